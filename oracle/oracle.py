@@ -1,0 +1,238 @@
+"""ctypes wrapper around the CPU oracle (wc_oracle.c).
+
+TEST INFRASTRUCTURE ONLY.  The oracle is the plain scalar statement of the
+exponent-plane rANS container; only the tests, the smoke check and the
+CPU-baseline leg of the benchmark may import this module.  The CUDA library
+never calls it and shares no code with it.
+
+Pins of every oracle function (worked traces, normalisation examples, brute
+force, the rANS accounting bound, exhaustive bf16 round trip, fp32 special
+values) live in tests/test_oracle_*.py.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(HERE, "wc_oracle.c")
+LIB = os.path.join(HERE, "liboracle.so")
+
+OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CORRUPT = 0, 1, 2, 4
+BF16, FP32 = 1, 2
+CHUNK = 65536
+
+
+def build(force: bool = False) -> str:
+    """Compile wc_oracle.c into liboracle.so (plain -O2, single thread)."""
+    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(
+        os.path.getmtime(SRC), os.path.getmtime(os.path.join(HERE, "wc_oracle.h"))
+    ):
+        tmp = LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c99", "-Wall", "-Wextra", "-shared", "-fPIC",
+             SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, LIB)
+    return LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(LIB)
+        u8p = ctypes.POINTER(ctypes.c_uint8)
+        u16p = ctypes.POINTER(ctypes.c_uint16)
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        u64p = ctypes.POINTER(ctypes.c_uint64)
+        vp = ctypes.c_void_p
+        L.oracle_encode_bound.restype = ctypes.c_uint64
+        L.oracle_encode_bound.argtypes = [ctypes.c_uint64, ctypes.c_int]
+        L.oracle_split_bf16.argtypes = [vp, ctypes.c_uint64, vp, vp]
+        L.oracle_split_fp32.argtypes = [vp, ctypes.c_uint64, vp, vp, vp]
+        L.oracle_histogram.argtypes = [vp, ctypes.c_uint64, vp]
+        L.oracle_normalize.argtypes = [vp, vp]
+        L.oracle_rans_encode.argtypes = [vp, ctypes.c_uint32, vp, ctypes.c_uint32, vp, vp, u32p]
+        L.oracle_rans_decode.argtypes = [vp, vp, ctypes.c_uint32, ctypes.c_uint32, vp,
+                                         ctypes.c_uint32, vp]
+        L.oracle_encode.argtypes = [vp, ctypes.c_uint64, ctypes.c_int, vp, ctypes.c_uint64, u64p]
+        L.oracle_decode.argtypes = [vp, ctypes.c_uint64, vp, ctypes.c_uint64]
+        L.oracle_decode_chunk.argtypes = [vp, ctypes.c_uint64, ctypes.c_uint64, vp, ctypes.c_uint64]
+        L.oracle_read_header.argtypes = [vp, ctypes.c_uint64, u64p, ctypes.POINTER(ctypes.c_int), u64p]
+        L.oracle_chunk_accounting.argtypes = [vp, ctypes.c_uint32, vp,
+                                              ctypes.POINTER(ctypes.c_double),
+                                              ctypes.POINTER(ctypes.c_double),
+                                              ctypes.POINTER(ctypes.c_double)]
+        del u8p, u16p, u64p
+        _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def dtype_code(arr: np.ndarray) -> int:
+    if arr.dtype == np.uint16:
+        return BF16
+    if arr.dtype == np.uint32:
+        return FP32
+    raise TypeError("oracle takes bf16 bits as uint16 or fp32 bits as uint32")
+
+
+class OracleError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: oracle status {code}")
+        self.code = code
+
+
+def encode_bound(n: int, dtype: int) -> int:
+    return int(lib().oracle_encode_bound(n, dtype))
+
+
+def split_bf16(bits: np.ndarray):
+    bits = np.ascontiguousarray(bits, dtype=np.uint16)
+    n = bits.size
+    e = np.empty(n, np.uint8)
+    sm = np.empty(n, np.uint8)
+    lib().oracle_split_bf16(_ptr(bits), n, _ptr(e), _ptr(sm))
+    return e, sm
+
+
+def split_fp32(bits: np.ndarray):
+    bits = np.ascontiguousarray(bits, dtype=np.uint32)
+    n = bits.size
+    e = np.empty(n, np.uint8)
+    sign = np.zeros((n + 7) // 8, np.uint8)
+    mant = np.empty(3 * n, np.uint8)
+    lib().oracle_split_fp32(_ptr(bits), n, _ptr(e), _ptr(sign) if sign.size else None,
+                            _ptr(mant) if mant.size else None)
+    return e, sign, mant
+
+
+def histogram(e: np.ndarray) -> np.ndarray:
+    e = np.ascontiguousarray(e, dtype=np.uint8)
+    c = np.zeros(256, np.uint64)
+    lib().oracle_histogram(_ptr(e) if e.size else None, e.size, _ptr(c))
+    return c
+
+
+def normalize(counts) -> np.ndarray:
+    c = np.zeros(256, np.uint64)
+    if isinstance(counts, dict):
+        for s, v in counts.items():
+            c[s] = v
+    else:
+        c[:] = np.asarray(counts, dtype=np.uint64)
+    f = np.zeros(256, np.uint16)
+    st = lib().oracle_normalize(_ptr(c), _ptr(f))
+    if st:
+        raise OracleError(st, "normalize")
+    return f
+
+
+def rans_encode(sym, freq, lanes: int = 32):
+    sym = np.ascontiguousarray(sym, dtype=np.uint8)
+    freq = np.ascontiguousarray(freq, dtype=np.uint16)
+    assert freq.size == 256
+    states = np.zeros(lanes, np.uint32)
+    words = np.zeros(max(sym.size, 1), np.uint16)
+    w = ctypes.c_uint32(0)
+    st = lib().oracle_rans_encode(_ptr(sym), sym.size, _ptr(freq), lanes, _ptr(states),
+                                  _ptr(words), ctypes.byref(w))
+    if st:
+        raise OracleError(st, "rans_encode")
+    return states, words[: w.value].copy()
+
+
+def rans_decode(states, words, nsym: int, freq, lanes: int = 32):
+    states = np.ascontiguousarray(states, dtype=np.uint32)
+    words = np.ascontiguousarray(words, dtype=np.uint16)
+    if words.size == 0:
+        words = np.zeros(1, np.uint16)[:0].copy()
+    freq = np.ascontiguousarray(freq, dtype=np.uint16)
+    out = np.zeros(max(nsym, 1), np.uint8)
+    wbuf = words if words.size else np.zeros(1, np.uint16)
+    st = lib().oracle_rans_decode(_ptr(states), _ptr(wbuf), words.size, nsym, _ptr(freq),
+                                  lanes, _ptr(out))
+    return st, out[:nsym]
+
+
+def encode(bits: np.ndarray) -> np.ndarray:
+    """Container bytes for a flat array of bf16 (uint16) or fp32 (uint32) bits."""
+    bits = np.ascontiguousarray(bits).reshape(-1)
+    dt = dtype_code(bits)
+    n = bits.size
+    cap = encode_bound(n, dt)
+    out = np.empty(cap, np.uint8)
+    size = ctypes.c_uint64(0)
+    st = lib().oracle_encode(_ptr(bits) if n else None, n, dt, _ptr(out), cap, ctypes.byref(size))
+    if st:
+        raise OracleError(st, "encode")
+    return out[: size.value].copy()
+
+
+def read_header(cont: np.ndarray):
+    cont = np.ascontiguousarray(cont, dtype=np.uint8)
+    n = ctypes.c_uint64(0)
+    dt = ctypes.c_int(0)
+    nc = ctypes.c_uint64(0)
+    st = lib().oracle_read_header(_ptr(cont), cont.size, ctypes.byref(n), ctypes.byref(dt),
+                                  ctypes.byref(nc))
+    if st:
+        raise OracleError(st, "read_header")
+    return n.value, dt.value, nc.value
+
+
+def decode_status(cont: np.ndarray, n_hint: int | None = None, dtype_hint: int | None = None):
+    """(status, values) without raising; values is None when the header is bad."""
+    cont = np.ascontiguousarray(cont, dtype=np.uint8)
+    n = ctypes.c_uint64(0)
+    dt = ctypes.c_int(0)
+    nc = ctypes.c_uint64(0)
+    st = lib().oracle_read_header(_ptr(cont), cont.size, ctypes.byref(n), ctypes.byref(dt),
+                                  ctypes.byref(nc))
+    if st:
+        return st, None
+    npdt = np.uint16 if dt.value == BF16 else np.uint32
+    out = np.zeros(max(n.value, 1), npdt)
+    st = lib().oracle_decode(_ptr(cont), cont.size, _ptr(out), out.nbytes)
+    return st, out[: n.value]
+
+
+def decode(cont: np.ndarray) -> np.ndarray:
+    st, out = decode_status(cont)
+    if st:
+        raise OracleError(st, "decode")
+    return out
+
+
+def decode_chunk(cont: np.ndarray, k: int) -> np.ndarray:
+    cont = np.ascontiguousarray(cont, dtype=np.uint8)
+    n, dt, nc = read_header(cont)
+    npdt = np.uint16 if dt == BF16 else np.uint32
+    nsym = min(CHUNK, n - k * CHUNK) if k < nc else 0
+    out = np.zeros(max(nsym, 1), npdt)
+    st = lib().oracle_decode_chunk(_ptr(cont), cont.size, k, _ptr(out), out.nbytes)
+    if st:
+        raise OracleError(st, "decode_chunk")
+    return out[:nsym]
+
+
+def chunk_accounting(sym, freq):
+    sym = np.ascontiguousarray(sym, dtype=np.uint8)
+    freq = np.ascontiguousarray(freq, dtype=np.uint16)
+    a, b, c = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+    st = lib().oracle_chunk_accounting(_ptr(sym), sym.size, _ptr(freq), ctypes.byref(a),
+                                       ctypes.byref(b), ctypes.byref(c))
+    if st:
+        raise OracleError(st, "chunk_accounting")
+    return a.value, b.value, c.value

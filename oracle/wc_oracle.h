@@ -1,0 +1,74 @@
+/*
+ * wc_oracle.h -- declarations of the CPU oracle for the exponent-plane rANS
+ * weight container.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This header and wc_oracle.c are the slow, plain,
+ * scalar reference that the CUDA library is checked against.  Only the test
+ * suite, the smoke check and the CPU-baseline leg of the benchmark may load
+ * it.  It shares no code, header, table or constant with the CUDA library:
+ * every constant below is restated here on purpose.
+ *
+ * All functions return 0 on success and one of the OR_ERR_* codes otherwise.
+ */
+#ifndef WC_ORACLE_H
+#define WC_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+    OR_OK = 0,
+    OR_ERR_INVALID_ARG = 1,
+    OR_ERR_CAPACITY = 2,
+    OR_ERR_CORRUPT = 4
+};
+
+enum { OR_BF16 = 1, OR_FP32 = 2 };
+
+/* Worst-case container size (every chunk stored raw). */
+uint64_t oracle_encode_bound(uint64_t n, int dtype);
+
+/* Plane split (PTWM README, "How it works" 1-2; SMEF README, pass 3). */
+void oracle_split_bf16(const uint16_t *in, uint64_t n, uint8_t *exp_plane,
+                       uint8_t *sm_plane);
+void oracle_split_fp32(const uint32_t *in, uint64_t n, uint8_t *exp_plane,
+                       uint8_t *sign_bits, uint8_t *mant3);
+
+/* 256-bin count of an exponent plane. */
+void oracle_histogram(const uint8_t *exp_plane, uint64_t n, uint64_t counts[256]);
+
+/* counts -> 12-bit table (sum 4096, every present symbol >= 1). */
+int oracle_normalize(const uint64_t counts[256], uint16_t freq[256]);
+
+/* Static rANS core for one chunk, with a lane count parameter (1 or 32 are
+ * used by the tests).  words must hold nsym entries.  No raw fallback here. */
+int oracle_rans_encode(const uint8_t *sym, uint32_t nsym, const uint16_t freq[256],
+                       uint32_t lanes, uint32_t *states_out, uint16_t *words_out,
+                       uint32_t *nwords_out);
+int oracle_rans_decode(const uint32_t *states_in, const uint16_t *words,
+                       uint32_t nwords, uint32_t nsym, const uint16_t freq[256],
+                       uint32_t lanes, uint8_t *sym_out);
+
+/* Whole container. */
+int oracle_encode(const void *in, uint64_t n, int dtype, uint8_t *out,
+                  uint64_t out_cap, uint64_t *out_size);
+int oracle_decode(const uint8_t *cont, uint64_t cont_bytes, void *out,
+                  uint64_t out_cap);
+int oracle_decode_chunk(const uint8_t *cont, uint64_t cont_bytes, uint64_t k,
+                        void *out, uint64_t out_cap);
+int oracle_read_header(const uint8_t *cont, uint64_t cont_bytes, uint64_t *n,
+                       int *dtype, uint64_t *nchunks);
+
+/* Diagnostic: for one chunk coded with the given table, the exact rANS
+ * accounting terms (see wc_oracle.c). */
+int oracle_chunk_accounting(const uint8_t *sym, uint32_t nsym,
+                            const uint16_t freq[256], double *coded_bits,
+                            double *ideal_bits, double *slack_bound);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

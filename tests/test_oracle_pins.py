@@ -1,0 +1,226 @@
+"""Pins of the CPU oracle against things other than itself: hand-worked traces
+and containers (tests/golden/), normalisation examples worked by hand, brute
+force over tiny inputs, the exact rANS accounting bound, and information
+theory.  No GPU needed."""
+import itertools
+
+import numpy as np
+import pytest
+
+from _golden import load_container, load_traces
+
+L = 65536
+
+
+# ---------------------------------------------------------------- traces
+@pytest.mark.parametrize("name", ["T1", "T2", "T3"])
+def test_hand_traces(orc, name):
+    tr = load_traces()[name]
+    states, words = orc.rans_encode(tr["syms"], tr["freq"], lanes=tr["lanes"])
+    assert states.tolist() == tr["states"]
+    assert words.tolist() == tr["words"]
+    st, back = orc.rans_decode(states, words, tr["syms"].size, tr["freq"], lanes=tr["lanes"])
+    assert st == 0
+    assert back.tolist() == tr["syms"].tolist()
+
+
+def test_T2_table_from_counts(orc):
+    """T2's table comes out of the normalisation of its own counts."""
+    e = np.array([127, 127, 127, 126], np.uint8)
+    f = orc.normalize(orc.histogram(e))
+    assert f[126] == 1024 and f[127] == 3072 and int(f.sum()) == 4096
+
+
+# ---------------------------------------------------------------- normalisation
+@pytest.mark.parametrize("counts,expect", [
+    ({0: 9997, 1: 1, 2: 1, 3: 1}, {0: 4093, 1: 1, 2: 1, 3: 1}),   # d = -1
+    ({5: 1, 6: 1, 7: 1}, {5: 1366, 6: 1365, 7: 1365}),            # d = +1, tie -> lowest
+    ({126: 1, 127: 3}, {126: 1024, 127: 3072}),                   # exact
+    ({42: 7}, {42: 4096}),                                        # single symbol
+    ({255: 123456789}, {255: 4096}),
+    # d = -4 with a tie between two equal maxima: 10, 20, 10, 20 give up 1 each
+    (dict([(10, 5000), (20, 5000)] + [(s, 1) for s in range(30, 40)]),
+     dict([(10, 2043), (20, 2043)] + [(s, 1) for s in range(30, 40)])),
+    # 255 rare symbols bumped to 1: the big one gives up 253 -> 4094 - 253
+    (dict([(0, 1000000)] + [(s, 1) for s in range(1, 256)]),
+     dict([(0, 3841)] + [(s, 1) for s in range(1, 256)])),
+    # all 256 symbols equally likely
+    ({s: 3 for s in range(256)}, {s: 16 for s in range(256)}),
+])
+def test_normalize_worked_examples(orc, counts, expect):
+    f = orc.normalize(counts)
+    want = np.zeros(256, np.uint16)
+    for s, v in expect.items():
+        want[s] = v
+    assert f.tolist() == want.tolist()
+
+
+def test_normalize_properties_random(orc):
+    rng = np.random.default_rng(123)
+    for trial in range(400):
+        k = int(rng.integers(1, 257))
+        present = rng.choice(256, size=k, replace=False)
+        counts = np.zeros(256, np.uint64)
+        scale = 10 ** int(rng.integers(0, 9))
+        counts[present] = rng.integers(1, scale + 2, size=k).astype(np.uint64)
+        if trial % 3 == 0:  # heavy skew
+            counts[present[0]] *= np.uint64(10 ** 6)
+        f = orc.normalize(counts).astype(np.int64)
+        assert int(f.sum()) == 4096
+        assert np.all(f[counts > 0] >= 1)
+        assert np.all(f[counts == 0] == 0)
+        # each frequency stays within its rounding window plus the correction:
+        # |f - c*4096/n| < 1 + |d| where |d| <= number of present symbols
+        n = float(counts.sum())
+        ideal = counts.astype(np.float64) * 4096.0 / n
+        assert np.all(np.abs(f - ideal)[counts > 0] <= 1 + k)
+
+
+def test_normalize_empty(orc):
+    assert orc.normalize(np.zeros(256, np.uint64)).tolist() == [0] * 256
+
+
+# ---------------------------------------------------------------- brute force
+def _tables(nsym_alpha, rng):
+    """A few valid tables over symbols 0..nsym_alpha-1: extremes and random."""
+    tabs = []
+    a = nsym_alpha
+    f = np.zeros(256, np.uint16)
+    f[:a] = 1
+    f[0] = 4096 - (a - 1)
+    tabs.append(f.copy())
+    f[:a] = 1
+    f[a - 1] = 4096 - (a - 1)
+    tabs.append(f.copy())
+    for _ in range(2):
+        cuts = np.sort(rng.choice(np.arange(1, 4096), size=a - 1, replace=False))
+        parts = np.diff(np.concatenate([[0], cuts, [4096]]))
+        g = np.zeros(256, np.uint16)
+        g[:a] = parts
+        tabs.append(g)
+    return tabs
+
+
+@pytest.mark.parametrize("lanes", [1, 32])
+def test_brute_force_round_trip(orc, lanes):
+    """Every sequence of length <= 6 over 2..4 symbols, several tables:
+    decode(encode(x)) == x, every lane back at 2^16, every word read."""
+    rng = np.random.default_rng(7)
+    for alpha in (2, 3, 4):
+        for tab in _tables(alpha, rng):
+            for length in range(1, 7):
+                for seq in itertools.product(range(alpha), repeat=length):
+                    sym = np.array(seq, np.uint8)
+                    states, words = orc.rans_encode(sym, tab, lanes=lanes)
+                    assert np.all(states >= L)
+                    st, back = orc.rans_decode(states, words, length, tab, lanes=lanes)
+                    assert st == 0 and back.tolist() == list(seq)
+
+
+def test_decoder_rejects_wrong_word_count(orc):
+    tr = load_traces()["T3"]
+    states, words = orc.rans_encode(tr["syms"], tr["freq"], lanes=32)
+    st, _ = orc.rans_decode(states, words[:-1], tr["syms"].size, tr["freq"], lanes=32)
+    assert st == 4
+    st, _ = orc.rans_decode(states, np.concatenate([words, [7]]), tr["syms"].size, tr["freq"], lanes=32)
+    assert st == 4
+    bad = states.copy()
+    bad[5] += 1
+    st, _ = orc.rans_decode(bad, words, tr["syms"].size, tr["freq"], lanes=32)
+    assert st == 4
+
+
+# ---------------------------------------------------------------- accounting
+def test_accounting_bound_and_entropy(orc):
+    """|coded - ideal| <= exact slack for every chunk of workload 1, and the
+    coded size is within 0.5% of the cross-entropy under the 12-bit table
+    plus the fixed per-chunk overhead (128 state bytes, <= 15 pad bytes)."""
+    import workloads
+    bits = workloads.generate_tensor(1, 0)
+    e, _ = orc.split_bf16(bits)
+    f = orc.normalize(orc.histogram(e))
+    cont = orc.encode(bits)
+    n, dt, nc = orc.read_header(cont)
+    off_len = 576 + 8 * (nc + 1)
+    lens = cont[off_len: off_len + 4 * nc].view(np.uint32)
+    for k in range(nc):
+        sym = e[k * 65536:(k + 1) * 65536]
+        coded, ideal, slack = orc.chunk_accounting(sym, f)
+        assert abs(coded - ideal) <= slack + 1e-6
+        assert slack < 5e-3 * ideal          # the bound itself is within 0.5%
+        assert abs(coded - ideal) < 1e-4 * ideal
+        assert lens[k] < 65536  # coded, not raw
+        # coded bits = payload bits beyond the 32 x 16 state bits of L
+        assert abs(8 * (int(lens[k]) - 128) + 32 * 16 - coded) < 32 * 17
+        assert 8 * int(lens[k]) <= 1.005 * ideal + 8 * (128 + 15)
+
+
+def test_exponent_statistics_sanity(orc):
+    """N(0, 0.02) bf16: ~20 distinct exponents, ~2.5 bits/byte ("PTWM" How it
+    works 2 reports ~20 values and ~2.6 bits/byte on trained weights)."""
+    import workloads
+    e, _ = orc.split_bf16(workloads.generate_tensor(1, 0))
+    c = orc.histogram(e).astype(np.float64)
+    p = c[c > 0] / c.sum()
+    assert 15 <= (c > 0).sum() <= 30
+    assert 2.3 < -(p * np.log2(p)).sum() < 2.8
+
+
+# ---------------------------------------------------------------- planes
+def test_split_bf16_worked(orc):
+    bits = np.array([0xBF80, 0x3F81, 0x0001, 0xFFFF, 0x7F80], np.uint16)
+    e, sm = orc.split_bf16(bits)
+    assert e.tolist() == [127, 127, 0, 255, 255]
+    assert sm.tolist() == [0x80, 0x01, 0x01, 0xFF, 0x00]
+
+
+def test_split_fp32_worked(orc):
+    bits = np.array([0x3F800000, 0xBF800000, 0x00000001, 0x7FC00000,
+                     0x807FFFFF, 0x00000000, 0x00000000, 0x00000000,
+                     0x80000000], np.uint32)
+    e, sign, mant = orc.split_fp32(bits)
+    assert e.tolist() == [127, 127, 0, 255, 0, 0, 0, 0, 0]
+    assert sign.tolist() == [0b00010010, 0b00000001]
+    assert mant[:15].tolist() == [0, 0, 0, 0, 0, 0, 1, 0, 0, 0, 0, 0x40, 0xFF, 0xFF, 0x7F]
+
+
+# ---------------------------------------------------------------- containers
+def test_golden_container_raw_chunk(orc):
+    bits = np.array([0x3F80, 0x3F80, 0x3F80, 0x3F00], np.uint16)
+    want = load_container("container_bf16_n4_raw.txt")
+    got = orc.encode(bits)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert orc.decode(got).tolist() == bits.tolist()
+
+
+def test_golden_container_single_symbol(orc):
+    bits = np.full(200, 0x3F80, np.uint16)
+    want = load_container("container_bf16_n200_single_symbol.txt")
+    got = orc.encode(bits)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert orc.decode(got).tolist() == bits.tolist()
+
+
+def test_coded_payload_layout(orc):
+    """A coded chunk's payload read as [32 x u32 states][w x u16 words]
+    decodes with the rANS core to the chunk's exponents."""
+    import workloads
+    bits = workloads.generate_tensor(1, 0)[:100000]
+    cont = orc.encode(bits)
+    n, dt, nc = orc.read_header(cont)
+    off_exp = int(cont[40:48].view(np.uint64)[0])
+    choff = cont[576:576 + 8 * (nc + 1)].view(np.uint64)
+    lens = cont[576 + 8 * (nc + 1): 576 + 8 * (nc + 1) + 4 * nc].view(np.uint32)
+    f = cont[64:576].view(np.uint16)
+    e, _ = orc.split_bf16(bits)
+    for k in range(nc):
+        nsym = min(65536, n - 65536 * k)
+        p = off_exp + int(choff[k])
+        assert lens[k] < nsym
+        states = cont[p:p + 128].view(np.uint32)
+        w = (int(lens[k]) - 128) // 2
+        words = cont[p + 128:p + 128 + 2 * w].view(np.uint16)
+        st, sym = orc.rans_decode(states, words, nsym, f)
+        assert st == 0 and np.array_equal(sym, e[65536 * k:65536 * k + nsym])
+        pad = cont[p + int(lens[k]): p + int(choff[k + 1] - choff[k])]
+        assert not pad.any()
