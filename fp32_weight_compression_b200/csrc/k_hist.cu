@@ -1,0 +1,235 @@
+// k_hist.cu -- encoder stage 1: container header, per-tensor exponent
+// histogram, and the 12-bit frequency table.
+//
+//  k_prep   one block per tensor: clears the tensor's scratch counters and
+//           writes the fixed header fields and the zero padding of the
+//           container (everything that depends on n alone).
+//  k_hist   one block per 65,536-value chunk: reads the chunk's values as
+//           integers (a NaN payload is never touched as a float), counts the
+//           8-bit exponents ("PTWM" How it works 1-2: after the bit reorder the
+//           exponent is a whole byte; "SMEF" pass3_streams.py) into a
+//           shared-memory histogram with one column per lane (so the 32 lanes
+//           of a warp never collide on an address), folds it into the tensor's
+//           global histogram, and the last block of each tensor turns the
+//           counts into the table.
+//
+// Table rule (the pages fix none; this is the container's rule):
+// f_s = 0 if c_s = 0 else max(1, floor(c_s 4096 / n));
+// d = 4096 - sum f; d > 0: the symbol with the largest count (lowest symbol on
+// ties) takes d; d < 0: -d times the symbol with the largest f among f > 1
+// (lowest symbol on ties) gives up one.  The repeated give-up is evaluated in
+// closed form here: with D(T) = sum max(0, f_s - T), let T be the smallest
+// level >= 1 with D(T) <= -d; every f_s >= T becomes T, and the r = -d - D(T)
+// lowest-numbered of them go on to T - 1.  This is the state the one-at-a-time
+// rule reaches: it always lowers a current maximum, so it flattens everything
+// above T to T first, and then takes the tied symbols at T in symbol order.
+#include "wc_block.cuh"
+#include "wc_format.cuh"
+
+namespace wc {
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_prep(const __grid_constant__ EncParams p) {
+  const EncItem &it = p.items[blockIdx.x];
+  const int tid = threadIdx.x;
+  const int dtype = int(it.dtype);
+  const Layout L = make_layout(it.n, dtype);
+  uint8_t *out = it.out;
+
+  uint64_t *hist = reinterpret_cast<uint64_t *>(it.scratch + kScrHist);
+  uint32_t *ctr = reinterpret_cast<uint32_t *>(it.scratch + kScrCtr);
+  hist[tid] = 0;
+  if (tid < 4) ctr[tid] = 0;
+
+  // table: all zero until the last histogram block writes it (n = 0 keeps it)
+  reinterpret_cast<uint16_t *>(out + kFreqOffset)[tid] = 0;
+
+  if (tid == 0) {
+    uint32_t *h32 = reinterpret_cast<uint32_t *>(out);
+    uint64_t *h64 = reinterpret_cast<uint64_t *>(out);
+    h32[0] = 0x315A4357u;  // "WCZ1"
+    h32[1] = kVersion | (uint32_t(dtype) << 16) | (kLanes << 24);
+    h64[1] = it.n;
+    h32[4] = kChunk;
+    h32[5] = uint32_t(L.nc);
+    h32[6] = kProbBits;  // u16 12, u16 0
+    h32[7] = 0;
+    h64[4] = L.off_raw;
+    h64[5] = L.off_exp;
+    if (it.n == 0) {
+      h64[6] = 0;
+      h64[7] = L.off_exp;
+      *reinterpret_cast<uint64_t *>(out + L.off_chunk_off) = 0;
+      *it.out_size = L.off_exp;
+    }
+  }
+  // zero padding: after the chunk-length table, and after each raw plane
+  if (tid < 16) {
+    uint64_t a = L.off_chunk_len + 4 * L.nc + tid;
+    if (a < L.off_raw) out[a] = 0;
+    if (dtype == WC_BF16) {
+      uint64_t b = L.off_raw + it.n + tid;
+      if (b < L.off_exp) out[b] = 0;
+    } else {
+      uint64_t b = L.off_raw + (it.n + 7) / 8 + tid;
+      if (b < L.off_mant) out[b] = 0;
+      uint64_t c = L.off_mant + 3 * it.n + tid;
+      if (c < L.off_exp) out[c] = 0;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+constexpr int kHistThreads = 512;
+
+__device__ __forceinline__ void count_bf16_word(uint32_t *sh, int lane, uint32_t w) {
+  atomicAdd(&sh[(((w >> 7) & 0xFFu) << 5) | lane], 1u);
+  atomicAdd(&sh[(((w >> 23) & 0xFFu) << 5) | lane], 1u);
+}
+__device__ __forceinline__ void count_fp32_word(uint32_t *sh, int lane, uint32_t u) {
+  atomicAdd(&sh[(((u >> 23) & 0xFFu) << 5) | lane], 1u);
+}
+
+// The last block of a tensor: counts -> table, published to the container
+// header (u16 freq[256]) and to the coder's scratch entries.
+__device__ void publish_table(const EncItem &it, uint64_t *red) {
+  const int tid = threadIdx.x;
+  const bool own = tid < 256;  // thread s owns symbol s
+  const uint64_t n = it.n;
+  const uint64_t *ghist = reinterpret_cast<const uint64_t *>(it.scratch + kScrHist);
+  uint64_t c = own ? __ldcg(&ghist[tid]) : 0;
+  uint64_t f = 0;
+  if (c) {
+    f = c * uint64_t(kProbScale) / n;
+    if (f < 1) f = 1;
+  }
+  const int64_t d = int64_t(kProbScale) - int64_t(block_sum_u64<kHistThreads>(f, red));
+  if (d > 0) {
+    uint64_t key = c ? ((c << 8) | uint64_t(255 - tid)) : 0;
+    uint64_t best = block_max_u64<kHistThreads>(key, red);
+    if (own && tid == int(255 - (best & 0xFF))) f += uint64_t(d);
+  } else if (d < 0) {
+    const uint64_t k = uint64_t(-d);
+    uint32_t lo = 1, hi = kProbScale;
+    while (lo < hi) {  // smallest T in [1, 4096] with D(T) <= k
+      uint32_t mid = (lo + hi) >> 1;
+      uint64_t Dm = block_sum_u64<kHistThreads>(f > mid ? f - mid : 0, red);
+      if (Dm <= k) hi = mid; else lo = mid + 1;
+    }
+    const uint32_t T = lo;
+    const uint64_t DT = block_sum_u64<kHistThreads>(f > T ? f - T : 0, red);
+    const uint64_t r = k - DT;
+    const bool ge = own && f >= T;
+    const uint64_t rank = block_excl_scan_u64<kHistThreads>(ge ? 1 : 0, red);
+    if (ge) f = T - (rank < r ? 1 : 0);
+  }
+  const uint64_t cum = block_excl_scan_u64<kHistThreads>(f, red);
+  if (own) {
+    const uint32_t ff = uint32_t(f);
+    reinterpret_cast<uint16_t *>(it.out + kFreqOffset)[tid] = uint16_t(ff);
+    uint4 e = make_uint4(0, 0, 0, 0);
+    uint32_t bias = 0;
+    if (ff) {
+      // q = floor(x / f) = floor(x * m / 2^64) with m = ceil(2^64 / f), exact
+      // for every x < 2^32 (x * (m f - 2^64) < 2^32 * f < 2^64); f = 1 uses
+      // m = 2^64 - 1, which yields q = x - 1, repaid by bias += 4095.
+      const uint64_t m = ff >= 2 ? (~uint64_t(0) / ff + 1) : ~uint64_t(0);
+      e.x = uint32_t(m);
+      e.y = uint32_t(m >> 32);
+      e.z = uint32_t((uint64_t(ff) << 20) - 1);  // renormalise while x > xmax
+      e.w = kProbScale - ff;
+      bias = uint32_t(cum) + (ff == 1 ? kProbScale - 1 : 0);
+    }
+    reinterpret_cast<uint4 *>(it.scratch + kScrTab)[tid] = e;
+    reinterpret_cast<uint32_t *>(it.scratch + kScrBias)[tid] = bias;
+  }
+}
+
+__global__ void __launch_bounds__(kHistThreads, 2) k_hist(const __grid_constant__ EncParams p) {
+  __shared__ __align__(16) uint32_t sh[256 * 32];  // [exponent][lane]
+  __shared__ uint64_t red[kHistThreads / 32 + 1];
+  __shared__ int s_last;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint32_t g = blockIdx.x;
+  const EncItem &it = p.items[find_item_by_chunk(p, g)];
+  const uint64_t k = g - it.chunk_base;
+  const uint32_t nsym = chunk_nsym(it.n, k);
+  const uint64_t nc = num_chunks(it.n);
+
+  for (int i = tid; i < 256 * 32 / 4; i += kHistThreads)
+    reinterpret_cast<uint4 *>(sh)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+
+  // Each thread takes 16-value groups tid, tid + 512, ... (8 per full chunk).
+  if (it.dtype == WC_BF16) {
+    const uint16_t *src = reinterpret_cast<const uint16_t *>(it.in) + k * kChunk;
+#pragma unroll 4
+    for (int j = 0; j < int(kChunk / 16 / kHistThreads); j++) {
+      const uint32_t v0 = (uint32_t(j) * kHistThreads + tid) * 16;
+      if (v0 + 16 <= nsym) {
+        uint4 a = ld_nc_v4(src + v0);
+        uint4 b = ld_nc_v4(src + v0 + 8);
+        count_bf16_word(sh, lane, a.x); count_bf16_word(sh, lane, a.y);
+        count_bf16_word(sh, lane, a.z); count_bf16_word(sh, lane, a.w);
+        count_bf16_word(sh, lane, b.x); count_bf16_word(sh, lane, b.y);
+        count_bf16_word(sh, lane, b.z); count_bf16_word(sh, lane, b.w);
+      } else if (v0 < nsym) {
+        for (uint32_t v = v0; v < nsym; v++)
+          atomicAdd(&sh[((uint32_t(src[v] >> 7) & 0xFFu) << 5) | lane], 1u);
+      }
+    }
+  } else {
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(it.in) + k * kChunk;
+#pragma unroll 2
+    for (int j = 0; j < int(kChunk / 16 / kHistThreads); j++) {
+      const uint32_t v0 = (uint32_t(j) * kHistThreads + tid) * 16;
+      if (v0 + 16 <= nsym) {
+        uint4 a = ld_nc_v4(src + v0), b = ld_nc_v4(src + v0 + 4);
+        uint4 c = ld_nc_v4(src + v0 + 8), d = ld_nc_v4(src + v0 + 12);
+        count_fp32_word(sh, lane, a.x); count_fp32_word(sh, lane, a.y);
+        count_fp32_word(sh, lane, a.z); count_fp32_word(sh, lane, a.w);
+        count_fp32_word(sh, lane, b.x); count_fp32_word(sh, lane, b.y);
+        count_fp32_word(sh, lane, b.z); count_fp32_word(sh, lane, b.w);
+        count_fp32_word(sh, lane, c.x); count_fp32_word(sh, lane, c.y);
+        count_fp32_word(sh, lane, c.z); count_fp32_word(sh, lane, c.w);
+        count_fp32_word(sh, lane, d.x); count_fp32_word(sh, lane, d.y);
+        count_fp32_word(sh, lane, d.z); count_fp32_word(sh, lane, d.w);
+      } else if (v0 < nsym) {
+        for (uint32_t v = v0; v < nsym; v++) count_fp32_word(sh, lane, src[v]);
+      }
+    }
+  }
+  __syncthreads();
+
+  uint64_t *ghist = reinterpret_cast<uint64_t *>(it.scratch + kScrHist);
+  if (tid < 256) {
+    uint32_t sum = 0;
+#pragma unroll 8
+    for (int j = 0; j < 32; j++) sum += sh[(tid << 5) | ((j + tid) & 31)];
+    if (sum) atomicAdd(reinterpret_cast<unsigned long long *>(&ghist[tid]),
+                       static_cast<unsigned long long>(sum));
+  }
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t *ctr = reinterpret_cast<uint32_t *>(it.scratch + kScrCtr);
+    s_last = (atomicAdd(&ctr[0], 1u) == uint32_t(nc - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  publish_table(it, red);
+}
+
+cudaError_t launch_prep(const EncParams &p, cudaStream_t s) {
+  k_prep<<<p.count, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_hist(const EncParams &p, cudaStream_t s) {
+  if (p.total_chunks == 0) return cudaSuccess;
+  k_hist<<<p.total_chunks, kHistThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace wc

@@ -1,0 +1,310 @@
+"""Python binding of libwc.so (include/wc.h): argument marshalling only.
+
+Every step of encoding and decoding runs in the library's CUDA kernels; this
+module only allocates device buffers through PyTorch, passes pointers, sizes
+and the current stream, and turns status codes into exceptions.  There is no
+CPU path: if libwc.so is missing or no CUDA device is present the calls fail.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libwc.so")
+
+OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CUDA, ERR_CORRUPT, ERR_UNSUPPORTED = 0, 1, 2, 3, 4, 5
+BF16, FP32 = 1, 2
+CHUNK = 65536
+
+_DT = {torch.bfloat16: BF16, torch.float32: FP32}
+_TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32}
+_ELEM = {BF16: 2, FP32: 4}
+
+EXPORTS = (
+    "wc_encode_bound", "wc_scratch_bytes", "wc_encode", "wc_decode", "wc_decode_chunk",
+    "wc_read_header", "wc_encode_batch", "wc_decode_batch", "wc_status_string", "wc_last_error",
+)
+
+
+class EncodeItem(ctypes.Structure):
+    _fields_ = [("in_", ctypes.c_void_p), ("n", ctypes.c_uint64), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("out", ctypes.c_void_p), ("out_cap", ctypes.c_uint64),
+                ("scratch", ctypes.c_void_p), ("scratch_cap", ctypes.c_uint64),
+                ("out_size", ctypes.c_void_p)]
+
+
+class DecodeItem(ctypes.Structure):
+    _fields_ = [("cont", ctypes.c_void_p), ("cont_bytes", ctypes.c_uint64),
+                ("out", ctypes.c_void_p), ("out_cap", ctypes.c_uint64)]
+
+
+class WCError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {status_string(code)}"
+                         + (f" ({last_error()})" if code == ERR_CUDA else ""))
+        self.code = code
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libwc.so from this package directory (no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run `python -m fp32_weight_compression_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    u64, i32, u32, vp = ctypes.c_uint64, ctypes.c_int32, ctypes.c_uint32, ctypes.c_void_p
+    L.wc_encode_bound.restype = u64
+    L.wc_encode_bound.argtypes = [u64, i32]
+    L.wc_scratch_bytes.restype = u64
+    L.wc_scratch_bytes.argtypes = [u64, i32]
+    L.wc_encode.restype = i32
+    L.wc_encode.argtypes = [vp, u64, i32, vp, u64, vp, u64, vp, vp]
+    L.wc_decode.restype = i32
+    L.wc_decode.argtypes = [vp, u64, vp, u64, vp, vp]
+    L.wc_decode_chunk.restype = i32
+    L.wc_decode_chunk.argtypes = [vp, u64, u64, vp, u64, vp, vp]
+    L.wc_read_header.restype = i32
+    L.wc_read_header.argtypes = [vp, u64, ctypes.POINTER(u64), ctypes.POINTER(i32), ctypes.POINTER(u64)]
+    L.wc_encode_batch.restype = i32
+    L.wc_encode_batch.argtypes = [ctypes.POINTER(EncodeItem), u32, vp]
+    L.wc_decode_batch.restype = i32
+    L.wc_decode_batch.argtypes = [ctypes.POINTER(DecodeItem), u32, vp, vp]
+    L.wc_status_string.restype = ctypes.c_char_p
+    L.wc_status_string.argtypes = [i32]
+    L.wc_last_error.restype = ctypes.c_char_p
+    L.wc_last_error.argtypes = []
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return load().wc_status_string(code).decode()
+
+
+def last_error() -> str:
+    return load().wc_last_error().decode()
+
+
+def _check(code: int, what: str):
+    if code != OK:
+        raise WCError(code, what)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def dtype_code(dtype: torch.dtype) -> int:
+    try:
+        return _DT[dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {dtype}: bf16 and fp32 only") from None
+
+
+def encode_bound(n: int, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return int(load().wc_encode_bound(n, code))
+
+
+def scratch_bytes(n: int, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return int(load().wc_scratch_bytes(n, code))
+
+
+def read_header(cont) -> tuple[int, int, int]:
+    """(n, dtype code, chunks) from a host copy of a container (bytes, numpy
+    array or CPU uint8 tensor)."""
+    if isinstance(cont, torch.Tensor):
+        cont = cont.detach().cpu().numpy()
+    import numpy as np
+    buf = np.ascontiguousarray(np.frombuffer(bytes(cont), np.uint8) if isinstance(cont, (bytes, bytearray)) else cont,
+                               dtype=np.uint8)
+    n, dt, nc = ctypes.c_uint64(), ctypes.c_int32(), ctypes.c_uint64()
+    _check(load().wc_read_header(buf.ctypes.data, buf.size, ctypes.byref(n), ctypes.byref(dt),
+                                 ctypes.byref(nc)), "wc_read_header")
+    return n.value, dt.value, nc.value
+
+
+def _flat(t: torch.Tensor) -> torch.Tensor:
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.reshape(-1)
+
+
+def _align_up(v: int, a: int) -> int:
+    return (v + a - 1) // a * a
+
+
+class BatchEncoder:
+    """Encodes a fixed list of tensor shapes/dtypes into preallocated device
+    buffers with one wc_encode_batch call.  Containers stay on the device;
+    `sizes` (u64 per tensor) is filled on the device."""
+
+    def __init__(self, numels, dtypes, device="cuda"):
+        self.numels = [int(n) for n in numels]
+        self.codes = [d if isinstance(d, int) else dtype_code(d) for d in dtypes]
+        self.device = torch.device(device)
+        caps = [encode_bound(n, c) for n, c in zip(self.numels, self.codes)]
+        scr = [scratch_bytes(n, c) for n, c in zip(self.numels, self.codes)]
+        self.out_offsets, off = [], 0
+        for c in caps:
+            self.out_offsets.append(off)
+            off = _align_up(off + c, 256)
+        self.caps = caps
+        self.out = torch.empty(max(off, 256), dtype=torch.uint8, device=self.device)
+        self.scr_offsets, off = [], 0
+        for c in scr:
+            self.scr_offsets.append(off)
+            off = _align_up(off + c, 256)
+        self.scratch = torch.empty(max(off, 256), dtype=torch.uint8, device=self.device)
+        self.sizes = torch.zeros(len(caps), dtype=torch.int64, device=self.device)
+        self._items = (EncodeItem * len(caps))()
+        self._key = None
+
+    def containers(self, sizes=None) -> list[torch.Tensor]:
+        """Views of the containers trimmed to size (reads the sizes back)."""
+        if sizes is None:
+            sizes = self.sizes.cpu().tolist()
+        return [self.out[o:o + int(s)] for o, s in zip(self.out_offsets, sizes)]
+
+    def encode(self, tensors, stream=None):
+        flats = [_flat(t) for t in tensors]
+        if len(flats) != len(self.numels):
+            raise ValueError("tensor count does not match the encoder")
+        key = tuple(t.data_ptr() for t in flats)
+        if key != self._key:
+            base_o, base_s, base_z = self.out.data_ptr(), self.scratch.data_ptr(), self.sizes.data_ptr()
+            for i, t in enumerate(flats):
+                if t.numel() != self.numels[i] or dtype_code(t.dtype) != self.codes[i]:
+                    raise ValueError(f"tensor {i} does not match the encoder's shape/dtype")
+                it = self._items[i]
+                it.in_ = t.data_ptr() if t.numel() else None
+                it.n = t.numel()
+                it.dtype = self.codes[i]
+                it.reserved = 0
+                it.out = base_o + self.out_offsets[i]
+                it.out_cap = self.caps[i]
+                it.scratch = base_s + self.scr_offsets[i]
+                it.scratch_cap = scratch_bytes(self.numels[i], self.codes[i])
+                it.out_size = base_z + 8 * i
+            self._key = key
+        _check(load().wc_encode_batch(self._items, len(flats), _stream(stream)), "wc_encode_batch")
+        return self
+
+
+class BatchDecoder:
+    """Decodes a fixed list of containers (device uint8 buffers) into
+    preallocated outputs with one wc_decode_batch call."""
+
+    def __init__(self, device="cuda"):
+        self.device = torch.device(device)
+        self.status = torch.zeros(1, dtype=torch.int32, device=self.device)
+        self._items = None
+        self._key = None
+
+    def decode(self, conts, outs, cont_bytes=None, stream=None):
+        if cont_bytes is None:
+            cont_bytes = [c.numel() for c in conts]
+        key = tuple(c.data_ptr() for c in conts) + tuple(o.data_ptr() for o in outs) + tuple(cont_bytes)
+        if key != self._key:
+            self._items = (DecodeItem * len(conts))()
+            for i, (c, o, nb) in enumerate(zip(conts, outs, cont_bytes)):
+                of = _flat(o)
+                it = self._items[i]
+                it.cont = c.data_ptr()
+                it.cont_bytes = int(nb)
+                it.out = of.data_ptr() if of.numel() else None
+                it.out_cap = of.numel() * of.element_size()
+            self._key = key
+        _check(load().wc_decode_batch(self._items, len(conts), self.status.data_ptr(),
+                                      _stream(stream)), "wc_decode_batch")
+        return self
+
+    def check(self):
+        """Synchronising read of the device status; raises on a bad container."""
+        st = int(self.status.item())
+        if st != OK:
+            raise WCError(st, "decode (device status)")
+
+
+# ---------------------------------------------------------------------------
+# Convenience single-tensor calls (allocate through torch, sync to trim).
+# ---------------------------------------------------------------------------
+def encode(t: torch.Tensor, stream=None) -> torch.Tensor:
+    """Container (device uint8 tensor, trimmed) for a bf16 / fp32 tensor."""
+    f = _flat(t)
+    code = dtype_code(f.dtype)
+    n = f.numel()
+    cap = encode_bound(n, code)
+    out = torch.empty(cap, dtype=torch.uint8, device=f.device)
+    scr = torch.empty(max(scratch_bytes(n, code), 256), dtype=torch.uint8, device=f.device)
+    size = torch.zeros(1, dtype=torch.int64, device=f.device)
+    _check(load().wc_encode(f.data_ptr() if n else None, n, code, out.data_ptr(), cap,
+                            scr.data_ptr(), scr.numel(), size.data_ptr(), _stream(stream)),
+           "wc_encode")
+    return out[: int(size.item())]
+
+
+def encode_batch(tensors, stream=None) -> list[torch.Tensor]:
+    if not tensors:
+        return []
+    enc = BatchEncoder([t.numel() for t in tensors], [t.dtype for t in tensors],
+                       device=tensors[0].device)
+    enc.encode(tensors, stream)
+    return [c.clone() for c in enc.containers()]
+
+
+def decode(cont: torch.Tensor, shape=None, dtype=None, out=None, stream=None) -> torch.Tensor:
+    """Decode a device container.  Without shape/dtype/out the header is
+    copied to the host once to size the output."""
+    if out is None:
+        if shape is None or dtype is None:
+            n, code, _ = read_header(cont[:64].cpu())
+            dtype = _TORCH_DT[code]
+            shape = (n,) if shape is None else shape
+        out = torch.empty(shape, dtype=dtype, device=cont.device)
+    of = _flat(out)
+    status = torch.zeros(1, dtype=torch.int32, device=cont.device)
+    _check(load().wc_decode(cont.data_ptr(), cont.numel(), of.data_ptr() if of.numel() else None,
+                            of.numel() * of.element_size(), status.data_ptr(), _stream(stream)),
+           "wc_decode")
+    st = int(status.item())
+    if st != OK:
+        raise WCError(st, "wc_decode (device status)")
+    return out
+
+
+def decode_chunk(cont: torch.Tensor, k: int, dtype=None, stream=None) -> torch.Tensor:
+    """Values [65536 k, min(n, 65536 (k + 1))) of a device container."""
+    n, code, nc = read_header(cont[:64].cpu())
+    if dtype is not None and dtype_code(dtype) != code:
+        raise TypeError("dtype does not match the container")
+    nvals = max(0, min(CHUNK, n - k * CHUNK)) if k < nc else 0
+    out = torch.empty(max(nvals, 1), dtype=_TORCH_DT[code], device=cont.device)
+    status = torch.zeros(1, dtype=torch.int32, device=cont.device)
+    _check(load().wc_decode_chunk(cont.data_ptr(), cont.numel(), k, out.data_ptr(),
+                                  nvals * _ELEM[code], status.data_ptr(), _stream(stream)),
+           "wc_decode_chunk")
+    st = int(status.item())
+    if st != OK:
+        raise WCError(st, "wc_decode_chunk (device status)")
+    return out[:nvals]
+
+
+def decode_batch(conts, shapes, dtypes, stream=None) -> list[torch.Tensor]:
+    outs = [torch.empty(s, dtype=d, device=c.device) for c, s, d in zip(conts, shapes, dtypes)]
+    dec = BatchDecoder(device=conts[0].device if conts else "cuda")
+    dec.decode(conts, outs, stream=stream)
+    dec.check()
+    return outs

@@ -1,0 +1,164 @@
+/*
+ * wc.h -- C ABI of the B200 (sm_100a) exponent-plane rANS weight codec.
+ *
+ * Lossless compression of bf16 / fp32 weight tensors.  Each float is split
+ * into planes; the skewed 8-bit exponent plane is entropy-coded with a
+ * static, 32-lane interleaved rANS coder, chunk by chunk; the sign and
+ * mantissa bits are stored raw.  Decoding re-merges the planes into the
+ * original bits.  The method follows:
+ *   - "PTWM" (PyPI README), "How it works": 1. Bit reorder (the exponent
+ *     moves to the top byte, the sign is tucked under it) and 2. Byte /
+ *     nibble split (bf16: 2 planes, plane 1 = exponent); the exponent plane
+ *     holds ~20 distinct values, the mantissa planes look random;
+ *   - "SMEF -- blog companion code", file table: pass3_streams.py splits
+ *     sign / exponent / mantissa streams, pass4_rans.py is the rANS coder;
+ *   - "PTWM", Configuration table: compression_threshold (store raw when
+ *     coding does not pay) and is_streaming / streaming_chunk (independently
+ *     decodable chunks);
+ *   - "seedpack 0.2.0 -> 0.2.2", README: a container of chunks plus an index,
+ *     with random access.
+ *
+ * Container (every field little-endian, sections 16-byte aligned, pad bytes
+ * zero):  "WCZ1", u16 version 1, u8 dtype, u8 lanes (32), u64 n,
+ * u32 chunk symbols (65536), u32 nc, u16 table bits (12), u16 0, u32 0,
+ * u64 off_raw, u64 off_exp, u64 exp_bytes, u64 total_bytes (64 bytes), then
+ * u16 freq[256], u64 chunk_off[nc+1], u32 chunk_len[nc], the raw planes
+ * (bf16: n sign+mantissa bytes; fp32: ceil(n/8) sign-bit bytes, 3n mantissa
+ * bytes) and the exponent chunks.  A coded chunk is 32 final u32 states then
+ * w u16 renormalisation words (128 + 2w bytes); a chunk whose coded form is
+ * not smaller than its nsym exponent bytes is stored raw.  The format is
+ * fully determined by the input bits: one input has exactly one container.
+ *
+ * Conventions for every call below:
+ *   - Pointers named d_* are device pointers on the current CUDA device;
+ *     h_* are host pointers.  The caller owns every buffer.  The library
+ *     allocates no memory and never synchronises the device: all work is
+ *     queued on `stream` (a cudaStream_t / CUstream handle; NULL is the
+ *     legacy default stream) and the call returns before it runs.
+ *   - Tensor and container buffers must be 16-byte aligned, scratch 256-byte
+ *     aligned.  Values are passed as raw bits (bf16 = 2 bytes, fp32 = 4).
+ *   - Argument, alignment and capacity errors are returned synchronously and
+ *     queue no work.  Corrupt containers are found on the device: the decode
+ *     calls clear *d_status (an int32 in device memory) in stream order and a
+ *     kernel stores a non-zero wc_status code there when it rejects a
+ *     container; read it after the stream has finished.  A decoder never
+ *     writes outside [d_out, d_out + out_cap) and never reads outside
+ *     [d_cont, d_cont + cont_bytes).
+ *   - WC_ERR_CUDA means a kernel launch failed; cudaGetLastError() in the
+ *     library's runtime was consumed and its text is available through
+ *     wc_last_error().
+ */
+#ifndef WC_H
+#define WC_H
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define WC_API __attribute__((visibility("default")))
+#else
+#define WC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    WC_OK = 0,
+    WC_ERR_INVALID_ARG = 1,
+    WC_ERR_CAPACITY = 2,
+    WC_ERR_CUDA = 3,
+    WC_ERR_CORRUPT = 4,
+    WC_ERR_UNSUPPORTED = 5
+} wc_status;
+
+typedef enum { WC_BF16 = 1, WC_FP32 = 2 } wc_dtype;
+
+/* Worst-case container size in bytes for n values of dtype: every chunk
+ * stored raw ("PTWM" Configuration table, compression_threshold: the coded
+ * form is only kept when it is smaller).  0 for an unknown dtype. */
+WC_API uint64_t wc_encode_bound(uint64_t n, int32_t dtype);
+
+/* Device scratch bytes wc_encode needs for n values (about 66 KiB per
+ * 65,536-value chunk plus a 6.25 KiB table area).  0 for an unknown dtype. */
+WC_API uint64_t wc_scratch_bytes(uint64_t n, int32_t dtype);
+
+/* Encode n values at d_in into a container at d_out.
+ *   d_in        n raw values (bf16 bits or fp32 bits), 16-byte aligned.
+ *   out_cap     bytes available at d_out; must be >= wc_encode_bound(n).
+ *   d_scratch   >= wc_scratch_bytes(n) bytes, 256-byte aligned; its content
+ *               on entry does not matter and is garbage on return.
+ *   d_out_size  device u64 receiving the container size in bytes.
+ * Steps ("PTWM" How it works 1-2; "SMEF" pass 3 and pass 4): plane split and
+ * per-tensor exponent histogram, the 12-bit table (sum 4096, every present
+ * exponent >= 1), 32-lane rANS per 65,536-value chunk with the raw fallback,
+ * exclusive scan of the chunk sizes into the offset table, and compaction.
+ * Returns WC_OK, WC_ERR_INVALID_ARG, WC_ERR_CAPACITY or WC_ERR_CUDA. */
+WC_API int32_t wc_encode(const void *d_in, uint64_t n, int32_t dtype, void *d_out,
+                  uint64_t out_cap, void *d_scratch, uint64_t scratch_cap,
+                  uint64_t *d_out_size, void *stream);
+
+/* Decode a whole container into d_out (n values of the container's dtype,
+ * 16-byte aligned, out_cap bytes).  The header is read on the device, so the
+ * host needs no copy of it; a container whose n values do not fit in out_cap
+ * is rejected on the device with WC_ERR_CAPACITY in *d_status.  Decoding
+ * inverts each chunk's rANS stream and re-merges the planes into the
+ * original bits ("PTWM" How it works; "SMEF" pass 3 merge_streams).
+ * Returns WC_OK, WC_ERR_INVALID_ARG or WC_ERR_CUDA; container problems go to
+ * *d_status (WC_ERR_CORRUPT / WC_ERR_CAPACITY). */
+WC_API int32_t wc_decode(const void *d_cont, uint64_t cont_bytes, void *d_out,
+                  uint64_t out_cap, int32_t *d_status, void *stream);
+
+/* Random access: decode only chunk k, i.e. values [65536 k, min(n, 65536 (k+1)))
+ * into d_out[0 ...] ("PTWM" Random access; "seedpack" README, chunks plus
+ * index).  k >= nc is reported as WC_ERR_INVALID_ARG in *d_status. */
+WC_API int32_t wc_decode_chunk(const void *d_cont, uint64_t cont_bytes, uint64_t k,
+                        void *d_out, uint64_t out_cap, int32_t *d_status,
+                        void *stream);
+
+/* Parse and check the fixed header at h_cont (host memory, >= 64 bytes;
+ * the offset table is checked too when it is present in the bytes given).
+ * Returns WC_OK or WC_ERR_CORRUPT / WC_ERR_INVALID_ARG. */
+WC_API int32_t wc_read_header(const void *h_cont, uint64_t bytes, uint64_t *n,
+                       int32_t *dtype, uint64_t *nchunks);
+
+/* Batched calls: many tensors in one launch per kernel (a whole model's
+ * weight set in a handful of launches).  The item arrays are host memory;
+ * the pointers inside are device pointers with the meaning and alignment of
+ * the single-tensor calls.  Every item is validated before anything is
+ * queued; on an error no work is queued.  Items may use any sizes, including
+ * n = 0. */
+typedef struct {
+    const void *in;       /* n values, 16-byte aligned                   */
+    uint64_t n;
+    int32_t dtype;        /* WC_BF16 or WC_FP32                          */
+    int32_t reserved;     /* must be 0                                   */
+    void *out;            /* container, out_cap >= wc_encode_bound(n)    */
+    uint64_t out_cap;
+    void *scratch;        /* >= wc_scratch_bytes(n), 256-byte aligned    */
+    uint64_t scratch_cap;
+    uint64_t *out_size;   /* device u64                                  */
+} wc_encode_item;
+
+typedef struct {
+    const void *cont;     /* container, 16-byte aligned                  */
+    uint64_t cont_bytes;
+    void *out;            /* decoded values, 16-byte aligned             */
+    uint64_t out_cap;
+} wc_decode_item;
+
+WC_API int32_t wc_encode_batch(const wc_encode_item *h_items, uint32_t count,
+                        void *stream);
+WC_API int32_t wc_decode_batch(const wc_decode_item *h_items, uint32_t count,
+                        int32_t *d_status, void *stream);
+
+/* Human-readable name of a wc_status code (static storage). */
+WC_API const char *wc_status_string(int32_t status);
+
+/* Text of the last CUDA error the library saw on this thread ("" if none). */
+WC_API const char *wc_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WC_H */
