@@ -1,0 +1,430 @@
+#!/usr/bin/env python3
+"""Throughput of the exponent-plane rANS codec on B200.
+
+One step = the whole hot path over the 0.6B-decoder-LM bf16 weight set
+(254 tensors, 596,042,752 values, 1.19 GB; see workloads.py): one batched
+encode (plane split + histogram + 12-bit table, 32-lane rANS with raw
+fallback, offset scan, compaction) and one batched decode (rANS + plane
+re-merge) of all tensors, inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).  `value` is uncompressed GB per second of
+round trip: bytes of all tensors / (encode time + decode time), summed over
+ranks (each rank codes its own copy of the set: weak scaling, no collective on
+the data path).  Timing: CUDA events on the launching stream over exactly K
+steps, barrier + synchronize on both sides, max over ranks.  The inputs
+(1.19 GB) exceed the 126 MB L2, so no flush is needed between steps.
+`--impl reference` times the CPU oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+WORKLOAD = 2
+HBM_FALLBACK_GBS = 6650.0
+METRIC = "decode & encode GB/s (uncompressed bytes) on 1 B200, % HBM roofline; ratio"
+WORKLOAD_NAME = ("bf16 tensor set shaped like a 0.6B decoder LM (hidden 1024, 28 layers, "
+                 "embedding 151936x1024, 57 norms): 254 tensors")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="oracle work budget of the CPU baseline sample (0: skip)")
+    ap.add_argument("--tensors", type=int, default=0,
+                    help="profiling only: use the first N tensors of the set (0: all)")
+    ap.add_argument("--no-e2e", action="store_true", help="profiling only: skip the e2e leg")
+    return ap.parse_args()
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def load_oracle():
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import oracle  # test infrastructure: the CPU baseline / reference arm only
+    oracle.build()
+    return oracle
+
+
+def oracle_round_trip_sample(oracle, budget_s: float, first_index: int = 0, max_tensors=None):
+    """Oracle encode + decode of workload tensors in order until the budget is
+    spent.  Returns (bytes, seconds, tensors, description)."""
+    specs = workloads.tensor_specs(WORKLOAD)
+    done_b, spent, count = 0, 0.0, 0
+    i = first_index
+    while True:
+        bits = workloads.generate_tensor(WORKLOAD, i % len(specs))
+        t0 = time.perf_counter()
+        cont = oracle.encode(bits)
+        back = oracle.decode(cont)
+        spent += time.perf_counter() - t0
+        assert np.array_equal(back, bits)
+        done_b += bits.nbytes
+        count += 1
+        i += 1
+        if spent >= budget_s or (max_tensors is not None and count >= max_tensors):
+            break
+    names = f"tensors {first_index}..{first_index + count - 1} of 254 ({specs[first_index].name} ..)"
+    return done_b, spent, count, f"{names}, {done_b / 1e6:.1f} MB, single thread"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 50):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", f"-lms={period_ms}"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def peak_hbm():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as fh:
+            return float(json.load(fh)["hbm_gbs"]), "of measured"
+    except (OSError, KeyError, ValueError):
+        return HBM_FALLBACK_GBS, "of fallback"
+
+
+def recorded_traffic(kernel: str, src_files) -> float | None:
+    """dram bytes per launch recorded by an ncu capture in profiles/, valid
+    only while the kernel's sources are unchanged."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_workload2.md")
+    if not os.path.exists(path):
+        return None
+    want = None
+    val = None
+    for line in open(path):
+        if line.startswith("source_sha256:"):
+            want = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_launch:"):
+            val = float(line.split(":", 1)[1].strip())
+    h = hashlib.sha256()
+    for f in src_files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    if want != h.hexdigest():
+        return None
+    return val
+
+
+def kernel_sources_sha(files) -> str:
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()
+
+
+DECODE_SOURCES = ["fp32_weight_compression_b200/csrc/k_decode.cu",
+                  "fp32_weight_compression_b200/csrc/wc_format.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_block.cuh"]
+CODER_SOURCES = ["fp32_weight_compression_b200/csrc/k_encode.cu",
+                 "fp32_weight_compression_b200/csrc/wc_format.cuh",
+                 "fp32_weight_compression_b200/csrc/wc_block.cuh"]
+
+
+# ---------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle as it stands, on the host cores,
+    rank 0 only.  Each step is a bounded sample of the workload: one tensor
+    (layer (step mod 28) k projection, 1024x1024 bf16)."""
+    if rank != 0:
+        return
+    oracle = load_oracle()
+    specs = workloads.tensor_specs(WORKLOAD)
+    k_idx = [i for i, s in enumerate(specs) if s.name.endswith(".k")]
+    data = {i: workloads.generate_tensor(WORKLOAD, i) for i in k_idx}
+    for s in range(args.warmup):
+        b = data[k_idx[s % len(k_idx)]]
+        oracle.decode(oracle.encode(b))
+    tot_b, tot_t = 0, 0.0
+    for s in range(args.steps):
+        b = data[k_idx[s % len(k_idx)]]
+        t0 = time.perf_counter()
+        c = oracle.encode(b)
+        back = oracle.decode(c)
+        tot_t += time.perf_counter() - t0
+        tot_b += b.nbytes
+        assert np.array_equal(back, b)
+    gbs = tot_b / tot_t / 1e9
+    sample = "per step one 1024x1024 bf16 tensor (layers.<step mod 28>.k) of the set, encode + decode"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u32", "data": "synthetic (seeded numpy PCG64)",
+        "config": {"workload": WORKLOAD_NAME, "sample": sample},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def e2e_leg(args, enc, sizes, outs, dev, dev_in, dev_out, host_in, stream, barrier, world):
+    """End-to-end through the public API with host buffers: every step copies
+    the inputs host->device, encodes, copies the containers device->host,
+    copies them back host->device, decodes, and copies the outputs
+    device->host (pinned host memory)."""
+    import torch
+    import torch.distributed as dist
+    from fp32_weight_compression_b200 import wc
+    if args.no_e2e:
+        return None, 0
+    # end-to-end through host buffers: H2D inputs -> encode -> D2H containers,
+    # H2D containers -> decode -> D2H outputs, every step
+    host_cont = torch.empty(max(sum((s + 255) // 256 * 256 for s in sizes), 256),
+                            dtype=torch.uint8, pin_memory=True)
+    coffs, o = [], 0
+    for s in sizes:
+        coffs.append(o)
+        o += (int(s) + 255) // 256 * 256
+    dev_cont = torch.empty(host_cont.numel(), dtype=torch.uint8, device=dev)
+    conts_packed = [dev_cont[co:co + int(s)] for co, s in zip(coffs, sizes)]
+    dec2 = wc.BatchDecoder(device=dev).prepare(conts_packed, outs)
+    host_out = torch.empty_like(host_in, pin_memory=True)
+    E = max(1, args.e2e_steps)
+    barrier()
+    torch.cuda.synchronize(dev)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        dev_in.copy_(host_in, non_blocking=True)
+        enc.run()
+        szs = enc.sizes.cpu().tolist()          # D2H of the sizes (sync)
+        for i, (s, co) in enumerate(zip(szs, coffs)):
+            host_cont[co:co + int(s)].copy_(enc.out[enc.out_offsets[i]:enc.out_offsets[i] + int(s)],
+                                            non_blocking=True)
+        dev_cont.copy_(host_cont, non_blocking=True)
+        dec2.run()
+        host_out.copy_(dev_out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    t_e2e = e0.elapsed_time(e1) / 1e3
+    dec2.check()
+    assert torch.equal(host_out, host_in), "end-to-end round trip is not bit-exact"
+    if world > 1:
+        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_e2e = tt.item()
+    return t_e2e, E
+
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    # Host-side work first (the oracle sample and the input draw use no GPU).
+    cpu_base = None
+    if rank == 0 and world == 1 and args.cpu_seconds > 0:
+        oracle = load_oracle()
+        b, t, cnt, desc = oracle_round_trip_sample(oracle, args.cpu_seconds)
+        cpu_base = {"value": b / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                    "sample": desc + f"; {t:.1f} s of encode + decode"}
+    specs = workloads.tensor_specs(WORKLOAD)
+    idx = list(range(len(specs) if args.tensors <= 0 else min(args.tensors, len(specs))))
+    specs = [specs[i] for i in idx]
+    arrs = workloads.generate_config(WORKLOAD, indices=idx,
+                                     workers=min(16, workloads.default_workers()))
+
+    import torch
+    import torch.distributed as dist
+    from fp32_weight_compression_b200 import wc
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev,
+                                timeout=__import__("datetime").timedelta(seconds=120))
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    # inputs: one pinned host buffer, one device buffer, per-tensor views
+    offs, off = [], 0
+    for a in arrs:
+        offs.append(off)
+        off = (off + a.nbytes + 255) // 256 * 256
+    total_in = sum(a.nbytes for a in arrs)
+    host_in = torch.empty(off, dtype=torch.uint8, pin_memory=True)
+    hv = host_in.numpy()
+    for a, o in zip(arrs, offs):
+        hv[o:o + a.nbytes] = a.view(np.uint8)
+    dev_in = host_in.to(dev)
+    ins = [dev_in[o:o + a.nbytes].view(torch.bfloat16).view(*s.shape)
+           for a, o, s in zip(arrs, offs, specs)]
+    dev_out = torch.empty_like(dev_in)
+    outs = [dev_out[o:o + a.nbytes].view(torch.bfloat16).view(*s.shape)
+            for a, o, s in zip(arrs, offs, specs)]
+
+    enc = wc.BatchEncoder([a.size for a in arrs], [torch.bfloat16] * len(arrs), device=dev)
+    enc.prepare(ins)
+    conts_cap = [enc.out[o:o + c] for o, c in zip(enc.out_offsets, enc.caps)]
+    dec = wc.BatchDecoder(device=dev).prepare(conts_cap, outs)
+    stream = torch.cuda.current_stream(dev)
+
+    # warm-up + a correctness check of the timed configuration
+    for _ in range(max(args.warmup, 1)):
+        enc.run()
+        dec.run()
+    torch.cuda.synchronize(dev)
+    dec.check()
+    assert torch.equal(dev_out, dev_in), "round trip is not bit-exact"
+    sizes = enc.sizes.cpu().tolist()
+    total_cont = int(sum(sizes))
+
+    # timed region
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    time.sleep(0.05)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        enc.run()
+        ev[k][1].record(stream)
+        dec.run()
+        ev[k][2].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    barrier()
+    t_total = start.elapsed_time(end) / 1e3
+    t_enc = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    dec.check()
+    if world > 1:
+        tt = torch.tensor([t_total, t_enc, t_dec], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        t_total, t_enc, t_dec = tt.tolist()
+
+    t_e2e, E = e2e_leg(args, enc, sizes, outs, dev, dev_in, dev_out, host_in, stream, barrier, world)
+
+    peak, peak_note = peak_hbm()
+    B = total_in
+    enc_bytes = B + total_cont     # read input, write container
+    dec_bytes = total_cont + B     # read container, write output
+    enc_gbs = B * K / t_enc / 1e9
+    dec_gbs = B * K / t_dec / 1e9
+    dec_achieved = dec_bytes * K / t_dec / 1e9
+    enc_achieved = enc_bytes * K / t_enc / 1e9
+    value = world * B * K / t_total / 1e9
+    traffic = recorded_traffic("k_decode", DECODE_SOURCES)
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": t_total / K * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "u32",
+        "data": "synthetic (seeded numpy PCG64; no checkpoints available)",
+        "config": {"workload": WORKLOAD_NAME, "tensors": len(arrs), "values": int(sum(a.size for a in arrs)),
+                   "input_bytes": B, "parallelism": f"replicas x{world} (one full set per GPU)",
+                   "l2": "inputs 1.19 GB > 126 MB L2, no flush"},
+        "encode": {"gbs": enc_gbs, "ms": t_enc / K * 1e3, "hbm_gbs": enc_achieved,
+                   "roofline_frac": enc_achieved / peak},
+        "decode": {"gbs": dec_gbs, "ms": t_dec / K * 1e3, "hbm_gbs": dec_achieved,
+                   "roofline_frac": dec_achieved / peak},
+        "ratio": total_cont / B,
+        "roofline": {"bound": "hbm", "kernel": "k_decode", "achieved": dec_achieved, "peak": peak,
+                     "unit": "GB/s", "frac": dec_achieved / peak, "traffic": traffic,
+                     "peak_note": peak_note,
+                     "algorithmic_bytes_per_launch": dec_bytes},
+        "e2e": None if t_e2e is None else {
+            "value": world * B * E / t_e2e / 1e9, "unit": "GB/s",
+            "h2d_bytes_per_step": B + total_cont, "d2h_bytes_per_step": total_cont + B + 8 * len(arrs),
+            "steps": E},
+        "gpu_launches": K * 5,
+        "clocks": clocks,
+        "cpu_baseline": cpu_base,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -2,18 +2,22 @@
 // re-merge of the planes into the original bits ("PTWM" How it works 1-2 run
 // backwards; "SMEF" pass3_streams.py merge_streams).
 //
-// Persistent grid.  Work is split into groups of kDecWarps consecutive chunks
-// of one tensor; a block takes groups blockIdx.x, + gridDim.x, ...  A block
-// stages its tensor's 4096-slot decoding table in shared memory (entry =
-// symbol | (slot - cum) << 8 | f << 20), then each warp decodes one chunk:
+// Persistent grid of 8-warp blocks.  Work is split into groups of 16
+// consecutive chunks of one tensor; a block takes groups blockIdx.x,
+// + gridDim.x, ...  The block stages its tensor's 4096-slot decoding table in
+// shared memory (entry = symbol | (slot - cum) << 8 | f << 20) and each warp
+// decodes two chunks.  When both are full 65,536-symbol coded chunks the warp
+// runs them in lock-step, so every lane carries two independent state chains;
+// otherwise it decodes them one after the other.  One decoding step:
 //   slot = x & 4095; e = tab[slot]; x = f (x >> 12) + (slot - cum);
 //   if x < 2^16: x = x << 16 | next word
-// where the lanes needing a word at a step take consecutive words in lane
-// order (__ballot_sync / __popc), from a per-warp shared-memory ring that
-// cp.async keeps filled with 16-byte loads of the chunk's word stream.  Every
-// 16 steps the warp has 512 exponent bytes; they are transposed through shared
-// memory so that each lane holds 16 consecutive ones, merged with the matching
-// raw-plane bytes, and written with 16-byte stores.
+// The lanes that need a word at a step take consecutive words in lane order
+// (__ballot_sync / __popc prefix), from a per-chunk 512-word shared-memory
+// ring that cp.async keeps filled with 16-byte loads of the chunk's word
+// stream.  Every 8 steps a chunk has 256 new exponent bytes; they are
+// transposed through shared memory so that each lane holds 8 consecutive
+// ones, merged with the matching raw-plane bytes, and written with one
+// 16-byte store (bf16) or two (fp32).
 //
 // Everything read from the container is checked before use (header fields
 // against the layout implied by n, the table sum, each chunk's offset pair and
@@ -26,19 +30,27 @@
 namespace wc {
 
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr uint32_t kRing = 1024;  // words per warp (4 units of 256)
-constexpr uint32_t kUnit = 256;   // words per cp.async round (32 lanes x 16 B)
+constexpr uint32_t kDecGroup = kDecWarps * 2;  // chunks per block group
+constexpr uint32_t kRing = 1024;                // words per chunk ring
+constexpr uint32_t kUnit = 256;                 // words per cp.async round (32 lanes x 16 B)
+constexpr uint32_t kHalf = 256;                 // values per half-group (8 steps)
 
 struct DecSmem {
-  uint32_t tab[kProbScale];                      // 16 KiB
-  __align__(16) uint16_t ring[kDecWarps][kRing];  // also holds freq/cum while a table is built
-  __align__(16) uint8_t tbuf[kDecWarps][kGroupValues];
+  uint32_t tab[kProbScale];                          // 16 KiB
+  __align__(16) uint16_t ring[kDecWarps][2][kRing];  // 32 KiB; freq/cum while a table is built
+  __align__(16) uint8_t tbuf[kDecWarps][2][kHalf];   // 4 KiB
   uint32_t gpre[kMaxItems + 1];
   uint64_t red[kDecThreads / 32 + 1];
   int cur_item;
   int tab_ok;
   int single_sym;
 };
+
+// The block's dynamic shared memory (a DecSmem).  Functions below reach it
+// through this symbol, not through pointer arguments, so that every access
+// compiles to a shared-memory instruction.
+extern __shared__ __align__(16) uint8_t dyn_smem[];
+__device__ __forceinline__ DecSmem &smem() { return *reinterpret_cast<DecSmem *>(dyn_smem); }
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) {
   atomicCAS(status, 0, code);
@@ -54,7 +66,7 @@ struct ItemView {
 };
 
 // Header checks that need no table or chunk data.
-__device__ ItemView view_item(const DecItem &it) {
+__device__ __noinline__ ItemView view_item(const DecItem &it) {
   ItemView v;
   v.ok = false;
   v.err = WC_ERR_CORRUPT;
@@ -95,279 +107,372 @@ __device__ ItemView view_item(const DecItem &it) {
   return v;
 }
 
-// ---------------------------------------------------------------------------
-// raw-plane bytes of 16 values and the merge
-template <int DT>
-struct Raw {
-  uint4 a;            // bf16: 16 sign+mantissa bytes; fp32: mantissa words 0..3
-  uint4 b, c;         // fp32: mantissa words 4..11
-  uint32_t sbits;     // fp32: 16 sign bits
+// A chunk's offset-table entry, checked.
+struct ChunkView {
+  bool ok, raw;
+  uint32_t nsym, len;
+  const uint8_t *pay;  // payload in the exponent section
+  uint8_t *out;        // output slot of the chunk's first value
 };
 
 template <int DT>
-__device__ __forceinline__ void load_raw(const uint8_t *cont, const Layout &L, uint64_t vg, uint32_t nv,
-                                         Raw<DT> &r) {
-  if (DT == WC_BF16) {
-    const uint8_t *s = cont + L.off_raw + vg;
-    if (nv == 16) {
-      r.a = ld_nc_v4(s);
-    } else {
-      uint32_t w[4] = {0, 0, 0, 0};
-      for (uint32_t j = 0; j < nv; j++) {
-        uint32_t byte = s[j];
-#pragma unroll
-        for (int q = 0; q < 4; q++)
-          if (q == int(j >> 2)) w[q] |= byte << (8 * (j & 3));
-      }
-      r.a = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-  } else {
-    const uint8_t *ss = cont + L.off_raw + vg / 8;
-    const uint8_t *ms = cont + L.off_mant + 3 * vg;
-    if (nv == 16) {
-      r.sbits = *reinterpret_cast<const uint16_t *>(ss);
-      r.a = ld_nc_v4(ms);
-      r.b = ld_nc_v4(ms + 16);
-      r.c = ld_nc_v4(ms + 32);
-    } else {
-      r.sbits = ss[0] | (nv > 8 ? uint32_t(ss[1]) << 8 : 0u);
-      uint32_t w[12];
-#pragma unroll
-      for (int q = 0; q < 12; q++) w[q] = 0;
-      for (uint32_t j = 0; j < 3 * nv; j++) {
-        uint32_t byte = ms[j];
-#pragma unroll
-        for (int q = 0; q < 12; q++)
-          if (q == int(j >> 2)) w[q] |= byte << (8 * (j & 3));
-      }
-      r.a = make_uint4(w[0], w[1], w[2], w[3]);
-      r.b = make_uint4(w[4], w[5], w[6], w[7]);
-      r.c = make_uint4(w[8], w[9], w[10], w[11]);
-    }
-  }
-}
-
-// bf16 pair from exponent word ew and sign+mantissa word sw (bytes 2h, 2h+1):
-// b = sm + 128 e + 255 (sm & 0x80)   (= s << 15 | e << 7 | m)
-__device__ __forceinline__ uint32_t merge_bf16_pair(uint32_t ew, uint32_t sw, int h) {
-  const uint32_t sel = h ? 0x4342u : 0x4140u;
-  const uint32_t eh = __byte_perm(ew, 0, sel);
-  const uint32_t sh = __byte_perm(sw, 0, sel);
-  return sh + (eh << 7) + (sh & 0x00800080u) * 255u;
-}
-
-template <int DT>
-__device__ __forceinline__ void merge_store(uint4 e, const Raw<DT> &r, uint8_t *dst, uint32_t nv) {
-  if (DT == WC_BF16) {
-    uint32_t o[8];
-    o[0] = merge_bf16_pair(e.x, r.a.x, 0); o[1] = merge_bf16_pair(e.x, r.a.x, 1);
-    o[2] = merge_bf16_pair(e.y, r.a.y, 0); o[3] = merge_bf16_pair(e.y, r.a.y, 1);
-    o[4] = merge_bf16_pair(e.z, r.a.z, 0); o[5] = merge_bf16_pair(e.z, r.a.z, 1);
-    o[6] = merge_bf16_pair(e.w, r.a.w, 0); o[7] = merge_bf16_pair(e.w, r.a.w, 1);
-    if (nv == 16) {
-      st_cs_v4(dst, make_uint4(o[0], o[1], o[2], o[3]));
-      st_cs_v4(dst + 16, make_uint4(o[4], o[5], o[6], o[7]));
-    } else {
-      uint16_t *d16 = reinterpret_cast<uint16_t *>(dst);
-      for (uint32_t j = 0; j < nv; j++) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int q = 0; q < 8; q++)
-          if (q == int(j >> 1)) word = o[q];
-        d16[j] = uint16_t(word >> (16 * (j & 1)));
-      }
-    }
-  } else {
-    const uint32_t mw[12] = {r.a.x, r.a.y, r.a.z, r.a.w, r.b.x, r.b.y, r.b.z, r.b.w,
-                             r.c.x, r.c.y, r.c.z, r.c.w};
-    const uint32_t ew[4] = {e.x, e.y, e.z, e.w};
-    uint32_t o[16];
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-      const uint32_t w0 = mw[3 * q], w1 = mw[3 * q + 1], w2 = mw[3 * q + 2];
-      const uint32_t m[4] = {w0 & 0x7FFFFFu, __funnelshift_r(w0, w1, 24) & 0x7FFFFFu,
-                             __funnelshift_r(w1, w2, 16) & 0x7FFFFFu, (w2 >> 8) & 0x7FFFFFu};
-#pragma unroll
-      for (int j = 0; j < 4; j++) {
-        const uint32_t ex = (ew[q] >> (8 * j)) & 0xFFu;
-        const uint32_t sg = (r.sbits >> (4 * q + j)) & 1u;
-        o[4 * q + j] = (sg << 31) | (ex << 23) | m[j];
-      }
-    }
-    if (nv == 16) {
-#pragma unroll
-      for (int q = 0; q < 4; q++)
-        st_cs_v4(dst + 16 * q, make_uint4(o[4 * q], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]));
-    } else {
-      uint32_t *d32 = reinterpret_cast<uint32_t *>(dst);
-#pragma unroll
-      for (int q = 0; q < 16; q++)
-        if (uint32_t(q) < nv) d32[q] = o[q];
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-template <int DT>
-__device__ void decode_chunk(DecSmem &s, const DecItem &it, const ItemView &v, uint64_t k,
-                             int32_t *status) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+__device__ __forceinline__ ChunkView view_chunk(const DecItem &it, const ItemView &v, uint64_t k) {
+  ChunkView c;
   const Layout &L = v.L;
   const uint8_t *cont = it.cont;
-  const uint32_t nsym = chunk_nsym(v.n, k);
+  c.nsym = chunk_nsym(v.n, k);
   const uint64_t *choff = reinterpret_cast<const uint64_t *>(cont + L.off_chunk_off);
   const uint32_t *chlen = reinterpret_cast<const uint32_t *>(cont + L.off_chunk_len);
   const uint64_t exp_bytes = reinterpret_cast<const uint64_t *>(cont)[6];
   const uint64_t o0 = choff[k], o1 = choff[k + 1];
-  const uint32_t len = chlen[k];
-  const bool raw = len == nsym;
-  const bool coded = len >= kStateBytes && len < nsym && (len & 1u) == 0;
-  bool ok = (raw || coded) && o0 <= o1 && o1 - o0 == round16(len) && o1 <= exp_bytes &&
-            (k != 0 || o0 == 0) && (k + 1 != L.nc || o1 == exp_bytes);
-  if (!ok) {
-    if (lane == 0) report(status, WC_ERR_CORRUPT);
-    return;
-  }
+  c.len = chlen[k];
+  c.raw = c.len == c.nsym;
+  const bool coded = c.len >= kStateBytes && c.len < c.nsym && (c.len & 1u) == 0;
+  c.ok = (c.raw || coded) && o0 <= o1 && o1 - o0 == round16(c.len) && o1 <= exp_bytes &&
+         (k != 0 || o0 == 0) && (k + 1 != L.nc || o1 == exp_bytes);
+  c.pay = cont + L.off_exp + o0;
   constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
-  const uint8_t *pay = cont + L.off_exp + o0;
-  uint8_t *outc = it.out + (k - v.first) * kChunk * elem;
-  const int ngroups = int((nsym + kGroupValues - 1) / kGroupValues);
-  auto lane_nv = [&](int G) -> uint32_t {
-    int64_t r = int64_t(nsym) - (int64_t(G) * kGroupValues + 16 * lane);
-    return r <= 0 ? 0u : (r >= 16 ? 16u : uint32_t(r));
-  };
+  c.out = it.out + (k - v.first) * kChunk * elem;
+  return c;
+}
 
-  if (raw || s.single_sym >= 0) {
-    uint4 ec = make_uint4(0, 0, 0, 0);
-    if (!raw) {
-      // single-symbol table: coding never moves a state and never emits a word
-      const uint32_t x = reinterpret_cast<const uint32_t *>(pay)[lane];
-      const bool good = __all_sync(0xffffffffu, x == kStateLow) && len == kStateBytes;
-      if (!good) {
-        if (lane == 0) report(status, WC_ERR_CORRUPT);
-        return;
-      }
-      const uint32_t b = uint32_t(s.single_sym) * 0x01010101u;
-      ec = make_uint4(b, b, b, b);
-    }
-    for (int G = 0; G < ngroups; G++) {
-      const uint32_t nv = lane_nv(G);
-      if (nv == 0) continue;
-      const uint32_t vl = uint32_t(G) * kGroupValues + 16 * lane;
-      Raw<DT> r;
-      load_raw<DT>(cont, L, k * kChunk + vl, nv, r);
-      const uint4 e = raw ? ld_nc_v4(pay + vl) : ec;  // raw payload is padded to 16
-      merge_store<DT>(e, r, outc + uint64_t(vl) * elem, nv);
-    }
-    return;
+// ---------------------------------------------------------------------------
+// Raw-plane bytes of 8 consecutive values and the merge.
+template <int DT>
+struct Raw8 {
+  uint2 a;        // bf16: 8 sign+mantissa bytes; fp32: mantissa bytes 0..7
+  uint2 b, c;     // fp32: mantissa bytes 8..23
+  uint32_t s;     // fp32: 8 sign bits
+};
+
+template <int DT>
+__device__ __forceinline__ void load_raw8(const uint8_t *cont, const Layout &L, uint64_t vg, Raw8<DT> &r) {
+  if (DT == WC_BF16) {
+    r.a = __ldg(reinterpret_cast<const uint2 *>(cont + L.off_raw + vg));
+  } else {
+    r.s = __ldg(cont + L.off_raw + vg / 8);
+    const uint2 *m = reinterpret_cast<const uint2 *>(cont + L.off_mant + 3 * vg);
+    r.a = __ldg(m);
+    r.b = __ldg(m + 1);
+    r.c = __ldg(m + 2);
   }
+}
 
-  // ---- rANS chunk
-  const uint32_t lt = lanemask_lt();
-  uint32_t x = reinterpret_cast<const uint32_t *>(pay)[lane];
-  const uint32_t w = (len - kStateBytes) >> 1;
-  const uint8_t *wsrc = pay + kStateBytes;
-  const uint32_t wavail = uint32_t(round16(len) - kStateBytes) >> 1;  // readable words
-  uint16_t *ring = s.ring[warp];
-  uint8_t *tb = s.tbuf[warp];
-  const uint32_t *tab = s.tab;
-  uint32_t req = 0, cons = 0;
+// 4 bf16 values from 4 exponent bytes and 4 sign+mantissa bytes, byte-parallel:
+// low byte = (sm & 0x7F) | (e & 1) << 7, high byte = e >> 1 | (sm & 0x80).
+__device__ __forceinline__ uint2 merge4_bf16(uint32_t e4, uint32_t s4) {
+  const uint32_t lo = (s4 & 0x7F7F7F7Fu) | ((e4 << 7) & 0x80808080u);
+  const uint32_t hi = ((e4 >> 1) & 0x7F7F7F7Fu) | (s4 & 0x80808080u);
+  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
 
-  auto issue = [&]() {
+// fp32 value j of 4 from 3 mantissa words: u = s << 31 | e << 23 | m
+__device__ __forceinline__ uint4 merge4_fp32(uint32_t e4, uint32_t w0, uint32_t w1, uint32_t w2,
+                                             uint32_t s4) {
+  const uint32_t m0 = w0 & 0x7FFFFFu;
+  const uint32_t m1 = __funnelshift_r(w0, w1, 24) & 0x7FFFFFu;
+  const uint32_t m2 = __funnelshift_r(w1, w2, 16) & 0x7FFFFFu;
+  const uint32_t m3 = (w2 >> 8) & 0x7FFFFFu;
+  uint4 o;
+  o.x = ((s4 & 1u) << 31) | ((e4 & 0xFFu) << 23) | m0;
+  o.y = ((s4 & 2u) << 30) | (((e4 >> 8) & 0xFFu) << 23) | m1;
+  o.z = ((s4 & 4u) << 29) | (((e4 >> 16) & 0xFFu) << 23) | m2;
+  o.w = ((s4 & 8u) << 28) | ((e4 >> 24) << 23) | m3;
+  return o;
+}
+
+// 8 values (exponents e8 = 8 bytes) -> output at dst (16-byte aligned).
+template <int DT>
+__device__ __forceinline__ void merge_store8(uint2 e8, const Raw8<DT> &r, uint8_t *dst) {
+  if (DT == WC_BF16) {
+    const uint2 p = merge4_bf16(e8.x, r.a.x);
+    const uint2 q = merge4_bf16(e8.y, r.a.y);
+    st_cs_v4(dst, make_uint4(p.x, p.y, q.x, q.y));
+  } else {
+    // mantissa words: a.x a.y b.x | b.y c.x c.y
+    st_cs_v4(dst, merge4_fp32(e8.x, r.a.x, r.a.y, r.b.x, r.s));
+    st_cs_v4(dst + 16, merge4_fp32(e8.y, r.b.y, r.c.x, r.c.y, r.s >> 4));
+  }
+}
+
+// One value, for ragged tails (scalar; no register arrays).
+template <int DT>
+__device__ __forceinline__ void merge_store1(uint32_t e, const uint8_t *cont, const Layout &L, uint64_t vg,
+                                             uint8_t *dst) {
+  if (DT == WC_BF16) {
+    const uint32_t sm = cont[L.off_raw + vg];
+    reinterpret_cast<uint16_t *>(dst)[0] =
+        uint16_t(((sm & 0x80u) << 8) | (e << 7) | (sm & 0x7Fu));
+  } else {
+    const uint32_t s = (cont[L.off_raw + vg / 8] >> (vg & 7)) & 1u;
+    const uint8_t *m = cont + L.off_mant + 3 * vg;
+    const uint32_t mant = (uint32_t(m[0]) | uint32_t(m[1]) << 8 | uint32_t(m[2]) << 16) & 0x7FFFFFu;
+    reinterpret_cast<uint32_t *>(dst)[0] = (s << 31) | (e << 23) | mant;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// The word ring of one chunk.
+struct Ring {
+  uint16_t *buf;
+  const uint8_t *src;  // first word
+  uint32_t avail;      // readable words (payload rounded to 16 bytes)
+  uint32_t req;        // words requested so far (multiple of kUnit)
+  uint32_t f1, f2;     // requested frontier after the call before last / before that
+
+  __device__ __forceinline__ void issue(int lane) {
     const uint32_t j0 = req + 8 * lane;
-    if (j0 < wavail) cp_async16(ring + (j0 & (kRing - 1)), wsrc + 2 * j0, 16);
-    else cp_async16(ring + (j0 & (kRing - 1)), wsrc, 0);  // zero fill, reads nothing
+    if (j0 < avail) cp_async16(buf + (j0 & (kRing - 1)), src + 2 * j0, 16);
+    else cp_async16(buf + (j0 & (kRing - 1)), src, 0);  // zero fill, reads nothing
     req += kUnit;
-  };
+  }
+  // Called once per half-group, followed by one commit.  Issues the next unit
+  // if it fits without overwriting unread words (a half-group consumes at
+  // most one unit, so the requested frontier stays >= cons + 513 words).
+  // Returns how many of the most recent commit groups may still be in flight
+  // while the words [cons, cons + 256) are already in shared memory: 3 if
+  // they were requested three calls ago or earlier, ..., 0 if only now.
+  __device__ __forceinline__ int top_up(uint32_t cons, int lane) {
+    const uint32_t f0 = req;  // frontier after the previous call
+    if (req < avail && req + kUnit <= (cons & ~(kUnit - 1)) + kRing) issue(lane);
+    const uint32_t need = min(cons + kHalf, avail);
+    const int depth = f2 >= need ? 3 : (f1 >= need ? 2 : (f0 >= need ? 1 : 0));
+    f2 = f1;
+    f1 = f0;
+    return depth;
+  }
+};
+
+__device__ __forceinline__ void cp_async_wait_depth(int d) {
+  if (d >= 3) cp_async_wait<3>();
+  else if (d == 2) cp_async_wait<2>();
+  else if (d == 1) cp_async_wait<1>();
+  else cp_async_wait<0>();
+}
+
+// One decoding step of one lane.
+__device__ __forceinline__ void dstep(uint32_t &x, uint32_t &cons, const uint32_t *tab,
+                                      const uint16_t *ring, uint8_t *tbp, uint32_t lt) {
+  const uint32_t e = tab[x & (kProbScale - 1)];
+  x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
+  const bool rn = x < kStateLow;
+  const uint32_t m = __ballot_sync(0xffffffffu, rn);
+  const uint32_t w = ring[(cons + __popc(m & lt)) & (kRing - 1)];
+  const uint32_t xr = __byte_perm(x, w, 0x1054);  // x << 16 | w
+  x = rn ? xr : x;
+  cons += __popc(m);
+  *tbp = uint8_t(e);
+}
+
+// Where a chunk's raw planes start, per dtype (value 0 of the chunk).
+struct RawPtrs {
+  const uint8_t *a;  // bf16: sign+mantissa bytes; fp32: mantissa bytes
+  const uint8_t *s;  // fp32: sign bits
+};
+
+template <int DT>
+__device__ __forceinline__ void load_raw8p(const RawPtrs &p, uint32_t vl, Raw8<DT> &r) {
+  if (DT == WC_BF16) {
+    r.a = __ldg(reinterpret_cast<const uint2 *>(p.a + vl));
+  } else {
+    r.s = __ldg(p.s + vl / 8);
+    const uint2 *m = reinterpret_cast<const uint2 *>(p.a + 3 * vl);
+    r.a = __ldg(m);
+    r.b = __ldg(m + 1);
+    r.c = __ldg(m + 2);
+  }
+}
+
+// Two full coded chunks in lock-step.  Everything arrives by value so that no
+// argument lives in local memory.
+template <int DT>
+__device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *payB, uint32_t lenA,
+                                         uint32_t lenB, RawPtrs rpA, RawPtrs rpB, uint8_t *outA,
+                                         uint8_t *outB, int32_t *status) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  DecSmem &s = smem();
+  const uint32_t *tab = s.tab;
+  uint16_t *ringA = s.ring[warp][0], *ringB = s.ring[warp][1];
+  uint8_t *tbA = s.tbuf[warp][0], *tbB = s.tbuf[warp][1];
+  const uint32_t lt = lanemask_lt();
+  constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
+  Ring ra{ringA, payA + kStateBytes, uint32_t(round16(lenA) - kStateBytes) >> 1, 0, 0, 0};
+  Ring rb{ringB, payB + kStateBytes, uint32_t(round16(lenB) - kStateBytes) >> 1, 0, 0, 0};
+  uint32_t xA = reinterpret_cast<const uint32_t *>(payA)[lane];
+  uint32_t xB = reinterpret_cast<const uint32_t *>(payB)[lane];
+  uint32_t cA = 0, cB = 0;
 #pragma unroll
-  for (int u = 0; u < int(kRing / kUnit); u++) issue();
+  for (int u = 0; u < int(kRing / kUnit); u++) {
+    ra.issue(lane);
+    rb.issue(lane);
+  }
   cp_async_commit();
 
-  for (int G = 0; G < ngroups; G++) {
-    const uint32_t before = req;
-    while (req < wavail && req + kUnit <= (cons & ~(kUnit - 1)) + kRing) issue();
+  constexpr uint32_t NH = kChunk / kHalf;
+  // raw planes are prefetched three half-groups ahead
+  Raw8<DT> nA, nB, mA, mB, oA, oB;
+  load_raw8p<DT>(rpA, 8 * lane, nA);
+  load_raw8p<DT>(rpB, 8 * lane, nB);
+  load_raw8p<DT>(rpA, kHalf + 8 * lane, mA);
+  load_raw8p<DT>(rpB, kHalf + 8 * lane, mB);
+  load_raw8p<DT>(rpA, 2 * kHalf + 8 * lane, oA);
+  load_raw8p<DT>(rpB, 2 * kHalf + 8 * lane, oB);
+  for (uint32_t h = 0; h < NH; h++) {
+    const int dA = ra.top_up(cA, lane);
+    const int dB = rb.top_up(cB, lane);
     cp_async_commit();
-    const uint32_t need = min(cons + kGroupValues, wavail);
-    if (before >= need) cp_async_wait<1>(); else cp_async_wait<0>();
+    cp_async_wait_depth(min(dA, dB));
     __syncwarp();
-
-    const uint32_t nv = lane_nv(G);
-    const uint32_t vl = uint32_t(G) * kGroupValues + 16 * lane;
-    Raw<DT> r;
-    if (nv) load_raw<DT>(cont, L, k * kChunk + vl, nv, r);
-
-    const uint32_t gbase = uint32_t(G) * kGroupValues;
-    if (gbase + kGroupValues <= nsym) {
+    const Raw8<DT> rA = nA, rB = nB;
+    nA = mA;
+    nB = mB;
+    mA = oA;
+    mB = oB;
+    if (h + 3 < NH) {
+      load_raw8p<DT>(rpA, (h + 3) * kHalf + 8 * lane, oA);
+      load_raw8p<DT>(rpB, (h + 3) * kHalf + 8 * lane, oB);
+    }
 #pragma unroll
-      for (int t = 0; t < int(kStepsPerGroup); t++) {
-        const uint32_t e = tab[x & (kProbScale - 1)];
-        x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
-        const bool rn = x < kStateLow;
-        const uint32_t m = __ballot_sync(0xffffffffu, rn);
-        if (rn) x = (x << 16) | ring[(cons + __popc(m & lt)) & (kRing - 1)];
-        cons += __popc(m);
-        tb[32 * t + lane] = uint8_t(e);
-      }
-    } else {
-      const int steps = int((nsym - gbase + 31) / 32);
-      for (int t = 0; t < steps; t++) {
-        const bool valid = gbase + 32 * t + lane < nsym;
-        uint32_t e = 0;
-        if (valid) {
-          e = tab[x & (kProbScale - 1)];
-          x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
-        }
-        const bool rn = valid && x < kStateLow;
-        const uint32_t m = __ballot_sync(0xffffffffu, rn);
-        if (rn) x = (x << 16) | ring[(cons + __popc(m & lt)) & (kRing - 1)];
-        cons += __popc(m);
-        tb[32 * t + lane] = uint8_t(e);
-      }
+    for (int t = 0; t < 8; t++) {
+      dstep(xA, cA, tab, ringA, tbA + 32 * t + lane, lt);
+      dstep(xB, cB, tab, ringB, tbB + 32 * t + lane, lt);
     }
     __syncwarp();
-    if (nv) {
-      const uint4 e = *reinterpret_cast<const uint4 *>(tb + 16 * lane);
-      merge_store<DT>(e, r, outc + uint64_t(vl) * elem, nv);
-    }
+    const uint2 eA = *reinterpret_cast<const uint2 *>(tbA + 8 * lane);
+    const uint2 eB = *reinterpret_cast<const uint2 *>(tbB + 8 * lane);
+    merge_store8<DT>(eA, rA, outA + (h * kHalf + 8 * lane) * elem);
+    merge_store8<DT>(eB, rB, outB + (h * kHalf + 8 * lane) * elem);
     __syncwarp();
   }
   cp_async_wait<0>();
   __syncwarp();
-  const bool good = __all_sync(0xffffffffu, x == kStateLow) && cons == w;
-  if (!good && lane == 0) report(status, WC_ERR_CORRUPT);
+  const uint32_t wA = (lenA - kStateBytes) >> 1, wB = (lenB - kStateBytes) >> 1;
+  if (!__all_sync(0xffffffffu, xA == kStateLow) || cA != wA) {
+    if (lane == 0) report(status, WC_ERR_CORRUPT);
+  }
+  if (!__all_sync(0xffffffffu, xB == kStateLow) || cB != wB) {
+    if (lane == 0) report(status, WC_ERR_CORRUPT);
+  }
+}
+
+// One chunk of any kind (raw, single-symbol, coded, ragged).
+template <int DT>
+__device__ __noinline__ void decode_one(const ItemView &v, const DecItem &it, const ChunkView &c,
+                           uint64_t k, int slot, int32_t *status) {
+  DecSmem &s = smem();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t lt = lanemask_lt();
+  const Layout &L = v.L;
+  constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
+  const uint64_t vg0 = k * kChunk;
+  const uint32_t nsym = c.nsym;
+  const uint32_t nhalf = (nsym + kHalf - 1) / kHalf;
+  uint8_t *tb = s.tbuf[warp][slot];
+
+  int mode = c.raw ? 0 : (s.single_sym >= 0 ? 1 : 2);
+  uint32_t x = 0, cons = 0;
+  Ring r{s.ring[warp][slot], c.pay + kStateBytes, 0, 0, 0, 0};
+  if (mode == 1) {
+    // single-symbol table: coding never moves a state and never emits a word
+    x = reinterpret_cast<const uint32_t *>(c.pay)[lane];
+    if (!__all_sync(0xffffffffu, x == kStateLow) || c.len != kStateBytes) {
+      if (lane == 0) report(status, WC_ERR_CORRUPT);
+      return;
+    }
+  } else if (mode == 2) {
+    x = reinterpret_cast<const uint32_t *>(c.pay)[lane];
+    r.avail = uint32_t(round16(c.len) - kStateBytes) >> 1;
+#pragma unroll
+    for (int u = 0; u < int(kRing / kUnit); u++) r.issue(lane);
+    cp_async_commit();
+  }
+  const uint32_t single_e = uint32_t(s.single_sym) * 0x01010101u;
+  for (uint32_t h = 0; h < nhalf; h++) {
+    const uint32_t hb = h * kHalf;
+    const bool full = hb + kHalf <= nsym;
+    if (mode == 2) {
+      const int d = r.top_up(cons, lane);
+      cp_async_commit();
+      cp_async_wait_depth(d);
+      __syncwarp();
+      if (full) {
+#pragma unroll
+        for (int t = 0; t < 8; t++) dstep(x, cons, s.tab, r.buf, tb + 32 * t + lane, lt);
+      } else {
+        const uint32_t steps = (nsym - hb + 31) / 32;
+        for (uint32_t t = 0; t < steps; t++) {
+          const bool valid = hb + 32 * t + lane < nsym;
+          uint32_t e = 0;
+          if (valid) {
+            e = s.tab[x & (kProbScale - 1)];
+            x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xFFFu);
+          }
+          const bool rn = valid && x < kStateLow;
+          const uint32_t m = __ballot_sync(0xffffffffu, rn);
+          const uint32_t w = r.buf[(cons + __popc(m & lt)) & (kRing - 1)];
+          if (rn) x = __byte_perm(x, w, 0x1054);
+          cons += __popc(m);
+          tb[32 * t + lane] = uint8_t(e);
+        }
+      }
+      __syncwarp();
+    }
+    const uint32_t vl = hb + 8 * lane;  // this lane's first value in the chunk
+    if (full) {
+      uint2 e8;
+      if (mode == 0) e8 = __ldg(reinterpret_cast<const uint2 *>(c.pay + vl));
+      else if (mode == 1) e8 = make_uint2(single_e, single_e);
+      else e8 = *reinterpret_cast<const uint2 *>(tb + 8 * lane);
+      Raw8<DT> rr;
+      load_raw8<DT>(it.cont, L, vg0 + vl, rr);
+      merge_store8<DT>(e8, rr, c.out + uint64_t(vl) * elem);
+    } else {
+      for (uint32_t j = 0; j < 8 && vl + j < nsym; j++) {
+        uint32_t e;
+        if (mode == 0) e = c.pay[vl + j];
+        else if (mode == 1) e = uint32_t(s.single_sym);
+        else e = tb[8 * lane + j];
+        merge_store1<DT>(e, it.cont, L, vg0 + vl + j, c.out + uint64_t(vl + j) * elem);
+      }
+    }
+    if (mode == 2) __syncwarp();
+  }
+  if (mode == 2) {
+    cp_async_wait<0>();
+    __syncwarp();
+    if (!__all_sync(0xffffffffu, x == kStateLow) || cons != ((c.len - kStateBytes) >> 1)) {
+      if (lane == 0) report(status, WC_ERR_CORRUPT);
+    }
+  }
 }
 
 // ---------------------------------------------------------------------------
 // Build the decoding table of item ii (whole block).
-__device__ void build_table(DecSmem &s, const DecItem &it, int ii, int32_t *status) {
+__device__ __noinline__ void build_table(const DecItem &it, int ii, int32_t *status) {
+  DecSmem &s = smem();
   const int tid = threadIdx.x;
   __syncthreads();  // all warps are done with the previous table and rings
-  uint32_t *sfreq = reinterpret_cast<uint32_t *>(&s.ring[0][0]);
+  uint32_t *sfreq = reinterpret_cast<uint32_t *>(&s.ring[0][0][0]);
   uint32_t *scum = sfreq + 256;
   const uint16_t *f16 = reinterpret_cast<const uint16_t *>(it.cont + kFreqOffset);
-  const uint32_t f0 = f16[2 * tid], f1 = f16[2 * tid + 1];
-  const uint64_t sum = block_sum_u64<kDecThreads>(f0 + f1, s.red);
-  const uint64_t ex = block_excl_scan_u64<kDecThreads>(f0 + f1, s.red);
-  uint64_t single = 0;
-  if (f0 == kProbScale) single = 2 * tid + 1;
-  if (f1 == kProbScale) single = 2 * tid + 2;
-  single = block_max_u64<kDecThreads>(single, s.red);
-  sfreq[2 * tid] = f0;
-  sfreq[2 * tid + 1] = f1;
-  scum[2 * tid] = uint32_t(ex);
-  scum[2 * tid + 1] = uint32_t(ex) + f0;
+  const uint32_t f = f16[tid];
+  const uint64_t sum = block_sum_u64<kDecThreads>(f, s.red);
+  const uint64_t cum = block_excl_scan_u64<kDecThreads>(f, s.red);
+  const uint64_t single = block_max_u64<kDecThreads>(f == kProbScale ? uint64_t(tid) + 1 : 0, s.red);
+  sfreq[tid] = f;
+  scum[tid] = uint32_t(cum);
   const bool ok = sum == kProbScale;
   __syncthreads();
   if (ok && single == 0) {
-    // thread t fills slots [32 t, 32 t + 32)
-    const uint32_t j0 = uint32_t(tid) * (kProbScale / kDecThreads);
+    constexpr uint32_t per = kProbScale / kDecThreads;  // 16 slots per thread
+    const uint32_t j0 = uint32_t(tid) * per;
     uint32_t lo = 0, hi = 255;  // last symbol with cum <= j0
     while (lo < hi) {
       uint32_t mid = (lo + hi + 1) >> 1;
       if (scum[mid] <= j0) lo = mid; else hi = mid - 1;
     }
     uint32_t sym = lo;
-    for (uint32_t j = j0; j < j0 + kProbScale / kDecThreads; j++) {
+    for (uint32_t j = j0; j < j0 + per; j++) {
       while (j >= scum[sym] + sfreq[sym]) sym++;
       s.tab[j] = sym | ((j - scum[sym]) << 8) | (sfreq[sym] << 20);
     }
@@ -381,26 +486,56 @@ __device__ void build_table(DecSmem &s, const DecItem &it, int ii, int32_t *stat
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kDecThreads, 8) k_decode(const __grid_constant__ DecParams p) {
-  __shared__ DecSmem s;
+template <int DT>
+__device__ __forceinline__ void decode_warp_chunks(const ItemView &v, const DecItem &it,
+                                                   uint64_t kA, uint64_t kend, int32_t *status) {
+  DecSmem &s = smem();
+  const int lane = threadIdx.x & 31;
+  if (kA >= kend) return;
+  const ChunkView A = view_chunk<DT>(it, v, kA);
+  const bool hasB = kA + 1 < kend;
+  ChunkView B;
+  if (hasB) B = view_chunk<DT>(it, v, kA + 1);
+  if (!A.ok || (hasB && !B.ok)) {
+    if (lane == 0) report(status, WC_ERR_CORRUPT);
+    return;
+  }
+  if (hasB && s.single_sym < 0 && !A.raw && !B.raw && A.nsym == kChunk && B.nsym == kChunk) {
+    const Layout &L = v.L;
+    const uint64_t vgA = kA * kChunk;
+    RawPtrs rpA, rpB;
+    if (DT == WC_BF16) {
+      rpA.a = it.cont + L.off_raw + vgA;
+      rpB.a = rpA.a + kChunk;
+      rpA.s = rpB.s = nullptr;
+    } else {
+      rpA.a = it.cont + L.off_mant + 3 * vgA;
+      rpB.a = rpA.a + 3 * kChunk;
+      rpA.s = it.cont + L.off_raw + vgA / 8;
+      rpB.s = rpA.s + kChunk / 8;
+    }
+    decode_pair<DT>(A.pay, B.pay, A.len, B.len, rpA, rpB, A.out, B.out, status);
+    return;
+  }
+  decode_one<DT>(v, it, A, kA, 0, status);
+  if (hasB) decode_one<DT>(v, it, B, kA + 1, 1, status);
+}
+
+__global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant__ DecParams p) {
+  DecSmem &s = smem();
   const int tid = threadIdx.x, warp = tid >> 5;
   int32_t *status = p.status;
 
-  // prologue: groups per item -> prefix (two items per thread)
-  uint32_t g2[2] = {0, 0};
-#pragma unroll
-  for (int h = 0; h < 2; h++) {
-    const uint32_t i = 2 * tid + h;
-    if (i < p.count) {
-      const ItemView v = view_item(p.items[i]);
-      if (v.ok) g2[h] = uint32_t((v.cnt + kDecWarps - 1) / kDecWarps);
-      else if (blockIdx.x == 0) report(status, v.err);
-    }
+  // prologue: groups per item -> prefix (one item per thread)
+  uint32_t g = 0;
+  if (uint32_t(tid) < p.count) {
+    const ItemView v = view_item(p.items[tid]);
+    if (v.ok) g = uint32_t((v.cnt + kDecGroup - 1) / kDecGroup);
+    else if (blockIdx.x == 0) report(status, v.err);
   }
-  const uint64_t ex = block_excl_scan_u64<kDecThreads>(g2[0] + g2[1], s.red);
-  if (2 * tid < kMaxItems) s.gpre[2 * tid] = uint32_t(ex);
-  if (2 * tid + 1 < kMaxItems) s.gpre[2 * tid + 1] = uint32_t(ex) + g2[0];
-  if (tid == kDecThreads - 1) s.gpre[kMaxItems] = uint32_t(ex) + g2[0] + g2[1];
+  const uint64_t ex = block_excl_scan_u64<kDecThreads>(g, s.red);
+  s.gpre[tid] = uint32_t(ex);
+  if (tid == kDecThreads - 1) s.gpre[kMaxItems] = uint32_t(ex) + g;
   if (tid == 0) s.cur_item = -1;
   __syncthreads();
   const uint32_t total = s.gpre[kMaxItems];
@@ -414,24 +549,30 @@ __global__ void __launch_bounds__(kDecThreads, 8) k_decode(const __grid_constant
     const int ii = int(lo);
     const DecItem &it = p.items[ii];
     const ItemView v = view_item(it);
-    if (ii != s.cur_item) build_table(s, it, ii, status);
+    if (ii != s.cur_item) build_table(it, ii, status);
     if (!s.tab_ok) continue;
-    const uint64_t k = v.first + uint64_t(grp - s.gpre[ii]) * kDecWarps + warp;
-    if (k >= v.first + v.cnt) continue;
-    if (v.dtype == WC_BF16) decode_chunk<WC_BF16>(s, it, v, k, status);
-    else decode_chunk<WC_FP32>(s, it, v, k, status);
+    const uint64_t kA = v.first + uint64_t(grp - s.gpre[ii]) * kDecGroup + 2 * warp;
+    const uint64_t kend = v.first + v.cnt;
+    if (v.dtype == WC_BF16) decode_warp_chunks<WC_BF16>(v, it, kA, kend, status);
+    else decode_warp_chunks<WC_FP32>(v, it, kA, kend, status);
   }
 }
 
+// Per device, before the first launch: allow the kernel its dynamic shared
+// memory and return how many blocks fit on one SM.
 int decode_blocks_per_sm() {
+  if (cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(sizeof(DecSmem))) != cudaSuccess)
+    return 0;
   int nb = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode, kDecThreads, 0) != cudaSuccess)
-    return 1;
-  return nb > 0 ? nb : 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_decode, kDecThreads, sizeof(DecSmem)) !=
+      cudaSuccess)
+    return 0;
+  return nb;
 }
 
 cudaError_t launch_decode(const DecParams &p, int grid, cudaStream_t s) {
-  k_decode<<<grid, kDecThreads, 0, s>>>(p);
+  k_decode<<<grid, kDecThreads, sizeof(DecSmem), s>>>(p);
   return cudaGetLastError();
 }
 

@@ -1,14 +1,17 @@
 // k_encode.cu -- encoder stage 2: plane split + rANS coding per chunk, and the
 // exclusive scan of chunk sizes into the container's offset table.
 //
-// One warp codes one 65,536-value chunk (one rANS state per lane, symbol i in
-// lane i mod 32).  The warp walks its chunk backwards in groups of 512 values
-// (16 steps): each lane loads its 16 consecutive values, writes their raw
-// planes straight into the container's raw section (bf16: the sign+mantissa
-// byte; fp32: sign bits and 3 little-endian mantissa bytes -- "PTWM" How it
-// works 1-2, "SMEF" pass3_streams.py), and parks their exponent bytes in shared
-// memory, where step t reads byte 32 t + lane.  Coding a symbol s with
-// frequency f from state x (12-bit table, L = 2^16, 16-bit words):
+// A block of 8 warps codes 16 consecutive chunks of one tensor, two per warp
+// (one rANS state per lane per chunk, symbol i in lane i mod 32).  Two full
+// bf16 chunks are coded in lock-step, so every lane carries two independent
+// state chains; other chunks are coded one at a time.  A warp walks a chunk
+// backwards in groups of 512 values (16 steps): each lane loads its 16
+// consecutive values, writes their raw planes straight into the container's
+// raw section (bf16: the sign+mantissa byte; fp32: sign bits and 3
+// little-endian mantissa bytes -- "PTWM" How it works 1-2, "SMEF"
+// pass3_streams.py), and parks their exponent bytes in shared memory, where
+// step t reads byte 32 t + lane.  Coding a symbol s with frequency f from
+// state x (12-bit table, L = 2^16, 16-bit words):
 //   if x >= f 2^20: emit x & 0xFFFF, x >>= 16;   x = (x / f) 4096 + x % f + cum_s
 // with x / f computed exactly as floor(x m / 2^64), m = ceil(2^64 / f) split in
 // two 32-bit halves (two integer multiply-adds; see publish_table).  The lanes
@@ -27,132 +30,93 @@ namespace wc {
 
 constexpr int kCoderThreads = kCoderWarps * 32;
 
-// 16 values of one lane, as raw 32-bit words (bf16: 8 words, fp32: 16 words).
-template <int DT>
-struct Vals {
-  uint32_t w[DT == WC_BF16 ? 8 : 16];
+// Per-block shared state of the coder, at namespace scope so that helper
+// functions reach it as shared memory (not through generic pointers).
+__shared__ uint4 s_tab[256];
+__shared__ uint32_t s_bias[256];
+__shared__ __align__(16) uint8_t s_ebuf[kCoderWarps][2][kGroupValues];
+
+// ---------------------------------------------------------------------------
+// 16 consecutive bf16 values (8 words) of one lane: exponents and raw plane.
+struct Bf16x16 {
+  uint4 a, b;
 };
 
-template <int DT>
-__device__ __forceinline__ void load_vals(const uint8_t *src, uint32_t nv, Vals<DT> &v) {
-  if (nv == 16) {
-#pragma unroll
-    for (int q = 0; q < (DT == WC_BF16 ? 2 : 4); q++) {
-      uint4 a = ld_nc_v4(src + 16 * q);
-      v.w[4 * q + 0] = a.x; v.w[4 * q + 1] = a.y; v.w[4 * q + 2] = a.z; v.w[4 * q + 3] = a.w;
-    }
-  } else {
-#pragma unroll
-    for (int q = 0; q < (DT == WC_BF16 ? 8 : 16); q++) v.w[q] = 0;
-    if (DT == WC_BF16) {
-      const uint16_t *s16 = reinterpret_cast<const uint16_t *>(src);
-      for (uint32_t j = 0; j < nv; j++) {
-        uint32_t b = s16[j];
-        // place value j in half (j & 1) of word j >> 1 (dynamic index kept in
-        // a small loop to stay in registers)
-#pragma unroll
-        for (int q = 0; q < 8; q++)
-          if (q == int(j >> 1)) v.w[q] |= b << (16 * (j & 1));
-      }
-    } else {
-      const uint32_t *s32 = reinterpret_cast<const uint32_t *>(src);
-#pragma unroll
-      for (int q = 0; q < 16; q++)
-        if (uint32_t(q) < nv) v.w[q] = s32[q];
-    }
-  }
+__device__ __forceinline__ uint32_t exp4_bf16(uint32_t w0, uint32_t w1) {
+  // bf16 word = [v1 : v0]; the exponent of a value is bits 7..14 of its half
+  return __byte_perm(w0 >> 7, w1 >> 7, 0x6420);
+}
+__device__ __forceinline__ uint32_t sm4_bf16(uint32_t w0, uint32_t w1) {
+  // sign+mantissa byte = (high byte & 0x80) | (low byte & 0x7F)
+  const uint32_t lo = __byte_perm(w0, w1, 0x6420);
+  const uint32_t hi = __byte_perm(w0, w1, 0x7531);
+  return (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
+}
+__device__ __forceinline__ uint4 exps_bf16(const Bf16x16 &v) {
+  return make_uint4(exp4_bf16(v.a.x, v.a.y), exp4_bf16(v.a.z, v.a.w), exp4_bf16(v.b.x, v.b.y),
+                    exp4_bf16(v.b.z, v.b.w));
+}
+__device__ __forceinline__ uint4 sms_bf16(const Bf16x16 &v) {
+  return make_uint4(sm4_bf16(v.a.x, v.a.y), sm4_bf16(v.a.z, v.a.w), sm4_bf16(v.b.x, v.b.y),
+                    sm4_bf16(v.b.z, v.b.w));
 }
 
-// Exponent bytes of the 16 values, packed little-endian into a uint4.
+// fp32: exponent byte = byte 3 of (u << 1)
+__device__ __forceinline__ uint32_t exp4_fp32(uint4 u) {
+  const uint32_t p01 = __byte_perm(u.x << 1, u.y << 1, 0x0073);
+  const uint32_t p23 = __byte_perm(u.z << 1, u.w << 1, 0x0073);
+  return __byte_perm(p01, p23, 0x5410);
+}
+// 4 mantissas (23 bits) as 12 little-endian bytes
+__device__ __forceinline__ uint3 mant4_fp32(uint4 u) {
+  const uint32_t m0 = u.x & 0x7FFFFFu, m1 = u.y & 0x7FFFFFu, m2 = u.z & 0x7FFFFFu, m3 = u.w & 0x7FFFFFu;
+  return make_uint3(m0 | (m1 << 24), (m1 >> 8) | (m2 << 16), (m2 >> 16) | (m3 << 8));
+}
+__device__ __forceinline__ uint32_t sign4_fp32(uint4 u) {
+  return (u.x >> 31) | ((u.y >> 31) << 1) | ((u.z >> 31) << 2) | ((u.w >> 31) << 3);
+}
+
+// Raw planes and exponents of one value (ragged tails only).
 template <int DT>
-__device__ __forceinline__ uint4 exponents(const Vals<DT> &v) {
-  uint32_t e[4];
+__device__ __forceinline__ uint32_t one_value(const uint8_t *in, uint64_t vg, uint8_t *out, const Layout &L) {
   if (DT == WC_BF16) {
-    // bf16 word = [v1 : v0]; exponent of a value = bits 7..14 of its half
-#pragma unroll
-    for (int q = 0; q < 4; q++)
-      e[q] = __byte_perm(v.w[2 * q] >> 7, v.w[2 * q + 1] >> 7, 0x6420);
+    const uint32_t b = reinterpret_cast<const uint16_t *>(in)[vg];
+    out[L.off_raw + vg] = uint8_t(((b >> 8) & 0x80u) | (b & 0x7Fu));
+    return (b >> 7) & 0xFFu;
   } else {
-    // fp32: exponent = byte 3 of (u << 1)
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-      uint32_t p01 = __byte_perm(v.w[4 * q] << 1, v.w[4 * q + 1] << 1, 0x0073);
-      uint32_t p23 = __byte_perm(v.w[4 * q + 2] << 1, v.w[4 * q + 3] << 1, 0x0073);
-      e[q] = __byte_perm(p01, p23, 0x5410);
-    }
-  }
-  return make_uint4(e[0], e[1], e[2], e[3]);
-}
-
-// Raw planes of the 16 values (value index vg within the tensor) into the
-// container's raw section.
-template <int DT>
-__device__ __forceinline__ void store_raw(uint8_t *out, const Layout &L, uint64_t vg, uint32_t nv,
-                                          const Vals<DT> &v) {
-  if (DT == WC_BF16) {
-    // sm byte = sign << 7 | mantissa = (high byte & 0x80) | (low byte & 0x7F)
-    uint32_t sm[4];
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-      uint32_t lo = __byte_perm(v.w[2 * q], v.w[2 * q + 1], 0x6420);
-      uint32_t hi = __byte_perm(v.w[2 * q], v.w[2 * q + 1], 0x7531);
-      sm[q] = (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
-    }
-    uint8_t *dst = out + L.off_raw + vg;
-    if (nv == 16) {
-      st_cs_v4(dst, make_uint4(sm[0], sm[1], sm[2], sm[3]));
-    } else {
-      for (uint32_t j = 0; j < nv; j++) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int q = 0; q < 4; q++)
-          if (q == int(j >> 2)) word = sm[q];
-        dst[j] = uint8_t(word >> (8 * (j & 3)));
-      }
-    }
-  } else {
-    uint32_t sbits = 0;
-#pragma unroll
-    for (int j = 0; j < 16; j++) sbits |= (v.w[j] >> 31) << j;
-    uint32_t mw[12];
-#pragma unroll
-    for (int q = 0; q < 4; q++) {
-      uint32_t m0 = v.w[4 * q] & 0x7FFFFFu, m1 = v.w[4 * q + 1] & 0x7FFFFFu;
-      uint32_t m2 = v.w[4 * q + 2] & 0x7FFFFFu, m3 = v.w[4 * q + 3] & 0x7FFFFFu;
-      mw[3 * q + 0] = m0 | (m1 << 24);
-      mw[3 * q + 1] = (m1 >> 8) | (m2 << 16);
-      mw[3 * q + 2] = (m2 >> 16) | (m3 << 8);
-    }
-    uint8_t *sdst = out + L.off_raw + vg / 8;
-    uint8_t *mdst = out + L.off_mant + 3 * vg;
-    if (nv == 16) {
-      *reinterpret_cast<uint16_t *>(sdst) = uint16_t(sbits);
-      st_cs_v4(mdst, make_uint4(mw[0], mw[1], mw[2], mw[3]));
-      st_cs_v4(mdst + 16, make_uint4(mw[4], mw[5], mw[6], mw[7]));
-      st_cs_v4(mdst + 32, make_uint4(mw[8], mw[9], mw[10], mw[11]));
-    } else {
-      // padding values are zero, so their sign bits are zero
-      sdst[0] = uint8_t(sbits);
-      if (nv > 8) sdst[1] = uint8_t(sbits >> 8);
-      for (uint32_t j = 0; j < 3 * nv; j++) {
-        uint32_t word = 0;
-#pragma unroll
-        for (int q = 0; q < 12; q++)
-          if (q == int(j >> 2)) word = mw[q];
-        mdst[j] = uint8_t(word >> (8 * (j & 3)));
-      }
-    }
+    const uint32_t u = reinterpret_cast<const uint32_t *>(in)[vg];
+    const uint32_t m = u & 0x7FFFFFu;
+    uint8_t *md = out + L.off_mant + 3 * vg;
+    md[0] = uint8_t(m);
+    md[1] = uint8_t(m >> 8);
+    md[2] = uint8_t(m >> 16);
+    return (u >> 23) & 0xFFu;
   }
 }
 
-// One coding step of one lane.  CHECK: the step may hold lanes past nsym.
-template <bool CHECK>
-__device__ __forceinline__ void code_step(uint32_t &x, uint32_t &tail, uint16_t *win16,
-                                          const uint4 *tab, const uint32_t *bias, uint32_t s,
-                                          bool valid, uint32_t lt) {
+// ---------------------------------------------------------------------------
+// One coding step of one lane.
+__device__ __forceinline__ void cstep(uint32_t &x, uint32_t &tail, uint16_t *win16, const uint4 *tab,
+                                      const uint32_t *bias, uint32_t s, uint32_t lt) {
   const uint4 te = tab[s];
   const uint32_t bi = bias[s];
-  const bool emit = (CHECK ? valid : true) && x > te.z;
+  const bool emit = x > te.z;
+  const uint32_t m = __ballot_sync(0xffffffffu, emit);
+  tail -= __popc(m);
+  if (emit) win16[tail + __popc(m & lt)] = uint16_t(x);
+  x = emit ? (x >> 16) : x;
+  const uint32_t qlo = __umulhi(x, te.x);
+  const uint64_t prod = uint64_t(x) * te.y + qlo;
+  x = x + uint32_t(prod >> 32) * te.w + bi;
+}
+
+// A step that may hold lanes past nsym.
+__device__ __forceinline__ void cstep_checked(uint32_t &x, uint32_t &tail, uint16_t *win16,
+                                              const uint4 *tab, const uint32_t *bias, uint32_t s,
+                                              bool valid, uint32_t lt) {
+  const uint4 te = tab[s];
+  const uint32_t bi = bias[s];
+  const bool emit = valid && x > te.z;
   const uint32_t m = __ballot_sync(0xffffffffu, emit);
   const uint32_t k = __popc(m);
   if (emit) {
@@ -160,85 +124,162 @@ __device__ __forceinline__ void code_step(uint32_t &x, uint32_t &tail, uint16_t 
     x >>= 16;
   }
   tail -= k;
-  if (!CHECK || valid) {
+  if (valid) {
     const uint32_t qlo = __umulhi(x, te.x);
     const uint64_t prod = uint64_t(x) * te.y + qlo;
-    const uint32_t q = uint32_t(prod >> 32);
-    x = x + q * te.w + bi;
+    x = x + uint32_t(prod >> 32) * te.w + bi;
   }
 }
 
-template <int DT>
-__device__ __forceinline__ void code_chunk(const EncItem &it, const Layout &L, uint64_t k,
-                                           const uint4 *tab, const uint32_t *bias, uint8_t *ebuf) {
+struct CoderOut {
+  uint32_t *lens;
+  uint8_t *win0;  // window of chunk 0 of the tensor
+};
+
+__device__ __forceinline__ void finish_chunk(const CoderOut &co, uint64_t k, uint32_t nsym, uint32_t x,
+                                             uint32_t tail, bool bail, int lane) {
+  const uint32_t w = kWinWords - tail;
+  const bool raw = bail || (kStateBytes + 2 * w >= nsym);
+  const uint32_t len = raw ? nsym : kStateBytes + 2 * w;
+  if (!raw) reinterpret_cast<uint32_t *>(co.win0 + k * kWin)[lane] = x;
+  if (lane == 0) co.lens[k] = len;
+}
+
+// Two full bf16 chunks kA, kA + 1 in lock-step.
+__device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
+                               const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
-  const uint64_t nc = L.nc;
+  const uint64_t vgA = kA * kChunk, vgB = vgA + kChunk;
+  const uint16_t *in16 = reinterpret_cast<const uint16_t *>(it.in);
+  uint16_t *wA = reinterpret_cast<uint16_t *>(co.win0 + kA * kWin);
+  uint16_t *wB = reinterpret_cast<uint16_t *>(co.win0 + (kA + 1) * kWin);
+  uint32_t xA = kStateLow, xB = kStateLow, tA = kWinWords, tB = kWinWords;
+  bool bailA = false, bailB = false;
+  constexpr int NG = int(kChunk / kGroupValues);
+
+  Bf16x16 cA, cB, nA, nB;
+  {
+    const uint64_t o = uint64_t(NG - 1) * kGroupValues + 16 * lane;
+    cA.a = ld_nc_v4(in16 + vgA + o); cA.b = ld_nc_v4(in16 + vgA + o + 8);
+    cB.a = ld_nc_v4(in16 + vgB + o); cB.b = ld_nc_v4(in16 + vgB + o + 8);
+  }
+  for (int G = NG - 1; G >= 0; --G) {
+    const uint64_t o = uint64_t(G) * kGroupValues + 16 * lane;
+    st_cs_v4(it.out + L.off_raw + vgA + o, sms_bf16(cA));
+    st_cs_v4(it.out + L.off_raw + vgB + o, sms_bf16(cB));
+    *reinterpret_cast<uint4 *>(ebA + 16 * lane) = exps_bf16(cA);
+    *reinterpret_cast<uint4 *>(ebB + 16 * lane) = exps_bf16(cB);
+    if (G > 0) {
+      const uint64_t on = o - kGroupValues;
+      nA.a = ld_nc_v4(in16 + vgA + on); nA.b = ld_nc_v4(in16 + vgA + on + 8);
+      nB.a = ld_nc_v4(in16 + vgB + on); nB.b = ld_nc_v4(in16 + vgB + on + 8);
+    }
+    __syncwarp();
+    if (!bailA && !bailB) {
+#pragma unroll
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t) {
+        cstep(xA, tA, wA, tab, bias, ebA[32 * t + lane], lt);
+        cstep(xB, tB, wB, tab, bias, ebB[32 * t + lane], lt);
+      }
+    } else if (!bailA) {
+#pragma unroll 4
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep(xA, tA, wA, tab, bias, ebA[32 * t + lane], lt);
+    } else if (!bailB) {
+#pragma unroll 4
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep(xB, tB, wB, tab, bias, ebB[32 * t + lane], lt);
+    }
+    if (kStateBytes + 2 * (kWinWords - tA) >= kChunk) bailA = true;
+    if (kStateBytes + 2 * (kWinWords - tB) >= kChunk) bailB = true;
+    __syncwarp();
+    cA = nA;
+    cB = nB;
+  }
+  finish_chunk(co, kA, kChunk, xA, tA, bailA, lane);
+  finish_chunk(co, kA + 1, kChunk, xB, tB, bailB, lane);
+}
+
+// Any single chunk (either dtype, possibly ragged).
+template <int DT>
+__device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64_t k, int slot,
+                                      const CoderOut &co) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint4 *tab = s_tab;
+  const uint32_t *bias = s_bias;
+  uint8_t *eb = s_ebuf[warp][slot];
+  const uint32_t lt = lanemask_lt();
   const uint32_t nsym = chunk_nsym(it.n, k);
   const int ngroups = int((nsym + kGroupValues - 1) / kGroupValues);
-  constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
-  const uint8_t *src = it.in + (k * kChunk) * elem;
-  uint8_t *win = it.scratch + scratch_win_offset(nc) + k * kWin;
-  uint16_t *win16 = reinterpret_cast<uint16_t *>(win);
-
-  uint32_t x = kStateLow;
-  uint32_t tail = kWinWords;
+  const uint64_t vg0 = k * kChunk;
+  uint16_t *win16 = reinterpret_cast<uint16_t *>(co.win0 + k * kWin);
+  uint32_t x = kStateLow, tail = kWinWords;
   bool bail = false;
 
-  auto lane_nv = [&](int G) -> uint32_t {
-    int64_t r = int64_t(nsym) - (int64_t(G) * kGroupValues + 16 * lane);
-    return r <= 0 ? 0u : (r >= 16 ? 16u : uint32_t(r));
-  };
-
-  Vals<DT> cur, nxt;
-  {
-    const int G = ngroups - 1;
-    const uint32_t nv = lane_nv(G);
-    if (nv) load_vals<DT>(src + (uint64_t(G) * kGroupValues + 16 * lane) * elem, nv, cur);
-    else {
-#pragma unroll
-      for (int q = 0; q < (DT == WC_BF16 ? 8 : 16); q++) cur.w[q] = 0;
-    }
-  }
   for (int G = ngroups - 1; G >= 0; --G) {
-    const uint32_t nv = lane_nv(G);
-    const uint64_t vg = k * kChunk + uint64_t(G) * kGroupValues + 16 * lane;
-    if (nv) store_raw<DT>(it.out, L, vg, nv, cur);
-    uint4 e = exponents<DT>(cur);
-    *reinterpret_cast<uint4 *>(ebuf + 16 * lane) = e;
-    if (G > 0) load_vals<DT>(src + (uint64_t(G - 1) * kGroupValues + 16 * lane) * elem, 16, nxt);
+    const uint32_t gb = uint32_t(G) * kGroupValues;
+    const uint32_t vl = gb + 16 * lane;  // lane's first value in the chunk
+    const uint64_t vg = vg0 + vl;
+    if (vl + 16 <= nsym) {
+      uint4 e;
+      if (DT == WC_BF16) {
+        const uint16_t *p = reinterpret_cast<const uint16_t *>(it.in) + vg;
+        Bf16x16 v;
+        v.a = ld_nc_v4(p);
+        v.b = ld_nc_v4(p + 8);
+        st_cs_v4(it.out + L.off_raw + vg, sms_bf16(v));
+        e = exps_bf16(v);
+      } else {
+        const uint32_t *p = reinterpret_cast<const uint32_t *>(it.in) + vg;
+        const uint4 u0 = ld_nc_v4(p), u1 = ld_nc_v4(p + 4), u2 = ld_nc_v4(p + 8), u3 = ld_nc_v4(p + 12);
+        e = make_uint4(exp4_fp32(u0), exp4_fp32(u1), exp4_fp32(u2), exp4_fp32(u3));
+        const uint32_t sb = sign4_fp32(u0) | (sign4_fp32(u1) << 4) | (sign4_fp32(u2) << 8) |
+                            (sign4_fp32(u3) << 12);
+        *reinterpret_cast<uint16_t *>(it.out + L.off_raw + vg / 8) = uint16_t(sb);
+        const uint3 m0 = mant4_fp32(u0), m1 = mant4_fp32(u1), m2 = mant4_fp32(u2), m3 = mant4_fp32(u3);
+        uint8_t *md = it.out + L.off_mant + 3 * vg;
+        st_cs_v4(md, make_uint4(m0.x, m0.y, m0.z, m1.x));
+        st_cs_v4(md + 16, make_uint4(m1.y, m1.z, m2.x, m2.y));
+        st_cs_v4(md + 32, make_uint4(m2.z, m3.x, m3.y, m3.z));
+      }
+      *reinterpret_cast<uint4 *>(eb + 16 * lane) = e;
+    } else {
+      // ragged tail: value by value; exponent bytes past nsym are zero
+      for (uint32_t j = 0; j < 16; j++) {
+        uint32_t e = 0;
+        if (vl + j < nsym) e = one_value<DT>(it.in, vg + j, it.out, L);
+        eb[16 * lane + j] = uint8_t(e);
+      }
+      if (DT == WC_FP32) {
+        for (uint32_t bsel = 0; bsel < 2; bsel++) {
+          if (vl + 8 * bsel >= nsym) break;
+          uint32_t byte = 0;
+          for (uint32_t j = 0; j < 8 && vl + 8 * bsel + j < nsym; j++)
+            byte |= (reinterpret_cast<const uint32_t *>(it.in)[vg + 8 * bsel + j] >> 31) << j;
+          it.out[L.off_raw + (vg + 8 * bsel) / 8] = uint8_t(byte);
+        }
+      }
+    }
     __syncwarp();
     if (!bail) {
-      const uint32_t gbase = uint32_t(G) * kGroupValues;
-      if (gbase + kGroupValues <= nsym) {
-#pragma unroll
-        for (int t = kStepsPerGroup - 1; t >= 0; --t)
-          code_step<false>(x, tail, win16, tab, bias, ebuf[32 * t + lane], true, lt);
+      if (gb + kGroupValues <= nsym) {
+#pragma unroll 4
+        for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+          cstep(x, tail, win16, tab, bias, eb[32 * t + lane], lt);
       } else {
-        const int steps = int((nsym - gbase + 31) / 32);
-        for (int t = steps - 1; t >= 0; --t) {
-          const bool valid = gbase + 32 * t + lane < nsym;
-          code_step<true>(x, tail, win16, tab, bias, ebuf[32 * t + lane], valid, lt);
-        }
+        const int steps = int((nsym - gb + 31) / 32);
+        for (int t = steps - 1; t >= 0; --t)
+          cstep_checked(x, tail, win16, tab, bias, eb[32 * t + lane], gb + 32 * t + lane < nsym, lt);
       }
       if (kStateBytes + 2 * (kWinWords - tail) >= nsym) bail = true;
     }
     __syncwarp();
-    if (G > 0) cur = nxt;
   }
-
-  const uint32_t w = kWinWords - tail;
-  const bool raw = bail || (kStateBytes + 2 * w >= nsym);
-  const uint32_t len = raw ? nsym : kStateBytes + 2 * w;
-  if (!raw) reinterpret_cast<uint32_t *>(win)[lane] = x;
-  uint32_t *lens = reinterpret_cast<uint32_t *>(it.scratch + kScrLen);
-  if (lane == 0) lens[k] = len;
+  finish_chunk(co, k, nsym, x, tail, bail, lane);
 }
 
 __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constant__ EncParams p) {
-  __shared__ uint4 s_tab[256];
-  __shared__ uint32_t s_bias[256];
-  __shared__ __align__(16) uint8_t s_ebuf[kCoderWarps][kGroupValues];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t b = blockIdx.x;
   const EncItem &it = p.items[find_item_by_block(p, b)];
@@ -249,19 +290,31 @@ __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constan
   s_bias[tid] = reinterpret_cast<const uint32_t *>(it.scratch + kScrBias)[tid];
   __syncthreads();
 
-  const uint64_t k = uint64_t(b - it.block_base) * kCoderWarps + warp;
-  if (k >= L.nc) return;
-  if (dtype == WC_BF16) code_chunk<WC_BF16>(it, L, k, s_tab, s_bias, s_ebuf[warp]);
-  else code_chunk<WC_FP32>(it, L, k, s_tab, s_bias, s_ebuf[warp]);
+  const uint64_t kA = uint64_t(b - it.block_base) * kCoderChunks + 2 * warp;
+  if (kA >= L.nc) return;
+  const bool hasB = kA + 1 < L.nc;
+  CoderOut co{reinterpret_cast<uint32_t *>(it.scratch + kScrLen), it.scratch + scratch_win_offset(L.nc)};
+  if (dtype == WC_BF16) {
+    if (hasB && chunk_nsym(it.n, kA + 1) == kChunk)
+      code_pair_bf16(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+    else {
+      code_one<WC_BF16>(it, L, kA, 0, co);
+      if (hasB) code_one<WC_BF16>(it, L, kA + 1, 1, co);
+    }
+  } else {
+    code_one<WC_FP32>(it, L, kA, 0, co);
+    if (hasB) code_one<WC_FP32>(it, L, kA + 1, 1, co);
+  }
 
   // last warp of the tensor: offset table and the rest of the header
+  const uint32_t done = hasB ? 2u : 1u;
   __threadfence();
   uint32_t prev = 0;
-  if (lane == 0) prev = atomicAdd(reinterpret_cast<uint32_t *>(it.scratch + kScrCtr) + 1, 1u);
+  if (lane == 0) prev = atomicAdd(reinterpret_cast<uint32_t *>(it.scratch + kScrCtr) + 1, done);
   prev = __shfl_sync(0xffffffffu, prev, 0);
-  if (prev != uint32_t(L.nc - 1)) return;
+  if (prev + done != uint32_t(L.nc)) return;
   __threadfence();
-  const uint32_t *lens = reinterpret_cast<const uint32_t *>(it.scratch + kScrLen);
+  const uint32_t *lens = co.lens;
   uint64_t *choff = reinterpret_cast<uint64_t *>(it.out + L.off_chunk_off);
   uint32_t *chlen = reinterpret_cast<uint32_t *>(it.out + L.off_chunk_len);
   uint64_t run = 0;

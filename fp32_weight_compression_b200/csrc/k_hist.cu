@@ -4,7 +4,7 @@
 //  k_prep   one block per tensor: clears the tensor's scratch counters and
 //           writes the fixed header fields and the zero padding of the
 //           container (everything that depends on n alone).
-//  k_hist   one block per 65,536-value chunk: reads the chunk's values as
+//  k_hist   one block per tile of up to 4 chunks: reads the values as
 //           integers (a NaN payload is never touched as a float), counts the
 //           8-bit exponents ("PTWM" How it works 1-2: after the bit reorder the
 //           exponent is a whole byte; "SMEF" pass3_streams.py) into a
@@ -145,59 +145,75 @@ __device__ void publish_table(const EncItem &it, uint64_t *red) {
   }
 }
 
+// 16 values' worth of exponent counts (one group) from raw words.
+__device__ __forceinline__ void count_group_bf16(uint32_t *sh, int lane, uint4 a, uint4 b) {
+  count_bf16_word(sh, lane, a.x); count_bf16_word(sh, lane, a.y);
+  count_bf16_word(sh, lane, a.z); count_bf16_word(sh, lane, a.w);
+  count_bf16_word(sh, lane, b.x); count_bf16_word(sh, lane, b.y);
+  count_bf16_word(sh, lane, b.z); count_bf16_word(sh, lane, b.w);
+}
+__device__ __forceinline__ void count_quad_fp32(uint32_t *sh, int lane, uint4 a) {
+  count_fp32_word(sh, lane, a.x); count_fp32_word(sh, lane, a.y);
+  count_fp32_word(sh, lane, a.z); count_fp32_word(sh, lane, a.w);
+}
+
+// One block counts a tile of up to kHistChunks chunks of one tensor.  Each
+// thread takes 16-value groups tid, tid + 512, ... and keeps four groups of
+// loads in flight.
 __global__ void __launch_bounds__(kHistThreads, 2) k_hist(const __grid_constant__ EncParams p) {
   __shared__ __align__(16) uint32_t sh[256 * 32];  // [exponent][lane]
   __shared__ uint64_t red[kHistThreads / 32 + 1];
   __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31;
-  const uint32_t g = blockIdx.x;
-  const EncItem &it = p.items[find_item_by_chunk(p, g)];
-  const uint64_t k = g - it.chunk_base;
-  const uint32_t nsym = chunk_nsym(it.n, k);
+  const uint32_t b = blockIdx.x;
+  const EncItem &it = p.items[find_item_by_hist(p, b)];
+  const uint64_t tile = b - it.hist_base;
+  const uint64_t v0 = tile * kHistChunks * kChunk;
+  const uint64_t left = it.n - v0;
+  const uint32_t count = uint32_t(left < uint64_t(kHistChunks) * kChunk ? left : uint64_t(kHistChunks) * kChunk);
   const uint64_t nc = num_chunks(it.n);
+  const uint32_t nfull = count / 16;  // full 16-value groups
 
   for (int i = tid; i < 256 * 32 / 4; i += kHistThreads)
     reinterpret_cast<uint4 *>(sh)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
 
-  // Each thread takes 16-value groups tid, tid + 512, ... (8 per full chunk).
   if (it.dtype == WC_BF16) {
-    const uint16_t *src = reinterpret_cast<const uint16_t *>(it.in) + k * kChunk;
-#pragma unroll 4
-    for (int j = 0; j < int(kChunk / 16 / kHistThreads); j++) {
-      const uint32_t v0 = (uint32_t(j) * kHistThreads + tid) * 16;
-      if (v0 + 16 <= nsym) {
-        uint4 a = ld_nc_v4(src + v0);
-        uint4 b = ld_nc_v4(src + v0 + 8);
-        count_bf16_word(sh, lane, a.x); count_bf16_word(sh, lane, a.y);
-        count_bf16_word(sh, lane, a.z); count_bf16_word(sh, lane, a.w);
-        count_bf16_word(sh, lane, b.x); count_bf16_word(sh, lane, b.y);
-        count_bf16_word(sh, lane, b.z); count_bf16_word(sh, lane, b.w);
-      } else if (v0 < nsym) {
-        for (uint32_t v = v0; v < nsym; v++)
-          atomicAdd(&sh[((uint32_t(src[v] >> 7) & 0xFFu) << 5) | lane], 1u);
-      }
+    const uint16_t *src = reinterpret_cast<const uint16_t *>(it.in) + v0;
+    uint32_t g = tid;
+    for (; g + 3 * kHistThreads < nfull; g += 4 * kHistThreads) {
+      uint4 a0 = ld_nc_v4(src + 16 * g), b0 = ld_nc_v4(src + 16 * g + 8);
+      uint4 a1 = ld_nc_v4(src + 16 * (g + kHistThreads)), b1 = ld_nc_v4(src + 16 * (g + kHistThreads) + 8);
+      uint4 a2 = ld_nc_v4(src + 16 * (g + 2 * kHistThreads)), b2 = ld_nc_v4(src + 16 * (g + 2 * kHistThreads) + 8);
+      uint4 a3 = ld_nc_v4(src + 16 * (g + 3 * kHistThreads)), b3 = ld_nc_v4(src + 16 * (g + 3 * kHistThreads) + 8);
+      count_group_bf16(sh, lane, a0, b0);
+      count_group_bf16(sh, lane, a1, b1);
+      count_group_bf16(sh, lane, a2, b2);
+      count_group_bf16(sh, lane, a3, b3);
     }
+    for (; g < nfull; g += kHistThreads) count_group_bf16(sh, lane, ld_nc_v4(src + 16 * g), ld_nc_v4(src + 16 * g + 8));
+    if (g == nfull)  // the thread whose next group is the ragged tail
+      for (uint32_t v = 16 * nfull; v < count; v++)
+        atomicAdd(&sh[((uint32_t(src[v] >> 7) & 0xFFu) << 5) | lane], 1u);
   } else {
-    const uint32_t *src = reinterpret_cast<const uint32_t *>(it.in) + k * kChunk;
-#pragma unroll 2
-    for (int j = 0; j < int(kChunk / 16 / kHistThreads); j++) {
-      const uint32_t v0 = (uint32_t(j) * kHistThreads + tid) * 16;
-      if (v0 + 16 <= nsym) {
-        uint4 a = ld_nc_v4(src + v0), b = ld_nc_v4(src + v0 + 4);
-        uint4 c = ld_nc_v4(src + v0 + 8), d = ld_nc_v4(src + v0 + 12);
-        count_fp32_word(sh, lane, a.x); count_fp32_word(sh, lane, a.y);
-        count_fp32_word(sh, lane, a.z); count_fp32_word(sh, lane, a.w);
-        count_fp32_word(sh, lane, b.x); count_fp32_word(sh, lane, b.y);
-        count_fp32_word(sh, lane, b.z); count_fp32_word(sh, lane, b.w);
-        count_fp32_word(sh, lane, c.x); count_fp32_word(sh, lane, c.y);
-        count_fp32_word(sh, lane, c.z); count_fp32_word(sh, lane, c.w);
-        count_fp32_word(sh, lane, d.x); count_fp32_word(sh, lane, d.y);
-        count_fp32_word(sh, lane, d.z); count_fp32_word(sh, lane, d.w);
-      } else if (v0 < nsym) {
-        for (uint32_t v = v0; v < nsym; v++) count_fp32_word(sh, lane, src[v]);
-      }
+    const uint32_t *src = reinterpret_cast<const uint32_t *>(it.in) + v0;
+    uint32_t g = tid;
+    for (; g + kHistThreads < nfull; g += 2 * kHistThreads) {
+      const uint32_t *s0 = src + 16 * g, *s1 = src + 16 * (g + kHistThreads);
+      uint4 a0 = ld_nc_v4(s0), b0 = ld_nc_v4(s0 + 4), c0 = ld_nc_v4(s0 + 8), d0 = ld_nc_v4(s0 + 12);
+      uint4 a1 = ld_nc_v4(s1), b1 = ld_nc_v4(s1 + 4), c1 = ld_nc_v4(s1 + 8), d1 = ld_nc_v4(s1 + 12);
+      count_quad_fp32(sh, lane, a0); count_quad_fp32(sh, lane, b0);
+      count_quad_fp32(sh, lane, c0); count_quad_fp32(sh, lane, d0);
+      count_quad_fp32(sh, lane, a1); count_quad_fp32(sh, lane, b1);
+      count_quad_fp32(sh, lane, c1); count_quad_fp32(sh, lane, d1);
     }
+    for (; g < nfull; g += kHistThreads) {
+      const uint32_t *s0 = src + 16 * g;
+      count_quad_fp32(sh, lane, ld_nc_v4(s0)); count_quad_fp32(sh, lane, ld_nc_v4(s0 + 4));
+      count_quad_fp32(sh, lane, ld_nc_v4(s0 + 8)); count_quad_fp32(sh, lane, ld_nc_v4(s0 + 12));
+    }
+    if (g == nfull)
+      for (uint32_t v = 16 * nfull; v < count; v++) count_fp32_word(sh, lane, src[v]);
   }
   __syncthreads();
 
@@ -208,12 +224,13 @@ __global__ void __launch_bounds__(kHistThreads, 2) k_hist(const __grid_constant_
     for (int j = 0; j < 32; j++) sum += sh[(tid << 5) | ((j + tid) & 31)];
     if (sum) atomicAdd(reinterpret_cast<unsigned long long *>(&ghist[tid]),
                        static_cast<unsigned long long>(sum));
+    __threadfence();
   }
-  __threadfence();
   __syncthreads();
   if (tid == 0) {
     uint32_t *ctr = reinterpret_cast<uint32_t *>(it.scratch + kScrCtr);
-    s_last = (atomicAdd(&ctr[0], 1u) == uint32_t(nc - 1));
+    const uint32_t nb = uint32_t((nc + kHistChunks - 1) / kHistChunks);
+    s_last = (atomicAdd(&ctr[0], 1u) == nb - 1);
   }
   __syncthreads();
   if (!s_last) return;
@@ -227,8 +244,8 @@ cudaError_t launch_prep(const EncParams &p, cudaStream_t s) {
 }
 
 cudaError_t launch_hist(const EncParams &p, cudaStream_t s) {
-  if (p.total_chunks == 0) return cudaSuccess;
-  k_hist<<<p.total_chunks, kHistThreads, 0, s>>>(p);
+  if (p.total_hist_blocks == 0) return cudaSuccess;
+  k_hist<<<p.total_hist_blocks, kHistThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -4,10 +4,10 @@
 // Encode, per launch of up to kMaxItems tensors (all on `stream`):
 //   k_prep     header fields + scratch counters            (1 block / tensor)
 //   k_hist     exponent histogram -> 12-bit table          (1 block / chunk)
-//   k_coder    raw planes + rANS per chunk + offset scan   (1 warp / chunk)
+//   k_coder    raw planes + rANS per chunk + offset scan   (1 warp / 2 chunks)
 //   k_compact  payloads into the exponent section          (1 block / chunk)
 // Decode, per launch of up to kMaxItems containers:
-//   k_decode   persistent grid, one warp per chunk
+//   k_decode   persistent grid, one warp per 2 chunks
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -52,7 +52,12 @@ DeviceInfo device_info(int32_t *err) {
       *err = cuda_fail(e, "cudaDeviceGetAttribute");
       return DeviceInfo{};
     }
-    cache[dev].dec_blocks_per_sm = wc::decode_blocks_per_sm();
+    const int nb = wc::decode_blocks_per_sm();
+    if (nb <= 0) {
+      *err = cuda_fail(cudaGetLastError(), "decoder set-up");
+      return DeviceInfo{};
+    }
+    cache[dev].dec_blocks_per_sm = nb;
     cache[dev].sms = sms;
   }
   *err = WC_OK;
@@ -111,7 +116,7 @@ int32_t wc_encode_batch(const wc_encode_item *items, uint32_t count, void *strea
     const uint32_t cnt = count - b0 < wc::kMaxItems ? count - b0 : wc::kMaxItems;
     memset(&P, 0, sizeof(P));
     P.count = cnt;
-    uint64_t chunks = 0, blocks = 0;
+    uint64_t chunks = 0, blocks = 0, hblocks = 0;
     for (uint32_t i = 0; i < cnt; i++) {
       const wc_encode_item &src = items[b0 + i];
       wc::EncItem &d = P.items[i];
@@ -123,13 +128,16 @@ int32_t wc_encode_batch(const wc_encode_item *items, uint32_t count, void *strea
       d.dtype = uint32_t(src.dtype);
       d.chunk_base = uint32_t(chunks);
       d.block_base = uint32_t(blocks);
+      d.hist_base = uint32_t(hblocks);
       const uint64_t nc = wc::num_chunks(src.n);
       chunks += nc;
-      blocks += (nc + wc::kCoderWarps - 1) / wc::kCoderWarps;
+      blocks += (nc + wc::kCoderChunks - 1) / wc::kCoderChunks;
+      hblocks += (nc + wc::kHistChunks - 1) / wc::kHistChunks;
       if (chunks >= (uint64_t(1) << 31)) return WC_ERR_UNSUPPORTED;
     }
     P.total_chunks = uint32_t(chunks);
     P.total_coder_blocks = uint32_t(blocks);
+    P.total_hist_blocks = uint32_t(hblocks);
     cudaError_t e;
     if ((e = wc::launch_prep(P, s)) != cudaSuccess) return cuda_fail(e, "k_prep");
     if ((e = wc::launch_hist(P, s)) != cudaSuccess) return cuda_fail(e, "k_hist");

@@ -98,14 +98,14 @@ struct EncItem {
   uint32_t chunk_base;  // first global chunk index of this item in the launch
   uint32_t block_base;  // first coder block of this item in the launch
   uint32_t dtype;
-  uint32_t pad;
+  uint32_t hist_base;   // first histogram block of this item in the launch
 };
 
 struct EncParams {
   uint32_t count;
   uint32_t total_chunks;
   uint32_t total_coder_blocks;
-  uint32_t pad;
+  uint32_t total_hist_blocks;
   EncItem items[kMaxItems];
 };
 
@@ -125,10 +125,13 @@ struct DecParams {
   DecItem items[kMaxItems];
 };
 
-// Encoder coder blocks: 8 warps, one chunk each, all of one tensor.
+// Histogram blocks: one tile of up to 4 chunks of one tensor.
+constexpr uint32_t kHistChunks = 4;
+// Encoder coder blocks: 8 warps, two chunks each, all of one tensor.
 constexpr uint32_t kCoderWarps = 8;
-// Decoder blocks: 4 warps, one chunk each, all of one tensor.
-constexpr uint32_t kDecWarps = 4;
+constexpr uint32_t kCoderChunks = 2 * kCoderWarps;
+// Decoder blocks: 8 warps, two chunks each, all of one tensor.
+constexpr uint32_t kDecWarps = 8;
 
 // Host launchers (one per kernel file).
 cudaError_t launch_prep(const EncParams &p, cudaStream_t s);
@@ -156,6 +159,15 @@ __device__ __forceinline__ uint32_t find_item_by_block(const EncParams &p, uint3
   while (lo < hi) {
     uint32_t mid = (lo + hi + 1) >> 1;
     if (p.items[mid].block_base <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint32_t find_item_by_hist(const EncParams &p, uint32_t b) {
+  uint32_t lo = 0, hi = p.count - 1;
+  while (lo < hi) {
+    uint32_t mid = (lo + hi + 1) >> 1;
+    if (p.items[mid].hist_base <= b) lo = mid; else hi = mid - 1;
   }
   return lo;
 }

@@ -178,8 +178,23 @@ class BatchEncoder:
             sizes = self.sizes.cpu().tolist()
         return [self.out[o:o + int(s)] for o, s in zip(self.out_offsets, sizes)]
 
+    def prepare(self, tensors):
+        """Bind input tensors once; run() then encodes them without any
+        per-call Python work beyond one library call."""
+        self._bind([_flat(t) for t in tensors])
+        self._bound = list(tensors)
+        return self
+
+    def run(self, stream=None):
+        _check(load().wc_encode_batch(self._items, len(self.numels), _stream(stream)),
+               "wc_encode_batch")
+        return self
+
     def encode(self, tensors, stream=None):
-        flats = [_flat(t) for t in tensors]
+        self._bind([_flat(t) for t in tensors])
+        return self.run(stream)
+
+    def _bind(self, flats):
         if len(flats) != len(self.numels):
             raise ValueError("tensor count does not match the encoder")
         key = tuple(t.data_ptr() for t in flats)
@@ -199,8 +214,6 @@ class BatchEncoder:
                 it.scratch_cap = scratch_bytes(self.numels[i], self.codes[i])
                 it.out_size = base_z + 8 * i
             self._key = key
-        _check(load().wc_encode_batch(self._items, len(flats), _stream(stream)), "wc_encode_batch")
-        return self
 
 
 class BatchDecoder:
@@ -213,7 +226,22 @@ class BatchDecoder:
         self._items = None
         self._key = None
 
+    def prepare(self, conts, outs, cont_bytes=None):
+        self._bind(conts, outs, cont_bytes)
+        self._n = len(conts)
+        return self
+
+    def run(self, stream=None):
+        _check(load().wc_decode_batch(self._items, self._n, self.status.data_ptr(),
+                                      _stream(stream)), "wc_decode_batch")
+        return self
+
     def decode(self, conts, outs, cont_bytes=None, stream=None):
+        self._bind(conts, outs, cont_bytes)
+        self._n = len(conts)
+        return self.run(stream)
+
+    def _bind(self, conts, outs, cont_bytes):
         if cont_bytes is None:
             cont_bytes = [c.numel() for c in conts]
         key = tuple(c.data_ptr() for c in conts) + tuple(o.data_ptr() for o in outs) + tuple(cont_bytes)
@@ -227,9 +255,6 @@ class BatchDecoder:
                 it.out = of.data_ptr() if of.numel() else None
                 it.out_cap = of.numel() * of.element_size()
             self._key = key
-        _check(load().wc_decode_batch(self._items, len(conts), self.status.data_ptr(),
-                                      _stream(stream)), "wc_decode_batch")
-        return self
 
     def check(self):
         """Synchronising read of the device status; raises on a bad container."""
