@@ -283,6 +283,32 @@ __device__ __forceinline__ void load_raw8p(const RawPtrs &p, uint32_t vl, Raw8<D
   }
 }
 
+// One decoding step of two independent chains (chunks A and B), written
+// interleaved operation by operation so that each warp always has an
+// independent instruction to issue while the other chain waits.
+__device__ __forceinline__ void dstep2(uint32_t &xA, uint32_t &cA, uint32_t &xB, uint32_t &cB,
+                                       const uint32_t *tab, const uint16_t *ringA,
+                                       const uint16_t *ringB, uint8_t *tbpA, uint8_t *tbpB,
+                                       uint32_t lt) {
+  const uint32_t eA = tab[xA & (kProbScale - 1)];
+  const uint32_t eB = tab[xB & (kProbScale - 1)];
+  const uint32_t sA = xA >> kProbBits, sB = xB >> kProbBits;
+  xA = (eA >> 20) * sA + ((eA >> 8) & 0xFFFu);
+  xB = (eB >> 20) * sB + ((eB >> 8) & 0xFFFu);
+  const bool rA = xA < kStateLow, rB = xB < kStateLow;
+  const uint32_t mA = __ballot_sync(0xffffffffu, rA);
+  const uint32_t mB = __ballot_sync(0xffffffffu, rB);
+  const uint32_t wA = ringA[(cA + __popc(mA & lt)) & (kRing - 1)];
+  const uint32_t wB = ringB[(cB + __popc(mB & lt)) & (kRing - 1)];
+  cA += __popc(mA);
+  cB += __popc(mB);
+  *tbpA = uint8_t(eA);
+  *tbpB = uint8_t(eB);
+  const uint32_t yA = __byte_perm(xA, wA, 0x1054), yB = __byte_perm(xB, wB, 0x1054);
+  xA = rA ? yA : xA;
+  xB = rB ? yB : xB;
+}
+
 // Two full coded chunks in lock-step.  Everything arrives by value so that no
 // argument lives in local memory.
 template <int DT>
@@ -309,40 +335,39 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   cp_async_commit();
 
   constexpr uint32_t NH = kChunk / kHalf;
-  // raw planes are prefetched three half-groups ahead
-  Raw8<DT> nA, nB, mA, mB, oA, oB;
-  load_raw8p<DT>(rpA, 8 * lane, nA);
-  load_raw8p<DT>(rpB, 8 * lane, nB);
-  load_raw8p<DT>(rpA, kHalf + 8 * lane, mA);
-  load_raw8p<DT>(rpB, kHalf + 8 * lane, mB);
-  load_raw8p<DT>(rpA, 2 * kHalf + 8 * lane, oA);
-  load_raw8p<DT>(rpB, 2 * kHalf + 8 * lane, oB);
-  for (uint32_t h = 0; h < NH; h++) {
-    const int dA = ra.top_up(cA, lane);
-    const int dB = rb.top_up(cB, lane);
-    cp_async_commit();
-    cp_async_wait_depth(min(dA, dB));
-    __syncwarp();
-    const Raw8<DT> rA = nA, rB = nB;
-    nA = mA;
-    nB = mB;
-    mA = oA;
-    mB = oB;
-    if (h + 3 < NH) {
-      load_raw8p<DT>(rpA, (h + 3) * kHalf + 8 * lane, oA);
-      load_raw8p<DT>(rpB, (h + 3) * kHalf + 8 * lane, oB);
-    }
+  // Raw planes are prefetched S half-groups ahead into S register sets used
+  // in rotation; the loop is unrolled S times so each set is consumed where it
+  // was loaded (no register moves that would wait on loads in flight).
+  constexpr int S = 2;
+  Raw8<DT> pa[S], pb[S];
 #pragma unroll
-    for (int t = 0; t < 8; t++) {
-      dstep(xA, cA, tab, ringA, tbA + 32 * t + lane, lt);
-      dstep(xB, cB, tab, ringB, tbB + 32 * t + lane, lt);
+  for (int j = 0; j < S; j++) {
+    load_raw8p<DT>(rpA, j * kHalf + 8 * lane, pa[j]);
+    load_raw8p<DT>(rpB, j * kHalf + 8 * lane, pb[j]);
+  }
+  for (uint32_t h0 = 0; h0 < NH; h0 += S) {
+#pragma unroll
+    for (int j = 0; j < S; j++) {
+      const uint32_t h = h0 + j;
+      const int dA = ra.top_up(cA, lane);
+      const int dB = rb.top_up(cB, lane);
+      cp_async_commit();
+      cp_async_wait_depth(min(dA, dB));
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < 8; t++)
+        dstep2(xA, cA, xB, cB, tab, ringA, ringB, tbA + 32 * t + lane, tbB + 32 * t + lane, lt);
+      __syncwarp();
+      const uint2 eA = *reinterpret_cast<const uint2 *>(tbA + 8 * lane);
+      const uint2 eB = *reinterpret_cast<const uint2 *>(tbB + 8 * lane);
+      merge_store8<DT>(eA, pa[j], outA + (h * kHalf + 8 * lane) * elem);
+      merge_store8<DT>(eB, pb[j], outB + (h * kHalf + 8 * lane) * elem);
+      if (h + S < NH) {
+        load_raw8p<DT>(rpA, (h + S) * kHalf + 8 * lane, pa[j]);
+        load_raw8p<DT>(rpB, (h + S) * kHalf + 8 * lane, pb[j]);
+      }
+      __syncwarp();
     }
-    __syncwarp();
-    const uint2 eA = *reinterpret_cast<const uint2 *>(tbA + 8 * lane);
-    const uint2 eB = *reinterpret_cast<const uint2 *>(tbB + 8 * lane);
-    merge_store8<DT>(eA, rA, outA + (h * kHalf + 8 * lane) * elem);
-    merge_store8<DT>(eB, rB, outB + (h * kHalf + 8 * lane) * elem);
-    __syncwarp();
   }
   cp_async_wait<0>();
   __syncwarp();

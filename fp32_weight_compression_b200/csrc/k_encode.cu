@@ -110,6 +110,27 @@ __device__ __forceinline__ void cstep(uint32_t &x, uint32_t &tail, uint16_t *win
   x = x + uint32_t(prod >> 32) * te.w + bi;
 }
 
+// One coding step of two chains, interleaved operation by operation.
+__device__ __forceinline__ void cstep2(uint32_t &xA, uint32_t &tA, uint16_t *wA, uint32_t sA,
+                                       uint32_t &xB, uint32_t &tB, uint16_t *wB, uint32_t sB,
+                                       const uint4 *tab, const uint32_t *bias, uint32_t lt) {
+  const uint4 eA = tab[sA], eB = tab[sB];
+  const uint32_t bA = bias[sA], bB = bias[sB];
+  const bool pA = xA > eA.z, pB = xB > eB.z;
+  const uint32_t mA = __ballot_sync(0xffffffffu, pA);
+  const uint32_t mB = __ballot_sync(0xffffffffu, pB);
+  tA -= __popc(mA);
+  tB -= __popc(mB);
+  if (pA) wA[tA + __popc(mA & lt)] = uint16_t(xA);
+  if (pB) wB[tB + __popc(mB & lt)] = uint16_t(xB);
+  xA = pA ? (xA >> 16) : xA;
+  xB = pB ? (xB >> 16) : xB;
+  const uint32_t qA = __umulhi(xA, eA.x), qB = __umulhi(xB, eB.x);
+  const uint64_t rA = uint64_t(xA) * eA.y + qA, rB = uint64_t(xB) * eB.y + qB;
+  xA = xA + uint32_t(rA >> 32) * eA.w + bA;
+  xB = xB + uint32_t(rB >> 32) * eB.w + bB;
+}
+
 // A step that may hold lanes past nsym.
 __device__ __forceinline__ void cstep_checked(uint32_t &x, uint32_t &tail, uint16_t *win16,
                                               const uint4 *tab, const uint32_t *bias, uint32_t s,
@@ -178,10 +199,8 @@ __device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, 
     __syncwarp();
     if (!bailA && !bailB) {
 #pragma unroll
-      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t) {
-        cstep(xA, tA, wA, tab, bias, ebA[32 * t + lane], lt);
-        cstep(xB, tB, wB, tab, bias, ebB[32 * t + lane], lt);
-      }
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep2(xA, tA, wA, ebA[32 * t + lane], xB, tB, wB, ebB[32 * t + lane], tab, bias, lt);
     } else if (!bailA) {
 #pragma unroll 4
       for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
