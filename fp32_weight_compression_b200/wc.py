@@ -26,7 +26,10 @@ _ELEM = {BF16: 2, FP32: 4}
 EXPORTS = (
     "wc_encode_bound", "wc_scratch_bytes", "wc_encode", "wc_decode", "wc_decode_chunk",
     "wc_read_header", "wc_encode_batch", "wc_decode_batch", "wc_status_string", "wc_last_error",
+    "wc_encode_noalloc",
 )
+# Library-held scratch of wc_encode_noalloc (WC_NOALLOC_SCRATCH_BYTES in wc.h).
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class EncodeItem(ctypes.Structure):
@@ -80,6 +83,8 @@ def load() -> ctypes.CDLL:
     L.wc_status_string.argtypes = [i32]
     L.wc_last_error.restype = ctypes.c_char_p
     L.wc_last_error.argtypes = []
+    L.wc_encode_noalloc.restype = i32
+    L.wc_encode_noalloc.argtypes = [vp, u64, i32, vp, u64, vp, vp]
     _lib = L
     return L
 
@@ -279,6 +284,20 @@ def encode(t: torch.Tensor, stream=None) -> torch.Tensor:
                             scr.data_ptr(), scr.numel(), size.data_ptr(), _stream(stream)),
            "wc_encode")
     return out[: int(size.item())]
+
+
+def encode_noalloc(t: torch.Tensor, out: torch.Tensor, size: torch.Tensor, stream=None) -> None:
+    """wc_encode_noalloc: encode into a caller-provided container buffer
+    (`out`, uint8, >= encode_bound bytes) and size word (`size`, one int64),
+    with the library-held scratch instead of a scratch buffer.  For callers
+    that cannot allocate device memory at the call site; at most 16,252,928
+    values.  Nothing is allocated and nothing is synchronised."""
+    f = _flat(t)
+    code = dtype_code(f.dtype)
+    n = f.numel()
+    _check(load().wc_encode_noalloc(f.data_ptr() if n else None, n, code, out.data_ptr(),
+                                    out.numel(), size.data_ptr(), _stream(stream)),
+           "wc_encode_noalloc")
 
 
 def encode_batch(tensors, stream=None) -> list[torch.Tensor]:

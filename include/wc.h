@@ -152,6 +152,33 @@ WC_API int32_t wc_encode_batch(const wc_encode_item *h_items, uint32_t count,
 WC_API int32_t wc_decode_batch(const wc_decode_item *h_items, uint32_t count,
                         int32_t *d_status, void *stream);
 
+/* Encoding with no scratch buffer from the caller.  (The pages have no
+ * counterpart; this exists for callers of the library.)
+ *
+ * For callers that cannot allocate device memory where they encode: a runtime
+ * that owns all device memory through a fixed, pre-planned arena and forbids
+ * allocations outside it, a plug-in that another framework calls with only
+ * its input and output buffers, or a latency-critical path that cannot afford
+ * an allocator's implicit synchronisation.  Arguments and results are those of
+ * wc_encode without d_scratch / scratch_cap; the scratch is a device array of
+ * WC_NOALLOC_SCRATCH_BYTES that the library holds on every GPU that loads it,
+ * from load until the process exits.  That limits n to values whose
+ * wc_scratch_bytes(n) fits: 16,252,928 values (248 chunks) for either dtype;
+ * larger inputs are rejected with WC_ERR_CAPACITY before any work is queued,
+ * and a failed device-address lookup returns WC_ERR_CUDA.
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current (a host-side lookup, cached per device); make that first call
+ * before capturing any stream on that device.  All calls on a GPU share the
+ * one array: calls whose work overlaps on the GPU (for example on two streams
+ * without ordering between them) race and corrupt each other's output; calls
+ * queued on one stream, or otherwise ordered, do not.  The array's contents
+ * between calls do not matter: each call clears the parts that must start at
+ * zero. */
+#define WC_NOALLOC_SCRATCH_BYTES (16u << 20)
+WC_API int32_t wc_encode_noalloc(const void *d_in, uint64_t n, int32_t dtype, void *d_out,
+                                 uint64_t out_cap, uint64_t *d_out_size, void *stream);
+
 /* Human-readable name of a wc_status code (static storage). */
 WC_API const char *wc_status_string(int32_t status);
 
