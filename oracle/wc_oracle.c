@@ -13,7 +13,7 @@
  * What the method is, and where each step comes from:
  *
  *  - Plane split.  A float is split into byte/bit planes so that the skewed
- *    exponent is separated from the near-random mantissa ("SMEF -- blog
+ *    exponent is separated from the mantissa, whose bits look random ("SMEF -- blog
  *    companion code", file table, pass3_streams.py, and "Reading order" item 1;
  *    "PTWM", "How it works" 1. Bit reorder and 2. Byte / nibble split).  For
  *    bf16 the exponent byte is the high byte after the reorder
