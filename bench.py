@@ -89,7 +89,8 @@ def oracle_round_trip_sample(oracle, budget_s: float, first_index: int = 0, max_
         i += 1
         if spent >= budget_s or (max_tensors is not None and count >= max_tensors):
             break
-    names = f"tensors {first_index}..{first_index + count - 1} of 254 ({specs[first_index].name} ..)"
+    names = (f"{count} tensors taken in order from the {len(specs)}-tensor set, starting at "
+             f"{specs[first_index % len(specs)].name} and wrapping around")
     return done_b, spent, count, f"{names}, {done_b / 1e6:.1f} MB, single thread"
 
 

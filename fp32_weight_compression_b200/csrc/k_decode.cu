@@ -37,13 +37,16 @@ constexpr uint32_t kHalf = 256;                 // values per half-group (8 step
 
 struct DecSmem {
   uint32_t tab[kProbScale];                          // 16 KiB
-  __align__(16) uint16_t ring[kDecWarps][2][kRing];  // 32 KiB; freq/cum while a table is built
   __align__(16) uint8_t tbuf[kDecWarps][2][kHalf];   // 4 KiB
   uint32_t gpre[kMaxItems + 1];
   uint64_t red[kDecThreads / 32 + 1];
   int cur_item;
   int tab_ok;
   int single_sym;
+  // Word rings, kRing u16 per chunk, each starting on a 2 KiB boundary of the
+  // shared window (the slack lets ring_ptr align them at run time); freq/cum
+  // while a table is built.
+  __align__(16) uint8_t ring_raw[kDecWarps * 2 * kRing * 2 + 2048];
 };
 
 // The block's dynamic shared memory (a DecSmem).  Functions below reach it
@@ -51,6 +54,14 @@ struct DecSmem {
 // compiles to a shared-memory instruction.
 extern __shared__ __align__(16) uint8_t dyn_smem[];
 __device__ __forceinline__ DecSmem &smem() { return *reinterpret_cast<DecSmem *>(dyn_smem); }
+
+// Ring of chunk slot c of warp w.
+__device__ __forceinline__ uint16_t *ring_ptr(int w, int c) {
+  uint8_t *r = smem().ring_raw;
+  const uint32_t a = uint32_t(__cvta_generic_to_shared(r));
+  const uint32_t pad = ((a + 2047u) & ~2047u) - a;
+  return reinterpret_cast<uint16_t *>(r + pad + (w * 2 + c) * kRing * 2);
+}
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) {
   atomicCAS(status, 0, code);
@@ -283,30 +294,46 @@ __device__ __forceinline__ void load_raw8p(const RawPtrs &p, uint32_t vl, Raw8<D
   }
 }
 
-// One decoding step of two independent chains (chunks A and B), written
-// interleaved operation by operation so that each warp always has an
-// independent instruction to issue while the other chain waits.
+// Renormalisation of one chain whose ring starts at the 2 KiB-aligned shared
+// address rs; c2 counts the bytes of words consumed.  A lane whose state fell
+// below 2^16 takes the word at c2 / 2 + (renormalising lanes below it), so the
+// ring address is (c2 + 2 popc(m & lt)) mod 2048 ORed onto rs, and the state
+// takes the word under the same predicate that voted.
+static_assert(kRing * 2 == 2048, "renorm wraps ring offsets at 2 KiB");
+__device__ __forceinline__ void renorm(uint32_t &x, uint32_t &c2, uint32_t rs, uint32_t lt) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b32 m, t, w;\n\t"
+      "setp.lt.u32 p, %0, 65536;\n\t"
+      "vote.sync.ballot.b32 m, p, -1;\n\t"
+      "and.b32 t, m, %3;\n\t"
+      "popc.b32 t, t;\n\t"
+      "shl.b32 t, t, 1;\n\t"
+      "add.u32 t, t, %1;\n\t"
+      "and.b32 t, t, 2046;\n\t"
+      "or.b32 t, t, %2;\n\t"
+      "ld.shared.u16 w, [t];\n\t"
+      "@p prmt.b32 %0, %0, w, 0x1054;\n\t"
+      "popc.b32 t, m;\n\t"
+      "shl.b32 t, t, 1;\n\t"
+      "add.u32 %1, %1, t;\n\t}"
+      : "+r"(x), "+r"(c2)
+      : "r"(rs), "r"(lt));
+}
+
+// One decoding step of two independent chains (chunks A and B), the table
+// lookups and state updates written side by side so that each warp always
+// has an independent instruction to issue while the other chain waits.
 __device__ __forceinline__ void dstep2(uint32_t &xA, uint32_t &cA, uint32_t &xB, uint32_t &cB,
-                                       const uint32_t *tab, const uint16_t *ringA,
-                                       const uint16_t *ringB, uint8_t *tbpA, uint8_t *tbpB,
-                                       uint32_t lt) {
+                                       const uint32_t *tab, uint32_t rsA, uint32_t rsB,
+                                       uint8_t *tbpA, uint8_t *tbpB, uint32_t lt) {
   const uint32_t eA = tab[xA & (kProbScale - 1)];
   const uint32_t eB = tab[xB & (kProbScale - 1)];
-  const uint32_t sA = xA >> kProbBits, sB = xB >> kProbBits;
-  xA = (eA >> 20) * sA + ((eA >> 8) & 0xFFFu);
-  xB = (eB >> 20) * sB + ((eB >> 8) & 0xFFFu);
-  const bool rA = xA < kStateLow, rB = xB < kStateLow;
-  const uint32_t mA = __ballot_sync(0xffffffffu, rA);
-  const uint32_t mB = __ballot_sync(0xffffffffu, rB);
-  const uint32_t wA = ringA[(cA + __popc(mA & lt)) & (kRing - 1)];
-  const uint32_t wB = ringB[(cB + __popc(mB & lt)) & (kRing - 1)];
-  cA += __popc(mA);
-  cB += __popc(mB);
+  xA = (eA >> 20) * (xA >> kProbBits) + ((eA >> 8) & 0xFFFu);
+  xB = (eB >> 20) * (xB >> kProbBits) + ((eB >> 8) & 0xFFFu);
   *tbpA = uint8_t(eA);
   *tbpB = uint8_t(eB);
-  const uint32_t yA = __byte_perm(xA, wA, 0x1054), yB = __byte_perm(xB, wB, 0x1054);
-  xA = rA ? yA : xA;
-  xB = rB ? yB : xB;
+  renorm(xA, cA, rsA, lt);
+  renorm(xB, cB, rsB, lt);
 }
 
 // Two full coded chunks in lock-step.  Everything arrives by value so that no
@@ -318,7 +345,7 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   DecSmem &s = smem();
   const uint32_t *tab = s.tab;
-  uint16_t *ringA = s.ring[warp][0], *ringB = s.ring[warp][1];
+  uint16_t *ringA = ring_ptr(warp, 0), *ringB = ring_ptr(warp, 1);
   uint8_t *tbA = s.tbuf[warp][0], *tbB = s.tbuf[warp][1];
   const uint32_t lt = lanemask_lt();
   constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
@@ -326,7 +353,9 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   Ring rb{ringB, payB + kStateBytes, uint32_t(round16(lenB) - kStateBytes) >> 1, 0, 0, 0};
   uint32_t xA = reinterpret_cast<const uint32_t *>(payA)[lane];
   uint32_t xB = reinterpret_cast<const uint32_t *>(payB)[lane];
-  uint32_t cA = 0, cB = 0;
+  uint32_t cA = 0, cB = 0;  // bytes of words consumed
+  const uint32_t rsA = uint32_t(__cvta_generic_to_shared(ringA));
+  const uint32_t rsB = uint32_t(__cvta_generic_to_shared(ringB));
 #pragma unroll
   for (int u = 0; u < int(kRing / kUnit); u++) {
     ra.issue(lane);
@@ -349,14 +378,14 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
 #pragma unroll
     for (int j = 0; j < S; j++) {
       const uint32_t h = h0 + j;
-      const int dA = ra.top_up(cA, lane);
-      const int dB = rb.top_up(cB, lane);
+      const int dA = ra.top_up(cA >> 1, lane);
+      const int dB = rb.top_up(cB >> 1, lane);
       cp_async_commit();
       cp_async_wait_depth(min(dA, dB));
       __syncwarp();
 #pragma unroll
       for (int t = 0; t < 8; t++)
-        dstep2(xA, cA, xB, cB, tab, ringA, ringB, tbA + 32 * t + lane, tbB + 32 * t + lane, lt);
+        dstep2(xA, cA, xB, cB, tab, rsA, rsB, tbA + 32 * t + lane, tbB + 32 * t + lane, lt);
       __syncwarp();
       const uint2 eA = *reinterpret_cast<const uint2 *>(tbA + 8 * lane);
       const uint2 eB = *reinterpret_cast<const uint2 *>(tbB + 8 * lane);
@@ -372,10 +401,10 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   cp_async_wait<0>();
   __syncwarp();
   const uint32_t wA = (lenA - kStateBytes) >> 1, wB = (lenB - kStateBytes) >> 1;
-  if (!__all_sync(0xffffffffu, xA == kStateLow) || cA != wA) {
+  if (!__all_sync(0xffffffffu, xA == kStateLow) || (cA >> 1) != wA) {
     if (lane == 0) report(status, WC_ERR_CORRUPT);
   }
-  if (!__all_sync(0xffffffffu, xB == kStateLow) || cB != wB) {
+  if (!__all_sync(0xffffffffu, xB == kStateLow) || (cB >> 1) != wB) {
     if (lane == 0) report(status, WC_ERR_CORRUPT);
   }
 }
@@ -396,7 +425,7 @@ __device__ __noinline__ void decode_one(const ItemView &v, const DecItem &it, co
 
   int mode = c.raw ? 0 : (s.single_sym >= 0 ? 1 : 2);
   uint32_t x = 0, cons = 0;
-  Ring r{s.ring[warp][slot], c.pay + kStateBytes, 0, 0, 0, 0};
+  Ring r{ring_ptr(warp, slot), c.pay + kStateBytes, 0, 0, 0, 0};
   if (mode == 1) {
     // single-symbol table: coding never moves a state and never emits a word
     x = reinterpret_cast<const uint32_t *>(c.pay)[lane];
@@ -477,7 +506,7 @@ __device__ __noinline__ void build_table(const DecItem &it, int ii, int32_t *sta
   DecSmem &s = smem();
   const int tid = threadIdx.x;
   __syncthreads();  // all warps are done with the previous table and rings
-  uint32_t *sfreq = reinterpret_cast<uint32_t *>(&s.ring[0][0][0]);
+  uint32_t *sfreq = reinterpret_cast<uint32_t *>(ring_ptr(0, 0));
   uint32_t *scum = sfreq + 256;
   const uint16_t *f16 = reinterpret_cast<const uint16_t *>(it.cont + kFreqOffset);
   const uint32_t f = f16[tid];

@@ -13,8 +13,10 @@
 // step t reads byte 32 t + lane.  Coding a symbol s with frequency f from
 // state x (12-bit table, L = 2^16, 16-bit words):
 //   if x >= f 2^20: emit x & 0xFFFF, x >>= 16;   x = (x / f) 4096 + x % f + cum_s
-// with x / f computed exactly as floor(x m / 2^64), m = ceil(2^64 / f) split in
-// two 32-bit halves (two integer multiply-adds; see publish_table).  The lanes
+// with x / f computed exactly by a multiply-high and a shift when every f of
+// the tensor is at most 2048 (the usual case), else by a 64-bit reciprocal in
+// two 32-bit halves (see publish_table); the coder is compiled for both and
+// each block takes the form its tensor's table was written in.  The lanes
 // that emit at a step form one block of the word stream, in ascending lane
 // order, placed with __ballot_sync / __popc prefix offsets; blocks are laid
 // down back to front, so the decoder (which runs the steps forwards) reads
@@ -95,28 +97,42 @@ __device__ __forceinline__ uint32_t one_value(const uint8_t *in, uint64_t vg, ui
 }
 
 // ---------------------------------------------------------------------------
+// x = (x / f) 4096 + x % f + cum for a renormalised state x < f 2^20, from the
+// symbol's table entry (narrow: {m, xmax, cmpl, sh | bias << 5}; wide: {ml,
+// xmax, cmpl, mh} with the bias in its own array).
+template <bool W>
+__device__ __forceinline__ uint32_t advance(uint32_t x, const uint4 &te, uint32_t bi) {
+  if (W) {
+    const uint32_t qlo = __umulhi(x, te.x);
+    const uint64_t prod = uint64_t(x) * te.w + qlo;
+    return x + uint32_t(prod >> 32) * te.z + bi;
+  }
+  const uint32_t q = __funnelshift_r(__umulhi(x, te.x), 0u, te.w);  // shift = te.w & 31
+  return x + q * te.z + (te.w >> 5);
+}
+
 // One coding step of one lane.
+template <bool W>
 __device__ __forceinline__ void cstep(uint32_t &x, uint32_t &tail, uint16_t *win16, const uint4 *tab,
                                       const uint32_t *bias, uint32_t s, uint32_t lt) {
   const uint4 te = tab[s];
-  const uint32_t bi = bias[s];
-  const bool emit = x > te.z;
+  const uint32_t bi = W ? bias[s] : 0u;
+  const bool emit = x > te.y;
   const uint32_t m = __ballot_sync(0xffffffffu, emit);
   tail -= __popc(m);
   if (emit) win16[tail + __popc(m & lt)] = uint16_t(x);
   x = emit ? (x >> 16) : x;
-  const uint32_t qlo = __umulhi(x, te.x);
-  const uint64_t prod = uint64_t(x) * te.y + qlo;
-  x = x + uint32_t(prod >> 32) * te.w + bi;
+  x = advance<W>(x, te, bi);
 }
 
 // One coding step of two chains, interleaved operation by operation.
+template <bool W>
 __device__ __forceinline__ void cstep2(uint32_t &xA, uint32_t &tA, uint16_t *wA, uint32_t sA,
                                        uint32_t &xB, uint32_t &tB, uint16_t *wB, uint32_t sB,
                                        const uint4 *tab, const uint32_t *bias, uint32_t lt) {
   const uint4 eA = tab[sA], eB = tab[sB];
-  const uint32_t bA = bias[sA], bB = bias[sB];
-  const bool pA = xA > eA.z, pB = xB > eB.z;
+  const uint32_t bA = W ? bias[sA] : 0u, bB = W ? bias[sB] : 0u;
+  const bool pA = xA > eA.y, pB = xB > eB.y;
   const uint32_t mA = __ballot_sync(0xffffffffu, pA);
   const uint32_t mB = __ballot_sync(0xffffffffu, pB);
   tA -= __popc(mA);
@@ -125,19 +141,18 @@ __device__ __forceinline__ void cstep2(uint32_t &xA, uint32_t &tA, uint16_t *wA,
   if (pB) wB[tB + __popc(mB & lt)] = uint16_t(xB);
   xA = pA ? (xA >> 16) : xA;
   xB = pB ? (xB >> 16) : xB;
-  const uint32_t qA = __umulhi(xA, eA.x), qB = __umulhi(xB, eB.x);
-  const uint64_t rA = uint64_t(xA) * eA.y + qA, rB = uint64_t(xB) * eB.y + qB;
-  xA = xA + uint32_t(rA >> 32) * eA.w + bA;
-  xB = xB + uint32_t(rB >> 32) * eB.w + bB;
+  xA = advance<W>(xA, eA, bA);
+  xB = advance<W>(xB, eB, bB);
 }
 
 // A step that may hold lanes past nsym.
+template <bool W>
 __device__ __forceinline__ void cstep_checked(uint32_t &x, uint32_t &tail, uint16_t *win16,
                                               const uint4 *tab, const uint32_t *bias, uint32_t s,
                                               bool valid, uint32_t lt) {
   const uint4 te = tab[s];
-  const uint32_t bi = bias[s];
-  const bool emit = valid && x > te.z;
+  const uint32_t bi = W ? bias[s] : 0u;
+  const bool emit = valid && x > te.y;
   const uint32_t m = __ballot_sync(0xffffffffu, emit);
   const uint32_t k = __popc(m);
   if (emit) {
@@ -145,11 +160,7 @@ __device__ __forceinline__ void cstep_checked(uint32_t &x, uint32_t &tail, uint1
     x >>= 16;
   }
   tail -= k;
-  if (valid) {
-    const uint32_t qlo = __umulhi(x, te.x);
-    const uint64_t prod = uint64_t(x) * te.y + qlo;
-    x = x + uint32_t(prod >> 32) * te.w + bi;
-  }
+  if (valid) x = advance<W>(x, te, bi);
 }
 
 struct CoderOut {
@@ -167,6 +178,7 @@ __device__ __forceinline__ void finish_chunk(const CoderOut &co, uint64_t k, uin
 }
 
 // Two full bf16 chunks kA, kA + 1 in lock-step.
+template <bool W>
 __device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
                                const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
   const int lane = threadIdx.x & 31;
@@ -200,15 +212,15 @@ __device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, 
     if (!bailA && !bailB) {
 #pragma unroll
       for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
-        cstep2(xA, tA, wA, ebA[32 * t + lane], xB, tB, wB, ebB[32 * t + lane], tab, bias, lt);
+        cstep2<W>(xA, tA, wA, ebA[32 * t + lane], xB, tB, wB, ebB[32 * t + lane], tab, bias, lt);
     } else if (!bailA) {
 #pragma unroll 4
       for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
-        cstep(xA, tA, wA, tab, bias, ebA[32 * t + lane], lt);
+        cstep<W>(xA, tA, wA, tab, bias, ebA[32 * t + lane], lt);
     } else if (!bailB) {
 #pragma unroll 4
       for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
-        cstep(xB, tB, wB, tab, bias, ebB[32 * t + lane], lt);
+        cstep<W>(xB, tB, wB, tab, bias, ebB[32 * t + lane], lt);
     }
     if (kStateBytes + 2 * (kWinWords - tA) >= kChunk) bailA = true;
     if (kStateBytes + 2 * (kWinWords - tB) >= kChunk) bailB = true;
@@ -221,7 +233,7 @@ __device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, 
 }
 
 // Any single chunk (either dtype, possibly ragged).
-template <int DT>
+template <int DT, bool W>
 __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64_t k, int slot,
                                       const CoderOut &co) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -285,11 +297,11 @@ __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64
       if (gb + kGroupValues <= nsym) {
 #pragma unroll 4
         for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
-          cstep(x, tail, win16, tab, bias, eb[32 * t + lane], lt);
+          cstep<W>(x, tail, win16, tab, bias, eb[32 * t + lane], lt);
       } else {
         const int steps = int((nsym - gb + 31) / 32);
         for (int t = steps - 1; t >= 0; --t)
-          cstep_checked(x, tail, win16, tab, bias, eb[32 * t + lane], gb + 32 * t + lane < nsym, lt);
+          cstep_checked<W>(x, tail, win16, tab, bias, eb[32 * t + lane], gb + 32 * t + lane < nsym, lt);
       }
       if (kStateBytes + 2 * (kWinWords - tail) >= nsym) bail = true;
     }
@@ -313,16 +325,24 @@ __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constan
   if (kA >= L.nc) return;
   const bool hasB = kA + 1 < L.nc;
   CoderOut co{reinterpret_cast<uint32_t *>(it.scratch + kScrLen), it.scratch + scratch_win_offset(L.nc)};
+  const bool wide = reinterpret_cast<const uint32_t *>(it.scratch + kScrCtr)[2] != 0;
   if (dtype == WC_BF16) {
-    if (hasB && chunk_nsym(it.n, kA + 1) == kChunk)
-      code_pair_bf16(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
-    else {
-      code_one<WC_BF16>(it, L, kA, 0, co);
-      if (hasB) code_one<WC_BF16>(it, L, kA + 1, 1, co);
+    if (hasB && chunk_nsym(it.n, kA + 1) == kChunk) {
+      if (wide) code_pair_bf16<true>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+      else code_pair_bf16<false>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+    } else if (wide) {
+      code_one<WC_BF16, true>(it, L, kA, 0, co);
+      if (hasB) code_one<WC_BF16, true>(it, L, kA + 1, 1, co);
+    } else {
+      code_one<WC_BF16, false>(it, L, kA, 0, co);
+      if (hasB) code_one<WC_BF16, false>(it, L, kA + 1, 1, co);
     }
+  } else if (wide) {
+    code_one<WC_FP32, true>(it, L, kA, 0, co);
+    if (hasB) code_one<WC_FP32, true>(it, L, kA + 1, 1, co);
   } else {
-    code_one<WC_FP32>(it, L, kA, 0, co);
-    if (hasB) code_one<WC_FP32>(it, L, kA + 1, 1, co);
+    code_one<WC_FP32, false>(it, L, kA, 0, co);
+    if (hasB) code_one<WC_FP32, false>(it, L, kA + 1, 1, co);
   }
 
   // last warp of the tensor: offset table and the rest of the header

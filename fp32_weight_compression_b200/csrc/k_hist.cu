@@ -124,25 +124,43 @@ __device__ void publish_table(const EncItem &it, uint64_t *red) {
     if (ge) f = T - (rank < r ? 1 : 0);
   }
   const uint64_t cum = block_excl_scan_u64<kHistThreads>(f, red);
+  // The coder divides the state x by f after renormalisation, when
+  // x < f 2^20.  Narrow format (every f <= 2048): q = floor(x m / 2^k) with
+  // k = 31 + c, c = ceil(log2 f), m = ceil(2^k / f) < 2^32, computed as
+  // umulhi(x, m) >> (c - 1).  With e = m f - 2^k < f, the error term
+  // x e / (f 2^k) < f 2^20 f / (f 2^(31 + c)) <= 1 / f when f <= 2^11, so the
+  // floor is exact.  Wide format (some f > 2048): m = ceil(2^64 / f) as two
+  // 32-bit halves, exact for every x < 2^32.  In both, f = 1 uses the all-ones
+  // multiplier, which yields q = x - 1, repaid by bias += 4095.
+  const bool wide = block_max_u64<kHistThreads>(f, red) > 2048;
   if (own) {
     const uint32_t ff = uint32_t(f);
     reinterpret_cast<uint16_t *>(it.out + kFreqOffset)[tid] = uint16_t(ff);
     uint4 e = make_uint4(0, 0, 0, 0);
     uint32_t bias = 0;
     if (ff) {
-      // q = floor(x / f) = floor(x * m / 2^64) with m = ceil(2^64 / f), exact
-      // for every x < 2^32 (x * (m f - 2^64) < 2^32 * f < 2^64); f = 1 uses
-      // m = 2^64 - 1, which yields q = x - 1, repaid by bias += 4095.
-      const uint64_t m = ff >= 2 ? (~uint64_t(0) / ff + 1) : ~uint64_t(0);
-      e.x = uint32_t(m);
-      e.y = uint32_t(m >> 32);
-      e.z = uint32_t((uint64_t(ff) << 20) - 1);  // renormalise while x > xmax
-      e.w = kProbScale - ff;
       bias = uint32_t(cum) + (ff == 1 ? kProbScale - 1 : 0);
+      e.y = uint32_t((uint64_t(ff) << 20) - 1);  // renormalise while x > xmax
+      e.z = kProbScale - ff;
+      if (wide) {
+        const uint64_t m = ff >= 2 ? (~uint64_t(0) / ff + 1) : ~uint64_t(0);
+        e.x = uint32_t(m);
+        e.w = uint32_t(m >> 32);
+      } else {
+        uint32_t m = 0xFFFFFFFFu, sh = 0;
+        if (ff >= 2) {
+          const uint32_t c = 32 - __clz(ff - 1);
+          m = uint32_t(((uint64_t(1) << (31 + c)) - 1) / ff + 1);
+          sh = c - 1;
+        }
+        e.x = m;
+        e.w = sh | (bias << 5);
+      }
     }
     reinterpret_cast<uint4 *>(it.scratch + kScrTab)[tid] = e;
     reinterpret_cast<uint32_t *>(it.scratch + kScrBias)[tid] = bias;
   }
+  if (tid == 0) reinterpret_cast<uint32_t *>(it.scratch + kScrCtr)[2] = wide ? 1u : 0u;
 }
 
 // 16 values' worth of exponent counts (one group) from raw words.

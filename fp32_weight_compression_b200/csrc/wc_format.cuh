@@ -31,9 +31,11 @@ constexpr uint32_t kStepsPerGroup = 16;
 
 // Encoder scratch, per tensor (offsets in bytes from the tensor's scratch).
 //   hist     u64[256]       exponent counts
-//   ctr      u32[4]         blocks done (histogram), warps done (coder)
-//   tab      uint4[256]     per-symbol coding entry {ml, mh, xmax, cmpl}
-//   bias     u32[256]       per-symbol additive term
+//   ctr      u32[4]         blocks done (histogram), warps done (coder),
+//                           table format (0 narrow, 1 wide), unused
+//   tab      uint4[256]     per-symbol coding entry: narrow {m, xmax, cmpl,
+//                           sh | bias << 5}, wide {ml, xmax, cmpl, mh}
+//   bias     u32[256]       per-symbol additive term (wide format)
 //   len      u32[nc]        chunk lengths
 //   windows  nc x kWin      coded chunk staging (states at the front,
 //                           words filled backwards from the end)

@@ -229,3 +229,37 @@ def test_random_flips_never_escape(orc, gu):
         assert (st == 0) == (ost == 0), (st, ost)
         if st == 0:
             assert np.array_equal(vals, ovals)
+
+
+@pytest.mark.parametrize("fmax", [1024, 2047, 2048, 2049, 2964, 4000, 4095])
+@pytest.mark.parametrize("dt", ["bf16", "fp32"])
+def test_table_format_boundary(orc, gu, dt, fmax):
+    """Exact counts that put the largest frequency at fmax, with several f = 1
+    symbols: the coder's narrow table (every f <= 2048) and its wide one on
+    both sides of the limit, through the paired-chunk path (4 full chunks)
+    and a ragged tail."""
+    rng = np.random.default_rng(fmax)
+    n = 4 * C                        # f = count / 64 exactly when counts are multiples of 64
+    ones = [3, 200, 250][:4096 - fmax]  # f = 1
+    rest = 4096 - fmax - len(ones)
+    fr = {120: fmax}
+    for s in ones:
+        fr[s] = 1
+    others = [118, 119, 121, 122, 123]
+    for i, s in enumerate(others):
+        fr[s] = rest // len(others) + (1 if i < rest % len(others) else 0)
+    fr = {s: f for s, f in fr.items() if f > 0}
+    assert sum(fr.values()) == 4096
+    e = np.concatenate([np.full(64 * f, s, np.uint32) for s, f in fr.items()])
+    rng.shuffle(e)
+    assert e.size == n
+    assert np.array_equal(orc.normalize(np.bincount(e, minlength=256).astype(np.uint64)),
+                          np.array([fr.get(s, 0) for s in range(256)], np.uint32))
+    if dt == "bf16":
+        sm = rng.integers(0, 256, n, dtype=np.uint32)
+        bits = (((sm & 0x80) << 8) | (e << 7) | (sm & 0x7F)).astype(np.uint16)
+    else:
+        bits = ((rng.integers(0, 2, n, dtype=np.uint32) << 31) | (e << 23) |
+                rng.integers(0, 1 << 23, n, dtype=np.uint32)).astype(np.uint32)
+    _check(orc, gu, bits)
+    _check(orc, gu, bits[:3 * C + 333])
