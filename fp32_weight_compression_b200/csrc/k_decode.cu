@@ -43,9 +43,9 @@ struct DecSmem {
   int cur_item;
   int tab_ok;
   int single_sym;
-  // Word rings, kRing u16 per chunk, each starting on a 2 KiB boundary of the
-  // shared window (the slack lets ring_ptr align them at run time); freq/cum
-  // while a table is built.
+  // Word rings, kRing u16 per chunk, each on a 2 KiB boundary of the shared
+  // window (the slack lets ring_ptr align them at run time); freq/cum while a
+  // table is built.
   __align__(16) uint8_t ring_raw[kDecWarps * 2 * kRing * 2 + 2048];
 };
 
@@ -225,16 +225,18 @@ __device__ __forceinline__ void merge_store1(uint32_t e, const uint8_t *cont, co
 // ---------------------------------------------------------------------------
 // The word ring of one chunk.
 struct Ring {
-  uint16_t *buf;
+  uint32_t rs;         // shared address of the ring
   const uint8_t *src;  // first word
   uint32_t avail;      // readable words (payload rounded to 16 bytes)
   uint32_t req;        // words requested so far (multiple of kUnit)
   uint32_t f1, f2;     // requested frontier after the call before last / before that
+  uint32_t landed;     // words known to be in shared memory (after a wait)
 
   __device__ __forceinline__ void issue(int lane) {
     const uint32_t j0 = req + 8 * lane;
-    if (j0 < avail) cp_async16(buf + (j0 & (kRing - 1)), src + 2 * j0, 16);
-    else cp_async16(buf + (j0 & (kRing - 1)), src, 0);  // zero fill, reads nothing
+    const uint32_t dst = rs + ((j0 & (kRing - 1)) << 1);
+    if (j0 < avail) cp_async16_s(dst, src + 2 * j0, 16);
+    else cp_async16_s(dst, src, 0);  // zero fill, reads nothing
     req += kUnit;
   }
   // Called once per half-group, followed by one commit.  Issues the next unit
@@ -244,13 +246,29 @@ struct Ring {
   // while the words [cons, cons + 256) are already in shared memory: 3 if
   // they were requested three calls ago or earlier, ..., 0 if only now.
   __device__ __forceinline__ int top_up(uint32_t cons, int lane) {
+    const uint32_t f0 = top(cons, lane);
+    const int d = depth(min(cons + kHalf, avail), f0);
+    shift(f0);
+    return d;
+  }
+  // The same in parts, for a caller that skips the wait while the words it
+  // needs are known to have landed: top() issues and returns the frontier
+  // before this call; depth(); frontier(d) is what a wait at depth d
+  // guarantees; shift() moves the history on.
+  __device__ __forceinline__ uint32_t top(uint32_t cons, int lane) {
     const uint32_t f0 = req;  // frontier after the previous call
     if (req < avail && req + kUnit <= (cons & ~(kUnit - 1)) + kRing) issue(lane);
-    const uint32_t need = min(cons + kHalf, avail);
-    const int depth = f2 >= need ? 3 : (f1 >= need ? 2 : (f0 >= need ? 1 : 0));
+    return f0;
+  }
+  __device__ __forceinline__ int depth(uint32_t need, uint32_t f0) const {
+    return f2 >= need ? 3 : (f1 >= need ? 2 : (f0 >= need ? 1 : 0));
+  }
+  __device__ __forceinline__ uint32_t frontier(int d, uint32_t f0) const {
+    return d >= 3 ? f2 : (d == 2 ? f1 : (d == 1 ? f0 : req));
+  }
+  __device__ __forceinline__ void shift(uint32_t f0) {
     f2 = f1;
     f1 = f0;
-    return depth;
   }
 };
 
@@ -296,9 +314,9 @@ __device__ __forceinline__ void load_raw8p(const RawPtrs &p, uint32_t vl, Raw8<D
 
 // Renormalisation of one chain whose ring starts at the 2 KiB-aligned shared
 // address rs; c2 counts the bytes of words consumed.  A lane whose state fell
-// below 2^16 takes the word at c2 / 2 + (renormalising lanes below it), so the
-// ring address is (c2 + 2 popc(m & lt)) mod 2048 ORed onto rs, and the state
-// takes the word under the same predicate that voted.
+// below 2^16 takes the word c2 / 2 + (renormalising lanes below it): its
+// address is (c2 + 2 popc(m & lt)) mod 2048 ORed onto rs, and the state takes
+// the word under the same predicate that voted.
 static_assert(kRing * 2 == 2048, "renorm wraps ring offsets at 2 KiB");
 __device__ __forceinline__ void renorm(uint32_t &x, uint32_t &c2, uint32_t rs, uint32_t lt) {
   asm volatile(
@@ -307,15 +325,13 @@ __device__ __forceinline__ void renorm(uint32_t &x, uint32_t &c2, uint32_t rs, u
       "vote.sync.ballot.b32 m, p, -1;\n\t"
       "and.b32 t, m, %3;\n\t"
       "popc.b32 t, t;\n\t"
-      "shl.b32 t, t, 1;\n\t"
-      "add.u32 t, t, %1;\n\t"
+      "mad.lo.u32 t, t, 2, %1;\n\t"
       "and.b32 t, t, 2046;\n\t"
       "or.b32 t, t, %2;\n\t"
       "ld.shared.u16 w, [t];\n\t"
       "@p prmt.b32 %0, %0, w, 0x1054;\n\t"
       "popc.b32 t, m;\n\t"
-      "shl.b32 t, t, 1;\n\t"
-      "add.u32 %1, %1, t;\n\t}"
+      "mad.lo.u32 %1, t, 2, %1;\n\t}"
       : "+r"(x), "+r"(c2)
       : "r"(rs), "r"(lt));
 }
@@ -328,8 +344,9 @@ __device__ __forceinline__ void dstep2(uint32_t &xA, uint32_t &cA, uint32_t &xB,
                                        uint8_t *tbpA, uint8_t *tbpB, uint32_t lt) {
   const uint32_t eA = tab[xA & (kProbScale - 1)];
   const uint32_t eB = tab[xB & (kProbScale - 1)];
-  xA = (eA >> 20) * (xA >> kProbBits) + ((eA >> 8) & 0xFFFu);
-  xB = (eB >> 20) * (xB >> kProbBits) + ((eB >> 8) & 0xFFFu);
+  // f (x >> 12) + d = f ((x >> 12) - 4096) + (e >> 8), as e >> 8 = f 4096 + d
+  xA = (eA >> 20) * ((xA >> kProbBits) - 4096u) + (eA >> 8);
+  xB = (eB >> 20) * ((xB >> kProbBits) - 4096u) + (eB >> 8);
   *tbpA = uint8_t(eA);
   *tbpB = uint8_t(eB);
   renorm(xA, cA, rsA, lt);
@@ -338,24 +355,28 @@ __device__ __forceinline__ void dstep2(uint32_t &xA, uint32_t &cA, uint32_t &xB,
 
 // Two full coded chunks in lock-step.  Everything arrives by value so that no
 // argument lives in local memory.
+// Chunk B is the one after A: its raw planes and output follow A's.
 template <int DT>
 __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *payB, uint32_t lenA,
-                                         uint32_t lenB, RawPtrs rpA, RawPtrs rpB, uint8_t *outA,
-                                         uint8_t *outB, int32_t *status) {
+                                         uint32_t lenB, RawPtrs rpA, uint8_t *outA,
+                                         int32_t *status) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   DecSmem &s = smem();
   const uint32_t *tab = s.tab;
-  uint16_t *ringA = ring_ptr(warp, 0), *ringB = ring_ptr(warp, 1);
+  const uint32_t rsA = uint32_t(__cvta_generic_to_shared(ring_ptr(warp, 0)));
+  const uint32_t rsB = uint32_t(__cvta_generic_to_shared(ring_ptr(warp, 1)));
   uint8_t *tbA = s.tbuf[warp][0], *tbB = s.tbuf[warp][1];
   const uint32_t lt = lanemask_lt();
   constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
-  Ring ra{ringA, payA + kStateBytes, uint32_t(round16(lenA) - kStateBytes) >> 1, 0, 0, 0};
-  Ring rb{ringB, payB + kStateBytes, uint32_t(round16(lenB) - kStateBytes) >> 1, 0, 0, 0};
+  Ring ra{rsA, payA + kStateBytes, uint32_t(round16(lenA) - kStateBytes) >> 1, 0, 0, 0, 0};
+  Ring rb{rsB, payB + kStateBytes, uint32_t(round16(lenB) - kStateBytes) >> 1, 0, 0, 0, 0};
+  RawPtrs rpB;
+  rpB.a = rpA.a + (DT == WC_BF16 ? kChunk : 3 * kChunk);
+  rpB.s = DT == WC_BF16 ? nullptr : rpA.s + kChunk / 8;
+  uint8_t *outB = outA + kChunk * elem;
   uint32_t xA = reinterpret_cast<const uint32_t *>(payA)[lane];
   uint32_t xB = reinterpret_cast<const uint32_t *>(payB)[lane];
   uint32_t cA = 0, cB = 0;  // bytes of words consumed
-  const uint32_t rsA = uint32_t(__cvta_generic_to_shared(ringA));
-  const uint32_t rsB = uint32_t(__cvta_generic_to_shared(ringB));
 #pragma unroll
   for (int u = 0; u < int(kRing / kUnit); u++) {
     ra.issue(lane);
@@ -366,8 +387,9 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   constexpr uint32_t NH = kChunk / kHalf;
   // Raw planes are prefetched S half-groups ahead into S register sets used
   // in rotation; the loop is unrolled S times so each set is consumed where it
-  // was loaded (no register moves that would wait on loads in flight).
-  constexpr int S = 2;
+  // was loaded (no register moves that would wait on loads in flight).  fp32
+  // needs 3x the raw bytes per value, so it keeps fewer sets in registers.
+  constexpr int S = DT == WC_BF16 ? 4 : 2;
   Raw8<DT> pa[S], pb[S];
 #pragma unroll
   for (int j = 0; j < S; j++) {
@@ -378,10 +400,21 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
 #pragma unroll
     for (int j = 0; j < S; j++) {
       const uint32_t h = h0 + j;
-      const int dA = ra.top_up(cA >> 1, lane);
-      const int dB = rb.top_up(cB >> 1, lane);
+      const uint32_t f0A = ra.top(cA >> 1, lane), f0B = rb.top(cB >> 1, lane);
       cp_async_commit();
-      cp_async_wait_depth(min(dA, dB));
+      // wait only when a word this half-group may read is not known to have
+      // landed (a wait is followed by __syncwarp, so landed words are visible
+      // to every lane)
+      const uint32_t needA = min((cA >> 1) + kHalf, ra.avail);
+      const uint32_t needB = min((cB >> 1) + kHalf, rb.avail);
+      if (needA > ra.landed || needB > rb.landed) {
+        const int d = min(ra.depth(needA, f0A), rb.depth(needB, f0B));
+        cp_async_wait_depth(d);
+        ra.landed = ra.frontier(d, f0A);
+        rb.landed = rb.frontier(d, f0B);
+      }
+      ra.shift(f0A);
+      rb.shift(f0B);
       __syncwarp();
 #pragma unroll
       for (int t = 0; t < 8; t++)
@@ -425,7 +458,8 @@ __device__ __noinline__ void decode_one(const ItemView &v, const DecItem &it, co
 
   int mode = c.raw ? 0 : (s.single_sym >= 0 ? 1 : 2);
   uint32_t x = 0, cons = 0;
-  Ring r{ring_ptr(warp, slot), c.pay + kStateBytes, 0, 0, 0, 0};
+  const uint16_t *rbuf = ring_ptr(warp, slot);
+  Ring r{uint32_t(__cvta_generic_to_shared(rbuf)), c.pay + kStateBytes, 0, 0, 0, 0, 0};
   if (mode == 1) {
     // single-symbol table: coding never moves a state and never emits a word
     x = reinterpret_cast<const uint32_t *>(c.pay)[lane];
@@ -451,7 +485,7 @@ __device__ __noinline__ void decode_one(const ItemView &v, const DecItem &it, co
       __syncwarp();
       if (full) {
 #pragma unroll
-        for (int t = 0; t < 8; t++) dstep(x, cons, s.tab, r.buf, tb + 32 * t + lane, lt);
+        for (int t = 0; t < 8; t++) dstep(x, cons, s.tab, rbuf, tb + 32 * t + lane, lt);
       } else {
         const uint32_t steps = (nsym - hb + 31) / 32;
         for (uint32_t t = 0; t < steps; t++) {
@@ -463,7 +497,7 @@ __device__ __noinline__ void decode_one(const ItemView &v, const DecItem &it, co
           }
           const bool rn = valid && x < kStateLow;
           const uint32_t m = __ballot_sync(0xffffffffu, rn);
-          const uint32_t w = r.buf[(cons + __popc(m & lt)) & (kRing - 1)];
+          const uint32_t w = rbuf[(cons + __popc(m & lt)) & (kRing - 1)];
           if (rn) x = __byte_perm(x, w, 0x1054);
           cons += __popc(m);
           tb[32 * t + lane] = uint8_t(e);
@@ -557,18 +591,15 @@ __device__ __forceinline__ void decode_warp_chunks(const ItemView &v, const DecI
   if (hasB && s.single_sym < 0 && !A.raw && !B.raw && A.nsym == kChunk && B.nsym == kChunk) {
     const Layout &L = v.L;
     const uint64_t vgA = kA * kChunk;
-    RawPtrs rpA, rpB;
+    RawPtrs rpA;
     if (DT == WC_BF16) {
       rpA.a = it.cont + L.off_raw + vgA;
-      rpB.a = rpA.a + kChunk;
-      rpA.s = rpB.s = nullptr;
+      rpA.s = nullptr;
     } else {
       rpA.a = it.cont + L.off_mant + 3 * vgA;
-      rpB.a = rpA.a + 3 * kChunk;
       rpA.s = it.cont + L.off_raw + vgA / 8;
-      rpB.s = rpA.s + kChunk / 8;
     }
-    decode_pair<DT>(A.pay, B.pay, A.len, B.len, rpA, rpB, A.out, B.out, status);
+    decode_pair<DT>(A.pay, B.pay, A.len, B.len, rpA, A.out, status);
     return;
   }
   decode_one<DT>(v, it, A, kA, 0, status);

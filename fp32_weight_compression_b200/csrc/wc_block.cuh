@@ -108,6 +108,11 @@ __device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src,
                "r"(src_bytes)
                : "memory");
 }
+__device__ __forceinline__ void cp_async16_s(uint32_t smem_dst, const void *gmem_src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(smem_dst), "l"(gmem_src),
+               "r"(src_bytes)
+               : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {
