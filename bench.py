@@ -225,28 +225,28 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def e2e_leg(args, enc, sizes, outs, dev, dev_in, dev_out, host_in, stream, barrier, world):
-    """End-to-end through the public API with host buffers: every step copies
-    the inputs host->device, encodes, copies the containers device->host,
-    copies them back host->device, decodes, and copies the outputs
-    device->host (pinned host memory)."""
+def e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world):
+    """End-to-end through the public host API (wc.HostCodec: wc_encode_host /
+    wc_decode_host): every step encodes the host-resident inputs (pinned) into
+    host containers and decodes those back into host outputs.  The library
+    streams windows of tensors through the device with copies in both
+    directions overlapping the kernels."""
     import torch
     import torch.distributed as dist
     from fp32_weight_compression_b200 import wc
     if args.no_e2e:
         return None, 0
-    # end-to-end through host buffers: H2D inputs -> encode -> D2H containers,
-    # H2D containers -> decode -> D2H outputs, every step
-    host_cont = torch.empty(max(sum((s + 255) // 256 * 256 for s in sizes), 256),
-                            dtype=torch.uint8, pin_memory=True)
-    coffs, o = [], 0
-    for s in sizes:
-        coffs.append(o)
-        o += (int(s) + 255) // 256 * 256
-    dev_cont = torch.empty(host_cont.numel(), dtype=torch.uint8, device=dev)
-    conts_packed = [dev_cont[co:co + int(s)] for co, s in zip(coffs, sizes)]
-    dec2 = wc.BatchDecoder(device=dev).prepare(conts_packed, outs)
+    hts = [host_in[o:o + a.nbytes].view(torch.bfloat16) for a, o in zip(arrs, offs)]
     host_out = torch.empty_like(host_in, pin_memory=True)
+    hos = [host_out[o:o + a.nbytes].view(torch.bfloat16) for a, o in zip(arrs, offs)]
+    big = max(wc.host_encode_footprint(a.size, torch.bfloat16) for a in arrs)
+    slot = (big + 256 + 255) // 256 * 256
+    codec = wc.HostCodec(256 * ((4 * len(arrs) + 255) // 256) + 3 * slot, device=dev)
+    enc_bufs, sizes = codec.encode_buffers(hts)
+    conts = codec.encode(hts, enc_bufs, sizes)      # warm-up + check
+    codec.decode(conts, hos)
+    assert torch.equal(host_out, host_in), "end-to-end round trip is not bit-exact"
+    host_out.zero_()
     E = max(1, args.e2e_steps)
     barrier()
     torch.cuda.synchronize(dev)
@@ -254,26 +254,17 @@ def e2e_leg(args, enc, sizes, outs, dev, dev_in, dev_out, host_in, stream, barri
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(E):
-        dev_in.copy_(host_in, non_blocking=True)
-        enc.run()
-        szs = enc.sizes.cpu().tolist()          # D2H of the sizes (sync)
-        for i, (s, co) in enumerate(zip(szs, coffs)):
-            host_cont[co:co + int(s)].copy_(enc.out[enc.out_offsets[i]:enc.out_offsets[i] + int(s)],
-                                            non_blocking=True)
-        dev_cont.copy_(host_cont, non_blocking=True)
-        dec2.run()
-        host_out.copy_(dev_out, non_blocking=True)
+        conts = codec.encode(hts, enc_bufs, sizes)
+        codec.decode(conts, hos)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     t_e2e = e0.elapsed_time(e1) / 1e3
-    dec2.check()
     assert torch.equal(host_out, host_in), "end-to-end round trip is not bit-exact"
     if world > 1:
         tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         t_e2e = tt.item()
     return t_e2e, E
-
 
 
 # ---------------------------------------------------------------------------
@@ -376,7 +367,7 @@ def main():
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         t_total, t_enc, t_dec = tt.tolist()
 
-    t_e2e, E = e2e_leg(args, enc, sizes, outs, dev, dev_in, dev_out, host_in, stream, barrier, world)
+    t_e2e, E = e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world)
 
     peak, peak_note = peak_hbm()
     B = total_in

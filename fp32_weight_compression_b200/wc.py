@@ -26,7 +26,8 @@ _ELEM = {BF16: 2, FP32: 4}
 EXPORTS = (
     "wc_encode_bound", "wc_scratch_bytes", "wc_encode", "wc_decode", "wc_decode_chunk",
     "wc_read_header", "wc_encode_batch", "wc_decode_batch", "wc_status_string", "wc_last_error",
-    "wc_encode_noalloc",
+    "wc_encode_noalloc", "wc_host_encode_footprint", "wc_host_decode_footprint", "wc_host_plan",
+    "wc_encode_host", "wc_decode_host",
 )
 # Library-held scratch of wc_encode_noalloc (WC_NOALLOC_SCRATCH_BYTES in wc.h).
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -42,6 +43,17 @@ class EncodeItem(ctypes.Structure):
 class DecodeItem(ctypes.Structure):
     _fields_ = [("cont", ctypes.c_void_p), ("cont_bytes", ctypes.c_uint64),
                 ("out", ctypes.c_void_p), ("out_cap", ctypes.c_uint64)]
+
+
+class HostEncodeItem(ctypes.Structure):
+    _fields_ = [("h_in", ctypes.c_void_p), ("n", ctypes.c_uint64), ("dtype", ctypes.c_int32),
+                ("reserved", ctypes.c_int32), ("h_out", ctypes.c_void_p), ("h_out_cap", ctypes.c_uint64),
+                ("h_out_size", ctypes.c_void_p)]
+
+
+class HostDecodeItem(ctypes.Structure):
+    _fields_ = [("h_cont", ctypes.c_void_p), ("cont_bytes", ctypes.c_uint64),
+                ("h_out", ctypes.c_void_p), ("out_cap", ctypes.c_uint64)]
 
 
 class WCError(RuntimeError):
@@ -85,6 +97,17 @@ def load() -> ctypes.CDLL:
     L.wc_last_error.argtypes = []
     L.wc_encode_noalloc.restype = i32
     L.wc_encode_noalloc.argtypes = [vp, u64, i32, vp, u64, vp, vp]
+    L.wc_host_encode_footprint.restype = u64
+    L.wc_host_encode_footprint.argtypes = [u64, i32]
+    L.wc_host_decode_footprint.restype = u64
+    L.wc_host_decode_footprint.argtypes = [u64, u64, i32]
+    L.wc_host_plan.restype = i32
+    L.wc_host_plan.argtypes = [vp, u32, u64, u64, ctypes.POINTER(u32), vp, ctypes.POINTER(u32)]
+    L.wc_encode_host.restype = i32
+    L.wc_encode_host.argtypes = [ctypes.POINTER(HostEncodeItem), u32, vp, u64, u64, vp, vp, vp]
+    L.wc_decode_host.restype = i32
+    L.wc_decode_host.argtypes = [ctypes.POINTER(HostDecodeItem), u32, vp, u64, u64, vp, vp, vp,
+                                 ctypes.POINTER(i32)]
     _lib = L
     return L
 
@@ -352,3 +375,104 @@ def decode_batch(conts, shapes, dtypes, stream=None) -> list[torch.Tensor]:
     dec.decode(conts, outs, stream=stream)
     dec.check()
     return outs
+
+
+# ---------------------------------------------------------------------------
+# Host-resident tensors through the device in windows (wc_encode_host /
+# wc_decode_host): the library runs the copy / kernel pipeline; this class
+# only owns the device workspace, the three streams and pinned host buffers.
+
+def host_plan(footprints, slot_area: int, window_bytes: int = 0) -> tuple[int, list[int]]:
+    """(slots, window ends) of wc_host_plan for the given item footprints."""
+    import numpy as np
+    fp = np.ascontiguousarray(np.asarray(footprints, dtype=np.uint64))
+    ends = np.zeros(max(1, fp.size), np.uint32)
+    k, w = ctypes.c_uint32(), ctypes.c_uint32()
+    _check(load().wc_host_plan(fp.ctypes.data if fp.size else None, fp.size, slot_area,
+                               window_bytes, ctypes.byref(k), ends.ctypes.data, ctypes.byref(w)),
+           "wc_host_plan")
+    return k.value, ends[:w.value].tolist()
+
+
+def host_encode_footprint(n: int, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return int(load().wc_host_encode_footprint(n, code))
+
+
+def host_decode_footprint(cont_bytes: int, n: int, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else dtype_code(dtype)
+    return int(load().wc_host_decode_footprint(cont_bytes, n, code))
+
+
+def _host_flat(t: torch.Tensor) -> torch.Tensor:
+    if t.is_cuda:
+        raise ValueError("host pipeline: tensor must be in host memory")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.reshape(-1)
+
+
+class HostCodec:
+    """Encodes host tensors into host containers and decodes them back,
+    streaming windows of about `window_bytes` of slot space through a device
+    workspace of `work_bytes` with three CUDA streams (copy in, kernels, copy
+    out).  Host buffers should be pinned (`torch.empty(..., pin_memory=True)`)
+    for the copies to overlap."""
+
+    def __init__(self, work_bytes: int, device="cuda", window_bytes: int = 128 << 20):
+        self.device = torch.device(device)
+        self.window_bytes = int(window_bytes)
+        self.work = torch.empty(int(work_bytes), dtype=torch.uint8, device=self.device)
+        self.streams = [torch.cuda.Stream(device=self.device) for _ in range(3)]
+
+    def _s(self):
+        return [s.cuda_stream for s in self.streams]
+
+    def encode_buffers(self, tensors, pin=True) -> tuple[list[torch.Tensor], torch.Tensor]:
+        """Host buffers of wc_encode_bound bytes for the given tensors, and the
+        host u64 size array; reuse them across encode() calls."""
+        outs = [torch.empty(max(16, encode_bound(t.numel(), t.dtype)), dtype=torch.uint8,
+                            pin_memory=pin) for t in tensors]
+        return outs, torch.zeros(len(tensors), dtype=torch.int64)
+
+    def encode(self, tensors, outs=None, sizes=None) -> list[torch.Tensor]:
+        """Containers (host uint8 views, trimmed) of host tensors."""
+        flats = [_host_flat(t) for t in tensors]
+        if outs is None or sizes is None:
+            outs, sizes = self.encode_buffers(tensors, pin=all(t.is_pinned() for t in flats))
+        items = (HostEncodeItem * len(flats))()
+        for i, t in enumerate(flats):
+            it = items[i]
+            it.h_in = t.data_ptr() if t.numel() else None
+            it.n = t.numel()
+            it.dtype = dtype_code(t.dtype)
+            it.reserved = 0
+            it.h_out = outs[i].data_ptr()
+            it.h_out_cap = outs[i].numel()
+            it.h_out_size = sizes.data_ptr() + 8 * i
+        si, sc, so = self._s()
+        _check(load().wc_encode_host(items, len(flats), self.work.data_ptr(), self.work.numel(),
+                                     self.window_bytes, si, sc, so), "wc_encode_host")
+        return [o[:int(z)] for o, z in zip(outs, sizes.tolist())]
+
+    def decode(self, conts, outs=None, pin=True) -> list[torch.Tensor]:
+        """Decoded host tensors (1-D) of host containers."""
+        hdr = [read_header(c) for c in conts]
+        if outs is None:
+            outs = [torch.empty(n, dtype=_TORCH_DT[dt], pin_memory=pin) for n, dt, _ in hdr]
+        items = (HostDecodeItem * len(conts))()
+        for i, (c, o) in enumerate(zip(conts, outs)):
+            if c.is_cuda or not c.is_contiguous():
+                raise ValueError("host pipeline: containers must be contiguous host buffers")
+            it = items[i]
+            it.h_cont = c.data_ptr()
+            it.cont_bytes = c.numel()
+            it.h_out = o.data_ptr() if o.numel() else None
+            it.out_cap = o.numel() * o.element_size()
+        st = ctypes.c_int32()
+        si, sc, so = self._s()
+        _check(load().wc_decode_host(items, len(conts), self.work.data_ptr(), self.work.numel(),
+                                     self.window_bytes, si, sc, so, ctypes.byref(st)),
+               "wc_decode_host")
+        _check(st.value, "wc_decode_host (device status)")
+        return outs

@@ -179,6 +179,78 @@ WC_API int32_t wc_decode_batch(const wc_decode_item *h_items, uint32_t count,
 WC_API int32_t wc_encode_noalloc(const void *d_in, uint64_t n, int32_t dtype, void *d_out,
                                  uint64_t out_cap, uint64_t *d_out_size, void *stream);
 
+/* Host-resident tensors, encoded and decoded through the device in windows
+ * ("seedpack 0.2.0 -> 0.2.2", README: a model is streamed through the GPU in
+ * windows of about 1 GB, tensor by tensor).
+ *
+ * The items' buffers (h_*) are host memory; on the device the calls use only
+ * the caller's workspace d_work (256-byte aligned, work_cap bytes).  The
+ * workspace is cut into slots; consecutive items are grouped into windows
+ * that fit one slot (wc_host_plan), and the windows go through a pipeline:
+ * host->device copies on stream_in, the batched kernels on stream_compute,
+ * device->host copies on stream_out, ordered by events, so that copies in
+ * both directions and the kernels of consecutive windows overlap.  Host
+ * buffers must be page-locked for the copies to overlap; pageable memory
+ * works but serialises them.  The three streams may be one stream (no
+ * overlap).  Containers and decoded values are exactly those of
+ * wc_encode_batch / wc_decode_batch.
+ *
+ * Unlike the calls above, these two block: they return after every copy has
+ * finished (or at the first error, after the work already queued is done) and
+ * synchronise the three streams.  Each call creates and destroys a few CUDA
+ * events; no memory is allocated.  Argument, header and capacity checks come
+ * first and queue no work.
+ *
+ * Workspace: 256-byte rounded 4 * count bytes of status words, then the
+ * slots.  An item needs wc_host_encode_footprint / wc_host_decode_footprint
+ * bytes of a slot (a window adds 256).  Three slots are used when each can
+ * hold the largest item, else two, else one; if one slot cannot hold it the
+ * call returns WC_ERR_CAPACITY. */
+typedef struct {
+    const void *h_in;       /* n values (host)                              */
+    uint64_t n;
+    int32_t dtype;          /* WC_BF16 or WC_FP32                           */
+    int32_t reserved;       /* must be 0                                    */
+    void *h_out;            /* container (host)                             */
+    uint64_t h_out_cap;     /* must be >= wc_encode_bound(n, dtype)         */
+    uint64_t *h_out_size;   /* host u64: the container's size               */
+} wc_host_encode_item;
+
+typedef struct {
+    const void *h_cont;     /* container (host); its header is read here    */
+    uint64_t cont_bytes;
+    void *h_out;            /* decoded values (host), n * element bytes     */
+    uint64_t out_cap;
+} wc_host_decode_item;
+
+/* Slot bytes one item needs (0 for an unknown dtype or n > 2^44). */
+WC_API uint64_t wc_host_encode_footprint(uint64_t n, int32_t dtype);
+WC_API uint64_t wc_host_decode_footprint(uint64_t cont_bytes, uint64_t n, int32_t dtype);
+
+/* The window plan the two calls use (host arithmetic only, no CUDA call):
+ * *slots = 3, 2 or 1 -- the most slots of 256-byte rounded (slot_area /
+ * slots) bytes that each hold the largest footprint plus 256 -- and greedy
+ * windows of consecutive items whose footprints plus 256 stay within
+ * min(slot, window_bytes) (window_bytes = 0: the slot), except that an item
+ * larger than that gets a window of its own.  Window w holds items
+ * [window_end[w-1], window_end[w]) (window_end[-1] = 0); *n_windows <= count
+ * and window_end needs room for count entries.  Smaller windows give the
+ * pipeline more stages to overlap.  WC_ERR_CAPACITY if no slot count fits,
+ * WC_ERR_INVALID_ARG for a null pointer or a zero footprint. */
+WC_API int32_t wc_host_plan(const uint64_t *h_footprints, uint32_t count, uint64_t slot_area,
+                            uint64_t window_bytes, uint32_t *slots, uint32_t *window_end,
+                            uint32_t *n_windows);
+
+WC_API int32_t wc_encode_host(const wc_host_encode_item *h_items, uint32_t count, void *d_work,
+                              uint64_t work_cap, uint64_t window_bytes, void *stream_in,
+                              void *stream_compute, void *stream_out);
+
+/* *h_status: WC_OK, or the device status of the first window with a
+ * rejected container (its outputs are then undefined). */
+WC_API int32_t wc_decode_host(const wc_host_decode_item *h_items, uint32_t count, void *d_work,
+                              uint64_t work_cap, uint64_t window_bytes, void *stream_in,
+                              void *stream_compute, void *stream_out, int32_t *h_status);
+
 /* Human-readable name of a wc_status code (static storage). */
 WC_API const char *wc_status_string(int32_t status);
 
