@@ -188,6 +188,25 @@ CODER_SOURCES = ["fp32_weight_compression_b200/csrc/k_encode.cu",
 
 
 # ---------------------------------------------------------------------------
+def max_over_ranks(vals, dev, world):
+    """Element-wise maximum of per-rank timings (seconds) over all ranks; every
+    rank gets the result.  The only collective of a multi-GPU run: the path
+    itself has no exchange (each rank encodes and decodes its own set)."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_gbs(world, bytes_per_rank, steps, seconds):
+    """Whole-job throughput: the bytes all ranks processed over the slowest
+    rank's time."""
+    return world * bytes_per_rank * steps / seconds / 1e9
+
+
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, on the host cores,
     rank 0 only.  Each step is a bounded sample of the workload: one tensor
@@ -260,10 +279,7 @@ def e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world):
     torch.cuda.synchronize(dev)
     t_e2e = e0.elapsed_time(e1) / 1e3
     assert torch.equal(host_out, host_in), "end-to-end round trip is not bit-exact"
-    if world > 1:
-        tt = torch.tensor([t_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_e2e = tt.item()
+    t_e2e, = max_over_ranks([t_e2e], dev, world)
     return t_e2e, E
 
 
@@ -362,10 +378,7 @@ def main():
     t_enc = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
     t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
     dec.check()
-    if world > 1:
-        tt = torch.tensor([t_total, t_enc, t_dec], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_total, t_enc, t_dec = tt.tolist()
+    t_total, t_enc, t_dec = max_over_ranks([t_total, t_enc, t_dec], dev, world)
 
     t_e2e, E = e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world)
 
@@ -377,7 +390,7 @@ def main():
     dec_gbs = B * K / t_dec / 1e9
     dec_achieved = dec_bytes * K / t_dec / 1e9
     enc_achieved = enc_bytes * K / t_enc / 1e9
-    value = world * B * K / t_total / 1e9
+    value = job_gbs(world, B, K, t_total)
     traffic = recorded_traffic("k_decode", DECODE_SOURCES)
     line = {
         "metric": METRIC,
@@ -405,7 +418,7 @@ def main():
                      "peak_note": peak_note,
                      "algorithmic_bytes_per_launch": dec_bytes},
         "e2e": None if t_e2e is None else {
-            "value": world * B * E / t_e2e / 1e9, "unit": "GB/s",
+            "value": job_gbs(world, B, E, t_e2e), "unit": "GB/s",
             "h2d_bytes_per_step": B + total_cont, "d2h_bytes_per_step": total_cont + B + 8 * len(arrs),
             "steps": E},
         "gpu_launches": K * 5,

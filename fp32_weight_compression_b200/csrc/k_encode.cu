@@ -3,8 +3,8 @@
 //
 // A block of 8 warps codes 16 consecutive chunks of one tensor, two per warp
 // (one rANS state per lane per chunk, symbol i in lane i mod 32).  Two full
-// bf16 chunks are coded in lock-step, so every lane carries two independent
-// state chains; other chunks are coded one at a time.  A warp walks a chunk
+// chunks (bf16 or fp32) are coded in lock-step, so every lane carries two
+// independent state chains; other chunks are coded one at a time.  A warp walks a chunk
 // backwards in groups of 512 values (16 steps): each lane loads its 16
 // consecutive values, writes their raw planes straight into the container's
 // raw section (bf16: the sign+mantissa byte; fp32: sign bits and 3
@@ -232,6 +232,85 @@ __device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, 
   finish_chunk(co, kA + 1, kChunk, xB, tB, bailB, lane);
 }
 
+// 16 consecutive fp32 values of one lane.
+struct Fp32x16 {
+  uint4 a, b, c, d;
+};
+
+__device__ __forceinline__ void load_fp32x16(const uint32_t *p, Fp32x16 &v) {
+  v.a = ld_nc_v4(p);
+  v.b = ld_nc_v4(p + 4);
+  v.c = ld_nc_v4(p + 8);
+  v.d = ld_nc_v4(p + 12);
+}
+
+// Raw planes of 16 fp32 values (value vg is a multiple of 16) into the
+// container; their exponent bytes into eb.
+__device__ __forceinline__ void split_fp32x16(const Fp32x16 &v, uint8_t *out, const Layout &L,
+                                              uint64_t vg, uint8_t *eb) {
+  const uint32_t sb = sign4_fp32(v.a) | (sign4_fp32(v.b) << 4) | (sign4_fp32(v.c) << 8) |
+                      (sign4_fp32(v.d) << 12);
+  *reinterpret_cast<uint16_t *>(out + L.off_raw + vg / 8) = uint16_t(sb);
+  const uint3 m0 = mant4_fp32(v.a), m1 = mant4_fp32(v.b), m2 = mant4_fp32(v.c), m3 = mant4_fp32(v.d);
+  uint8_t *md = out + L.off_mant + 3 * vg;
+  st_cs_v4(md, make_uint4(m0.x, m0.y, m0.z, m1.x));
+  st_cs_v4(md + 16, make_uint4(m1.y, m1.z, m2.x, m2.y));
+  st_cs_v4(md + 32, make_uint4(m2.z, m3.x, m3.y, m3.z));
+  *reinterpret_cast<uint4 *>(eb) = make_uint4(exp4_fp32(v.a), exp4_fp32(v.b), exp4_fp32(v.c), exp4_fp32(v.d));
+}
+
+// Two full fp32 chunks kA, kA + 1 in lock-step (as code_pair_bf16; the next
+// group's values are loaded into the registers the current group's split
+// has just freed).
+template <bool W>
+__device__ void code_pair_fp32(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
+                               const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = lanemask_lt();
+  const uint64_t vgA = kA * kChunk, vgB = vgA + kChunk;
+  const uint32_t *in32 = reinterpret_cast<const uint32_t *>(it.in);
+  uint16_t *wA = reinterpret_cast<uint16_t *>(co.win0 + kA * kWin);
+  uint16_t *wB = reinterpret_cast<uint16_t *>(co.win0 + (kA + 1) * kWin);
+  uint32_t xA = kStateLow, xB = kStateLow, tA = kWinWords, tB = kWinWords;
+  bool bailA = false, bailB = false;
+  constexpr int NG = int(kChunk / kGroupValues);
+
+  Fp32x16 vA, vB;
+  {
+    const uint64_t o = uint64_t(NG - 1) * kGroupValues + 16 * lane;
+    load_fp32x16(in32 + vgA + o, vA);
+    load_fp32x16(in32 + vgB + o, vB);
+  }
+  for (int G = NG - 1; G >= 0; --G) {
+    const uint64_t o = uint64_t(G) * kGroupValues + 16 * lane;
+    split_fp32x16(vA, it.out, L, vgA + o, ebA + 16 * lane);
+    split_fp32x16(vB, it.out, L, vgB + o, ebB + 16 * lane);
+    if (G > 0) {
+      load_fp32x16(in32 + vgA + o - kGroupValues, vA);
+      load_fp32x16(in32 + vgB + o - kGroupValues, vB);
+    }
+    __syncwarp();
+    if (!bailA && !bailB) {
+#pragma unroll
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep2<W>(xA, tA, wA, ebA[32 * t + lane], xB, tB, wB, ebB[32 * t + lane], tab, bias, lt);
+    } else if (!bailA) {
+#pragma unroll 4
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep<W>(xA, tA, wA, tab, bias, ebA[32 * t + lane], lt);
+    } else if (!bailB) {
+#pragma unroll 4
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep<W>(xB, tB, wB, tab, bias, ebB[32 * t + lane], lt);
+    }
+    if (kStateBytes + 2 * (kWinWords - tA) >= kChunk) bailA = true;
+    if (kStateBytes + 2 * (kWinWords - tB) >= kChunk) bailB = true;
+    __syncwarp();
+  }
+  finish_chunk(co, kA, kChunk, xA, tA, bailA, lane);
+  finish_chunk(co, kA + 1, kChunk, xB, tB, bailB, lane);
+}
+
 // Any single chunk (either dtype, possibly ragged).
 template <int DT, bool W>
 __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64_t k, int slot,
@@ -337,6 +416,9 @@ __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constan
       code_one<WC_BF16, false>(it, L, kA, 0, co);
       if (hasB) code_one<WC_BF16, false>(it, L, kA + 1, 1, co);
     }
+  } else if (hasB && chunk_nsym(it.n, kA + 1) == kChunk) {
+    if (wide) code_pair_fp32<true>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+    else code_pair_fp32<false>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
   } else if (wide) {
     code_one<WC_FP32, true>(it, L, kA, 0, co);
     if (hasB) code_one<WC_FP32, true>(it, L, kA + 1, 1, co);
