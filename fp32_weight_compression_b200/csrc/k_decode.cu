@@ -388,8 +388,9 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   // Raw planes are prefetched S half-groups ahead into S register sets used
   // in rotation; the loop is unrolled S times so each set is consumed where it
   // was loaded (no register moves that would wait on loads in flight).  fp32
-  // needs 3x the raw bytes per value, so it keeps fewer sets in registers.
-  constexpr int S = DT == WC_BF16 ? 4 : 2;
+  // needs 3.5x the raw bytes per value: one set, loaded a half-group ahead,
+  // keeps it clear of register spills.
+  constexpr int S = DT == WC_BF16 ? 4 : 1;
   Raw8<DT> pa[S], pb[S];
 #pragma unroll
   for (int j = 0; j < S; j++) {
