@@ -401,22 +401,31 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
 #pragma unroll
     for (int j = 0; j < S; j++) {
       const uint32_t h = h0 + j;
-      const uint32_t f0A = ra.top(cA >> 1, lane), f0B = rb.top(cB >> 1, lane);
-      cp_async_commit();
-      // wait only when a word this half-group may read is not known to have
-      // landed (a wait is followed by __syncwarp, so landed words are visible
-      // to every lane)
-      const uint32_t needA = min((cA >> 1) + kHalf, ra.avail);
-      const uint32_t needB = min((cB >> 1) + kHalf, rb.avail);
-      if (needA > ra.landed || needB > rb.landed) {
-        const int d = min(ra.depth(needA, f0A), rb.depth(needB, f0B));
-        cp_async_wait_depth(d);
-        ra.landed = ra.frontier(d, f0A);
-        rb.landed = rb.frontier(d, f0B);
+      // The ring is checked every kSpan half-groups: up to kSpan units are
+      // issued and the words of the next kSpan half-groups (at most
+      // kSpan * 256; the ring keeps >= 769 requested ahead) must have landed;
+      // a wait happens only when some of them are not known to have.  A wait
+      // is followed by __syncwarp, so landed words are visible to every lane.
+      constexpr int kSpan = S >= 2 ? 2 : 1;
+      if (j % kSpan == 0) {
+        const uint32_t f0A = ra.top(cA >> 1, lane), f0B = rb.top(cB >> 1, lane);
+        if (kSpan == 2) {
+          ra.top(cA >> 1, lane);
+          rb.top(cB >> 1, lane);
+        }
+        cp_async_commit();
+        const uint32_t needA = min((cA >> 1) + kSpan * kHalf, ra.avail);
+        const uint32_t needB = min((cB >> 1) + kSpan * kHalf, rb.avail);
+        if (needA > ra.landed || needB > rb.landed) {
+          const int d = min(ra.depth(needA, f0A), rb.depth(needB, f0B));
+          cp_async_wait_depth(d);
+          ra.landed = ra.frontier(d, f0A);
+          rb.landed = rb.frontier(d, f0B);
+        }
+        ra.shift(f0A);
+        rb.shift(f0B);
+        __syncwarp();
       }
-      ra.shift(f0A);
-      rb.shift(f0B);
-      __syncwarp();
 #pragma unroll
       for (int t = 0; t < 8; t++)
         dstep2(xA, cA, xB, cB, tab, rsA, rsB, tbA + 32 * t + lane, tbB + 32 * t + lane, lt);
