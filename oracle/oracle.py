@@ -22,7 +22,7 @@ SRC = os.path.join(HERE, "wc_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CORRUPT = 0, 1, 2, 4
-BF16, FP32 = 1, 2
+BF16, FP32, FP16 = 1, 2, 3
 CHUNK = 65536
 
 
@@ -57,6 +57,7 @@ def lib():
         L.oracle_encode_bound.argtypes = [ctypes.c_uint64, ctypes.c_int]
         L.oracle_split_bf16.argtypes = [vp, ctypes.c_uint64, vp, vp]
         L.oracle_split_fp32.argtypes = [vp, ctypes.c_uint64, vp, vp, vp]
+        L.oracle_split_fp16.argtypes = [vp, ctypes.c_uint64, vp, vp]
         L.oracle_histogram.argtypes = [vp, ctypes.c_uint64, vp]
         L.oracle_normalize.argtypes = [vp, vp]
         L.oracle_rans_encode.argtypes = [vp, ctypes.c_uint32, vp, ctypes.c_uint32, vp, vp, u32p]
@@ -85,7 +86,9 @@ def dtype_code(arr: np.ndarray) -> int:
         return BF16
     if arr.dtype == np.uint32:
         return FP32
-    raise TypeError("oracle takes bf16 bits as uint16 or fp32 bits as uint32")
+    if arr.dtype == np.float16:
+        return FP16
+    raise TypeError("oracle takes bf16 bits as uint16, fp32 bits as uint32, fp16 as float16")
 
 
 class OracleError(RuntimeError):
@@ -105,6 +108,15 @@ def split_bf16(bits: np.ndarray):
     sm = np.empty(n, np.uint8)
     lib().oracle_split_bf16(_ptr(bits), n, _ptr(e), _ptr(sm))
     return e, sm
+
+
+def split_fp16(bits: np.ndarray):
+    """(coded high-byte plane, raw low-byte plane) of fp16 bits (uint16)."""
+    bits = np.ascontiguousarray(bits).view(np.uint16).reshape(-1)
+    hi = np.zeros(bits.size, np.uint8)
+    lo = np.zeros(bits.size, np.uint8)
+    lib().oracle_split_fp16(_ptr(bits), bits.size, _ptr(hi), _ptr(lo))
+    return hi, lo
 
 
 def split_fp32(bits: np.ndarray):
@@ -166,10 +178,13 @@ def rans_decode(states, words, nsym: int, freq, lanes: int = 32):
     return st, out[:nsym]
 
 
-def encode(bits: np.ndarray) -> np.ndarray:
-    """Container bytes for a flat array of bf16 (uint16) or fp32 (uint32) bits."""
+def encode(bits: np.ndarray, dtype: int | None = None) -> np.ndarray:
+    """Container bytes for a flat array of bf16 (uint16) or fp32 (uint32) bits,
+    or fp16 values (float16, or uint16 bits with dtype=FP16)."""
     bits = np.ascontiguousarray(bits).reshape(-1)
-    dt = dtype_code(bits)
+    dt = dtype_code(bits) if dtype is None else dtype
+    if dt == FP16:
+        bits = bits.view(np.uint16)
     n = bits.size
     cap = encode_bound(n, dt)
     out = np.empty(cap, np.uint8)
@@ -202,7 +217,7 @@ def decode_status(cont: np.ndarray, n_hint: int | None = None, dtype_hint: int |
                                   ctypes.byref(nc))
     if st:
         return st, None
-    npdt = np.uint16 if dt.value == BF16 else np.uint32
+    npdt = np.uint32 if dt.value == FP32 else np.uint16
     out = np.zeros(max(n.value, 1), npdt)
     st = lib().oracle_decode(_ptr(cont), cont.size, _ptr(out), out.nbytes)
     return st, out[: n.value]
@@ -218,7 +233,7 @@ def decode(cont: np.ndarray) -> np.ndarray:
 def decode_chunk(cont: np.ndarray, k: int) -> np.ndarray:
     cont = np.ascontiguousarray(cont, dtype=np.uint8)
     n, dt, nc = read_header(cont)
-    npdt = np.uint16 if dt == BF16 else np.uint32
+    npdt = np.uint32 if dt == FP32 else np.uint16
     nsym = min(CHUNK, n - k * CHUNK) if k < nc else 0
     out = np.zeros(max(nsym, 1), npdt)
     st = lib().oracle_decode_chunk(_ptr(cont), cont.size, k, _ptr(out), out.nbytes)

@@ -18,7 +18,11 @@
  *    "PTWM", "How it works" 1. Bit reorder and 2. Byte / nibble split).  For
  *    bf16 the exponent byte is the high byte after the reorder
  *    [S E M] -> [E S M], and the low byte holds the sign above the 7 mantissa
- *    bits.  For fp32 the container keeps three streams: sign bits, the 8-bit
+ *    bits.  For fp16 the same reorder and 2-plane byte split give a coded
+ *    high byte of 5 exponent bits, the sign and the top 2 mantissa bits, and
+ *    a raw low byte of the other 8 mantissa bits ("PTWM", "How it works" 2:
+ *    float16 / bfloat16 are split into 2 byte planes, plane 1 = exponent).
+ *    For fp32 the container keeps three streams: sign bits, the 8-bit
  *    exponent, and the 23-bit mantissa stored as 3 little-endian bytes.
  *
  *  - Entropy coder.  Only the exponent plane is coded, with static rANS ("SMEF
@@ -43,13 +47,13 @@
  *
  * Container layout (all fields little-endian, sections 16-byte aligned,
  * padding bytes zero):
- *   0  "WCZ1"            4  u16 version = 1    6  u8 dtype (1 bf16, 2 fp32)
+ *   0  "WCZ1"            4  u16 version = 1    6  u8 dtype (1 bf16, 2 fp32, 3 fp16)
  *   7  u8 lanes = 32     8  u64 n              16 u32 chunk symbols = 65536
  *   20 u32 nc            24 u16 prob bits = 12 26 u16 0      28 u32 0
  *   32 u64 off_raw       40 u64 off_exp        48 u64 exp_bytes
  *   56 u64 total_bytes   64 u16 freq[256]      576 u64 chunk_off[nc + 1]
  *   then u32 chunk_len[nc]; pad; raw section; pad; exponent section.
- *   bf16 raw section: n sign+mantissa bytes.
+ *   bf16 raw section: n sign+mantissa bytes; fp16: n low bytes.
  *   fp32 raw section: ceil(n/8) sign bytes (value 8j+b is bit b of byte j),
  *   pad, then 3n mantissa bytes.
  *   Exponent section: chunk k at off_exp + chunk_off[k], chunk_len[k] bytes,
@@ -116,7 +120,7 @@ static void or_make_layout(uint64_t n, int dtype, or_layout *lay) {
     lay->off_chunk_off = OR_CHUNK_OFF_OFFSET;
     lay->off_chunk_len = lay->off_chunk_off + 8 * (lay->nc + 1);
     lay->off_raw = round_up16(lay->off_chunk_len + 4 * lay->nc);
-    if (dtype == OR_BF16) {
+    if (dtype == OR_BF16 || dtype == OR_FP16) {
         lay->off_sign = 0;
         lay->off_mant = 0;
         lay->off_exp = round_up16(lay->off_raw + n);
@@ -133,9 +137,16 @@ static uint32_t or_chunk_nsym(uint64_t n, uint64_t k) {
     return (uint32_t)(left < OR_CHUNK_SYMBOLS ? left : OR_CHUNK_SYMBOLS);
 }
 
+static int or_dtype_ok(int dtype) {
+    return dtype == OR_BF16 || dtype == OR_FP32 || dtype == OR_FP16;
+}
+
+/* Bytes per value of a dtype. */
+static uint64_t or_elem(int dtype) { return dtype == OR_FP32 ? 4 : 2; }
+
 uint64_t oracle_encode_bound(uint64_t n, int dtype) {
     or_layout lay;
-    if (dtype != OR_BF16 && dtype != OR_FP32) return 0;
+    if (!or_dtype_ok(dtype)) return 0;
     or_make_layout(n, dtype, &lay);
     uint64_t exp_bytes = 0;
     for (uint64_t k = 0; k < lay.nc; k++) exp_bytes += round_up16(or_chunk_nsym(n, k));
@@ -175,6 +186,23 @@ void oracle_split_fp32(const uint32_t *in, uint64_t n, uint8_t *exp_plane,
         mant3[3 * i + 0] = (uint8_t)(mant & 0xFFu);
         mant3[3 * i + 1] = (uint8_t)((mant >> 8) & 0xFFu);
         mant3[3 * i + 2] = (uint8_t)((mant >> 16) & 0xFFu);
+    }
+}
+
+/* fp16 bits b = [S:1][E:5][M:10].  The reorder puts E on top with S below
+ * it: r = E<<11 | S<<10 | M; the byte split gives the high byte r >> 8
+ * (E, S and the top two mantissa bits; the coded plane) and the low byte
+ * r & 0xFF (the low eight mantissa bits; stored raw). */
+void oracle_split_fp16(const uint16_t *in, uint64_t n, uint8_t *hi_plane,
+                       uint8_t *lo_plane) {
+    for (uint64_t i = 0; i < n; i++) {
+        uint16_t b = in[i];
+        uint16_t sign = (uint16_t)((b >> 15) & 1u);
+        uint16_t expo = (uint16_t)((b >> 10) & 0x1Fu);
+        uint16_t mant = (uint16_t)(b & 0x3FFu);
+        uint16_t r = (uint16_t)((expo << 11) | (sign << 10) | mant);
+        hi_plane[i] = (uint8_t)(r >> 8);
+        lo_plane[i] = (uint8_t)(r & 0xFFu);
     }
 }
 
@@ -413,7 +441,7 @@ int oracle_chunk_accounting(const uint8_t *sym, uint32_t nsym,
 /* ------------------------------------------------------------------ */
 int oracle_encode(const void *in, uint64_t n, int dtype, uint8_t *out,
                   uint64_t out_cap, uint64_t *out_size) {
-    if (dtype != OR_BF16 && dtype != OR_FP32) return OR_ERR_INVALID_ARG;
+    if (!or_dtype_ok(dtype)) return OR_ERR_INVALID_ARG;
     if (n > 0 && in == NULL) return OR_ERR_INVALID_ARG;
     if (out == NULL || out_size == NULL) return OR_ERR_INVALID_ARG;
     if (out_cap < oracle_encode_bound(n, dtype)) return OR_ERR_CAPACITY;
@@ -427,6 +455,8 @@ int oracle_encode(const void *in, uint64_t n, int dtype, uint8_t *out,
     if (!expo) return OR_ERR_INVALID_ARG;
     if (dtype == OR_BF16)
         oracle_split_bf16((const uint16_t *)in, n, expo, out + lay.off_raw);
+    else if (dtype == OR_FP16)
+        oracle_split_fp16((const uint16_t *)in, n, expo, out + lay.off_raw);
     else
         oracle_split_fp32((const uint32_t *)in, n, expo, out + lay.off_sign,
                           out + lay.off_mant);
@@ -503,7 +533,7 @@ static int or_parse(const uint8_t *c, uint64_t bytes, or_header *h) {
     if (c[0] != 'W' || c[1] != 'C' || c[2] != 'Z' || c[3] != '1') return OR_ERR_CORRUPT;
     if (get_u16(c + 4) != 1) return OR_ERR_CORRUPT;
     int dtype = c[6];
-    if (dtype != OR_BF16 && dtype != OR_FP32) return OR_ERR_CORRUPT;
+    if (!or_dtype_ok(dtype)) return OR_ERR_CORRUPT;
     if (c[7] != OR_LANES) return OR_ERR_CORRUPT;
     uint64_t n = get_u64(c + 8);
     if (get_u32(c + 16) != OR_CHUNK_SYMBOLS) return OR_ERR_CORRUPT;
@@ -583,6 +613,13 @@ static int or_decode_one_chunk(const uint8_t *c, const or_header *h, uint64_t k,
             uint16_t sign = (uint16_t)((sm >> 7) & 1u);
             uint16_t mant = (uint16_t)(sm & 0x7Fu);
             ((uint16_t *)out_vals)[j] = (uint16_t)((sign << 15) | ((uint16_t)expo[j] << 7) | mant);
+        } else if (h->dtype == OR_FP16) {
+            /* undo the byte split, then the reorder E S M -> S E M */
+            uint16_t r = (uint16_t)(((uint16_t)expo[j] << 8) | c[h->lay.off_raw + i]);
+            uint16_t e5 = (uint16_t)(r >> 11);
+            uint16_t sign = (uint16_t)((r >> 10) & 1u);
+            uint16_t mant = (uint16_t)(r & 0x3FFu);
+            ((uint16_t *)out_vals)[j] = (uint16_t)((sign << 15) | (e5 << 10) | mant);
         } else {
             uint32_t sign = (c[h->lay.off_sign + i / 8] >> (i % 8)) & 1u;
             const uint8_t *m = c + h->lay.off_mant + 3 * i;
@@ -598,7 +635,7 @@ int oracle_decode(const uint8_t *cont, uint64_t cont_bytes, void *out,
     or_header h;
     int st = or_parse(cont, cont_bytes, &h);
     if (st != OR_OK) return st;
-    uint64_t elem = h.dtype == OR_BF16 ? 2 : 4;
+    uint64_t elem = or_elem(h.dtype);
     if (h.lay.n * elem > out_cap) return OR_ERR_CAPACITY;
     if (h.lay.n > 0 && out == NULL) return OR_ERR_INVALID_ARG;
     uint8_t *expo = (uint8_t *)malloc(OR_CHUNK_SYMBOLS);
@@ -619,7 +656,7 @@ int oracle_decode_chunk(const uint8_t *cont, uint64_t cont_bytes, uint64_t k,
     int st = or_parse(cont, cont_bytes, &h);
     if (st != OR_OK) return st;
     if (k >= h.lay.nc) return OR_ERR_INVALID_ARG;
-    uint64_t elem = h.dtype == OR_BF16 ? 2 : 4;
+    uint64_t elem = or_elem(h.dtype);
     if ((uint64_t)or_chunk_nsym(h.lay.n, k) * elem > out_cap) return OR_ERR_CAPACITY;
     if (out == NULL) return OR_ERR_INVALID_ARG;
     uint8_t *expo = (uint8_t *)malloc(OR_CHUNK_SYMBOLS);

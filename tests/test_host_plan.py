@@ -72,7 +72,7 @@ def test_footprints(wcm, n, dt):
     assert wcm.host_encode_footprint(n, dt) == (r256(n * e) + r256(wcm.encode_bound(n, dt))
                                                 + r256(wcm.scratch_bytes(n, dt)) + 8)
     assert wcm.host_decode_footprint(1000, n, dt) == r256(1000) + r256(n * e)
-    assert wcm.host_encode_footprint(n, 3) == 0
+    assert wcm.host_encode_footprint(n, 4) == 0
 
 
 def test_bad_arguments_rejected_before_device(wcm, orc):

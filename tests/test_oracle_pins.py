@@ -184,7 +184,46 @@ def test_split_fp32_worked(orc):
     assert mant[:15].tolist() == [0, 0, 0, 0, 0, 0, 1, 0, 0, 0, 0, 0x40, 0xFF, 0xFF, 0x7F]
 
 
+def test_split_fp16_worked(orc):
+    # fp16 S E5 M10; reordered E5 S M10; high byte coded, low byte raw
+    bits = np.array([0x3C00, 0x8001, 0x7C00, 0xFC01, 0x7BFF, 0x3555, 0x0001, 0x8000], np.uint16)
+    hi, lo = orc.split_fp16(bits)
+    assert hi.tolist() == [0x78, 0x04, 0xF8, 0xFC, 0xF3, 0x69, 0x00, 0x04]
+    assert lo.tolist() == [0x00, 0x01, 0x00, 0x01, 0xFF, 0x55, 0x01, 0x00]
+
+
+def test_split_fp16_plane_structure(orc):
+    # the coded byte is exponent << 3 | sign << 2 | top two mantissa bits
+    rng = np.random.default_rng(3)
+    bits = rng.integers(0, 1 << 16, 4096, dtype=np.uint16)
+    hi, lo = orc.split_fp16(bits)
+    b = bits.astype(np.uint32)
+    assert np.array_equal(hi >> 3, (b >> 10) & 0x1F)
+    assert np.array_equal((hi >> 2) & 1, b >> 15)
+    assert np.array_equal(hi & 3, (b >> 8) & 3)
+    assert np.array_equal(lo, b & 0xFF)
+
+
+def test_fp16_all_patterns_round_trip(orc):
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    cont = orc.encode(bits, dtype=orc.FP16)
+    assert orc.read_header(cont) == (1 << 16, orc.FP16, 1)
+    assert np.array_equal(orc.decode(cont), bits)
+    vals = (np.random.default_rng(4).standard_normal(5 * 65536 + 7) * 0.02).astype(np.float16)
+    cont = orc.encode(vals)
+    assert np.array_equal(orc.decode(cont), vals.view(np.uint16))
+    assert cont.size < vals.nbytes          # the coded plane shrinks
+
+
 # ---------------------------------------------------------------- containers
+def test_golden_container_fp16_raw_chunk(orc):
+    bits = np.array([0x3C00, 0x3C00, 0x3C00, 0x3800], np.uint16)
+    want = load_container("container_fp16_n4_raw.txt")
+    got = orc.encode(bits, dtype=orc.FP16)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert orc.decode(got).tolist() == bits.tolist()
+
+
 def test_golden_container_raw_chunk(orc):
     bits = np.array([0x3F80, 0x3F80, 0x3F80, 0x3F00], np.uint16)
     want = load_container("container_bf16_n4_raw.txt")
