@@ -9,6 +9,7 @@
 //                does not compress is stored as it is).
 #include "wc_block.cuh"
 #include "wc_format.cuh"
+#include "wc_planes.cuh"
 
 namespace wc {
 
@@ -48,8 +49,9 @@ __global__ void __launch_bounds__(kCompactThreads) k_compact(const __grid_consta
 
   if (len == nsym) {
     const uint32_t ngran = uint32_t(round16(nsym) / 16);
-    if (dtype == WC_BF16) {
+    if (dtype != WC_FP32) {
       const uint16_t *src = reinterpret_cast<const uint16_t *>(it.in) + k * kChunk;
+      const bool bf = dtype == WC_BF16;
       for (uint32_t gi = tid; gi < ngran; gi += kCompactThreads) {
         const uint32_t v0 = gi * 16;
         uint32_t w[8];
@@ -65,10 +67,13 @@ __global__ void __launch_bounds__(kCompactThreads) k_compact(const __grid_consta
           }
         }
         uint4 e;
-        e.x = __byte_perm(w[0] >> 7, w[1] >> 7, 0x6420);
-        e.y = __byte_perm(w[2] >> 7, w[3] >> 7, 0x6420);
-        e.z = __byte_perm(w[4] >> 7, w[5] >> 7, 0x6420);
-        e.w = __byte_perm(w[6] >> 7, w[7] >> 7, 0x6420);
+        if (bf) {
+          e.x = code4<WC_BF16>(w[0], w[1]); e.y = code4<WC_BF16>(w[2], w[3]);
+          e.z = code4<WC_BF16>(w[4], w[5]); e.w = code4<WC_BF16>(w[6], w[7]);
+        } else {
+          e.x = code4<WC_FP16>(w[0], w[1]); e.y = code4<WC_FP16>(w[2], w[3]);
+          e.z = code4<WC_FP16>(w[4], w[5]); e.w = code4<WC_FP16>(w[6], w[7]);
+        }
         if (v0 + 16 > nsym) {  // zero the padding bytes
           const int keep = int(nsym - v0);
           e.x = keep_bytes(e.x, keep); e.y = keep_bytes(e.y, keep - 4);

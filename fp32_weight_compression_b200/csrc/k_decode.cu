@@ -26,6 +26,7 @@
 // No loop waits on another block; each wait is on this warp's own copies.
 #include "wc_block.cuh"
 #include "wc_format.cuh"
+#include "wc_planes.cuh"
 
 namespace wc {
 
@@ -90,7 +91,7 @@ __device__ __noinline__ ItemView view_item(const DecItem &it) {
   const uint32_t w1 = h32[1];
   const int dtype = int((w1 >> 16) & 0xFF);
   if (h32[0] != 0x315A4357u || (w1 & 0xFFFF) != kVersion || (w1 >> 24) != kLanes) return v;
-  if (dtype != WC_BF16 && dtype != WC_FP32) return v;
+  if (dtype != WC_BF16 && dtype != WC_FP32 && dtype != WC_FP16) return v;
   const uint64_t n = h64[1];
   if (n > (uint64_t(1) << 44)) return v;
   if (h32[4] != kChunk || h32[6] != kProbBits || h32[7] != 0) return v;
@@ -109,7 +110,7 @@ __device__ __noinline__ ItemView view_item(const DecItem &it) {
     v.first = it.chunk_first;
     v.cnt = min(it.chunk_count, L.nc - it.chunk_first);
   }
-  const uint64_t elem = dtype == WC_BF16 ? 2 : 4;
+  const uint64_t elem = dtype == WC_FP32 ? 4 : 2;
   const uint64_t vals = v.cnt == 0 ? 0
                         : (v.first + v.cnt == L.nc ? n - v.first * kChunk : v.cnt * kChunk);
   if (vals * elem > it.out_cap || (vals > 0 && it.out == nullptr)) { v.err = WC_ERR_CAPACITY; return v; }
@@ -142,7 +143,7 @@ __device__ __forceinline__ ChunkView view_chunk(const DecItem &it, const ItemVie
   c.ok = (c.raw || coded) && o0 <= o1 && o1 - o0 == round16(c.len) && o1 <= exp_bytes &&
          (k != 0 || o0 == 0) && (k + 1 != L.nc || o1 == exp_bytes);
   c.pay = cont + L.off_exp + o0;
-  constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
+  constexpr uint32_t elem = DT == WC_FP32 ? 4 : 2;
   c.out = it.out + (k - v.first) * kChunk * elem;
   return c;
 }
@@ -151,14 +152,14 @@ __device__ __forceinline__ ChunkView view_chunk(const DecItem &it, const ItemVie
 // Raw-plane bytes of 8 consecutive values and the merge.
 template <int DT>
 struct Raw8 {
-  uint2 a;        // bf16: 8 sign+mantissa bytes; fp32: mantissa bytes 0..7
+  uint2 a;        // bf16 / fp16: the 8 raw bytes; fp32: mantissa bytes 0..7
   uint2 b, c;     // fp32: mantissa bytes 8..23
   uint32_t s;     // fp32: 8 sign bits
 };
 
 template <int DT>
 __device__ __forceinline__ void load_raw8(const uint8_t *cont, const Layout &L, uint64_t vg, Raw8<DT> &r) {
-  if (DT == WC_BF16) {
+  if (DT != WC_FP32) {
     r.a = __ldg(reinterpret_cast<const uint2 *>(cont + L.off_raw + vg));
   } else {
     r.s = __ldg(cont + L.off_raw + vg / 8);
@@ -167,14 +168,6 @@ __device__ __forceinline__ void load_raw8(const uint8_t *cont, const Layout &L, 
     r.b = __ldg(m + 1);
     r.c = __ldg(m + 2);
   }
-}
-
-// 4 bf16 values from 4 exponent bytes and 4 sign+mantissa bytes, byte-parallel:
-// low byte = (sm & 0x7F) | (e & 1) << 7, high byte = e >> 1 | (sm & 0x80).
-__device__ __forceinline__ uint2 merge4_bf16(uint32_t e4, uint32_t s4) {
-  const uint32_t lo = (s4 & 0x7F7F7F7Fu) | ((e4 << 7) & 0x80808080u);
-  const uint32_t hi = ((e4 >> 1) & 0x7F7F7F7Fu) | (s4 & 0x80808080u);
-  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
 // fp32 value j of 4 from 3 mantissa words: u = s << 31 | e << 23 | m
@@ -192,12 +185,13 @@ __device__ __forceinline__ uint4 merge4_fp32(uint32_t e4, uint32_t w0, uint32_t 
   return o;
 }
 
-// 8 values (exponents e8 = 8 bytes) -> output at dst (16-byte aligned).
+// 8 values (coded bytes e8 = 8 bytes) -> output at dst (16-byte aligned);
+// 2-byte values merge byte-parallel (merge4, wc_planes.cuh).
 template <int DT>
 __device__ __forceinline__ void merge_store8(uint2 e8, const Raw8<DT> &r, uint8_t *dst) {
-  if (DT == WC_BF16) {
-    const uint2 p = merge4_bf16(e8.x, r.a.x);
-    const uint2 q = merge4_bf16(e8.y, r.a.y);
+  if (DT != WC_FP32) {
+    const uint2 p = merge4<DT>(e8.x, r.a.x);
+    const uint2 q = merge4<DT>(e8.y, r.a.y);
     st_cs_v4(dst, make_uint4(p.x, p.y, q.x, q.y));
   } else {
     // mantissa words: a.x a.y b.x | b.y c.x c.y
@@ -210,10 +204,8 @@ __device__ __forceinline__ void merge_store8(uint2 e8, const Raw8<DT> &r, uint8_
 template <int DT>
 __device__ __forceinline__ void merge_store1(uint32_t e, const uint8_t *cont, const Layout &L, uint64_t vg,
                                              uint8_t *dst) {
-  if (DT == WC_BF16) {
-    const uint32_t sm = cont[L.off_raw + vg];
-    reinterpret_cast<uint16_t *>(dst)[0] =
-        uint16_t(((sm & 0x80u) << 8) | (e << 7) | (sm & 0x7Fu));
+  if (DT != WC_FP32) {
+    reinterpret_cast<uint16_t *>(dst)[0] = uint16_t(merge16<DT>(e, cont[L.off_raw + vg]));
   } else {
     const uint32_t s = (cont[L.off_raw + vg / 8] >> (vg & 7)) & 1u;
     const uint8_t *m = cont + L.off_mant + 3 * vg;
@@ -301,7 +293,7 @@ struct RawPtrs {
 
 template <int DT>
 __device__ __forceinline__ void load_raw8p(const RawPtrs &p, uint32_t vl, Raw8<DT> &r) {
-  if (DT == WC_BF16) {
+  if (DT != WC_FP32) {
     r.a = __ldg(reinterpret_cast<const uint2 *>(p.a + vl));
   } else {
     r.s = __ldg(p.s + vl / 8);
@@ -367,12 +359,12 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   const uint32_t rsB = uint32_t(__cvta_generic_to_shared(ring_ptr(warp, 1)));
   uint8_t *tbA = s.tbuf[warp][0], *tbB = s.tbuf[warp][1];
   const uint32_t lt = lanemask_lt();
-  constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
+  constexpr uint32_t elem = DT == WC_FP32 ? 4 : 2;
   Ring ra{rsA, payA + kStateBytes, uint32_t(round16(lenA) - kStateBytes) >> 1, 0, 0, 0, 0};
   Ring rb{rsB, payB + kStateBytes, uint32_t(round16(lenB) - kStateBytes) >> 1, 0, 0, 0, 0};
   RawPtrs rpB;
-  rpB.a = rpA.a + (DT == WC_BF16 ? kChunk : 3 * kChunk);
-  rpB.s = DT == WC_BF16 ? nullptr : rpA.s + kChunk / 8;
+  rpB.a = rpA.a + (DT == WC_FP32 ? 3 * kChunk : kChunk);
+  rpB.s = DT == WC_FP32 ? rpA.s + kChunk / 8 : nullptr;
   uint8_t *outB = outA + kChunk * elem;
   uint32_t xA = reinterpret_cast<const uint32_t *>(payA)[lane];
   uint32_t xB = reinterpret_cast<const uint32_t *>(payB)[lane];
@@ -390,7 +382,7 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   // was loaded (no register moves that would wait on loads in flight).  fp32
   // needs 3.5x the raw bytes per value: one set, loaded a half-group ahead,
   // keeps it clear of register spills.
-  constexpr int S = DT == WC_BF16 ? 4 : 1;
+  constexpr int S = DT == WC_FP32 ? 1 : 4;
   Raw8<DT> pa[S], pb[S];
 #pragma unroll
   for (int j = 0; j < S; j++) {
@@ -460,7 +452,7 @@ __device__ __noinline__ void decode_one(const ItemView &v, const DecItem &it, co
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t lt = lanemask_lt();
   const Layout &L = v.L;
-  constexpr uint32_t elem = DT == WC_BF16 ? 2 : 4;
+  constexpr uint32_t elem = DT == WC_FP32 ? 4 : 2;
   const uint64_t vg0 = k * kChunk;
   const uint32_t nsym = c.nsym;
   const uint32_t nhalf = (nsym + kHalf - 1) / kHalf;
@@ -602,7 +594,7 @@ __device__ __forceinline__ void decode_warp_chunks(const ItemView &v, const DecI
     const Layout &L = v.L;
     const uint64_t vgA = kA * kChunk;
     RawPtrs rpA;
-    if (DT == WC_BF16) {
+    if (DT != WC_FP32) {
       rpA.a = it.cont + L.off_raw + vgA;
       rpA.s = nullptr;
     } else {
@@ -649,6 +641,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
     const uint64_t kA = v.first + uint64_t(grp - s.gpre[ii]) * kDecGroup + 2 * warp;
     const uint64_t kend = v.first + v.cnt;
     if (v.dtype == WC_BF16) decode_warp_chunks<WC_BF16>(v, it, kA, kend, status);
+    else if (v.dtype == WC_FP16) decode_warp_chunks<WC_FP16>(v, it, kA, kend, status);
     else decode_warp_chunks<WC_FP32>(v, it, kA, kend, status);
   }
 }

@@ -3,14 +3,15 @@
 //
 // A block of 8 warps codes 16 consecutive chunks of one tensor, two per warp
 // (one rANS state per lane per chunk, symbol i in lane i mod 32).  Two full
-// chunks (bf16 or fp32) are coded in lock-step, so every lane carries two
-// independent state chains; other chunks are coded one at a time.  A warp walks a chunk
-// backwards in groups of 512 values (16 steps): each lane loads its 16
-// consecutive values, writes their raw planes straight into the container's
-// raw section (bf16: the sign+mantissa byte; fp32: sign bits and 3
-// little-endian mantissa bytes -- "PTWM" How it works 1-2, "SMEF"
-// pass3_streams.py), and parks their exponent bytes in shared memory, where
-// step t reads byte 32 t + lane.  Coding a symbol s with frequency f from
+// chunks (any dtype) are coded in lock-step, so every lane carries two
+// independent state chains; other chunks are coded one at a time.  A warp
+// walks a chunk backwards in groups of 512 values (16 steps): each lane loads
+// its 16 consecutive values, writes their raw planes straight into the
+// container's raw section (bf16: the sign+mantissa byte; fp16: the low byte;
+// fp32: sign bits and 3 little-endian mantissa bytes -- "PTWM" How it works
+// 1-2, "SMEF" pass3_streams.py), and parks their coded bytes (the exponent;
+// for fp16 the reordered high byte) in shared memory, where step t reads byte
+// 32 t + lane.  Coding a symbol s with frequency f from
 // state x (12-bit table, L = 2^16, 16-bit words):
 //   if x >= f 2^20: emit x & 0xFFFF, x >>= 16;   x = (x / f) 4096 + x % f + cum_s
 // with x / f computed exactly by a multiply-high and a shift when every f of
@@ -27,6 +28,7 @@
 // chunk_off[] (16-byte rounded) and chunk_len[] and completes the header.
 #include "wc_block.cuh"
 #include "wc_format.cuh"
+#include "wc_planes.cuh"
 
 namespace wc {
 
@@ -39,28 +41,21 @@ __shared__ uint32_t s_bias[256];
 __shared__ __align__(16) uint8_t s_ebuf[kCoderWarps][2][kGroupValues];
 
 // ---------------------------------------------------------------------------
-// 16 consecutive bf16 values (8 words) of one lane: exponents and raw plane.
-struct Bf16x16 {
+// 16 consecutive 2-byte values (bf16 or fp16, 8 words) of one lane: their
+// coded bytes and raw bytes (wc_planes.cuh).
+struct V16x16 {
   uint4 a, b;
 };
 
-__device__ __forceinline__ uint32_t exp4_bf16(uint32_t w0, uint32_t w1) {
-  // bf16 word = [v1 : v0]; the exponent of a value is bits 7..14 of its half
-  return __byte_perm(w0 >> 7, w1 >> 7, 0x6420);
+template <int DT>
+__device__ __forceinline__ uint4 codes16(const V16x16 &v) {
+  return make_uint4(code4<DT>(v.a.x, v.a.y), code4<DT>(v.a.z, v.a.w), code4<DT>(v.b.x, v.b.y),
+                    code4<DT>(v.b.z, v.b.w));
 }
-__device__ __forceinline__ uint32_t sm4_bf16(uint32_t w0, uint32_t w1) {
-  // sign+mantissa byte = (high byte & 0x80) | (low byte & 0x7F)
-  const uint32_t lo = __byte_perm(w0, w1, 0x6420);
-  const uint32_t hi = __byte_perm(w0, w1, 0x7531);
-  return (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
-}
-__device__ __forceinline__ uint4 exps_bf16(const Bf16x16 &v) {
-  return make_uint4(exp4_bf16(v.a.x, v.a.y), exp4_bf16(v.a.z, v.a.w), exp4_bf16(v.b.x, v.b.y),
-                    exp4_bf16(v.b.z, v.b.w));
-}
-__device__ __forceinline__ uint4 sms_bf16(const Bf16x16 &v) {
-  return make_uint4(sm4_bf16(v.a.x, v.a.y), sm4_bf16(v.a.z, v.a.w), sm4_bf16(v.b.x, v.b.y),
-                    sm4_bf16(v.b.z, v.b.w));
+template <int DT>
+__device__ __forceinline__ uint4 raws16(const V16x16 &v) {
+  return make_uint4(raw4<DT>(v.a.x, v.a.y), raw4<DT>(v.a.z, v.a.w), raw4<DT>(v.b.x, v.b.y),
+                    raw4<DT>(v.b.z, v.b.w));
 }
 
 // fp32: exponent byte = byte 3 of (u << 1)
@@ -81,10 +76,10 @@ __device__ __forceinline__ uint32_t sign4_fp32(uint4 u) {
 // Raw planes and exponents of one value (ragged tails only).
 template <int DT>
 __device__ __forceinline__ uint32_t one_value(const uint8_t *in, uint64_t vg, uint8_t *out, const Layout &L) {
-  if (DT == WC_BF16) {
+  if (DT != WC_FP32) {
     const uint32_t b = reinterpret_cast<const uint16_t *>(in)[vg];
-    out[L.off_raw + vg] = uint8_t(((b >> 8) & 0x80u) | (b & 0x7Fu));
-    return (b >> 7) & 0xFFu;
+    out[L.off_raw + vg] = uint8_t(raw_byte<DT>(b));
+    return code_byte<DT>(b);
   } else {
     const uint32_t u = reinterpret_cast<const uint32_t *>(in)[vg];
     const uint32_t m = u & 0x7FFFFFu;
@@ -177,9 +172,9 @@ __device__ __forceinline__ void finish_chunk(const CoderOut &co, uint64_t k, uin
   if (lane == 0) co.lens[k] = len;
 }
 
-// Two full bf16 chunks kA, kA + 1 in lock-step.
-template <bool W>
-__device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
+// Two full 2-byte-value chunks (bf16 or fp16) kA, kA + 1 in lock-step.
+template <int DT, bool W>
+__device__ void code_pair16(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
                                const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
@@ -191,7 +186,7 @@ __device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, 
   bool bailA = false, bailB = false;
   constexpr int NG = int(kChunk / kGroupValues);
 
-  Bf16x16 cA, cB, nA, nB;
+  V16x16 cA, cB, nA, nB;
   {
     const uint64_t o = uint64_t(NG - 1) * kGroupValues + 16 * lane;
     cA.a = ld_nc_v4(in16 + vgA + o); cA.b = ld_nc_v4(in16 + vgA + o + 8);
@@ -199,10 +194,10 @@ __device__ void code_pair_bf16(const EncItem &it, const Layout &L, uint64_t kA, 
   }
   for (int G = NG - 1; G >= 0; --G) {
     const uint64_t o = uint64_t(G) * kGroupValues + 16 * lane;
-    st_cs_v4(it.out + L.off_raw + vgA + o, sms_bf16(cA));
-    st_cs_v4(it.out + L.off_raw + vgB + o, sms_bf16(cB));
-    *reinterpret_cast<uint4 *>(ebA + 16 * lane) = exps_bf16(cA);
-    *reinterpret_cast<uint4 *>(ebB + 16 * lane) = exps_bf16(cB);
+    st_cs_v4(it.out + L.off_raw + vgA + o, raws16<DT>(cA));
+    st_cs_v4(it.out + L.off_raw + vgB + o, raws16<DT>(cB));
+    *reinterpret_cast<uint4 *>(ebA + 16 * lane) = codes16<DT>(cA);
+    *reinterpret_cast<uint4 *>(ebB + 16 * lane) = codes16<DT>(cB);
     if (G > 0) {
       const uint64_t on = o - kGroupValues;
       nA.a = ld_nc_v4(in16 + vgA + on); nA.b = ld_nc_v4(in16 + vgA + on + 8);
@@ -259,7 +254,7 @@ __device__ __forceinline__ void split_fp32x16(const Fp32x16 &v, uint8_t *out, co
   *reinterpret_cast<uint4 *>(eb) = make_uint4(exp4_fp32(v.a), exp4_fp32(v.b), exp4_fp32(v.c), exp4_fp32(v.d));
 }
 
-// Two full fp32 chunks kA, kA + 1 in lock-step (as code_pair_bf16; the next
+// Two full fp32 chunks kA, kA + 1 in lock-step (as code_pair16; the next
 // group's values are loaded into the registers the current group's split
 // has just freed).
 template <bool W>
@@ -333,13 +328,13 @@ __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64
     const uint64_t vg = vg0 + vl;
     if (vl + 16 <= nsym) {
       uint4 e;
-      if (DT == WC_BF16) {
+      if (DT != WC_FP32) {
         const uint16_t *p = reinterpret_cast<const uint16_t *>(it.in) + vg;
-        Bf16x16 v;
+        V16x16 v;
         v.a = ld_nc_v4(p);
         v.b = ld_nc_v4(p + 8);
-        st_cs_v4(it.out + L.off_raw + vg, sms_bf16(v));
-        e = exps_bf16(v);
+        st_cs_v4(it.out + L.off_raw + vg, raws16<DT>(v));
+        e = codes16<DT>(v);
       } else {
         const uint32_t *p = reinterpret_cast<const uint32_t *>(it.in) + vg;
         const uint4 u0 = ld_nc_v4(p), u1 = ld_nc_v4(p + 4), u2 = ld_nc_v4(p + 8), u3 = ld_nc_v4(p + 12);
@@ -389,6 +384,19 @@ __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64
   finish_chunk(co, k, nsym, x, tail, bail, lane);
 }
 
+// The warp's two chunks kA and (if hasB) kA + 1.
+template <int DT, bool W>
+__device__ __forceinline__ void code_warp(const EncItem &it, const Layout &L, uint64_t kA, bool hasB,
+                                          int warp, const CoderOut &co) {
+  if (hasB && chunk_nsym(it.n, kA + 1) == kChunk) {
+    if (DT == WC_FP32) code_pair_fp32<W>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+    else code_pair16<DT, W>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+  } else {
+    code_one<DT, W>(it, L, kA, 0, co);
+    if (hasB) code_one<DT, W>(it, L, kA + 1, 1, co);
+  }
+}
+
 __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constant__ EncParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t b = blockIdx.x;
@@ -406,25 +414,15 @@ __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constan
   CoderOut co{reinterpret_cast<uint32_t *>(it.scratch + kScrLen), it.scratch + scratch_win_offset(L.nc)};
   const bool wide = reinterpret_cast<const uint32_t *>(it.scratch + kScrCtr)[2] != 0;
   if (dtype == WC_BF16) {
-    if (hasB && chunk_nsym(it.n, kA + 1) == kChunk) {
-      if (wide) code_pair_bf16<true>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
-      else code_pair_bf16<false>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
-    } else if (wide) {
-      code_one<WC_BF16, true>(it, L, kA, 0, co);
-      if (hasB) code_one<WC_BF16, true>(it, L, kA + 1, 1, co);
-    } else {
-      code_one<WC_BF16, false>(it, L, kA, 0, co);
-      if (hasB) code_one<WC_BF16, false>(it, L, kA + 1, 1, co);
-    }
-  } else if (hasB && chunk_nsym(it.n, kA + 1) == kChunk) {
-    if (wide) code_pair_fp32<true>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
-    else code_pair_fp32<false>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+    if (wide) code_warp<WC_BF16, true>(it, L, kA, hasB, warp, co);
+    else code_warp<WC_BF16, false>(it, L, kA, hasB, warp, co);
+  } else if (dtype == WC_FP16) {
+    if (wide) code_warp<WC_FP16, true>(it, L, kA, hasB, warp, co);
+    else code_warp<WC_FP16, false>(it, L, kA, hasB, warp, co);
   } else if (wide) {
-    code_one<WC_FP32, true>(it, L, kA, 0, co);
-    if (hasB) code_one<WC_FP32, true>(it, L, kA + 1, 1, co);
+    code_warp<WC_FP32, true>(it, L, kA, hasB, warp, co);
   } else {
-    code_one<WC_FP32, false>(it, L, kA, 0, co);
-    if (hasB) code_one<WC_FP32, false>(it, L, kA + 1, 1, co);
+    code_warp<WC_FP32, false>(it, L, kA, hasB, warp, co);
   }
 
   // last warp of the tensor: offset table and the rest of the header

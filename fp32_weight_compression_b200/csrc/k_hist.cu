@@ -6,8 +6,9 @@
 //           container (everything that depends on n alone).
 //  k_hist   one block per tile of up to 4 chunks: reads the values as
 //           integers (a NaN payload is never touched as a float), counts the
-//           8-bit exponents ("PTWM" How it works 1-2: after the bit reorder the
-//           exponent is a whole byte; "SMEF" pass3_streams.py) into a
+//           coded bytes -- the 8-bit exponent of bf16 / fp32, the reordered
+//           high byte of fp16 ("PTWM" How it works 1-2: after the bit reorder
+//           the exponent leads a whole byte; "SMEF" pass3_streams.py) -- into a
 //           shared-memory histogram with one column per lane (so the 32 lanes
 //           of a warp never collide on an address), folds it into the tensor's
 //           global histogram, and the last block of each tensor turns the
@@ -25,6 +26,7 @@
 // above T to T first, and then takes the tied symbols at T in symbol order.
 #include "wc_block.cuh"
 #include "wc_format.cuh"
+#include "wc_planes.cuh"
 
 namespace wc {
 
@@ -67,7 +69,7 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ EncParams 
   if (tid < 16) {
     uint64_t a = L.off_chunk_len + 4 * L.nc + tid;
     if (a < L.off_raw) out[a] = 0;
-    if (dtype == WC_BF16) {
+    if (dtype != WC_FP32) {
       uint64_t b = L.off_raw + it.n + tid;
       if (b < L.off_exp) out[b] = 0;
     } else {
@@ -82,9 +84,11 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ EncParams 
 // ---------------------------------------------------------------------------
 constexpr int kHistThreads = 512;
 
-__device__ __forceinline__ void count_bf16_word(uint32_t *sh, int lane, uint32_t w) {
-  atomicAdd(&sh[(((w >> 7) & 0xFFu) << 5) | lane], 1u);
-  atomicAdd(&sh[(((w >> 23) & 0xFFu) << 5) | lane], 1u);
+// a word holds two 2-byte values (bf16 or fp16): count their coded bytes
+template <int DT>
+__device__ __forceinline__ void count_word16(uint32_t *sh, int lane, uint32_t w) {
+  atomicAdd(&sh[(code_byte<DT>(w & 0xFFFFu) << 5) | lane], 1u);
+  atomicAdd(&sh[(code_byte<DT>(w >> 16) << 5) | lane], 1u);
 }
 __device__ __forceinline__ void count_fp32_word(uint32_t *sh, int lane, uint32_t u) {
   atomicAdd(&sh[(((u >> 23) & 0xFFu) << 5) | lane], 1u);
@@ -163,12 +167,36 @@ __device__ void publish_table(const EncItem &it, uint64_t *red) {
   if (tid == 0) reinterpret_cast<uint32_t *>(it.scratch + kScrCtr)[2] = wide ? 1u : 0u;
 }
 
-// 16 values' worth of exponent counts (one group) from raw words.
-__device__ __forceinline__ void count_group_bf16(uint32_t *sh, int lane, uint4 a, uint4 b) {
-  count_bf16_word(sh, lane, a.x); count_bf16_word(sh, lane, a.y);
-  count_bf16_word(sh, lane, a.z); count_bf16_word(sh, lane, a.w);
-  count_bf16_word(sh, lane, b.x); count_bf16_word(sh, lane, b.y);
-  count_bf16_word(sh, lane, b.z); count_bf16_word(sh, lane, b.w);
+// 16 values' worth of coded-byte counts (one group) from raw words.
+template <int DT>
+__device__ __forceinline__ void count_group16(uint32_t *sh, int lane, uint4 a, uint4 b) {
+  count_word16<DT>(sh, lane, a.x); count_word16<DT>(sh, lane, a.y);
+  count_word16<DT>(sh, lane, a.z); count_word16<DT>(sh, lane, a.w);
+  count_word16<DT>(sh, lane, b.x); count_word16<DT>(sh, lane, b.y);
+  count_word16<DT>(sh, lane, b.z); count_word16<DT>(sh, lane, b.w);
+}
+
+// One thread's share of a tile of 2-byte values: groups tid, tid + 512, ...
+// with four groups of loads in flight.
+template <int DT>
+__device__ __forceinline__ void count_tile16(uint32_t *sh, int lane, int tid, const uint16_t *src,
+                                             uint32_t nfull, uint32_t count) {
+  uint32_t g = tid;
+  for (; g + 3 * kHistThreads < nfull; g += 4 * kHistThreads) {
+    uint4 a0 = ld_nc_v4(src + 16 * g), b0 = ld_nc_v4(src + 16 * g + 8);
+    uint4 a1 = ld_nc_v4(src + 16 * (g + kHistThreads)), b1 = ld_nc_v4(src + 16 * (g + kHistThreads) + 8);
+    uint4 a2 = ld_nc_v4(src + 16 * (g + 2 * kHistThreads)), b2 = ld_nc_v4(src + 16 * (g + 2 * kHistThreads) + 8);
+    uint4 a3 = ld_nc_v4(src + 16 * (g + 3 * kHistThreads)), b3 = ld_nc_v4(src + 16 * (g + 3 * kHistThreads) + 8);
+    count_group16<DT>(sh, lane, a0, b0);
+    count_group16<DT>(sh, lane, a1, b1);
+    count_group16<DT>(sh, lane, a2, b2);
+    count_group16<DT>(sh, lane, a3, b3);
+  }
+  for (; g < nfull; g += kHistThreads)
+    count_group16<DT>(sh, lane, ld_nc_v4(src + 16 * g), ld_nc_v4(src + 16 * g + 8));
+  if (g == nfull)  // the thread whose next group is the ragged tail
+    for (uint32_t v = 16 * nfull; v < count; v++)
+      atomicAdd(&sh[(code_byte<DT>(src[v]) << 5) | lane], 1u);
 }
 __device__ __forceinline__ void count_quad_fp32(uint32_t *sh, int lane, uint4 a) {
   count_fp32_word(sh, lane, a.x); count_fp32_word(sh, lane, a.y);
@@ -197,22 +225,9 @@ __global__ void __launch_bounds__(kHistThreads, 2) k_hist(const __grid_constant_
   __syncthreads();
 
   if (it.dtype == WC_BF16) {
-    const uint16_t *src = reinterpret_cast<const uint16_t *>(it.in) + v0;
-    uint32_t g = tid;
-    for (; g + 3 * kHistThreads < nfull; g += 4 * kHistThreads) {
-      uint4 a0 = ld_nc_v4(src + 16 * g), b0 = ld_nc_v4(src + 16 * g + 8);
-      uint4 a1 = ld_nc_v4(src + 16 * (g + kHistThreads)), b1 = ld_nc_v4(src + 16 * (g + kHistThreads) + 8);
-      uint4 a2 = ld_nc_v4(src + 16 * (g + 2 * kHistThreads)), b2 = ld_nc_v4(src + 16 * (g + 2 * kHistThreads) + 8);
-      uint4 a3 = ld_nc_v4(src + 16 * (g + 3 * kHistThreads)), b3 = ld_nc_v4(src + 16 * (g + 3 * kHistThreads) + 8);
-      count_group_bf16(sh, lane, a0, b0);
-      count_group_bf16(sh, lane, a1, b1);
-      count_group_bf16(sh, lane, a2, b2);
-      count_group_bf16(sh, lane, a3, b3);
-    }
-    for (; g < nfull; g += kHistThreads) count_group_bf16(sh, lane, ld_nc_v4(src + 16 * g), ld_nc_v4(src + 16 * g + 8));
-    if (g == nfull)  // the thread whose next group is the ragged tail
-      for (uint32_t v = 16 * nfull; v < count; v++)
-        atomicAdd(&sh[((uint32_t(src[v] >> 7) & 0xFFu) << 5) | lane], 1u);
+    count_tile16<WC_BF16>(sh, lane, tid, reinterpret_cast<const uint16_t *>(it.in) + v0, nfull, count);
+  } else if (it.dtype == WC_FP16) {
+    count_tile16<WC_FP16>(sh, lane, tid, reinterpret_cast<const uint16_t *>(it.in) + v0, nfull, count);
   } else {
     const uint32_t *src = reinterpret_cast<const uint32_t *>(it.in) + v0;
     uint32_t g = tid;

@@ -25,7 +25,9 @@ namespace {
 
 inline uint64_t r256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
 
-uint64_t elem_bytes(int32_t dt) { return dt == WC_BF16 ? 2 : 4; }
+uint64_t elem_bytes(int32_t dt) { return dt == WC_FP32 ? 4 : 2; }
+
+bool dtype_ok(int32_t dt) { return dt == WC_BF16 || dt == WC_FP32 || dt == WC_FP16; }
 
 constexpr uint64_t kWindowReserve = 256;  // per window: the rounding of its size array
 
@@ -58,7 +60,7 @@ uint64_t wc_host_encode_footprint(uint64_t n, int32_t dtype) {
 }
 
 uint64_t wc_host_decode_footprint(uint64_t cont_bytes, uint64_t n, int32_t dtype) {
-  if (dtype != WC_BF16 && dtype != WC_FP32) return 0;
+  if (!dtype_ok(dtype)) return 0;
   return r256(cont_bytes) + r256(n * elem_bytes(dtype));
 }
 
@@ -105,7 +107,7 @@ int32_t wc_encode_host(const wc_host_encode_item *items, uint32_t count, void *d
   std::vector<uint64_t> fp(count);
   for (uint32_t i = 0; i < count; i++) {
     const wc_host_encode_item &it = items[i];
-    if ((it.dtype != WC_BF16 && it.dtype != WC_FP32) || it.reserved != 0) return WC_ERR_INVALID_ARG;
+    if (!dtype_ok(it.dtype) || it.reserved != 0) return WC_ERR_INVALID_ARG;
     if ((it.n > 0 && it.h_in == nullptr) || it.h_out == nullptr || it.h_out_size == nullptr)
       return WC_ERR_INVALID_ARG;
     fp[i] = wc_host_encode_footprint(it.n, it.dtype);

@@ -1,0 +1,66 @@
+// wc_planes.cuh -- the two byte planes of a 2-byte value and back ("PTWM",
+// How it works 1-2: the reorder S E M -> E S M, then a 2-plane byte split
+// whose high byte, plane 1, is the coded one).
+//   bf16 [S:1 E:8 M:7]   coded byte E                       raw byte S<<7 | M
+//   fp16 [S:1 E:5 M:10]  coded byte E<<3 | S<<2 | M>>8      raw byte M & 0xFF
+// The scalar forms take one 16-bit value.  The x4 forms work on four values
+// at once, one per byte lane: w0 = [v1:v0] and w1 = [v3:v2] are the values as
+// two 32-bit words; c4 / r4 hold the four coded / raw bytes, value j in byte j.
+#pragma once
+
+#include <cstdint>
+
+#include "wc.h"
+
+namespace wc {
+
+template <int DT>
+__device__ __forceinline__ uint32_t code_byte(uint32_t v) {
+  if (DT == WC_BF16) return (v >> 7) & 0xFFu;
+  return ((v >> 7) & 0xF8u) | ((v >> 13) & 0x04u) | ((v >> 8) & 0x03u);
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t raw_byte(uint32_t v) {
+  if (DT == WC_BF16) return ((v >> 8) & 0x80u) | (v & 0x7Fu);
+  return v & 0xFFu;
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t merge16(uint32_t code, uint32_t raw) {
+  if (DT == WC_BF16) return ((raw & 0x80u) << 8) | (code << 7) | (raw & 0x7Fu);
+  const uint32_t hi = ((code >> 1) & 0x7Cu) | ((code << 5) & 0x80u) | (code & 0x03u);
+  return (hi << 8) | raw;
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t code4(uint32_t w0, uint32_t w1) {
+  if (DT == WC_BF16) return __byte_perm(w0 >> 7, w1 >> 7, 0x6420);
+  const uint32_t hb = __byte_perm(w0, w1, 0x7531);  // the four high bytes
+  return ((hb << 1) & 0xF8F8F8F8u) | ((hb >> 5) & 0x04040404u) | (hb & 0x03030303u);
+}
+
+template <int DT>
+__device__ __forceinline__ uint32_t raw4(uint32_t w0, uint32_t w1) {
+  const uint32_t lo = __byte_perm(w0, w1, 0x6420);  // the four low bytes
+  if (DT == WC_BF16) {
+    const uint32_t hi = __byte_perm(w0, w1, 0x7531);
+    return (lo & 0x7F7F7F7Fu) | (hi & 0x80808080u);
+  }
+  return lo;
+}
+
+template <int DT>
+__device__ __forceinline__ uint2 merge4(uint32_t c4, uint32_t r4) {
+  uint32_t lo, hi;  // the four values' low and high bytes
+  if (DT == WC_BF16) {
+    lo = (r4 & 0x7F7F7F7Fu) | ((c4 << 7) & 0x80808080u);
+    hi = ((c4 >> 1) & 0x7F7F7F7Fu) | (r4 & 0x80808080u);
+  } else {
+    lo = r4;
+    hi = ((c4 >> 1) & 0x7C7C7C7Cu) | ((c4 << 5) & 0x80808080u) | (c4 & 0x03030303u);
+  }
+  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
+
+}  // namespace wc

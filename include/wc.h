@@ -24,7 +24,8 @@
  * u64 off_raw, u64 off_exp, u64 exp_bytes, u64 total_bytes (64 bytes), then
  * u16 freq[256], u64 chunk_off[nc+1], u32 chunk_len[nc], the raw planes
  * (bf16: n sign+mantissa bytes; fp32: ceil(n/8) sign-bit bytes, 3n mantissa
- * bytes) and the exponent chunks.  A coded chunk is 32 final u32 states then
+ * bytes; fp16: n low bytes) and the exponent chunks (bf16 / fp32: the
+ * exponent byte; fp16: the reordered high byte).  A coded chunk is 32 final u32 states then
  * w u16 renormalisation words (128 + 2w bytes); a chunk whose coded form is
  * not smaller than its nsym exponent bytes is stored raw.  The format is
  * fully determined by the input bits: one input has exactly one container.
@@ -72,7 +73,11 @@ typedef enum {
     WC_ERR_UNSUPPORTED = 5
 } wc_status;
 
-typedef enum { WC_BF16 = 1, WC_FP32 = 2 } wc_dtype;
+/* WC_FP16: the same 2-plane byte split as bf16 after the reorder S E M ->
+ * E S M ("PTWM", How it works 1-2: float16 / bfloat16 are split into 2 byte
+ * planes, plane 1 coded); for fp16 the coded byte holds the 5 exponent bits,
+ * the sign and the top 2 mantissa bits, the raw byte the other 8. */
+typedef enum { WC_BF16 = 1, WC_FP32 = 2, WC_FP16 = 3 } wc_dtype;
 
 /* Worst-case container size in bytes for n values of dtype: every chunk
  * stored raw ("PTWM" Configuration table, compression_threshold: the coded
@@ -131,7 +136,7 @@ WC_API int32_t wc_read_header(const void *h_cont, uint64_t bytes, uint64_t *n,
 typedef struct {
     const void *in;       /* n values, 16-byte aligned                   */
     uint64_t n;
-    int32_t dtype;        /* WC_BF16 or WC_FP32                          */
+    int32_t dtype;        /* WC_BF16, WC_FP32 or WC_FP16                 */
     int32_t reserved;     /* must be 0                                   */
     void *out;            /* container, out_cap >= wc_encode_bound(n)    */
     uint64_t out_cap;
@@ -209,7 +214,7 @@ WC_API int32_t wc_encode_noalloc(const void *d_in, uint64_t n, int32_t dtype, vo
 typedef struct {
     const void *h_in;       /* n values (host)                              */
     uint64_t n;
-    int32_t dtype;          /* WC_BF16 or WC_FP32                           */
+    int32_t dtype;          /* WC_BF16, WC_FP32 or WC_FP16                  */
     int32_t reserved;       /* must be 0                                    */
     void *h_out;            /* container (host)                             */
     uint64_t h_out_cap;     /* must be >= wc_encode_bound(n, dtype)         */

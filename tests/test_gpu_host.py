@@ -22,18 +22,25 @@ def _cuda():
 
 def _bits(n, dt, seed):
     x = np.random.default_rng(seed).standard_normal(n).astype(np.float32) * np.float32(0.02)
+    if dt == "fp16":
+        return x.astype(np.float16)
     return workloads.rne_bf16(x) if dt == "bf16" else x.view(np.uint32).copy()
 
 
 def _host(bits, pin=True):
-    t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16) if bits.dtype == np.uint16 \
-        else torch.from_numpy(bits.view(np.int32)).view(torch.float32)
+    if bits.dtype == np.uint16:
+        t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+    elif bits.dtype == np.float16:
+        t = torch.from_numpy(bits.view(np.int16)).view(torch.float16)
+    else:
+        t = torch.from_numpy(bits.view(np.int32)).view(torch.float32)
     return t.pin_memory() if pin else t.clone()
 
 
 def _set():
     sizes = [0, 1, 100, C - 3, C, C + 5, 3 * C + 17, 5 * C, 17, 2 * C + 1]
-    return [_bits(n, "bf16" if i % 3 else "fp32", 500 + i) for i, n in enumerate(sizes)]
+    kinds = ["fp32", "bf16", "fp16"]
+    return [_bits(n, kinds[i % 3], 500 + i) for i, n in enumerate(sizes)]
 
 
 @pytest.mark.parametrize("window", [1, 1 << 20, 0])    # one item per window .. one slot per window
@@ -42,7 +49,8 @@ def test_host_round_trip_matches_oracle(orc, slots, window):
     from fp32_weight_compression_b200 import wc
     arrs = _set()
     ts = [_host(a) for a in arrs]
-    big = max(wc.host_encode_footprint(a.size, 1 if a.dtype == np.uint16 else 2) for a in arrs)
+    code = {np.dtype(np.uint16): 1, np.dtype(np.uint32): 2, np.dtype(np.float16): 3}
+    big = max(wc.host_encode_footprint(a.size, code[a.dtype]) for a in arrs)
     slot = (big + 256 + 255) // 256 * 256
     work = 256 * ((4 * len(arrs) + 255) // 256) + slots * slot   # status words + slots
     codec = wc.HostCodec(work, window_bytes=window)
@@ -51,7 +59,7 @@ def test_host_round_trip_matches_oracle(orc, slots, window):
         assert np.array_equal(c.numpy(), orc.encode(a))
     outs = codec.decode(conts)
     for a, o in zip(arrs, outs):
-        got = o.view(torch.int16 if a.dtype == np.uint16 else torch.int32).numpy()
+        got = o.view(torch.int32 if a.dtype == np.uint32 else torch.int16).numpy()
         assert np.array_equal(got.view(a.dtype), a)
 
 

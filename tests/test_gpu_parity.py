@@ -263,3 +263,54 @@ def test_table_format_boundary(orc, gu, dt, fmax):
                 rng.integers(0, 1 << 23, n, dtype=np.uint32)).astype(np.uint32)
     _check(orc, gu, bits)
     _check(orc, gu, bits[:3 * C + 333])
+
+
+# ---------------------------------------------------------------- fp16
+def _fp16(n, seed, scale=0.02):
+    return (np.random.default_rng(seed).standard_normal(n) * scale).astype(np.float16)
+
+
+def _check16(orc, gu, vals):
+    want = orc.encode(vals)
+    got, back = gu.gpu_roundtrip(vals)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert np.array_equal(back.view(np.uint16), vals.view(np.uint16))
+
+
+@pytest.mark.parametrize("n", [0, 1, 17, 33, 513, 65535, 65536, 65537, 3 * C + 17, 5 * C + 511])
+def test_fp16_edge_sizes(orc, gu, n):
+    _check16(orc, gu, _fp16(n, seed=n + 3))
+
+
+def test_fp16_all_patterns(orc, gu):
+    pats = np.arange(1 << 16, dtype=np.uint16).view(np.float16)
+    _check16(orc, gu, pats)                                          # raw path
+    base = _fp16(8 * C, seed=5)
+    pos = np.random.default_rng(6).choice(base.size, size=1 << 16, replace=False)
+    base[pos] = pats
+    _check16(orc, gu, base)                                          # coded path
+
+
+def test_fp16_single_symbol_and_random_access(orc, gu):
+    from fp32_weight_compression_b200 import wc
+    _check16(orc, gu, np.full(3 * C + 5, 1.0, np.float16))
+    vals = _fp16(4 * C + 999, seed=8)
+    cont = orc.encode(vals)
+    d = gu.cont_device(cont)
+    for k in range(5):
+        got = wc.decode_chunk(d, k).view(torch.int16).cpu().numpy().view(np.uint16)
+        assert np.array_equal(got, vals.view(np.uint16)[k * C:(k + 1) * C])
+
+
+def test_mixed_dtype_batch(orc, gu):
+    """bf16, fp16 and fp32 tensors in one batched launch."""
+    from fp32_weight_compression_b200 import wc
+    arrs = [_normal_bits(2 * C + 7, "bf16", seed=1), _fp16(3 * C + 1, seed=2),
+            _normal_bits(C + 5, "fp32", seed=3), _fp16(100, seed=4), _fp16(2 * C, seed=5)]
+    ts = [gu.to_device(a) for a in arrs]
+    conts = wc.encode_batch(ts)
+    for a, c in zip(arrs, conts):
+        assert np.array_equal(c.cpu().numpy(), orc.encode(a))
+    outs = wc.decode_batch(conts, [(a.size,) for a in arrs], [t.dtype for t in ts])
+    for a, o in zip(arrs, outs):
+        assert np.array_equal(gu.to_bits(o).view(a.dtype), a)

@@ -85,7 +85,7 @@ def test_bad_arguments_rejected_before_device(wcm, orc):
     assert L.wc_encode_host(it, 0, None, 0, 0, None, None, None) == wcm.OK
     assert L.wc_encode_host(None, 1, 256, 1 << 20, 0, None, None, None) == wcm.ERR_INVALID_ARG
     assert L.wc_encode_host(it, 1, 257, 1 << 20, 0, None, None, None) == wcm.ERR_INVALID_ARG
-    it[0].dtype = 3
+    it[0].dtype = 4
     assert L.wc_encode_host(it, 1, 256, 1 << 20, 0, None, None, None) == wcm.ERR_INVALID_ARG
     it[0].dtype, it[0].h_out_cap = 1, 10          # below wc_encode_bound
     assert L.wc_encode_host(it, 1, 256, 1 << 20, 0, None, None, None) == wcm.ERR_CAPACITY
