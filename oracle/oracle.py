@@ -22,7 +22,8 @@ SRC = os.path.join(HERE, "wc_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CORRUPT = 0, 1, 2, 4
-BF16, FP32, FP16 = 1, 2, 3
+BF16, FP32, FP16, FP8E4M3 = 1, 2, 3, 4
+_NP = {BF16: np.uint16, FP32: np.uint32, FP16: np.uint16, FP8E4M3: np.uint8}
 CHUNK = 65536
 
 
@@ -58,6 +59,7 @@ def lib():
         L.oracle_split_bf16.argtypes = [vp, ctypes.c_uint64, vp, vp]
         L.oracle_split_fp32.argtypes = [vp, ctypes.c_uint64, vp, vp, vp]
         L.oracle_split_fp16.argtypes = [vp, ctypes.c_uint64, vp, vp]
+        L.oracle_split_fp8e4m3.argtypes = [vp, ctypes.c_uint64, vp, vp]
         L.oracle_histogram.argtypes = [vp, ctypes.c_uint64, vp]
         L.oracle_normalize.argtypes = [vp, vp]
         L.oracle_rans_encode.argtypes = [vp, ctypes.c_uint32, vp, ctypes.c_uint32, vp, vp, u32p]
@@ -88,7 +90,10 @@ def dtype_code(arr: np.ndarray) -> int:
         return FP32
     if arr.dtype == np.float16:
         return FP16
-    raise TypeError("oracle takes bf16 bits as uint16, fp32 bits as uint32, fp16 as float16")
+    if arr.dtype == np.uint8:
+        return FP8E4M3
+    raise TypeError("oracle takes bf16 bits as uint16, fp32 bits as uint32, fp16 as float16, "
+                    "fp8 e4m3 bits as uint8")
 
 
 class OracleError(RuntimeError):
@@ -117,6 +122,15 @@ def split_fp16(bits: np.ndarray):
     lo = np.zeros(bits.size, np.uint8)
     lib().oracle_split_fp16(_ptr(bits), bits.size, _ptr(hi), _ptr(lo))
     return hi, lo
+
+
+def split_fp8e4m3(bits: np.ndarray):
+    """(exponent-nibble plane, packed low-nibble plane) of fp8 e4m3 bits (uint8)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint8).reshape(-1)
+    e = np.zeros(bits.size, np.uint8)
+    nib = np.zeros((bits.size + 1) // 2, np.uint8)
+    lib().oracle_split_fp8e4m3(_ptr(bits), bits.size, _ptr(e), _ptr(nib) if nib.size else None)
+    return e, nib
 
 
 def split_fp32(bits: np.ndarray):
@@ -217,7 +231,7 @@ def decode_status(cont: np.ndarray, n_hint: int | None = None, dtype_hint: int |
                                   ctypes.byref(nc))
     if st:
         return st, None
-    npdt = np.uint32 if dt.value == FP32 else np.uint16
+    npdt = _NP[dt.value]
     out = np.zeros(max(n.value, 1), npdt)
     st = lib().oracle_decode(_ptr(cont), cont.size, _ptr(out), out.nbytes)
     return st, out[: n.value]
@@ -233,7 +247,7 @@ def decode(cont: np.ndarray) -> np.ndarray:
 def decode_chunk(cont: np.ndarray, k: int) -> np.ndarray:
     cont = np.ascontiguousarray(cont, dtype=np.uint8)
     n, dt, nc = read_header(cont)
-    npdt = np.uint32 if dt == FP32 else np.uint16
+    npdt = _NP[dt]
     nsym = min(CHUNK, n - k * CHUNK) if k < nc else 0
     out = np.zeros(max(nsym, 1), npdt)
     st = lib().oracle_decode_chunk(_ptr(cont), cont.size, k, _ptr(out), out.nbytes)

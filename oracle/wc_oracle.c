@@ -22,6 +22,11 @@
  *    high byte of 5 exponent bits, the sign and the top 2 mantissa bits, and
  *    a raw low byte of the other 8 mantissa bits ("PTWM", "How it works" 2:
  *    float16 / bfloat16 are split into 2 byte planes, plane 1 = exponent).
+ *    For fp8 e4m3 the reorder S E M -> E S M puts the 4 exponent bits in the
+ *    high nibble and a nibble split separates them ("PTWM", "How it works"
+ *    1-2: float8 formats are split into 2 nibble planes, plane 0 = exponent
+ *    nibbles): the coded symbol is the exponent nibble, and the low nibbles
+ *    (sign above 3 mantissa bits) are stored raw, two per byte.
  *    For fp32 the container keeps three streams: sign bits, the 8-bit
  *    exponent, and the 23-bit mantissa stored as 3 little-endian bytes.
  *
@@ -47,13 +52,15 @@
  *
  * Container layout (all fields little-endian, sections 16-byte aligned,
  * padding bytes zero):
- *   0  "WCZ1"            4  u16 version = 1    6  u8 dtype (1 bf16, 2 fp32, 3 fp16)
+ *   0  "WCZ1"            4  u16 version = 1    6  u8 dtype (1 bf16, 2 fp32, 3 fp16,
+ *                                              4 fp8 e4m3)
  *   7  u8 lanes = 32     8  u64 n              16 u32 chunk symbols = 65536
  *   20 u32 nc            24 u16 prob bits = 12 26 u16 0      28 u32 0
  *   32 u64 off_raw       40 u64 off_exp        48 u64 exp_bytes
  *   56 u64 total_bytes   64 u16 freq[256]      576 u64 chunk_off[nc + 1]
  *   then u32 chunk_len[nc]; pad; raw section; pad; exponent section.
- *   bf16 raw section: n sign+mantissa bytes; fp16: n low bytes.
+ *   bf16 raw section: n sign+mantissa bytes; fp16: n low bytes; fp8 e4m3:
+ *   ceil(n/2) bytes of low nibbles (value 2j in the low half of byte j).
  *   fp32 raw section: ceil(n/8) sign bytes (value 8j+b is bit b of byte j),
  *   pad, then 3n mantissa bytes.
  *   Exponent section: chunk k at off_exp + chunk_off[k], chunk_len[k] bytes,
@@ -124,6 +131,10 @@ static void or_make_layout(uint64_t n, int dtype, or_layout *lay) {
         lay->off_sign = 0;
         lay->off_mant = 0;
         lay->off_exp = round_up16(lay->off_raw + n);
+    } else if (dtype == OR_FP8E4M3) {
+        lay->off_sign = 0;
+        lay->off_mant = 0;
+        lay->off_exp = round_up16(lay->off_raw + (n + 1) / 2);
     } else {
         lay->off_sign = lay->off_raw;
         lay->off_mant = round_up16(lay->off_raw + (n + 7) / 8);
@@ -138,11 +149,13 @@ static uint32_t or_chunk_nsym(uint64_t n, uint64_t k) {
 }
 
 static int or_dtype_ok(int dtype) {
-    return dtype == OR_BF16 || dtype == OR_FP32 || dtype == OR_FP16;
+    return dtype == OR_BF16 || dtype == OR_FP32 || dtype == OR_FP16 || dtype == OR_FP8E4M3;
 }
 
 /* Bytes per value of a dtype. */
-static uint64_t or_elem(int dtype) { return dtype == OR_FP32 ? 4 : 2; }
+static uint64_t or_elem(int dtype) {
+    return dtype == OR_FP32 ? 4 : (dtype == OR_FP8E4M3 ? 1 : 2);
+}
 
 uint64_t oracle_encode_bound(uint64_t n, int dtype) {
     or_layout lay;
@@ -203,6 +216,24 @@ void oracle_split_fp16(const uint16_t *in, uint64_t n, uint8_t *hi_plane,
         uint16_t r = (uint16_t)((expo << 11) | (sign << 10) | mant);
         hi_plane[i] = (uint8_t)(r >> 8);
         lo_plane[i] = (uint8_t)(r & 0xFFu);
+    }
+}
+
+/* fp8 e4m3 bits b = [S:1][E:4][M:3].  The reorder gives E<<4 | S<<3 | M; the
+ * nibble split gives the exponent nibble E (coded) and the low nibble
+ * S<<3 | M (raw), packed two per byte: value i goes to byte i/2, in the low
+ * nibble when i is even.  nibble_plane must be zeroed by the caller. */
+void oracle_split_fp8e4m3(const uint8_t *in, uint64_t n, uint8_t *exp_plane,
+                          uint8_t *nibble_plane) {
+    for (uint64_t i = 0; i < n; i++) {
+        uint8_t b = in[i];
+        uint8_t sign = (uint8_t)((b >> 7) & 1u);
+        uint8_t expo = (uint8_t)((b >> 3) & 0xFu);
+        uint8_t mant = (uint8_t)(b & 7u);
+        uint8_t r = (uint8_t)((expo << 4) | (sign << 3) | mant);
+        exp_plane[i] = (uint8_t)(r >> 4);
+        uint8_t lo = (uint8_t)(r & 0xFu);
+        nibble_plane[i / 2] = (uint8_t)(nibble_plane[i / 2] | (i % 2 ? lo << 4 : lo));
     }
 }
 
@@ -457,6 +488,8 @@ int oracle_encode(const void *in, uint64_t n, int dtype, uint8_t *out,
         oracle_split_bf16((const uint16_t *)in, n, expo, out + lay.off_raw);
     else if (dtype == OR_FP16)
         oracle_split_fp16((const uint16_t *)in, n, expo, out + lay.off_raw);
+    else if (dtype == OR_FP8E4M3)  /* the raw nibbles land in the zeroed section */
+        oracle_split_fp8e4m3((const uint8_t *)in, n, expo, out + lay.off_raw);
     else
         oracle_split_fp32((const uint32_t *)in, n, expo, out + lay.off_sign,
                           out + lay.off_mant);
@@ -620,6 +653,14 @@ static int or_decode_one_chunk(const uint8_t *c, const or_header *h, uint64_t k,
             uint16_t sign = (uint16_t)((r >> 10) & 1u);
             uint16_t mant = (uint16_t)(r & 0x3FFu);
             ((uint16_t *)out_vals)[j] = (uint16_t)((sign << 15) | (e5 << 10) | mant);
+        } else if (h->dtype == OR_FP8E4M3) {
+            /* undo the nibble split, then the reorder E S M -> S E M */
+            uint8_t lo = (uint8_t)((c[h->lay.off_raw + i / 2] >> (i % 2 ? 4 : 0)) & 0xFu);
+            uint8_t r = (uint8_t)((expo[j] << 4) | lo);
+            uint8_t e4 = (uint8_t)(r >> 4);
+            uint8_t sign = (uint8_t)((r >> 3) & 1u);
+            uint8_t mant = (uint8_t)(r & 7u);
+            ((uint8_t *)out_vals)[j] = (uint8_t)((sign << 7) | (e4 << 3) | mant);
         } else {
             uint32_t sign = (c[h->lay.off_sign + i / 8] >> (i % 8)) & 1u;
             const uint8_t *m = c + h->lay.off_mant + 3 * i;

@@ -26,7 +26,7 @@ enum {
     OR_ERR_CORRUPT = 4
 };
 
-enum { OR_BF16 = 1, OR_FP32 = 2, OR_FP16 = 3 };
+enum { OR_BF16 = 1, OR_FP32 = 2, OR_FP16 = 3, OR_FP8E4M3 = 4 };
 
 /* Worst-case container size (every chunk stored raw). */
 uint64_t oracle_encode_bound(uint64_t n, int dtype);
@@ -38,6 +38,8 @@ void oracle_split_fp32(const uint32_t *in, uint64_t n, uint8_t *exp_plane,
                        uint8_t *sign_bits, uint8_t *mant3);
 void oracle_split_fp16(const uint16_t *in, uint64_t n, uint8_t *hi_plane,
                        uint8_t *lo_plane);
+void oracle_split_fp8e4m3(const uint8_t *in, uint64_t n, uint8_t *exp_plane,
+                          uint8_t *nibble_plane);
 
 /* 256-bin count of an exponent plane. */
 void oracle_histogram(const uint8_t *exp_plane, uint64_t n, uint64_t counts[256]);

@@ -215,7 +215,56 @@ def test_fp16_all_patterns_round_trip(orc):
     assert cont.size < vals.nbytes          # the coded plane shrinks
 
 
+def test_split_fp8e4m3_worked(orc):
+    # fp8 e4m3 S E4 M3; reordered E4 | S M3; exponent nibble coded, low nibbles
+    # raw, two per byte (even value in the low half)
+    bits = np.array([0x38, 0xB8, 0x7E, 0x01, 0x80], np.uint8)
+    e, nib = orc.split_fp8e4m3(bits)
+    assert e.tolist() == [7, 7, 15, 0, 0]
+    assert nib.tolist() == [0x80, 0x16, 0x08]
+
+
+def test_split_fp8e4m3_plane_structure(orc):
+    rng = np.random.default_rng(7)
+    for n in (4096, 4097):
+        bits = rng.integers(0, 256, n, dtype=np.uint8)
+        e, nib = orc.split_fp8e4m3(bits)
+        assert np.array_equal(e, (bits >> 3) & 0xF)
+        lo = np.zeros(2 * nib.size, np.uint8)
+        lo[0::2], lo[1::2] = nib & 0xF, nib >> 4
+        assert np.array_equal(lo[:n], ((bits >> 4) & 8) | (bits & 7))
+        assert n % 2 == 0 or lo[n] == 0          # the pad nibble is zero
+
+
+def test_fp8e4m3_round_trips(orc):
+    pats = np.arange(256, dtype=np.uint8)
+    cont = orc.encode(pats)
+    assert orc.read_header(cont) == (256, orc.FP8E4M3, 1)
+    assert np.array_equal(orc.decode(cont), pats)
+    rng = np.random.default_rng(8)
+    # skewed: exponents around 7, with every pattern present
+    vals = ((rng.integers(0, 2, 3 * 65536 + 7) << 7) | (np.clip(rng.normal(6, 1.2, 3 * 65536 + 7), 0, 15).astype(np.int64) << 3)
+            | rng.integers(0, 8, 3 * 65536 + 7)).astype(np.uint8)
+    vals[rng.choice(vals.size, 256, replace=False)] = pats
+    cont = orc.encode(vals)
+    assert np.array_equal(orc.decode(cont), vals)
+    assert cont.size < vals.nbytes
+    for n in (0, 1, 2, 3, 31, 33, 65535, 65537):
+        v = vals[:n]
+        c = orc.encode(v)
+        assert np.array_equal(orc.decode(c), v)
+        for k in range((n + 65535) // 65536):
+            assert np.array_equal(orc.decode_chunk(c, k), v[k * 65536:(k + 1) * 65536])
+
+
 # ---------------------------------------------------------------- containers
+def test_golden_container_fp8e4m3_raw_chunk(orc):
+    bits = np.array([0x38, 0x38, 0x38, 0x30], np.uint8)
+    want = load_container("container_fp8e4m3_n4_raw.txt")
+    got = orc.encode(bits)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert orc.decode(got).tolist() == bits.tolist()
+
 def test_golden_container_fp16_raw_chunk(orc):
     bits = np.array([0x3C00, 0x3C00, 0x3C00, 0x3800], np.uint16)
     want = load_container("container_fp16_n4_raw.txt")
