@@ -4,7 +4,8 @@
 //   coded chunk: the 32 final states (front of the chunk's scratch window) and
 //                the w words (back of the window, at a 2-byte aligned start;
 //                realigned here with funnel shifts into 16-byte stores);
-//   raw chunk:   the chunk's exponent bytes, re-extracted from the input
+//   raw chunk:   the chunk's coded bytes (exponents; fp16 high bytes; fp8
+//                exponent nibbles), re-extracted from the input
 //                ("PTWM" Configuration table, compression_threshold: data that
 //                does not compress is stored as it is).
 #include "wc_block.cuh"
@@ -49,7 +50,24 @@ __global__ void __launch_bounds__(kCompactThreads) k_compact(const __grid_consta
 
   if (len == nsym) {
     const uint32_t ngran = uint32_t(round16(nsym) / 16);
-    if (dtype != WC_FP32) {
+    if (dtype == WC_FP8E4M3) {
+      const uint8_t *src = it.in + k * kChunk;
+      for (uint32_t gi = tid; gi < ngran; gi += kCompactThreads) {
+        const uint32_t v0 = gi * 16;
+        uint4 e;
+        if (v0 + 16 <= nsym) {
+          const uint4 a = ld_nc_v4(src + v0);
+          e = make_uint4(fp8_code4(a.x), fp8_code4(a.y), fp8_code4(a.z), fp8_code4(a.w));
+        } else {  // ragged: exponent nibbles, zero padding bytes
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+          for (uint32_t q = 0; q < 16; q++)
+            if (v0 + q < nsym) w[q / 4] |= fp8_code(src[v0 + q]) << (8 * (q % 4));
+          e = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *reinterpret_cast<uint4 *>(dst + v0) = e;
+      }
+    } else if (dtype != WC_FP32) {
       const uint16_t *src = reinterpret_cast<const uint16_t *>(it.in) + k * kChunk;
       const bool bf = dtype == WC_BF16;
       for (uint32_t gi = tid; gi < ngran; gi += kCompactThreads) {

@@ -91,7 +91,7 @@ __device__ __noinline__ ItemView view_item(const DecItem &it) {
   const uint32_t w1 = h32[1];
   const int dtype = int((w1 >> 16) & 0xFF);
   if (h32[0] != 0x315A4357u || (w1 & 0xFFFF) != kVersion || (w1 >> 24) != kLanes) return v;
-  if (dtype != WC_BF16 && dtype != WC_FP32 && dtype != WC_FP16) return v;
+  if (dtype != WC_BF16 && dtype != WC_FP32 && dtype != WC_FP16 && dtype != WC_FP8E4M3) return v;
   const uint64_t n = h64[1];
   if (n > (uint64_t(1) << 44)) return v;
   if (h32[4] != kChunk || h32[6] != kProbBits || h32[7] != 0) return v;
@@ -110,7 +110,7 @@ __device__ __noinline__ ItemView view_item(const DecItem &it) {
     v.first = it.chunk_first;
     v.cnt = min(it.chunk_count, L.nc - it.chunk_first);
   }
-  const uint64_t elem = dtype == WC_FP32 ? 4 : 2;
+  const uint64_t elem = dtype_bytes(dtype);
   const uint64_t vals = v.cnt == 0 ? 0
                         : (v.first + v.cnt == L.nc ? n - v.first * kChunk : v.cnt * kChunk);
   if (vals * elem > it.out_cap || (vals > 0 && it.out == nullptr)) { v.err = WC_ERR_CAPACITY; return v; }
@@ -143,7 +143,7 @@ __device__ __forceinline__ ChunkView view_chunk(const DecItem &it, const ItemVie
   c.ok = (c.raw || coded) && o0 <= o1 && o1 - o0 == round16(c.len) && o1 <= exp_bytes &&
          (k != 0 || o0 == 0) && (k + 1 != L.nc || o1 == exp_bytes);
   c.pay = cont + L.off_exp + o0;
-  constexpr uint32_t elem = DT == WC_FP32 ? 4 : 2;
+  constexpr uint32_t elem = dtype_bytes(DT);
   c.out = it.out + (k - v.first) * kChunk * elem;
   return c;
 }
@@ -152,14 +152,17 @@ __device__ __forceinline__ ChunkView view_chunk(const DecItem &it, const ItemVie
 // Raw-plane bytes of 8 consecutive values and the merge.
 template <int DT>
 struct Raw8 {
-  uint2 a;        // bf16 / fp16: the 8 raw bytes; fp32: mantissa bytes 0..7
+  uint2 a;        // bf16 / fp16: the 8 raw bytes; fp8: a.x = 8 packed nibbles;
+                  // fp32: mantissa bytes 0..7
   uint2 b, c;     // fp32: mantissa bytes 8..23
   uint32_t s;     // fp32: 8 sign bits
 };
 
 template <int DT>
 __device__ __forceinline__ void load_raw8(const uint8_t *cont, const Layout &L, uint64_t vg, Raw8<DT> &r) {
-  if (DT != WC_FP32) {
+  if (DT == WC_FP8E4M3) {
+    r.a.x = __ldg(reinterpret_cast<const uint32_t *>(cont + L.off_raw + vg / 2));
+  } else if (DT != WC_FP32) {
     r.a = __ldg(reinterpret_cast<const uint2 *>(cont + L.off_raw + vg));
   } else {
     r.s = __ldg(cont + L.off_raw + vg / 8);
@@ -189,7 +192,9 @@ __device__ __forceinline__ uint4 merge4_fp32(uint32_t e4, uint32_t w0, uint32_t 
 // 2-byte values merge byte-parallel (merge4, wc_planes.cuh).
 template <int DT>
 __device__ __forceinline__ void merge_store8(uint2 e8, const Raw8<DT> &r, uint8_t *dst) {
-  if (DT != WC_FP32) {
+  if (DT == WC_FP8E4M3) {
+    st_cs_v2(dst, fp8_merge8(e8, r.a.x));  // 8 one-byte values
+  } else if (DT != WC_FP32) {
     const uint2 p = merge4<DT>(e8.x, r.a.x);
     const uint2 q = merge4<DT>(e8.y, r.a.y);
     st_cs_v4(dst, make_uint4(p.x, p.y, q.x, q.y));
@@ -204,7 +209,9 @@ __device__ __forceinline__ void merge_store8(uint2 e8, const Raw8<DT> &r, uint8_
 template <int DT>
 __device__ __forceinline__ void merge_store1(uint32_t e, const uint8_t *cont, const Layout &L, uint64_t vg,
                                              uint8_t *dst) {
-  if (DT != WC_FP32) {
+  if (DT == WC_FP8E4M3) {
+    dst[0] = uint8_t(fp8_merge(e, (cont[L.off_raw + vg / 2] >> (4 * (vg & 1))) & 0xFu));
+  } else if (DT != WC_FP32) {
     reinterpret_cast<uint16_t *>(dst)[0] = uint16_t(merge16<DT>(e, cont[L.off_raw + vg]));
   } else {
     const uint32_t s = (cont[L.off_raw + vg / 8] >> (vg & 7)) & 1u;
@@ -293,7 +300,9 @@ struct RawPtrs {
 
 template <int DT>
 __device__ __forceinline__ void load_raw8p(const RawPtrs &p, uint32_t vl, Raw8<DT> &r) {
-  if (DT != WC_FP32) {
+  if (DT == WC_FP8E4M3) {
+    r.a.x = __ldg(reinterpret_cast<const uint32_t *>(p.a + vl / 2));
+  } else if (DT != WC_FP32) {
     r.a = __ldg(reinterpret_cast<const uint2 *>(p.a + vl));
   } else {
     r.s = __ldg(p.s + vl / 8);
@@ -359,11 +368,11 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   const uint32_t rsB = uint32_t(__cvta_generic_to_shared(ring_ptr(warp, 1)));
   uint8_t *tbA = s.tbuf[warp][0], *tbB = s.tbuf[warp][1];
   const uint32_t lt = lanemask_lt();
-  constexpr uint32_t elem = DT == WC_FP32 ? 4 : 2;
+  constexpr uint32_t elem = dtype_bytes(DT);
   Ring ra{rsA, payA + kStateBytes, uint32_t(round16(lenA) - kStateBytes) >> 1, 0, 0, 0, 0};
   Ring rb{rsB, payB + kStateBytes, uint32_t(round16(lenB) - kStateBytes) >> 1, 0, 0, 0, 0};
   RawPtrs rpB;
-  rpB.a = rpA.a + (DT == WC_FP32 ? 3 * kChunk : kChunk);
+  rpB.a = rpA.a + (DT == WC_FP32 ? 3 * kChunk : (DT == WC_FP8E4M3 ? kChunk / 2 : kChunk));
   rpB.s = DT == WC_FP32 ? rpA.s + kChunk / 8 : nullptr;
   uint8_t *outB = outA + kChunk * elem;
   uint32_t xA = reinterpret_cast<const uint32_t *>(payA)[lane];
@@ -452,7 +461,7 @@ __device__ __noinline__ void decode_one(const ItemView &v, const DecItem &it, co
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint32_t lt = lanemask_lt();
   const Layout &L = v.L;
-  constexpr uint32_t elem = DT == WC_FP32 ? 4 : 2;
+  constexpr uint32_t elem = dtype_bytes(DT);
   const uint64_t vg0 = k * kChunk;
   const uint32_t nsym = c.nsym;
   const uint32_t nhalf = (nsym + kHalf - 1) / kHalf;
@@ -594,7 +603,10 @@ __device__ __forceinline__ void decode_warp_chunks(const ItemView &v, const DecI
     const Layout &L = v.L;
     const uint64_t vgA = kA * kChunk;
     RawPtrs rpA;
-    if (DT != WC_FP32) {
+    if (DT == WC_FP8E4M3) {
+      rpA.a = it.cont + L.off_raw + vgA / 2;
+      rpA.s = nullptr;
+    } else if (DT != WC_FP32) {
       rpA.a = it.cont + L.off_raw + vgA;
       rpA.s = nullptr;
     } else {
@@ -642,6 +654,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
     const uint64_t kend = v.first + v.cnt;
     if (v.dtype == WC_BF16) decode_warp_chunks<WC_BF16>(v, it, kA, kend, status);
     else if (v.dtype == WC_FP16) decode_warp_chunks<WC_FP16>(v, it, kA, kend, status);
+    else if (v.dtype == WC_FP8E4M3) decode_warp_chunks<WC_FP8E4M3>(v, it, kA, kend, status);
     else decode_warp_chunks<WC_FP32>(v, it, kA, kend, status);
   }
 }

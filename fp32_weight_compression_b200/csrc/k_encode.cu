@@ -76,6 +76,7 @@ __device__ __forceinline__ uint32_t sign4_fp32(uint4 u) {
 // Raw planes and exponents of one value (ragged tails only).
 template <int DT>
 __device__ __forceinline__ uint32_t one_value(const uint8_t *in, uint64_t vg, uint8_t *out, const Layout &L) {
+  static_assert(DT != WC_FP8E4M3, "fp8 raw nibbles are written a byte (two values) at a time");
   if (DT != WC_FP32) {
     const uint32_t b = reinterpret_cast<const uint16_t *>(in)[vg];
     out[L.off_raw + vg] = uint8_t(raw_byte<DT>(b));
@@ -306,6 +307,62 @@ __device__ void code_pair_fp32(const EncItem &it, const Layout &L, uint64_t kA, 
   finish_chunk(co, kA + 1, kChunk, xB, tB, bailB, lane);
 }
 
+// Two full fp8 e4m3 chunks kA, kA + 1 in lock-step (as code_pair16: 16
+// values are one 16-byte load; their low nibbles are 8 bytes of the plane).
+template <bool W>
+__device__ void code_pair8(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
+                           const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t lt = lanemask_lt();
+  const uint64_t vgA = kA * kChunk, vgB = vgA + kChunk;
+  uint16_t *wA = reinterpret_cast<uint16_t *>(co.win0 + kA * kWin);
+  uint16_t *wB = reinterpret_cast<uint16_t *>(co.win0 + (kA + 1) * kWin);
+  uint32_t xA = kStateLow, xB = kStateLow, tA = kWinWords, tB = kWinWords;
+  bool bailA = false, bailB = false;
+  constexpr int NG = int(kChunk / kGroupValues);
+
+  uint4 cA, cB, nA, nB;
+  {
+    const uint64_t o = uint64_t(NG - 1) * kGroupValues + 16 * lane;
+    cA = ld_nc_v4(it.in + vgA + o);
+    cB = ld_nc_v4(it.in + vgB + o);
+  }
+  for (int G = NG - 1; G >= 0; --G) {
+    const uint64_t o = uint64_t(G) * kGroupValues + 16 * lane;
+    st_cs_v2(it.out + L.off_raw + (vgA + o) / 2, make_uint2(fp8_pack8(cA.x, cA.y), fp8_pack8(cA.z, cA.w)));
+    st_cs_v2(it.out + L.off_raw + (vgB + o) / 2, make_uint2(fp8_pack8(cB.x, cB.y), fp8_pack8(cB.z, cB.w)));
+    *reinterpret_cast<uint4 *>(ebA + 16 * lane) =
+        make_uint4(fp8_code4(cA.x), fp8_code4(cA.y), fp8_code4(cA.z), fp8_code4(cA.w));
+    *reinterpret_cast<uint4 *>(ebB + 16 * lane) =
+        make_uint4(fp8_code4(cB.x), fp8_code4(cB.y), fp8_code4(cB.z), fp8_code4(cB.w));
+    if (G > 0) {
+      nA = ld_nc_v4(it.in + vgA + o - kGroupValues);
+      nB = ld_nc_v4(it.in + vgB + o - kGroupValues);
+    }
+    __syncwarp();
+    if (!bailA && !bailB) {
+#pragma unroll
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep2<W>(xA, tA, wA, ebA[32 * t + lane], xB, tB, wB, ebB[32 * t + lane], tab, bias, lt);
+    } else if (!bailA) {
+#pragma unroll 4
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep<W>(xA, tA, wA, tab, bias, ebA[32 * t + lane], lt);
+    } else if (!bailB) {
+#pragma unroll 4
+      for (int t = int(kStepsPerGroup) - 1; t >= 0; --t)
+        cstep<W>(xB, tB, wB, tab, bias, ebB[32 * t + lane], lt);
+    }
+    if (kStateBytes + 2 * (kWinWords - tA) >= kChunk) bailA = true;
+    if (kStateBytes + 2 * (kWinWords - tB) >= kChunk) bailB = true;
+    __syncwarp();
+    cA = nA;
+    cB = nB;
+  }
+  finish_chunk(co, kA, kChunk, xA, tA, bailA, lane);
+  finish_chunk(co, kA + 1, kChunk, xB, tB, bailB, lane);
+}
+
 // Any single chunk (either dtype, possibly ragged).
 template <int DT, bool W>
 __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64_t k, int slot,
@@ -328,7 +385,11 @@ __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64
     const uint64_t vg = vg0 + vl;
     if (vl + 16 <= nsym) {
       uint4 e;
-      if (DT != WC_FP32) {
+      if constexpr (DT == WC_FP8E4M3) {
+        const uint4 v = ld_nc_v4(it.in + vg);
+        st_cs_v2(it.out + L.off_raw + vg / 2, make_uint2(fp8_pack8(v.x, v.y), fp8_pack8(v.z, v.w)));
+        e = make_uint4(fp8_code4(v.x), fp8_code4(v.y), fp8_code4(v.z), fp8_code4(v.w));
+      } else if constexpr (DT != WC_FP32) {
         const uint16_t *p = reinterpret_cast<const uint16_t *>(it.in) + vg;
         V16x16 v;
         v.a = ld_nc_v4(p);
@@ -349,6 +410,16 @@ __device__ __noinline__ void code_one(const EncItem &it, const Layout &L, uint64
         st_cs_v4(md + 32, make_uint4(m2.z, m3.x, m3.y, m3.z));
       }
       *reinterpret_cast<uint4 *>(eb + 16 * lane) = e;
+    } else if constexpr (DT == WC_FP8E4M3) {
+      // ragged tail: a byte of the nibble plane holds two values (the second
+      // nibble is zero past nsym); coded bytes past nsym are zero
+      for (uint32_t q = 0; q < 8; q++) {
+        const bool v0 = vl + 2 * q < nsym, v1 = vl + 2 * q + 1 < nsym;
+        const uint32_t b0 = v0 ? it.in[vg + 2 * q] : 0u, b1 = v1 ? it.in[vg + 2 * q + 1] : 0u;
+        eb[16 * lane + 2 * q] = uint8_t(v0 ? fp8_code(b0) : 0u);
+        eb[16 * lane + 2 * q + 1] = uint8_t(v1 ? fp8_code(b1) : 0u);
+        if (v0) it.out[L.off_raw + (vg + 2 * q) / 2] = uint8_t(fp8_nibble(b0) | (v1 ? fp8_nibble(b1) << 4 : 0u));
+      }
     } else {
       // ragged tail: value by value; exponent bytes past nsym are zero
       for (uint32_t j = 0; j < 16; j++) {
@@ -390,6 +461,7 @@ __device__ __forceinline__ void code_warp(const EncItem &it, const Layout &L, ui
                                           int warp, const CoderOut &co) {
   if (hasB && chunk_nsym(it.n, kA + 1) == kChunk) {
     if (DT == WC_FP32) code_pair_fp32<W>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
+    else if (DT == WC_FP8E4M3) code_pair8<W>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
     else code_pair16<DT, W>(it, L, kA, s_tab, s_bias, s_ebuf[warp][0], s_ebuf[warp][1], co);
   } else {
     code_one<DT, W>(it, L, kA, 0, co);
@@ -419,6 +491,9 @@ __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constan
   } else if (dtype == WC_FP16) {
     if (wide) code_warp<WC_FP16, true>(it, L, kA, hasB, warp, co);
     else code_warp<WC_FP16, false>(it, L, kA, hasB, warp, co);
+  } else if (dtype == WC_FP8E4M3) {
+    if (wide) code_warp<WC_FP8E4M3, true>(it, L, kA, hasB, warp, co);
+    else code_warp<WC_FP8E4M3, false>(it, L, kA, hasB, warp, co);
   } else if (wide) {
     code_warp<WC_FP32, true>(it, L, kA, hasB, warp, co);
   } else {

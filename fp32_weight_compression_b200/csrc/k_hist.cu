@@ -7,7 +7,8 @@
 //  k_hist   one block per tile of up to 4 chunks: reads the values as
 //           integers (a NaN payload is never touched as a float), counts the
 //           coded bytes -- the 8-bit exponent of bf16 / fp32, the reordered
-//           high byte of fp16 ("PTWM" How it works 1-2: after the bit reorder
+//           high byte of fp16, the exponent nibble of fp8 e4m3 ("PTWM" How it
+//           works 1-2: after the bit reorder
 //           the exponent leads a whole byte; "SMEF" pass3_streams.py) -- into a
 //           shared-memory histogram with one column per lane (so the 32 lanes
 //           of a warp never collide on an address), folds it into the tensor's
@@ -70,7 +71,8 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ EncParams 
     uint64_t a = L.off_chunk_len + 4 * L.nc + tid;
     if (a < L.off_raw) out[a] = 0;
     if (dtype != WC_FP32) {
-      uint64_t b = L.off_raw + it.n + tid;
+      const uint64_t raw_bytes = dtype == WC_FP8E4M3 ? (it.n + 1) / 2 : it.n;
+      uint64_t b = L.off_raw + raw_bytes + tid;
       if (b < L.off_exp) out[b] = 0;
     } else {
       uint64_t b = L.off_raw + (it.n + 7) / 8 + tid;
@@ -176,6 +178,36 @@ __device__ __forceinline__ void count_group16(uint32_t *sh, int lane, uint4 a, u
   count_word16<DT>(sh, lane, b.z); count_word16<DT>(sh, lane, b.w);
 }
 
+// fp8 e4m3: a word holds four values; count their exponent nibbles.
+__device__ __forceinline__ void count_word8(uint32_t *sh, int lane, uint32_t w) {
+  atomicAdd(&sh[(fp8_code(w) << 5) | lane], 1u);
+  atomicAdd(&sh[(fp8_code(w >> 8) << 5) | lane], 1u);
+  atomicAdd(&sh[(fp8_code(w >> 16) << 5) | lane], 1u);
+  atomicAdd(&sh[(fp8_code(w >> 24) << 5) | lane], 1u);
+}
+__device__ __forceinline__ void count_quad8(uint32_t *sh, int lane, uint4 a) {
+  count_word8(sh, lane, a.x); count_word8(sh, lane, a.y);
+  count_word8(sh, lane, a.z); count_word8(sh, lane, a.w);
+}
+
+// One thread's share of a tile of fp8 values (16-value groups of 16 bytes).
+__device__ __forceinline__ void count_tile8(uint32_t *sh, int lane, int tid, const uint8_t *src,
+                                            uint32_t nfull, uint32_t count) {
+  uint32_t g = tid;
+  for (; g + 3 * kHistThreads < nfull; g += 4 * kHistThreads) {
+    uint4 a0 = ld_nc_v4(src + 16 * g), a1 = ld_nc_v4(src + 16 * (g + kHistThreads));
+    uint4 a2 = ld_nc_v4(src + 16 * (g + 2 * kHistThreads)), a3 = ld_nc_v4(src + 16 * (g + 3 * kHistThreads));
+    count_quad8(sh, lane, a0);
+    count_quad8(sh, lane, a1);
+    count_quad8(sh, lane, a2);
+    count_quad8(sh, lane, a3);
+  }
+  for (; g < nfull; g += kHistThreads) count_quad8(sh, lane, ld_nc_v4(src + 16 * g));
+  if (g == nfull)  // the thread whose next group is the ragged tail
+    for (uint32_t v = 16 * nfull; v < count; v++)
+      atomicAdd(&sh[(fp8_code(src[v]) << 5) | lane], 1u);
+}
+
 // One thread's share of a tile of 2-byte values: groups tid, tid + 512, ...
 // with four groups of loads in flight.
 template <int DT>
@@ -228,6 +260,8 @@ __global__ void __launch_bounds__(kHistThreads, 2) k_hist(const __grid_constant_
     count_tile16<WC_BF16>(sh, lane, tid, reinterpret_cast<const uint16_t *>(it.in) + v0, nfull, count);
   } else if (it.dtype == WC_FP16) {
     count_tile16<WC_FP16>(sh, lane, tid, reinterpret_cast<const uint16_t *>(it.in) + v0, nfull, count);
+  } else if (it.dtype == WC_FP8E4M3) {
+    count_tile8(sh, lane, tid, it.in + v0, nfull, count);
   } else {
     const uint32_t *src = reinterpret_cast<const uint32_t *>(it.in) + v0;
     uint32_t g = tid;

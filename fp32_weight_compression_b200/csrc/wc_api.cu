@@ -28,7 +28,9 @@ constexpr uint64_t kMaxN = uint64_t(1) << 44;
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
-bool dtype_ok(int32_t dt) { return dt == WC_BF16 || dt == WC_FP32 || dt == WC_FP16; }
+bool dtype_ok(int32_t dt) {
+  return dt == WC_BF16 || dt == WC_FP32 || dt == WC_FP16 || dt == WC_FP8E4M3;
+}
 
 struct DeviceInfo {
   int sms = 0;

@@ -127,6 +127,9 @@ __device__ __forceinline__ uint4 ld_nc_v4(const void *p) {
                : "l"(p));
   return r;
 }
+__device__ __forceinline__ void st_cs_v2(void *p, uint2 v) {
+  asm volatile("st.global.cs.v2.u32 [%0], {%1,%2};\n" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
 __device__ __forceinline__ void st_cs_v4(void *p, uint4 v) {
   asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};\n" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w)

@@ -60,7 +60,7 @@ __host__ __device__ inline uint32_t chunk_nsym(uint64_t n, uint64_t k) {
 struct Layout {
   uint64_t n, nc;
   uint64_t off_chunk_off, off_chunk_len;
-  uint64_t off_raw;   // bf16: sign+mantissa bytes; fp16: low bytes; fp32: sign bits
+  uint64_t off_raw;   // bf16: sign+mantissa bytes; fp16: low bytes; fp8: low nibbles; fp32: sign bits
   uint64_t off_mant;  // fp32 only
   uint64_t off_exp;
 };
@@ -72,14 +72,22 @@ __host__ __device__ inline Layout make_layout(uint64_t n, int dtype) {
   L.off_chunk_off = kChunkOffOffset;
   L.off_chunk_len = L.off_chunk_off + 8 * (L.nc + 1);
   L.off_raw = round16(L.off_chunk_len + 4 * L.nc);
-  if (dtype != WC_FP32) {  // 2-byte dtypes: one raw byte per value
+  if (dtype == WC_BF16 || dtype == WC_FP16) {  // one raw byte per value
     L.off_mant = 0;
     L.off_exp = round16(L.off_raw + n);
+  } else if (dtype == WC_FP8E4M3) {  // one raw nibble per value
+    L.off_mant = 0;
+    L.off_exp = round16(L.off_raw + (n + 1) / 2);
   } else {
     L.off_mant = round16(L.off_raw + (n + 7) / 8);
     L.off_exp = round16(L.off_mant + 3 * n);
   }
   return L;
+}
+
+// Bytes per value.
+__host__ __device__ constexpr uint32_t dtype_bytes(int dtype) {
+  return dtype == WC_FP32 ? 4 : (dtype == WC_FP8E4M3 ? 1 : 2);
 }
 
 __host__ __device__ inline uint64_t scratch_win_offset(uint64_t nc) {

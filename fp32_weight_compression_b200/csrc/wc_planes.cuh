@@ -63,4 +63,33 @@ __device__ __forceinline__ uint2 merge4(uint32_t c4, uint32_t r4) {
   return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
 }
 
+// ---------------------------------------------------------------------------
+// fp8 e4m3 [S:1 E:4 M:3]: the reorder gives E<<4 | S<<3 | M; the coded symbol
+// is the exponent nibble E, the raw plane holds the low nibbles S<<3 | M two
+// per byte (even value in the low half).  Four values per 32-bit word, one per
+// byte lane.
+
+__device__ __forceinline__ uint32_t fp8_code(uint32_t b) { return (b >> 3) & 0xFu; }
+__device__ __forceinline__ uint32_t fp8_nibble(uint32_t b) { return ((b >> 4) & 8u) | (b & 7u); }
+__device__ __forceinline__ uint32_t fp8_merge(uint32_t code, uint32_t nib) {
+  return ((nib & 8u) << 4) | ((code & 0xFu) << 3) | (nib & 7u);
+}
+
+__device__ __forceinline__ uint32_t fp8_code4(uint32_t w) { return (w >> 3) & 0x0F0F0F0Fu; }
+__device__ __forceinline__ uint32_t fp8_nibble4(uint32_t w) {
+  return ((w >> 4) & 0x08080808u) | (w & 0x07070707u);
+}
+// the low nibbles of 8 values (two words) packed into 4 bytes
+__device__ __forceinline__ uint32_t fp8_pack8(uint32_t w0, uint32_t w1) {
+  const uint32_t t0 = fp8_nibble4(w0), t1 = fp8_nibble4(w1);
+  return __byte_perm(t0 | (t0 >> 4), t1 | (t1 >> 4), 0x6420);
+}
+// 8 values (coded bytes c8, packed nibbles r) -> 8 value bytes as two words
+__device__ __forceinline__ uint2 fp8_merge8(uint2 c8, uint32_t r) {
+  const uint32_t lo = r & 0x0F0F0F0Fu, hi = (r >> 4) & 0x0F0F0F0Fu;
+  const uint32_t n0 = __byte_perm(lo, hi, 0x5140), n1 = __byte_perm(lo, hi, 0x7362);
+  return make_uint2(((n0 & 0x08080808u) << 4) | ((c8.x & 0x0F0F0F0Fu) << 3) | (n0 & 0x07070707u),
+                    ((n1 & 0x08080808u) << 4) | ((c8.y & 0x0F0F0F0Fu) << 3) | (n1 & 0x07070707u));
+}
+
 }  // namespace wc

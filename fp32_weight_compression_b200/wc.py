@@ -16,12 +16,14 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libwc.so")
 
 OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CUDA, ERR_CORRUPT, ERR_UNSUPPORTED = 0, 1, 2, 3, 4, 5
-BF16, FP32, FP16 = 1, 2, 3
+BF16, FP32, FP16, FP8E4M3 = 1, 2, 3, 4
 CHUNK = 65536
 
-_DT = {torch.bfloat16: BF16, torch.float32: FP32, torch.float16: FP16}
-_TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32, FP16: torch.float16}
-_ELEM = {BF16: 2, FP32: 4, FP16: 2}
+_DT = {torch.bfloat16: BF16, torch.float32: FP32, torch.float16: FP16,
+       torch.float8_e4m3fn: FP8E4M3}
+_TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32, FP16: torch.float16,
+             FP8E4M3: torch.float8_e4m3fn}
+_ELEM = {BF16: 2, FP32: 4, FP16: 2, FP8E4M3: 1}
 
 EXPORTS = (
     "wc_encode_bound", "wc_scratch_bytes", "wc_encode", "wc_decode", "wc_decode_chunk",
@@ -135,7 +137,7 @@ def dtype_code(dtype: torch.dtype) -> int:
     try:
         return _DT[dtype]
     except KeyError:
-        raise TypeError(f"unsupported dtype {dtype}: bf16, fp16 and fp32 only") from None
+        raise TypeError(f"unsupported dtype {dtype}: bf16, fp16, fp32 and fp8 e4m3 only") from None
 
 
 def encode_bound(n: int, dtype) -> int:

@@ -24,8 +24,10 @@
  * u64 off_raw, u64 off_exp, u64 exp_bytes, u64 total_bytes (64 bytes), then
  * u16 freq[256], u64 chunk_off[nc+1], u32 chunk_len[nc], the raw planes
  * (bf16: n sign+mantissa bytes; fp32: ceil(n/8) sign-bit bytes, 3n mantissa
- * bytes; fp16: n low bytes) and the exponent chunks (bf16 / fp32: the
- * exponent byte; fp16: the reordered high byte).  A coded chunk is 32 final u32 states then
+ * bytes; fp16: n low bytes; fp8 e4m3: ceil(n/2) bytes of low nibbles) and
+ * the exponent chunks (bf16 / fp32: the exponent byte; fp16: the reordered
+ * high byte; fp8 e4m3: the exponent nibble).  Values are passed as raw bits
+ * (bf16 / fp16 2 bytes, fp32 4, fp8 1).  A coded chunk is 32 final u32 states then
  * w u16 renormalisation words (128 + 2w bytes); a chunk whose coded form is
  * not smaller than its nsym exponent bytes is stored raw.  The format is
  * fully determined by the input bits: one input has exactly one container.
@@ -77,7 +79,11 @@ typedef enum {
  * E S M ("PTWM", How it works 1-2: float16 / bfloat16 are split into 2 byte
  * planes, plane 1 coded); for fp16 the coded byte holds the 5 exponent bits,
  * the sign and the top 2 mantissa bits, the raw byte the other 8. */
-typedef enum { WC_BF16 = 1, WC_FP32 = 2, WC_FP16 = 3 } wc_dtype;
+/* WC_FP8E4M3: the reorder puts the 4 exponent bits in the high nibble and a
+ * nibble split codes them ("PTWM", How it works 1-2: float8 formats are split
+ * into 2 nibble planes, plane 0 = exponent nibbles); the low nibbles (sign
+ * above 3 mantissa bits) are stored raw, two per byte, even value low. */
+typedef enum { WC_BF16 = 1, WC_FP32 = 2, WC_FP16 = 3, WC_FP8E4M3 = 4 } wc_dtype;
 
 /* Worst-case container size in bytes for n values of dtype: every chunk
  * stored raw ("PTWM" Configuration table, compression_threshold: the coded
@@ -136,7 +142,7 @@ WC_API int32_t wc_read_header(const void *h_cont, uint64_t bytes, uint64_t *n,
 typedef struct {
     const void *in;       /* n values, 16-byte aligned                   */
     uint64_t n;
-    int32_t dtype;        /* WC_BF16, WC_FP32 or WC_FP16                 */
+    int32_t dtype;        /* a wc_dtype                                  */
     int32_t reserved;     /* must be 0                                   */
     void *out;            /* container, out_cap >= wc_encode_bound(n)    */
     uint64_t out_cap;
@@ -214,7 +220,7 @@ WC_API int32_t wc_encode_noalloc(const void *d_in, uint64_t n, int32_t dtype, vo
 typedef struct {
     const void *h_in;       /* n values (host)                              */
     uint64_t n;
-    int32_t dtype;          /* WC_BF16, WC_FP32 or WC_FP16                  */
+    int32_t dtype;          /* a wc_dtype                                   */
     int32_t reserved;       /* must be 0                                    */
     void *h_out;            /* container (host)                             */
     uint64_t h_out_cap;     /* must be >= wc_encode_bound(n, dtype)         */

@@ -9,13 +9,15 @@ from fp32_weight_compression_b200 import wc
 
 
 def to_device(bits: np.ndarray) -> torch.Tensor:
-    """uint16 bits -> bf16 tensor, float16 values -> fp16 tensor, uint32 bits
-    -> fp32 tensor, on cuda:0."""
+    """uint16 bits -> bf16 tensor, float16 values -> fp16 tensor, uint8 bits
+    -> fp8 e4m3 tensor, uint32 bits -> fp32 tensor, on cuda:0."""
     bits = np.ascontiguousarray(bits)
     if bits.dtype == np.uint16:
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
     elif bits.dtype == np.float16:
         t = torch.from_numpy(bits.view(np.int16)).view(torch.float16)
+    elif bits.dtype == np.uint8:
+        t = torch.from_numpy(bits.copy()).view(torch.float8_e4m3fn)
     elif bits.dtype == np.uint32:
         t = torch.from_numpy(bits.view(np.int32)).view(torch.float32)
     else:
@@ -29,6 +31,8 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
         return t.view(torch.int16).cpu().numpy().view(np.uint16)
     if t.dtype == torch.float16:
         return t.view(torch.int16).cpu().numpy().view(np.float16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).cpu().numpy()
     if t.dtype == torch.float32:
         return t.view(torch.int32).cpu().numpy().view(np.uint32)
     raise TypeError(t.dtype)

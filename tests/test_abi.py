@@ -44,7 +44,7 @@ def test_every_declared_symbol_is_exported(wcm):
 def test_bound_matches_oracle(wcm, orc, n, dt):
     assert wcm.encode_bound(n, dt) == orc.encode_bound(n, dt)
     assert wcm.scratch_bytes(n, dt) >= 7424
-    assert wcm.encode_bound(n, 4) == 0
+    assert wcm.encode_bound(n, 5) == 0
 
 
 def test_read_header_matches_oracle(wcm, orc):

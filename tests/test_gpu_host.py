@@ -24,6 +24,9 @@ def _bits(n, dt, seed):
     x = np.random.default_rng(seed).standard_normal(n).astype(np.float32) * np.float32(0.02)
     if dt == "fp16":
         return x.astype(np.float16)
+    if dt == "fp8":
+        e = np.clip(np.random.default_rng(seed).normal(6, 1.3, n), 0, 15).astype(np.int64)
+        return ((e << 3) | (np.arange(n) % 8) | ((np.arange(n) % 3 == 0) << 7)).astype(np.uint8)
     return workloads.rne_bf16(x) if dt == "bf16" else x.view(np.uint32).copy()
 
 
@@ -32,6 +35,8 @@ def _host(bits, pin=True):
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
     elif bits.dtype == np.float16:
         t = torch.from_numpy(bits.view(np.int16)).view(torch.float16)
+    elif bits.dtype == np.uint8:
+        t = torch.from_numpy(bits.copy()).view(torch.float8_e4m3fn)
     else:
         t = torch.from_numpy(bits.view(np.int32)).view(torch.float32)
     return t.pin_memory() if pin else t.clone()
@@ -39,8 +44,8 @@ def _host(bits, pin=True):
 
 def _set():
     sizes = [0, 1, 100, C - 3, C, C + 5, 3 * C + 17, 5 * C, 17, 2 * C + 1]
-    kinds = ["fp32", "bf16", "fp16"]
-    return [_bits(n, kinds[i % 3], 500 + i) for i, n in enumerate(sizes)]
+    kinds = ["fp32", "bf16", "fp16", "fp8"]
+    return [_bits(n, kinds[i % 4], 500 + i) for i, n in enumerate(sizes)]
 
 
 @pytest.mark.parametrize("window", [1, 1 << 20, 0])    # one item per window .. one slot per window
@@ -49,7 +54,8 @@ def test_host_round_trip_matches_oracle(orc, slots, window):
     from fp32_weight_compression_b200 import wc
     arrs = _set()
     ts = [_host(a) for a in arrs]
-    code = {np.dtype(np.uint16): 1, np.dtype(np.uint32): 2, np.dtype(np.float16): 3}
+    code = {np.dtype(np.uint16): 1, np.dtype(np.uint32): 2, np.dtype(np.float16): 3,
+            np.dtype(np.uint8): 4}
     big = max(wc.host_encode_footprint(a.size, code[a.dtype]) for a in arrs)
     slot = (big + 256 + 255) // 256 * 256
     work = 256 * ((4 * len(arrs) + 255) // 256) + slots * slot   # status words + slots
@@ -59,7 +65,7 @@ def test_host_round_trip_matches_oracle(orc, slots, window):
         assert np.array_equal(c.numpy(), orc.encode(a))
     outs = codec.decode(conts)
     for a, o in zip(arrs, outs):
-        got = o.view(torch.int32 if a.dtype == np.uint32 else torch.int16).numpy()
+        got = o.view({4: torch.int32, 2: torch.int16, 1: torch.uint8}[a.dtype.itemsize]).numpy()
         assert np.array_equal(got.view(a.dtype), a)
 
 

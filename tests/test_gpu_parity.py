@@ -314,3 +314,51 @@ def test_mixed_dtype_batch(orc, gu):
     outs = wc.decode_batch(conts, [(a.size,) for a in arrs], [t.dtype for t in ts])
     for a, o in zip(arrs, outs):
         assert np.array_equal(gu.to_bits(o).view(a.dtype), a)
+
+
+# ---------------------------------------------------------------- fp8 e4m3
+def _fp8(n, seed):
+    """Bits of e4m3 values with a weight-like skew: exponents around 6."""
+    rng = np.random.default_rng(seed)
+    e = np.clip(rng.normal(6, 1.3, n), 0, 15).astype(np.int64)
+    return ((rng.integers(0, 2, n) << 7) | (e << 3) | rng.integers(0, 8, n)).astype(np.uint8)
+
+
+def _check8(orc, gu, bits):
+    want = orc.encode(bits)
+    got, back = gu.gpu_roundtrip(bits)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert np.array_equal(back, bits)
+
+
+@pytest.mark.parametrize("n", [0, 1, 2, 3, 15, 16, 17, 33, 511, 513, 65535, 65536, 65537,
+                               3 * C + 17, 5 * C + 511])
+def test_fp8_edge_sizes(orc, gu, n):
+    _check8(orc, gu, _fp8(n, seed=n + 11))
+
+
+def test_fp8_all_patterns_and_kinds(orc, gu):
+    pats = np.arange(256, dtype=np.uint8)
+    _check8(orc, gu, np.tile(pats, 300))                           # near-uniform: raw chunks
+    base = _fp8(4 * C + 3, seed=12)
+    base[np.random.default_rng(13).choice(base.size, 256, replace=False)] = pats
+    _check8(orc, gu, base)                                        # coded with every pattern
+    _check8(orc, gu, np.full(2 * C + 9, 0x38, np.uint8))           # single symbol
+
+
+def test_fp8_random_access_and_mixed_batch(orc, gu):
+    from fp32_weight_compression_b200 import wc
+    bits = _fp8(4 * C + 999, seed=14)
+    d = gu.cont_device(orc.encode(bits))
+    for k in range(5):
+        got = wc.decode_chunk(d, k).view(torch.uint8).cpu().numpy()
+        assert np.array_equal(got, bits[k * C:(k + 1) * C])
+    arrs = [_fp8(2 * C + 7, 15), _normal_bits(C + 3, "bf16", 16), _fp8(101, 17), _fp16(C, 18),
+            _normal_bits(77, "fp32", 19), _fp8(3 * C, 20)]
+    ts = [gu.to_device(a) for a in arrs]
+    conts = wc.encode_batch(ts)
+    for a, c in zip(arrs, conts):
+        assert np.array_equal(c.cpu().numpy(), orc.encode(a))
+    outs = wc.decode_batch(conts, [(a.size,) for a in arrs], [t.dtype for t in ts])
+    for a, o in zip(arrs, outs):
+        assert np.array_equal(gu.to_bits(o).view(a.dtype), a)
