@@ -1,6 +1,7 @@
 // wc_host.cu -- encode and decode of host-resident tensors through the device
-// in windows ("seedpack 0.2.0 -> 0.2.2", README: models are streamed through
-// the GPU in windows of about 1 GB, tensor by tensor).
+// in windows ("seedpack 0.2.0 -> 0.2.2", README: a BF16 model larger than the
+// GPU's memory is handled in groups of tensors of roughly a gigabyte and
+// unpacked on the GPU one tensor after another).
 //
 // The caller's device workspace is cut into K slots (K = 3 when the largest
 // item allows it, else 2, else 1).  Consecutive items are grouped into

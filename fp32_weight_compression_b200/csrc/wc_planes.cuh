@@ -1,6 +1,6 @@
 // wc_planes.cuh -- the two byte planes of a 2-byte value and back ("PTWM",
-// How it works 1-2: the reorder S E M -> E S M, then a 2-plane byte split
-// whose high byte, plane 1, is the coded one).
+// How it works 1-2: the reorder S E M -> E S M, then the value is cut into its
+// bytes and the high, exponent-bearing byte is the one that is coded).
 //   bf16 [S:1 E:8 M:7]   coded byte E                       raw byte S<<7 | M
 //   fp16 [S:1 E:5 M:10]  coded byte E<<3 | S<<2 | M>>8      raw byte M & 0xFF
 // The scalar forms take one 16-bit value.  The x4 forms work on four values

@@ -8,7 +8,8 @@
  * original bits.  The method follows:
  *   - "PTWM" (PyPI README), "How it works": 1. Bit reorder (the exponent
  *     moves to the top byte, the sign is tucked under it) and 2. Byte /
- *     nibble split (bf16: 2 planes, plane 1 = exponent); the exponent plane
+ *     nibble split (a bf16 value becomes two byte planes, the high one the
+ *     exponent); the exponent plane
  *     holds ~20 distinct values, the mantissa planes look random;
  *   - "SMEF -- blog companion code", file table: pass3_streams.py splits
  *     sign / exponent / mantissa streams, pass4_rans.py is the rANS coder;
@@ -75,14 +76,14 @@ typedef enum {
     WC_ERR_UNSUPPORTED = 5
 } wc_status;
 
-/* WC_FP16: the same 2-plane byte split as bf16 after the reorder S E M ->
- * E S M ("PTWM", How it works 1-2: float16 / bfloat16 are split into 2 byte
- * planes, plane 1 coded); for fp16 the coded byte holds the 5 exponent bits,
- * the sign and the top 2 mantissa bits, the raw byte the other 8. */
-/* WC_FP8E4M3: the reorder puts the 4 exponent bits in the high nibble and a
- * nibble split codes them ("PTWM", How it works 1-2: float8 formats are split
- * into 2 nibble planes, plane 0 = exponent nibbles); the low nibbles (sign
- * above 3 mantissa bits) are stored raw, two per byte, even value low. */
+/* WC_FP16: after the reorder S E M -> E S M an fp16 value is cut into its
+ * two bytes like a bf16 one and the high byte is coded ("PTWM", How it works
+ * 1-2); for fp16 that byte holds the 5 exponent bits, the sign and the top 2
+ * mantissa bits, and the raw byte the other 8. */
+/* WC_FP8E4M3: the reorder puts the 4 exponent bits in the high nibble and the
+ * value is cut into its two nibbles, the exponent nibbles being the coded
+ * stream ("PTWM", How it works 1-2); the low nibbles (sign above 3 mantissa
+ * bits) are stored raw, two per byte, even value low. */
 typedef enum { WC_BF16 = 1, WC_FP32 = 2, WC_FP16 = 3, WC_FP8E4M3 = 4 } wc_dtype;
 
 /* Worst-case container size in bytes for n values of dtype: every chunk
@@ -191,8 +192,9 @@ WC_API int32_t wc_encode_noalloc(const void *d_in, uint64_t n, int32_t dtype, vo
                                  uint64_t out_cap, uint64_t *d_out_size, void *stream);
 
 /* Host-resident tensors, encoded and decoded through the device in windows
- * ("seedpack 0.2.0 -> 0.2.2", README: a model is streamed through the GPU in
- * windows of about 1 GB, tensor by tensor).
+ * ("seedpack 0.2.0 -> 0.2.2", README: a BF16 model larger than the GPU's
+ * memory is handled in groups of tensors of roughly a gigabyte and unpacked
+ * on the GPU one tensor after another).
  *
  * The items' buffers (h_*) are host memory; on the device the calls use only
  * the caller's workspace d_work (256-byte aligned, work_cap bytes).  The

@@ -21,11 +21,12 @@
  *    bits.  For fp16 the same reorder and 2-plane byte split give a coded
  *    high byte of 5 exponent bits, the sign and the top 2 mantissa bits, and
  *    a raw low byte of the other 8 mantissa bits ("PTWM", "How it works" 2:
- *    float16 / bfloat16 are split into 2 byte planes, plane 1 = exponent).
+ *    16-bit floats are cut into their two bytes, the high byte being the
+ *    exponent-bearing one).
  *    For fp8 e4m3 the reorder S E M -> E S M puts the 4 exponent bits in the
  *    high nibble and a nibble split separates them ("PTWM", "How it works"
- *    1-2: float8 formats are split into 2 nibble planes, plane 0 = exponent
- *    nibbles): the coded symbol is the exponent nibble, and the low nibbles
+ *    1-2: 8-bit floats are cut into two nibbles, the exponent nibbles forming
+ *    a stream of their own): the coded symbol is the exponent nibble, and the low nibbles
  *    (sign above 3 mantissa bits) are stored raw, two per byte.
  *    For fp32 the container keeps three streams: sign bits, the 8-bit
  *    exponent, and the 23-bit mantissa stored as 3 little-endian bytes.
