@@ -185,10 +185,12 @@ def kernel_sources_sha(files) -> str:
 
 DECODE_SOURCES = ["fp32_weight_compression_b200/csrc/k_decode.cu",
                   "fp32_weight_compression_b200/csrc/wc_format.cuh",
-                  "fp32_weight_compression_b200/csrc/wc_block.cuh"]
+                  "fp32_weight_compression_b200/csrc/wc_block.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_planes.cuh"]
 CODER_SOURCES = ["fp32_weight_compression_b200/csrc/k_encode.cu",
                  "fp32_weight_compression_b200/csrc/wc_format.cuh",
-                 "fp32_weight_compression_b200/csrc/wc_block.cuh"]
+                 "fp32_weight_compression_b200/csrc/wc_block.cuh",
+                 "fp32_weight_compression_b200/csrc/wc_planes.cuh"]
 
 
 # ---------------------------------------------------------------------------
