@@ -13,9 +13,9 @@
 //   out(w) waits for compute(w)
 // so that with K = 3 the copies in both directions and the kernels of three
 // consecutive windows overlap.  Encoding needs each container's size on the
-// host before its copy back: the host reads the sizes of window w - 1 (a
-// copy that returns when the encode of w - 1 is done) after it has queued
-// window w, so the device never waits for the host.
+// host before its copy back: the host reads the sizes of window w - 1 (on a
+// stream of its own, so the read waits for the encode of w - 1 and nothing
+// else) after it has queued window w, so the device never waits for the host.
 #include <cstring>
 #include <vector>
 
@@ -47,6 +47,16 @@ struct Events {
   ~Events() {
     for (auto &e : ev)
       if (e) cudaEventDestroy(e);
+  }
+};
+
+// A non-blocking stream owned by one call.
+struct OwnStream {
+  cudaStream_t s = nullptr;
+  bool ok = false;
+  OwnStream() { ok = cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) == cudaSuccess; }
+  ~OwnStream() {
+    if (s) cudaStreamDestroy(s);
   }
 };
 
@@ -129,7 +139,8 @@ int32_t wc_encode_host(const wc_host_encode_item *items, uint32_t count, void *d
   cudaStream_t s_cp = static_cast<cudaStream_t>(stream_compute);
   cudaStream_t s_out = static_cast<cudaStream_t>(stream_out);
   Events E(3 * K);  // [0, K) copied in, [K, 2K) encoded, [2K, 3K) copied out
-  if (!E.ok) return WC_ERR_CUDA;
+  OwnStream szs;    // size read-back, so that it waits for nothing but its window
+  if (!E.ok || !szs.ok) return WC_ERR_CUDA;
 
   // device addresses of window w's items
   std::vector<wc_encode_item> di(count);
@@ -156,15 +167,18 @@ int32_t wc_encode_host(const wc_host_encode_item *items, uint32_t count, void *d
       d.out_size = sz + (i - b);
     }
   };
-  // Copy window v's containers back (blocks the host until v is encoded).
+  // Copy window v's containers back.  The host waits for window v's encode
+  // only (its sizes come back on a stream of their own), not for the copies
+  // of earlier windows still queued on stream_out.
   auto finish = [&](uint32_t v) -> int32_t {
     const uint32_t b = v ? wend[v - 1] : 0, e = wend[v];
     const uint32_t s = v % K;
-    cudaError_t ce = cudaStreamWaitEvent(s_out, E.ev[K + s], 0);
+    cudaError_t ce = cudaStreamWaitEvent(szs.s, E.ev[K + s], 0);
     if (ce == cudaSuccess)  // pageable destination: returns once the copy is done
       ce = cudaMemcpyAsync(sizes.data() + b, di[b].out_size, 8 * uint64_t(e - b),
-                           cudaMemcpyDeviceToHost, s_out);
-    if (ce == cudaSuccess) ce = cudaStreamSynchronize(s_out);
+                           cudaMemcpyDeviceToHost, szs.s);
+    if (ce == cudaSuccess) ce = cudaStreamSynchronize(szs.s);
+    if (ce == cudaSuccess) ce = cudaStreamWaitEvent(s_out, E.ev[K + s], 0);
     if (ce != cudaSuccess) return fail(ce);
     for (uint32_t i = b; i < e; i++) {
       if (sizes[i] > items[i].h_out_cap) return WC_ERR_CAPACITY;

@@ -211,7 +211,8 @@ WC_API int32_t wc_encode_noalloc(const void *d_in, uint64_t n, int32_t dtype, vo
  * Unlike the calls above, these two block: they return after every copy has
  * finished (or at the first error, after the work already queued is done) and
  * synchronise the three streams.  Each call creates and destroys a few CUDA
- * events; no memory is allocated.  Argument, header and capacity checks come
+ * events (and wc_encode_host one more stream, for reading sizes back); no
+ * memory is allocated.  Argument, header and capacity checks come
  * first and queue no work.
  *
  * Workspace: 256-byte rounded 4 * count bytes of status words, then the
