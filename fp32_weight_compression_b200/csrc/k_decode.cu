@@ -12,12 +12,12 @@
 //   slot = x & 4095; e = tab[slot]; x = f (x >> 12) + (slot - cum);
 //   if x < 2^16: x = x << 16 | next word
 // The lanes that need a word at a step take consecutive words in lane order
-// (__ballot_sync / __popc prefix), from a per-chunk 512-word shared-memory
+// (__ballot_sync / __popc prefix), from a per-chunk 1024-word shared-memory
 // ring that cp.async keeps filled with 16-byte loads of the chunk's word
-// stream.  Every 8 steps a chunk has 256 new exponent bytes; they are
-// transposed through shared memory so that each lane holds 8 consecutive
-// ones, merged with the matching raw-plane bytes, and written with one
-// 16-byte store (bf16) or two (fp32).
+// stream.  Every 8 steps a chunk has 256 new coded bytes; they are transposed
+// through shared memory so that each lane holds 8 consecutive ones, merged
+// with the matching raw-plane bytes, and written with one 16-byte store (bf16,
+// fp16), two (fp32) or one 8-byte store (fp8 e4m3).
 //
 // Everything read from the container is checked before use (header fields
 // against the layout implied by n, the table sum, each chunk's offset pair and

@@ -3,7 +3,7 @@
 //
 // Encode, per launch of up to kMaxItems tensors (all on `stream`):
 //   k_prep     header fields + scratch counters            (1 block / tensor)
-//   k_hist     exponent histogram -> 12-bit table          (1 block / chunk)
+//   k_hist     coded-byte histogram -> 12-bit table        (1 block / 4 chunks)
 //   k_coder    raw planes + rANS per chunk + offset scan   (1 warp / 2 chunks)
 //   k_compact  payloads into the exponent section          (1 block / chunk)
 // Decode, per launch of up to kMaxItems containers:

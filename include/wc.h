@@ -1,16 +1,16 @@
 /*
  * wc.h -- C ABI of the B200 (sm_100a) exponent-plane rANS weight codec.
  *
- * Lossless compression of bf16 / fp32 weight tensors.  Each float is split
- * into planes; the skewed 8-bit exponent plane is entropy-coded with a
- * static, 32-lane interleaved rANS coder, chunk by chunk; the sign and
+ * Lossless compression of bf16 / fp32 / fp16 / fp8 e4m3 weight tensors.
+ * Each float is split into planes; the skewed exponent plane is entropy-coded
+ * with a static, 32-lane interleaved rANS coder, chunk by chunk; the sign and
  * mantissa bits are stored raw.  Decoding re-merges the planes into the
  * original bits.  The method follows:
  *   - "PTWM" (PyPI README), "How it works": 1. Bit reorder (the exponent
- *     moves to the top byte, the sign is tucked under it) and 2. Byte /
- *     nibble split (a bf16 value becomes two byte planes, the high one the
- *     exponent); the exponent plane
- *     holds ~20 distinct values, the mantissa planes look random;
+ *     moves to the top, the sign is tucked under it) and 2. Byte / nibble
+ *     split (a bf16 value becomes two byte planes, the high one the
+ *     exponent); the exponent plane holds ~20 distinct values, the mantissa
+ *     planes look random;
  *   - "SMEF -- blog companion code", file table: pass3_streams.py splits
  *     sign / exponent / mantissa streams, pass4_rans.py is the rANS coder;
  *   - "PTWM", Configuration table: compression_threshold (store raw when
