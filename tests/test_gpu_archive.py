@@ -1,0 +1,58 @@
+"""The archive file on the GPU: save() writes the library's containers (byte
+for byte the oracle's) under their names, and load / load_chunk / load_all
+give the tensors back bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+C = 65536
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fp32_weight_compression_b200 import build
+    build.build()
+
+
+def _tensors():
+    import gpu_util as gu
+    rng = np.random.default_rng(21)
+    bf = workloads.rne_bf16(rng.standard_normal(3 * C + 5).astype(np.float32) * np.float32(0.02))
+    f32 = (rng.standard_normal(2 * C + 1).astype(np.float32) * np.float32(0.02)).view(np.uint32)
+    f16 = (rng.standard_normal(C + 77) * 0.05).astype(np.float16)
+    e = np.clip(rng.normal(6, 1.3, 2 * C + 9), 0, 15).astype(np.int64)
+    f8 = ((rng.integers(0, 2, e.size) << 7) | (e << 3) | rng.integers(0, 8, e.size)).astype(np.uint8)
+    bits = {"blk.0.attn.q": (bf, (5, 39325)), "norm": (f32, (2 * C + 1,)),
+            "h16": (f16, (C + 77, 1)), "f8": (f8, (2 * C + 9,)), "none": (np.zeros(0, np.uint16), (0,))}
+    return {k: (b, gu.to_device(b).reshape(s)) for k, (b, s) in bits.items()}
+
+
+def test_save_load_bit_exact(orc, tmp_path):
+    import gpu_util as gu
+    from fp32_weight_compression_b200 import archive
+    ts = _tensors()
+    path = str(tmp_path / "m.wca")
+    archive.save(path, {k: t for k, (_, t) in ts.items()})
+    with archive.Archive(path) as a:
+        assert a.names() == list(ts)
+        for k, (b, t) in ts.items():
+            assert a.info(k)[:2] == (t.dtype, tuple(t.shape))
+            assert np.array_equal(a.container(k), orc.encode(b))
+            got = a.load(k)
+            assert got.dtype == t.dtype and tuple(got.shape) == tuple(t.shape)
+            assert np.array_equal(gu.to_bits(got).reshape(-1).view(np.uint8), b.view(np.uint8))
+        # one chunk: the second of the bf16 tensor and the ragged last of fp8
+        part = a.load_chunk("blk.0.attn.q", 1)
+        assert np.array_equal(gu.to_bits(part), ts["blk.0.attn.q"][0][C:2 * C])
+        part = a.load_chunk("f8", 2)
+        assert np.array_equal(gu.to_bits(part), ts["f8"][0][2 * C:])
+        allv = a.load_all()
+        for k, (b, t) in ts.items():
+            assert torch.equal(allv[k].view(torch.uint8), t.view(torch.uint8))
+        some = a.load_all(["h16", "norm"])
+        assert list(some) == ["h16", "norm"]
