@@ -7,7 +7,7 @@ never calls it and shares no code with it.
 
 Pins of every oracle function (worked traces, normalisation examples, brute
 force, the rANS accounting bound, exhaustive bf16 round trip, fp32 special
-values) live in tests/test_oracle_*.py.
+values, CRC-32 check values and zlib) live in tests/test_oracle_*.py.
 """
 from __future__ import annotations
 
@@ -73,6 +73,9 @@ def lib():
                                               ctypes.POINTER(ctypes.c_double),
                                               ctypes.POINTER(ctypes.c_double),
                                               ctypes.POINTER(ctypes.c_double)]
+        L.oracle_crc32.restype = ctypes.c_uint32
+        L.oracle_crc32.argtypes = [vp, ctypes.c_uint64]
+        L.oracle_crc32_blocks.argtypes = [vp, ctypes.c_uint64, ctypes.c_uint64, vp]
         del u8p, u16p, u64p
         _lib = L
     return _lib
@@ -265,3 +268,27 @@ def chunk_accounting(sym, freq):
     if st:
         raise OracleError(st, "chunk_accounting")
     return a.value, b.value, c.value
+
+
+def _bytes_view(data) -> np.ndarray:
+    if isinstance(data, (bytes, bytearray, memoryview)):
+        return np.frombuffer(bytes(data), dtype=np.uint8)
+    return np.ascontiguousarray(data).reshape(-1).view(np.uint8)
+
+
+def crc32(data) -> int:
+    """CRC-32 (zlib / IEEE 802.3) of a byte string or array's bytes."""
+    buf = _bytes_view(data)
+    return int(lib().oracle_crc32(_ptr(buf) if buf.size else None, buf.size))
+
+
+def crc32_blocks(data, block_bytes: int) -> np.ndarray:
+    """CRC-32 of each block_bytes-sized block (the last one may be shorter)."""
+    buf = _bytes_view(data)
+    nb = -(-buf.size // block_bytes) if block_bytes > 0 else 0
+    out = np.zeros(nb, dtype=np.uint32)
+    st = lib().oracle_crc32_blocks(_ptr(buf) if buf.size else None, buf.size, block_bytes,
+                                   _ptr(out) if nb else None)
+    if st != OK:
+        raise OracleError(st, "oracle_crc32_blocks")
+    return out

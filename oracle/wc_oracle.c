@@ -709,3 +709,31 @@ int oracle_decode_chunk(const uint8_t *cont, uint64_t cont_bytes, uint64_t k,
     free(words);
     return st;
 }
+
+/* ---------------------------------------------------------------------------
+ * CRC-32, one bit at a time: the register holds the remainder with the
+ * coefficient of x^31 in bit 0 (bits are taken least significant first), so
+ * a step shifts right and, when a 1 falls out, subtracts (xors) the generator
+ * without its x^32 term, written in that same reversed order: 0xEDB88320. */
+uint32_t oracle_crc32(const uint8_t *data, uint64_t bytes) {
+    const uint32_t gen_reversed = 0xEDB88320u;
+    uint32_t r = 0xFFFFFFFFu;
+    for (uint64_t i = 0; i < bytes; i++) {
+        r ^= data[i];
+        for (int b = 0; b < 8; b++)
+            r = (r & 1u) ? (r >> 1) ^ gen_reversed : (r >> 1);
+    }
+    return r ^ 0xFFFFFFFFu;
+}
+
+int oracle_crc32_blocks(const uint8_t *data, uint64_t bytes, uint64_t block_bytes,
+                        uint32_t *crc) {
+    if (block_bytes == 0 || (bytes > 0 && (data == NULL || crc == NULL)))
+        return OR_ERR_INVALID_ARG;
+    for (uint64_t i = 0; i * block_bytes < bytes; i++) {
+        uint64_t len = bytes - i * block_bytes;
+        if (len > block_bytes) len = block_bytes;
+        crc[i] = oracle_crc32(data + i * block_bytes, len);
+    }
+    return OR_OK;
+}

@@ -72,6 +72,17 @@ int oracle_chunk_accounting(const uint8_t *sym, uint32_t nsym,
                             const uint16_t freq[256], double *coded_bits,
                             double *ideal_bits, double *slack_bound);
 
+/* CRC-32 of a byte string as zlib and IEEE 802.3 define it: generator
+ * x^32 + x^26 + x^23 + x^22 + x^16 + x^12 + x^11 + x^10 + x^8 + x^7 + x^5 +
+ * x^4 + x^2 + x + 1, bits taken least significant first, register preset to
+ * all ones and complemented at the end ("seedpack 0.2.0 -> 0.2.2", README:
+ * every chunk of an archive carries a CRC32). */
+uint32_t oracle_crc32(const uint8_t *data, uint64_t bytes);
+/* The CRC-32 of each block [i*block_bytes, min((i+1)*block_bytes, bytes)),
+ * i < ceil(bytes / block_bytes), into crc[i]. */
+int oracle_crc32_blocks(const uint8_t *data, uint64_t bytes, uint64_t block_bytes,
+                        uint32_t *crc);
+
 #ifdef __cplusplus
 }
 #endif
