@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--tensors", type=int, default=0,
                     help="profiling only: use the first N tensors of the set (0: all)")
     ap.add_argument("--no-e2e", action="store_true", help="profiling only: skip the e2e leg")
+    ap.add_argument("--checksum", action="store_true",
+                    help="also time wc_crc32_blocks (1 MiB blocks) over the container arena, "
+                         "outside the timed step; adds a 'checksum' object to the line")
     return ap.parse_args()
 
 
@@ -290,6 +293,27 @@ def e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world):
 
 
 # ---------------------------------------------------------------------------
+def checksum_leg(arena, dev, stream, reps: int = 10):
+    """wc_crc32_blocks over the whole container arena (larger than L2), 1 MiB
+    blocks: algorithmic bytes = the arena's bytes read (the CRCs written are
+    1/262144 of that)."""
+    import torch
+    from fp32_weight_compression_b200 import wc
+    for _ in range(3):
+        wc.crc32_blocks(arena, wc.CRC_BLOCK, stream)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * reps)]
+    torch.cuda.synchronize(dev)
+    for r in range(reps):
+        evs[2 * r].record(stream)
+        wc.crc32_blocks(arena, wc.CRC_BLOCK, stream)
+        evs[2 * r + 1].record(stream)
+    torch.cuda.synchronize(dev)
+    t = sum(evs[2 * r].elapsed_time(evs[2 * r + 1]) for r in range(reps)) / reps / 1e3
+    nbytes = arena.numel()
+    return {"kernel": "k_crc32", "bytes": nbytes, "block_bytes": wc.CRC_BLOCK, "ms": t * 1e3,
+            "gbs": nbytes / t / 1e9, "reps": reps}
+
+
 def main():
     args = parse()
     rank = int(os.environ.get("RANK", "0"))
@@ -387,6 +411,7 @@ def main():
     t_total, t_enc, t_dec = max_over_ranks([t_total, t_enc, t_dec], dev, world)
 
     t_e2e, E = e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world)
+    checksum = checksum_leg(enc.out, dev, stream) if args.checksum else None
 
     peak, peak_note = peak_hbm()
     B = total_in
@@ -431,6 +456,9 @@ def main():
         "clocks": clocks,
         "cpu_baseline": cpu_base,
     }
+    if checksum is not None:
+        checksum["roofline_frac"] = checksum["gbs"] / peak
+        line["checksum"] = checksum
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -7,17 +7,19 @@ Layout (little-endian):
     0   "WCA1"
     4   u32 version (1)
     8   u32 number of entries
-    12  u32 0
+    12  u32 checksum block B in bytes (0: no checksums)
     16  u64 offset of the index
     24  u64 bytes of the index
     32  the containers, each starting on a 16-byte boundary, zero padding
     index: per entry  u16 name bytes, the UTF-8 name, u8 dtype code,
            u8 number of dimensions, u64 per dimension, u64 container offset,
-           u64 container bytes
+           u64 container bytes, then (B > 0) one u32 CRC-32 per B-byte block
+           of the container, the last block short
 
 The containers are exactly those of the library (include/wc.h); this module
-only places them in a file and finds them again.  Encoding and decoding run on
-the GPU through the binding.
+only places them in a file and finds them again.  Encoding, decoding and the
+checksums ("seedpack 0.2.0 -> 0.2.2", README: a CRC32 per archive chunk) run
+on the GPU through the binding.
 """
 from __future__ import annotations
 
@@ -39,43 +41,59 @@ def _align16(v: int) -> int:
     return (v + 15) // 16 * 16
 
 
-def write(path: str, entries) -> None:
-    """Write an archive from (name, dtype code, shape, container bytes)
-    entries, in the given order."""
-    entries = list(entries)
+def _nblocks(nbytes: int, block: int) -> int:
+    return -(-nbytes // block) if block else 0
+
+
+def write(path: str, entries, crc_block: int = 0) -> None:
+    """Write an archive from (name, dtype code, shape, container bytes[,
+    CRCs]) entries, in the given order.  With crc_block > 0 every entry
+    carries the CRC-32 of each crc_block-byte block of its container."""
+    entries = [tuple(e) for e in entries]
     names = [e[0] for e in entries]
     if len(set(names)) != len(names):
         raise ValueError("duplicate tensor names")
+    if crc_block < 0 or crc_block >= 1 << 32:
+        raise ValueError("checksum block size out of range")
     offsets, off = [], _HEAD.size
-    for _, _, _, cont in entries:
+    for e in entries:
         offsets.append(off)
-        off = _align16(off + len(cont))
+        off = _align16(off + len(e[3]))
     index = bytearray()
-    for (name, code, shape, cont), o in zip(entries, offsets):
+    for e, o in zip(entries, offsets):
+        name, code, shape, cont = e[:4]
         nb = name.encode("utf-8")
         if len(nb) > 0xFFFF or len(shape) > 255:
             raise ValueError(f"entry {name!r}: name or rank too large")
         index += struct.pack("<H", len(nb)) + nb + struct.pack("<BB", int(code), len(shape))
         index += struct.pack(f"<{len(shape)}Q", *[int(d) for d in shape])
         index += struct.pack("<QQ", o, len(cont))
+        crcs = np.asarray(e[4] if len(e) > 4 and e[4] is not None else [], dtype=np.uint32)
+        if crcs.size != _nblocks(len(cont), crc_block):
+            raise ValueError(f"entry {name!r}: {crcs.size} checksums for "
+                             f"{_nblocks(len(cont), crc_block)} blocks")
+        index += crcs.astype("<u4").tobytes()
     with open(path, "wb") as fh:
-        fh.write(_HEAD.pack(MAGIC, VERSION, len(entries), 0, off, len(index)))
+        fh.write(_HEAD.pack(MAGIC, VERSION, len(entries), crc_block, off, len(index)))
         pos = _HEAD.size
-        for (_, _, _, cont), o in zip(entries, offsets):
+        for e, o in zip(entries, offsets):
             fh.write(b"\0" * (o - pos))
-            fh.write(bytes(cont))
-            pos = o + len(cont)
+            fh.write(bytes(e[3]))
+            pos = o + len(e[3])
         fh.write(b"\0" * (off - pos))
         fh.write(index)
 
 
-def save(path: str, tensors: dict, stream=None) -> None:
-    """Encode every tensor (CUDA tensors; one batched launch per kernel) and
-    write them to an archive under their names."""
+def save(path: str, tensors: dict, stream=None, crc_block: int = wc.CRC_BLOCK) -> None:
+    """Encode every tensor (CUDA tensors; one batched launch per kernel),
+    checksum each container on the device (crc_block 0: none) and write them
+    to an archive under their names."""
     items = list(tensors.items())
     conts = wc.encode_batch([t.contiguous() for _, t in items], stream)
-    write(path, [(name, wc.dtype_code(t.dtype), tuple(t.shape), c.cpu().numpy().tobytes())
-                 for (name, t), c in zip(items, conts)])
+    crcs = [wc.crc32_blocks(c, crc_block, stream) if crc_block else None for c in conts]
+    write(path, [(name, wc.dtype_code(t.dtype), tuple(t.shape), c.cpu().numpy().tobytes(),
+                  None if k is None else k.cpu().numpy().view(np.uint32))
+                 for (name, t), c, k in zip(items, conts, crcs)], crc_block)
 
 
 class Archive:
@@ -98,9 +116,10 @@ class Archive:
             raise
 
     def _read_index(self, size: int) -> None:
-        magic, version, count, _, ioff, ibytes = _HEAD.unpack_from(self._mm, 0)
+        magic, version, count, crc_block, ioff, ibytes = _HEAD.unpack_from(self._mm, 0)
         if magic != MAGIC or version != VERSION or ioff + ibytes > size:
             raise ValueError("not an archive or unsupported version")
+        self.crc_block = crc_block
         self._entries = {}
         p = ioff
         for _ in range(count):
@@ -114,10 +133,13 @@ class Archive:
             p += 8 * ndim
             off, nbytes = struct.unpack_from("<QQ", self._mm, p)
             p += 16
-            if p > ioff + ibytes:
-                raise ValueError("index runs past its stated size")
             if off < _HEAD.size or off + nbytes > ioff or off % 16:
                 raise ValueError(f"entry {name!r}: container outside the data section")
+            nck = _nblocks(nbytes, crc_block)
+            if p + 4 * nck > ioff + ibytes:
+                raise ValueError("index runs past its stated size")
+            crcs = np.frombuffer(self._mm, dtype="<u4", count=nck, offset=p).astype(np.uint32)
+            p += 4 * nck
             if code not in wc._TORCH_DT:
                 raise ValueError(f"entry {name!r}: unknown dtype code {code}")
             if name in self._entries:
@@ -125,7 +147,7 @@ class Archive:
             n, hcode, _ = wc.read_header(bytes(self._mm[off:off + min(nbytes, 64)]))
             if hcode != code or n != int(np.prod(shape, dtype=np.uint64)):
                 raise ValueError(f"entry {name!r}: container header disagrees with the index")
-            self._entries[name] = (code, tuple(shape), off, nbytes)
+            self._entries[name] = (code, tuple(shape), off, nbytes, crcs)
         if p != ioff + ibytes:
             raise ValueError("index size does not match its entries")
 
@@ -150,33 +172,58 @@ class Archive:
 
     def info(self, name: str) -> tuple[torch.dtype, tuple, int]:
         """(dtype, shape, container bytes) of an entry."""
-        code, shape, _, nbytes = self._entries[name]
+        code, shape, _, nbytes, _ = self._entries[name]
         return wc._TORCH_DT[code], shape, nbytes
+
+    def checksums(self, name: str) -> np.ndarray:
+        """The stored CRC-32 of each checksum block of the entry's container
+        (empty when the archive has none)."""
+        return self._entries[name][4].copy()
 
     def container(self, name: str) -> np.ndarray:
         """A copy of the entry's container bytes."""
-        _, _, off, nbytes = self._entries[name]
+        _, _, off, nbytes, _ = self._entries[name]
         return np.frombuffer(self._mm, dtype=np.uint8, count=nbytes, offset=off).copy()
 
-    def _device_container(self, name: str, device) -> torch.Tensor:
-        return torch.from_numpy(self.container(name)).to(device)
+    def _device_container(self, name: str, device, verify: bool, stream) -> torch.Tensor:
+        cont = torch.from_numpy(self.container(name)).to(device)
+        if verify and self.crc_block:
+            bad = self._bad_blocks(name, cont, stream)
+            if bad:
+                raise ValueError(f"entry {name!r}: checksum mismatch in block(s) {bad[:8]}")
+        return cont
 
-    def load(self, name: str, device="cuda", stream=None) -> torch.Tensor:
-        """Decode one tensor onto the device."""
-        code, shape, _, _ = self._entries[name]
-        cont = self._device_container(name, device)
+    def _bad_blocks(self, name: str, cont: torch.Tensor, stream) -> list[int]:
+        got = wc.crc32_blocks(cont, self.crc_block, stream).cpu().numpy().view(np.uint32)
+        return np.nonzero(got != self._entries[name][4])[0].tolist()
+
+    def verify(self, name: str, device="cuda", stream=None) -> list[int]:
+        """Indices of the checksum blocks of an entry whose CRC-32, computed on
+        the device, differs from the stored one (empty: intact, or no
+        checksums in this archive)."""
+        if not self.crc_block:
+            return []
+        cont = torch.from_numpy(self.container(name)).to(device)
+        return self._bad_blocks(name, cont, stream)
+
+    def load(self, name: str, device="cuda", stream=None, verify: bool = True) -> torch.Tensor:
+        """Decode one tensor onto the device (checksums checked first unless
+        verify is False; a mismatch raises ValueError)."""
+        code, shape = self._entries[name][:2]
+        cont = self._device_container(name, device, verify, stream)
         return wc.decode(cont, shape=shape, dtype=wc._TORCH_DT[code], stream=stream)
 
-    def load_chunk(self, name: str, k: int, device="cuda", stream=None) -> torch.Tensor:
+    def load_chunk(self, name: str, k: int, device="cuda", stream=None,
+                   verify: bool = True) -> torch.Tensor:
         """Values k * 65536 .. of one tensor (1-D), decoding that chunk only."""
         code = self._entries[name][0]
-        cont = self._device_container(name, device)
+        cont = self._device_container(name, device, verify, stream)
         return wc.decode_chunk(cont, k, dtype=wc._TORCH_DT[code], stream=stream)
 
-    def load_all(self, names=None, device="cuda", stream=None) -> dict:
+    def load_all(self, names=None, device="cuda", stream=None, verify: bool = True) -> dict:
         """Decode several tensors with one batched launch."""
         names = self.names() if names is None else list(names)
-        conts = [self._device_container(n, device) for n in names]
+        conts = [self._device_container(n, device, verify, stream) for n in names]
         shapes = [self._entries[n][1] for n in names]
         dtypes = [wc._TORCH_DT[self._entries[n][0]] for n in names]
         outs = wc.decode_batch(conts, shapes, dtypes, stream)

@@ -8,6 +8,8 @@
 //   k_compact  payloads into the exponent section          (1 block / chunk)
 // Decode, per launch of up to kMaxItems containers:
 //   k_decode   persistent grid, one warp per 2 chunks
+// Block checksums (wc_crc32_blocks):
+//   k_crc32    persistent grid, one block of the buffer per CTA at a time
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -35,6 +37,8 @@ bool dtype_ok(int32_t dt) {
 struct DeviceInfo {
   int sms = 0;
   int dec_blocks_per_sm = 0;
+  int crc_blocks_per_sm = 0;
+  cudaError_t crc_err = cudaSuccess;
 };
 
 DeviceInfo device_info(int32_t *err) {
@@ -59,6 +63,9 @@ DeviceInfo device_info(int32_t *err) {
       *err = cuda_fail(cudaGetLastError(), "decoder set-up");
       return DeviceInfo{};
     }
+    // the checksum kernel's set-up failing leaves the codec usable
+    cache[dev].crc_blocks_per_sm = wc::crc_blocks_per_sm();
+    if (cache[dev].crc_blocks_per_sm <= 0) cache[dev].crc_err = cudaGetLastError();
     cache[dev].dec_blocks_per_sm = nb;
     cache[dev].sms = sms;
   }
@@ -82,6 +89,27 @@ uint64_t wc_scratch_bytes(uint64_t n, int32_t dtype) {
   if (!dtype_ok(dtype) || n > kMaxN) return 0;
   const uint64_t nc = wc::num_chunks(n);
   return wc::scratch_win_offset(nc) + nc * wc::kWin;
+}
+
+int32_t wc_crc32_blocks(const void *d_buf, uint64_t bytes, uint64_t block_bytes, uint32_t *d_crc,
+                        void *stream) {
+  if (block_bytes == 0 || block_bytes % 8192 != 0 || block_bytes > (uint64_t(1) << 30))
+    return WC_ERR_INVALID_ARG;
+  if (bytes == 0) return WC_OK;
+  if (d_buf == nullptr || d_crc == nullptr || !aligned(d_buf, 16) || !aligned(d_crc, 4))
+    return WC_ERR_INVALID_ARG;
+  int32_t err = WC_OK;
+  const DeviceInfo di = device_info(&err);
+  if (err != WC_OK) return err;
+  if (di.crc_blocks_per_sm <= 0)
+    return cuda_fail(di.crc_err == cudaSuccess ? cudaErrorInvalidConfiguration : di.crc_err,
+                     "k_crc32 set-up");
+  const uint64_t nblocks = (bytes + block_bytes - 1) / block_bytes;
+  const uint64_t cap = uint64_t(di.sms) * uint64_t(di.crc_blocks_per_sm);
+  const int grid = int(nblocks < cap ? nblocks : cap);
+  const cudaError_t e = wc::launch_crc32(static_cast<const uint8_t *>(d_buf), bytes, block_bytes,
+                                         d_crc, grid, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? WC_OK : cuda_fail(e, "k_crc32 launch");
 }
 
 const char *wc_status_string(int32_t st) {

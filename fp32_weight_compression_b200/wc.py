@@ -110,6 +110,8 @@ def load() -> ctypes.CDLL:
     L.wc_decode_host.restype = i32
     L.wc_decode_host.argtypes = [ctypes.POINTER(HostDecodeItem), u32, vp, u64, u64, vp, vp, vp,
                                  ctypes.POINTER(i32)]
+    L.wc_crc32_blocks.restype = i32
+    L.wc_crc32_blocks.argtypes = [vp, u64, u64, vp, vp]
     _lib = L
     return L
 
@@ -377,6 +379,23 @@ def decode_batch(conts, shapes, dtypes, stream=None) -> list[torch.Tensor]:
     dec.decode(conts, outs, stream=stream)
     dec.check()
     return outs
+
+
+CRC_BLOCK = 1 << 20
+
+
+def crc32_blocks(buf: torch.Tensor, block_bytes: int = CRC_BLOCK, stream=None) -> torch.Tensor:
+    """CRC-32 (zlib's code) of each block_bytes-sized block of a contiguous
+    device tensor's bytes (wc_crc32_blocks); int32 tensor on the device, one
+    entry per block, the bits of the unsigned CRC."""
+    if not buf.is_cuda or not buf.is_contiguous():
+        raise ValueError("buffer must be a contiguous CUDA tensor")
+    nbytes = buf.numel() * buf.element_size()
+    nb = -(-nbytes // block_bytes) if block_bytes > 0 else 0
+    out = torch.empty(max(nb, 1), dtype=torch.int32, device=buf.device)
+    _check(load().wc_crc32_blocks(buf.data_ptr() if nbytes else None, nbytes, block_bytes,
+                                  out.data_ptr(), _stream(stream)), "wc_crc32_blocks")
+    return out[:nb]
 
 
 # ---------------------------------------------------------------------------

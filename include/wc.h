@@ -265,6 +265,22 @@ WC_API int32_t wc_decode_host(const wc_host_decode_item *h_items, uint32_t count
                               uint64_t work_cap, uint64_t window_bytes, void *stream_in,
                               void *stream_compute, void *stream_out, int32_t *h_status);
 
+/* CRC-32 of fixed-size blocks of a device buffer, the per-block check that
+ * an archive file keeps ("seedpack 0.2.0 -> 0.2.2", README: every chunk of an
+ * archive carries a CRC32).  The code is zlib's and IEEE 802.3's CRC-32
+ * (generator 0x04C11DB7, bits least significant first, register preset to
+ * all ones, result complemented; "123456789" gives 0xCBF43926).
+ *   d_buf        device, 16-byte aligned, `bytes` bytes (read only).  bytes
+ *                = 0 is allowed and queues nothing.
+ *   block_bytes  the block size: a multiple of 8192, at most 2^30.  Block i
+ *                is [i * block_bytes, min((i + 1) * block_bytes, bytes)).
+ *   d_crc        device, ceil(bytes / block_bytes) uint32, written in block
+ *                order.
+ * Queued on `stream`; returns WC_OK, WC_ERR_INVALID_ARG (null or misaligned
+ * pointer, bad block size) or WC_ERR_CUDA. */
+WC_API int32_t wc_crc32_blocks(const void *d_buf, uint64_t bytes, uint64_t block_bytes,
+                               uint32_t *d_crc, void *stream);
+
 /* Human-readable name of a wc_status code (static storage). */
 WC_API const char *wc_status_string(int32_t status);
 

@@ -86,6 +86,14 @@ def test_bad_arguments_rejected_without_device(wcm):
     assert L.wc_decode(ok_in, 1000, ok_out + 2, 100, ok_sz, None) == wcm.ERR_INVALID_ARG
     assert L.wc_decode(ok_in, 1000, ok_out, 100, None, None) == wcm.ERR_INVALID_ARG
     assert L.wc_decode_chunk(ok_in, 1000, 0, ok_out, 100, ok_sz + 2, None) == wcm.ERR_INVALID_ARG
+    # block checksums: block size, alignment and null pointers
+    assert L.wc_crc32_blocks(ok_in, 1000, 0, ok_out, None) == wcm.ERR_INVALID_ARG
+    assert L.wc_crc32_blocks(ok_in, 1000, 4096, ok_out, None) == wcm.ERR_INVALID_ARG
+    assert L.wc_crc32_blocks(ok_in, 1000, (1 << 30) + 8192, ok_out, None) == wcm.ERR_INVALID_ARG
+    assert L.wc_crc32_blocks(ok_in + 8, 1000, 8192, ok_out, None) == wcm.ERR_INVALID_ARG
+    assert L.wc_crc32_blocks(ok_in, 1000, 8192, ok_out + 2, None) == wcm.ERR_INVALID_ARG
+    assert L.wc_crc32_blocks(None, 1000, 8192, ok_out, None) == wcm.ERR_INVALID_ARG
+    assert L.wc_crc32_blocks(None, 0, 8192, None, None) == wcm.OK   # nothing to do
     assert wcm.status_string(4) == "WC_ERR_CORRUPT"
 
 

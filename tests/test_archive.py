@@ -130,3 +130,26 @@ def test_damaged_counts_and_headers_refused(orc, arc, tmp_path):
         with pytest.raises(ValueError):
             arc.Archive(str(p))
     assert ioff % 16 == 0
+
+
+def test_checksums_stored_and_read_back(orc, arc, tmp_path):
+    ents = _entries(orc)
+    block = 8192
+    path = str(tmp_path / "c.wca")
+    arc.write(path, [(n, c, s, cont.tobytes(), orc.crc32_blocks(cont, block))
+                     for n, c, s, _, cont in ents], crc_block=block)
+    with arc.Archive(path) as a:
+        assert a.crc_block == block
+        for name, _, _, _, cont in ents:
+            assert np.array_equal(a.container(name), cont)
+            assert np.array_equal(a.checksums(name), orc.crc32_blocks(cont, block))
+    # a wrong number of checksums is refused when writing
+    n, c, s, _, cont = ents[0]
+    with pytest.raises(ValueError):
+        arc.write(path, [(n, c, s, cont.tobytes(), orc.crc32_blocks(cont, block)[:-1])], crc_block=block)
+    with pytest.raises(ValueError):
+        arc.write(path, [(n, c, s, cont.tobytes())], crc_block=block)
+    # without checksums the list is empty
+    arc.write(path, [(n, c, s, cont.tobytes())])
+    with arc.Archive(path) as a:
+        assert a.crc_block == 0 and a.checksums(n).size == 0

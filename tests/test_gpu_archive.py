@@ -56,3 +56,34 @@ def test_save_load_bit_exact(orc, tmp_path):
             assert torch.equal(allv[k].view(torch.uint8), t.view(torch.uint8))
         some = a.load_all(["h16", "norm"])
         assert list(some) == ["h16", "norm"]
+
+
+def test_checksums_catch_a_damaged_container(orc, tmp_path):
+    import gpu_util as gu
+    from fp32_weight_compression_b200 import archive
+    ts = _tensors()
+    path = tmp_path / "c.wca"
+    block = 65536
+    archive.save(str(path), {k: t for k, (_, t) in ts.items()}, crc_block=block)
+    with archive.Archive(str(path)) as a:
+        assert a.crc_block == block
+        for k in ts:
+            assert np.array_equal(a.checksums(k), orc.crc32_blocks(a.container(k), block))
+            assert a.verify(k) == []
+        off = a._entries["blk.0.attn.q"][2]
+        size = a.info("blk.0.attn.q")[2]
+    # flip one bit in the second checksum block of that container
+    raw = bytearray(path.read_bytes())
+    pos = off + block + 1234
+    assert pos < off + size
+    raw[pos] ^= 0x04
+    path.write_bytes(bytes(raw))
+    with archive.Archive(str(path)) as a:
+        assert a.verify("blk.0.attn.q") == [1]
+        with pytest.raises(ValueError):
+            a.load("blk.0.attn.q")
+        with pytest.raises(ValueError):
+            a.load_all()
+        # the other entries are untouched
+        got = a.load("h16")
+        assert np.array_equal(gu.to_bits(got).reshape(-1), ts["h16"][0])
