@@ -12,18 +12,25 @@
 //     raw(A B) = raw(A) * x^(8|B|) + raw(B)          (mod G, over GF(2)),
 // while the CRC proper is  ~( raw(M) + 0xFFFFFFFF * x^(8|M|) ).
 //
-// Work split.  One CTA (512 threads) per block at a time, grid-strided over
-// the blocks; thread t takes the t-th of 512 equal contiguous segments of the
-// block (block_bytes / 512 bytes, a multiple of 16), computes raw() of it with
-// 4-byte slicing tables, multiplies it by x^(8 * bytes after the segment) and
-// the CTA xors the 512 products.  For full blocks the multiplier of each
-// thread is the same in every block and is computed once per launch.
+// Work split.  One CTA (16 warps) per block at a time, grid-strided over the
+// blocks.  Warp w owns the w-th sixteenth of the block; inside it lane l takes
+// the 16-byte pieces l, l+32, l+64, ... so that every warp load covers 512
+// contiguous bytes.  A lane keeps one running register over its pieces: the
+// next piece starts 512 bytes after the previous one began, so between pieces
+// the register jumps over 496 bytes (c -> c * x^(8*496), a linear map done
+// with four byte tables J_k) before the 16 bytes are fed in.  At the end each
+// lane multiplies its register by x^(8 * bytes after its last piece) and the
+// CTA xors the 512 products.  For full blocks that multiplier is the same in
+// every block and is computed once per launch; a block's ragged tail (< 16
+// bytes) is fed in byte by byte.
 //
 // Tables.  S_k[b] = raw(byte b followed by k zero bytes), k = 0..3, give one
 // 4-byte step:  r ^= w;  r = S_3[r0] ^ S_2[r1] ^ S_1[r2] ^ S_0[r3]  (ri the
-// bytes of r, r0 lowest).  Lookups are data-dependent, so the 4 KiB of
-// tables are held 32 times over in shared memory, entry (k, b) of lane l at
-// word ((k * 256 + b) * 32 + l): every lane reads its own bank.
+// bytes of r, r0 lowest); J_k[b] = (b << 8k) * x^(8*496).  Lookups are
+// data-dependent: the S tables are held 32 times over in shared memory,
+// entry (k, b) of lane l at word ((k * 256 + b) * 32 + l), so every lane
+// reads its own bank; the J tables (a quarter of the lookups) 16 times, lane
+// l reading copy l mod 16 (at most two lanes per bank).
 #include <cstdint>
 
 #include "wc.h"
@@ -32,13 +39,17 @@
 namespace wc {
 namespace {
 
-constexpr int kCrcThreads = 512;
+constexpr int kCrcWarps = 16;
+constexpr int kCrcThreads = 32 * kCrcWarps;
 constexpr uint32_t kGenReversed = 0xEDB88320u;
+constexpr uint32_t kJump = 512 - 16;  // bytes between one lane's pieces
 
 struct CrcSmem {
-  uint32_t rep[4 * 256 * 32];  // lane-replicated slicing tables, 128 KiB
-  uint32_t base[4 * 256];      // the tables once
-  uint32_t red[kCrcThreads / 32];
+  uint32_t srep[4 * 256 * 32];  // S tables, one copy per lane      128 KiB
+  uint32_t jrep[4 * 256 * 16];  // J tables, one copy per half-warp  64 KiB
+  uint32_t sbase[4 * 256];      // the tables once
+  uint32_t jbase[4 * 256];
+  uint32_t red[kCrcWarps];
 };
 
 extern __shared__ __align__(16) uint8_t crc_smem[];
@@ -66,99 +77,134 @@ __device__ uint32_t xpow8(uint64_t n) {
   return r;
 }
 
-// t = this lane's column of the replicated tables
-__device__ __forceinline__ uint32_t step4(uint32_t r, uint32_t w, const uint32_t *t) {
+__device__ __forceinline__ uint32_t byte_of(uint32_t r, int k) {
+  return __byte_perm(r, 0u, 0x4440u + uint32_t(k));
+}
+
+// one 4-byte step; s = this lane's column of the S copies
+__device__ __forceinline__ uint32_t step4(uint32_t r, uint32_t w, const uint32_t *s) {
   r ^= w;
-  return t[(768u + (r & 0xFFu)) << 5] ^ t[(512u + ((r >> 8) & 0xFFu)) << 5] ^
-         t[(256u + ((r >> 16) & 0xFFu)) << 5] ^ t[(r >> 24) << 5];
+  return s[(768u + byte_of(r, 0)) << 5] ^ s[(512u + byte_of(r, 1)) << 5] ^
+         s[(256u + byte_of(r, 2)) << 5] ^ s[byte_of(r, 3) << 5];
 }
 
-__device__ __forceinline__ uint32_t step16(uint32_t r, uint4 v, const uint32_t *t) {
-  r = step4(r, v.x, t);
-  r = step4(r, v.y, t);
-  r = step4(r, v.z, t);
-  return step4(r, v.w, t);
+// c * x^(8*496); j = this lane's column of the J copies
+__device__ __forceinline__ uint32_t jump(uint32_t c, const uint32_t *j) {
+  return j[byte_of(c, 0) << 4] ^ j[(256u + byte_of(c, 1)) << 4] ^
+         j[(512u + byte_of(c, 2)) << 4] ^ j[(768u + byte_of(c, 3)) << 4];
 }
 
-// raw() of n bytes at p (p 16-byte aligned)
-__device__ uint32_t raw_segment(const uint8_t *p, uint64_t n, const uint32_t *t) {
-  const uint4 *q = reinterpret_cast<const uint4 *>(p);
-  const uint64_t n16 = n >> 4, groups = n16 >> 2;
-  uint32_t r = 0;
+__device__ __forceinline__ uint32_t piece(uint32_t c, uint4 v, const uint32_t *s, const uint32_t *j) {
+  c = jump(c, j);
+  c = step4(c, v.x, s);
+  c = step4(c, v.y, s);
+  c = step4(c, v.z, s);
+  return step4(c, v.w, s);
+}
+
+// The register over this lane's `cnt` pieces; q = its first piece, the
+// others 32 uint4 apart.
+__device__ uint32_t lane_chain(const uint4 *q, uint32_t cnt, const uint32_t *s, const uint32_t *j) {
+  uint32_t c = 0;
+  const uint32_t groups = cnt >> 2;
   if (groups) {
-    // 64 bytes in registers while the next 64 are on their way
-    uint4 c0 = __ldg(q), c1 = __ldg(q + 1), c2 = __ldg(q + 2), c3 = __ldg(q + 3);
-    for (uint64_t g = 1; g < groups; g++) {
-      const uint4 *qg = q + 4 * g;
-      const uint4 d0 = __ldg(qg), d1 = __ldg(qg + 1), d2 = __ldg(qg + 2), d3 = __ldg(qg + 3);
-      r = step16(r, c0, t);
-      r = step16(r, c1, t);
-      r = step16(r, c2, t);
-      r = step16(r, c3, t);
-      c0 = d0;
-      c1 = d1;
-      c2 = d2;
-      c3 = d3;
+    // four pieces in registers while the next four are on their way
+    uint4 a0 = __ldg(q), a1 = __ldg(q + 32), a2 = __ldg(q + 64), a3 = __ldg(q + 96);
+    for (uint32_t g = 1; g < groups; g++) {
+      const uint4 *qg = q + 128 * g;
+      const uint4 b0 = __ldg(qg), b1 = __ldg(qg + 32), b2 = __ldg(qg + 64), b3 = __ldg(qg + 96);
+      c = piece(c, a0, s, j);
+      c = piece(c, a1, s, j);
+      c = piece(c, a2, s, j);
+      c = piece(c, a3, s, j);
+      a0 = b0;
+      a1 = b1;
+      a2 = b2;
+      a3 = b3;
     }
-    r = step16(r, c0, t);
-    r = step16(r, c1, t);
-    r = step16(r, c2, t);
-    r = step16(r, c3, t);
+    c = piece(c, a0, s, j);
+    c = piece(c, a1, s, j);
+    c = piece(c, a2, s, j);
+    c = piece(c, a3, s, j);
   }
-  for (uint64_t i = groups * 4; i < n16; i++) r = step16(r, __ldg(q + i), t);
-  const uint8_t *b = p + (n16 << 4);
-  uint32_t rem = uint32_t(n & 15u);
-  for (; rem >= 4; rem -= 4, b += 4) r = step4(r, __ldg(reinterpret_cast<const uint32_t *>(b)), t);
-  for (; rem; rem--, b++) r = t[((r ^ __ldg(b)) & 0xFFu) << 5] ^ (r >> 8);
-  return r;
+  for (uint32_t i = groups * 4; i < cnt; i++) c = piece(c, __ldg(q + 32 * i), s, j);
+  return c;
 }
 
 __global__ void __launch_bounds__(kCrcThreads, 1)
 k_crc32(const uint8_t *__restrict__ buf, uint64_t bytes, uint64_t block_bytes,
         uint32_t *__restrict__ crc) {
-  CrcSmem &s = *reinterpret_cast<CrcSmem *>(crc_smem);
+  CrcSmem &sm = *reinterpret_cast<CrcSmem *>(crc_smem);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   if (tid < 256) {
     uint32_t r = uint32_t(tid);
     for (int i = 0; i < 8; i++) r = (r >> 1) ^ (kGenReversed & (0u - (r & 1u)));
-    s.base[tid] = r;
+    sm.sbase[tid] = r;
+  }
+  {
+    const uint32_t x496 = xpow8(kJump);
+    for (int i = tid; i < 1024; i += kCrcThreads)
+      sm.jbase[i] = gf_mul(uint32_t(i & 255) << (8 * (i >> 8)), x496);
   }
   __syncthreads();
   if (tid < 256) {
-    uint32_t r = s.base[tid];
+    uint32_t r = sm.sbase[tid];
     for (int k = 1; k < 4; k++) {
-      r = s.base[r & 0xFFu] ^ (r >> 8);  // one more zero byte
-      s.base[k * 256 + tid] = r;
+      r = sm.sbase[r & 0xFFu] ^ (r >> 8);  // one more zero byte
+      sm.sbase[k * 256 + tid] = r;
     }
   }
   __syncthreads();
-  for (int i = tid; i < 4 * 256 * 32; i += kCrcThreads) s.rep[i] = s.base[i >> 5];
+  for (int i = tid; i < 4 * 256 * 32; i += kCrcThreads) sm.srep[i] = sm.sbase[i >> 5];
+  for (int i = tid; i < 4 * 256 * 16; i += kCrcThreads) sm.jrep[i] = sm.jbase[i >> 4];
   __syncthreads();
 
-  const uint32_t *t = s.rep + lane;
+  const uint32_t *s = sm.srep + lane;
+  const uint32_t *j = sm.jrep + (lane & 15);
   const uint64_t nblocks = (bytes + block_bytes - 1) / block_bytes;
-  const uint64_t seg = block_bytes / kCrcThreads;
-  // full blocks: what follows thread tid's segment, and the preset's image
-  const uint32_t mul_full = xpow8(uint64_t(kCrcThreads - 1 - tid) * seg);
+  const uint64_t region = block_bytes / kCrcWarps;  // a multiple of 512
+  const uint32_t cnt_full = uint32_t(region / 512);
+  // full blocks: bytes after this lane's last piece, and the preset's image
+  const uint32_t mul_full =
+      xpow8(block_bytes - uint64_t(warp + 1) * region + 16u * uint32_t(31 - lane));
   const uint32_t preset_full = gf_mul(0xFFFFFFFFu, xpow8(block_bytes));
 
   for (uint64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
     const uint64_t start = blk * block_bytes;
     const uint64_t len = bytes - start < block_bytes ? bytes - start : block_bytes;
-    const uint64_t s0 = uint64_t(tid) * seg < len ? uint64_t(tid) * seg : len;
-    const uint64_t s1 = s0 + seg < len ? s0 + seg : len;
-    const uint32_t r = raw_segment(buf + start + s0, s1 - s0, t);
+    const uint64_t r0 = uint64_t(warp) * region;
+    const uint8_t *rb = buf + start + r0;
     uint32_t part = 0;
-    if (r != 0) part = gf_mul(r, len == block_bytes ? mul_full : xpow8(len - s1));
+    if (len == block_bytes) {
+      const uint32_t c = lane_chain(reinterpret_cast<const uint4 *>(rb) + lane, cnt_full, s, j);
+      if (c) part = gf_mul(c, mul_full);
+    } else if (len > r0) {
+      // the ragged block: this warp's share may be short or end in a tail
+      const uint64_t rlen = len - r0 < region ? len - r0 : region;
+      const uint32_t np = uint32_t(rlen >> 4);
+      const uint32_t cnt = np > uint32_t(lane) ? (np - uint32_t(lane) + 31) / 32 : 0;
+      if (cnt) {
+        const uint32_t c = lane_chain(reinterpret_cast<const uint4 *>(rb) + lane, cnt, s, j);
+        const uint64_t end = r0 + 16u * (uint64_t(lane) + 32u * (cnt - 1) + 1);
+        if (c) part = gf_mul(c, xpow8(len - end));
+      }
+      const uint32_t tail = uint32_t(rlen & 15u);
+      if (tail && lane == 0) {
+        uint32_t c = 0;
+        for (uint32_t i = 0; i < tail; i++)
+          c = s[((c ^ __ldg(rb + 16u * np + i)) & 0xFFu) << 5] ^ (c >> 8);
+        part ^= gf_mul(c, xpow8(len - (r0 + rlen)));
+      }
+    }
 #pragma unroll
     for (int o = 16; o; o >>= 1) part ^= __shfl_xor_sync(0xFFFFFFFFu, part, o);
-    if (lane == 0) s.red[warp] = part;
+    if (lane == 0) sm.red[warp] = part;
     __syncthreads();
     if (tid == 0) {
       uint32_t x = 0;
 #pragma unroll
-      for (int w = 0; w < kCrcThreads / 32; w++) x ^= s.red[w];
+      for (int w = 0; w < kCrcWarps; w++) x ^= sm.red[w];
       const uint32_t preset = len == block_bytes ? preset_full : gf_mul(0xFFFFFFFFu, xpow8(len));
       crc[blk] = ~(x ^ preset);
     }
