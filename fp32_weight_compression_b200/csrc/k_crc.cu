@@ -15,18 +15,19 @@
 // Work split.  One CTA (16 warps) per block at a time, grid-strided over the
 // blocks.  Warp w owns the w-th sixteenth of the block; inside it lane l takes
 // the 16-byte pieces l, l+32, l+64, ... so that every warp load covers 512
-// contiguous bytes.  A lane keeps one running register over its pieces: the
-// next piece starts 512 bytes after the previous one began, so between pieces
-// the register jumps over 496 bytes (c -> c * x^(8*496), a linear map done
-// with four byte tables J_k) before the 16 bytes are fed in.  At the end each
-// lane multiplies its register by x^(8 * bytes after its last piece) and the
-// CTA xors the 512 products.  For full blocks that multiplier is the same in
-// every block and is computed once per launch; a block's ragged tail (< 16
-// bytes) is fed in byte by byte.
+// contiguous bytes.  A lane keeps two running registers, one over its even
+// and one over its odd pieces (two independent chains of lookups in flight):
+// the next piece of a chain starts 1024 bytes after the previous one began,
+// so between pieces the register jumps over 1008 bytes (c -> c * x^(8*1008),
+// a linear map done with four byte tables J_k) before the 16 bytes are fed
+// in.  At the end each register is multiplied by x^(8 * bytes after its last
+// piece) and the CTA xors the 1024 products.  For full blocks those
+// multipliers are the same in every block and are computed once per launch;
+// a block's ragged tail (< 16 bytes) is fed in byte by byte.
 //
 // Tables.  S_k[b] = raw(byte b followed by k zero bytes), k = 0..3, give one
 // 4-byte step:  r ^= w;  r = S_3[r0] ^ S_2[r1] ^ S_1[r2] ^ S_0[r3]  (ri the
-// bytes of r, r0 lowest); J_k[b] = (b << 8k) * x^(8*496).  Lookups are
+// bytes of r, r0 lowest); J_k[b] = (b << 8k) * x^(8*1008).  Lookups are
 // data-dependent: the S tables are held 32 times over in shared memory,
 // entry (k, b) of lane l at word ((k * 256 + b) * 32 + l), so every lane
 // reads its own bank; the J tables (a quarter of the lookups) 16 times, lane
@@ -42,7 +43,7 @@ namespace {
 constexpr int kCrcWarps = 16;
 constexpr int kCrcThreads = 32 * kCrcWarps;
 constexpr uint32_t kGenReversed = 0xEDB88320u;
-constexpr uint32_t kJump = 512 - 16;  // bytes between one lane's pieces
+constexpr uint32_t kJump = 1024 - 16;  // bytes between two pieces of one chain
 
 struct CrcSmem {
   uint32_t srep[4 * 256 * 32];  // S tables, one copy per lane      128 KiB
@@ -88,7 +89,7 @@ __device__ __forceinline__ uint32_t step4(uint32_t r, uint32_t w, const uint32_t
          s[(256u + byte_of(r, 2)) << 5] ^ s[byte_of(r, 3) << 5];
 }
 
-// c * x^(8*496); j = this lane's column of the J copies
+// c * x^(8*1008); j = this lane's column of the J copies
 __device__ __forceinline__ uint32_t jump(uint32_t c, const uint32_t *j) {
   return j[byte_of(c, 0) << 4] ^ j[(256u + byte_of(c, 1)) << 4] ^
          j[(512u + byte_of(c, 2)) << 4] ^ j[(768u + byte_of(c, 3)) << 4];
@@ -102,10 +103,11 @@ __device__ __forceinline__ uint32_t piece(uint32_t c, uint4 v, const uint32_t *s
   return step4(c, v.w, s);
 }
 
-// The register over this lane's `cnt` pieces; q = its first piece, the
-// others 32 uint4 apart.
-__device__ uint32_t lane_chain(const uint4 *q, uint32_t cnt, const uint32_t *s, const uint32_t *j) {
-  uint32_t c = 0;
+// The two registers over this lane's `cnt` pieces (even ones into ca, odd
+// ones into cb); q = its first piece, the others 32 uint4 apart.
+__device__ void lane_chains(const uint4 *q, uint32_t cnt, const uint32_t *s, const uint32_t *j,
+                            uint32_t &ca, uint32_t &cb) {
+  uint32_t a = 0, b = 0;
   const uint32_t groups = cnt >> 2;
   if (groups) {
     // four pieces in registers while the next four are on their way
@@ -113,22 +115,37 @@ __device__ uint32_t lane_chain(const uint4 *q, uint32_t cnt, const uint32_t *s, 
     for (uint32_t g = 1; g < groups; g++) {
       const uint4 *qg = q + 128 * g;
       const uint4 b0 = __ldg(qg), b1 = __ldg(qg + 32), b2 = __ldg(qg + 64), b3 = __ldg(qg + 96);
-      c = piece(c, a0, s, j);
-      c = piece(c, a1, s, j);
-      c = piece(c, a2, s, j);
-      c = piece(c, a3, s, j);
+      a = piece(a, a0, s, j);
+      b = piece(b, a1, s, j);
+      a = piece(a, a2, s, j);
+      b = piece(b, a3, s, j);
       a0 = b0;
       a1 = b1;
       a2 = b2;
       a3 = b3;
     }
-    c = piece(c, a0, s, j);
-    c = piece(c, a1, s, j);
-    c = piece(c, a2, s, j);
-    c = piece(c, a3, s, j);
+    a = piece(a, a0, s, j);
+    b = piece(b, a1, s, j);
+    a = piece(a, a2, s, j);
+    b = piece(b, a3, s, j);
   }
-  for (uint32_t i = groups * 4; i < cnt; i++) c = piece(c, __ldg(q + 32 * i), s, j);
-  return c;
+  for (uint32_t i = groups * 4; i < cnt; i++) {
+    const uint4 v = __ldg(q + 32 * i);
+    if (i & 1u) b = piece(b, v, s, j);
+    else a = piece(a, v, s, j);
+  }
+  ca = a;
+  cb = b;
+}
+
+// Bytes of the lane's share of the region after the last piece of the chain
+// of parity `par` (region r0 + [0, 512 * cnt) of which the lane holds pieces
+// lane + 32 i, i < cnt), counted to `len`; ~0 when that chain is empty.
+__device__ __forceinline__ uint64_t after_last(uint64_t len, uint64_t r0, int lane, uint32_t cnt,
+                                               uint32_t par) {
+  if (cnt == 0 || (cnt == 1 && par == 1)) return ~uint64_t(0);
+  const uint32_t last = ((cnt - 1) & 1u) == par ? cnt - 1 : cnt - 2;
+  return len - (r0 + 16u * (uint64_t(lane) + 32u * uint64_t(last) + 1u));
 }
 
 __global__ void __launch_bounds__(kCrcThreads, 1)
@@ -165,29 +182,34 @@ k_crc32(const uint8_t *__restrict__ buf, uint64_t bytes, uint64_t block_bytes,
   const uint64_t nblocks = (bytes + block_bytes - 1) / block_bytes;
   const uint64_t region = block_bytes / kCrcWarps;  // a multiple of 512
   const uint32_t cnt_full = uint32_t(region / 512);
-  // full blocks: bytes after this lane's last piece, and the preset's image
-  const uint32_t mul_full =
-      xpow8(block_bytes - uint64_t(warp + 1) * region + 16u * uint32_t(31 - lane));
+  // full blocks: bytes after each chain's last piece, and the preset's image
+  const uint64_t r0 = uint64_t(warp) * region;
+  const uint64_t da = after_last(block_bytes, r0, lane, cnt_full, 0);
+  const uint64_t db = after_last(block_bytes, r0, lane, cnt_full, 1);
+  const uint32_t mul_a = xpow8(da);
+  const uint32_t mul_b = db == ~uint64_t(0) ? 0u : xpow8(db);
   const uint32_t preset_full = gf_mul(0xFFFFFFFFu, xpow8(block_bytes));
 
   for (uint64_t blk = blockIdx.x; blk < nblocks; blk += gridDim.x) {
     const uint64_t start = blk * block_bytes;
     const uint64_t len = bytes - start < block_bytes ? bytes - start : block_bytes;
-    const uint64_t r0 = uint64_t(warp) * region;
     const uint8_t *rb = buf + start + r0;
     uint32_t part = 0;
     if (len == block_bytes) {
-      const uint32_t c = lane_chain(reinterpret_cast<const uint4 *>(rb) + lane, cnt_full, s, j);
-      if (c) part = gf_mul(c, mul_full);
+      uint32_t ca, cb;
+      lane_chains(reinterpret_cast<const uint4 *>(rb) + lane, cnt_full, s, j, ca, cb);
+      if (ca) part = gf_mul(ca, mul_a);
+      if (cb) part ^= gf_mul(cb, mul_b);
     } else if (len > r0) {
       // the ragged block: this warp's share may be short or end in a tail
       const uint64_t rlen = len - r0 < region ? len - r0 : region;
       const uint32_t np = uint32_t(rlen >> 4);
       const uint32_t cnt = np > uint32_t(lane) ? (np - uint32_t(lane) + 31) / 32 : 0;
       if (cnt) {
-        const uint32_t c = lane_chain(reinterpret_cast<const uint4 *>(rb) + lane, cnt, s, j);
-        const uint64_t end = r0 + 16u * (uint64_t(lane) + 32u * (cnt - 1) + 1);
-        if (c) part = gf_mul(c, xpow8(len - end));
+        uint32_t ca, cb;
+        lane_chains(reinterpret_cast<const uint4 *>(rb) + lane, cnt, s, j, ca, cb);
+        if (ca) part = gf_mul(ca, xpow8(after_last(len, r0, lane, cnt, 0)));
+        if (cb) part ^= gf_mul(cb, xpow8(after_last(len, r0, lane, cnt, 1)));
       }
       const uint32_t tail = uint32_t(rlen & 15u);
       if (tail && lane == 0) {
