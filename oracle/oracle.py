@@ -22,8 +22,9 @@ SRC = os.path.join(HERE, "wc_oracle.c")
 LIB = os.path.join(HERE, "liboracle.so")
 
 OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CORRUPT = 0, 1, 2, 4
-BF16, FP32, FP16, FP8E4M3 = 1, 2, 3, 4
-_NP = {BF16: np.uint16, FP32: np.uint32, FP16: np.uint16, FP8E4M3: np.uint8}
+BF16, FP32, FP16, FP8E4M3, FP8E5M2, BF16_HIGHBYTE = 1, 2, 3, 4, 5, 6
+_NP = {BF16: np.uint16, FP32: np.uint32, FP16: np.uint16, FP8E4M3: np.uint8,
+       FP8E5M2: np.uint8, BF16_HIGHBYTE: np.uint16}
 CHUNK = 65536
 
 
@@ -60,6 +61,8 @@ def lib():
         L.oracle_split_fp32.argtypes = [vp, ctypes.c_uint64, vp, vp, vp]
         L.oracle_split_fp16.argtypes = [vp, ctypes.c_uint64, vp, vp]
         L.oracle_split_fp8e4m3.argtypes = [vp, ctypes.c_uint64, vp, vp]
+        L.oracle_split_fp8e5m2.argtypes = [vp, ctypes.c_uint64, vp, vp]
+        L.oracle_split_bf16_highbyte.argtypes = [vp, ctypes.c_uint64, vp, vp]
         L.oracle_histogram.argtypes = [vp, ctypes.c_uint64, vp]
         L.oracle_normalize.argtypes = [vp, vp]
         L.oracle_rans_encode.argtypes = [vp, ctypes.c_uint32, vp, ctypes.c_uint32, vp, vp, u32p]
@@ -136,6 +139,24 @@ def split_fp8e4m3(bits: np.ndarray):
     return e, nib
 
 
+def split_fp8e5m2(bits: np.ndarray):
+    """(high-nibble plane, packed low-nibble plane) of fp8 e5m2 bits (uint8)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint8).reshape(-1)
+    hi = np.zeros(bits.size, np.uint8)
+    nib = np.zeros((bits.size + 1) // 2, np.uint8)
+    lib().oracle_split_fp8e5m2(_ptr(bits), bits.size, _ptr(hi), _ptr(nib) if nib.size else None)
+    return hi, nib
+
+
+def split_bf16_highbyte(bits: np.ndarray):
+    """(high-byte plane, low-byte plane) of bf16 bits (uint16), no reorder."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16).reshape(-1)
+    hi = np.zeros(bits.size, np.uint8)
+    lo = np.zeros(bits.size, np.uint8)
+    lib().oracle_split_bf16_highbyte(_ptr(bits), bits.size, _ptr(hi), _ptr(lo))
+    return hi, lo
+
+
 def split_fp32(bits: np.ndarray):
     bits = np.ascontiguousarray(bits, dtype=np.uint32)
     n = bits.size
@@ -197,7 +218,8 @@ def rans_decode(states, words, nsym: int, freq, lanes: int = 32):
 
 def encode(bits: np.ndarray, dtype: int | None = None) -> np.ndarray:
     """Container bytes for a flat array of bf16 (uint16) or fp32 (uint32) bits,
-    or fp16 values (float16, or uint16 bits with dtype=FP16)."""
+    fp16 values (float16, or uint16 bits with dtype=FP16), fp8 bits (uint8:
+    e4m3 unless dtype=FP8E5M2), or bf16 bits with dtype=BF16_HIGHBYTE."""
     bits = np.ascontiguousarray(bits).reshape(-1)
     dt = dtype_code(bits) if dtype is None else dtype
     if dt == FP16:

@@ -128,11 +128,11 @@ static void or_make_layout(uint64_t n, int dtype, or_layout *lay) {
     lay->off_chunk_off = OR_CHUNK_OFF_OFFSET;
     lay->off_chunk_len = lay->off_chunk_off + 8 * (lay->nc + 1);
     lay->off_raw = round_up16(lay->off_chunk_len + 4 * lay->nc);
-    if (dtype == OR_BF16 || dtype == OR_FP16) {
+    if (dtype == OR_BF16 || dtype == OR_FP16 || dtype == OR_BF16_HIGHBYTE) {
         lay->off_sign = 0;
         lay->off_mant = 0;
         lay->off_exp = round_up16(lay->off_raw + n);
-    } else if (dtype == OR_FP8E4M3) {
+    } else if (dtype == OR_FP8E4M3 || dtype == OR_FP8E5M2) {
         lay->off_sign = 0;
         lay->off_mant = 0;
         lay->off_exp = round_up16(lay->off_raw + (n + 1) / 2);
@@ -150,12 +150,13 @@ static uint32_t or_chunk_nsym(uint64_t n, uint64_t k) {
 }
 
 static int or_dtype_ok(int dtype) {
-    return dtype == OR_BF16 || dtype == OR_FP32 || dtype == OR_FP16 || dtype == OR_FP8E4M3;
+    return dtype == OR_BF16 || dtype == OR_FP32 || dtype == OR_FP16 || dtype == OR_FP8E4M3 ||
+           dtype == OR_FP8E5M2 || dtype == OR_BF16_HIGHBYTE;
 }
 
 /* Bytes per value of a dtype. */
 static uint64_t or_elem(int dtype) {
-    return dtype == OR_FP32 ? 4 : (dtype == OR_FP8E4M3 ? 1 : 2);
+    return dtype == OR_FP32 ? 4 : (dtype == OR_FP8E4M3 || dtype == OR_FP8E5M2 ? 1 : 2);
 }
 
 uint64_t oracle_encode_bound(uint64_t n, int dtype) {
@@ -235,6 +236,37 @@ void oracle_split_fp8e4m3(const uint8_t *in, uint64_t n, uint8_t *exp_plane,
         exp_plane[i] = (uint8_t)(r >> 4);
         uint8_t lo = (uint8_t)(r & 0xFu);
         nibble_plane[i / 2] = (uint8_t)(nibble_plane[i / 2] | (i % 2 ? lo << 4 : lo));
+    }
+}
+
+/* fp8 e5m2 bits b = [S:1][E:5][M:2].  The same reorder gives E<<3 | S<<2 | M:
+ * the five exponent bits on top.  The nibble split then takes the high nibble
+ * (the top four exponent bits; coded) and the low nibble (lowest exponent bit,
+ * sign, two mantissa bits; raw), packed as for e4m3. */
+void oracle_split_fp8e5m2(const uint8_t *in, uint64_t n, uint8_t *hi_nibbles,
+                          uint8_t *nibble_plane) {
+    for (uint64_t i = 0; i < n; i++) {
+        uint8_t b = in[i];
+        uint8_t sign = (uint8_t)((b >> 7) & 1u);
+        uint8_t expo = (uint8_t)((b >> 2) & 0x1Fu);
+        uint8_t mant = (uint8_t)(b & 3u);
+        uint8_t r = (uint8_t)((expo << 3) | (sign << 2) | mant);
+        hi_nibbles[i] = (uint8_t)(r >> 4);
+        uint8_t lo = (uint8_t)(r & 0xFu);
+        nibble_plane[i / 2] = (uint8_t)(nibble_plane[i / 2] | (i % 2 ? lo << 4 : lo));
+    }
+}
+
+/* bf16 bits cut into bytes as they are, no reorder: the high byte (sign and
+ * the top seven exponent bits) is coded, the low byte (lowest exponent bit
+ * and the mantissa) is stored raw ("weight-compression" README: Split12
+ * splits bf16 into bytes, rebuilds the high byte from a codebook and keeps the
+ * low byte raw). */
+void oracle_split_bf16_highbyte(const uint16_t *in, uint64_t n, uint8_t *hi_plane,
+                                uint8_t *lo_plane) {
+    for (uint64_t i = 0; i < n; i++) {
+        hi_plane[i] = (uint8_t)(in[i] >> 8);
+        lo_plane[i] = (uint8_t)(in[i] & 0xFFu);
     }
 }
 
@@ -491,6 +523,10 @@ int oracle_encode(const void *in, uint64_t n, int dtype, uint8_t *out,
         oracle_split_fp16((const uint16_t *)in, n, expo, out + lay.off_raw);
     else if (dtype == OR_FP8E4M3)  /* the raw nibbles land in the zeroed section */
         oracle_split_fp8e4m3((const uint8_t *)in, n, expo, out + lay.off_raw);
+    else if (dtype == OR_FP8E5M2)
+        oracle_split_fp8e5m2((const uint8_t *)in, n, expo, out + lay.off_raw);
+    else if (dtype == OR_BF16_HIGHBYTE)
+        oracle_split_bf16_highbyte((const uint16_t *)in, n, expo, out + lay.off_raw);
     else
         oracle_split_fp32((const uint32_t *)in, n, expo, out + lay.off_sign,
                           out + lay.off_mant);
@@ -662,6 +698,15 @@ static int or_decode_one_chunk(const uint8_t *c, const or_header *h, uint64_t k,
             uint8_t sign = (uint8_t)((r >> 3) & 1u);
             uint8_t mant = (uint8_t)(r & 7u);
             ((uint8_t *)out_vals)[j] = (uint8_t)((sign << 7) | (e4 << 3) | mant);
+        } else if (h->dtype == OR_FP8E5M2) {
+            uint8_t lo = (uint8_t)((c[h->lay.off_raw + i / 2] >> (i % 2 ? 4 : 0)) & 0xFu);
+            uint8_t r = (uint8_t)((expo[j] << 4) | lo);
+            uint8_t e5 = (uint8_t)(r >> 3);
+            uint8_t sign = (uint8_t)((r >> 2) & 1u);
+            uint8_t mant = (uint8_t)(r & 3u);
+            ((uint8_t *)out_vals)[j] = (uint8_t)((sign << 7) | (e5 << 2) | mant);
+        } else if (h->dtype == OR_BF16_HIGHBYTE) {
+            ((uint16_t *)out_vals)[j] = (uint16_t)(((uint16_t)expo[j] << 8) | c[h->lay.off_raw + i]);
         } else {
             uint32_t sign = (c[h->lay.off_sign + i / 8] >> (i % 8)) & 1u;
             const uint8_t *m = c + h->lay.off_mant + 3 * i;

@@ -26,7 +26,11 @@ enum {
     OR_ERR_CORRUPT = 4
 };
 
-enum { OR_BF16 = 1, OR_FP32 = 2, OR_FP16 = 3, OR_FP8E4M3 = 4 };
+/* 5: fp8 e5m2; 6: bf16 split into its bytes without the reorder (the high
+ * byte S E7..E1 coded, the low byte E0 M7 raw): the Split12 split, kept as a
+ * comparison against the reorder. */
+enum { OR_BF16 = 1, OR_FP32 = 2, OR_FP16 = 3, OR_FP8E4M3 = 4, OR_FP8E5M2 = 5,
+       OR_BF16_HIGHBYTE = 6 };
 
 /* Worst-case container size (every chunk stored raw). */
 uint64_t oracle_encode_bound(uint64_t n, int dtype);
@@ -40,6 +44,10 @@ void oracle_split_fp16(const uint16_t *in, uint64_t n, uint8_t *hi_plane,
                        uint8_t *lo_plane);
 void oracle_split_fp8e4m3(const uint8_t *in, uint64_t n, uint8_t *exp_plane,
                           uint8_t *nibble_plane);
+void oracle_split_fp8e5m2(const uint8_t *in, uint64_t n, uint8_t *hi_nibbles,
+                          uint8_t *nibble_plane);
+void oracle_split_bf16_highbyte(const uint16_t *in, uint64_t n, uint8_t *hi_plane,
+                                uint8_t *lo_plane);
 
 /* 256-bin count of an exponent plane. */
 void oracle_histogram(const uint8_t *exp_plane, uint64_t n, uint64_t counts[256]);

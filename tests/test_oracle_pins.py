@@ -257,7 +257,90 @@ def test_fp8e4m3_round_trips(orc):
             assert np.array_equal(orc.decode_chunk(c, k), v[k * 65536:(k + 1) * 65536])
 
 
+def test_split_fp8e5m2_worked(orc):
+    # fp8 e5m2 S E5 M2; reordered E5 S M2; high nibble (top four exponent bits)
+    # coded, low nibble (lowest exponent bit, sign, mantissa) raw
+    bits = np.array([0x3C, 0xBE, 0x7B, 0x01, 0x80], np.uint8)
+    hi, nib = orc.split_fp8e5m2(bits)
+    assert hi.tolist() == [7, 7, 15, 0, 0]
+    # low nibbles 8, 0xE, 3, 1, 4 -> bytes 0xE8, 0x13, 0x04
+    assert nib.tolist() == [0xE8, 0x13, 0x04]
+
+
+def test_split_fp8e5m2_plane_structure(orc):
+    rng = np.random.default_rng(17)
+    for n in (4096, 4097):
+        bits = rng.integers(0, 256, n, dtype=np.uint8)
+        hi, nib = orc.split_fp8e5m2(bits)
+        e5 = (bits >> 2) & 0x1F
+        assert np.array_equal(hi, e5 >> 1)
+        lo = ((e5 & 1) << 3) | ((bits >> 7) << 2) | (bits & 3)
+        padded = np.zeros(2 * nib.size, np.uint8)
+        padded[:n] = lo
+        assert np.array_equal(nib, padded[0::2] | (padded[1::2] << 4))
+
+
+def test_fp8e5m2_round_trips(orc):
+    pats = np.arange(256, dtype=np.uint8)
+    cont = orc.encode(pats, dtype=orc.FP8E5M2)
+    assert orc.read_header(cont) == (256, orc.FP8E5M2, 1)
+    assert np.array_equal(orc.decode(cont), pats)
+    rng = np.random.default_rng(18)
+    e = np.clip(rng.normal(13, 1.5, 3 * 65536 + 7), 0, 31).astype(np.int64)
+    vals = ((rng.integers(0, 2, e.size) << 7) | (e << 2) | rng.integers(0, 4, e.size)).astype(np.uint8)
+    vals[rng.choice(vals.size, 256, replace=False)] = pats
+    cont = orc.encode(vals, dtype=orc.FP8E5M2)
+    assert np.array_equal(orc.decode(cont), vals)
+    assert cont.size < vals.nbytes
+    for n in (0, 1, 2, 3, 33, 65537):
+        v = vals[:n]
+        c = orc.encode(v, dtype=orc.FP8E5M2)
+        assert np.array_equal(orc.decode(c), v)
+        for k in range((n + 65535) // 65536):
+            assert np.array_equal(orc.decode_chunk(c, k), v[k * 65536:(k + 1) * 65536])
+
+
+def test_split_bf16_highbyte_worked(orc):
+    bits = np.array([0x3F80, 0xBF00, 0x0001, 0x7F80], np.uint16)
+    hi, lo = orc.split_bf16_highbyte(bits)
+    assert hi.tolist() == [0x3F, 0xBF, 0x00, 0x7F]
+    assert lo.tolist() == [0x80, 0x00, 0x01, 0x80]
+
+
+def test_bf16_highbyte_round_trips(orc):
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    cont = orc.encode(bits, dtype=orc.BF16_HIGHBYTE)
+    assert orc.read_header(cont) == (1 << 16, orc.BF16_HIGHBYTE, 1)
+    assert np.array_equal(orc.decode(cont), bits)
+    x = np.random.default_rng(19).standard_normal(3 * 65536 + 5).astype(np.float32) * np.float32(0.02)
+    import workloads
+    b = workloads.rne_bf16(x)
+    cont = orc.encode(b, dtype=orc.BF16_HIGHBYTE)
+    assert np.array_equal(orc.decode(cont), b)
+    assert np.array_equal(orc.decode_chunk(cont, 3), b[3 * 65536:])
+    # the coded plane is the high byte: same values, same table as counting
+    # the high bytes directly
+    hi, _ = orc.split_bf16_highbyte(b)
+    assert np.array_equal(orc.histogram(hi), np.bincount(b >> 8, minlength=256))
+
+
 # ---------------------------------------------------------------- containers
+def test_golden_container_fp8e5m2_raw_chunk(orc):
+    bits = np.array([0x3C, 0x3C, 0x3C, 0x38], np.uint8)
+    want = load_container("container_fp8e5m2_n4_raw.txt")
+    got = orc.encode(bits, dtype=orc.FP8E5M2)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert orc.decode(got).tolist() == bits.tolist()
+
+
+def test_golden_container_bf16_highbyte_raw_chunk(orc):
+    bits = np.array([0x3F80, 0x3F80, 0x3F80, 0x3F00], np.uint16)
+    want = load_container("container_bf16_highbyte_n4_raw.txt")
+    got = orc.encode(bits, dtype=orc.BF16_HIGHBYTE)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert orc.decode(got).tolist() == bits.tolist()
+
+
 def test_golden_container_fp8e4m3_raw_chunk(orc):
     bits = np.array([0x38, 0x38, 0x38, 0x30], np.uint8)
     want = load_container("container_fp8e4m3_n4_raw.txt")

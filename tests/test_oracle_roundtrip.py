@@ -134,7 +134,7 @@ def test_corrupt_header_fields(orc):
     cases = []
     c = good.copy(); c[0] ^= 1; cases.append(c)                       # magic
     c = good.copy(); c[4] = 2; cases.append(c)                        # version
-    c = good.copy(); c[6] = 5; cases.append(c)                        # dtype (unknown)
+    c = good.copy(); c[6] = 7; cases.append(c)                        # dtype (unknown)
     c = good.copy(); c[7] = 16; cases.append(c)                       # lanes
     c = good.copy(); _field(c, 16, np.uint32)[0] = 4096; cases.append(c)
     c = good.copy(); _field(c, 24, np.uint16)[0] = 11; cases.append(c)
