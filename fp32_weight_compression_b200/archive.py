@@ -215,9 +215,31 @@ class Archive:
 
     def load_chunk(self, name: str, k: int, device="cuda", stream=None,
                    verify: bool = True) -> torch.Tensor:
-        """Values k * 65536 .. of one tensor (1-D), decoding that chunk only."""
-        code = self._entries[name][0]
-        cont = self._device_container(name, device, verify, stream)
+        """Values k * 65536 .. of one tensor (1-D), decoding that chunk only.
+        Only the bytes the chunk needs leave the file: the header and tables,
+        the chunk's raw-plane bytes and its payload (wc_chunk_ranges), widened
+        to whole checksum blocks when those are checked."""
+        code, _, off, nbytes, crcs = self._entries[name]
+        (off_raw,) = struct.unpack_from("<Q", self._mm, off + 32)
+        if off_raw > nbytes:
+            raise ValueError(f"entry {name!r}: container header out of range")
+        ranges = wc.chunk_ranges(bytes(self._mm[off:off + off_raw]), k)
+        check = verify and self.crc_block > 0
+        if check:
+            B = self.crc_block
+            blocks = sorted({b for o, n in ranges if n for b in range(o // B, (o + n - 1) // B + 1)})
+            ranges = [(b * B, min(B, nbytes - b * B)) for b in blocks]
+        cont = torch.zeros(nbytes, dtype=torch.uint8, device=device)
+        for o, n in ranges:
+            if o + n > nbytes:
+                raise ValueError(f"entry {name!r}: chunk {k} reaches past its container")
+            cont[o:o + n].copy_(torch.from_numpy(
+                np.frombuffer(self._mm, dtype=np.uint8, count=n, offset=off + o).copy()))
+        if check:
+            got = wc.crc32_blocks(cont, self.crc_block, stream).cpu().numpy().view(np.uint32)
+            bad = [b for b in blocks if got[b] != crcs[b]]
+            if bad:
+                raise ValueError(f"entry {name!r}: checksum mismatch in block(s) {bad[:8]}")
         return wc.decode_chunk(cont, k, dtype=wc._TORCH_DT[code], stream=stream)
 
     def load_all(self, names=None, device="cuda", stream=None, verify: bool = True) -> dict:

@@ -321,4 +321,41 @@ int32_t wc_read_header(const void *h_cont, uint64_t bytes, uint64_t *n, int32_t 
   return WC_OK;
 }
 
+int32_t wc_chunk_ranges(const void *h_prefix, uint64_t prefix_bytes, uint64_t k, uint64_t *ranges,
+                        uint32_t *count) {
+  if (h_prefix == nullptr || ranges == nullptr || count == nullptr) return WC_ERR_INVALID_ARG;
+  uint64_t n = 0, nc = 0;
+  int32_t dt = 0;
+  const int32_t st = wc_read_header(h_prefix, prefix_bytes, &n, &dt, &nc);
+  if (st != WC_OK) return st;
+  const wc::Layout L = wc::make_layout(n, dt);
+  // with the whole prefix present, wc_read_header has checked every table entry
+  if (prefix_bytes < L.off_raw) return WC_ERR_CAPACITY;
+  if (k >= nc) return WC_ERR_INVALID_ARG;
+  const uint8_t *c = static_cast<const uint8_t *>(h_prefix);
+  uint64_t choff = 0;
+  uint32_t len = 0;
+  memcpy(&choff, c + L.off_chunk_off + 8 * k, 8);
+  memcpy(&len, c + L.off_chunk_len + 4 * k, 4);
+  const uint64_t first = k * wc::kChunk, nsym = wc::chunk_nsym(n, k);
+  uint32_t m = 0;
+  auto put = [&](uint64_t off, uint64_t bytes) {
+    ranges[2 * m] = off;
+    ranges[2 * m + 1] = bytes;
+    m++;
+  };
+  put(0, L.off_raw);
+  if (dt == WC_FP32) {
+    put(L.off_raw + first / 8, (nsym + 7) / 8);
+    put(L.off_mant + 3 * first, 3 * nsym);
+  } else if (dt == WC_FP8E4M3) {
+    put(L.off_raw + first / 2, (nsym + 1) / 2);
+  } else {
+    put(L.off_raw + first, nsym);
+  }
+  put(L.off_exp + choff, wc::round16(len));
+  *count = m;
+  return WC_OK;
+}
+
 }  // extern "C"

@@ -110,6 +110,8 @@ def load() -> ctypes.CDLL:
     L.wc_decode_host.restype = i32
     L.wc_decode_host.argtypes = [ctypes.POINTER(HostDecodeItem), u32, vp, u64, u64, vp, vp, vp,
                                  ctypes.POINTER(i32)]
+    L.wc_chunk_ranges.restype = i32
+    L.wc_chunk_ranges.argtypes = [vp, u64, u64, ctypes.POINTER(u64), ctypes.POINTER(u32)]
     L.wc_crc32_blocks.restype = i32
     L.wc_crc32_blocks.argtypes = [vp, u64, u64, vp, vp]
     _lib = L
@@ -379,6 +381,20 @@ def decode_batch(conts, shapes, dtypes, stream=None) -> list[torch.Tensor]:
     dec.decode(conts, outs, stream=stream)
     dec.check()
     return outs
+
+
+def chunk_ranges(prefix, k: int) -> list[tuple[int, int]]:
+    """(offset, bytes) ranges of a container that decoding chunk k reads
+    (wc_chunk_ranges); `prefix` is a host copy of the container's start
+    (bytes or uint8 array) reaching at least the raw-plane offset."""
+    import numpy as np
+    buf = np.ascontiguousarray(np.frombuffer(prefix, np.uint8) if isinstance(prefix, (bytes, bytearray))
+                               else prefix, dtype=np.uint8)
+    out = (ctypes.c_uint64 * 8)()
+    cnt = ctypes.c_uint32(0)
+    _check(load().wc_chunk_ranges(buf.ctypes.data, buf.size, k, out, ctypes.byref(cnt)),
+           "wc_chunk_ranges")
+    return [(int(out[2 * i]), int(out[2 * i + 1])) for i in range(cnt.value)]
 
 
 CRC_BLOCK = 1 << 20

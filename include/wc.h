@@ -265,6 +265,24 @@ WC_API int32_t wc_decode_host(const wc_host_decode_item *h_items, uint32_t count
                               uint64_t work_cap, uint64_t window_bytes, void *stream_in,
                               void *stream_compute, void *stream_out, int32_t *h_status);
 
+/* The byte ranges of a container that wc_decode_chunk reads for chunk k:
+ * random access inside a stored tensor ("PTWM", Random access: a reader
+ * fetches what one tensor needs without reading the rest) can copy just these
+ * to the device and leave the rest of a container-sized buffer unwritten.
+ *   h_prefix      host copy of the container's first prefix_bytes bytes; it
+ *                 must reach the end of the tables, i.e. the raw-plane offset
+ *                 stored at header byte 32 (WC_ERR_CAPACITY otherwise).
+ *   k             the chunk (WC_ERR_INVALID_ARG if k >= nchunks).
+ *   ranges        host, 8 uint64: up to 4 {offset, bytes} pairs in ascending
+ *                 order, written for *count of them: the header and tables
+ *                 [0, raw-plane offset), the chunk's raw-plane bytes (two
+ *                 ranges for fp32: sign bits and mantissa bytes), and its
+ *                 exponent payload rounded up to 16 bytes.
+ * The header and chunk k's offset-table entries are checked as wc_read_header
+ * and the decoder check them (WC_ERR_CORRUPT).  Host only; no device work. */
+WC_API int32_t wc_chunk_ranges(const void *h_prefix, uint64_t prefix_bytes, uint64_t k,
+                               uint64_t *ranges, uint32_t *count);
+
 /* CRC-32 of fixed-size blocks of a device buffer, the per-block check that
  * an archive file keeps ("seedpack 0.2.0 -> 0.2.2", README: every chunk of an
  * archive carries a CRC32).  The code is zlib's and IEEE 802.3's CRC-32

@@ -107,3 +107,72 @@ def test_product_path_has_no_oracle_dependency():
                 for pat in ("import oracle", "from oracle", "liboracle", "wc_oracle",
                             "sys.path"):
                     assert pat not in text, (fn, pat)
+
+
+def _masked_to_ranges(cont, ranges):
+    keep = np.zeros_like(cont)
+    for off, size in ranges:
+        keep[off:off + size] = cont[off:off + size]
+    return keep
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp32", "fp16", "fp8"])
+def test_chunk_ranges_hold_all_a_chunk_needs(wcm, orc, dt):
+    """Every byte outside wc_chunk_ranges(k) zeroed: the oracle still decodes
+    chunk k exactly, so the ranges hold everything that chunk needs."""
+    rng = np.random.default_rng(31)
+    n = 3 * 65536 + 100       # the last chunk (100 values) is always stored raw
+    x = rng.standard_normal(n).astype(np.float32) * np.float32(0.02)
+    if dt == "bf16":
+        bits = workloads.rne_bf16(x)
+    elif dt == "fp32":
+        bits = x.view(np.uint32).copy()
+    elif dt == "fp16":
+        bits = x.astype(np.float16)
+    else:
+        e = np.clip(rng.normal(6, 1.3, n), 0, 15).astype(np.int64)
+        bits = ((rng.integers(0, 2, n) << 7) | (e << 3) | rng.integers(0, 8, n)).astype(np.uint8)
+    # random bits in chunk 1 (stored raw except for fp8, whose 16-symbol
+    # alphabet always codes below a byte per value)
+    bits[65536:2 * 65536] = np.frombuffer(rng.bytes(65536 * bits.itemsize), bits.dtype)
+    cont = orc.encode(bits)
+    off_raw = int(cont[32:40].view(np.uint64)[0])
+    raws = []
+    for k in range(4):
+        ranges = wcm.chunk_ranges(cont[:off_raw], k)
+        assert ranges[0] == (0, off_raw)
+        assert all(o % 16 == 0 or i > 0 for i, (o, _) in enumerate(ranges))
+        assert sum(s for _, s in ranges) < cont.size
+        part = _masked_to_ranges(cont, ranges)
+        want = bits.reshape(-1)[k * 65536:(k + 1) * 65536]
+        got = orc.decode_chunk(part, k)
+        assert np.array_equal(got.view(np.uint8), want.view(np.uint8)), k
+        # without any one of the data ranges the chunk no longer decodes
+        for drop in range(1, len(ranges)):
+            short = _masked_to_ranges(cont, ranges[:drop] + ranges[drop + 1:])
+            try:
+                bad = orc.decode_chunk(short, k)
+                assert not np.array_equal(bad.view(np.uint8), want.view(np.uint8)), (k, drop)
+            except orc.OracleError:
+                pass
+        n_, _, nc = orc.read_header(cont)
+        lens = cont[576 + 8 * (nc + 1): 576 + 8 * (nc + 1) + 4 * nc].view(np.uint32)
+        raws.append(int(lens[k]) == min(65536, n - k * 65536))
+    assert raws[3] and not raws[0] and raws[1] == (dt != "fp8")
+
+
+def test_chunk_ranges_rejects(wcm, orc):
+    bits = workloads.rne_bf16(np.random.default_rng(2).standard_normal(70000).astype(np.float32))
+    cont = orc.encode(bits)
+    off_raw = int(cont[32:40].view(np.uint64)[0])
+    with pytest.raises(wcm.WCError) as e:
+        wcm.chunk_ranges(cont[:off_raw - 1], 0)               # prefix short of the tables
+    assert e.value.code == wcm.ERR_CAPACITY
+    with pytest.raises(wcm.WCError) as e:
+        wcm.chunk_ranges(cont[:off_raw], 2)                   # only 2 chunks
+    assert e.value.code == wcm.ERR_INVALID_ARG
+    bad = cont[:off_raw].copy()
+    bad[576 + 8] ^= 0x10                                      # chunk_off[1] off by 16
+    with pytest.raises(wcm.WCError) as e:
+        wcm.chunk_ranges(bad, 0)
+    assert e.value.code == wcm.ERR_CORRUPT

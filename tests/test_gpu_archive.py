@@ -51,6 +51,9 @@ def test_save_load_bit_exact(orc, tmp_path):
         assert np.array_equal(gu.to_bits(part), ts["blk.0.attn.q"][0][C:2 * C])
         part = a.load_chunk("f8", 2)
         assert np.array_equal(gu.to_bits(part), ts["f8"][0][2 * C:])
+        for k in range(3):   # fp32 (sign-bit and mantissa ranges), and without checks
+            part = a.load_chunk("norm", k, verify=k != 1)
+            assert np.array_equal(gu.to_bits(part), ts["norm"][0][k * C:(k + 1) * C])
         allv = a.load_all()
         for k, (b, t) in ts.items():
             assert allv[k].dtype == t.dtype and tuple(allv[k].shape) == tuple(t.shape)
@@ -85,6 +88,12 @@ def test_checksums_catch_a_damaged_container(orc, tmp_path):
             a.load("blk.0.attn.q")
         with pytest.raises(ValueError):
             a.load_all()
+        # one chunk: its bytes include the damaged block (chunk 0's raw plane
+        # reaches into checksum block 1) or do not (chunk 2)
+        with pytest.raises(ValueError):
+            a.load_chunk("blk.0.attn.q", 0)
+        part = a.load_chunk("blk.0.attn.q", 2)
+        assert np.array_equal(gu.to_bits(part), ts["blk.0.attn.q"][0][2 * C:3 * C])
         # the other entries are untouched
         got = a.load("h16")
         assert np.array_equal(gu.to_bits(got).reshape(-1), ts["h16"][0])
