@@ -176,3 +176,37 @@ def test_chunk_ranges_rejects(wcm, orc):
     with pytest.raises(wcm.WCError) as e:
         wcm.chunk_ranges(bad, 0)
     assert e.value.code == wcm.ERR_CORRUPT
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp32", "fp16", "fp8"])
+def test_header_fuzz_agrees_with_oracle(wcm, orc, dt):
+    """Random byte flips in the header and tables: the library's host parser
+    (wc_read_header) and the oracle accept and reject the same containers and
+    read the same fields; where both accept, wc_chunk_ranges accepts too."""
+    rng = np.random.default_rng(["bf16", "fp32", "fp16", "fp8"].index(dt) + 40)
+    n = 3 * 65536 + 777
+    x = rng.standard_normal(n).astype(np.float32) * np.float32(0.02)
+    bits = {"bf16": lambda: workloads.rne_bf16(x), "fp32": lambda: x.view(np.uint32).copy(),
+            "fp16": lambda: x.astype(np.float16),
+            "fp8": lambda: (np.clip(rng.normal(6, 1.3, n), 0, 15).astype(np.uint8) << 3)}[dt]()
+    good = orc.encode(bits)
+    off_raw = int(good[32:40].view(np.uint64)[0])
+    both = 0
+    for _ in range(600):
+        c = good.copy()
+        for _ in range(int(rng.integers(1, 3))):
+            c[int(rng.integers(0, off_raw))] ^= np.uint8(rng.integers(1, 256))
+        try:
+            a = wcm.read_header(c)
+        except wcm.WCError:
+            a = None
+        try:
+            b = orc.read_header(c)
+        except orc.OracleError:
+            b = None
+        assert a == b
+        if a is not None:
+            both += 1
+            for k in range(a[2]):
+                wcm.chunk_ranges(c[:off_raw], k)
+    assert both < 600   # most flips must be caught
