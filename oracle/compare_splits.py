@@ -8,6 +8,8 @@ involved).  For each workload's bf16 tensors:
   high byte  dtype 6: bf16 cut into bytes as they are, high byte (sign and
              exponent bits 7..1) coded, low byte raw (the Split12 split of the
              "weight-compression" README)
+  split12    the Split12 codec itself (oracle/split12.py): a 4-bit index into
+             a 16-entry codebook of high bytes, the low byte raw, exceptions
 and, with the values scaled by 64 and rounded to fp8 (torch's CPU casts):
   e4m3       dtype 4: exponent nibble coded
   e5m2       dtype 5: top four exponent bits coded
@@ -29,6 +31,7 @@ sys.path.insert(0, HERE)
 sys.path.insert(0, os.path.dirname(HERE))
 
 import oracle  # noqa: E402
+import split12  # noqa: E402
 import workloads  # noqa: E402
 
 
@@ -57,7 +60,8 @@ def main() -> None:
         idx = list(range(len(specs)))
         if cid == 4:
             idx = idx[: 7 * args.layers]
-        tot = {k: 0 for k in ("in", "reorder", "highbyte", "in8", "e4m3", "e5m2")}
+        tot = {k: 0 for k in ("in", "reorder", "highbyte", "split12", "in8", "e4m3", "e5m2")}
+        n_exc = 0
         ent = {k: 0.0 for k in ("reorder", "highbyte", "e4m3", "e5m2")}
         nvals = 0
         for i in idx:
@@ -69,6 +73,9 @@ def main() -> None:
             tot["in"] += b.nbytes
             tot["reorder"] += oracle.encode(b).size
             tot["highbyte"] += oracle.encode(b, dtype=oracle.BF16_HIGHBYTE).size
+            c12 = split12.encode(b)
+            tot["split12"] += c12.size
+            n_exc += split12.read_header(c12)["ne"]
             ent["reorder"] += entropy_bits(oracle.split_bf16(b)[0]) * n
             ent["highbyte"] += entropy_bits(oracle.split_bf16_highbyte(b)[0]) * n
             for kind, code, split in (("e4m3", oracle.FP8E4M3, oracle.split_fp8e4m3),
@@ -84,6 +91,8 @@ def main() -> None:
               f"{ent['reorder'] / nvals:.3f} bits/value")
         print(f"  bf16 high byte  ratio {tot['highbyte'] / tot['in']:.4f}  coded plane "
               f"{ent['highbyte'] / nvals:.3f} bits/value")
+        print(f"  Split12 codec   ratio {tot['split12'] / tot['in']:.4f}  exceptions "
+              f"{100 * n_exc / nvals:.4f} % of values")
         print(f"  fp8 e4m3 (x64)  ratio {tot['e4m3'] / tot['in8']:.4f}  coded plane "
               f"{ent['e4m3'] / nvals:.3f} bits/value")
         print(f"  fp8 e5m2 (x64)  ratio {tot['e5m2'] / tot['in8']:.4f}  coded plane "

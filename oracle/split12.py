@@ -1,0 +1,162 @@
+"""Split12 weight format, stated plainly in numpy.
+
+TEST INFRASTRUCTURE ONLY: the slow reference for a bf16 format read from the
+"weight-compression" README (Split12: bf16 split into its two bytes, the high
+byte rebuilt from a codebook, the low byte kept raw; 24.967 % smaller on a
+753B model, i.e. 12 bits a value plus a little).  Only the tests, the smoke
+check and the benchmark's CPU leg may import it; the CUDA library never does.
+
+Reading (the page gives the idea, not the format):
+  * high byte h = b >> 8 (sign and exponent bits 7..1), low byte l = b & 0xFF;
+  * codebook: the K <= 16 most frequent high bytes of the tensor (ties to the
+    smaller byte), stored in ascending order;
+  * each value stores a 4-bit index into the codebook (value i in byte i // 2,
+    low nibble when i is even; 0 for a value whose high byte is not in the
+    codebook) and its low byte;
+  * values whose high byte is not in the codebook are exceptions, listed per
+    65,536-value chunk in ascending position: u16 position in the chunk and
+    the u8 high byte; a u32 offset table gives each chunk's first exception.
+
+Container (little-endian, sections 16-byte aligned, zero padding):
+    0   "W12C"  u16 version 1  u8 dtype 1 (bf16)  u8 K (codebook entries)
+    8   u64 n
+    16  u32 chunk values 65536  u32 nc = ceil(n / 65536)
+    24  u64 ne (exceptions)
+    32  u64 off_idx   40 u64 off_lo   48 u64 off_exc   56 u64 total bytes
+    64  u8 codebook[16] (entries >= K are 0)
+    80  u32 exc_off[nc + 1]
+    off_idx   ceil(n / 2) index bytes
+    off_lo    n low bytes
+    off_exc   u16 position[ne], then (16-aligned) u8 high byte[ne]
+"""
+from __future__ import annotations
+
+import numpy as np
+
+CHUNK = 65536
+MAGIC = b"W12C"
+HEADER = 64
+BOOK = 16
+
+
+def _r16(v: int) -> int:
+    return (v + 15) // 16 * 16
+
+
+def layout(n: int, ne: int) -> dict:
+    nc = -(-n // CHUNK)
+    off_excoff = HEADER + BOOK
+    off_idx = _r16(off_excoff + 4 * (nc + 1))
+    off_lo = _r16(off_idx + (n + 1) // 2)
+    off_exc = _r16(off_lo + n)
+    off_excval = off_exc + _r16(2 * ne)
+    total = off_excval + _r16(ne)
+    return dict(nc=nc, off_excoff=off_excoff, off_idx=off_idx, off_lo=off_lo,
+                off_exc=off_exc, off_excval=off_excval, total=total)
+
+
+def codebook(high: np.ndarray) -> np.ndarray:
+    """The up to 16 most frequent bytes of `high` (ties to the smaller byte),
+    ascending."""
+    counts = np.bincount(high, minlength=256)
+    ranked = sorted(range(256), key=lambda b: (-int(counts[b]), b))
+    chosen = [b for b in ranked[:BOOK] if counts[b] > 0]
+    return np.array(sorted(chosen), dtype=np.uint8)
+
+
+def encode(bits: np.ndarray) -> np.ndarray:
+    """Container bytes for bf16 bits (uint16)."""
+    bits = np.ascontiguousarray(bits, dtype=np.uint16).reshape(-1)
+    n = bits.size
+    high = (bits >> 8).astype(np.uint8)
+    low = (bits & 0xFF).astype(np.uint8)
+    book = codebook(high)
+    k = book.size
+    where = np.full(256, -1, np.int64)
+    where[book] = np.arange(k)
+    slot = where[high]
+    is_exc = slot < 0
+    idx = np.where(is_exc, 0, slot).astype(np.uint8)
+    pos = np.nonzero(is_exc)[0]                      # ascending
+    ne = pos.size
+    L = layout(n, ne)
+    # exceptions before the start of each chunk, and at the end
+    exc_off = np.searchsorted(pos, np.arange(L["nc"] + 1, dtype=np.int64) * CHUNK)
+    exc_off[-1] = ne
+    out = np.zeros(L["total"], np.uint8)
+    out[0:4] = np.frombuffer(MAGIC, np.uint8)
+    out[4:6] = np.array([1], "<u2").view(np.uint8)
+    out[6] = 1
+    out[7] = k
+    out[8:16] = np.array([n], "<u8").view(np.uint8)
+    out[16:24] = np.array([CHUNK, L["nc"]], "<u4").view(np.uint8)
+    out[24:32] = np.array([ne], "<u8").view(np.uint8)
+    out[32:64] = np.array([L["off_idx"], L["off_lo"], L["off_exc"], L["total"]], "<u8").view(np.uint8)
+    out[HEADER:HEADER + k] = book
+    o = L["off_excoff"]
+    out[o:o + 4 * (L["nc"] + 1)] = exc_off.astype("<u4").view(np.uint8)
+    padded = np.zeros(2 * ((n + 1) // 2), np.uint8)
+    padded[:n] = idx
+    out[L["off_idx"]:L["off_idx"] + padded.size // 2] = padded[0::2] | (padded[1::2] << 4)
+    out[L["off_lo"]:L["off_lo"] + n] = low
+    if ne:
+        out[L["off_exc"]:L["off_exc"] + 2 * ne] = (pos % CHUNK).astype("<u2").view(np.uint8)
+        out[L["off_excval"]:L["off_excval"] + ne] = high[pos]
+    return out
+
+
+def _u(c: np.ndarray, off: int, fmt: str) -> int:
+    return int(np.frombuffer(c[off:off + np.dtype(fmt).itemsize].tobytes(), fmt)[0])
+
+
+def read_header(cont: np.ndarray) -> dict:
+    c = np.ascontiguousarray(cont, dtype=np.uint8)
+    if c.size < HEADER + BOOK or c[:4].tobytes() != MAGIC or _u(c, 4, "<u2") != 1 or c[6] != 1:
+        raise ValueError("not a Split12 container")
+    n, ne = _u(c, 8, "<u8"), _u(c, 24, "<u8")
+    k = int(c[7])
+    L = layout(n, ne)
+    if (_u(c, 16, "<u4") != CHUNK or _u(c, 20, "<u4") != L["nc"] or not 0 <= k <= BOOK
+            or (n > 0) != (k > 0)):
+        raise ValueError("bad Split12 header")
+    if [_u(c, 32 + 8 * j, "<u8") for j in range(4)] != [L["off_idx"], L["off_lo"], L["off_exc"], L["total"]]:
+        raise ValueError("bad Split12 layout")
+    if c.size < L["total"]:
+        raise ValueError("Split12 container cut short")
+    return dict(n=n, ne=ne, k=k, **L)
+
+
+def decode(cont: np.ndarray) -> np.ndarray:
+    """bf16 bits (uint16) of a container; ValueError if it is not the one
+    container the format allows for some input."""
+    c = np.ascontiguousarray(cont, dtype=np.uint8)
+    h = read_header(c)
+    n, ne, k, nc = h["n"], h["ne"], h["k"], h["nc"]
+    book = c[HEADER:HEADER + BOOK]
+    if k and (np.any(np.diff(book[:k].astype(np.int64)) <= 0) or np.any(book[k:] != 0)):
+        raise ValueError("codebook not ascending or padded with non-zero bytes")
+    o = h["off_excoff"]
+    exc_off = c[o:o + 4 * (nc + 1)].view("<u4").astype(np.int64)
+    if exc_off[0] != 0 or exc_off[-1] != ne or np.any(np.diff(exc_off) < 0):
+        raise ValueError("bad Split12 exception table")
+    packed = c[h["off_idx"]:h["off_idx"] + (n + 1) // 2]
+    idx = np.empty(2 * packed.size, np.uint8)
+    idx[0::2] = packed & 0xF
+    idx[1::2] = packed >> 4
+    idx = idx[:n]
+    if np.any(idx >= max(k, 1)):
+        raise ValueError("codebook index out of range")
+    low = c[h["off_lo"]:h["off_lo"] + n].astype(np.uint16)
+    out = (book[idx].astype(np.uint16) << 8) | low
+    if ne:
+        chunk_of = np.repeat(np.arange(nc, dtype=np.int64), np.diff(exc_off))
+        pos = chunk_of * CHUNK + c[h["off_exc"]:h["off_exc"] + 2 * ne].view("<u2").astype(np.int64)
+        if np.any(np.diff(pos) <= 0) or pos[-1] >= n:
+            raise ValueError("bad Split12 exception position")
+        val = c[h["off_excval"]:h["off_excval"] + ne]
+        if np.any(idx[pos] != 0) or np.any(np.isin(val, book[:k])):
+            raise ValueError("exception not in canonical form")
+        out[pos] = (val.astype(np.uint16) << 8) | low[pos]
+    if not np.array_equal(codebook((out >> 8).astype(np.uint8)), book[:k]):
+        raise ValueError("codebook is not the values' most frequent high bytes")
+    return out

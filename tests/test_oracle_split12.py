@@ -1,0 +1,107 @@
+"""Pins of the Split12 oracle (oracle/split12.py): a hand-worked container,
+the 12-bits-a-value size, the codebook rule checked by brute force, round
+trips over every bf16 pattern, and refusal of non-canonical containers."""
+import numpy as np
+import pytest
+
+import workloads
+from _golden import load_container
+
+C = 65536
+
+
+@pytest.fixture(scope="module")
+def s12():
+    import split12
+    return split12
+
+
+def _golden_bits():
+    v = [0x3F80, 0x3F00] + [((i - 1) << 8) | (0xA0 + i) for i in range(2, 18)]
+    return np.array(v, np.uint16)
+
+
+def test_golden_container(s12):
+    bits = _golden_bits()
+    want = load_container("split12_n18_one_exception.txt")
+    got = s12.encode(bits)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert np.array_equal(s12.decode(got), bits)
+
+
+def test_size_is_twelve_bits_a_value(s12):
+    # no exceptions: header 64 + codebook 16 + offset table + n/2 + n bytes
+    for n in (1, 2, 17, C, C + 1, 5 * C + 3):
+        bits = np.full(n, 0x3C00, np.uint16) | np.arange(n, dtype=np.uint16) % 256
+        cont = s12.encode(bits)
+        nc = -(-n // C)
+        r16 = lambda v: (v + 15) // 16 * 16
+        assert cont.size == r16(r16(r16(80 + 4 * (nc + 1)) + (n + 1) // 2) + n)
+        assert np.array_equal(s12.decode(cont), bits)
+    big = s12.encode(np.full(64 * C, 0x3F80, np.uint16))
+    assert abs(big.size / (2 * 64 * C) - 0.75) < 1e-4
+
+
+def test_codebook_rule_by_brute_force(s12):
+    rng = np.random.default_rng(12)
+    for trial in range(200):
+        nd = int(rng.integers(1, 40))
+        alphabet = rng.choice(256, nd, replace=False)
+        high = rng.choice(alphabet, int(rng.integers(1, 300))).astype(np.uint8)
+        book = s12.codebook(high)
+        counts = np.bincount(high, minlength=256)
+        present = np.nonzero(counts)[0]
+        assert book.size == min(16, present.size)
+        assert np.all(np.diff(book.astype(int)) > 0)
+        inside = set(book.tolist())
+        for b in present:
+            if b in inside:
+                continue
+            for a in inside:   # every member beats every outsider
+                assert counts[a] > counts[b] or (counts[a] == counts[b] and a < b)
+
+
+def test_round_trips(s12):
+    every = np.arange(1 << 16, dtype=np.uint16)
+    cont = s12.encode(every)
+    h = s12.read_header(cont)
+    assert h["k"] == 16 and h["ne"] == (256 - 16) * 256   # ties: bytes 0..15 win
+    assert np.array_equal(s12.decode(cont), every)
+    for n in (0, 1, 15, 16, 17, C - 1, C, C + 1):
+        b = workloads.generate_tensor(4, 1)[:n]
+        assert np.array_equal(s12.decode(s12.encode(b)), b)
+    # exceptions in several chunks, the last one ragged
+    b = workloads.generate_tensor(4, 1)[: 3 * C + 123].copy()
+    b[[5, C + 7, 2 * C, 3 * C + 122]] = 0x0101
+    cont = s12.encode(b)
+    assert s12.read_header(cont)["ne"] >= 4
+    assert np.array_equal(s12.decode(cont), b)
+
+
+def test_ratio_on_weights(s12):
+    # bf16 N(0, 0.02): a handful of exceptions, 12 bits a value plus a little
+    b = workloads.generate_tensor(1, 0)
+    cont = s12.encode(b)
+    h = s12.read_header(cont)
+    assert 0 < h["ne"] < b.size // 1000
+    assert 0.75 < cont.size / b.nbytes < 0.7505
+
+
+def test_non_canonical_refused(s12):
+    good = s12.encode(_golden_bits())
+    s12.decode(good)
+    cases = []
+    c = good.copy(); c[64:66] = [0x02, 0x01]; cases.append(c)        # codebook not ascending
+    c = good.copy(); c[160] = 0x05; cases.append(c)                   # exception byte in the book
+    c = good.copy(); c[104] = 0x1E; cases.append(c)                   # exception's index not 0
+    c = good.copy(); c[144] = 30; cases.append(c)                     # exception past n
+    c = good.copy(); c[0] = 0; cases.append(c)                        # magic
+    c = good.copy(); c[84] = 2; cases.append(c)                       # exception count
+    # entry 14 (0x0F) replaced by 0x11: still ascending, but the decoded values
+    # would then have 0x10 and 0x11 tied at one and 0x10 must win
+    c = good.copy(); c[78] = 0x11; cases.append(c)                    # book not the top 16
+    for c in cases:
+        with pytest.raises(ValueError):
+            s12.decode(c)
+    with pytest.raises(ValueError):
+        s12.decode(good[:-1])                                         # cut short
