@@ -127,14 +127,14 @@ def read_header(cont: np.ndarray) -> dict:
 
 
 def decode(cont: np.ndarray) -> np.ndarray:
-    """bf16 bits (uint16) of a container; ValueError if it is not the one
-    container the format allows for some input."""
+    """bf16 bits (uint16) of a container.  Checks what decoding relies on:
+    the header and layout, a non-decreasing exception table ending at ne,
+    every index below K, and exception positions inside their chunk, inside
+    n and ascending within the chunk (ValueError otherwise)."""
     c = np.ascontiguousarray(cont, dtype=np.uint8)
     h = read_header(c)
     n, ne, k, nc = h["n"], h["ne"], h["k"], h["nc"]
     book = c[HEADER:HEADER + BOOK]
-    if k and (np.any(np.diff(book[:k].astype(np.int64)) <= 0) or np.any(book[k:] != 0)):
-        raise ValueError("codebook not ascending or padded with non-zero bytes")
     o = h["off_excoff"]
     exc_off = c[o:o + 4 * (nc + 1)].view("<u4").astype(np.int64)
     if exc_off[0] != 0 or exc_off[-1] != ne or np.any(np.diff(exc_off) < 0):
@@ -148,15 +148,24 @@ def decode(cont: np.ndarray) -> np.ndarray:
         raise ValueError("codebook index out of range")
     low = c[h["off_lo"]:h["off_lo"] + n].astype(np.uint16)
     out = (book[idx].astype(np.uint16) << 8) | low
-    if ne:
-        chunk_of = np.repeat(np.arange(nc, dtype=np.int64), np.diff(exc_off))
-        pos = chunk_of * CHUNK + c[h["off_exc"]:h["off_exc"] + 2 * ne].view("<u2").astype(np.int64)
-        if np.any(np.diff(pos) <= 0) or pos[-1] >= n:
+    for ch in range(nc):
+        e0, e1 = int(exc_off[ch]), int(exc_off[ch + 1])
+        if e0 == e1:
+            continue
+        p = c[h["off_exc"] + 2 * e0:h["off_exc"] + 2 * e1].view("<u2").astype(np.int64)
+        if np.any(np.diff(p) <= 0) or ch * CHUNK + p[-1] >= n:
             raise ValueError("bad Split12 exception position")
-        val = c[h["off_excval"]:h["off_excval"] + ne]
-        if np.any(idx[pos] != 0) or np.any(np.isin(val, book[:k])):
-            raise ValueError("exception not in canonical form")
-        out[pos] = (val.astype(np.uint16) << 8) | low[pos]
-    if not np.array_equal(codebook((out >> 8).astype(np.uint8)), book[:k]):
-        raise ValueError("codebook is not the values' most frequent high bytes")
+        val = c[h["off_excval"] + e0:h["off_excval"] + e1].astype(np.uint16)
+        i = ch * CHUNK + p
+        out[i] = (val << 8) | low[i]
     return out
+
+
+def canonical(cont: np.ndarray) -> bool:
+    """Whether a decodable container is the one that encode() writes for its
+    values: codebook ascending, zero-padded and equal to the values' 16 most
+    frequent high bytes; every exception marked by index 0 and missing from
+    the codebook; padding zero."""
+    c = np.ascontiguousarray(cont, dtype=np.uint8)
+    vals = decode(c)
+    return c.size == read_header(c)["total"] and np.array_equal(encode(vals), c)

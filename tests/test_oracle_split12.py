@@ -87,21 +87,44 @@ def test_ratio_on_weights(s12):
     assert 0.75 < cont.size / b.nbytes < 0.7505
 
 
-def test_non_canonical_refused(s12):
+def test_structural_damage_refused(s12):
     good = s12.encode(_golden_bits())
-    s12.decode(good)
+    assert s12.canonical(good)
     cases = []
-    c = good.copy(); c[64:66] = [0x02, 0x01]; cases.append(c)        # codebook not ascending
-    c = good.copy(); c[160] = 0x05; cases.append(c)                   # exception byte in the book
-    c = good.copy(); c[104] = 0x1E; cases.append(c)                   # exception's index not 0
     c = good.copy(); c[144] = 30; cases.append(c)                     # exception past n
     c = good.copy(); c[0] = 0; cases.append(c)                        # magic
     c = good.copy(); c[84] = 2; cases.append(c)                       # exception count
-    # entry 14 (0x0F) replaced by 0x11: still ascending, but the decoded values
-    # would then have 0x10 and 0x11 tied at one and 0x10 must win
-    c = good.copy(); c[78] = 0x11; cases.append(c)                    # book not the top 16
+    c = good.copy(); c[7] = 3; cases.append(c)                        # K = 3: index 15 out of range
+    c = good.copy(); c[56] ^= 0x10; cases.append(c)                   # total
     for c in cases:
         with pytest.raises(ValueError):
             s12.decode(c)
     with pytest.raises(ValueError):
         s12.decode(good[:-1])                                         # cut short
+    # two exceptions in one chunk must ascend
+    b = np.arange(40, dtype=np.uint16) << 8 | 7
+    cont = s12.encode(b)
+    h = s12.read_header(cont)
+    assert h["ne"] == 40 - 16
+    bad = cont.copy()
+    first_two = bad[h["off_exc"]:h["off_exc"] + 4].view("<u2").copy()
+    bad[h["off_exc"]:h["off_exc"] + 4] = first_two[::-1].copy().view(np.uint8)
+    with pytest.raises(ValueError):
+        s12.decode(bad)
+
+
+def test_non_canonical_detected(s12):
+    good = s12.encode(_golden_bits())
+    cases = []
+    c = good.copy(); c[64:66] = [0x02, 0x01]; cases.append(c)        # codebook not ascending
+    c = good.copy(); c[160] = 0x05; cases.append(c)                   # exception byte in the book
+    c = good.copy(); c[104] = 0x1E; cases.append(c)                   # exception's index not 0
+    # entry 14 (0x0F) replaced by 0x11: still ascending, but the decoded values
+    # would then have 0x10 and 0x11 tied at one and 0x10 must win
+    c = good.copy(); c[78] = 0x11; cases.append(c)
+    for c in cases:
+        s12.decode(c)                     # decodable, but not what encode writes
+        assert not s12.canonical(c)
+    # the valid container of other values is canonical
+    c = good.copy(); c[79] = 0x3E
+    assert s12.canonical(c)
