@@ -15,7 +15,7 @@ Reading (the page gives the idea, not the format):
     codebook) and its low byte;
   * values whose high byte is not in the codebook are exceptions, listed per
     65,536-value chunk in ascending position: u16 position in the chunk and
-    the u8 high byte; a u32 offset table gives each chunk's first exception.
+    the u8 high byte; a u64 offset table gives each chunk's first exception.
 
 Container (little-endian, sections 16-byte aligned, zero padding):
     0   "W12C"  u16 version 1  u8 dtype 1 (bf16)  u8 K (codebook entries)
@@ -24,7 +24,7 @@ Container (little-endian, sections 16-byte aligned, zero padding):
     24  u64 ne (exceptions)
     32  u64 off_idx   40 u64 off_lo   48 u64 off_exc   56 u64 total bytes
     64  u8 codebook[16] (entries >= K are 0)
-    80  u32 exc_off[nc + 1]
+    80  u64 exc_off[nc + 1]
     off_idx   ceil(n / 2) index bytes
     off_lo    n low bytes
     off_exc   u16 position[ne], then (16-aligned) u8 high byte[ne]
@@ -46,7 +46,7 @@ def _r16(v: int) -> int:
 def layout(n: int, ne: int) -> dict:
     nc = -(-n // CHUNK)
     off_excoff = HEADER + BOOK
-    off_idx = _r16(off_excoff + 4 * (nc + 1))
+    off_idx = _r16(off_excoff + 8 * (nc + 1))
     off_lo = _r16(off_idx + (n + 1) // 2)
     off_exc = _r16(off_lo + n)
     off_excval = off_exc + _r16(2 * ne)
@@ -94,7 +94,7 @@ def encode(bits: np.ndarray) -> np.ndarray:
     out[32:64] = np.array([L["off_idx"], L["off_lo"], L["off_exc"], L["total"]], "<u8").view(np.uint8)
     out[HEADER:HEADER + k] = book
     o = L["off_excoff"]
-    out[o:o + 4 * (L["nc"] + 1)] = exc_off.astype("<u4").view(np.uint8)
+    out[o:o + 8 * (L["nc"] + 1)] = exc_off.astype("<u8").view(np.uint8)
     padded = np.zeros(2 * ((n + 1) // 2), np.uint8)
     padded[:n] = idx
     out[L["off_idx"]:L["off_idx"] + padded.size // 2] = padded[0::2] | (padded[1::2] << 4)
@@ -136,7 +136,7 @@ def decode(cont: np.ndarray) -> np.ndarray:
     n, ne, k, nc = h["n"], h["ne"], h["k"], h["nc"]
     book = c[HEADER:HEADER + BOOK]
     o = h["off_excoff"]
-    exc_off = c[o:o + 4 * (nc + 1)].view("<u4").astype(np.int64)
+    exc_off = c[o:o + 8 * (nc + 1)].view("<u8").astype(np.int64)
     if exc_off[0] != 0 or exc_off[-1] != ne or np.any(np.diff(exc_off) < 0):
         raise ValueError("bad Split12 exception table")
     packed = c[h["off_idx"]:h["off_idx"] + (n + 1) // 2]

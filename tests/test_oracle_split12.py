@@ -36,7 +36,7 @@ def test_size_is_twelve_bits_a_value(s12):
         cont = s12.encode(bits)
         nc = -(-n // C)
         r16 = lambda v: (v + 15) // 16 * 16
-        assert cont.size == r16(r16(r16(80 + 4 * (nc + 1)) + (n + 1) // 2) + n)
+        assert cont.size == r16(r16(r16(80 + 8 * (nc + 1)) + (n + 1) // 2) + n)
         assert np.array_equal(s12.decode(cont), bits)
     big = s12.encode(np.full(64 * C, 0x3F80, np.uint16))
     assert abs(big.size / (2 * 64 * C) - 0.75) < 1e-4
@@ -93,7 +93,7 @@ def test_structural_damage_refused(s12):
     cases = []
     c = good.copy(); c[144] = 30; cases.append(c)                     # exception past n
     c = good.copy(); c[0] = 0; cases.append(c)                        # magic
-    c = good.copy(); c[84] = 2; cases.append(c)                       # exception count
+    c = good.copy(); c[88] = 2; cases.append(c)                       # exception count
     c = good.copy(); c[7] = 3; cases.append(c)                        # K = 3: index 15 out of range
     c = good.copy(); c[56] ^= 0x10; cases.append(c)                   # total
     for c in cases:
