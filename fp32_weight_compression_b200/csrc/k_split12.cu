@@ -1,0 +1,505 @@
+// k_split12.cu -- the Split12 serving format for bf16 (include/wc_split12.h;
+// "weight-compression" README: the high byte from a codebook, the low byte
+// raw): encoder in five kernels, decoder in one, and their C ABI.
+//
+// Encode (all on one stream, sizes from n alone):
+//   k12_prep   1 block    header fields that depend on n, zero padding,
+//                         clears the global high-byte histogram
+//   k12_hist   1 block / chunk   high-byte counts of the chunk (one column
+//                         per lane in shared memory), kept per chunk and
+//                         added to the global histogram
+//   k12_book   1 block    the 16 most frequent high bytes (ties to the smaller
+//                         byte), ascending -> codebook, K, and a 256-entry
+//                         byte -> slot table (0xFF: missed)
+//   k12_count  1 warp / chunk   the chunk's exceptions from its histogram
+//   k12_scan   1 block    exclusive scan -> exc_off[], ne, total size, the
+//                         padding after the exception lists
+//   k12_pack   1 block / chunk   index nibbles and low bytes; exceptions in
+//                         ascending position at the chunk's exc_off
+// Decode: k12_decode, a persistent grid, one block per chunk at a time:
+// expands 16 values per thread per step (the codebook lives in four
+// registers; byte permutes do the lookup), then patches the chunk's
+// exceptions after a block barrier.
+#include <cstdint>
+#include <mutex>
+
+#include "wc.h"
+#include "wc_block.cuh"
+#include "wc_split12.h"
+
+namespace wc12 {
+
+constexpr uint64_t kChunk = 65536;
+constexpr uint32_t kBookOff = 64;
+constexpr uint32_t kExcOffOff = 80;
+constexpr uint32_t kMagic = 0x43323157u;  // "W12C"
+constexpr uint64_t kMaxN = uint64_t(1) << 44;
+
+constexpr uint64_t kScrHist = 0;           // u64[256]
+constexpr uint64_t kScrLut = 2048;         // u8[256]
+constexpr uint64_t kScrChunkHist = 2560;   // u32[nc][256]
+
+__host__ __device__ inline uint64_t r16(uint64_t v) { return (v + 15) & ~uint64_t(15); }
+
+struct Lay {
+  uint64_t nc, off_idx, off_lo, off_exc, off_excval, total;
+};
+
+__host__ __device__ inline Lay lay(uint64_t n, uint64_t ne) {
+  Lay L;
+  L.nc = (n + kChunk - 1) / kChunk;
+  L.off_idx = r16(kExcOffOff + 8 * (L.nc + 1));
+  L.off_lo = r16(L.off_idx + (n + 1) / 2);
+  L.off_exc = r16(L.off_lo + n);
+  L.off_excval = L.off_exc + r16(2 * ne);
+  L.total = L.off_excval + r16(ne);
+  return L;
+}
+
+__device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k12_prep(uint64_t n, uint8_t *out, uint8_t *scr) {
+  const int tid = threadIdx.x;
+  const Lay L = lay(n, 0);
+  reinterpret_cast<unsigned long long *>(scr + kScrHist)[tid] = 0;
+  if (tid == 0) {
+    uint32_t *h32 = reinterpret_cast<uint32_t *>(out);
+    uint64_t *h64 = reinterpret_cast<uint64_t *>(out);
+    h32[0] = kMagic;
+    h32[1] = 1u | (1u << 16);  // version 1, dtype bf16; K follows from k12_book
+    h64[1] = n;
+    h32[4] = uint32_t(kChunk);
+    h32[5] = uint32_t(L.nc);
+    h64[3] = 0;                // ne: k12_scan
+    h64[4] = L.off_idx;
+    h64[5] = L.off_lo;
+    h64[6] = L.off_exc;
+    h64[7] = 0;                // total: k12_scan
+  }
+  // padding that depends on n alone (each run is shorter than 16 bytes)
+  const uint64_t z0 = kExcOffOff + 8 * (L.nc + 1), z1 = L.off_idx + (n + 1) / 2, z2 = L.off_lo + n;
+  if (tid < 16) {
+    if (z0 + tid < L.off_idx) out[z0 + tid] = 0;
+  } else if (tid < 32) {
+    if (z1 + (tid - 16) < L.off_lo) out[z1 + (tid - 16)] = 0;
+  } else if (tid < 48) {
+    if (z2 + (tid - 32) < L.off_exc) out[z2 + (tid - 32)] = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+constexpr int kHistThreads = 512;
+
+__device__ __forceinline__ void count_hi(uint32_t *sh, int lane, uint32_t w) {
+  atomicAdd(&sh[(((w >> 8) & 0xFFu) << 5) | lane], 1u);
+  atomicAdd(&sh[((w >> 24) << 5) | lane], 1u);
+}
+
+__device__ __forceinline__ void count_group(uint32_t *sh, int lane, uint4 a, uint4 b) {
+  count_hi(sh, lane, a.x); count_hi(sh, lane, a.y); count_hi(sh, lane, a.z); count_hi(sh, lane, a.w);
+  count_hi(sh, lane, b.x); count_hi(sh, lane, b.y); count_hi(sh, lane, b.z); count_hi(sh, lane, b.w);
+}
+
+__global__ void __launch_bounds__(kHistThreads, 2)
+k12_hist(const uint16_t *__restrict__ in, uint64_t n, uint8_t *scr) {
+  __shared__ __align__(16) uint32_t sh[256 * 32];  // [high byte][lane]
+  const int tid = threadIdx.x, lane = tid & 31;
+  const uint64_t c = blockIdx.x, v0 = c * kChunk;
+  const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
+  const uint32_t nfull = count / 16;
+  for (int i = tid; i < 256 * 32 / 4; i += kHistThreads)
+    reinterpret_cast<uint4 *>(sh)[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  const uint16_t *src = in + v0;
+  uint32_t g = tid;
+  for (; g + kHistThreads < nfull; g += 2 * kHistThreads) {
+    const uint16_t *s0 = src + 16 * g, *s1 = src + 16 * (g + kHistThreads);
+    const uint4 a0 = wc::ld_nc_v4(s0), b0 = wc::ld_nc_v4(s0 + 8);
+    const uint4 a1 = wc::ld_nc_v4(s1), b1 = wc::ld_nc_v4(s1 + 8);
+    count_group(sh, lane, a0, b0);
+    count_group(sh, lane, a1, b1);
+  }
+  for (; g < nfull; g += kHistThreads)
+    count_group(sh, lane, wc::ld_nc_v4(src + 16 * g), wc::ld_nc_v4(src + 16 * g + 8));
+  if (g == nfull)  // the thread whose next group is the ragged tail
+    for (uint32_t v = 16 * nfull; v < count; v++) atomicAdd(&sh[((uint32_t(src[v]) >> 8) << 5) | lane], 1u);
+  __syncthreads();
+  if (tid < 256) {
+    uint32_t sum = 0;
+#pragma unroll 8
+    for (int j = 0; j < 32; j++) sum += sh[(tid << 5) | ((j + tid) & 31)];
+    reinterpret_cast<uint32_t *>(scr + kScrChunkHist)[c * 256 + tid] = sum;
+    if (sum)
+      atomicAdd(reinterpret_cast<unsigned long long *>(scr + kScrHist) + tid,
+                static_cast<unsigned long long>(sum));
+  }
+}
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k12_book(uint8_t *out, uint8_t *scr) {
+  __shared__ unsigned long long cnt[256];
+  __shared__ uint32_t wsel[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  cnt[tid] = reinterpret_cast<const unsigned long long *>(scr + kScrHist)[tid];
+  __syncthreads();
+  const unsigned long long mine = cnt[tid];
+  uint32_t rank = 0;  // bytes that beat this one: more values, or as many and smaller
+  for (int b = 0; b < 256; b++) {
+    const unsigned long long o = cnt[b];
+    rank += (o > mine || (o == mine && b < tid)) ? 1u : 0u;
+  }
+  const bool sel = mine > 0 && rank < 16;
+  const uint32_t bal = __ballot_sync(0xFFFFFFFFu, sel);
+  if (lane == 0) wsel[warp] = __popc(bal);
+  __syncthreads();
+  uint32_t before = 0, k = 0;
+  for (int w = 0; w < 8; w++) {
+    before += w < warp ? wsel[w] : 0;
+    k += wsel[w];
+  }
+  const uint32_t pos = before + __popc(bal & ((1u << lane) - 1u));
+  scr[kScrLut + tid] = sel ? uint8_t(pos) : uint8_t(0xFF);
+  if (sel) out[kBookOff + pos] = uint8_t(tid);
+  if (tid < 16 && uint32_t(tid) >= k) out[kBookOff + tid] = 0;
+  if (tid == 0) out[7] = uint8_t(k);
+}
+
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k12_count(uint64_t nc, uint8_t *out, const uint8_t *scr) {
+  __shared__ uint8_t lut[256];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  lut[tid] = scr[kScrLut + tid];
+  __syncthreads();
+  const uint64_t c = uint64_t(blockIdx.x) * 8 + warp;
+  uint64_t *exc_off = reinterpret_cast<uint64_t *>(out + kExcOffOff);
+  if (blockIdx.x == 0 && tid == 0) exc_off[0] = 0;
+  if (c >= nc) return;
+  const uint32_t *h = reinterpret_cast<const uint32_t *>(scr + kScrChunkHist) + c * 256;
+  uint32_t s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; j++) {
+    const int b = lane * 8 + j;
+    s += lut[b] == 0xFF ? h[b] : 0u;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if (lane == 0) exc_off[c + 1] = s;  // this chunk's count; k12_scan sums
+}
+
+// ---------------------------------------------------------------------------
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads) k12_scan(uint64_t n, uint8_t *out, uint64_t *out_size) {
+  __shared__ uint64_t red[kScanThreads / 32 + 1];
+  __shared__ uint64_t s_ne;
+  const int tid = threadIdx.x;
+  const uint64_t nc = (n + kChunk - 1) / kChunk;
+  uint64_t *exc_off = reinterpret_cast<uint64_t *>(out + kExcOffOff);
+  uint64_t carry = 0;
+  for (uint64_t base = 1; base <= nc; base += kScanThreads) {  // entries 1..nc, in place
+    const uint64_t i = base + tid;
+    const uint64_t v = i <= nc ? exc_off[i] : 0;
+    const uint64_t ex = wc::block_excl_scan_u64<kScanThreads>(v, red);
+    const uint64_t tot = wc::block_sum_u64<kScanThreads>(v, red);
+    if (i <= nc) exc_off[i] = carry + ex + v;
+    carry += tot;
+  }
+  if (tid == 0) s_ne = carry;
+  __syncthreads();
+  const uint64_t ne = s_ne;
+  const Lay L = lay(n, ne);
+  if (tid == 0) {
+    uint64_t *h64 = reinterpret_cast<uint64_t *>(out);
+    h64[3] = ne;
+    h64[7] = L.total;
+    *out_size = L.total;
+  }
+  const uint64_t z0 = L.off_exc + 2 * ne, z1 = L.off_excval + ne;
+  if (tid < 16) {
+    if (z0 + tid < L.off_excval) out[z0 + tid] = 0;
+  } else if (tid < 32) {
+    if (z1 + (tid - 16) < L.total) out[z1 + (tid - 16)] = 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+constexpr int kPackThreads = 256;
+
+// slot of each of the 4 values' high bytes in byte j of the result
+__device__ __forceinline__ uint32_t slots4(const uint8_t *lut, uint32_t w0, uint32_t w1) {
+  const uint32_t hb = __byte_perm(w0, w1, 0x7531);
+  return uint32_t(lut[hb & 0xFFu]) | (uint32_t(lut[(hb >> 8) & 0xFFu]) << 8) |
+         (uint32_t(lut[(hb >> 16) & 0xFFu]) << 16) | (uint32_t(lut[hb >> 24]) << 24);
+}
+
+// 4 slots (bytes, 0xFF = missed) -> 4 index nibbles in the low 16 bits, and
+// the number missed
+__device__ __forceinline__ uint32_t nibbles4(uint32_t s4, uint32_t &missed) {
+  const uint32_t miss = s4 & 0x80808080u;  // slots are < 16 or 0xFF
+  missed += __popc(miss);
+  const uint32_t idx = s4 & ~((miss >> 7) * 0xFFu);  // missed -> 0
+  return (idx & 0xFu) | ((idx >> 4) & 0xF0u) | ((idx >> 8) & 0xF00u) | ((idx >> 12) & 0xF000u);
+}
+
+__global__ void __launch_bounds__(kPackThreads)
+k12_pack(const uint16_t *__restrict__ in, uint64_t n, uint8_t *out, const uint8_t *scr) {
+  __shared__ uint8_t lut[256];
+  __shared__ uint64_t red[kPackThreads / 32 + 1];
+  const int tid = threadIdx.x;
+  lut[tid] = scr[kScrLut + tid];
+  const uint64_t c = blockIdx.x, v0 = c * kChunk;
+  const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
+  const uint32_t nfull = count / 16, tail = count % 16;
+  const uint32_t ngroups = nfull + (tail ? 1u : 0u);
+  const uint64_t *h64 = reinterpret_cast<const uint64_t *>(out);
+  const uint64_t ne = h64[3];
+  const Lay L = lay(n, ne);
+  const uint64_t e_base = reinterpret_cast<const uint64_t *>(out + kExcOffOff)[c];
+  uint16_t *exc_pos = reinterpret_cast<uint16_t *>(out + L.off_exc);
+  uint8_t *exc_val = out + L.off_excval;
+  uint8_t *idx_plane = out + L.off_idx + v0 / 2;
+  uint8_t *lo_plane = out + L.off_lo + v0;
+  const uint16_t *src = in + v0;
+  __syncthreads();
+
+  uint64_t run = 0;  // exceptions of this chunk written so far
+  for (uint32_t it = 0; it * kPackThreads < ngroups; it++) {
+    const uint32_t g = tid + it * kPackThreads;
+    uint32_t missed = 0;
+    uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+    if (g < nfull) {
+      a = wc::ld_nc_v4(src + 16 * g);
+      b = wc::ld_nc_v4(src + 16 * g + 8);
+      const uint32_t q0 = nibbles4(slots4(lut, a.x, a.y), missed);
+      const uint32_t q1 = nibbles4(slots4(lut, a.z, a.w), missed);
+      const uint32_t q2 = nibbles4(slots4(lut, b.x, b.y), missed);
+      const uint32_t q3 = nibbles4(slots4(lut, b.z, b.w), missed);
+      *reinterpret_cast<uint2 *>(idx_plane + 8 * g) = make_uint2(q0 | (q1 << 16), q2 | (q3 << 16));
+      *reinterpret_cast<uint4 *>(lo_plane + 16 * g) =
+          make_uint4(__byte_perm(a.x, a.y, 0x6420), __byte_perm(a.z, a.w, 0x6420),
+                     __byte_perm(b.x, b.y, 0x6420), __byte_perm(b.z, b.w, 0x6420));
+    } else if (g == nfull && tail) {
+      uint32_t pair = 0;
+      for (uint32_t j = 0; j < tail; j++) {
+        const uint32_t v = src[16 * g + j];
+        const uint32_t s = lut[v >> 8];
+        const uint32_t nib = s == 0xFFu ? 0u : s;
+        missed += s == 0xFFu ? 1u : 0u;
+        pair |= nib << (4 * (j & 1));
+        if (j & 1) {
+          idx_plane[8 * g + j / 2] = uint8_t(pair);
+          pair = 0;
+        }
+        lo_plane[16 * g + j] = uint8_t(v & 0xFFu);
+      }
+      if (tail & 1) idx_plane[8 * g + tail / 2] = uint8_t(pair);  // high nibble 0
+    }
+    // exceptions, in ascending position: this step's groups in thread order
+    if (__syncthreads_or(missed != 0)) {
+      const uint64_t before = wc::block_excl_scan_u64<kPackThreads>(missed, red);
+      const uint64_t total = wc::block_sum_u64<kPackThreads>(missed, red);
+      uint64_t e = e_base + run + before;
+      const uint32_t nv = g < nfull ? 16u : (g == nfull ? tail : 0u);
+      for (uint32_t j = 0; j < nv && missed; j++) {
+        uint32_t v;
+        if (g < nfull) {
+          const uint32_t w = j < 8 ? (&a.x)[j >> 1] : (&b.x)[(j - 8) >> 1];
+          v = (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+        } else {
+          v = src[16 * g + j];
+        }
+        const uint32_t h = v >> 8;
+        if (lut[h] == 0xFFu) {
+          exc_pos[e] = uint16_t(16 * g + j);
+          exc_val[e] = uint8_t(h);
+          e++;
+          missed--;
+        }
+      }
+      run += total;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+constexpr int kDecThreads = 256;
+
+// 4 index nibbles (low 16 bits of q), the codebook in four words, 4 low bytes
+// -> the 4 bf16 values as two words
+__device__ __forceinline__ uint2 expand4(uint32_t q, uint4 book, uint32_t lo4) {
+  const uint32_t sel = q & 0x7777u;              // entry within its half
+  const uint32_t upper = (q >> 3) & 0x1111u;     // 1: entries 8..15
+  const uint32_t r0 = __byte_perm(book.x, book.y, sel);
+  const uint32_t r1 = __byte_perm(book.z, book.w, sel);
+  const uint32_t m = __byte_perm(0x0000FF00u, 0u, upper);  // 0xFF where upper
+  const uint32_t hi4 = (r0 & ~m) | (r1 & m);
+  return make_uint2(__byte_perm(lo4, hi4, 0x5140), __byte_perm(lo4, hi4, 0x7362));
+}
+
+// any of the 8 nibbles of w at or above k (1 <= k <= 16)
+__device__ __forceinline__ uint32_t over8(uint32_t w, uint32_t add) {
+  const uint32_t e = w & 0x0F0F0F0Fu, o = (w >> 4) & 0x0F0F0F0Fu;
+  return ((e + add) | (o + add)) & 0x10101010u;
+}
+
+__global__ void __launch_bounds__(kDecThreads)
+k12_decode(const uint8_t *__restrict__ cont, uint64_t cont_bytes, uint16_t *__restrict__ out,
+           uint64_t out_cap, int32_t *status) {
+  const int tid = threadIdx.x;
+  // header checks (every block; block 0 reports)
+  if (cont_bytes < 96) {
+    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CORRUPT);
+    return;
+  }
+  const uint32_t *h32 = reinterpret_cast<const uint32_t *>(cont);
+  const uint64_t *h64 = reinterpret_cast<const uint64_t *>(cont);
+  const uint64_t n = h64[1], ne = h64[3];
+  const uint32_t k = h32[1] >> 24;
+  bool ok = h32[0] == kMagic && (h32[1] & 0xFFFFFFu) == (1u | (1u << 16)) && k <= 16 &&
+            (n > 0) == (k > 0) && n <= kMaxN && ne <= n && h32[4] == uint32_t(kChunk);
+  Lay L{};
+  if (ok) {
+    L = lay(n, ne);
+    ok = h32[5] == uint32_t(L.nc) && h64[4] == L.off_idx && h64[5] == L.off_lo &&
+         h64[6] == L.off_exc && h64[7] == L.total && L.total <= cont_bytes;
+  }
+  if (!ok) {
+    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CORRUPT);
+    return;
+  }
+  if (2 * n > out_cap) {
+    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CAPACITY);
+    return;
+  }
+  const uint4 book = *reinterpret_cast<const uint4 *>(cont + kBookOff);
+  const uint32_t add = (16u - k) * 0x01010101u;
+  const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(cont + kExcOffOff);
+  const uint16_t *exc_pos = reinterpret_cast<const uint16_t *>(cont + L.off_exc);
+  const uint8_t *exc_val = cont + L.off_excval;
+  const uint8_t *idx_plane = cont + L.off_idx;
+  const uint8_t *lo_plane = cont + L.off_lo;
+  if (L.nc == 0 && exc_off[0] != 0) {  // an empty tensor's table is one zero
+    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CORRUPT);
+    return;
+  }
+
+  for (uint64_t c = blockIdx.x; c < L.nc; c += gridDim.x) {
+    const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
+    if (!(e0 <= e1 && e1 <= ne && (c != 0 || e0 == 0) && (c + 1 != L.nc || e1 == ne))) {
+      if (tid == 0) report(status, WC_ERR_CORRUPT);
+      continue;
+    }
+    const uint64_t v0 = c * kChunk;
+    const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
+    const uint32_t nfull = count / 16, tail = count % 16;
+    uint32_t bad = 0;
+    for (uint32_t g = tid; g < nfull; g += kDecThreads) {
+      const uint2 q = *reinterpret_cast<const uint2 *>(idx_plane + v0 / 2 + 8 * g);
+      const uint4 lo = *reinterpret_cast<const uint4 *>(lo_plane + v0 + 16 * g);
+      bad |= over8(q.x, add) | over8(q.y, add);
+      const uint2 o0 = expand4(q.x, book, lo.x), o1 = expand4(q.x >> 16, book, lo.y);
+      const uint2 o2 = expand4(q.y, book, lo.z), o3 = expand4(q.y >> 16, book, lo.w);
+      uint4 *dst = reinterpret_cast<uint4 *>(out + v0 + 16 * g);
+      dst[0] = make_uint4(o0.x, o0.y, o1.x, o1.y);
+      dst[1] = make_uint4(o2.x, o2.y, o3.x, o3.y);
+    }
+    if (tid == 0) {  // the ragged tail, value by value
+      for (uint32_t j = 0; j < tail; j++) {
+        const uint64_t v = v0 + 16 * uint64_t(nfull) + j;
+        const uint32_t nib = (uint32_t(idx_plane[v / 2]) >> (4 * (v & 1))) & 0xFu;
+        bad |= nib >= k ? 1u : 0u;
+        const uint32_t hi = (nib < 8 ? ((&book.x)[nib >> 2] >> (8 * (nib & 3)))
+                                     : ((&book.z)[(nib - 8) >> 2] >> (8 * (nib & 3)))) & 0xFFu;
+        out[v] = uint16_t((hi << 8) | lo_plane[v]);
+      }
+    }
+    if (bad) report(status, WC_ERR_CORRUPT);
+    __syncthreads();  // the chunk's values are written; patch its exceptions
+    for (uint64_t e = e0 + tid; e < e1; e += kDecThreads) {
+      const uint32_t p = exc_pos[e];
+      if (p >= count || (e > e0 && p <= exc_pos[e - 1])) {
+        report(status, WC_ERR_CORRUPT);
+        continue;
+      }
+      const uint64_t v = v0 + p;
+      out[v] = uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[v]);
+    }
+    __syncthreads();
+  }
+}
+
+int sms_of_current_device() {
+  static std::mutex mu;
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache[dev] == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = sms;
+  }
+  return cache[dev];
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace wc12
+
+extern "C" {
+
+uint64_t wc12_encode_bound(uint64_t n) {
+  if (n > wc12::kMaxN) return 0;
+  return wc12::lay(n, n - (n + 15) / 16).total;
+}
+
+uint64_t wc12_scratch_bytes(uint64_t n) {
+  if (n > wc12::kMaxN) return 0;
+  return wc12::kScrChunkHist + 1024 * ((n + wc12::kChunk - 1) / wc12::kChunk);
+}
+
+int32_t wc12_encode(const void *d_in, uint64_t n, void *d_out, uint64_t out_cap, void *d_scratch,
+                    uint64_t scratch_cap, uint64_t *d_out_size, void *stream) {
+  if (n > wc12::kMaxN || d_out == nullptr || d_scratch == nullptr || d_out_size == nullptr)
+    return WC_ERR_INVALID_ARG;
+  if (n > 0 && d_in == nullptr) return WC_ERR_INVALID_ARG;
+  if (!wc12::aligned(d_in, 16) || !wc12::aligned(d_out, 16) || !wc12::aligned(d_scratch, 16) ||
+      !wc12::aligned(d_out_size, 8))
+    return WC_ERR_INVALID_ARG;
+  if (out_cap < wc12_encode_bound(n) || scratch_cap < wc12_scratch_bytes(n)) return WC_ERR_CAPACITY;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const uint16_t *in = static_cast<const uint16_t *>(d_in);
+  uint8_t *out = static_cast<uint8_t *>(d_out);
+  uint8_t *scr = static_cast<uint8_t *>(d_scratch);
+  const uint64_t nc = (n + wc12::kChunk - 1) / wc12::kChunk;
+  if (nc > 0x7FFFFFFFull) return WC_ERR_INVALID_ARG;
+  wc12::k12_prep<<<1, 256, 0, s>>>(n, out, scr);
+  if (nc) wc12::k12_hist<<<unsigned(nc), wc12::kHistThreads, 0, s>>>(in, n, scr);
+  wc12::k12_book<<<1, 256, 0, s>>>(out, scr);
+  if (nc) wc12::k12_count<<<unsigned((nc + 7) / 8), 256, 0, s>>>(nc, out, scr);
+  else wc12::k12_count<<<1, 256, 0, s>>>(0, out, scr);  // writes exc_off[0]
+  wc12::k12_scan<<<1, wc12::kScanThreads, 0, s>>>(n, out, d_out_size);
+  if (nc) wc12::k12_pack<<<unsigned(nc), wc12::kPackThreads, 0, s>>>(in, n, out, scr);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return WC_ERR_CUDA;
+  return WC_OK;
+}
+
+int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out, uint64_t out_cap,
+                    int32_t *d_status, void *stream) {
+  if (d_cont == nullptr || d_status == nullptr) return WC_ERR_INVALID_ARG;
+  if (!wc12::aligned(d_cont, 16) || !wc12::aligned(d_out, 16) || !wc12::aligned(d_status, 4))
+    return WC_ERR_INVALID_ARG;
+  if (out_cap > 0 && d_out == nullptr) return WC_ERR_INVALID_ARG;
+  const int sms = wc12::sms_of_current_device();
+  if (sms <= 0) return WC_ERR_CUDA;
+  wc12::k12_decode<<<unsigned(sms * 8), wc12::kDecThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t *>(d_cont), cont_bytes, static_cast<uint16_t *>(d_out), out_cap,
+      d_status);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return WC_ERR_CUDA;
+  return WC_OK;
+}
+
+}  // extern "C"

@@ -112,6 +112,14 @@ def load() -> ctypes.CDLL:
                                  ctypes.POINTER(i32)]
     L.wc_chunk_ranges.restype = i32
     L.wc_chunk_ranges.argtypes = [vp, u64, u64, ctypes.POINTER(u64), ctypes.POINTER(u32)]
+    L.wc12_encode_bound.restype = u64
+    L.wc12_encode_bound.argtypes = [u64]
+    L.wc12_scratch_bytes.restype = u64
+    L.wc12_scratch_bytes.argtypes = [u64]
+    L.wc12_encode.restype = i32
+    L.wc12_encode.argtypes = [vp, u64, vp, u64, vp, u64, vp, vp]
+    L.wc12_decode.restype = i32
+    L.wc12_decode.argtypes = [vp, u64, vp, u64, vp, vp]
     L.wc_crc32_blocks.restype = i32
     L.wc_crc32_blocks.argtypes = [vp, u64, u64, vp, vp]
     _lib = L
@@ -395,6 +403,49 @@ def chunk_ranges(prefix, k: int) -> list[tuple[int, int]]:
     _check(load().wc_chunk_ranges(buf.ctypes.data, buf.size, k, out, ctypes.byref(cnt)),
            "wc_chunk_ranges")
     return [(int(out[2 * i]), int(out[2 * i + 1])) for i in range(cnt.value)]
+
+
+# ---------------------------------------------------------------------------
+# Split12 serving format (include/wc_split12.h): bf16 only.
+
+def split12_encode_bound(n: int) -> int:
+    return int(load().wc12_encode_bound(n))
+
+
+def split12_scratch_bytes(n: int) -> int:
+    return int(load().wc12_scratch_bytes(n))
+
+
+def split12_encode(t: torch.Tensor, stream=None) -> torch.Tensor:
+    """Split12 container (device uint8, trimmed) of a bf16 CUDA tensor."""
+    if t.dtype != torch.bfloat16:
+        raise TypeError("Split12 takes bf16 tensors")
+    f = _flat(t)
+    n = f.numel()
+    out = torch.empty(split12_encode_bound(n), dtype=torch.uint8, device=f.device)
+    scr = torch.empty(split12_scratch_bytes(n), dtype=torch.uint8, device=f.device)
+    size = torch.zeros(1, dtype=torch.int64, device=f.device)
+    _check(load().wc12_encode(f.data_ptr() if n else None, n, out.data_ptr(), out.numel(),
+                              scr.data_ptr(), scr.numel(), size.data_ptr(), _stream(stream)),
+           "wc12_encode")
+    return out[: int(size.item())]
+
+
+def split12_decode(cont: torch.Tensor, shape=None, out=None, stream=None) -> torch.Tensor:
+    """Decode a device Split12 container into bf16 (shape from the header's
+    value count, bytes 8..15, unless given)."""
+    if out is None:
+        if shape is None:
+            shape = (int(cont[8:16].cpu().numpy().view("<u8")[0]),)
+        out = torch.empty(shape, dtype=torch.bfloat16, device=cont.device)
+    of = _flat(out)
+    status = torch.zeros(1, dtype=torch.int32, device=cont.device)
+    _check(load().wc12_decode(cont.data_ptr(), cont.numel(), of.data_ptr() if of.numel() else None,
+                              of.numel() * 2, status.data_ptr(), _stream(stream)), "wc12_decode")
+    st = int(status.item())
+    if st != OK:
+        raise WCError(st, "wc12_decode (device status)")
+    return out
 
 
 CRC_BLOCK = 1 << 20

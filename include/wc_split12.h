@@ -1,0 +1,74 @@
+/*
+ * wc_split12.h -- the Split12 serving format for bf16 weights, in libwc.so.
+ *
+ * "weight-compression" README: Split12 splits bf16 into its two bytes,
+ * rebuilds the high byte from a codebook and keeps the low byte raw (24.967 %
+ * smaller on a 753B model).  Read as 12 bits a value: a 4-bit index into the
+ * tensor's 16-entry codebook of high bytes plus the raw low byte; values
+ * whose high byte the codebook misses are listed as exceptions.  It decodes
+ * with a few instructions per value, so it is the format a GEMM can expand
+ * in its prologue; the rANS container of wc.h stays the smaller storage
+ * format.
+ *
+ * Container "W12C" (little-endian; sections 16-byte aligned, zero padding):
+ *   0   "W12C", u16 version 1, u8 dtype 1 (bf16), u8 K (codebook entries)
+ *   8   u64 n
+ *   16  u32 chunk values 65536, u32 nc = ceil(n / 65536)
+ *   24  u64 ne (exceptions)
+ *   32  u64 off_idx, u64 off_lo, u64 off_exc, u64 total bytes
+ *   64  u8 codebook[16]: the K most frequent high bytes (b >> 8) of the
+ *       tensor, ties to the smaller byte, ascending; entries >= K are 0
+ *   80  u64 exc_off[nc + 1]: first exception of each chunk; exc_off[nc] = ne
+ *   off_idx = round16(80 + 8 (nc + 1)): ceil(n / 2) bytes of 4-bit indices,
+ *       value i in byte i / 2, low nibble for even i; 0 for an exception
+ *   off_lo = round16(off_idx + ceil(n / 2)): the n low bytes (b & 0xFF)
+ *   off_exc = round16(off_lo + n): u16 position of each exception within its
+ *       chunk, ascending within the chunk, chunk by chunk
+ *   off_exc + round16(2 ne): the exceptions' u8 high bytes
+ *   total = off_exc + round16(2 ne) + round16(ne)
+ * Exactly one container is correct for an input.
+ *
+ * Conventions are those of wc.h: device pointers, caller-owned buffers, no
+ * allocation, no synchronisation, work queued on `stream`; argument errors
+ * return synchronously, container problems go to *d_status.
+ */
+#ifndef WC_SPLIT12_H
+#define WC_SPLIT12_H
+
+#include <stdint.h>
+
+#include "wc.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Largest container for n values (at most 15n/16 of them can be exceptions:
+ * the 16 most frequent high bytes hold at least n/16 of the values). */
+WC_API uint64_t wc12_encode_bound(uint64_t n);
+
+/* Device scratch wc12_encode needs for n values (2,560 B plus 1 KiB per
+ * 65,536-value chunk). */
+WC_API uint64_t wc12_scratch_bytes(uint64_t n);
+
+/* Encode n bf16 values (d_in, 16-byte aligned) into d_out (16-byte aligned,
+ * out_cap >= wc12_encode_bound(n)); the container's size goes to the device
+ * u64 *d_out_size.  d_scratch: 16-byte aligned, wc12_scratch_bytes(n) bytes.
+ * Returns WC_OK, WC_ERR_INVALID_ARG, WC_ERR_CAPACITY or WC_ERR_CUDA. */
+WC_API int32_t wc12_encode(const void *d_in, uint64_t n, void *d_out, uint64_t out_cap,
+                           void *d_scratch, uint64_t scratch_cap, uint64_t *d_out_size,
+                           void *stream);
+
+/* Decode a container (d_cont, cont_bytes, 16-byte aligned) into out_cap bytes
+ * at d_out (16-byte aligned).  *d_status (device i32, set to 0 by the caller)
+ * receives WC_ERR_CORRUPT for a bad header, offset table, index >= K or
+ * exception position, WC_ERR_CAPACITY if 2n > out_cap; the output is then
+ * unspecified but nothing outside [d_out, d_out + out_cap) is written.
+ * Returns WC_OK, WC_ERR_INVALID_ARG or WC_ERR_CUDA. */
+WC_API int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out, uint64_t out_cap,
+                           int32_t *d_status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* WC_SPLIT12_H */

@@ -210,3 +210,33 @@ def test_header_fuzz_agrees_with_oracle(wcm, orc, dt):
             for k in range(a[2]):
                 wcm.chunk_ranges(c[:off_raw], k)
     assert both < 600   # most flips must be caught
+
+
+def test_split12_sizes_match_the_oracle_layout(wcm):
+    import split12 as s12
+    for n in (0, 1, 15, 16, 17, 65535, 65536, 65537, 5 * 65536 + 3):
+        ne_max = n - (n + 15) // 16
+        assert wcm.split12_encode_bound(n) == s12.layout(n, ne_max)["total"]
+        assert wcm.split12_scratch_bytes(n) == 2560 + 1024 * (-(-n // 65536))
+    # every bf16 pattern once: 240 of 256 high bytes missed, exactly the bound
+    every = np.arange(1 << 16, dtype=np.uint16)
+    assert s12.encode(every).size == wcm.split12_encode_bound(1 << 16)
+
+
+def test_split12_bad_arguments_rejected_without_device(wcm):
+    L = wcm.load()
+    buf = (ctypes.c_uint8 * 4096)()
+    base = (ctypes.addressof(buf) + 255) // 256 * 256
+    n = 100
+    cap, scr = wcm.split12_encode_bound(n), wcm.split12_scratch_bytes(n)
+    assert L.wc12_encode(base + 2, n, base, cap, base, scr, base, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_encode(base, n, base + 8, cap, base, scr, base, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_encode(base, n, base, cap, base + 4, scr, base, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_encode(base, n, base, cap, base, scr, base + 4, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_encode(None, n, base, cap, base, scr, base, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_encode(base, n, base, cap - 1, base, scr, base, None) == wcm.ERR_CAPACITY
+    assert L.wc12_encode(base, n, base, cap, base, scr - 1, base, None) == wcm.ERR_CAPACITY
+    assert L.wc12_decode(base + 4, 1000, base, 200, base, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_decode(base, 1000, base + 2, 200, base, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_decode(base, 1000, base, 200, None, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_decode(base, 1000, None, 200, base, None) == wcm.ERR_INVALID_ARG

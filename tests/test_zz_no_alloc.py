@@ -6,7 +6,7 @@ array the library holds; this file checks, through the C ABI, that its
 containers are byte-identical to wc_encode's (which gets scratch from the
 caller) on calls in a row, and that inputs too large for the array are
 refused before any work is queued.  Kept in a file of its own that pytest
-collects last."""
+collects after the parity files."""
 import ctypes
 
 import numpy as np

@@ -1,0 +1,120 @@
+"""Split12 serving format on the GPU (wc12_encode / wc12_decode through the C
+ABI) against the numpy oracle (oracle/split12.py): containers byte-identical
+for ragged sizes, exceptions in several chunks and steps, every bf16 pattern,
+weight-like tensors; decoding of oracle-written containers; damaged
+containers refused exactly when the oracle refuses them.  Collected after the
+other GPU files."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+C = 65536
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from fp32_weight_compression_b200 import build
+    build.build()
+
+
+@pytest.fixture(scope="module")
+def s12():
+    import split12
+    return split12
+
+
+def _dev(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to("cuda")
+
+
+def _check(s12, bits):
+    from fp32_weight_compression_b200 import wc
+    want = s12.encode(bits)
+    cont = wc.split12_encode(_dev(bits))
+    got = cont.cpu().numpy()
+    assert got.size == want.size, (got.size, want.size)
+    if not np.array_equal(got, want):
+        diff = np.nonzero(got != want)[0]
+        raise AssertionError(f"{diff.size} bytes differ, first at {diff[:8].tolist()}")
+    back = wc.split12_decode(cont)
+    assert np.array_equal(back.view(torch.int16).cpu().numpy().view(np.uint16), bits)
+
+
+@pytest.mark.parametrize("n", [0, 1, 2, 15, 16, 17, 31, 4095, 4096, 4097, C - 1, C, C + 1,
+                               3 * C + 4099])
+def test_sizes(s12, n):
+    _check(s12, workloads.generate_tensor(4, 1)[:n].copy())
+
+
+def test_exceptions_across_chunks_and_steps(s12):
+    b = workloads.generate_tensor(4, 1)[: 3 * C + 4099].copy()
+    rng = np.random.default_rng(5)
+    # rare high bytes spread over every chunk, in the first and last step of a
+    # chunk, in neighbouring values and in the ragged tail
+    pos = np.concatenate([[0, 1, 2, 15, 16, 4095, 4096, C - 1, C, 2 * C + 17, 3 * C + 4098],
+                          rng.choice(b.size, 300, replace=False)])
+    b[pos] = (rng.integers(0x40, 0x80, pos.size) << 8 | rng.integers(0, 256, pos.size)).astype(np.uint16)
+    _check(s12, b)
+
+
+def test_every_pattern_and_tiny_alphabets(s12):
+    _check(s12, np.arange(1 << 16, dtype=np.uint16))                      # ne at its bound
+    _check(s12, np.full(3 * C + 5, 0x3F80, np.uint16))                    # K = 1
+    _check(s12, (np.arange(5 * C, dtype=np.uint16) % 16) << 8 | 0x55)     # K = 16, no exception
+
+
+def test_weight_sets(s12):
+    for cid, i in ((1, 0), (2, 0), (2, 196), (2, 200), (4, 4)):
+        b = workloads.generate_tensor(cid, i)
+        if b.size > 60_000_000:
+            b = b[: 60_000_000 // C * C + 777]
+        _check(s12, b)
+
+
+def test_decodes_oracle_containers_and_refuses_damage(s12):
+    from fp32_weight_compression_b200 import wc
+    b = workloads.generate_tensor(4, 1)[: 2 * C + 999].copy()
+    b[[3, C + 5, 2 * C + 998]] = 0x7001
+    good = s12.encode(b)
+    rng = np.random.default_rng(9)
+    cases = [good]
+    for _ in range(60):
+        c = good.copy()
+        for _ in range(int(rng.integers(1, 3))):
+            region = int(rng.integers(0, 3))
+            if region == 0:
+                p = int(rng.integers(0, 96))                 # header, codebook, table start
+            elif region == 1:
+                p = int(rng.integers(0, c.size))            # anywhere
+            else:
+                p = int(rng.integers(c.size - 64, c.size))  # the exception lists
+            c[p] ^= np.uint8(rng.integers(1, 256))
+        cases.append(c)
+    cases.append(good[:-16])
+    for c in cases:
+        try:
+            want = s12.decode(c)
+        except ValueError:
+            want = None
+        d = torch.zeros(c.size + 64, dtype=torch.uint8, device="cuda")
+        d[: c.size] = torch.from_numpy(c)
+        # room for a flipped n that still gives a valid, slightly longer
+        # header; a guard region after it must stay untouched
+        room = b.size + 1024
+        out = torch.full((room + 2048,), 0x5A5A, dtype=torch.int16, device="cuda")
+        status = torch.zeros(1, dtype=torch.int32, device="cuda")
+        assert wc.load().wc12_decode(d.data_ptr(), c.size, out.data_ptr(), 2 * room,
+                                     status.data_ptr(), torch.cuda.current_stream().cuda_stream) == 0
+        torch.cuda.synchronize()
+        st = int(status.item())
+        assert bool((out[room:] == 0x5A5A).all().item())
+        if want is None:
+            assert st != 0
+        else:
+            assert st == 0
+            assert np.array_equal(out[: want.size].cpu().numpy().view(np.uint16), want)
