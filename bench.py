@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--tensors", type=int, default=0,
                     help="profiling only: use the first N tensors of the set (0: all)")
     ap.add_argument("--no-e2e", action="store_true", help="profiling only: skip the e2e leg")
+    ap.add_argument("--split12", action="store_true",
+                    help="also time the Split12 serving format (wc12_encode / wc12_decode) on the "
+                         "same tensors, outside the timed step; adds a 'split12' object")
     ap.add_argument("--checksum", action="store_true",
                     help="also time wc_crc32_blocks (1 MiB blocks) over the container arena, "
                          "outside the timed step; adds a 'checksum' object to the line")
@@ -293,6 +296,59 @@ def e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world):
 
 
 # ---------------------------------------------------------------------------
+def split12_leg(ins, dev, stream, reps: int = 5):
+    """wc12_encode / wc12_decode over every tensor of the set (one call per
+    tensor, back to back on one stream), containers checked bit-exact once.
+    Algorithmic bytes: encode reads the input twice (histogram, pack) and
+    writes the container; decode reads the container and writes the values."""
+    import torch
+    from fp32_weight_compression_b200 import wc
+    L = wc.load()
+    outs, scrs, sizes = [], [], []
+    for t in ins:
+        n = t.numel()
+        outs.append(torch.empty(wc.split12_encode_bound(n), dtype=torch.uint8, device=dev))
+        scrs.append(torch.empty(wc.split12_scratch_bytes(n), dtype=torch.uint8, device=dev))
+        sizes.append(torch.zeros(1, dtype=torch.int64, device=dev))
+    vals = [torch.empty_like(t) for t in ins]
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    sh = stream.cuda_stream
+
+    def enc():
+        for t, o, sc, z in zip(ins, outs, scrs, sizes):
+            wc._check(L.wc12_encode(t.data_ptr(), t.numel(), o.data_ptr(), o.numel(), sc.data_ptr(),
+                                    sc.numel(), z.data_ptr(), sh), "wc12_encode")
+
+    def dec():
+        for o, v in zip(outs, vals):
+            wc._check(L.wc12_decode(o.data_ptr(), o.numel(), v.data_ptr(), 2 * v.numel(),
+                                    status.data_ptr(), sh), "wc12_decode")
+
+    enc()
+    dec()
+    torch.cuda.synchronize(dev)
+    assert int(status.item()) == 0 and all(torch.equal(a, b) for a, b in zip(vals, ins))
+    total = int(sum(int(z.item()) for z in sizes))
+    B = sum(t.numel() * 2 for t in ins)
+    res = {}
+    for name, fn, alg in (("encode", enc, 2 * B + total), ("decode", dec, total + B)):
+        for _ in range(2):
+            fn()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        t = a.elapsed_time(b) / reps / 1e3
+        res[name] = {"ms": t * 1e3, "gbs": B / t / 1e9, "hbm_gbs": alg / t / 1e9,
+                     "algorithmic_bytes": alg}
+    res["ratio"] = total / B
+    res["launches_per_tensor"] = {"encode": 6, "decode": 1}
+    return res
+
+
 def checksum_leg(arena, dev, stream, reps: int = 10):
     """wc_crc32_blocks over the whole container arena (larger than L2), 1 MiB
     blocks: algorithmic bytes = the arena's bytes read (the CRCs written are
@@ -412,6 +468,7 @@ def main():
 
     t_e2e, E = e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world)
     checksum = checksum_leg(enc.out, dev, stream) if args.checksum else None
+    s12 = split12_leg(ins, dev, stream) if args.split12 else None
 
     peak, peak_note = peak_hbm()
     B = total_in
@@ -459,6 +516,10 @@ def main():
     if checksum is not None:
         checksum["roofline_frac"] = checksum["gbs"] / peak
         line["checksum"] = checksum
+    if s12 is not None:
+        for leg in ("encode", "decode"):
+            s12[leg]["roofline_frac"] = s12[leg]["hbm_gbs"] / peak
+        line["split12"] = s12
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
