@@ -1,0 +1,375 @@
+// k_split12_linear.cu -- Y = X W^T with the weights W (N x K, bf16, row-major)
+// held as a Split12 container (include/wc_split12.h): the weight tile is
+// expanded from the index and low planes straight into the tensor cores'
+// shared-memory operand layout and multiplied with tcgen05.mma, accumulating
+// in tensor memory, so the weights cross HBM at 12 bits a value ("weight-
+// compression" README: Split12 serving, bf16 weights rebuilt on the fly).
+//
+// Work split.  A CTA owns 128 weight rows (the MMA's M) and a range of K;
+// the host splits K across CTAs until the grid covers the SMs, and the CTAs
+// of one row block add their partial sums into Y (fp32 atomics; Y is zeroed
+// first).  Per stage of 64 K-values:
+//   * thread r (128 threads) expands row r: 32 index bytes + 64 low bytes ->
+//     64 bf16, written as eight 16-byte rows of core matrices;
+//   * the tokens' X slice (n_mma x 64, rows past M zero) is copied the same
+//     way; the chunks' exceptions that fall in the tile are patched in;
+//   * one thread issues four MMAs (M = 128, N = n_mma = M rounded up to 16,
+//     K = 16) and commits them to the stage's mbarrier.
+// Two stages alternate, so the expansion of one overlaps the MMAs of the
+// other.  At the end each warp reads its 32 TMEM lanes (rows) and adds them
+// into Y.
+//
+// Operand layout (K-major, no swizzle): a core matrix is 8 rows x 16 bytes
+// stored as 128 contiguous bytes; the two 8-value halves of a K = 16 slice
+// are 128 bytes apart (leading byte offset) and consecutive 8-row groups 256
+// bytes apart (stride byte offset).  A slice of A is 16 groups = 4 KiB; a
+// slice of B is n_mma / 8 groups.
+//
+// Waits: every mbarrier wait is bounded; when one runs out the kernel records
+// WC_ERR_TIMEOUT, stops issuing, waits (bounded) for what it issued, frees its
+// tensor memory and returns.
+#include <cstdint>
+#include <mutex>
+
+#include "wc.h"
+#include "wc_split12.cuh"
+
+namespace wc12l {
+
+using wc12::kChunk;
+
+constexpr int kThreads = 128;
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr uint32_t kASlice = kBM * 16 * 2;   // bytes of one K = 16 slice of A
+constexpr uint32_t kAStage = 4 * kASlice;
+constexpr uint32_t kMaxTokens = 256;
+constexpr uint32_t kSpinLimit = 1u << 24;
+
+struct Params {
+  const uint8_t *w;
+  uint64_t w_bytes;
+  const uint16_t *x;  // [M, K]
+  float *y;           // [M, N]
+  uint32_t M, N, K;
+  uint32_t n_mma;     // M rounded up to 16
+  uint32_t per_split; // stages per CTA
+  uint32_t splits;
+  int32_t *status;
+};
+
+__host__ __device__ inline uint32_t b_stage_bytes(uint32_t n_mma) { return n_mma * kBK * 2; }
+__host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma) {
+  return 1024 + 2 * kAStage + 2 * b_stage_bytes(n_mma) + 64;
+}
+
+__device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// shared-memory matrix descriptor: K-major, no swizzle, LBO 128 B, SBO 256 B
+__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 16) | (uint64_t(256 >> 4) << 32) |
+         (uint64_t(1) << 46);
+}
+
+// instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128, N = n
+__device__ __forceinline__ uint32_t instr_desc(uint32_t n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((n >> 3) << 17) | ((uint32_t(kBM) >> 4) << 24);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+// true once the phase of the given parity has completed; false after the limit
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t i = 0; i < kSpinLimit; i++) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}"
+      ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(accumulate), "r"(0u)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void fence_after_sync() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_before_sync() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// byte offset of (row, k) in a stage laid out as K = 16 slices of core matrices
+__device__ __forceinline__ uint32_t op_offset(uint32_t row, uint32_t k, uint32_t slice_bytes) {
+  return (k >> 4) * slice_bytes + (row >> 3) * 256 + ((k >> 3) & 1) * 128 + (row & 7) * 16 + (k & 7) * 2;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant__ Params p) {
+  extern __shared__ uint8_t dyn[];
+  uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
+  uint8_t *a_st = base;                       // 2 x kAStage
+  uint8_t *b_st = base + 2 * kAStage;         // 2 x b_stage_bytes
+  const uint32_t b_bytes = b_stage_bytes(p.n_mma);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(b_st + 2 * b_bytes);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
+  int *flag = reinterpret_cast<int *>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t K = p.K, N = p.N;
+  const uint32_t n0 = blockIdx.x * kBM;
+  const uint32_t split = blockIdx.y;
+  const uint32_t total_stages = K / kBK;
+  const uint32_t s_begin = split * p.per_split;
+  const uint32_t s_end = s_begin + p.per_split < total_stages ? s_begin + p.per_split : total_stages;
+
+  // container header (every CTA checks; CTA (0, 0) reports)
+  const uint8_t *w = p.w;
+  const uint32_t *h32 = reinterpret_cast<const uint32_t *>(w);
+  const uint64_t *h64 = reinterpret_cast<const uint64_t *>(w);
+  const uint64_t n = h64[1], ne = h64[3];
+  const uint32_t kk = h32[1] >> 24;
+  bool ok = p.w_bytes >= 96 && h32[0] == wc12::kMagic && (h32[1] & 0xFFFFFFu) == (1u | (1u << 16)) &&
+            kk >= 1 && kk <= 16 && n == uint64_t(N) * K && ne <= n && h32[4] == uint32_t(kChunk);
+  wc12::Lay L{};
+  if (ok) {
+    L = wc12::lay(n, ne);
+    ok = h32[5] == uint32_t(L.nc) && h64[4] == L.off_idx && h64[5] == L.off_lo && h64[6] == L.off_exc &&
+         h64[7] == L.total && L.total <= p.w_bytes;
+  }
+  if (!ok || s_begin >= s_end) {
+    if (!ok && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) report(p.status, WC_ERR_CORRUPT);
+    return;
+  }
+  const uint4 book = *reinterpret_cast<const uint4 *>(w + wc12::kBookOff);
+  const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(w + wc12::kExcOffOff);
+  const uint16_t *exc_pos = reinterpret_cast<const uint16_t *>(w + L.off_exc);
+  const uint8_t *exc_val = w + L.off_excval;
+  const uint8_t *lo_plane = w + L.off_lo;
+  const uint64_t c_lo = uint64_t(n0) * K / kChunk, c_hi = (uint64_t(n0 + kBM) * K - 1) / kChunk;
+
+  // tensor memory: n_mma fp32 columns, rounded up to a power of two >= 32
+  uint32_t cols = 32;
+  while (cols < p.n_mma) cols <<= 1;
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 ::"r"(smem_u32(tmem_slot)), "r"(cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (tid == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    *flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  fence_before_sync();
+  __syncthreads();
+  fence_after_sync();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t idesc = instr_desc(p.n_mma);
+
+  uint32_t it = 0;
+  for (uint32_t st = s_begin; st < s_end; st++, it++) {
+    const uint32_t buf = it & 1u;
+    if (it >= 2) {  // this buffer's MMAs of two stages ago must be done
+      if (!mbar_wait(&bar[buf], ((it - 2) >> 1) & 1u)) {
+        if (tid == 0) report(p.status, WC_ERR_TIMEOUT);
+        *flag = 1;
+      }
+      __syncthreads();
+      if (*flag) break;
+    }
+    uint8_t *A = a_st + buf * kAStage;
+    uint8_t *B = b_st + buf * b_bytes;
+    const uint32_t k0 = st * kBK;
+
+    // A: row tid of the block, 64 values
+    {
+      const uint64_t f0 = uint64_t(n0 + tid) * K + k0;
+      const uint4 *iq = reinterpret_cast<const uint4 *>(w + L.off_idx + f0 / 2);
+      const uint4 *lq = reinterpret_cast<const uint4 *>(lo_plane + f0);
+      const uint4 i0 = __ldg(iq), i1 = __ldg(iq + 1);
+      const uint4 l0 = __ldg(lq), l1 = __ldg(lq + 1), l2 = __ldg(lq + 2), l3 = __ldg(lq + 3);
+      const uint32_t iw[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
+      const uint32_t lw[16] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w,
+                               l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
+#pragma unroll
+      for (int j = 0; j < 8; j++) {  // values 8j .. 8j + 7
+        const uint2 e0 = wc12::expand4(iw[j], book, lw[2 * j]);
+        const uint2 e1 = wc12::expand4(iw[j] >> 16, book, lw[2 * j + 1]);
+        *reinterpret_cast<uint4 *>(A + op_offset(tid, 8 * j, kASlice)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+      }
+    }
+    // B: the tokens' slice of X, rows >= M zero
+    for (uint32_t i = tid; i < p.n_mma * 8; i += kThreads) {
+      const uint32_t t = i >> 3, j = i & 7;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t < p.M) v = __ldg(reinterpret_cast<const uint4 *>(p.x + uint64_t(t) * K + k0 + 8 * j));
+      *reinterpret_cast<uint4 *>(B + op_offset(t, 8 * j, p.n_mma * 32)) = v;
+    }
+    __syncthreads();
+    // exceptions of the block's chunks that fall in this tile
+    for (uint64_t c = c_lo; c <= c_hi; c++) {
+      const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
+      if (e0 > e1 || e1 > ne) {
+        if (tid == 0) report(p.status, WC_ERR_CORRUPT);
+        continue;
+      }
+      const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
+      for (uint64_t e = e0 + tid; e < e1; e += kThreads) {
+        const uint32_t pos = exc_pos[e];
+        if (pos >= cnt) {
+          report(p.status, WC_ERR_CORRUPT);
+          continue;
+        }
+        const uint64_t f = c * kChunk + pos;
+        const uint64_t row = f / K, col = f % K;
+        if (row < n0 || row >= n0 + kBM || col < k0 || col >= k0 + kBK) continue;
+        *reinterpret_cast<uint16_t *>(A + op_offset(uint32_t(row - n0), uint32_t(col - k0), kASlice)) =
+            uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[f]);
+      }
+    }
+    fence_proxy_async();  // generic-proxy writes -> visible to the tensor cores
+    __syncthreads();
+    if (tid == 0) {
+      fence_after_sync();
+      const uint32_t a0 = smem_u32(A), b0 = smem_u32(B);
+#pragma unroll
+      for (uint32_t s = 0; s < 4; s++)
+        mma_bf16(tmem, operand_desc(a0 + s * kASlice), operand_desc(b0 + s * p.n_mma * 32), idesc,
+                 (it > 0 || s > 0) ? 1u : 0u);
+      mma_commit(&bar[buf]);
+    }
+  }
+
+  // wait for the last stage issued (its commit covers all earlier MMAs)
+  const uint32_t issued = it;
+  bool done = true;
+  if (issued > 0) {
+    const uint32_t last = issued - 1;
+    done = mbar_wait(&bar[last & 1u], (last >> 1) & 1u);
+    if (!done && tid == 0) report(p.status, WC_ERR_TIMEOUT);
+  }
+  fence_after_sync();
+  if (done && !*flag && issued > 0) {
+    const uint32_t row = n0 + 32 * warp + lane;
+    for (uint32_t c0 = 0; c0 < p.n_mma; c0 += 8) {
+      uint32_t v[8];
+      asm volatile(
+          "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+          : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+          : "r"(tmem + (uint32_t(32 * warp) << 16) + c0));
+      asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+      for (int i = 0; i < 8; i++) {
+        const uint32_t t = c0 + i;
+        if (t < p.M) {
+          float *dst = p.y + uint64_t(t) * N + row;
+          if (p.splits > 1) atomicAdd(dst, __uint_as_float(v[i]));
+          else *dst = __uint_as_float(v[i]);
+        }
+      }
+    }
+  }
+  fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    fence_after_sync();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(cols) : "memory");
+  }
+}
+
+__global__ void k12_zero(float *y, uint64_t count) {
+  for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
+       i += uint64_t(gridDim.x) * blockDim.x)
+    y[i] = 0.0f;
+}
+
+struct DevInfo {
+  int sms = 0;
+  bool attr = false;
+};
+
+DevInfo dev_info() {
+  static std::mutex mu;
+  static DevInfo cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DevInfo{};
+  std::lock_guard<std::mutex> lock(mu);
+  DevInfo &d = cache[dev];
+  if (d.sms == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DevInfo{};
+    d.attr = cudaFuncSetAttribute(k12_linear, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  int(smem_bytes(kMaxTokens))) == cudaSuccess;
+    d.sms = sms;
+  }
+  return d;
+}
+
+}  // namespace wc12l
+
+extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, uint32_t K,
+                               const void *d_x, uint32_t M, float *d_y, int32_t *d_status,
+                               void *stream) {
+  auto aligned = [](const void *q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; };
+  if (d_w == nullptr || d_x == nullptr || d_y == nullptr || d_status == nullptr) return WC_ERR_INVALID_ARG;
+  if (!aligned(d_w, 16) || !aligned(d_x, 16) || !aligned(d_y, 4) || !aligned(d_status, 4))
+    return WC_ERR_INVALID_ARG;
+  if (N == 0 || K == 0 || N % wc12l::kBM != 0 || K % wc12l::kBK != 0 || M == 0 || M > wc12l::kMaxTokens)
+    return WC_ERR_INVALID_ARG;
+  const wc12l::DevInfo di = wc12l::dev_info();
+  if (di.sms <= 0 || !di.attr) return WC_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  wc12l::Params p;
+  p.w = static_cast<const uint8_t *>(d_w);
+  p.w_bytes = w_bytes;
+  p.x = static_cast<const uint16_t *>(d_x);
+  p.y = d_y;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.n_mma = (M + 15) / 16 * 16;
+  p.status = d_status;
+  const uint32_t blocks = N / wc12l::kBM, stages = K / wc12l::kBK;
+  // split K until the grid covers the SMs twice, at least two stages a CTA
+  uint32_t splits = (2 * uint32_t(di.sms) + blocks - 1) / blocks;
+  if (splits > stages / 2) splits = stages / 2;
+  if (splits < 1) splits = 1;
+  p.per_split = (stages + splits - 1) / splits;
+  p.splits = (stages + p.per_split - 1) / p.per_split;
+  if (p.splits > 1) {
+    wc12l::k12_zero<<<unsigned(2 * di.sms), 256, 0, s>>>(d_y, uint64_t(M) * N);
+  }
+  dim3 grid(blocks, p.splits);
+  wc12l::k12_linear<<<grid, wc12l::kThreads, wc12l::smem_bytes(p.n_mma), s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+}

@@ -120,6 +120,7 @@ const char *wc_status_string(int32_t st) {
     case WC_ERR_CUDA: return "WC_ERR_CUDA";
     case WC_ERR_CORRUPT: return "WC_ERR_CORRUPT";
     case WC_ERR_UNSUPPORTED: return "WC_ERR_UNSUPPORTED";
+    case WC_ERR_TIMEOUT: return "WC_ERR_TIMEOUT";
     default: return "WC_ERR_UNKNOWN";
   }
 }

@@ -15,7 +15,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libwc.so")
 
-OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CUDA, ERR_CORRUPT, ERR_UNSUPPORTED = 0, 1, 2, 3, 4, 5
+OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CUDA, ERR_CORRUPT, ERR_UNSUPPORTED, ERR_TIMEOUT = 0, 1, 2, 3, 4, 5, 6
 BF16, FP32, FP16, FP8E4M3 = 1, 2, 3, 4
 CHUNK = 65536
 
@@ -120,6 +120,8 @@ def load() -> ctypes.CDLL:
     L.wc12_encode.argtypes = [vp, u64, vp, u64, vp, u64, vp, vp]
     L.wc12_decode.restype = i32
     L.wc12_decode.argtypes = [vp, u64, vp, u64, vp, vp]
+    L.wc12_linear.restype = i32
+    L.wc12_linear.argtypes = [vp, u64, u32, u32, vp, u32, vp, vp, vp]
     L.wc_crc32_blocks.restype = i32
     L.wc_crc32_blocks.argtypes = [vp, u64, u64, vp, vp]
     _lib = L
@@ -446,6 +448,22 @@ def split12_decode(cont: torch.Tensor, shape=None, out=None, stream=None) -> tor
     if st != OK:
         raise WCError(st, "wc12_decode (device status)")
     return out
+
+
+def split12_linear(cont: torch.Tensor, N: int, K: int, x: torch.Tensor, stream=None) -> torch.Tensor:
+    """Y = x W^T (fp32, M x N) with W (N x K bf16) given as a Split12
+    container on the device (wc12_linear)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != K:
+        raise ValueError("x must be a 2-D bf16 tensor with K columns")
+    xf = x.contiguous()
+    y = torch.empty(x.shape[0], N, dtype=torch.float32, device=x.device)
+    status = torch.zeros(1, dtype=torch.int32, device=x.device)
+    _check(load().wc12_linear(cont.data_ptr(), cont.numel(), N, K, xf.data_ptr(), x.shape[0],
+                              y.data_ptr(), status.data_ptr(), _stream(stream)), "wc12_linear")
+    st = int(status.item())
+    if st != OK:
+        raise WCError(st, "wc12_linear (device status)")
+    return y
 
 
 CRC_BLOCK = 1 << 20

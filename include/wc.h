@@ -73,7 +73,8 @@ typedef enum {
     WC_ERR_CAPACITY = 2,
     WC_ERR_CUDA = 3,
     WC_ERR_CORRUPT = 4,
-    WC_ERR_UNSUPPORTED = 5
+    WC_ERR_UNSUPPORTED = 5,
+    WC_ERR_TIMEOUT = 6      /* a kernel's bounded wait ran out (device status) */
 } wc_status;
 
 /* WC_FP16: after the reorder S E M -> E S M an fp16 value is cut into its

@@ -68,6 +68,21 @@ WC_API int32_t wc12_encode(const void *d_in, uint64_t n, void *d_out, uint64_t o
 WC_API int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out, uint64_t out_cap,
                            int32_t *d_status, void *stream);
 
+/* Y = X W^T with W (N x K bf16, row-major) given as a Split12 container:
+ * the weights are expanded tile by tile into the tensor cores' operand
+ * layout and multiplied with tcgen05.mma (fp32 accumulate), so they cross
+ * HBM at 12 bits a value.
+ *   d_w, w_bytes  the container (16-byte aligned), n = N * K
+ *   N, K          N a multiple of 128, K a multiple of 64
+ *   d_x           M x K bf16, row-major, 16-byte aligned; 1 <= M <= 256
+ *   d_y           M x N fp32, row-major (overwritten)
+ *   d_status      device i32 set to 0 by the caller: WC_ERR_CORRUPT for a bad
+ *                 container, WC_ERR_TIMEOUT if a bounded wait ran out
+ * Returns WC_OK, WC_ERR_INVALID_ARG or WC_ERR_CUDA. */
+WC_API int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, uint32_t K,
+                           const void *d_x, uint32_t M, float *d_y, int32_t *d_status,
+                           void *stream);
+
 #ifdef __cplusplus
 }
 #endif

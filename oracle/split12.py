@@ -169,3 +169,18 @@ def canonical(cont: np.ndarray) -> bool:
     c = np.ascontiguousarray(cont, dtype=np.uint8)
     vals = decode(c)
     return c.size == read_header(c)["total"] and np.array_equal(encode(vals), c)
+
+
+def linear(x_bits: np.ndarray, cont: np.ndarray, n_rows: int) -> np.ndarray:
+    """Y = X W^T in float64, W (n_rows x K, bf16) decoded from a container and
+    X (M x K) given as bf16 bits: the exact products of the bf16 values,
+    summed in float64 (the reference a fused decode-and-multiply kernel is
+    held to within its fp32 accumulation bound)."""
+    w = decode(cont)
+    k = w.size // n_rows
+    if n_rows * k != w.size:
+        raise ValueError("container size is not a multiple of the row count")
+    to_f = lambda b: (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
+    wf = to_f(w).astype(np.float64).reshape(n_rows, k)
+    xf = to_f(x_bits).astype(np.float64).reshape(-1, k)
+    return xf @ wf.T

@@ -240,3 +240,21 @@ def test_split12_bad_arguments_rejected_without_device(wcm):
     assert L.wc12_decode(base, 1000, base + 2, 200, base, None) == wcm.ERR_INVALID_ARG
     assert L.wc12_decode(base, 1000, base, 200, None, None) == wcm.ERR_INVALID_ARG
     assert L.wc12_decode(base, 1000, None, 200, base, None) == wcm.ERR_INVALID_ARG
+
+
+def test_split12_linear_bad_arguments_rejected_without_device(wcm):
+    L = wcm.load()
+    buf = (ctypes.c_uint8 * 4096)()
+    b = (ctypes.addressof(buf) + 255) // 256 * 256
+    ok = dict(N=256, K=128, M=4)
+    def call(w=b, N=ok["N"], K=ok["K"], x=b, M=ok["M"], y=b, st=b):
+        return L.wc12_linear(w, 1 << 20, N, K, x, M, y, st, None)
+    assert call(N=100) == wcm.ERR_INVALID_ARG          # N not a multiple of 128
+    assert call(K=96) == wcm.ERR_INVALID_ARG           # K not a multiple of 64
+    assert call(M=0) == wcm.ERR_INVALID_ARG
+    assert call(M=257) == wcm.ERR_INVALID_ARG
+    assert call(w=b + 8) == wcm.ERR_INVALID_ARG        # container not 16-byte aligned
+    assert call(x=b + 8) == wcm.ERR_INVALID_ARG
+    assert call(y=b + 2) == wcm.ERR_INVALID_ARG
+    assert call(w=None) == wcm.ERR_INVALID_ARG
+    assert call(st=None) == wcm.ERR_INVALID_ARG

@@ -128,3 +128,21 @@ def test_non_canonical_detected(s12):
     # the valid container of other values is canonical
     c = good.copy(); c[79] = 0x3E
     assert s12.canonical(c)
+
+
+def test_linear_worked_example(s12):
+    # W = [[1, 2, -1], [0.5, 4, 3]] and x = [1, -2, 3] as bf16 bits;
+    # x W^T = [1 - 4 - 3, 0.5 - 8 + 9] = [-6, 1.5], worked by hand
+    w = np.array([0x3F80, 0x4000, 0xBF80, 0x3F00, 0x4080, 0x4040], np.uint16)
+    x = np.array([[0x3F80, 0xC000, 0x4040]], np.uint16)
+    y = s12.linear(x, s12.encode(w), 2)
+    assert y.shape == (1, 2) and y.tolist() == [[-6.0, 1.5]]
+    # two tokens, one with an exception in W (18 distinct high bytes)
+    # 18 powers of four: exponents two apart, so 18 distinct high bytes
+    vals = np.array([4.0 ** e for e in range(-9, 9)], np.float32)
+    wb = (vals.view(np.uint32) >> 16).astype(np.uint16)               # exact in bf16
+    xb = np.array([[0x3F80] * 18, [0x4000] * 9 + [0x0000] * 9], np.uint16)   # ones; twos then zeros
+    y = s12.linear(xb, s12.encode(wb), 1)
+    assert s12.read_header(s12.encode(wb))["ne"] == 2
+    assert y[0, 0] == vals.astype(np.float64).sum()
+    assert y[1, 0] == 2 * vals[:9].astype(np.float64).sum()
