@@ -9,8 +9,9 @@
 // the host splits K across CTAs until the grid covers the SMs, and the CTAs
 // of one row block add their partial sums into Y (fp32 atomics; Y is zeroed
 // first).  Per stage of 64 K-values:
-//   * thread r (128 threads) expands row r: 32 index bytes + 64 low bytes ->
-//     64 bf16, written as eight 16-byte rows of core matrices;
+//   * the 128 threads expand the block's 128 x 64 values in segments of 16
+//     (8 index bytes + 16 low bytes -> 16 bf16, two 16-byte rows of core
+//     matrices), four threads per row, so a warp's loads touch 8 lines;
 //   * the tokens' X slice (n_mma x 64, rows past M zero) is copied the same
 //     way; the chunks' exceptions that fall in the tile are patched in;
 //   * one thread issues four MMAs (M = 128, N = n_mma = M rounded up to 16,
@@ -151,12 +152,14 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   const uint32_t s_end = s_begin + p.per_split < total_stages ? s_begin + p.per_split : total_stages;
 
   // container header (every CTA checks; CTA (0, 0) reports)
+  // (the host refuses containers shorter than 96 bytes, so the header is
+  // inside the buffer)
   const uint8_t *w = p.w;
   const uint32_t *h32 = reinterpret_cast<const uint32_t *>(w);
   const uint64_t *h64 = reinterpret_cast<const uint64_t *>(w);
   const uint64_t n = h64[1], ne = h64[3];
   const uint32_t kk = h32[1] >> 24;
-  bool ok = p.w_bytes >= 96 && h32[0] == wc12::kMagic && (h32[1] & 0xFFFFFFu) == (1u | (1u << 16)) &&
+  bool ok = h32[0] == wc12::kMagic && (h32[1] & 0xFFFFFFu) == (1u | (1u << 16)) &&
             kk >= 1 && kk <= 16 && n == uint64_t(N) * K && ne <= n && h32[4] == uint32_t(kChunk);
   wc12::Lay L{};
   if (ok) {
@@ -211,22 +214,18 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     uint8_t *B = b_st + buf * b_bytes;
     const uint32_t k0 = st * kBK;
 
-    // A: row tid of the block, 64 values
-    {
-      const uint64_t f0 = uint64_t(n0 + tid) * K + k0;
-      const uint4 *iq = reinterpret_cast<const uint4 *>(w + L.off_idx + f0 / 2);
-      const uint4 *lq = reinterpret_cast<const uint4 *>(lo_plane + f0);
-      const uint4 i0 = __ldg(iq), i1 = __ldg(iq + 1);
-      const uint4 l0 = __ldg(lq), l1 = __ldg(lq + 1), l2 = __ldg(lq + 2), l3 = __ldg(lq + 3);
-      const uint32_t iw[8] = {i0.x, i0.y, i0.z, i0.w, i1.x, i1.y, i1.z, i1.w};
-      const uint32_t lw[16] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w,
-                               l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
+    // A: 512 segments of 16 values (row = i / 4, values 16 (i % 4) ..), four
+    // per thread; a warp covers 8 rows, so its loads touch 8 lines, not 32
 #pragma unroll
-      for (int j = 0; j < 8; j++) {  // values 8j .. 8j + 7
-        const uint2 e0 = wc12::expand4(iw[j], book, lw[2 * j]);
-        const uint2 e1 = wc12::expand4(iw[j] >> 16, book, lw[2 * j + 1]);
-        *reinterpret_cast<uint4 *>(A + op_offset(tid, 8 * j, kASlice)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-      }
+    for (int q = 0; q < 4; q++) {
+      const uint32_t i = uint32_t(tid) + kThreads * q, row = i >> 2, seg = i & 3;
+      const uint64_t f = uint64_t(n0 + row) * K + k0 + 16 * seg;
+      const uint2 iw = __ldg(reinterpret_cast<const uint2 *>(w + L.off_idx + f / 2));
+      const uint4 lw = __ldg(reinterpret_cast<const uint4 *>(lo_plane + f));
+      const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
+      const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
+      *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg, kASlice)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+      *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg + 8, kASlice)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
     }
     // B: the tokens' slice of X, rows >= M zero
     for (uint32_t i = tid; i < p.n_mma * 8; i += kThreads) {
@@ -346,6 +345,7 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
     return WC_ERR_INVALID_ARG;
   if (N == 0 || K == 0 || N % wc12l::kBM != 0 || K % wc12l::kBK != 0 || M == 0 || M > wc12l::kMaxTokens)
     return WC_ERR_INVALID_ARG;
+  if (w_bytes < 96) return WC_ERR_INVALID_ARG;  // shorter than any container's header
   const wc12l::DevInfo di = wc12l::dev_info();
   if (di.sms <= 0 || !di.attr) return WC_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -72,7 +72,7 @@ WC_API int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out,
  * the weights are expanded tile by tile into the tensor cores' operand
  * layout and multiplied with tcgen05.mma (fp32 accumulate), so they cross
  * HBM at 12 bits a value.
- *   d_w, w_bytes  the container (16-byte aligned), n = N * K
+ *   d_w, w_bytes  the container (16-byte aligned, at least 96 bytes), n = N * K
  *   N, K          N a multiple of 128, K a multiple of 64
  *   d_x           M x K bf16, row-major, 16-byte aligned; 1 <= M <= 256
  *   d_y           M x N fp32, row-major (overwritten)

@@ -258,3 +258,4 @@ def test_split12_linear_bad_arguments_rejected_without_device(wcm):
     assert call(y=b + 2) == wcm.ERR_INVALID_ARG
     assert call(w=None) == wcm.ERR_INVALID_ARG
     assert call(st=None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_linear(b, 95, 256, 128, b, 4, b, b, None) == wcm.ERR_INVALID_ARG   # no room for a header
