@@ -146,3 +146,24 @@ def test_linear_worked_example(s12):
     assert s12.read_header(s12.encode(wb))["ne"] == 2
     assert y[0, 0] == vals.astype(np.float64).sum()
     assert y[1, 0] == 2 * vals[:9].astype(np.float64).sum()
+
+
+def test_random_inputs_round_trip_within_the_bound(s12):
+    """Random alphabets and sizes: the oracle round-trips, its containers are
+    canonical, and no container exceeds the size the library reserves
+    (wc12_encode_bound: at most 15/16 of the values can be exceptions)."""
+    from fp32_weight_compression_b200 import build, wc
+    build.build()
+    rng = np.random.default_rng(77)
+    for trial in range(40):
+        n = int(rng.choice([1, 2, 17, 255, 4097, C + 3, 2 * C + 1]))
+        width = int(rng.integers(1, 257))
+        highs = rng.choice(256, width, replace=False)
+        p = rng.dirichlet(np.full(width, float(rng.choice([0.05, 1.0, 20.0]))))
+        hi = rng.choice(highs, n, p=p).astype(np.uint16)
+        bits = (hi << 8) | rng.integers(0, 256, n, dtype=np.uint16)
+        cont = s12.encode(bits)
+        assert np.array_equal(s12.decode(cont), bits)
+        assert cont.size <= wc.split12_encode_bound(n)
+        if trial % 8 == 0:
+            assert s12.canonical(cont)
