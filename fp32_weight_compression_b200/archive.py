@@ -16,8 +16,10 @@ Layout (little-endian):
            u64 container bytes, then (B > 0) one u32 CRC-32 per B-byte block
            of the container, the last block short
 
-The containers are exactly those of the library (include/wc.h); this module
-only places them in a file and finds them again.  Encoding, decoding and the
+The containers are exactly those of the library: the rANS storage format
+(include/wc.h, magic "WCZ1") or the Split12 serving format
+(include/wc_split12.h, magic "W12C", bf16 only), told apart by their magic;
+this module only places them in a file and finds them again.  Encoding, decoding and the
 checksums ("seedpack 0.2.0 -> 0.2.2", README: a CRC32 per archive chunk) run
 on the GPU through the binding.
 """
@@ -84,12 +86,20 @@ def write(path: str, entries, crc_block: int = 0) -> None:
         fh.write(index)
 
 
-def save(path: str, tensors: dict, stream=None, crc_block: int = wc.CRC_BLOCK) -> None:
-    """Encode every tensor (CUDA tensors; one batched launch per kernel),
-    checksum each container on the device (crc_block 0: none) and write them
-    to an archive under their names."""
+def save(path: str, tensors: dict, stream=None, crc_block: int = wc.CRC_BLOCK,
+         codec: str = "rans") -> None:
+    """Encode every tensor (CUDA tensors) and write the containers to an
+    archive under their names, each checksummed on the device (crc_block 0:
+    none).  codec "rans": the storage format, one batched launch per kernel;
+    "split12": the serving format (bf16 tensors only), which wc12_linear
+    multiplies without decoding."""
     items = list(tensors.items())
-    conts = wc.encode_batch([t.contiguous() for _, t in items], stream)
+    if codec == "rans":
+        conts = wc.encode_batch([t.contiguous() for _, t in items], stream)
+    elif codec == "split12":
+        conts = [wc.split12_encode(t.contiguous(), stream) for _, t in items]
+    else:
+        raise ValueError(f"unknown codec {codec!r}")
     crcs = [wc.crc32_blocks(c, crc_block, stream) if crc_block else None for c in conts]
     write(path, [(name, wc.dtype_code(t.dtype), tuple(t.shape), c.cpu().numpy().tobytes(),
                   None if k is None else k.cpu().numpy().view(np.uint32))
@@ -144,10 +154,17 @@ class Archive:
                 raise ValueError(f"entry {name!r}: unknown dtype code {code}")
             if name in self._entries:
                 raise ValueError(f"entry {name!r} appears twice")
-            n, hcode, _ = wc.read_header(bytes(self._mm[off:off + min(nbytes, 64)]))
+            head = bytes(self._mm[off:off + min(nbytes, 64)])
+            if head[:4] == b"W12C":
+                codec = "split12"
+                n, _, _ = wc.split12_read_header(head, nbytes)
+                hcode = wc.BF16
+            else:
+                codec = "rans"
+                n, hcode, _ = wc.read_header(head)
             if hcode != code or n != int(np.prod(shape, dtype=np.uint64)):
                 raise ValueError(f"entry {name!r}: container header disagrees with the index")
-            self._entries[name] = (code, tuple(shape), off, nbytes, crcs)
+            self._entries[name] = (code, tuple(shape), off, nbytes, crcs, codec)
         if p != ioff + ibytes:
             raise ValueError("index size does not match its entries")
 
@@ -172,8 +189,12 @@ class Archive:
 
     def info(self, name: str) -> tuple[torch.dtype, tuple, int]:
         """(dtype, shape, container bytes) of an entry."""
-        code, shape, _, nbytes, _ = self._entries[name]
+        code, shape, _, nbytes = self._entries[name][:4]
         return wc._TORCH_DT[code], shape, nbytes
+
+    def codec(self, name: str) -> str:
+        """"rans" (storage format) or "split12" (serving format)."""
+        return self._entries[name][5]
 
     def checksums(self, name: str) -> np.ndarray:
         """The stored CRC-32 of each checksum block of the entry's container
@@ -182,8 +203,14 @@ class Archive:
 
     def container(self, name: str) -> np.ndarray:
         """A copy of the entry's container bytes."""
-        _, _, off, nbytes, _ = self._entries[name]
+        _, _, off, nbytes = self._entries[name][:4]
         return np.frombuffer(self._mm, dtype=np.uint8, count=nbytes, offset=off).copy()
+
+    def device_container(self, name: str, device="cuda", stream=None, verify: bool = True) -> torch.Tensor:
+        """The entry's container on the device (checksums checked unless
+        verify is False): the operand wc.split12_linear takes for a Split12
+        entry."""
+        return self._device_container(name, device, verify, stream)
 
     def _device_container(self, name: str, device, verify: bool, stream) -> torch.Tensor:
         cont = torch.from_numpy(self.container(name)).to(device)
@@ -211,6 +238,8 @@ class Archive:
         verify is False; a mismatch raises ValueError)."""
         code, shape = self._entries[name][:2]
         cont = self._device_container(name, device, verify, stream)
+        if self.codec(name) == "split12":
+            return wc.split12_decode(cont, shape=shape, stream=stream)
         return wc.decode(cont, shape=shape, dtype=wc._TORCH_DT[code], stream=stream)
 
     def load_chunk(self, name: str, k: int, device="cuda", stream=None,
@@ -219,7 +248,9 @@ class Archive:
         Only the bytes the chunk needs leave the file: the header and tables,
         the chunk's raw-plane bytes and its payload (wc_chunk_ranges), widened
         to whole checksum blocks when those are checked."""
-        code, _, off, nbytes, crcs = self._entries[name]
+        code, _, off, nbytes, crcs, codec = self._entries[name]
+        if codec != "rans":
+            raise ValueError(f"entry {name!r}: chunk access needs the rANS storage format")
         (off_raw,) = struct.unpack_from("<Q", self._mm, off + 32)
         if off_raw > nbytes:
             raise ValueError(f"entry {name!r}: container header out of range")
@@ -243,10 +274,15 @@ class Archive:
         return wc.decode_chunk(cont, k, dtype=wc._TORCH_DT[code], stream=stream)
 
     def load_all(self, names=None, device="cuda", stream=None, verify: bool = True) -> dict:
-        """Decode several tensors with one batched launch."""
+        """Decode several tensors: the rANS entries with one batched launch,
+        Split12 entries one call each."""
         names = self.names() if names is None else list(names)
-        conts = [self._device_container(n, device, verify, stream) for n in names]
-        shapes = [self._entries[n][1] for n in names]
-        dtypes = [wc._TORCH_DT[self._entries[n][0]] for n in names]
-        outs = wc.decode_batch(conts, shapes, dtypes, stream)
-        return dict(zip(names, outs))
+        rans = [n for n in names if self.codec(n) == "rans"]
+        conts = [self._device_container(n, device, verify, stream) for n in rans]
+        shapes = [self._entries[n][1] for n in rans]
+        dtypes = [wc._TORCH_DT[self._entries[n][0]] for n in rans]
+        got = dict(zip(rans, wc.decode_batch(conts, shapes, dtypes, stream)))
+        for n in names:
+            if n not in got:
+                got[n] = self.load(n, device, stream, verify)
+        return {n: got[n] for n in names}

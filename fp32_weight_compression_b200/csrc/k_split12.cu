@@ -21,6 +21,7 @@
 // registers; byte permutes do the lookup), then patches the chunk's
 // exceptions after a block barrier.
 #include <cstdint>
+#include <cstring>
 #include <mutex>
 
 #include "wc.h"
@@ -444,6 +445,28 @@ int32_t wc12_encode(const void *d_in, uint64_t n, void *d_out, uint64_t out_cap,
   if (nc) wc12::k12_pack<<<unsigned(nc), wc12::kPackThreads, 0, s>>>(in, n, out, scr);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return WC_ERR_CUDA;
+  return WC_OK;
+}
+
+int32_t wc12_read_header(const void *h_cont, uint64_t bytes, uint64_t *n, uint64_t *ne, uint32_t *k) {
+  if (h_cont == nullptr || n == nullptr || ne == nullptr || k == nullptr) return WC_ERR_INVALID_ARG;
+  if (bytes < 96) return WC_ERR_CORRUPT;
+  uint32_t h32[16];
+  memcpy(h32, h_cont, 64);
+  uint64_t h64[8];
+  memcpy(h64, h_cont, 64);
+  const uint64_t nn = h64[1], nne = h64[3];
+  const uint32_t kk = h32[1] >> 24;
+  if (h32[0] != wc12::kMagic || (h32[1] & 0xFFFFFFu) != (1u | (1u << 16)) || kk > 16 ||
+      (nn > 0) != (kk > 0) || nn > wc12::kMaxN || nne > nn || h32[4] != uint32_t(wc12::kChunk))
+    return WC_ERR_CORRUPT;
+  const wc12::Lay L = wc12::lay(nn, nne);
+  if (h32[5] != uint32_t(L.nc) || h64[4] != L.off_idx || h64[5] != L.off_lo || h64[6] != L.off_exc ||
+      h64[7] != L.total || L.total > bytes)
+    return WC_ERR_CORRUPT;
+  *n = nn;
+  *ne = nne;
+  *k = kk;
   return WC_OK;
 }
 

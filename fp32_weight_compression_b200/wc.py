@@ -120,6 +120,8 @@ def load() -> ctypes.CDLL:
     L.wc12_encode.argtypes = [vp, u64, vp, u64, vp, u64, vp, vp]
     L.wc12_decode.restype = i32
     L.wc12_decode.argtypes = [vp, u64, vp, u64, vp, vp]
+    L.wc12_read_header.restype = i32
+    L.wc12_read_header.argtypes = [vp, u64, ctypes.POINTER(u64), ctypes.POINTER(u64), ctypes.POINTER(u32)]
     L.wc12_linear.restype = i32
     L.wc12_linear.argtypes = [vp, u64, u32, u32, vp, u32, vp, vp, vp]
     L.wc_crc32_blocks.restype = i32
@@ -416,6 +418,22 @@ def split12_encode_bound(n: int) -> int:
 
 def split12_scratch_bytes(n: int) -> int:
     return int(load().wc12_scratch_bytes(n))
+
+
+def split12_read_header(cont, cont_bytes: int | None = None) -> tuple[int, int, int]:
+    """(n, exceptions, codebook entries) of a Split12 container, from a host
+    copy of (at least) its first 64 bytes (bytes or uint8 array); cont_bytes
+    is the container's size (default: the copy's)."""
+    import numpy as np
+    buf = np.ascontiguousarray(np.frombuffer(cont, np.uint8) if isinstance(cont, (bytes, bytearray))
+                               else cont, dtype=np.uint8)
+    size = buf.size if cont_bytes is None else int(cont_bytes)
+    if buf.size < 64:
+        raise WCError(ERR_CORRUPT, "wc12_read_header")
+    n, ne, k = ctypes.c_uint64(), ctypes.c_uint64(), ctypes.c_uint32()
+    _check(load().wc12_read_header(buf.ctypes.data, size, ctypes.byref(n), ctypes.byref(ne),
+                                   ctypes.byref(k)), "wc12_read_header")
+    return n.value, ne.value, k.value
 
 
 def split12_encode(t: torch.Tensor, stream=None) -> torch.Tensor:

@@ -59,6 +59,15 @@ WC_API int32_t wc12_encode(const void *d_in, uint64_t n, void *d_out, uint64_t o
                            void *d_scratch, uint64_t scratch_cap, uint64_t *d_out_size,
                            void *stream);
 
+/* Header of a container of `bytes` bytes, read from a host copy of its first
+ * 64 bytes (h_cont): n, exceptions, codebook entries.  Checks what
+ * wc12_decode checks of the header and layout (magic, version, dtype, K,
+ * chunk size and count, section offsets, total <= bytes; fewer than 96 bytes
+ * is corrupt).  Returns WC_OK, WC_ERR_INVALID_ARG (null pointer) or
+ * WC_ERR_CORRUPT.  Host only. */
+WC_API int32_t wc12_read_header(const void *h_cont, uint64_t bytes, uint64_t *n, uint64_t *ne,
+                                uint32_t *k);
+
 /* Decode a container (d_cont, cont_bytes, 16-byte aligned) into out_cap bytes
  * at d_out (16-byte aligned).  *d_status (device i32, set to 0 by the caller)
  * receives WC_ERR_CORRUPT for a bad header, offset table, index >= K or

@@ -259,3 +259,30 @@ def test_split12_linear_bad_arguments_rejected_without_device(wcm):
     assert call(w=None) == wcm.ERR_INVALID_ARG
     assert call(st=None) == wcm.ERR_INVALID_ARG
     assert L.wc12_linear(b, 95, 256, 128, b, 4, b, b, None) == wcm.ERR_INVALID_ARG   # no room for a header
+
+
+def test_split12_read_header_matches_the_oracle(wcm):
+    import split12 as s12
+    rng = np.random.default_rng(12)
+    for n in (0, 1, 17, 65537):
+        bits = (rng.integers(0, 40, n).astype(np.uint16) << 8) | rng.integers(0, 256, n).astype(np.uint16)
+        cont = s12.encode(bits)
+        h = s12.read_header(cont)
+        assert wcm.split12_read_header(cont) == (h["n"], h["ne"], h["k"])
+        # the library's header checks refuse what the oracle's refuse
+        for _ in range(200):
+            c = cont.copy()
+            c[int(rng.integers(0, 64))] ^= np.uint8(rng.integers(1, 256))
+            try:
+                s12.read_header(c)
+                ok = True
+            except ValueError:
+                ok = False
+            try:
+                wcm.split12_read_header(c)
+                got = True
+            except wcm.WCError:
+                got = False
+            assert got == ok
+        with pytest.raises(wcm.WCError):
+            wcm.split12_read_header(cont[:-1])

@@ -153,3 +153,35 @@ def test_checksums_stored_and_read_back(orc, arc, tmp_path):
     arc.write(path, [(n, c, s, cont.tobytes())])
     with arc.Archive(path) as a:
         assert a.crc_block == 0 and a.checksums(n).size == 0
+
+
+def test_split12_entries(orc, arc, tmp_path):
+    """Serving-format (Split12) containers stored beside rANS ones: told apart
+    by their magic, checked against the index, checksummed the same way."""
+    import split12 as s12
+    rng = np.random.default_rng(41)
+    b = workloads.rne_bf16(rng.standard_normal(C + 77).astype(np.float32) * np.float32(0.02))
+    b[[3, C + 5]] = 0x7A01
+    c12 = s12.encode(b)
+    crans = orc.encode(b)
+    path = str(tmp_path / "s.wca")
+    block = 8192
+    arc.write(path, [("w12", 1, (C + 77,), c12.tobytes(), orc.crc32_blocks(c12, block)),
+                     ("w", 1, (C + 77,), crans.tobytes(), orc.crc32_blocks(crans, block))],
+              crc_block=block)
+    with arc.Archive(path) as a:
+        assert a.codec("w12") == "split12" and a.codec("w") == "rans"
+        assert a.info("w12")[:2] == (a.info("w")[0], (C + 77,))
+        assert np.array_equal(a.container("w12"), c12)
+        assert np.array_equal(s12.decode(a.container("w12")), b)
+        assert np.array_equal(a.checksums("w12"), orc.crc32_blocks(c12, block))
+    # a Split12 entry must be bf16 and match the index's shape
+    for code, shape in ((2, (C + 77,)), (1, (C + 78,))):
+        arc.write(path, [("w12", code, shape, c12.tobytes())])
+        with pytest.raises(ValueError):
+            arc.Archive(path)
+    bad = c12.copy()
+    bad[20] ^= 1                                                   # chunk count
+    arc.write(path, [("w12", 1, (C + 77,), bad.tobytes())])
+    with pytest.raises(ValueError):
+        arc.Archive(path)

@@ -97,3 +97,28 @@ def test_checksums_catch_a_damaged_container(orc, tmp_path):
         # the other entries are untouched
         got = a.load("h16")
         assert np.array_equal(gu.to_bits(got).reshape(-1), ts["h16"][0])
+
+
+def test_split12_archive(orc, tmp_path):
+    import gpu_util as gu
+    import split12 as s12
+    from fp32_weight_compression_b200 import archive
+    ts = _tensors()
+    bf = {k: v for k, v in ts.items() if v[1].dtype == torch.bfloat16}
+    path = str(tmp_path / "serve.wca")
+    archive.save(path, {k: t for k, (_, t) in bf.items()}, codec="split12", crc_block=65536)
+    with archive.Archive(path) as a:
+        for k, (b, t) in bf.items():
+            assert a.codec(k) == "split12"
+            assert np.array_equal(a.container(k), s12.encode(b))
+            assert a.verify(k) == []
+            got = a.load(k)
+            assert got.dtype == torch.bfloat16 and tuple(got.shape) == tuple(t.shape)
+            assert np.array_equal(gu.to_bits(got).reshape(-1), b)
+            dc = a.device_container(k)
+            assert dc.is_cuda and np.array_equal(dc.cpu().numpy(), a.container(k))
+        allv = a.load_all()
+        for k, (b, t) in bf.items():
+            assert np.array_equal(gu.to_bits(allv[k]).reshape(-1), b)
+        with pytest.raises(ValueError):
+            a.load_chunk(next(iter(bf)), 0)
