@@ -298,12 +298,16 @@ def e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world):
 # ---------------------------------------------------------------------------
 def split12_leg(ins, dev, stream, reps: int = 5):
     """wc12_encode / wc12_decode over every tensor of the set (one call per
-    tensor, back to back on one stream), containers checked bit-exact once.
-    Algorithmic bytes: encode reads the input twice (histogram, pack) and
-    writes the container; decode reads the container and writes the values."""
+    tensor, back to back on one stream of its own), containers checked
+    bit-exact.  Algorithmic bytes: encode reads the input twice (histogram,
+    pack) and writes the container; decode reads the container and writes
+    the values.  Each pass is captured once in a CUDA graph and replayed
+    (one launch per kernel per tensor would otherwise be timed)."""
     import torch
     from fp32_weight_compression_b200 import wc
     L = wc.load()
+    side = torch.cuda.Stream(dev)       # graph capture needs a stream other than the default
+    side.wait_stream(stream)
     outs, scrs, sizes = [], [], []
     for t in ins:
         n = t.numel()
@@ -312,7 +316,7 @@ def split12_leg(ins, dev, stream, reps: int = 5):
         sizes.append(torch.zeros(1, dtype=torch.int64, device=dev))
     vals = [torch.empty_like(t) for t in ins]
     status = torch.zeros(1, dtype=torch.int32, device=dev)
-    sh = stream.cuda_stream
+    sh = side.cuda_stream
 
     def enc():
         for t, o, sc, z in zip(ins, outs, scrs, sizes):
@@ -324,33 +328,34 @@ def split12_leg(ins, dev, stream, reps: int = 5):
             wc._check(L.wc12_decode(o.data_ptr(), o.numel(), v.data_ptr(), 2 * v.numel(),
                                     status.data_ptr(), sh), "wc12_decode")
 
-    enc()
-    dec()
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(side)
+        for _ in range(reps):
+            fn()
+        b.record(side)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps / 1e3
+
+    with torch.cuda.stream(side):
+        enc()
+        dec()
     torch.cuda.synchronize(dev)
     assert int(status.item()) == 0 and all(torch.equal(a, b) for a, b in zip(vals, ins))
     total = int(sum(int(z.item()) for z in sizes))
     B = sum(t.numel() * 2 for t in ins)
-    def timed(fn):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize(dev)
-        a.record(stream)
-        for _ in range(reps):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        return a.elapsed_time(b) / reps / 1e3
-
     res = {}
     for name, fn, alg in (("encode", enc, 2 * B + total), ("decode", dec, total + B)):
-        for _ in range(2):
+        with torch.cuda.stream(side):
             fn()
         t_eager = timed(fn)
-        # the same launches captured once and replayed: per-launch host cost gone
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+        with torch.cuda.graph(g, stream=side):
             fn()
-        g.replay()
-        t = timed(g.replay)
+        with torch.cuda.stream(side):
+            g.replay()
+            t = timed(g.replay)
         del g
         res[name] = {"ms": t * 1e3, "gbs": B / t / 1e9, "hbm_gbs": alg / t / 1e9,
                      "algorithmic_bytes": alg, "ms_eager": t_eager * 1e3}
