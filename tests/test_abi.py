@@ -286,3 +286,33 @@ def test_split12_read_header_matches_the_oracle(wcm):
             assert got == ok
         with pytest.raises(wcm.WCError):
             wcm.split12_read_header(cont[:-1])
+
+
+def test_headers_are_plain_c_and_link(wcm, tmp_path):
+    """The public headers compile as C99 (-pedantic, no warnings), every
+    declared entry point links from libwc.so, and size queries answer from a
+    C program as they do through the binding."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    names = declared_entry_points()
+    src = ['#include <stdio.h>', '#include "wc.h"', '#include "wc_split12.h"',
+           'typedef void (*fn_t)(void);',
+           'int main(void) {', '  const fn_t fns[] = {']
+    src += [f'    (fn_t)&{n},' for n in names]
+    src += ['  };', '  (void)fns;',
+            '  printf("%llu %llu %llu\\n", (unsigned long long)wc_encode_bound(1000, WC_FP32),',
+            '         (unsigned long long)wc12_encode_bound(1000), (unsigned long long)wc_scratch_bytes(1000, WC_BF16));',
+            '  return 0;', '}']
+    c = tmp_path / "abi.c"
+    c.write_text("\n".join(src) + "\n")
+    pkg = os.path.join(ROOT, "fp32_weight_compression_b200")
+    exe = tmp_path / "abi"
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror",
+                        "-Wno-cast-function-type", "-I", os.path.join(ROOT, "include"), str(c), "-L", pkg,
+                        "-lwc", f"-Wl,-rpath,{pkg}", "-o", str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split()
+    assert [int(v) for v in out] == [wcm.encode_bound(1000, 2), wcm.split12_encode_bound(1000),
+                                     wcm.scratch_bytes(1000, 1)]
