@@ -17,6 +17,13 @@
 #include "wc.h"
 #include "wc_format.cuh"
 
+namespace wc {
+// block checksums (k_crc.cu)
+cudaError_t launch_crc32(const uint8_t *buf, uint64_t bytes, uint64_t block_bytes, uint32_t *crc,
+                         int grid, cudaStream_t s);
+int crc_blocks_per_sm();
+}  // namespace wc
+
 namespace {
 
 thread_local char g_last_error[256] = "";

@@ -150,9 +150,6 @@ cudaError_t launch_coder(const EncParams &p, cudaStream_t s);
 cudaError_t launch_compact(const EncParams &p, cudaStream_t s);
 cudaError_t launch_decode(const DecParams &p, int grid, cudaStream_t s);
 int decode_blocks_per_sm();
-cudaError_t launch_crc32(const uint8_t *buf, uint64_t bytes, uint64_t block_bytes, uint32_t *crc,
-                         int grid, cudaStream_t s);
-int crc_blocks_per_sm();
 
 // ---------------------------------------------------------------------------
 // Device helpers.
