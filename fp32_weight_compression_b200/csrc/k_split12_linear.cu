@@ -343,7 +343,7 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   if (d_w == nullptr || d_x == nullptr || d_y == nullptr || d_status == nullptr) return WC_ERR_INVALID_ARG;
   if (!aligned(d_w, 16) || !aligned(d_x, 16) || !aligned(d_y, 4) || !aligned(d_status, 4))
     return WC_ERR_INVALID_ARG;
-  if (N == 0 || K == 0 || N % wc12l::kBM != 0 || K % wc12l::kBK != 0 || M == 0 || M > wc12l::kMaxTokens)
+  if (N == 0 || K == 0 || N % wc12l::kBM != 0 || K % wc12l::kBK != 0 || M == 0)
     return WC_ERR_INVALID_ARG;
   if (w_bytes < 96) return WC_ERR_INVALID_ARG;  // shorter than any container's header
   const wc12l::DevInfo di = wc12l::dev_info();
@@ -352,12 +352,8 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   wc12l::Params p;
   p.w = static_cast<const uint8_t *>(d_w);
   p.w_bytes = w_bytes;
-  p.x = static_cast<const uint16_t *>(d_x);
-  p.y = d_y;
-  p.M = M;
   p.N = N;
   p.K = K;
-  p.n_mma = (M + 15) / 16 * 16;
   p.status = d_status;
   const uint32_t blocks = N / wc12l::kBM, stages = K / wc12l::kBK;
   // split K until the grid covers the SMs twice, at least two stages a CTA
@@ -366,10 +362,18 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   if (splits < 1) splits = 1;
   p.per_split = (stages + splits - 1) / splits;
   p.splits = (stages + p.per_split - 1) / p.per_split;
-  if (p.splits > 1) {
-    wc12l::k12_zero<<<unsigned(2 * di.sms), 256, 0, s>>>(d_y, uint64_t(M) * N);
+  // tokens in slices of at most kMaxTokens (the MMA's N); each slice's rows
+  // of X and Y are contiguous
+  for (uint32_t t0 = 0; t0 < M; t0 += wc12l::kMaxTokens) {
+    const uint32_t m = M - t0 < wc12l::kMaxTokens ? M - t0 : wc12l::kMaxTokens;
+    p.x = static_cast<const uint16_t *>(d_x) + uint64_t(t0) * K;
+    p.y = d_y + uint64_t(t0) * N;
+    p.M = m;
+    p.n_mma = (m + 15) / 16 * 16;
+    if (p.splits > 1) wc12l::k12_zero<<<unsigned(2 * di.sms), 256, 0, s>>>(p.y, uint64_t(m) * N);
+    dim3 grid(blocks, p.splits);
+    wc12l::k12_linear<<<grid, wc12l::kThreads, wc12l::smem_bytes(p.n_mma), s>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
   }
-  dim3 grid(blocks, p.splits);
-  wc12l::k12_linear<<<grid, wc12l::kThreads, wc12l::smem_bytes(p.n_mma), s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+  return WC_OK;
 }

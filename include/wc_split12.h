@@ -83,7 +83,8 @@ WC_API int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out,
  * HBM at 12 bits a value.
  *   d_w, w_bytes  the container (16-byte aligned, at least 96 bytes), n = N * K
  *   N, K          N a multiple of 128, K a multiple of 64
- *   d_x           M x K bf16, row-major, 16-byte aligned; 1 <= M <= 256
+ *   d_x           M x K bf16, row-major, 16-byte aligned; M >= 1 (taken in
+ *                 slices of 256 tokens, one launch each)
  *   d_y           M x N fp32, row-major (overwritten)
  *   d_status      device i32 set to 0 by the caller: WC_ERR_CORRUPT for a bad
  *                 container, WC_ERR_TIMEOUT if a bounded wait ran out

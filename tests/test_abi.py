@@ -252,7 +252,6 @@ def test_split12_linear_bad_arguments_rejected_without_device(wcm):
     assert call(N=100) == wcm.ERR_INVALID_ARG          # N not a multiple of 128
     assert call(K=96) == wcm.ERR_INVALID_ARG           # K not a multiple of 64
     assert call(M=0) == wcm.ERR_INVALID_ARG
-    assert call(M=257) == wcm.ERR_INVALID_ARG
     assert call(w=b + 8) == wcm.ERR_INVALID_ARG        # container not 16-byte aligned
     assert call(x=b + 8) == wcm.ERR_INVALID_ARG
     assert call(y=b + 2) == wcm.ERR_INVALID_ARG
