@@ -52,6 +52,8 @@ def load_container(fname: str) -> np.ndarray:
             if not line or line.startswith("#"):
                 continue
             key, val = line.split(":", 1)
+            if not key[0].isdigit() and key != "length":
+                continue  # a named field (load_fields)
             if key == "length":
                 data = np.zeros(int(val), np.uint8)
                 continue
@@ -63,3 +65,19 @@ def load_container(fname: str) -> np.ndarray:
             for r in range(cnt):
                 data[off + r * len(bs): off + (r + 1) * len(bs)] = bs
     return data
+
+
+def load_fields(fname: str) -> dict:
+    """The named (non-offset) fields of a fixture, e.g. 'exponents', as byte
+    lists parsed from hex."""
+    out = {}
+    with open(os.path.join(GOLDEN, fname)) as fh:
+        for line in fh:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = line.split(":", 1)
+            if key[0].isdigit() or key == "length":
+                continue
+            out[key] = [int(b, 16) for b in val.split()]
+    return out

@@ -362,3 +362,18 @@ def test_fp8_random_access_and_mixed_batch(orc, gu):
     outs = wc.decode_batch(conts, [(a.size,) for a in arrs], [t.dtype for t in ts])
     for a, o in zip(arrs, outs):
         assert np.array_equal(gu.to_bits(o).view(a.dtype), a)
+
+
+@pytest.mark.parametrize("fname,raw", [("container_bf16_n186_tie_raw.txt", True),
+                                       ("container_bf16_n186_near_coded.txt", False)])
+def test_raw_fallback_boundary(orc, gu, fname, raw):
+    """128 + 2w == nsym is stored raw, 128 + 2w == nsym - 2 stays coded:
+    the library's container equals the hand-laid-out fixture (and the
+    oracle's), and decodes bit-exactly."""
+    from _golden import load_container, load_fields
+    e = np.array(load_fields(fname)["exponents"], np.uint16)
+    bits = (e << 7).astype(np.uint16)
+    want = load_container(fname)
+    got = _check(orc, gu, bits)
+    assert np.array_equal(got, want)
+    assert int(want[592:596].view(np.uint32)[0]) == (186 if raw else 184)

@@ -395,3 +395,25 @@ def test_coded_payload_layout(orc):
         assert st == 0 and np.array_equal(sym, e[65536 * k:65536 * k + nsym])
         pad = cont[p + int(lens[k]): p + int(choff[k + 1] - choff[k])]
         assert not pad.any()
+
+
+@pytest.mark.parametrize("fname,raw", [("container_bf16_n186_tie_raw.txt", True),
+                                       ("container_bf16_n186_near_coded.txt", False)])
+def test_golden_raw_fallback_boundary(orc, fname, raw):
+    """The raw-fallback boundary ("PTWM" Configuration table,
+    compression_threshold, read as: raw iff 128 + 2w >= nsym, ties raw): a
+    chunk whose coded length equals nsym is stored raw, one 2 bytes shorter
+    stays coded.  w comes from the pinned rANS core; the container bytes
+    were laid out field by field, not by the oracle's encoder."""
+    from _golden import load_fields
+    e = np.array(load_fields(fname)["exponents"], np.uint8)
+    bits = e.astype(np.uint16) << 7
+    states, words = orc.rans_encode(e, orc.normalize(orc.histogram(e)))
+    assert (128 + 2 * words.size == e.size) == raw
+    assert (128 + 2 * words.size == e.size - 2) == (not raw)
+    want = load_container(fname)
+    got = orc.encode(bits)
+    assert got.size == want.size and np.array_equal(got, want)
+    chunk_len = int(got[592:596].view(np.uint32)[0])
+    assert chunk_len == (e.size if raw else e.size - 2)
+    assert orc.decode(got).tolist() == bits.tolist()

@@ -23,29 +23,15 @@ def oracle_digest(args):
     return idx, cont.size, hashlib.sha256(cont.tobytes()).hexdigest()
 
 
-def oracle_chunk_payloads(args):
-    """Payload bytes (as stored in the container) of a few chunks of one
-    tensor, computed with the oracle's rANS core and the whole tensor's table."""
-    cid, idx, chunks = args
-    import numpy as np
+def gen_tensor_and_digest(args):
+    """The tensor and the digest of the oracle's container for it, from one
+    draw."""
+    cid, idx = args
     import oracle
     import workloads
     bits = workloads.generate_tensor(cid, idx)
-    if bits.dtype == np.uint16:
-        e, _ = oracle.split_bf16(bits)
-    else:
-        e, _, _ = oracle.split_fp32(bits)
-    f = oracle.normalize(oracle.histogram(e))
-    out = {}
-    for k in chunks:
-        sym = e[k * 65536:(k + 1) * 65536]
-        states, words = oracle.rans_encode(sym, f)
-        if 128 + 2 * words.size < sym.size:
-            payload = states.astype("<u4").tobytes() + words.astype("<u2").tobytes()
-        else:
-            payload = sym.tobytes()
-        out[k] = hashlib.sha256(payload).hexdigest()
-    return idx, f.tobytes(), out
+    cont = oracle.encode(bits)
+    return idx, bits, cont.size, hashlib.sha256(cont.tobytes()).hexdigest()
 
 
 def gen_tensor(args):
