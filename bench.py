@@ -1,20 +1,31 @@
 #!/usr/bin/env python3
 """Throughput of the exponent-plane rANS codec on B200.
 
-One step = the whole hot path over the 0.6B-decoder-LM bf16 weight set
-(254 tensors, 596,042,752 values, 1.19 GB; see workloads.py): one batched
-encode (plane split + histogram + 12-bit table, 32-lane rANS with raw
-fallback, offset scan, compaction) and one batched decode (rANS + plane
-re-merge) of all tensors, inputs resident in HBM.
+One step = the whole hot path over one weight set, inputs resident in HBM:
+one batched encode (plane split + histogram + 12-bit table, 32-lane rANS
+with raw fallback, offset scan, compaction) and one batched decode (rANS +
+plane re-merge) of every tensor.  The headline set is workload 4, the
+largest that fits one GPU: 225 bf16 tensors shaped like an 8B dense LM
+(hidden 4096, 32 layers, GQA; embedding 128256x4096), 7,504,658,432 values,
+15.0 GB, values 0.015 * Student-t(4) (see workloads.py).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload 4] [--extra 1,2,3,5 | none]
 
 Prints one JSON line (rank 0).  `value` is uncompressed GB per second of
-round trip: bytes of all tensors / (encode time + decode time), summed over
-ranks (each rank codes its own copy of the set: weak scaling, no collective on
-the data path).  Timing: CUDA events on the launching stream over exactly K
-steps, barrier + synchronize on both sides, max over ranks.  The inputs
-(1.19 GB) exceed the 126 MB L2, so no flush is needed between steps.
+round trip: bytes of all tensors / (encode time + decode time).  Timing:
+CUDA events on the launching stream over exactly K steps, barrier +
+synchronize on both sides, max over ranks.  The inputs (15 GB) exceed the
+126 MB L2, so no flush is needed between steps.  The other workloads are
+timed the same way, each for --extra-steps steps, and reported under
+`workloads`.
+
+Several GPUs (torchrun): the tensors of the set are partitioned, whole
+tensors, across the ranks (largest first, each to the least-loaded rank);
+each rank encodes and decodes its share, with no collective on the data
+path; the job's time is the slowest rank's, so `value` = all bytes / that
+time (total work fixed: strong scaling).
+
 `--impl reference` times the CPU oracle instead (rank 0 only).
 """
 from __future__ import annotations
@@ -35,32 +46,43 @@ import numpy as np  # noqa: E402
 
 import workloads  # noqa: E402
 
-WORKLOAD = 2
 HBM_FALLBACK_GBS = 6650.0
 METRIC = "decode & encode GB/s (uncompressed bytes) on 1 B200, % HBM roofline; ratio"
-WORKLOAD_NAME = ("bf16 tensor set shaped like a 0.6B decoder LM (hidden 1024, 28 layers, "
-                 "embedding 151936x1024, 57 norms): 254 tensors")
+WORKLOAD_NAMES = {
+    1: "one bf16 1024x1024 tensor, N(0, 0.02)",
+    2: ("bf16 tensor set shaped like a 0.6B decoder LM (hidden 1024, 28 layers, "
+        "embedding 151936x1024, 57 norms): 254 tensors"),
+    3: "fp32 tensor set shaped like GPT-2 small (12 layers, embedding 50257x768): 49 tensors",
+    4: ("bf16 tensor set shaped like an 8B dense LM (hidden 4096, 32 layers, GQA, "
+        "embedding 128256x4096), 0.015 * Student-t(4): 225 tensors"),
+    5: "adversarial bf16 stream of 2^28 values (uniform, constant, special-value, N(0,1e-3) chunks)",
+}
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
-    ap.add_argument("--cpu-seconds", type=float, default=12.0,
-                    help="oracle work budget of the CPU baseline sample (0: skip)")
+    ap.add_argument("--workload", type=int, default=4, choices=[1, 2, 3, 4, 5],
+                    help="the headline set")
+    ap.add_argument("--extra", default="1,2,3,5",
+                    help="other workloads timed after the headline ('none' to skip)")
+    ap.add_argument("--extra-steps", type=int, default=10)
+    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--cpu-seconds", type=float, default=8.0,
+                    help="oracle time budget per worker of the all-cores CPU baseline (0: skip)")
     ap.add_argument("--tensors", type=int, default=0,
                     help="profiling only: use the first N tensors of the set (0: all)")
     ap.add_argument("--no-e2e", action="store_true", help="profiling only: skip the e2e leg")
     ap.add_argument("--split12", action="store_true",
                     help="also time the Split12 serving format (wc12_encode / wc12_decode) on the "
-                         "same tensors, outside the timed step; adds a 'split12' object")
+                         "headline tensors, outside the timed step; adds a 'split12' object")
     ap.add_argument("--checksum", action="store_true",
                     help="also time wc_crc32_blocks (1 MiB blocks) over the container arena, "
                          "outside the timed step; adds a 'checksum' object to the line")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def host_cores() -> int:
@@ -77,43 +99,127 @@ def load_oracle():
     return oracle
 
 
-def oracle_round_trip_sample(oracle, budget_s: float, first_index: int = 0, max_tensors=None):
-    """Oracle encode + decode of workload tensors in order until the budget is
-    spent.  Returns (bytes, seconds, tensors, description)."""
-    specs = workloads.tensor_specs(WORKLOAD)
-    done_b, spent, count = 0, 0.0, 0
-    i = first_index
-    while True:
-        bits = workloads.generate_tensor(WORKLOAD, i % len(specs))
-        t0 = time.perf_counter()
-        cont = oracle.encode(bits)
-        back = oracle.decode(cont)
-        spent += time.perf_counter() - t0
-        assert np.array_equal(back, bits)
-        done_b += bits.nbytes
-        count += 1
-        i += 1
-        if spent >= budget_s or (max_tensors is not None and count >= max_tensors):
-            break
-    names = (f"{count} tensors taken in order from the {len(specs)}-tensor set, starting at "
-             f"{specs[first_index % len(specs)].name} and wrapping around")
-    return done_b, spent, count, f"{names}, {done_b / 1e6:.1f} MB, single thread"
+# ---------------------------------------------------------------------------
+# Partitioning of a tensor set across ranks (whole tensors, no exchange).
+def partition(sizes, world: int) -> list[list[int]]:
+    """Indices of the tensors each rank codes: largest first, each to the
+    rank with the fewest bytes so far (ties to the lower rank); each share
+    is returned in set order."""
+    load = [0] * world
+    shares = [[] for _ in range(world)]
+    for i in sorted(range(len(sizes)), key=lambda j: (-sizes[j], j)):
+        r = min(range(world), key=lambda q: (load[q], q))
+        shares[r].append(i)
+        load[r] += sizes[i]
+    return [sorted(s) for s in shares]
 
 
+def max_over_ranks(vals, dev, world):
+    """Element-wise maximum of per-rank timings (seconds) over all ranks; every
+    rank gets the result.  The only collective of a multi-GPU run: the path
+    itself has no exchange (each rank encodes and decodes its own tensors)."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def sum_over_ranks(vals, dev, world):
+    if world <= 1:
+        return [float(v) for v in vals]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return t.tolist()
+
+
+def job_gbs(total_bytes, steps, seconds):
+    """Whole-job throughput: the bytes all ranks processed over the slowest
+    rank's time."""
+    return total_bytes * steps / seconds / 1e9
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle as it stands, one process per host core.
+def _oracle_worker(args):
+    """Encode + decode the given tensors of a workload with the oracle, over
+    and over, until `budget` seconds of oracle time are spent; the tensors
+    are drawn first and the timing starts when every worker is ready."""
+    cid, idx_list, budget, barrier = args
+    sys.path.insert(0, ROOT)
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import oracle
+    import workloads as wl
+    data = [wl.generate_tensor(cid, i) for i in idx_list]
+    oracle.decode(oracle.encode(data[0]))  # loads the library
+    if barrier is not None:
+        barrier.wait()
+    done, spent, j = 0, 0.0, 0
+    t0 = time.perf_counter()
+    while spent < budget:
+        b = data[j % len(data)]
+        c = oracle.encode(b)
+        back = oracle.decode(c)
+        assert np.array_equal(back, b)
+        done += b.nbytes
+        j += 1
+        spent = time.perf_counter() - t0
+    return done, spent, j
+
+
+def cpu_oracle_baseline(cid: int, budget: float, workers: int):
+    """GB/s of oracle encode + decode on `workers` processes at once (one per
+    host core), each coding its own tensors of workload cid."""
+    import multiprocessing as mp
+    specs = workloads.tensor_specs(cid)
+    if cid == 4:   # the k and v projections (4096x1024): many equal, modest tensors
+        pool_idx = [i for i, s in enumerate(specs) if s.name.endswith((".k", ".v"))]
+    elif cid == 2:
+        pool_idx = [i for i, s in enumerate(specs) if s.name.endswith((".k", ".v"))]
+    else:
+        pool_idx = [i for i, s in enumerate(specs) if s.numel <= (1 << 22)] or [0]
+    ctx = mp.get_context("spawn")
+    barrier = ctx.Manager().Barrier(workers)
+    assign = [[pool_idx[(w + k * workers) % len(pool_idx)] for k in range(2)] for w in range(workers)]
+    with ctx.Pool(workers) as pool:
+        res = pool.map(_oracle_worker, [(cid, a, budget, barrier) for a in assign])
+    total = sum(r[0] for r in res)
+    wall = max(r[1] for r in res)
+    names = sorted({specs[i].name.split(".")[-1] for a in assign for i in a})
+    return {"value": total / wall / 1e9, "unit": "GB/s", "cores": workers, "kind": "oracle",
+            "sample": (f"workload {cid}: {workers} processes at once (one per host core), each "
+                       f"coding 2 of the {'/'.join(names)} tensors of the set over and over "
+                       f"for {budget:.0f} s (encode + decode, {sum(r[2] for r in res)} tensor "
+                       f"round trips, {total / 1e9:.2f} GB)")}
+
+
+def cpu_oracle_single(budget: float):
+    """The oracle on one core: workload 1 (one 1024x1024 bf16 tensor)."""
+    done, spent, j = _oracle_worker((1, [0], budget, None))
+    return {"value": done / spent / 1e9, "unit": "GB/s", "cores": 1,
+            "sample": f"workload 1 tensor, {j} encode + decode round trips, {spent:.1f} s"}
+
+
+# ---------------------------------------------------------------------------
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+    """nvidia-smi clocks / throttle reasons, sampled every 20 ms from before
+    the warm-up to the end of the timed region; the summary uses the samples
+    taken inside the timed region (all of them if fewer than 3 fall there)."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int, period_ms: int = 50):
+    def __init__(self, gpu_index: int, period_ms: int = 20):
         import tempfile
         self.proc = None
-        # the raw samples go to WC_CLOCK_LOG_DIR if set (kept for inspection),
-        # else to the temp directory; the summary goes into the JSON line
         log_dir = os.environ.get("WC_CLOCK_LOG_DIR") or tempfile.gettempdir()
-        self.path = os.path.join(log_dir, f"clocks_gpu{gpu_index}.csv")
+        self.path = os.path.join(log_dir, f"clocks_gpu{gpu_index}_{os.getpid()}.csv")
+        self.window = None
         try:
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
@@ -123,33 +229,53 @@ class ClockSampler:
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < 3.0 and os.path.getsize(self.path) == 0:
+            time.sleep(0.01)
+
+    def mark(self, start: float, end: float):
+        self.window = (start, end)
 
     def stop(self) -> dict:
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.05)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
         self.fh.close()
-        sm, smax, reasons = [], [], set()
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                sm.append(float(f[1]))
-                smax.append(float(f[2]))
-            except ValueError:
+                ts = time.mktime(time.strptime(f[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                ts += float("0." + f[0].split(".")[1]) if "." in f[0] else 0.0
+                rows.append((ts, float(f[2]), float(f[3]), f[6:10]))
+            except (ValueError, IndexError):
                 continue
-            for nm, v in zip(names, f[5:9]):
+        inside = rows
+        if self.window is not None:
+            a, b = self.window
+            sel = [r for r in rows if a - 0.01 <= r[0] <= b + 0.03]
+            if len(sel) >= 3:
+                inside = sel
+        reasons = set()
+        for r in inside:
+            for nm, v in zip(names, r[3]):
                 if v.lower() == "active":
                     reasons.add(nm)
+        sm = [r[1] for r in inside]
         return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "sm_max_mhz": max(r[2] for r in inside) if inside else None,
+                "reasons": sorted(reasons), "samples": len(inside),
+                "period_ms": 20,
+                "scope": "timed region" if inside is not rows else "warm-up + timed region"}
 
 
 def peak_hbm():
@@ -161,25 +287,10 @@ def peak_hbm():
         return HBM_FALLBACK_GBS, "of fallback"
 
 
-def recorded_traffic(kernel: str, src_files) -> float | None:
-    """dram bytes per launch recorded by an ncu capture in profiles/, valid
-    only while the kernel's sources are unchanged."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_workload2.md")
-    if not os.path.exists(path):
-        return None
-    want = None
-    val = None
-    for line in open(path):
-        if line.startswith("source_sha256:"):
-            want = line.split(":", 1)[1].strip()
-        if line.startswith("traffic_bytes_per_launch:"):
-            val = float(line.split(":", 1)[1].strip())
-    h = hashlib.sha256()
-    for f in src_files:
-        h.update(open(os.path.join(ROOT, f), "rb").read())
-    if want != h.hexdigest():
-        return None
-    return val
+DECODE_SOURCES = ["fp32_weight_compression_b200/csrc/k_decode.cu",
+                  "fp32_weight_compression_b200/csrc/wc_format.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_block.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_planes.cuh"]
 
 
 def kernel_sources_sha(files) -> str:
@@ -189,52 +300,47 @@ def kernel_sources_sha(files) -> str:
     return h.hexdigest()
 
 
-DECODE_SOURCES = ["fp32_weight_compression_b200/csrc/k_decode.cu",
-                  "fp32_weight_compression_b200/csrc/wc_format.cuh",
-                  "fp32_weight_compression_b200/csrc/wc_block.cuh",
-                  "fp32_weight_compression_b200/csrc/wc_planes.cuh"]
-CODER_SOURCES = ["fp32_weight_compression_b200/csrc/k_encode.cu",
-                 "fp32_weight_compression_b200/csrc/wc_format.cuh",
-                 "fp32_weight_compression_b200/csrc/wc_block.cuh",
-                 "fp32_weight_compression_b200/csrc/wc_planes.cuh"]
+def recorded_traffic(kernel: str, workload: int, src_files, values: int) -> float | None:
+    """DRAM bytes per launch of `kernel` on the given set, from the ncu
+    summary in profiles/ (bytes per value there, times this launch's values),
+    valid only while the kernel's sources are unchanged."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_workload{workload}.md")
+    if not os.path.exists(path):
+        return None
+    want, per_value = None, None
+    for line in open(path):
+        if line.startswith("source_sha256:"):
+            want = line.split(":", 1)[1].strip()
+        if line.startswith("traffic_bytes_per_value:"):
+            per_value = float(line.split(":", 1)[1].strip())
+    if per_value is None or want != kernel_sources_sha(src_files):
+        return None
+    return per_value * values
 
 
 # ---------------------------------------------------------------------------
-def max_over_ranks(vals, dev, world):
-    """Element-wise maximum of per-rank timings (seconds) over all ranks; every
-    rank gets the result.  The only collective of a multi-GPU run: the path
-    itself has no exchange (each rank encodes and decodes its own set)."""
-    if world <= 1:
-        return [float(v) for v in vals]
-    import torch
-    import torch.distributed as dist
-    t = torch.tensor([float(v) for v in vals], dtype=torch.float64, device=dev)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return t.tolist()
-
-
-def job_gbs(world, bytes_per_rank, steps, seconds):
-    """Whole-job throughput: the bytes all ranks processed over the slowest
-    rank's time."""
-    return world * bytes_per_rank * steps / seconds / 1e9
-
-
 def run_reference(args, rank, world):
     """The reference arm: the CPU oracle as it stands, on the host cores,
-    rank 0 only.  Each step is a bounded sample of the workload: one tensor
-    (layer (step mod 28) k projection, 1024x1024 bf16)."""
+    rank 0 only.  Each step is a bounded sample of the headline set: one of
+    its k projections (4096x1024 bf16, 4.2M values), encode + decode."""
     if rank != 0:
         return
     oracle = load_oracle()
-    specs = workloads.tensor_specs(WORKLOAD)
-    k_idx = [i for i, s in enumerate(specs) if s.name.endswith(".k")]
-    data = {i: workloads.generate_tensor(WORKLOAD, i) for i in k_idx}
+    cid = args.workload
+    specs = workloads.tensor_specs(cid)
+    k_idx = [i for i, s in enumerate(specs) if s.name.endswith(".k")] or [0]
+    data = {}
+    for s in range(args.warmup + args.steps):
+        i = k_idx[s % len(k_idx)]
+        if i not in data and len(data) < 4:
+            data[i] = workloads.generate_tensor(cid, i)
+    keys = list(data)
     for s in range(args.warmup):
-        b = data[k_idx[s % len(k_idx)]]
+        b = data[keys[s % len(keys)]]
         oracle.decode(oracle.encode(b))
     tot_b, tot_t = 0, 0.0
     for s in range(args.steps):
-        b = data[k_idx[s % len(k_idx)]]
+        b = data[keys[s % len(keys)]]
         t0 = time.perf_counter()
         c = oracle.encode(b)
         back = oracle.decode(c)
@@ -242,13 +348,16 @@ def run_reference(args, rank, world):
         tot_b += b.nbytes
         assert np.array_equal(back, b)
     gbs = tot_b / tot_t / 1e9
-    sample = "per step one 1024x1024 bf16 tensor (layers.<step mod 28>.k) of the set, encode + decode"
+    shape = "x".join(str(d) for d in specs[keys[0]].shape)
+    sample = (f"per step one {shape} tensor of the set ({len(keys)} k projections in "
+              f"rotation), encode + decode, single thread")
     line = {
         "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u32", "data": "synthetic (seeded numpy PCG64)",
-        "config": {"workload": WORKLOAD_NAME, "sample": sample},
+        "ms_per_step": tot_t / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "strong", "vs_baseline": None, "dtype": "u32",
+        "data": "synthetic (seeded numpy PCG64)",
+        "config": {"workload": WORKLOAD_NAMES[cid], "sample": sample},
         "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -256,27 +365,139 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world):
+# ---------------------------------------------------------------------------
+def _gen_worker(args):
+    cid, i = args
+    sys.path.insert(0, ROOT)
+    import workloads as wl
+    return i, wl.generate_tensor(cid, i)
+
+
+def generate_pinned(pool, cid, idx):
+    """The listed tensors of a workload drawn in the process pool, packed into
+    one pinned host buffer (256-byte aligned views).  Returns (buffer, offsets,
+    nbytes, numels, dtypes)."""
+    import torch
+    specs = workloads.tensor_specs(cid)
+    offs, off = [], 0
+    for i in idx:
+        offs.append(off)
+        off = (off + specs[i].numel * specs[i].itemsize + 255) // 256 * 256
+    host = torch.empty(max(off, 256), dtype=torch.uint8, pin_memory=True)
+    hv = host.numpy()
+    where = {i: o for i, o in zip(idx, offs)}
+    if pool is None:
+        it = (_gen_worker((cid, i)) for i in idx)
+    else:
+        it = pool.imap_unordered(_gen_worker, [(cid, i) for i in idx])
+    for i, a in it:
+        hv[where[i]:where[i] + a.nbytes] = a.view(np.uint8)
+        del a
+    nbytes = [specs[i].numel * specs[i].itemsize for i in idx]
+    numels = [specs[i].numel for i in idx]
+    dts = [torch.bfloat16 if specs[i].dtype == "bf16" else torch.float32 for i in idx]
+    return host, offs, nbytes, numels, dts
+
+
+class DeviceSet:
+    """A tensor set resident in HBM with its encoder and decoder bound."""
+
+    def __init__(self, host, offs, nbytes, numels, dts, dev):
+        import torch
+        from fp32_weight_compression_b200 import wc
+        self.dev_in = host.to(dev)
+        self.dev_out = torch.zeros_like(self.dev_in)
+        self.ins = [self.dev_in[o:o + b].view(d) for o, b, d in zip(offs, nbytes, dts)]
+        self.outs = [self.dev_out[o:o + b].view(d) for o, b, d in zip(offs, nbytes, dts)]
+        self.enc = wc.BatchEncoder(numels, dts, device=dev)
+        self.enc.prepare(self.ins)
+        conts_cap = [self.enc.out[o:o + c] for o, c in zip(self.enc.out_offsets, self.enc.caps)]
+        self.dec = wc.BatchDecoder(device=dev).prepare(conts_cap, self.outs)
+        self.bytes = int(sum(nbytes))
+        self.n = len(numels)
+        self.launches_per_step = 5 * ((self.n + 255) // 256)
+
+    def check(self):
+        import torch
+        torch.cuda.synchronize()
+        self.dec.check()
+        assert torch.equal(self.dev_out, self.dev_in), "round trip is not bit-exact"
+
+    def container_bytes(self) -> int:
+        return int(self.enc.sizes.sum().item())
+
+
+def time_steps(ds, K, W, stream, dev, barrier, sampler=None):
+    """W warm-up steps, then exactly K timed steps (encode + decode each),
+    bracketed by barrier + synchronize.  Returns (total, encode, decode)
+    seconds on this rank."""
+    import torch
+    for _ in range(max(W, 1)):
+        ds.enc.run()
+        ds.dec.run()
+    ds.check()
+    ds.dev_out.zero_()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize(dev)
+    t_wall0 = time.time()
+    start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        ds.enc.run()
+        ev[k][1].record(stream)
+        ds.dec.run()
+        ev[k][2].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize(dev)
+    t_wall1 = time.time()
+    barrier()
+    if sampler is not None:
+        sampler.mark(t_wall0, t_wall1)
+    ds.check()
+    t_total = start.elapsed_time(end) / 1e3
+    t_enc = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
+    t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
+    return t_total, t_enc, t_dec
+
+
+def legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak):
+    enc_bytes = total_in + total_cont  # read input, write container
+    dec_bytes = total_cont + total_in  # read container, write output
+    return {
+        "value": job_gbs(total_in, K, t_total),
+        "ms_per_step": t_total / K * 1e3,
+        "encode": {"gbs": job_gbs(total_in, K, t_enc), "ms": t_enc / K * 1e3,
+                   "hbm_gbs": job_gbs(enc_bytes, K, t_enc),
+                   "roofline_frac": job_gbs(enc_bytes, K, t_enc) / peak},
+        "decode": {"gbs": job_gbs(total_in, K, t_dec), "ms": t_dec / K * 1e3,
+                   "hbm_gbs": job_gbs(dec_bytes, K, t_dec),
+                   "roofline_frac": job_gbs(dec_bytes, K, t_dec) / peak},
+        "ratio": total_cont / total_in,
+        "dec_bytes": dec_bytes,
+    }
+
+
+def e2e_leg(args, host, offs, nbytes, dts, dev, stream, barrier, world):
     """End-to-end through the public host API (wc.HostCodec: wc_encode_host /
     wc_decode_host): every step encodes the host-resident inputs (pinned) into
     host containers and decodes those back into host outputs.  The library
     streams windows of tensors through the device with copies in both
     directions overlapping the kernels."""
     import torch
-    import torch.distributed as dist
     from fp32_weight_compression_b200 import wc
-    if args.no_e2e:
-        return None, 0
-    hts = [host_in[o:o + a.nbytes].view(torch.bfloat16) for a, o in zip(arrs, offs)]
-    host_out = torch.empty_like(host_in, pin_memory=True)
-    hos = [host_out[o:o + a.nbytes].view(torch.bfloat16) for a, o in zip(arrs, offs)]
-    big = max(wc.host_encode_footprint(a.size, torch.bfloat16) for a in arrs)
+    hts = [host[o:o + b].view(d) for o, b, d in zip(offs, nbytes, dts)]
+    host_out = torch.empty_like(host, pin_memory=True)
+    hos = [host_out[o:o + b].view(d) for o, b, d in zip(offs, nbytes, dts)]
+    big = max(wc.host_encode_footprint(t.numel(), t.dtype) for t in hts)
     slot = (big + 256 + 255) // 256 * 256
-    codec = wc.HostCodec(256 * ((4 * len(arrs) + 255) // 256) + 3 * slot, device=dev)
+    codec = wc.HostCodec(256 * ((4 * len(hts) + 255) // 256) + 3 * slot, device=dev)
     enc_bufs, sizes = codec.encode_buffers(hts)
     conts = codec.encode(hts, enc_bufs, sizes)      # warm-up + check
     codec.decode(conts, hos)
-    assert torch.equal(host_out, host_in), "end-to-end round trip is not bit-exact"
+    assert torch.equal(host_out, host), "end-to-end round trip is not bit-exact"
     host_out.zero_()
     E = max(1, args.e2e_steps)
     barrier()
@@ -290,15 +511,16 @@ def e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     t_e2e = e0.elapsed_time(e1) / 1e3
-    assert torch.equal(host_out, host_in), "end-to-end round trip is not bit-exact"
-    t_e2e, = max_over_ranks([t_e2e], dev, world)
-    return t_e2e, E
+    assert torch.equal(host_out, host), "end-to-end round trip is not bit-exact"
+    total_cont = sum(int(c.numel()) for c in conts)
+    del codec, enc_bufs, host_out
+    return t_e2e, E, total_cont, len(hts)
 
 
 # ---------------------------------------------------------------------------
 def split12_leg(ins, dev, stream, reps: int = 5):
-    """wc12_encode / wc12_decode over every tensor of the set (one call per
-    tensor, back to back on one stream of its own), containers checked
+    """wc12_encode / wc12_decode over every bf16 tensor of the set (one call
+    per tensor, back to back on one stream of its own), containers checked
     bit-exact.  Algorithmic bytes: encode reads the input twice (histogram,
     pack) and writes the container; decode reads the container and writes
     the values.  Each pass is captured once in a CUDA graph and replayed
@@ -306,7 +528,8 @@ def split12_leg(ins, dev, stream, reps: int = 5):
     import torch
     from fp32_weight_compression_b200 import wc
     L = wc.load()
-    side = torch.cuda.Stream(dev)       # graph capture needs a stream other than the default
+    ins = [t for t in ins if t.dtype == torch.bfloat16]
+    side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
     outs, scrs, sizes = [], [], []
     for t in ins:
@@ -364,6 +587,7 @@ def split12_leg(ins, dev, stream, reps: int = 5):
     res["ratio"] = total / B
     res["launches_per_tensor"] = {"encode": 6, "decode": 1}
     res["timing"] = "CUDA graph of all tensors' launches, replayed; ms_eager: launched one by one"
+    del outs, scrs, vals
     return res
 
 
@@ -388,8 +612,9 @@ def checksum_leg(arena, dev, stream, reps: int = 10):
             "gbs": nbytes / t / 1e9, "reps": reps}
 
 
-def main():
-    args = parse()
+# ---------------------------------------------------------------------------
+def main(argv=None):
+    args = parse(argv)
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -398,138 +623,117 @@ def main():
         run_reference(args, rank, world)
         return
 
-    # Host-side work first (the oracle sample and the input draw use no GPU).
+    cid = args.workload
+    extra = [] if args.extra in ("", "none") else [int(x) for x in args.extra.split(",")]
+    extra = [c for c in extra if c != cid]
+
+    # Host-side work first: the CPU baseline (all cores, then one), the
+    # input draw.  Both use spawn-started processes, before any CUDA call.
     cpu_base = None
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
-        oracle = load_oracle()
-        b, t, cnt, desc = oracle_round_trip_sample(oracle, args.cpu_seconds)
-        cpu_base = {"value": b / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
-                    "sample": desc + f"; {t:.1f} s of encode + decode"}
-    specs = workloads.tensor_specs(WORKLOAD)
+        cpu_base = cpu_oracle_baseline(cid, args.cpu_seconds, host_cores())
+        cpu_base["single_thread"] = cpu_oracle_single(min(3.0, args.cpu_seconds))
+    specs = workloads.tensor_specs(cid)
     idx = list(range(len(specs) if args.tensors <= 0 else min(args.tensors, len(specs))))
-    specs = [specs[i] for i in idx]
-    arrs = workloads.generate_config(WORKLOAD, indices=idx,
-                                     workers=min(16, workloads.default_workers()))
+    shares = partition([specs[i].numel * specs[i].itemsize for i in idx], world)
+    mine = [idx[j] for j in shares[rank]]
+    import multiprocessing as mp
+    pool = mp.get_context("spawn").Pool(max(1, min(16, host_cores() // max(1, world))))
 
     import torch
     import torch.distributed as dist
-    from fp32_weight_compression_b200 import wc
-
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    host, offs, nbytes, numels, dts = generate_pinned(pool, cid, mine)
     if world > 1:
-        dist.init_process_group("nccl", device_id=dev,
-                                timeout=__import__("datetime").timedelta(seconds=120))
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
 
     def barrier():
         if world > 1:
             dist.barrier(device_ids=[local])
 
-    # inputs: one pinned host buffer, one device buffer, per-tensor views
-    offs, off = [], 0
-    for a in arrs:
-        offs.append(off)
-        off = (off + a.nbytes + 255) // 256 * 256
-    total_in = sum(a.nbytes for a in arrs)
-    host_in = torch.empty(off, dtype=torch.uint8, pin_memory=True)
-    hv = host_in.numpy()
-    for a, o in zip(arrs, offs):
-        hv[o:o + a.nbytes] = a.view(np.uint8)
-    dev_in = host_in.to(dev)
-    ins = [dev_in[o:o + a.nbytes].view(torch.bfloat16).view(*s.shape)
-           for a, o, s in zip(arrs, offs, specs)]
-    dev_out = torch.empty_like(dev_in)
-    outs = [dev_out[o:o + a.nbytes].view(torch.bfloat16).view(*s.shape)
-            for a, o, s in zip(arrs, offs, specs)]
-
-    enc = wc.BatchEncoder([a.size for a in arrs], [torch.bfloat16] * len(arrs), device=dev)
-    enc.prepare(ins)
-    conts_cap = [enc.out[o:o + c] for o, c in zip(enc.out_offsets, enc.caps)]
-    dec = wc.BatchDecoder(device=dev).prepare(conts_cap, outs)
     stream = torch.cuda.current_stream(dev)
-
-    # warm-up + a correctness check of the timed configuration
-    for _ in range(max(args.warmup, 1)):
-        enc.run()
-        dec.run()
-    torch.cuda.synchronize(dev)
-    dec.check()
-    assert torch.equal(dev_out, dev_in), "round trip is not bit-exact"
-    sizes = enc.sizes.cpu().tolist()
-    total_cont = int(sum(sizes))
-
-    # timed region
-    K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    barrier()
-    torch.cuda.synchronize(dev)
-    sampler = ClockSampler(local)
-    time.sleep(0.05)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for k in range(K):
-        ev[k][0].record(stream)
-        enc.run()
-        ev[k][1].record(stream)
-        dec.run()
-        ev[k][2].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize(dev)
-    clocks = sampler.stop()
-    barrier()
-    t_total = start.elapsed_time(end) / 1e3
-    t_enc = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    dec.check()
-    t_total, t_enc, t_dec = max_over_ranks([t_total, t_enc, t_dec], dev, world)
-
-    t_e2e, E = e2e_leg(args, arrs, specs, host_in, offs, dev, stream, barrier, world)
-    checksum = checksum_leg(enc.out, dev, stream) if args.checksum else None
-    s12 = split12_leg(ins, dev, stream) if args.split12 else None
-
     peak, peak_note = peak_hbm()
-    B = total_in
-    enc_bytes = B + total_cont     # read input, write container
-    dec_bytes = total_cont + B     # read container, write output
-    enc_gbs = B * K / t_enc / 1e9
-    dec_gbs = B * K / t_dec / 1e9
-    dec_achieved = dec_bytes * K / t_dec / 1e9
-    enc_achieved = enc_bytes * K / t_enc / 1e9
-    value = job_gbs(world, B, K, t_total)
-    traffic = recorded_traffic("k_decode", DECODE_SOURCES)
+    ds = DeviceSet(host, offs, nbytes, numels, dts, dev)
+    sampler = ClockSampler(local)
+    t_total, t_enc, t_dec = time_steps(ds, args.steps, args.warmup, stream, dev, barrier, sampler)
+    clocks = sampler.stop()
+    total_cont = ds.container_bytes()
+    t_total, t_enc, t_dec = max_over_ranks([t_total, t_enc, t_dec], dev, world)
+    total_in, total_cont = (int(v) for v in sum_over_ranks([ds.bytes, total_cont], dev, world))
+    K = args.steps
+    r = legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak)
+    values_mine = int(sum(numels))
+    checksum = checksum_leg(ds.enc.out, dev, stream) if args.checksum else None
+    s12 = split12_leg(ds.ins, dev, stream) if args.split12 else None
+    launches = ds.launches_per_step * K
+    del ds
+    torch.cuda.empty_cache()
+
+    e2e = None
+    if not args.no_e2e:
+        t_e2e, E, e2e_cont, ntens = e2e_leg(args, host, offs, nbytes, dts, dev, stream, barrier, world)
+        t_e2e, = max_over_ranks([t_e2e], dev, world)
+        e2e_cont, = sum_over_ranks([e2e_cont], dev, world)
+        e2e = {"value": job_gbs(total_in, E, t_e2e), "unit": "GB/s",
+               "h2d_bytes_per_step": int(total_in + e2e_cont),
+               "d2h_bytes_per_step": int(e2e_cont + 8 * len(idx) + total_in), "steps": E,
+               "api": "wc_encode_host + wc_decode_host (pinned host buffers, windows through HBM)"}
+    del host
+
+    per_workload = {}
+    if world == 1:
+        for c in extra:
+            cs = workloads.tensor_specs(c)
+            h, o, nb, nu, dt = generate_pinned(pool, c, list(range(len(cs))))
+            d = DeviceSet(h, o, nb, nu, dt, dev)
+            tt, te, td = time_steps(d, args.extra_steps, 3, stream, dev, barrier)
+            rr = legs(d.bytes, d.container_bytes(), args.extra_steps, tt, te, td, peak)
+            rr.pop("dec_bytes")
+            rr["workload"] = WORKLOAD_NAMES[c]
+            rr["input_bytes"] = d.bytes
+            rr["steps"] = args.extra_steps
+            per_workload[str(c)] = rr
+            launches += d.launches_per_step * args.extra_steps
+            del d, h
+            torch.cuda.empty_cache()
+    pool.close()
+
+    traffic = recorded_traffic("k_decode", cid, DECODE_SOURCES, values_mine) if world == 1 else None
+    dec_achieved = r["decode"]["hbm_gbs"]
     line = {
         "metric": METRIC,
-        "value": value,
+        "value": r["value"],
         "unit": "GB/s",
         "n_gpus": world,
         "steps": K,
         "warmup": args.warmup,
-        "ms_per_step": t_total / K * 1e3,
+        "ms_per_step": r["ms_per_step"],
         "higher_is_better": True,
-        "scaling": "weak",
+        "scaling": "strong",
         "vs_baseline": None,
         "dtype": "u32",
         "data": "synthetic (seeded numpy PCG64; no checkpoints available)",
-        "config": {"workload": WORKLOAD_NAME, "tensors": len(arrs), "values": int(sum(a.size for a in arrs)),
-                   "input_bytes": B, "parallelism": f"replicas x{world} (one full set per GPU)",
-                   "l2": "inputs 1.19 GB > 126 MB L2, no flush"},
-        "encode": {"gbs": enc_gbs, "ms": t_enc / K * 1e3, "hbm_gbs": enc_achieved,
-                   "roofline_frac": enc_achieved / peak},
-        "decode": {"gbs": dec_gbs, "ms": t_dec / K * 1e3, "hbm_gbs": dec_achieved,
-                   "roofline_frac": dec_achieved / peak},
-        "ratio": total_cont / B,
+        "config": {"workload": WORKLOAD_NAMES[cid] + (f" (first {len(idx)})" if args.tensors else ""),
+                   "tensors": len(idx), "values": int(sum(specs[i].numel for i in idx)),
+                   "input_bytes": total_in,
+                   "parallelism": ("one GPU" if world == 1 else
+                                   f"tensors partitioned over {world} GPUs (whole tensors, "
+                                   f"largest first to the least-loaded rank), no collective"),
+                   "l2": f"inputs {total_in / 1e9:.2f} GB > 126 MB L2, no flush"},
+        "encode": r["encode"],
+        "decode": r["decode"],
+        "ratio": r["ratio"],
         "roofline": {"bound": "hbm", "kernel": "k_decode", "achieved": dec_achieved, "peak": peak,
                      "unit": "GB/s", "frac": dec_achieved / peak, "traffic": traffic,
                      "peak_note": peak_note,
-                     "algorithmic_bytes_per_launch": dec_bytes},
-        "e2e": None if t_e2e is None else {
-            "value": job_gbs(world, B, E, t_e2e), "unit": "GB/s",
-            "h2d_bytes_per_step": B + total_cont, "d2h_bytes_per_step": total_cont + B + 8 * len(arrs),
-            "steps": E},
-        "gpu_launches": K * 5,
+                     "algorithmic_bytes_per_launch": r["dec_bytes"] // max(1, world)},
+        "e2e": e2e,
+        "gpu_launches": launches,
         "clocks": clocks,
         "cpu_baseline": cpu_base,
+        "workloads": per_workload,
     }
     if checksum is not None:
         checksum["roofline_frac"] = checksum["gbs"] / peak
