@@ -46,6 +46,11 @@ constexpr uint32_t kASlice = kBM * 16 * 2;   // bytes of one K = 16 slice of A
 constexpr uint32_t kAStage = 4 * kASlice;
 constexpr uint32_t kMaxTokens = 256;
 constexpr uint32_t kSpinLimit = 1u << 24;
+// A CTA's exceptions (its 128 rows, its range of K) are gathered once into a
+// shared-memory list of up to kExcCap entries {column in the CTA's K range,
+// row | high byte << 16 | low byte << 24}; a CTA with more walks its chunks'
+// exception lists at every stage instead.
+constexpr uint32_t kExcCap = 1024;
 
 struct Params {
   const uint8_t *w;
@@ -61,7 +66,7 @@ struct Params {
 
 __host__ __device__ inline uint32_t b_stage_bytes(uint32_t n_mma) { return n_mma * kBK * 2; }
 __host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma) {
-  return 1024 + 2 * kAStage + 2 * b_stage_bytes(n_mma) + 64;
+  return 1024 + 2 * kAStage + 2 * b_stage_bytes(n_mma) + 64 + 8 * kExcCap;
 }
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
@@ -142,6 +147,8 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   uint64_t *bar = reinterpret_cast<uint64_t *>(b_st + 2 * b_bytes);
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
+  uint32_t *exc_n = tmem_slot + 2;
+  uint2 *exc_list = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(bar) + 64);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t K = p.K, N = p.N;
@@ -191,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
     *flag = 0;
+    *exc_n = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   fence_before_sync();
@@ -198,6 +206,45 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const uint32_t idesc = instr_desc(p.n_mma);
+
+  // The CTA's exceptions, once: positions within a chunk become (row, column)
+  // relative to the CTA's tile with 32-bit arithmetic when 128 K fits it.
+  const uint64_t f_base = uint64_t(n0) * K, f_span = uint64_t(kBM) * K;
+  const uint32_t k_beg = s_begin * kBK, k_end = s_end * kBK;
+  for (uint64_t c = c_lo; c <= c_hi; c++) {
+    const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
+    if (e0 > e1 || e1 > ne) {
+      if (tid == 0) report(p.status, WC_ERR_CORRUPT);
+      continue;
+    }
+    const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
+    for (uint64_t e = e0 + tid; e < e1; e += kThreads) {
+      const uint32_t pos = exc_pos[e];
+      if (pos >= cnt) {
+        report(p.status, WC_ERR_CORRUPT);
+        continue;
+      }
+      const uint64_t f = c * kChunk + pos;
+      if (f < f_base || f - f_base >= f_span) continue;
+      const uint64_t lf = f - f_base;
+      uint32_t row, col;
+      if (f_span <= 0xFFFFFFFFull) {
+        row = uint32_t(lf) / K;
+        col = uint32_t(lf) - row * K;
+      } else {
+        row = uint32_t(lf / K);
+        col = uint32_t(lf - uint64_t(row) * K);
+      }
+      if (col < k_beg || col >= k_end) continue;
+      const uint32_t slot = atomicAdd(exc_n, 1u);
+      if (slot < kExcCap)
+        exc_list[slot] = make_uint2(col - k_beg, row | (uint32_t(exc_val[e]) << 16) |
+                                                     (uint32_t(lo_plane[f]) << 24));
+    }
+  }
+  __syncthreads();
+  const uint32_t n_exc = *exc_n;
+  const bool exc_walk = n_exc > kExcCap;
 
   uint32_t it = 0;
   for (uint32_t st = s_begin; st < s_end; st++, it++) {
@@ -235,25 +282,29 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
       *reinterpret_cast<uint4 *>(B + op_offset(t, 8 * j, p.n_mma * 32)) = v;
     }
     __syncthreads();
-    // exceptions of the block's chunks that fall in this tile
-    for (uint64_t c = c_lo; c <= c_hi; c++) {
-      const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
-      if (e0 > e1 || e1 > ne) {
-        if (tid == 0) report(p.status, WC_ERR_CORRUPT);
-        continue;
+    // exceptions that fall in this tile
+    if (!exc_walk) {
+      const uint32_t c0 = k0 - k_beg;
+      for (uint32_t i = tid; i < n_exc; i += kThreads) {
+        const uint2 ex = exc_list[i];
+        if (ex.x - c0 >= uint32_t(kBK)) continue;
+        *reinterpret_cast<uint16_t *>(A + op_offset(ex.y & 0xFFFFu, ex.x - c0, kASlice)) =
+            uint16_t(((ex.y >> 16) & 0xFFu) << 8 | (ex.y >> 24));
       }
-      const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
-      for (uint64_t e = e0 + tid; e < e1; e += kThreads) {
-        const uint32_t pos = exc_pos[e];
-        if (pos >= cnt) {
-          report(p.status, WC_ERR_CORRUPT);
-          continue;
+    } else {
+      for (uint64_t c = c_lo; c <= c_hi; c++) {
+        const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
+        if (e0 > e1 || e1 > ne) continue;  // reported by the gathering pass
+        const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
+        for (uint64_t e = e0 + tid; e < e1; e += kThreads) {
+          const uint32_t pos = exc_pos[e];
+          if (pos >= cnt) continue;
+          const uint64_t f = c * kChunk + pos;
+          const uint64_t row = f / K, col = f % K;
+          if (row < n0 || row >= n0 + kBM || col < k0 || col >= k0 + kBK) continue;
+          *reinterpret_cast<uint16_t *>(A + op_offset(uint32_t(row - n0), uint32_t(col - k0), kASlice)) =
+              uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[f]);
         }
-        const uint64_t f = c * kChunk + pos;
-        const uint64_t row = f / K, col = f % K;
-        if (row < n0 || row >= n0 + kBM || col < k0 || col >= k0 + kBK) continue;
-        *reinterpret_cast<uint16_t *>(A + op_offset(uint32_t(row - n0), uint32_t(col - k0), kASlice)) =
-            uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[f]);
       }
     }
     fence_proxy_async();  // generic-proxy writes -> visible to the tensor cores
@@ -275,8 +326,11 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   if (issued > 0) {
     const uint32_t last = issued - 1;
     done = mbar_wait(&bar[last & 1u], (last >> 1) & 1u);
-    if (!done && tid == 0) report(p.status, WC_ERR_TIMEOUT);
   }
+  // every thread takes the same branch below: the tensor-memory loads are
+  // warp-collective (.sync.aligned)
+  done = __syncthreads_and(done) != 0;
+  if (!done && tid == 0) report(p.status, WC_ERR_TIMEOUT);
   fence_after_sync();
   if (done && !*flag && issued > 0) {
     const uint32_t row = n0 + 32 * warp + lane;
@@ -315,7 +369,25 @@ __global__ void k12_zero(float *y, uint64_t count) {
 struct DevInfo {
   int sms = 0;
   bool attr = false;
+  int smem_per_sm = 0;     // shared memory of one SM
+  int smem_reserved = 0;   // per CTA, taken by the system
 };
+
+// Dynamic shared memory for a launch with n_mma token columns: at least what
+// the stages need, padded so that the CTAs that fit on one SM hold at most
+// the SM's 512 tensor-memory columns between them (otherwise a CTA's
+// tcgen05.alloc would wait for another CTA to finish).
+uint32_t launch_smem(const DevInfo &d, uint32_t n_mma) {
+  uint32_t cols = 32;
+  while (cols < n_mma) cols <<= 1;
+  const uint32_t max_ctas = 512 / cols;
+  uint32_t need = smem_bytes(n_mma);
+  const uint32_t per_sm = uint32_t(d.smem_per_sm), rsv = uint32_t(d.smem_reserved);
+  // CTAs per SM = floor(per_sm / (smem + rsv)); make it <= max_ctas
+  const uint32_t floor_smem = per_sm / (max_ctas + 1) + 1;
+  if (floor_smem > rsv && need + rsv < floor_smem) need = floor_smem - rsv;
+  return need;
+}
 
 DevInfo dev_info() {
   static std::mutex mu;
@@ -327,8 +399,19 @@ DevInfo dev_info() {
   if (d.sms == 0) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DevInfo{};
+    int per_sm = 0, rsv = 0;
+    if (cudaDeviceGetAttribute(&per_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+      return DevInfo{};
+    d.smem_per_sm = per_sm;
+    d.smem_reserved = rsv;
+    uint32_t most = 0;
+    for (uint32_t m = 16; m <= kMaxTokens; m += 16) {
+      const uint32_t b = launch_smem(d, m);
+      most = b > most ? b : most;
+    }
     d.attr = cudaFuncSetAttribute(k12_linear, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  int(smem_bytes(kMaxTokens))) == cudaSuccess;
+                                  int(most)) == cudaSuccess;
     d.sms = sms;
   }
   return d;
@@ -372,7 +455,7 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
     p.n_mma = (m + 15) / 16 * 16;
     if (p.splits > 1) wc12l::k12_zero<<<unsigned(2 * di.sms), 256, 0, s>>>(p.y, uint64_t(m) * N);
     dim3 grid(blocks, p.splits);
-    wc12l::k12_linear<<<grid, wc12l::kThreads, wc12l::smem_bytes(p.n_mma), s>>>(p);
+    wc12l::k12_linear<<<grid, wc12l::kThreads, wc12l::launch_smem(di, p.n_mma), s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
   }
   return WC_OK;
