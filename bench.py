@@ -76,12 +76,13 @@ def parse(argv=None):
     ap.add_argument("--tensors", type=int, default=0,
                     help="profiling only: use the first N tensors of the set (0: all)")
     ap.add_argument("--no-e2e", action="store_true", help="profiling only: skip the e2e leg")
-    ap.add_argument("--split12", action="store_true",
-                    help="also time the Split12 serving format (wc12_encode / wc12_decode) on the "
-                         "headline tensors, outside the timed step; adds a 'split12' object")
-    ap.add_argument("--checksum", action="store_true",
-                    help="also time wc_crc32_blocks (1 MiB blocks) over the container arena, "
-                         "outside the timed step; adds a 'checksum' object to the line")
+    ap.add_argument("--no-split12", dest="split12", action="store_false",
+                    help="skip the Split12 serving-format leg (wc12_encode / wc12_decode on the "
+                         "headline tensors and wc12_linear against cuBLAS bf16, timed after the "
+                         "step; the 'split12' object)")
+    ap.add_argument("--no-checksum", dest="checksum", action="store_false",
+                    help="skip the block-checksum leg (wc_crc32_blocks, 1 MiB blocks, over the "
+                         "container arena, timed after the step; the 'checksum' object)")
     return ap.parse_args(argv)
 
 
@@ -415,7 +416,7 @@ class DeviceSet:
         self.dec = wc.BatchDecoder(device=dev).prepare(conts_cap, self.outs)
         self.bytes = int(sum(nbytes))
         self.n = len(numels)
-        self.launches_per_step = 5 * ((self.n + 255) // 256)
+        self.launches_per_step = 3 * ((self.n + 255) // 256)   # k_prep, k_encode, k_decode
 
     def check(self):
         import torch
@@ -591,6 +592,63 @@ def split12_leg(ins, dev, stream, reps: int = 5):
     return res
 
 
+def linear_leg(ins, specs_mine, dev, reps: int = 20):
+    """wc12_linear (Y = X W^T with W held as a Split12 container, expanded
+    into the tensor cores' operand layout inside the kernel) against
+    torch.matmul on the bf16 weights (cuBLAS), for token counts M = 1 .. 256.
+    W: the first four gate projections of the set (4096 x 14336 bf16, 117 MB
+    each, 470 MB together > L2), used in rotation so that every call reads its
+    weights from HBM.  Reported per M: microseconds per call and the weight
+    bytes each call reads over its time."""
+    import torch
+    from fp32_weight_compression_b200 import wc
+    pick = [i for i, s in enumerate(specs_mine) if s.name.endswith(".gate")][:4]
+    if not pick:
+        return None
+    Ws = [ins[i].view(specs_mine[i].shape) for i in pick]
+    N, K = Ws[0].shape
+    conts = [wc.split12_encode(w.reshape(-1)) for w in Ws]
+    L = wc.load()
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    out = {}
+    for M in (1, 16, 64, 256):
+        x = torch.randn(M, K, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.float32, device=dev)
+        s = torch.cuda.current_stream(dev).cuda_stream
+
+        def ours(r):
+            c = conts[r % len(conts)]
+            wc._check(L.wc12_linear(c.data_ptr(), c.numel(), N, K, x.data_ptr(), M, y.data_ptr(),
+                                    status.data_ptr(), s), "wc12_linear")
+
+        def ref(r):
+            torch.matmul(x, Ws[r % len(Ws)].t())
+
+        res = {}
+        for name, fn in (("wc12_linear", ours), ("cublas_bf16", ref)):
+            for r in range(4):
+                fn(r)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize(dev)
+            a.record()
+            for r in range(reps):
+                fn(r)
+            b.record()
+            torch.cuda.synchronize(dev)
+            t = a.elapsed_time(b) / reps / 1e3
+            wbytes = conts[0].numel() if name == "wc12_linear" else 2 * N * K
+            res[name] = {"us": t * 1e6, "weight_gbs": wbytes / t / 1e9}
+        assert int(status.item()) == 0
+        ref_y = torch.matmul(x.float(), Ws[(reps - 1) % len(Ws)].float().t())
+        ours(reps - 1)
+        torch.cuda.synchronize(dev)
+        res["max_rel_err"] = float(((y - ref_y).abs().max() / ref_y.abs().max().clamp_min(1e-30)).item())
+        res["speedup"] = res["cublas_bf16"]["us"] / res["wc12_linear"]["us"]
+        out[str(M)] = res
+    return {"N": N, "K": K, "weights": len(Ws), "per_M": out,
+            "container_bytes": conts[0].numel(), "bf16_bytes": 2 * N * K}
+
+
 def checksum_leg(arena, dev, stream, reps: int = 10):
     """wc_crc32_blocks over the whole container arena (larger than L2), 1 MiB
     blocks: algorithmic bytes = the arena's bytes read (the CRCs written are
@@ -667,6 +725,11 @@ def main(argv=None):
     values_mine = int(sum(numels))
     checksum = checksum_leg(ds.enc.out, dev, stream) if args.checksum else None
     s12 = split12_leg(ds.ins, dev, stream) if args.split12 else None
+    if s12 is not None:
+        try:
+            s12["linear"] = linear_leg(ds.ins, [specs[i] for i in mine], dev)
+        except Exception as ex:  # reported, not fatal: the leg is outside the timed step
+            s12["linear"] = {"error": f"{type(ex).__name__}: {ex}"[:300]}
     launches = ds.launches_per_step * K
     del ds
     torch.cuda.empty_cache()

@@ -17,7 +17,7 @@
 // stream.  Every 8 steps a chunk has 256 new coded bytes; they are transposed
 // through shared memory so that each lane holds 8 consecutive ones, merged
 // with the matching raw-plane bytes, and written with one 16-byte store (bf16,
-// fp16), two (fp32) or one 8-byte store (fp8 e4m3).
+// fp16), two (fp32) or one 8-byte store (fp8).
 //
 // Everything read from the container is checked before use (header fields
 // against the layout implied by n, the table sum, each chunk's offset pair and
@@ -91,7 +91,7 @@ __device__ __noinline__ ItemView view_item(const DecItem &it) {
   const uint32_t w1 = h32[1];
   const int dtype = int((w1 >> 16) & 0xFF);
   if (h32[0] != 0x315A4357u || (w1 & 0xFFFF) != kVersion || (w1 >> 24) != kLanes) return v;
-  if (dtype != WC_BF16 && dtype != WC_FP32 && dtype != WC_FP16 && dtype != WC_FP8E4M3) return v;
+  if (dtype != WC_BF16 && dtype != WC_FP32 && dtype != WC_FP16 && !is_fp8(dtype)) return v;
   const uint64_t n = h64[1];
   if (n > (uint64_t(1) << 44)) return v;
   if (h32[4] != kChunk || h32[6] != kProbBits || h32[7] != 0) return v;
@@ -160,7 +160,7 @@ struct Raw8 {
 
 template <int DT>
 __device__ __forceinline__ void load_raw8(const uint8_t *cont, const Layout &L, uint64_t vg, Raw8<DT> &r) {
-  if (DT == WC_FP8E4M3) {
+  if (is_fp8(DT)) {
     r.a.x = __ldg(reinterpret_cast<const uint32_t *>(cont + L.off_raw + vg / 2));
   } else if (DT != WC_FP32) {
     r.a = __ldg(reinterpret_cast<const uint2 *>(cont + L.off_raw + vg));
@@ -192,8 +192,8 @@ __device__ __forceinline__ uint4 merge4_fp32(uint32_t e4, uint32_t w0, uint32_t 
 // 2-byte values merge byte-parallel (merge4, wc_planes.cuh).
 template <int DT>
 __device__ __forceinline__ void merge_store8(uint2 e8, const Raw8<DT> &r, uint8_t *dst) {
-  if (DT == WC_FP8E4M3) {
-    st_cs_v2(dst, fp8_merge8(e8, r.a.x));  // 8 one-byte values
+  if (is_fp8(DT)) {
+    st_cs_v2(dst, fp8_merge8<DT>(e8, r.a.x));  // 8 one-byte values
   } else if (DT != WC_FP32) {
     const uint2 p = merge4<DT>(e8.x, r.a.x);
     const uint2 q = merge4<DT>(e8.y, r.a.y);
@@ -209,8 +209,8 @@ __device__ __forceinline__ void merge_store8(uint2 e8, const Raw8<DT> &r, uint8_
 template <int DT>
 __device__ __forceinline__ void merge_store1(uint32_t e, const uint8_t *cont, const Layout &L, uint64_t vg,
                                              uint8_t *dst) {
-  if (DT == WC_FP8E4M3) {
-    dst[0] = uint8_t(fp8_merge(e, (cont[L.off_raw + vg / 2] >> (4 * (vg & 1))) & 0xFu));
+  if (is_fp8(DT)) {
+    dst[0] = uint8_t(fp8_merge<DT>(e, (cont[L.off_raw + vg / 2] >> (4 * (vg & 1))) & 0xFu));
   } else if (DT != WC_FP32) {
     reinterpret_cast<uint16_t *>(dst)[0] = uint16_t(merge16<DT>(e, cont[L.off_raw + vg]));
   } else {
@@ -300,7 +300,7 @@ struct RawPtrs {
 
 template <int DT>
 __device__ __forceinline__ void load_raw8p(const RawPtrs &p, uint32_t vl, Raw8<DT> &r) {
-  if (DT == WC_FP8E4M3) {
+  if (is_fp8(DT)) {
     r.a.x = __ldg(reinterpret_cast<const uint32_t *>(p.a + vl / 2));
   } else if (DT != WC_FP32) {
     r.a = __ldg(reinterpret_cast<const uint2 *>(p.a + vl));
@@ -372,7 +372,7 @@ __device__ __noinline__ void decode_pair(const uint8_t *payA, const uint8_t *pay
   Ring ra{rsA, payA + kStateBytes, uint32_t(round16(lenA) - kStateBytes) >> 1, 0, 0, 0, 0};
   Ring rb{rsB, payB + kStateBytes, uint32_t(round16(lenB) - kStateBytes) >> 1, 0, 0, 0, 0};
   RawPtrs rpB;
-  rpB.a = rpA.a + (DT == WC_FP32 ? 3 * kChunk : (DT == WC_FP8E4M3 ? kChunk / 2 : kChunk));
+  rpB.a = rpA.a + (DT == WC_FP32 ? 3 * kChunk : (is_fp8(DT) ? kChunk / 2 : kChunk));
   rpB.s = DT == WC_FP32 ? rpA.s + kChunk / 8 : nullptr;
   uint8_t *outB = outA + kChunk * elem;
   uint32_t xA = reinterpret_cast<const uint32_t *>(payA)[lane];
@@ -603,7 +603,7 @@ __device__ __forceinline__ void decode_warp_chunks(const ItemView &v, const DecI
     const Layout &L = v.L;
     const uint64_t vgA = kA * kChunk;
     RawPtrs rpA;
-    if (DT == WC_FP8E4M3) {
+    if (is_fp8(DT)) {
       rpA.a = it.cont + L.off_raw + vgA / 2;
       rpA.s = nullptr;
     } else if (DT != WC_FP32) {
@@ -655,6 +655,7 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
     if (v.dtype == WC_BF16) decode_warp_chunks<WC_BF16>(v, it, kA, kend, status);
     else if (v.dtype == WC_FP16) decode_warp_chunks<WC_FP16>(v, it, kA, kend, status);
     else if (v.dtype == WC_FP8E4M3) decode_warp_chunks<WC_FP8E4M3>(v, it, kA, kend, status);
+    else if (v.dtype == WC_FP8E5M2) decode_warp_chunks<WC_FP8E5M2>(v, it, kA, kend, status);
     else decode_warp_chunks<WC_FP32>(v, it, kA, kend, status);
   }
 }

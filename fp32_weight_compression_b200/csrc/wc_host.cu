@@ -29,7 +29,7 @@ inline uint64_t r256(uint64_t v) { return (v + 255) & ~uint64_t(255); }
 uint64_t elem_bytes(int32_t dt) { return wc::dtype_bytes(dt); }
 
 bool dtype_ok(int32_t dt) {
-  return dt == WC_BF16 || dt == WC_FP32 || dt == WC_FP16 || dt == WC_FP8E4M3;
+  return dt == WC_BF16 || dt == WC_FP32 || dt == WC_FP16 || dt == WC_FP8E4M3 || dt == WC_FP8E5M2;
 }
 
 constexpr uint64_t kWindowReserve = 256;  // per window: the rounding of its size array

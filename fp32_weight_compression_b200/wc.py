@@ -16,14 +16,14 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libwc.so")
 
 OK, ERR_INVALID_ARG, ERR_CAPACITY, ERR_CUDA, ERR_CORRUPT, ERR_UNSUPPORTED, ERR_TIMEOUT = 0, 1, 2, 3, 4, 5, 6
-BF16, FP32, FP16, FP8E4M3 = 1, 2, 3, 4
+BF16, FP32, FP16, FP8E4M3, FP8E5M2 = 1, 2, 3, 4, 5
 CHUNK = 65536
 
 _DT = {torch.bfloat16: BF16, torch.float32: FP32, torch.float16: FP16,
-       torch.float8_e4m3fn: FP8E4M3}
+       torch.float8_e4m3fn: FP8E4M3, torch.float8_e5m2: FP8E5M2}
 _TORCH_DT = {BF16: torch.bfloat16, FP32: torch.float32, FP16: torch.float16,
-             FP8E4M3: torch.float8_e4m3fn}
-_ELEM = {BF16: 2, FP32: 4, FP16: 2, FP8E4M3: 1}
+             FP8E4M3: torch.float8_e4m3fn, FP8E5M2: torch.float8_e5m2}
+_ELEM = {BF16: 2, FP32: 4, FP16: 2, FP8E4M3: 1, FP8E5M2: 1}
 
 EXPORTS = (
     "wc_encode_bound", "wc_scratch_bytes", "wc_encode", "wc_decode", "wc_decode_chunk",
@@ -126,6 +126,8 @@ def load() -> ctypes.CDLL:
     L.wc12_linear.argtypes = [vp, u64, u32, u32, vp, u32, vp, vp, vp]
     L.wc_crc32_blocks.restype = i32
     L.wc_crc32_blocks.argtypes = [vp, u64, u64, vp, vp]
+    L.wc_check_coder_division.restype = i32
+    L.wc_check_coder_division.argtypes = [i32, u32, u32, vp, vp]
     _lib = L
     return L
 
@@ -153,7 +155,7 @@ def dtype_code(dtype: torch.dtype) -> int:
     try:
         return _DT[dtype]
     except KeyError:
-        raise TypeError(f"unsupported dtype {dtype}: bf16, fp16, fp32 and fp8 e4m3 only") from None
+        raise TypeError(f"unsupported dtype {dtype}: bf16, fp16, fp32, fp8 e4m3 and fp8 e5m2 only") from None
 
 
 def encode_bound(n: int, dtype) -> int:
@@ -482,6 +484,16 @@ def split12_linear(cont: torch.Tensor, N: int, K: int, x: torch.Tensor, stream=N
     if st != OK:
         raise WCError(st, "wc12_linear (device status)")
     return y
+
+
+def check_coder_division(wide: bool, f_first: int, f_last: int, stream=None) -> tuple[int, int]:
+    """wc_check_coder_division: (mismatches, one failing f << 32 | x) of the
+    encoder's division by f over every state x < f 2^20 (synchronises)."""
+    res = torch.zeros(2, dtype=torch.int64, device="cuda")
+    _check(load().wc_check_coder_division(1 if wide else 0, f_first, f_last, res.data_ptr(),
+                                          _stream(stream)), "wc_check_coder_division")
+    out = res.cpu().tolist()
+    return int(out[0]), int(out[1])
 
 
 CRC_BLOCK = 1 << 20

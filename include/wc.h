@@ -1,7 +1,7 @@
 /*
  * wc.h -- C ABI of the B200 (sm_100a) exponent-plane rANS weight codec.
  *
- * Lossless compression of bf16 / fp32 / fp16 / fp8 e4m3 weight tensors.
+ * Lossless compression of bf16 / fp32 / fp16 / fp8 (e4m3, e5m2) weight tensors.
  * Each float is split into planes; the skewed exponent plane is entropy-coded
  * with a static, 32-lane interleaved rANS coder, chunk by chunk; the sign and
  * mantissa bits are stored raw.  Decoding re-merges the planes into the
@@ -25,9 +25,10 @@
  * u64 off_raw, u64 off_exp, u64 exp_bytes, u64 total_bytes (64 bytes), then
  * u16 freq[256], u64 chunk_off[nc+1], u32 chunk_len[nc], the raw planes
  * (bf16: n sign+mantissa bytes; fp32: ceil(n/8) sign-bit bytes, 3n mantissa
- * bytes; fp16: n low bytes; fp8 e4m3: ceil(n/2) bytes of low nibbles) and
+ * bytes; fp16: n low bytes; fp8: ceil(n/2) bytes of low nibbles) and
  * the exponent chunks (bf16 / fp32: the exponent byte; fp16: the reordered
- * high byte; fp8 e4m3: the exponent nibble).  Values are passed as raw bits
+ * high byte; fp8 e4m3: the exponent nibble; fp8 e5m2: the top four exponent
+ * bits).  Values are passed as raw bits
  * (bf16 / fp16 2 bytes, fp32 4, fp8 1).  A coded chunk is 32 final u32 states then
  * w u16 renormalisation words (128 + 2w bytes); a chunk whose coded form is
  * not smaller than its nsym exponent bytes is stored raw.  The format is
@@ -85,7 +86,12 @@ typedef enum {
  * value is cut into its two nibbles, the exponent nibbles being the coded
  * stream ("PTWM", How it works 1-2); the low nibbles (sign above 3 mantissa
  * bits) are stored raw, two per byte, even value low. */
-typedef enum { WC_BF16 = 1, WC_FP32 = 2, WC_FP16 = 3, WC_FP8E4M3 = 4 } wc_dtype;
+/* WC_FP8E5M2: the same reorder puts the 5 exponent bits on top; the value is
+ * cut into nibbles as for e4m3, so the coded stream is the high nibble
+ * (exponent bits 4..1) and the raw nibble holds exponent bit 0, the sign and
+ * the 2 mantissa bits ("PTWM", Supported dtypes: float8_e5m2 takes the same
+ * bit reorder and 2-plane nibble split as float8_e4m3). */
+typedef enum { WC_BF16 = 1, WC_FP32 = 2, WC_FP16 = 3, WC_FP8E4M3 = 4, WC_FP8E5M2 = 5 } wc_dtype;
 
 /* Worst-case container size in bytes for n values of dtype: every chunk
  * stored raw ("PTWM" Configuration table, compression_threshold: the coded
@@ -181,8 +187,10 @@ WC_API int32_t wc_decode_batch(const wc_decode_item *h_items, uint32_t count,
  * and a failed device-address lookup returns WC_ERR_CUDA.
  *
  * The first call on a device looks up the array's device address with that
- * device current (a host-side lookup, cached per device); make that first call
- * before capturing any stream on that device.  All calls on a GPU share the
+ * device current (a host-side lookup, cached per device and CUDA context: a
+ * call after the context was destroyed and created again, e.g. by
+ * cudaDeviceReset, looks it up again); make that first call before capturing
+ * any stream on that device.  All calls on a GPU share the
  * one array: calls whose work overlaps on the GPU (for example on two streams
  * without ordering between them) race and corrupt each other's output; calls
  * queued on one stream, or otherwise ordered, do not.  The array's contents

@@ -8,16 +8,17 @@ import torch
 from fp32_weight_compression_b200 import wc
 
 
-def to_device(bits: np.ndarray) -> torch.Tensor:
+def to_device(bits: np.ndarray, fp8=torch.float8_e4m3fn) -> torch.Tensor:
     """uint16 bits -> bf16 tensor, float16 values -> fp16 tensor, uint8 bits
-    -> fp8 e4m3 tensor, uint32 bits -> fp32 tensor, on cuda:0."""
+    -> fp8 tensor (e4m3 unless fp8=torch.float8_e5m2), uint32 bits -> fp32
+    tensor, on cuda:0."""
     bits = np.ascontiguousarray(bits)
     if bits.dtype == np.uint16:
         t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
     elif bits.dtype == np.float16:
         t = torch.from_numpy(bits.view(np.int16)).view(torch.float16)
     elif bits.dtype == np.uint8:
-        t = torch.from_numpy(bits.copy()).view(torch.float8_e4m3fn)
+        t = torch.from_numpy(bits.copy()).view(fp8)
     elif bits.dtype == np.uint32:
         t = torch.from_numpy(bits.view(np.int32)).view(torch.float32)
     else:
@@ -31,7 +32,7 @@ def to_bits(t: torch.Tensor) -> np.ndarray:
         return t.view(torch.int16).cpu().numpy().view(np.uint16)
     if t.dtype == torch.float16:
         return t.view(torch.int16).cpu().numpy().view(np.float16)
-    if t.dtype == torch.float8_e4m3fn:
+    if t.dtype in (torch.float8_e4m3fn, torch.float8_e5m2):
         return t.view(torch.uint8).cpu().numpy()
     if t.dtype == torch.float32:
         return t.view(torch.int32).cpu().numpy().view(np.uint32)
@@ -42,9 +43,9 @@ def gpu_encode(bits: np.ndarray) -> np.ndarray:
     return wc.encode(to_device(bits)).cpu().numpy()
 
 
-def gpu_roundtrip(bits: np.ndarray):
+def gpu_roundtrip(bits: np.ndarray, fp8=torch.float8_e4m3fn):
     """(container bytes, decoded bits) through wc_encode / wc_decode."""
-    t = to_device(bits)
+    t = to_device(bits, fp8)
     cont = wc.encode(t)
     out = wc.decode(cont, shape=(bits.size,), dtype=t.dtype)
     torch.cuda.synchronize()

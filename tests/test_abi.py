@@ -40,11 +40,11 @@ def test_every_declared_symbol_is_exported(wcm):
 
 
 @pytest.mark.parametrize("n", [0, 1, 15, 16, 17, 65535, 65536, 65537, 10 ** 6, 123456789])
-@pytest.mark.parametrize("dt", [1, 2])
+@pytest.mark.parametrize("dt", [1, 2, 3, 4, 5])
 def test_bound_matches_oracle(wcm, orc, n, dt):
     assert wcm.encode_bound(n, dt) == orc.encode_bound(n, dt)
     assert wcm.scratch_bytes(n, dt) >= 7424
-    assert wcm.encode_bound(n, 5) == 0
+    assert wcm.encode_bound(n, 6) == 0 and wcm.encode_bound(n, 0) == 0
 
 
 def test_read_header_matches_oracle(wcm, orc):
@@ -95,6 +95,14 @@ def test_bad_arguments_rejected_without_device(wcm):
     assert L.wc_crc32_blocks(None, 1000, 8192, ok_out, None) == wcm.ERR_INVALID_ARG
     assert L.wc_crc32_blocks(None, 0, 8192, None, None) == wcm.OK   # nothing to do
     assert wcm.status_string(4) == "WC_ERR_CORRUPT"
+    # the division self-check: ranges and the result pointer are checked first
+    res = ctypes.c_void_p(0x10000)
+    assert L.wc_check_coder_division(0, 1, 2049, res, None) == wcm.ERR_INVALID_ARG   # narrow <= 2048
+    assert L.wc_check_coder_division(1, 1, 4096, res, None) == wcm.ERR_INVALID_ARG   # f <= 4095
+    assert L.wc_check_coder_division(1, 0, 10, res, None) == wcm.ERR_INVALID_ARG     # f >= 1
+    assert L.wc_check_coder_division(1, 9, 8, res, None) == wcm.ERR_INVALID_ARG      # empty range
+    assert L.wc_check_coder_division(1, 1, 8, None, None) == wcm.ERR_INVALID_ARG
+    assert L.wc_check_coder_division(1, 1, 8, ctypes.c_void_p(0x10004), None) == wcm.ERR_INVALID_ARG
 
 
 def test_product_path_has_no_oracle_dependency():
@@ -296,7 +304,7 @@ def test_headers_are_plain_c_and_link(wcm, tmp_path):
     if shutil.which("gcc") is None:
         pytest.skip("no C compiler")
     names = declared_entry_points()
-    src = ['#include <stdio.h>', '#include "wc.h"', '#include "wc_split12.h"',
+    src = ['#include <stdio.h>', '#include "wc.h"', '#include "wc_split12.h"', '#include "wc_diag.h"',
            'typedef void (*fn_t)(void);',
            'int main(void) {', '  const fn_t fns[] = {']
     src += [f'    (fn_t)&{n},' for n in names]

@@ -377,3 +377,59 @@ def test_raw_fallback_boundary(orc, gu, fname, raw):
     got = _check(orc, gu, bits)
     assert np.array_equal(got, want)
     assert int(want[592:596].view(np.uint32)[0]) == (186 if raw else 184)
+
+
+# fp8 e5m2 (dtype 5): the coded nibble is exponent bits 4..1, the raw nibble
+# exponent bit 0, sign and mantissa ("PTWM", Supported dtypes, float8_e5m2).
+def _e5m2(n, seed):
+    """Bits of e5m2 values with a weight-like skew: exponents around 12."""
+    rng = np.random.default_rng(seed)
+    e = np.clip(rng.normal(12, 2.0, n), 0, 31).astype(np.int64)
+    return ((rng.integers(0, 2, n) << 7) | (e << 2) | rng.integers(0, 4, n)).astype(np.uint8)
+
+
+def _check5(orc, gu, bits):
+    want = orc.encode(bits, dtype=orc.FP8E5M2)
+    got, back = gu.gpu_roundtrip(bits, torch.float8_e5m2)
+    assert got.size == want.size and np.array_equal(got, want)
+    assert np.array_equal(back, bits)
+    return want
+
+
+@pytest.mark.parametrize("n", [0, 1, 2, 3, 15, 16, 17, 33, 511, 513, 65535, 65536, 65537,
+                               3 * C + 17, 5 * C + 511])
+def test_fp8e5m2_edge_sizes(orc, gu, n):
+    _check5(orc, gu, _e5m2(n, seed=n + 21))
+
+
+def test_fp8e5m2_all_patterns_and_kinds(orc, gu):
+    pats = np.arange(256, dtype=np.uint8)
+    _check5(orc, gu, np.tile(pats, 300))                           # near-uniform: raw chunks
+    base = _e5m2(4 * C + 3, seed=22)
+    base[np.random.default_rng(23).choice(base.size, 256, replace=False)] = pats
+    _check5(orc, gu, base)                                        # coded with every pattern
+    _check5(orc, gu, np.full(2 * C + 9, 0x3C, np.uint8))           # single symbol
+    # the golden hand-derived container
+    from _golden import load_container
+    want = load_container("container_fp8e5m2_n4_raw.txt")
+    got = _check5(orc, gu, np.array([0x3C, 0x3C, 0x3C, 0x38], np.uint8))
+    assert np.array_equal(got, want)
+
+
+def test_fp8e5m2_random_access_and_mixed_batch(orc, gu):
+    from fp32_weight_compression_b200 import wc
+    bits = _e5m2(4 * C + 999, seed=24)
+    d = gu.cont_device(orc.encode(bits, dtype=orc.FP8E5M2))
+    for k in range(5):
+        got = wc.decode_chunk(d, k).view(torch.uint8).cpu().numpy()
+        assert np.array_equal(got, bits[k * C:(k + 1) * C])
+    arrs = [_e5m2(2 * C + 7, 25), _fp8(C + 3, 26), _e5m2(101, 27), _normal_bits(77, "bf16", 28)]
+    fp8s = [torch.float8_e5m2, torch.float8_e4m3fn, torch.float8_e5m2, None]
+    ts = [gu.to_device(a, f) if f is not None else gu.to_device(a) for a, f in zip(arrs, fp8s)]
+    conts = wc.encode_batch(ts)
+    for a, f, c in zip(arrs, fp8s, conts):
+        want = orc.encode(a, dtype=orc.FP8E5M2) if f == torch.float8_e5m2 else orc.encode(a)
+        assert np.array_equal(c.cpu().numpy(), want)
+    outs = wc.decode_batch(conts, [(a.size,) for a in arrs], [t.dtype for t in ts])
+    for a, o in zip(arrs, outs):
+        assert np.array_equal(gu.to_bits(o).view(a.dtype), a)

@@ -72,7 +72,7 @@ def test_footprints(wcm, n, dt):
     assert wcm.host_encode_footprint(n, dt) == (r256(n * e) + r256(wcm.encode_bound(n, dt))
                                                 + r256(wcm.scratch_bytes(n, dt)) + 8)
     assert wcm.host_decode_footprint(1000, n, dt) == r256(1000) + r256(n * e)
-    assert wcm.host_encode_footprint(n, 5) == 0
+    assert wcm.host_encode_footprint(n, 6) == 0
 
 
 def test_bad_arguments_rejected_before_device(wcm, orc):
@@ -85,7 +85,7 @@ def test_bad_arguments_rejected_before_device(wcm, orc):
     assert L.wc_encode_host(it, 0, None, 0, 0, None, None, None) == wcm.OK
     assert L.wc_encode_host(None, 1, 256, 1 << 20, 0, None, None, None) == wcm.ERR_INVALID_ARG
     assert L.wc_encode_host(it, 1, 257, 1 << 20, 0, None, None, None) == wcm.ERR_INVALID_ARG
-    it[0].dtype = 5
+    it[0].dtype = 6
     assert L.wc_encode_host(it, 1, 256, 1 << 20, 0, None, None, None) == wcm.ERR_INVALID_ARG
     it[0].dtype, it[0].h_out_cap = 1, 10          # below wc_encode_bound
     assert L.wc_encode_host(it, 1, 256, 1 << 20, 0, None, None, None) == wcm.ERR_CAPACITY
