@@ -595,7 +595,8 @@ def split12_leg(ins, dev, stream, reps: int = 5):
 def linear_leg(ins, specs_mine, dev, reps: int = 20):
     """wc12_linear (Y = X W^T with W held as a Split12 container, expanded
     into the tensor cores' operand layout inside the kernel) against
-    torch.matmul on the bf16 weights (cuBLAS), for token counts M = 1 .. 256.
+    torch.matmul on the bf16 weights (cuBLAS), for token counts M = 1 .. 256
+    (M <= 8: the library's CUDA-core path; more: its tensor-core path).
     W: the first four gate projections of the set (4096 x 14336 bf16, 117 MB
     each, 470 MB together > L2), used in rotation so that every call reads its
     weights from HBM.  Reported per M: microseconds per call and the weight
@@ -611,7 +612,7 @@ def linear_leg(ins, specs_mine, dev, reps: int = 20):
     L = wc.load()
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     out = {}
-    for M in (1, 16, 64, 256):
+    for M in (1, 2, 4, 8, 16, 64, 256):
         x = torch.randn(M, K, device=dev, dtype=torch.float32).to(torch.bfloat16)
         y = torch.empty(M, N, dtype=torch.float32, device=dev)
         s = torch.cuda.current_stream(dev).cuda_stream

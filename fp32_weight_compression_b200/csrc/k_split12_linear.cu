@@ -360,6 +360,165 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   }
 }
 
+// ---------------------------------------------------------------------------
+// Few tokens (M <= kGemvMaxM): the layer is bound by reading W, so it runs on
+// the CUDA cores, one warp per weight row, streaming the row's index nibbles
+// and low bytes (12 bits a value) and expanding them in registers: each lane
+// takes 16 consecutive values per step of 512, expands them with the
+// codebook (four byte permutes and a select per 4 values), patches the
+// tile's exceptions, and adds the exact bf16 x bf16 products into fp32 sums
+// (one per token); a warp reduction ends the row.  Exceptions are met in
+// order: a warp-uniform cursor walks the container's exception list, which
+// is sorted by position within each chunk and chunk after chunk.
+constexpr int kGemvWarps = 8;
+constexpr uint32_t kGemvMaxM = 8;
+
+template <int MT>
+__global__ void __launch_bounds__(kGemvWarps * 32) k12_gemv(const __grid_constant__ Params p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint32_t K = p.K, N = p.N;
+  const uint8_t *w = p.w;
+  const uint32_t *h32 = reinterpret_cast<const uint32_t *>(w);
+  const uint64_t *h64 = reinterpret_cast<const uint64_t *>(w);
+  const uint64_t n = h64[1], ne = h64[3];
+  const uint32_t kk = h32[1] >> 24;
+  bool ok = h32[0] == wc12::kMagic && (h32[1] & 0xFFFFFFu) == (1u | (1u << 16)) &&
+            kk >= 1 && kk <= 16 && n == uint64_t(N) * K && ne <= n && h32[4] == uint32_t(kChunk);
+  wc12::Lay L{};
+  if (ok) {
+    L = wc12::lay(n, ne);
+    ok = h32[5] == uint32_t(L.nc) && h64[4] == L.off_idx && h64[5] == L.off_lo && h64[6] == L.off_exc &&
+         h64[7] == L.total && L.total <= p.w_bytes;
+  }
+  if (!ok) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) report(p.status, WC_ERR_CORRUPT);
+    return;
+  }
+  const uint32_t row = blockIdx.x * kGemvWarps + warp;
+  if (row >= N) return;
+  const uint4 book = *reinterpret_cast<const uint4 *>(w + wc12::kBookOff);
+  const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(w + wc12::kExcOffOff);
+  const uint16_t *exc_pos = reinterpret_cast<const uint16_t *>(w + L.off_exc);
+  const uint8_t *exc_val = w + L.off_excval;
+  const uint8_t *idx_plane = w + L.off_idx;
+  const uint8_t *lo_plane = w + L.off_lo;
+  const uint64_t r0 = uint64_t(row) * K;
+
+  // exception cursor: chunk c, list index e = the first exception at or
+  // after value r0 (a search in chunk c's sorted positions)
+  uint64_t c = r0 / kChunk;
+  uint64_t c_end = exc_off[c + 1];
+  uint64_t e;
+  {
+    uint64_t lo = exc_off[c], hi = c_end;
+    if (lo > hi || hi > ne) {
+      if (lane == 0) report(p.status, WC_ERR_CORRUPT);
+      return;
+    }
+    const uint32_t target = uint32_t(r0 % kChunk);
+    while (lo < hi) {
+      const uint64_t mid = (lo + hi) >> 1;
+      if (exc_pos[mid] < target) lo = mid + 1; else hi = mid;
+    }
+    e = lo;
+  }
+
+  float acc[MT];
+#pragma unroll
+  for (int m = 0; m < MT; m++) acc[m] = 0.0f;
+  for (uint32_t k0 = 0; k0 < K; k0 += 512) {
+    const uint32_t col = k0 + 16 * lane;
+    const bool act = col < K;  // K is a multiple of 64: a lane holds 16 values or none
+    uint2 iw = make_uint2(0, 0);
+    uint4 lw = make_uint4(0, 0, 0, 0);
+    if (act) {
+      iw = __ldg(reinterpret_cast<const uint2 *>(idx_plane + (r0 + col) / 2));
+      lw = __ldg(reinterpret_cast<const uint4 *>(lo_plane + r0 + col));
+    }
+    uint32_t v[8];
+    {
+      const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
+      const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
+      v[0] = e0.x; v[1] = e0.y; v[2] = e1.x; v[3] = e1.y; v[4] = e2.x; v[5] = e2.y; v[6] = e3.x; v[7] = e3.y;
+    }
+    // the exceptions among values [r0 + k0, r0 + min(k0 + 512, K))
+    const uint64_t s0 = r0 + k0, s1 = r0 + (k0 + 512 < K ? k0 + 512 : K);
+    for (;;) {
+      while (e >= c_end && c + 1 < L.nc) {  // on to the next chunk's list
+        c++;
+        const uint64_t nxt = exc_off[c + 1];
+        if (exc_off[c] != c_end || nxt < c_end || nxt > ne) {
+          if (lane == 0) report(p.status, WC_ERR_CORRUPT);
+          return;
+        }
+        c_end = nxt;
+      }
+      if (e >= c_end) break;
+      const uint32_t cpos = exc_pos[e];
+      const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
+      if (cpos >= cnt) {
+        if (lane == 0) report(p.status, WC_ERR_CORRUPT);
+        return;
+      }
+      const uint64_t pos = c * kChunk + cpos;
+      if (pos >= s1) break;
+      if (pos >= s0) {
+        const uint32_t rel = uint32_t(pos - s0);
+        if (lane == int(rel >> 4)) {
+          const uint32_t j = rel & 15u;
+          const uint32_t lo = (j < 4 ? lw.x : j < 8 ? lw.y : j < 12 ? lw.z : lw.w) >> (8 * (j & 3)) & 0xFFu;
+          const uint32_t val = (uint32_t(exc_val[e]) << 8) | lo;
+#pragma unroll
+          for (int q = 0; q < 8; q++)
+            if (int(j >> 1) == q) v[q] = (j & 1u) ? ((v[q] & 0xFFFFu) | (val << 16)) : ((v[q] & 0xFFFF0000u) | val);
+        }
+      }
+      e++;
+    }
+    if (act) {
+#pragma unroll
+      for (int m = 0; m < MT; m++) {
+        const uint4 *xp = reinterpret_cast<const uint4 *>(p.x + uint64_t(m) * K + col);
+        const uint4 xa = __ldg(xp), xb = __ldg(xp + 1);
+        const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
+        float a = acc[m];
+#pragma unroll
+        for (int q = 0; q < 8; q++) {
+          a = fmaf(__uint_as_float(v[q] << 16), __uint_as_float(xw[q] << 16), a);
+          a = fmaf(__uint_as_float(v[q] & 0xFFFF0000u), __uint_as_float(xw[q] & 0xFFFF0000u), a);
+        }
+        acc[m] = a;
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; m++) {
+    float a = acc[m];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) p.y[uint64_t(m) * N + row] = a;
+  }
+}
+
+template <int MT>
+cudaError_t launch_gemv(const Params &p, cudaStream_t s) {
+  k12_gemv<MT><<<(p.N + kGemvWarps - 1) / kGemvWarps, kGemvWarps * 32, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemv_m(const Params &p, cudaStream_t s) {
+  switch (p.M) {
+    case 1: return launch_gemv<1>(p, s);
+    case 2: return launch_gemv<2>(p, s);
+    case 3: return launch_gemv<3>(p, s);
+    case 4: return launch_gemv<4>(p, s);
+    case 5: return launch_gemv<5>(p, s);
+    case 6: return launch_gemv<6>(p, s);
+    case 7: return launch_gemv<7>(p, s);
+    default: return launch_gemv<8>(p, s);
+  }
+}
+
 __global__ void k12_zero(float *y, uint64_t count) {
   for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
        i += uint64_t(gridDim.x) * blockDim.x)
@@ -429,8 +588,6 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   if (N == 0 || K == 0 || N % wc12l::kBM != 0 || K % wc12l::kBK != 0 || M == 0)
     return WC_ERR_INVALID_ARG;
   if (w_bytes < 96) return WC_ERR_INVALID_ARG;  // shorter than any container's header
-  const wc12l::DevInfo di = wc12l::dev_info();
-  if (di.sms <= 0 || !di.attr) return WC_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   wc12l::Params p;
   p.w = static_cast<const uint8_t *>(d_w);
@@ -438,6 +595,16 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   p.N = N;
   p.K = K;
   p.status = d_status;
+  if (M <= wc12l::kGemvMaxM) {  // reading W bounds it: CUDA cores, no tensor memory
+    p.x = static_cast<const uint16_t *>(d_x);
+    p.y = d_y;
+    p.M = M;
+    p.n_mma = 0;
+    p.per_split = p.splits = 1;
+    return wc12l::launch_gemv_m(p, s) == cudaSuccess ? WC_OK : WC_ERR_CUDA;
+  }
+  const wc12l::DevInfo di = wc12l::dev_info();
+  if (di.sms <= 0 || !di.attr) return WC_ERR_CUDA;
   const uint32_t blocks = N / wc12l::kBM, stages = K / wc12l::kBK;
   // split K until the grid covers the SMs twice, at least two stages a CTA
   uint32_t splits = (2 * uint32_t(di.sms) + blocks - 1) / blocks;

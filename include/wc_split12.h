@@ -77,14 +77,17 @@ WC_API int32_t wc12_read_header(const void *h_cont, uint64_t bytes, uint64_t *n,
 WC_API int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out, uint64_t out_cap,
                            int32_t *d_status, void *stream);
 
-/* Y = X W^T with W (N x K bf16, row-major) given as a Split12 container:
- * the weights are expanded tile by tile into the tensor cores' operand
- * layout and multiplied with tcgen05.mma (fp32 accumulate), so they cross
- * HBM at 12 bits a value.
+/* Y = X W^T with W (N x K bf16, row-major) given as a Split12 container, the
+ * weights crossing HBM at 12 bits a value ("weight-compression" README:
+ * serving with the weights kept in this format).  For M <= 8 tokens the
+ * layer is bound by reading W and runs on the CUDA cores, a warp per weight
+ * row expanding the values in registers; for more tokens the weights are
+ * expanded tile by tile into the tensor cores' operand layout and multiplied
+ * with tcgen05.mma.  Both accumulate exact bf16 products in fp32.
  *   d_w, w_bytes  the container (16-byte aligned, at least 96 bytes), n = N * K
  *   N, K          N a multiple of 128, K a multiple of 64
- *   d_x           M x K bf16, row-major, 16-byte aligned; M >= 1 (taken in
- *                 slices of 256 tokens, one launch each)
+ *   d_x           M x K bf16, row-major, 16-byte aligned; M >= 1 (more than 8
+ *                 are taken in slices of 256 tokens, one launch each)
  *   d_y           M x N fp32, row-major (overwritten)
  *   d_status      device i32 set to 0 by the caller: WC_ERR_CORRUPT for a bad
  *                 container, WC_ERR_TIMEOUT if a bounded wait ran out

@@ -2,7 +2,9 @@
 Y = X W^T with W held as a Split12 container ("weight-compression" README:
 bf16 weights rebuilt from a codebook index and the raw low byte inside the
 serving kernels), against the oracle's float64 sum of the exact bf16
-products (oracle/split12.py linear).
+products (oracle/split12.py linear).  M <= 8 runs on the CUDA cores (one
+warp per weight row), larger M on the tensor cores (tcgen05); both are
+covered.
 
 Tolerance, from the arithmetic: every product of two bf16 values is exact in
 fp32, so an output is a sum of K exact terms; the tensor cores and the split-K
@@ -92,7 +94,7 @@ def test_one_small_shape_first(s12):
 
 
 @pytest.mark.parametrize("N,K", [(128, 64), (256, 128), (128, 4096), (256, 4096)])
-@pytest.mark.parametrize("M", [1, 17, 144, 256, 300])
+@pytest.mark.parametrize("M", [1, 3, 8, 9, 17, 144, 256, 300])
 def test_shapes(s12, N, K, M):
     _check(s12, N, K, M, seed=N + K + M)
 
@@ -102,21 +104,23 @@ def test_exceptions_in_the_tile(s12, K):
     """Outliers become exceptions: a few per tile (gathered into the CTA's
     list) and, at 20 %, more than the list holds (walked per stage)."""
     for frac in (0.002, 0.2):
-        ne = _check(s12, 256, K, 33, seed=K + int(frac * 1000), outliers=frac)
-        assert ne > 0
+        for M in (4, 33):  # the CUDA-core path (M <= 8) and the tensor-core path
+            ne = _check(s12, 256, K, M, seed=K + int(frac * 1000) + M, outliers=frac)
+            assert ne > 0
 
 
 def test_corrupt_header_is_reported(s12):
     from fp32_weight_compression_b200 import wc
     N, K = 128, 128
     cont = s12.encode(_weights(N, K, 3))
-    x = _bf16_dev(workloads.rne_bf16(np.ones(K, np.float32))).view(1, K)
-    for off, val in ((0, 0x00), (8, 0x01), (16, 0x00)):   # magic, n, chunk size
-        bad = cont.copy()
-        bad[off] ^= 0xFF if val == 0 else val
-        with pytest.raises(wc.WCError) as ei:
-            wc.split12_linear(torch.from_numpy(bad).to("cuda"), N, K, x)
-        assert ei.value.code == wc.ERR_CORRUPT
-    # the intact container still works after the refusals
-    y = wc.split12_linear(torch.from_numpy(cont).to("cuda"), N, K, x)
-    assert torch.isfinite(y).all()
+    for M in (1, 17):  # both paths
+        x = _bf16_dev(workloads.rne_bf16(np.ones(M * K, np.float32))).view(M, K)
+        for off, val in ((0, 0x00), (8, 0x01), (16, 0x00)):   # magic, n, chunk size
+            bad = cont.copy()
+            bad[off] ^= 0xFF if val == 0 else val
+            with pytest.raises(wc.WCError) as ei:
+                wc.split12_linear(torch.from_numpy(bad).to("cuda"), N, K, x)
+            assert ei.value.code == wc.ERR_CORRUPT
+        # the intact container still works after the refusals
+        y = wc.split12_linear(torch.from_numpy(cont).to("cuda"), N, K, x)
+        assert torch.isfinite(y).all()
