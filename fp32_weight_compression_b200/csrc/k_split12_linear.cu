@@ -6,19 +6,21 @@
 // compression" README: Split12 serving, bf16 weights rebuilt on the fly).
 //
 // Work split.  A CTA owns 128 weight rows (the MMA's M) and a range of K;
-// the host splits K across CTAs until the grid covers the SMs, and the CTAs
+// the host splits K across CTAs so that the grid is one wave, and the CTAs
 // of one row block add their partial sums into Y (fp32 atomics; Y is zeroed
 // first).  Per stage of 64 K-values:
-//   * the 128 threads expand the block's 128 x 64 values in segments of 16
-//     (8 index bytes + 16 low bytes -> 16 bf16, two 16-byte rows of core
-//     matrices), four threads per row, so a warp's loads touch 8 lines;
-//   * the tokens' X slice (n_mma x 64, rows past M zero) is copied the same
-//     way; the chunks' exceptions that fall in the tile are patched in;
+//   * cp.async brings the rows' 64 index nibbles and 64 low bytes each (12
+//     bits a value, as stored) and the tokens' X slice (n_mma x 64, rows past
+//     M zero-filled, straight into the B operand layout) into a ring slot,
+//     three stages ahead of the stage being expanded;
+//   * the 128 threads expand the 128 x 64 values from the ring slot in
+//     segments of 16 (8 index bytes + 16 low bytes -> 16 bf16, two 16-byte
+//     rows of core matrices) into one of two A operand slots and patch the
+//     tile's exceptions;
 //   * one thread issues four MMAs (M = 128, N = n_mma = M rounded up to 16,
-//     K = 16) and commits them to the stage's mbarrier.
-// Two stages alternate, so the expansion of one overlaps the MMAs of the
-// other.  At the end each warp reads its 32 TMEM lanes (rows) and adds them
-// into Y.
+//     K = 16) and commits them to the slot's mbarrier; once the previous
+//     stage's MMAs are done its ring slot takes the next loads.
+// At the end each warp reads its 32 TMEM lanes (rows) and adds them into Y.
 //
 // Operand layout (K-major, no swizzle): a core matrix is 8 rows x 16 bytes
 // stored as 128 contiguous bytes; the two 8-value halves of a K = 16 slice
@@ -64,9 +66,18 @@ struct Params {
   int32_t *status;
 };
 
+// Shared memory: two expanded A operand slots, then a ring of kDepth load
+// slots (the stage's index bytes and low bytes of the 128 rows, as stored,
+// and the tokens' X slice already in the B operand layout), the mbarriers,
+// and the CTA's exception list.
+constexpr uint32_t kDepth = 4;
+constexpr uint32_t kIdxBytes = kBM * kBK / 2;  // 4 KiB
+constexpr uint32_t kLoBytes = kBM * kBK;       // 8 KiB
+
 __host__ __device__ inline uint32_t b_stage_bytes(uint32_t n_mma) { return n_mma * kBK * 2; }
+__host__ __device__ inline uint32_t slot_bytes(uint32_t n_mma) { return kIdxBytes + kLoBytes + b_stage_bytes(n_mma); }
 __host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma) {
-  return 1024 + 2 * kAStage + 2 * b_stage_bytes(n_mma) + 64 + 8 * kExcCap;
+  return 1024 + 2 * kAStage + kDepth * slot_bytes(n_mma) + 64 + 8 * kExcCap;
 }
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
@@ -138,14 +149,21 @@ __device__ __forceinline__ uint32_t op_offset(uint32_t row, uint32_t k, uint32_t
   return (k >> 4) * slice_bytes + (row >> 3) * 256 + ((k >> 3) & 1) * 128 + (row & 7) * 16 + (k & 7) * 2;
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant__ Params p) {
   extern __shared__ uint8_t dyn[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
-  uint8_t *a_st = base;                       // 2 x kAStage
-  uint8_t *b_st = base + 2 * kAStage;         // 2 x b_stage_bytes
-  const uint32_t b_bytes = b_stage_bytes(p.n_mma);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(b_st + 2 * b_bytes);
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + 2);
+  uint8_t *a_op = base;                       // 2 x kAStage
+  uint8_t *ring = base + 2 * kAStage;         // kDepth x slot_bytes
+  const uint32_t sb = slot_bytes(p.n_mma);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(ring + kDepth * sb);  // kDepth
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + kDepth);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
   uint32_t *exc_n = tmem_slot + 2;
   uint2 *exc_list = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(bar) + 64);
@@ -178,12 +196,39 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     if (!ok && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) report(p.status, WC_ERR_CORRUPT);
     return;
   }
+  const uint32_t nst = s_end - s_begin;
   const uint4 book = *reinterpret_cast<const uint4 *>(w + wc12::kBookOff);
   const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(w + wc12::kExcOffOff);
   const uint16_t *exc_pos = reinterpret_cast<const uint16_t *>(w + L.off_exc);
   const uint8_t *exc_val = w + L.off_excval;
+  const uint8_t *idx_plane = w + L.off_idx;
   const uint8_t *lo_plane = w + L.off_lo;
   const uint64_t c_lo = uint64_t(n0) * K / kChunk, c_hi = (uint64_t(n0 + kBM) * K - 1) / kChunk;
+
+  // the loads of stage j (of this CTA) into ring slot j % kDepth: the rows'
+  // index and low bytes as stored, and the tokens' X slice straight into the
+  // B operand layout (one 16-byte core-matrix row per copy; tokens >= M are
+  // zero-filled)
+  const uint32_t ring_s = smem_u32(ring);
+  auto issue_loads = [&](uint32_t j) {
+    const uint32_t slot = ring_s + (j % kDepth) * sb;
+    const uint32_t k0 = (s_begin + j) * kBK;
+    const uint32_t total = 3 * kBM * 2 + p.n_mma * 8;  // 256 index + 512 low + B copies
+    for (uint32_t i = tid; i < total; i += kThreads) {
+      if (i < 2 * kBM) {
+        const uint32_t row = i >> 1, part = i & 1;
+        cp_async16(slot + row * 32 + 16 * part, idx_plane + (uint64_t(n0 + row) * K + k0) / 2 + 16 * part, 16);
+      } else if (i < 6 * kBM) {
+        const uint32_t j2 = i - 2 * kBM, row = j2 >> 2, part = j2 & 3;
+        cp_async16(slot + kIdxBytes + row * 64 + 16 * part, lo_plane + uint64_t(n0 + row) * K + k0 + 16 * part, 16);
+      } else {
+        const uint32_t j3 = i - 6 * kBM, t = j3 >> 3, jj = j3 & 7;
+        const bool real = t < p.M;
+        cp_async16(slot + kIdxBytes + kLoBytes + op_offset(t, 8 * jj, p.n_mma * 32),
+                   real ? static_cast<const void *>(p.x + uint64_t(t) * K + k0 + 8 * jj) : p.x, real ? 16 : 0);
+      }
+    }
+  };
 
   // tensor memory: n_mma fp32 columns, rounded up to a power of two >= 32
   uint32_t cols = 32;
@@ -195,11 +240,16 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (uint32_t d = 0; d < kDepth; d++) mbar_init(&bar[d], 1);
     *flag = 0;
     *exc_n = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // the first kDepth - 1 stages' loads are in flight while the exceptions
+  // are gathered
+  for (uint32_t j = 0; j + 1 < kDepth; j++) {
+    if (j < nst) issue_loads(j);
+    cp_async_commit();
   }
   fence_before_sync();
   __syncthreads();
@@ -247,39 +297,25 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   const bool exc_walk = n_exc > kExcCap;
 
   uint32_t it = 0;
-  for (uint32_t st = s_begin; st < s_end; st++, it++) {
-    const uint32_t buf = it & 1u;
-    if (it >= 2) {  // this buffer's MMAs of two stages ago must be done
-      if (!mbar_wait(&bar[buf], ((it - 2) >> 1) & 1u)) {
-        if (tid == 0) report(p.status, WC_ERR_TIMEOUT);
-        *flag = 1;
-      }
-      __syncthreads();
-      if (*flag) break;
-    }
-    uint8_t *A = a_st + buf * kAStage;
-    uint8_t *B = b_st + buf * b_bytes;
+  for (; it < nst; it++) {
+    const uint32_t st = s_begin + it;
     const uint32_t k0 = st * kBK;
+    uint8_t *A = a_op + (it & 1) * kAStage;
+    const uint8_t *slot = ring + (it % kDepth) * sb;
+    cp_async_wait<kDepth - 2>();  // this stage's loads (later stages may still be in flight)
+    __syncthreads();
 
     // A: 512 segments of 16 values (row = i / 4, values 16 (i % 4) ..), four
-    // per thread; a warp covers 8 rows, so its loads touch 8 lines, not 32
+    // per thread, expanded from the ring slot into the operand slot
 #pragma unroll
     for (int q = 0; q < 4; q++) {
       const uint32_t i = uint32_t(tid) + kThreads * q, row = i >> 2, seg = i & 3;
-      const uint64_t f = uint64_t(n0 + row) * K + k0 + 16 * seg;
-      const uint2 iw = __ldg(reinterpret_cast<const uint2 *>(w + L.off_idx + f / 2));
-      const uint4 lw = __ldg(reinterpret_cast<const uint4 *>(lo_plane + f));
+      const uint2 iw = *reinterpret_cast<const uint2 *>(slot + row * 32 + 8 * seg);
+      const uint4 lw = *reinterpret_cast<const uint4 *>(slot + kIdxBytes + row * 64 + 16 * seg);
       const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
       const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
       *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg, kASlice)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
       *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg + 8, kASlice)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
-    }
-    // B: the tokens' slice of X, rows >= M zero
-    for (uint32_t i = tid; i < p.n_mma * 8; i += kThreads) {
-      const uint32_t t = i >> 3, j = i & 7;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < p.M) v = __ldg(reinterpret_cast<const uint4 *>(p.x + uint64_t(t) * K + k0 + 8 * j));
-      *reinterpret_cast<uint4 *>(B + op_offset(t, 8 * j, p.n_mma * 32)) = v;
     }
     __syncthreads();
     // exceptions that fall in this tile
@@ -311,21 +347,38 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     __syncthreads();
     if (tid == 0) {
       fence_after_sync();
-      const uint32_t a0 = smem_u32(A), b0 = smem_u32(B);
+      const uint32_t a0 = smem_u32(A), b0 = smem_u32(slot + kIdxBytes + kLoBytes);
 #pragma unroll
-      for (uint32_t s = 0; s < 4; s++)
-        mma_bf16(tmem, operand_desc(a0 + s * kASlice), operand_desc(b0 + s * p.n_mma * 32), idesc,
-                 (it > 0 || s > 0) ? 1u : 0u);
-      mma_commit(&bar[buf]);
+      for (uint32_t sl = 0; sl < 4; sl++)
+        mma_bf16(tmem, operand_desc(a0 + sl * kASlice), operand_desc(b0 + sl * p.n_mma * 32), idesc,
+                 (it > 0 || sl > 0) ? 1u : 0u);
+      mma_commit(&bar[it % kDepth]);
     }
+    // the slot of stage it - 1 is free once its MMAs are done (which also
+    // frees the A slot stage it + 1 writes): load stage it + kDepth - 1 there
+    if (it >= 1) {
+      const uint32_t prev = it - 1;
+      if (!mbar_wait(&bar[prev % kDepth], (prev / kDepth) & 1u)) {
+        if (tid == 0) report(p.status, WC_ERR_TIMEOUT);
+        *flag = 1;
+      }
+      __syncthreads();
+      if (*flag) {
+        it++;  // stage it was issued
+        break;
+      }
+    }
+    if (it + kDepth - 1 < nst) issue_loads(it + kDepth - 1);
+    cp_async_commit();
   }
+  cp_async_wait<0>();
 
   // wait for the last stage issued (its commit covers all earlier MMAs)
   const uint32_t issued = it;
   bool done = true;
   if (issued > 0) {
     const uint32_t last = issued - 1;
-    done = mbar_wait(&bar[last & 1u], (last >> 1) & 1u);
+    done = mbar_wait(&bar[last % kDepth], (last / kDepth) & 1u);
   }
   // every thread takes the same branch below: the tensor-memory loads are
   // warp-collective (.sync.aligned)
@@ -606,12 +659,7 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   const wc12l::DevInfo di = wc12l::dev_info();
   if (di.sms <= 0 || !di.attr) return WC_ERR_CUDA;
   const uint32_t blocks = N / wc12l::kBM, stages = K / wc12l::kBK;
-  // split K until the grid covers the SMs twice, at least two stages a CTA
-  uint32_t splits = (2 * uint32_t(di.sms) + blocks - 1) / blocks;
-  if (splits > stages / 2) splits = stages / 2;
-  if (splits < 1) splits = 1;
-  p.per_split = (stages + splits - 1) / splits;
-  p.splits = (stages + p.per_split - 1) / p.per_split;
+  if (blocks == 0) return WC_ERR_INVALID_ARG;
   // tokens in slices of at most kMaxTokens (the MMA's N); each slice's rows
   // of X and Y are contiguous
   for (uint32_t t0 = 0; t0 < M; t0 += wc12l::kMaxTokens) {
@@ -620,9 +668,23 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
     p.y = d_y + uint64_t(t0) * N;
     p.M = m;
     p.n_mma = (m + 15) / 16 * 16;
+    // split K so that the grid is one wave of the CTAs an SM holds, with at
+    // least 4 stages a CTA when K allows (the load ring runs 3 ahead)
+    const uint32_t smem = wc12l::launch_smem(di, p.n_mma);
+    uint32_t cols = 32;
+    while (cols < p.n_mma) cols <<= 1;
+    uint32_t per_sm = uint32_t(di.smem_per_sm) / (smem + uint32_t(di.smem_reserved));
+    if (per_sm > 512 / cols) per_sm = 512 / cols;
+    if (per_sm < 1) per_sm = 1;
+    uint32_t splits = uint32_t(di.sms) * per_sm / blocks;
+    const uint32_t most = stages / 4 > 0 ? stages / 4 : 1;
+    if (splits > most) splits = most;
+    if (splits < 1) splits = 1;
+    p.per_split = (stages + splits - 1) / splits;
+    p.splits = (stages + p.per_split - 1) / p.per_split;
     if (p.splits > 1) wc12l::k12_zero<<<unsigned(2 * di.sms), 256, 0, s>>>(p.y, uint64_t(m) * N);
     dim3 grid(blocks, p.splits);
-    wc12l::k12_linear<<<grid, wc12l::kThreads, wc12l::launch_smem(di, p.n_mma), s>>>(p);
+    wc12l::k12_linear<<<grid, wc12l::kThreads, smem, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
   }
   return WC_OK;
