@@ -416,7 +416,7 @@ class DeviceSet:
         self.dec = wc.BatchDecoder(device=dev).prepare(conts_cap, self.outs)
         self.bytes = int(sum(nbytes))
         self.n = len(numels)
-        self.launches_per_step = 3 * ((self.n + 255) // 256)   # k_prep, k_encode, k_decode
+        self.launches_per_step = 5 * ((self.n + 255) // 256)   # k_prep, k_hist, k_coder, k_compact, k_decode
 
     def check(self):
         import torch

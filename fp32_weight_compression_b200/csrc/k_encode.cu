@@ -16,8 +16,8 @@
 //   if x >= f 2^20: emit x & 0xFFFF, x >>= 16;   x = (x / f) 4096 + x % f + cum_s
 // with x / f computed exactly by a multiply-high and a shift when every f of
 // the tensor is at most 2048 (the usual case), else by a 64-bit reciprocal in
-// two 32-bit halves (see publish_table); the coder is compiled for both and
-// each block takes the form its tensor's table was written in.  The lanes
+// two 32-bit halves (wc_coder.cuh); the coder is compiled for both and each
+// block takes the form its tensor's table was written in.  The lanes
 // that emit at a step form one block of the word stream, in ascending lane
 // order, placed with __ballot_sync / __popc prefix offsets; blocks are laid
 // down back to front, so the decoder (which runs the steps forwards) reads
@@ -29,7 +29,6 @@
 #include "wc_block.cuh"
 #include "wc_coder.cuh"
 #include "wc_format.cuh"
-#include "wc_hist.cuh"
 #include "wc_planes.cuh"
 
 namespace wc {
@@ -41,7 +40,6 @@ constexpr int kCoderThreads = kCoderWarps * 32;
 __shared__ uint4 s_tab[256];
 __shared__ uint32_t s_bias[256];
 __shared__ __align__(16) uint8_t s_ebuf[kCoderWarps][2][kGroupValues];
-__shared__ uint32_t s_len[kCoderWarps][2];
 
 // ---------------------------------------------------------------------------
 // 16 consecutive 2-byte values (bf16 or fp16, 8 words) of one lane: their
@@ -148,25 +146,22 @@ __device__ __forceinline__ void cstep_checked(uint32_t &x, uint32_t &tail, uint1
 }
 
 struct CoderOut {
-  uint32_t *lens;  // the warp's two chunk lengths (shared memory)
-  uint64_t k0;     // the warp's first chunk
-  uint8_t *win0;   // window of chunk 0 of the tensor
+  uint32_t *lens;
+  uint8_t *win0;  // window of chunk 0 of the tensor
 };
 
-// A chunk's stored length: 128 + 2w if that is smaller than nsym, else nsym
-// (raw).  A coded chunk's final states go to the front of its window.
 __device__ __forceinline__ void finish_chunk(const CoderOut &co, uint64_t k, uint32_t nsym, uint32_t x,
                                              uint32_t tail, bool bail, int lane) {
   const uint32_t w = kWinWords - tail;
   const bool raw = bail || (kStateBytes + 2 * w >= nsym);
   const uint32_t len = raw ? nsym : kStateBytes + 2 * w;
   if (!raw) reinterpret_cast<uint32_t *>(co.win0 + k * kWin)[lane] = x;
-  if (lane == 0) co.lens[k - co.k0] = len;
+  if (lane == 0) co.lens[k] = len;
 }
 
 // Two full 2-byte-value chunks (bf16 or fp16) kA, kA + 1 in lock-step.
 template <int DT, bool W>
-__device__ __forceinline__ void code_pair16(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
+__device__ void code_pair16(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
                                const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
@@ -250,7 +245,7 @@ __device__ __forceinline__ void split_fp32x16(const Fp32x16 &v, uint8_t *out, co
 // group's values are loaded into the registers the current group's split
 // has just freed).
 template <bool W>
-__device__ __forceinline__ void code_pair_fp32(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
+__device__ void code_pair_fp32(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
                                const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
@@ -301,7 +296,7 @@ __device__ __forceinline__ void code_pair_fp32(const EncItem &it, const Layout &
 // Two full fp8 e4m3 chunks kA, kA + 1 in lock-step (as code_pair16: 16
 // values are one 16-byte load; their low nibbles are 8 bytes of the plane).
 template <int DT, bool W>
-__device__ __forceinline__ void code_pair8(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
+__device__ void code_pair8(const EncItem &it, const Layout &L, uint64_t kA, const uint4 *tab,
                            const uint32_t *bias, uint8_t *ebA, uint8_t *ebB, const CoderOut &co) {
   const int lane = threadIdx.x & 31;
   const uint32_t lt = lanemask_lt();
@@ -462,446 +457,75 @@ __device__ __forceinline__ void code_warp(const EncItem &it, const Layout &L, ui
   }
 }
 
-// ---------------------------------------------------------------------------
-// Header fields, padding and scratch counters (one block per tensor).
-__global__ void __launch_bounds__(256) k_prep(const __grid_constant__ EncParams p) {
-  const EncItem &it = p.items[blockIdx.x];
-  const int tid = threadIdx.x;
-  const int dtype = int(it.dtype);
-  const Layout L = make_layout(it.n, dtype);
-  uint8_t *out = it.out;
-
-  uint64_t *hist = reinterpret_cast<uint64_t *>(it.scratch + kScrHist);
-  uint32_t *ctr = reinterpret_cast<uint32_t *>(it.scratch + kScrCtr);
-  uint64_t *stat = reinterpret_cast<uint64_t *>(it.scratch + kScrStat);
-  hist[tid] = 0;
-  if (tid < 4) ctr[tid] = 0;
-  for (uint64_t k = tid; k < L.nc; k += 256) stat[k] = 0;
-
-  // table: all zero until the last histogram tile writes it (n = 0 keeps it)
-  reinterpret_cast<uint16_t *>(out + kFreqOffset)[tid] = 0;
-
-  if (tid == 0) {
-    uint32_t *h32 = reinterpret_cast<uint32_t *>(out);
-    uint64_t *h64 = reinterpret_cast<uint64_t *>(out);
-    h32[0] = 0x315A4357u;  // "WCZ1"
-    h32[1] = kVersion | (uint32_t(dtype) << 16) | (kLanes << 24);
-    h64[1] = it.n;
-    h32[4] = kChunk;
-    h32[5] = uint32_t(L.nc);
-    h32[6] = kProbBits;  // u16 12, u16 0
-    h32[7] = 0;
-    h64[4] = L.off_raw;
-    h64[5] = L.off_exp;
-    if (it.n == 0) {
-      h64[6] = 0;
-      h64[7] = L.off_exp;
-      *reinterpret_cast<uint64_t *>(out + L.off_chunk_off) = 0;
-      *it.out_size = L.off_exp;
-    }
-  }
-  // zero padding: after the chunk-length table, and after each raw plane
-  if (tid < 16) {
-    uint64_t a = L.off_chunk_len + 4 * L.nc + tid;
-    if (a < L.off_raw) out[a] = 0;
-    if (dtype != WC_FP32) {
-      const uint64_t raw_bytes = is_fp8(dtype) ? (it.n + 1) / 2 : it.n;
-      uint64_t b = L.off_raw + raw_bytes + tid;
-      if (b < L.off_exp) out[b] = 0;
-    } else {
-      uint64_t b = L.off_raw + (it.n + 7) / 8 + tid;
-      if (b < L.off_mant) out[b] = 0;
-      uint64_t c = L.off_mant + 3 * it.n + tid;
-      if (c < L.off_exp) out[c] = 0;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------
-// k_hist: one block (512 threads) per tile of 4 chunks counts the tile's coded
-// bytes and adds them to the tensor's histogram; the tensor's last tile turns
-// the counts into the table.  The whole GPU reads the input at memory speed.
-//
-// k_encode: persistent coding.  Blocks take coding tasks (16 chunks of one
-// tensor, two per warp) in order from a counter, so every task that a task
-// waits for was taken earlier by a running block.  A warp that has coded its
-// chunks places them with a decoupled look-back over the tensor's per-chunk
-// words (stat): it publishes each chunk's padded length, reads its
-// predecessors' words (32 at a time) until one holds an inclusive prefix,
-// publishes its own inclusive prefix, writes the offset-table entries and
-// copies the payload from its window (or the raw exponent bytes from the
-// input) to the final place, zero-padded to 16 bytes.  The last chunk of a
-// tensor completes the header and the size.  A predecessor waits only for
-// its own coding, so the waits end; each is bounded all the same (kWaitNs),
-// and a tensor whose wait ran out gets size 0.
-
-constexpr int kHistThreads = 512;
-
-__shared__ uint32_t s_task;
-__shared__ uint32_t s_flag;
-
-// bytes [mis, mis + 16) of the 32 bytes a:b (mis even, 0..14)
-__device__ __forceinline__ uint4 extract16(uint4 a, uint4 b, uint32_t mis) {
-  const uint32_t sh = (mis & 3u) * 8u;
-  uint32_t r0, r1, r2, r3, r4;
-  switch (mis >> 2) {
-    case 0: r0 = a.x; r1 = a.y; r2 = a.z; r3 = a.w; r4 = b.x; break;
-    case 1: r0 = a.y; r1 = a.z; r2 = a.w; r3 = b.x; r4 = b.y; break;
-    case 2: r0 = a.z; r1 = a.w; r2 = b.x; r3 = b.y; r4 = b.z; break;
-    default: r0 = a.w; r1 = b.x; r2 = b.y; r3 = b.z; r4 = b.w; break;
-  }
-  return make_uint4(__funnelshift_r(r0, r1, sh), __funnelshift_r(r1, r2, sh),
-                    __funnelshift_r(r2, r3, sh), __funnelshift_r(r3, r4, sh));
-}
-
-__device__ __forceinline__ uint32_t keep_bytes(uint32_t v, int keep) {
-  if (keep >= 4) return v;
-  if (keep <= 0) return 0;
-  return v & ((1u << (8 * keep)) - 1u);
-}
-__device__ __forceinline__ uint4 keep16(uint4 o, int keep) {
-  if (keep >= 16) return o;
-  return make_uint4(keep_bytes(o.x, keep), keep_bytes(o.y, keep - 4), keep_bytes(o.z, keep - 8),
-                    keep_bytes(o.w, keep - 12));
-}
-
-// A coded chunk's payload: the 32 states (front of the window) and the w
-// words (the window's last 2w bytes, 2-byte aligned; realigned here).  Lane
-// l takes the 16-byte output granules l, l + 32, ..., kCopyUnroll at a time with
-// all their window loads issued before the first store, so that a warp keeps
-// many loads in flight.
-constexpr int kCopyUnroll = 2;
-
-__device__ __forceinline__ void copy_coded(const uint8_t *win, uint32_t len, uint8_t *dst, int lane) {
-  if (lane < int(kStateBytes / 16))
-    reinterpret_cast<uint4 *>(dst)[lane] = __ldcg(reinterpret_cast<const uint4 *>(win) + lane);
-  const uint32_t nbytes = len - kStateBytes;   // 2w
-  const uint32_t S = uint32_t(kWin) - nbytes;  // first word's byte offset in the window
-  const uint32_t mis = S & 15u;
-  const uint32_t A0 = S - mis;
-  const uint32_t ngran = (nbytes + 15) / 16;
-  const uint4 zero = make_uint4(0, 0, 0, 0);
-  constexpr int U = kCopyUnroll;
-  for (uint32_t j0 = 0; j0 < ngran; j0 += U * 32) {
-    uint4 a[U], b[U];
-#pragma unroll
-    for (int u = 0; u < U; u++) {
-      const uint32_t j = j0 + u * 32 + lane;
-      const uint32_t a_off = A0 + 16 * j;
-      a[u] = j < ngran ? __ldcg(reinterpret_cast<const uint4 *>(win + a_off)) : zero;
-      b[u] = j < ngran && a_off + 16 < uint32_t(kWin)
-                 ? __ldcg(reinterpret_cast<const uint4 *>(win + a_off + 16)) : zero;
-    }
-#pragma unroll
-    for (int u = 0; u < U; u++) {
-      const uint32_t j = j0 + u * 32 + lane;
-      if (j < ngran)
-        st_cs_v4(dst + kStateBytes + 16 * j, keep16(extract16(a[u], b[u], mis), int(nbytes) - int(16 * j)));
-    }
-  }
-}
-
-// A raw chunk: its nsym coded bytes, extracted again from the input.
-template <int DT>
-__device__ void copy_raw(const uint8_t *in, uint64_t k, uint32_t nsym, uint8_t *dst, int lane) {
-  const uint32_t ngran = uint32_t(round16(nsym) / 16);
-  for (uint32_t gi = lane; gi < ngran; gi += 32) {
-    const uint32_t v0 = gi * 16;
-    const int keep = int(nsym - v0);
-    uint4 e;
-    if (is_fp8(DT)) {
-      const uint8_t *src = in + k * kChunk;
-      if (keep >= 16) {
-        const uint4 a = ld_nc_v4(src + v0);
-        e = make_uint4(fp8_code4(a.x), fp8_code4(a.y), fp8_code4(a.z), fp8_code4(a.w));
-      } else {
-        uint32_t w[4] = {0u, 0u, 0u, 0u};
-        for (int q = 0; q < keep; q++) w[q / 4] |= fp8_code(src[v0 + q]) << (8 * (q % 4));
-        e = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    } else if (DT != WC_FP32) {
-      const uint16_t *src = reinterpret_cast<const uint16_t *>(in) + k * kChunk;
-      uint32_t w[8];
-      if (keep >= 16) {
-        const uint4 a = ld_nc_v4(src + v0), b = ld_nc_v4(src + v0 + 8);
-        w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w; w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; q++) {
-          const uint32_t lo = 2 * q < keep ? src[v0 + 2 * q] : 0u;
-          const uint32_t hi = 2 * q + 1 < keep ? src[v0 + 2 * q + 1] : 0u;
-          w[q] = lo | (hi << 16);
-        }
-      }
-      e = keep16(make_uint4(code4<DT>(w[0], w[1]), code4<DT>(w[2], w[3]), code4<DT>(w[4], w[5]),
-                            code4<DT>(w[6], w[7])), keep);
-    } else {
-      const uint32_t *src = reinterpret_cast<const uint32_t *>(in) + k * kChunk;
-      uint32_t u[16];
-#pragma unroll
-      for (int q = 0; q < 16; q++) u[q] = q < keep ? src[v0 + q] : 0u;
-      uint32_t ee[4];
-#pragma unroll
-      for (int q = 0; q < 4; q++) {
-        const uint32_t p01 = __byte_perm(u[4 * q] << 1, u[4 * q + 1] << 1, 0x0073);
-        const uint32_t p23 = __byte_perm(u[4 * q + 2] << 1, u[4 * q + 3] << 1, 0x0073);
-        ee[q] = __byte_perm(p01, p23, 0x5410);
-      }
-      e = keep16(make_uint4(ee[0], ee[1], ee[2], ee[3]), keep);
-    }
-    st_cs_v4(dst + v0, e);
-  }
-}
-
-// Exclusive prefix (padded bytes of chunks 0 .. k-1) of chunk k of a tensor
-// from the look-back words; false if a predecessor failed or the wait ran
-// out.  Lane l reads the word of chunk j - l; the words before chunk 0 count
-// as an inclusive prefix of 0.
-__device__ bool lookback(const uint64_t *stat, uint64_t k, uint64_t &excl, int lane) {
-  uint64_t sum = 0;
-  int64_t j = int64_t(k) - 1;
-  const uint64_t t0 = global_ns();
-  while (j >= 0) {
-    const int64_t idx = j - lane;
-    const uint64_t v = idx >= 0 ? ld_acquire_u64(stat + idx) : kStatInc;
-    const uint32_t fl = uint32_t(v >> 62);
-    const uint32_t bad = __ballot_sync(0xffffffffu, fl == 3u);
-    const uint32_t inc = __ballot_sync(0xffffffffu, fl == 2u);
-    const uint32_t stop = __ballot_sync(0xffffffffu, fl == 0u) | bad;
-    const int first_stop = stop ? __ffs(int(stop)) - 1 : 32;
-    const int first_inc = inc ? __ffs(int(inc)) - 1 : 32;
-    if (first_inc < first_stop) {
-      sum += warp_sum_u64(lane <= first_inc ? (v & kStatVal) : 0);
-      excl = sum;
-      return true;
-    }
-    if (first_stop < 32 && ((bad >> first_stop) & 1u)) return false;
-    sum += warp_sum_u64(lane < first_stop ? (v & kStatVal) : 0);
-    j -= first_stop;
-    if (first_stop == 0) {  // the nearest unread predecessor is still coding
-      if (global_ns() - t0 > kWaitNs) return false;
-      __nanosleep(512);     // leave the issue slots to the warps that code
-    }
-  }
-  excl = sum;
-  return true;
-}
-
-// What placing a warp's chunks needs of its tensor (passed by value to an
-// out-of-line function, so that the coding loops keep their registers).
-struct PlaceArgs {
-  uint64_t *stat;         // look-back words
-  const uint8_t *win0;    // window of chunk 0
-  const uint8_t *in;      // the tensor's values
-  uint8_t *out;           // the container
-  uint64_t *out_size;
-  uint64_t n, nc;
-  uint64_t off_chunk_off, off_chunk_len, off_exp;
-};
-
-// After the warp has coded chunks kA (and kA + 1 if hasB): place them.
-template <int DT>
-__device__ __noinline__ void place_chunks(const PlaceArgs a, uint64_t kA, bool hasB, uint32_t lenA,
-                                          uint32_t lenB) {
-  const int lane = threadIdx.x & 31;
-  const uint64_t padA = round16(lenA), padB = hasB ? round16(lenB) : 0;
-  if (lane == 0) {
-    st_release_u64(a.stat + kA, kStatAgg | padA);
-    if (hasB) st_release_u64(a.stat + kA + 1, kStatAgg | padB);
-  }
-  uint64_t excl = 0;
-  const bool ok = lookback(a.stat, kA, excl, lane);
-  if (!ok) {
-    if (lane == 0) {
-      st_release_u64(a.stat + kA, kStatBad);
-      if (hasB) st_release_u64(a.stat + kA + 1, kStatBad);
-      *a.out_size = 0;
-    }
-    return;
-  }
-  if (lane == 0) {
-    st_release_u64(a.stat + kA, kStatInc | (excl + padA));
-    if (hasB) st_release_u64(a.stat + kA + 1, kStatInc | (excl + padA + padB));
-  }
-  uint64_t *choff = reinterpret_cast<uint64_t *>(a.out + a.off_chunk_off);
-  uint32_t *chlen = reinterpret_cast<uint32_t *>(a.out + a.off_chunk_len);
-  for (int c = 0; c < (hasB ? 2 : 1); c++) {
-    const uint64_t k = kA + c;
-    const uint32_t len = c ? lenB : lenA;
-    const uint64_t off = excl + (c ? padA : 0);
-    const uint32_t nsym = chunk_nsym(a.n, k);
-    if (lane == 0) {
-      choff[k] = off;
-      chlen[k] = len;
-    }
-    uint8_t *dst = a.out + a.off_exp + off;
-    if (len == nsym) copy_raw<DT>(a.in, k, nsym, dst, lane);
-    else copy_coded(a.win0 + k * kWin, len, dst, lane);
-    if (k + 1 == a.nc && lane == 0) {
-      const uint64_t exp_bytes = off + round16(len);
-      choff[a.nc] = exp_bytes;
-      uint64_t *h64 = reinterpret_cast<uint64_t *>(a.out);
-      h64[6] = exp_bytes;
-      h64[7] = a.off_exp + exp_bytes;
-      *a.out_size = a.off_exp + exp_bytes;
-    }
-  }
-}
-
-template <int DT, bool W>
-__device__ __forceinline__ void code_and_place(const EncItem &it, const Layout &L, uint64_t kA, bool hasB,
-                                               int warp, int lane) {
-  CoderOut co{s_len[warp], kA, it.scratch + scratch_win_offset(L.nc)};
-  code_warp<DT, W>(it, L, kA, hasB, warp, co);
-  __syncwarp();
-  const uint32_t lenA = s_len[warp][0], lenB = hasB ? s_len[warp][1] : 0u;
-  PlaceArgs a;
-  a.stat = reinterpret_cast<uint64_t *>(it.scratch + kScrStat);
-  a.win0 = co.win0;
-  a.in = it.in;
-  a.out = it.out;
-  a.out_size = it.out_size;
-  a.n = it.n;
-  a.nc = L.nc;
-  a.off_chunk_off = L.off_chunk_off;
-  a.off_chunk_len = L.off_chunk_len;
-  a.off_exp = L.off_exp;
-  place_chunks<DT>(a, kA, hasB, lenA, lenB);
-}
-
-__global__ void __launch_bounds__(kHistThreads, 2) k_hist(const __grid_constant__ EncParams p) {
-  __shared__ __align__(16) uint32_t sh[256 * 32];  // [symbol][lane]
-  __shared__ uint64_t red[kHistThreads / 32 + 1];
-  __shared__ int s_last;
-  const int tid = threadIdx.x;
-  const uint32_t b = blockIdx.x;
-  uint32_t lo = 0, hi = p.ntseg - 1;  // last segment starting at or before b
-  while (lo < hi) {
-    const uint32_t mid = (lo + hi + 1) >> 1;
-    if (p.tseg_start[mid] <= b) lo = mid; else hi = mid - 1;
-  }
-  const EncItem &it = p.items[p.tseg_item[lo]];
-  const uint64_t tile = b - p.tseg_start[lo];
-  for (int i = tid; i < 256 * 32 / 4; i += kHistThreads)
-    reinterpret_cast<uint4 *>(sh)[i] = make_uint4(0, 0, 0, 0);
-  __syncthreads();
-  count_tile<kHistThreads>(it, tile, sh);
-  __syncthreads();
-  uint64_t *ghist = reinterpret_cast<uint64_t *>(it.scratch + kScrHist);
-  if (tid < 256) {
-    uint32_t sum = 0;
-#pragma unroll 8
-    for (int j = 0; j < 32; j++) sum += sh[(tid << 5) | ((j + tid) & 31)];
-    if (sum) atomicAdd(reinterpret_cast<unsigned long long *>(&ghist[tid]),
-                       static_cast<unsigned long long>(sum));
-    __threadfence();
-  }
-  __syncthreads();
-  if (tid == 0) {
-    uint32_t *ctr = reinterpret_cast<uint32_t *>(it.scratch + kScrCtr);
-    const uint64_t nc = num_chunks(it.n);
-    const uint32_t nt = uint32_t((nc + kHistChunks - 1) / kHistChunks);
-    s_last = (atomicAdd(&ctr[0], 1u) == nt - 1);
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  publish_table<kHistThreads>(it, red);
-}
-
-// Coding task: chunks [16 j, 16 j + 16) of item `it` (by value: the coding
-// loops get the registers the task loop does not need).
-__device__ __noinline__ void code_task(const EncItem it, uint64_t j) {
+__global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constant__ EncParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t b = blockIdx.x;
+  const EncItem &it = p.items[find_item_by_block(p, b)];
   const int dtype = int(it.dtype);
   const Layout L = make_layout(it.n, dtype);
-  if (tid == 0) {
-    const uint32_t *ready = reinterpret_cast<const uint32_t *>(it.scratch + kScrCtr) + 2;
-    const uint64_t t0 = global_ns();
-    uint32_t r = ld_acquire_u32(ready);
-    while (r == 0 && global_ns() - t0 <= kWaitNs) {
-      __nanosleep(256);
-      r = ld_acquire_u32(ready);
-    }
-    s_flag = r;
-  }
+
+  s_tab[tid] = reinterpret_cast<const uint4 *>(it.scratch + kScrTab)[tid];
+  s_bias[tid] = reinterpret_cast<const uint32_t *>(it.scratch + kScrBias)[tid];
   __syncthreads();
-  const uint32_t ready = s_flag;
-  const uint64_t kA = j * kCoderChunks + 2 * warp;
-  if (ready == 0) {  // no table (cannot happen after k_hist): the tensor fails
-    if (kA < L.nc && lane == 0) {
-      uint64_t *stat = reinterpret_cast<uint64_t *>(it.scratch + kScrStat);
-      st_release_u64(stat + kA, kStatBad);
-      if (kA + 1 < L.nc) st_release_u64(stat + kA + 1, kStatBad);
-      *it.out_size = 0;
-    }
-    return;
-  }
-  s_tab[tid] = __ldcg(reinterpret_cast<const uint4 *>(it.scratch + kScrTab) + tid);
-  s_bias[tid] = __ldcg(reinterpret_cast<const uint32_t *>(it.scratch + kScrBias) + tid);
-  __syncthreads();
+
+  const uint64_t kA = uint64_t(b - it.block_base) * kCoderChunks + 2 * warp;
   if (kA >= L.nc) return;
   const bool hasB = kA + 1 < L.nc;
-  const bool wide = ready == 2;
+  CoderOut co{reinterpret_cast<uint32_t *>(it.scratch + kScrLen), it.scratch + scratch_win_offset(L.nc)};
+  const bool wide = reinterpret_cast<const uint32_t *>(it.scratch + kScrCtr)[2] == 2;
   if (dtype == WC_BF16) {
-    if (wide) code_and_place<WC_BF16, true>(it, L, kA, hasB, warp, lane);
-    else code_and_place<WC_BF16, false>(it, L, kA, hasB, warp, lane);
+    if (wide) code_warp<WC_BF16, true>(it, L, kA, hasB, warp, co);
+    else code_warp<WC_BF16, false>(it, L, kA, hasB, warp, co);
   } else if (dtype == WC_FP16) {
-    if (wide) code_and_place<WC_FP16, true>(it, L, kA, hasB, warp, lane);
-    else code_and_place<WC_FP16, false>(it, L, kA, hasB, warp, lane);
+    if (wide) code_warp<WC_FP16, true>(it, L, kA, hasB, warp, co);
+    else code_warp<WC_FP16, false>(it, L, kA, hasB, warp, co);
   } else if (dtype == WC_FP8E4M3) {
-    if (wide) code_and_place<WC_FP8E4M3, true>(it, L, kA, hasB, warp, lane);
-    else code_and_place<WC_FP8E4M3, false>(it, L, kA, hasB, warp, lane);
+    if (wide) code_warp<WC_FP8E4M3, true>(it, L, kA, hasB, warp, co);
+    else code_warp<WC_FP8E4M3, false>(it, L, kA, hasB, warp, co);
   } else if (dtype == WC_FP8E5M2) {
-    if (wide) code_and_place<WC_FP8E5M2, true>(it, L, kA, hasB, warp, lane);
-    else code_and_place<WC_FP8E5M2, false>(it, L, kA, hasB, warp, lane);
+    if (wide) code_warp<WC_FP8E5M2, true>(it, L, kA, hasB, warp, co);
+    else code_warp<WC_FP8E5M2, false>(it, L, kA, hasB, warp, co);
   } else if (wide) {
-    code_and_place<WC_FP32, true>(it, L, kA, hasB, warp, lane);
+    code_warp<WC_FP32, true>(it, L, kA, hasB, warp, co);
   } else {
-    code_and_place<WC_FP32, false>(it, L, kA, hasB, warp, lane);
+    code_warp<WC_FP32, false>(it, L, kA, hasB, warp, co);
   }
-}
 
-__global__ void __launch_bounds__(kCoderThreads, 4) k_encode(const __grid_constant__ EncParams p) {
-  const int tid = threadIdx.x;
-  uint32_t *ticket = reinterpret_cast<uint32_t *>(p.items[0].scratch + kScrCtr) + 3;
-  for (;;) {
-    if (tid == 0) s_task = atomicAdd(ticket, 1u);
-    __syncthreads();
-    const uint32_t t = s_task;
-    if (t >= p.total_tasks) return;
-    uint32_t lo = 0, hi = p.ncseg - 1;  // last segment starting at or before t
-    while (lo < hi) {
-      const uint32_t mid = (lo + hi + 1) >> 1;
-      if (p.cseg_start[mid] <= t) lo = mid; else hi = mid - 1;
+  // last warp of the tensor: offset table and the rest of the header
+  const uint32_t done = hasB ? 2u : 1u;
+  __threadfence();
+  uint32_t prev = 0;
+  if (lane == 0) prev = atomicAdd(reinterpret_cast<uint32_t *>(it.scratch + kScrCtr) + 1, done);
+  prev = __shfl_sync(0xffffffffu, prev, 0);
+  if (prev + done != uint32_t(L.nc)) return;
+  __threadfence();
+  const uint32_t *lens = co.lens;
+  uint64_t *choff = reinterpret_cast<uint64_t *>(it.out + L.off_chunk_off);
+  uint32_t *chlen = reinterpret_cast<uint32_t *>(it.out + L.off_chunk_len);
+  uint64_t run = 0;
+  for (uint64_t base = 0; base < L.nc; base += 32) {
+    const uint64_t j = base + lane;
+    const uint32_t ln = j < L.nc ? __ldcg(&lens[j]) : 0u;
+    const uint64_t pd = round16(ln);
+    const uint64_t incl = warp_incl_scan_u64(pd);
+    if (j < L.nc) {
+      choff[j] = run + incl - pd;
+      chlen[j] = ln;
     }
-    code_task(p.items[p.cseg_item[lo]], t - p.cseg_start[lo]);
-    __syncthreads();  // the block is done with this task's shared memory
+    run += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  if (lane == 0) {
+    choff[L.nc] = run;
+    uint64_t *h64 = reinterpret_cast<uint64_t *>(it.out);
+    h64[6] = run;
+    h64[7] = L.off_exp + run;
+    *it.out_size = L.off_exp + run;
   }
 }
 
-int encode_blocks_per_sm() {
-  int nb = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, k_encode, kCoderThreads, 0) != cudaSuccess)
-    return 0;
-  return nb;
-}
-
-cudaError_t launch_prep(const EncParams &p, cudaStream_t s) {
-  k_prep<<<p.count, 256, 0, s>>>(p);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_hist(const EncParams &p, cudaStream_t s) {
-  if (p.total_tiles == 0) return cudaSuccess;
-  k_hist<<<p.total_tiles, kHistThreads, 0, s>>>(p);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_encode(const EncParams &p, int grid, cudaStream_t s) {
-  if (p.total_tasks == 0) return cudaSuccess;
-  const int g = int(p.total_tasks) < grid ? int(p.total_tasks) : grid;
-  k_encode<<<g, kCoderThreads, 0, s>>>(p);
+cudaError_t launch_coder(const EncParams &p, cudaStream_t s) {
+  if (p.total_coder_blocks == 0) return cudaSuccess;
+  k_coder<<<p.total_coder_blocks, kCoderThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

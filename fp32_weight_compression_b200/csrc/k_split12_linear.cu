@@ -41,7 +41,7 @@ namespace wc12l {
 
 using wc12::kChunk;
 
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;  // 8 warps: all expand; warps 0-3 (TMEM lanes) and 4-7 split the epilogue
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr uint32_t kASlice = kBM * 16 * 2;   // bytes of one K = 16 slice of A
@@ -52,7 +52,7 @@ constexpr uint32_t kSpinLimit = 1u << 24;
 // shared-memory list of up to kExcCap entries {column in the CTA's K range,
 // row | high byte << 16 | low byte << 24}; a CTA with more walks its chunks'
 // exception lists at every stage instead.
-constexpr uint32_t kExcCap = 1024;
+constexpr uint32_t kExcCap = 512;
 
 struct Params {
   const uint8_t *w;
@@ -76,8 +76,10 @@ constexpr uint32_t kLoBytes = kBM * kBK;       // 8 KiB
 
 __host__ __device__ inline uint32_t b_stage_bytes(uint32_t n_mma) { return n_mma * kBK * 2; }
 __host__ __device__ inline uint32_t slot_bytes(uint32_t n_mma) { return kIdxBytes + kLoBytes + b_stage_bytes(n_mma); }
+// per-stage exception bins: a count (then start) per stage of the CTA
+constexpr uint32_t kMaxStagesPerCta = 256;
 __host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma) {
-  return 1024 + 2 * kAStage + kDepth * slot_bytes(n_mma) + 64 + 8 * kExcCap;
+  return 1024 + 2 * kAStage + kDepth * slot_bytes(n_mma) + 64 + 2 * 8 * kExcCap + 2 * 4 * (kMaxStagesPerCta + 1);
 }
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
@@ -166,7 +168,10 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + kDepth);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
   uint32_t *exc_n = tmem_slot + 2;
-  uint2 *exc_list = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(bar) + 64);
+  uint2 *exc_raw = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(bar) + 64);  // gathered
+  uint2 *exc_bin = exc_raw + kExcCap;                                                  // by stage
+  uint32_t *bin = reinterpret_cast<uint32_t *>(exc_bin + kExcCap);                     // per stage
+  uint32_t *cur = bin + kMaxStagesPerCta + 1;                                          // scatter cursors
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const uint32_t K = p.K, N = p.N;
@@ -201,32 +206,43 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(w + wc12::kExcOffOff);
   const uint16_t *exc_pos = reinterpret_cast<const uint16_t *>(w + L.off_exc);
   const uint8_t *exc_val = w + L.off_excval;
-  const uint8_t *idx_plane = w + L.off_idx;
   const uint8_t *lo_plane = w + L.off_lo;
   const uint64_t c_lo = uint64_t(n0) * K / kChunk, c_hi = (uint64_t(n0 + kBM) * K - 1) / kChunk;
 
-  // the loads of stage j (of this CTA) into ring slot j % kDepth: the rows'
-  // index and low bytes as stored, and the tokens' X slice straight into the
-  // B operand layout (one 16-byte core-matrix row per copy; tokens >= M are
-  // zero-filled)
+  // This thread's copies of every stage, with their sources at stage 0 of
+  // the CTA (a stage adds 32 bytes to an index-plane source, 64 to a
+  // low-plane source, 128 to an X source): three of the 768 copies of the
+  // rows' index and low bytes, and n_mma / 32 of the X slice's (tokens >= M
+  // are zero-filled).
   const uint32_t ring_s = smem_u32(ring);
+  const uint32_t k_first = s_begin * kBK;
+  const uint8_t *a_src[3];
+  uint32_t a_dst[3];
+#pragma unroll
+  for (int r = 0; r < 3; r++) {
+    const uint32_t i = uint32_t(tid) + kThreads * r;
+    if (i < 2 * kBM) {
+      const uint32_t row = i >> 1, part = i & 1;
+      a_src[r] = w + L.off_idx + (uint64_t(n0 + row) * K + k_first) / 2 + 16 * part;
+      a_dst[r] = row * 32 + 16 * part;
+    } else {
+      const uint32_t j2 = i - 2 * kBM, row = j2 >> 2, part = j2 & 3;
+      a_src[r] = lo_plane + uint64_t(n0 + row) * K + k_first + 16 * part;
+      a_dst[r] = kIdxBytes + row * 64 + 16 * part;
+    }
+  }
+  const uint32_t nb = p.n_mma * 8;  // X copies per stage
   auto issue_loads = [&](uint32_t j) {
     const uint32_t slot = ring_s + (j % kDepth) * sb;
-    const uint32_t k0 = (s_begin + j) * kBK;
-    const uint32_t total = 3 * kBM * 2 + p.n_mma * 8;  // 256 index + 512 low + B copies
-    for (uint32_t i = tid; i < total; i += kThreads) {
-      if (i < 2 * kBM) {
-        const uint32_t row = i >> 1, part = i & 1;
-        cp_async16(slot + row * 32 + 16 * part, idx_plane + (uint64_t(n0 + row) * K + k0) / 2 + 16 * part, 16);
-      } else if (i < 6 * kBM) {
-        const uint32_t j2 = i - 2 * kBM, row = j2 >> 2, part = j2 & 3;
-        cp_async16(slot + kIdxBytes + row * 64 + 16 * part, lo_plane + uint64_t(n0 + row) * K + k0 + 16 * part, 16);
-      } else {
-        const uint32_t j3 = i - 6 * kBM, t = j3 >> 3, jj = j3 & 7;
-        const bool real = t < p.M;
-        cp_async16(slot + kIdxBytes + kLoBytes + op_offset(t, 8 * jj, p.n_mma * 32),
-                   real ? static_cast<const void *>(p.x + uint64_t(t) * K + k0 + 8 * jj) : p.x, real ? 16 : 0);
-      }
+    const uint32_t kofs = j * kBK;  // values past the CTA's first stage
+#pragma unroll
+    for (int r = 0; r < 3; r++) cp_async16(slot + a_dst[r], a_src[r] + (r == 0 && tid < 2 * kBM ? kofs / 2 : kofs), 16);
+    for (uint32_t j3 = tid; j3 < nb; j3 += kThreads) {
+      const uint32_t t = j3 >> 3, jj = j3 & 7;
+      const bool real = t < p.M;
+      cp_async16(slot + kIdxBytes + kLoBytes + op_offset(t, 8 * jj, p.n_mma * 32),
+                 real ? static_cast<const void *>(p.x + uint64_t(t) * K + k_first + kofs + 8 * jj) : p.x,
+                 real ? 16 : 0);
     }
   };
 
@@ -245,6 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     *exc_n = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
+  for (uint32_t i = tid; i <= nst && i <= kMaxStagesPerCta; i += kThreads) bin[i] = 0;
   // the first kDepth - 1 stages' loads are in flight while the exceptions
   // are gathered
   for (uint32_t j = 0; j + 1 < kDepth; j++) {
@@ -258,9 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   const uint32_t idesc = instr_desc(p.n_mma);
 
   // The CTA's exceptions, once: positions within a chunk become (row, column)
-  // relative to the CTA's tile with 32-bit arithmetic when 128 K fits it.
+  // relative to the CTA's tile with 32-bit arithmetic when 128 K fits it,
+  // counted per stage, then binned by stage so that each stage's are found
+  // without a search and patched by the thread that expanded their segment.
   const uint64_t f_base = uint64_t(n0) * K, f_span = uint64_t(kBM) * K;
   const uint32_t k_beg = s_begin * kBK, k_end = s_end * kBK;
+  const bool binned = nst <= kMaxStagesPerCta;
   for (uint64_t c = c_lo; c <= c_hi; c++) {
     const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
     if (e0 > e1 || e1 > ne) {
@@ -287,14 +307,42 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
       }
       if (col < k_beg || col >= k_end) continue;
       const uint32_t slot = atomicAdd(exc_n, 1u);
-      if (slot < kExcCap)
-        exc_list[slot] = make_uint2(col - k_beg, row | (uint32_t(exc_val[e]) << 16) |
-                                                     (uint32_t(lo_plane[f]) << 24));
+      if (slot < kExcCap) {
+        exc_raw[slot] = make_uint2(col - k_beg, row | (uint32_t(exc_val[e]) << 16) |
+                                                    (uint32_t(lo_plane[f]) << 24));
+        if (binned) atomicAdd(&bin[(col - k_beg) / kBK], 1u);
+      }
     }
   }
   __syncthreads();
   const uint32_t n_exc = *exc_n;
-  const bool exc_walk = n_exc > kExcCap;
+  const bool exc_walk = n_exc > kExcCap || !binned;
+  if (!exc_walk) {
+    // counts -> starts (one warp), then scatter by stage
+    if (warp == 0) {
+      uint32_t run = 0;
+      for (uint32_t b0 = 0; b0 <= nst; b0 += 32) {
+        const uint32_t b = b0 + lane;
+        const uint32_t v = b < nst ? bin[b] : 0u;
+        uint32_t incl = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += u;
+        }
+        if (b <= nst) bin[b] = run + incl - v;
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
+    }
+    __syncthreads();
+    for (uint32_t i = tid; i <= nst; i += kThreads) cur[i] = bin[i];
+    __syncthreads();
+    for (uint32_t i = tid; i < n_exc; i += kThreads) {
+      const uint2 ex = exc_raw[i];
+      exc_bin[atomicAdd(&cur[ex.x / kBK], 1u)] = ex;
+    }
+    __syncthreads();
+  }
 
   uint32_t it = 0;
   for (; it < nst; it++) {
@@ -305,10 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     cp_async_wait<kDepth - 2>();  // this stage's loads (later stages may still be in flight)
     __syncthreads();
 
-    // A: 512 segments of 16 values (row = i / 4, values 16 (i % 4) ..), four
+    // A: 512 segments of 16 values (row = i / 4, values 16 (i % 4) ..), two
     // per thread, expanded from the ring slot into the operand slot
 #pragma unroll
-    for (int q = 0; q < 4; q++) {
+    for (int q = 0; q < 2; q++) {
       const uint32_t i = uint32_t(tid) + kThreads * q, row = i >> 2, seg = i & 3;
       const uint2 iw = *reinterpret_cast<const uint2 *>(slot + row * 32 + 8 * seg);
       const uint4 lw = *reinterpret_cast<const uint4 *>(slot + kIdxBytes + row * 64 + 16 * seg);
@@ -317,17 +365,19 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
       *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg, kASlice)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
       *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg + 8, kASlice)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
     }
-    __syncthreads();
     // exceptions that fall in this tile
     if (!exc_walk) {
-      const uint32_t c0 = k0 - k_beg;
-      for (uint32_t i = tid; i < n_exc; i += kThreads) {
-        const uint2 ex = exc_list[i];
-        if (ex.x - c0 >= uint32_t(kBK)) continue;
-        *reinterpret_cast<uint16_t *>(A + op_offset(ex.y & 0xFFFFu, ex.x - c0, kASlice)) =
+      // each is patched by the thread that expanded its segment (program
+      // order after that thread's stores: no barrier needed)
+      for (uint32_t i = bin[it]; i < bin[it + 1]; i++) {
+        const uint2 ex = exc_bin[i];
+        const uint32_t row = ex.y & 0xFFFFu, col = ex.x - it * kBK;
+        if ((row * 4 + (col >> 4)) % kThreads != uint32_t(tid)) continue;
+        *reinterpret_cast<uint16_t *>(A + op_offset(row, col, kASlice)) =
             uint16_t(((ex.y >> 16) & 0xFFu) << 8 | (ex.y >> 24));
       }
     } else {
+      __syncthreads();  // every segment expanded before any thread patches
       for (uint64_t c = c_lo; c <= c_hi; c++) {
         const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
         if (e0 > e1 || e1 > ne) continue;  // reported by the gathering pass
@@ -353,20 +403,21 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
         mma_bf16(tmem, operand_desc(a0 + sl * kASlice), operand_desc(b0 + sl * p.n_mma * 32), idesc,
                  (it > 0 || sl > 0) ? 1u : 0u);
       mma_commit(&bar[it % kDepth]);
+      // the slot of stage it - 1 is free once its MMAs are done (which also
+      // frees the A slot stage it + 1 writes); one thread waits, the rest
+      // wait at the barrier below
+      if (it >= 1) {
+        const uint32_t prev = it - 1;
+        if (!mbar_wait(&bar[prev % kDepth], (prev / kDepth) & 1u)) {
+          report(p.status, WC_ERR_TIMEOUT);
+          *flag = 1;
+        }
+      }
     }
-    // the slot of stage it - 1 is free once its MMAs are done (which also
-    // frees the A slot stage it + 1 writes): load stage it + kDepth - 1 there
-    if (it >= 1) {
-      const uint32_t prev = it - 1;
-      if (!mbar_wait(&bar[prev % kDepth], (prev / kDepth) & 1u)) {
-        if (tid == 0) report(p.status, WC_ERR_TIMEOUT);
-        *flag = 1;
-      }
-      __syncthreads();
-      if (*flag) {
-        it++;  // stage it was issued
-        break;
-      }
+    __syncthreads();
+    if (*flag) {
+      it++;  // stage it was issued
+      break;
     }
     if (it + kDepth - 1 < nst) issue_loads(it + kDepth - 1);
     cp_async_commit();
@@ -376,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   // wait for the last stage issued (its commit covers all earlier MMAs)
   const uint32_t issued = it;
   bool done = true;
-  if (issued > 0) {
+  if (issued > 0 && tid == 0) {
     const uint32_t last = issued - 1;
     done = mbar_wait(&bar[last % kDepth], (last / kDepth) & 1u);
   }
@@ -386,13 +437,16 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   if (!done && tid == 0) report(p.status, WC_ERR_TIMEOUT);
   fence_after_sync();
   if (done && !*flag && issued > 0) {
-    const uint32_t row = n0 + 32 * warp + lane;
-    for (uint32_t c0 = 0; c0 < p.n_mma; c0 += 8) {
+    // warp w reads TMEM lanes 32 (w % 4) .. (its rows); warps 0-3 take the
+    // even 8-column groups, warps 4-7 the odd ones
+    const uint32_t lane_base = 32 * (warp & 3);
+    const uint32_t row = n0 + lane_base + lane;
+    for (uint32_t c0 = 8 * (warp >> 2); c0 < p.n_mma; c0 += 16) {
       uint32_t v[8];
       asm volatile(
           "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
           : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
-          : "r"(tmem + (uint32_t(32 * warp) << 16) + c0));
+          : "r"(tmem + (lane_base << 16) + c0));
       asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
       for (int i = 0; i < 8; i++) {
@@ -458,7 +512,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k12_gemv(const __grid_constan
   const uint64_t r0 = uint64_t(row) * K;
 
   // exception cursor: chunk c, list index e = the first exception at or
-  // after value r0 (a search in chunk c's sorted positions)
+  // after value r0 (a search in chunk c's sorted positions); next_pos is its
+  // position among all values (~0 when the list is done), kept in a register
+  // so that a step reads the list only when an exception falls in it
   uint64_t c = r0 / kChunk;
   uint64_t c_end = exc_off[c + 1];
   uint64_t e;
@@ -475,18 +531,46 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k12_gemv(const __grid_constan
     }
     e = lo;
   }
+  bool bad = false;
+  auto locate = [&]() -> uint64_t {  // position of exception e (warp-uniform)
+    while (e >= c_end && c + 1 < L.nc) {  // on to the next chunk's list
+      c++;
+      const uint64_t nxt = exc_off[c + 1];
+      if (exc_off[c] != c_end || nxt < c_end || nxt > ne) {
+        bad = true;
+        return ~uint64_t(0);
+      }
+      c_end = nxt;
+    }
+    if (e >= c_end) return ~uint64_t(0);
+    const uint32_t cpos = exc_pos[e];
+    const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
+    if (cpos >= cnt) {
+      bad = true;
+      return ~uint64_t(0);
+    }
+    return c * kChunk + cpos;
+  };
+  uint64_t next_pos = locate();
 
   float acc[MT];
 #pragma unroll
   for (int m = 0; m < MT; m++) acc[m] = 0.0f;
+  // the planes of the next step are loaded while this one is worked on
+  uint2 iw_n = make_uint2(0, 0);
+  uint4 lw_n = make_uint4(0, 0, 0, 0);
+  if (uint32_t(16 * lane) < K) {
+    iw_n = __ldg(reinterpret_cast<const uint2 *>(idx_plane + (r0 + 16 * lane) / 2));
+    lw_n = __ldg(reinterpret_cast<const uint4 *>(lo_plane + r0 + 16 * lane));
+  }
   for (uint32_t k0 = 0; k0 < K; k0 += 512) {
     const uint32_t col = k0 + 16 * lane;
     const bool act = col < K;  // K is a multiple of 64: a lane holds 16 values or none
-    uint2 iw = make_uint2(0, 0);
-    uint4 lw = make_uint4(0, 0, 0, 0);
-    if (act) {
-      iw = __ldg(reinterpret_cast<const uint2 *>(idx_plane + (r0 + col) / 2));
-      lw = __ldg(reinterpret_cast<const uint4 *>(lo_plane + r0 + col));
+    const uint2 iw = iw_n;
+    const uint4 lw = lw_n;
+    if (col + 512 < K) {
+      iw_n = __ldg(reinterpret_cast<const uint2 *>(idx_plane + (r0 + col + 512) / 2));
+      lw_n = __ldg(reinterpret_cast<const uint4 *>(lo_plane + r0 + col + 512));
     }
     uint32_t v[8];
     {
@@ -496,27 +580,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k12_gemv(const __grid_constan
     }
     // the exceptions among values [r0 + k0, r0 + min(k0 + 512, K))
     const uint64_t s0 = r0 + k0, s1 = r0 + (k0 + 512 < K ? k0 + 512 : K);
-    for (;;) {
-      while (e >= c_end && c + 1 < L.nc) {  // on to the next chunk's list
-        c++;
-        const uint64_t nxt = exc_off[c + 1];
-        if (exc_off[c] != c_end || nxt < c_end || nxt > ne) {
-          if (lane == 0) report(p.status, WC_ERR_CORRUPT);
-          return;
-        }
-        c_end = nxt;
-      }
-      if (e >= c_end) break;
-      const uint32_t cpos = exc_pos[e];
-      const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
-      if (cpos >= cnt) {
-        if (lane == 0) report(p.status, WC_ERR_CORRUPT);
-        return;
-      }
-      const uint64_t pos = c * kChunk + cpos;
-      if (pos >= s1) break;
-      if (pos >= s0) {
-        const uint32_t rel = uint32_t(pos - s0);
+    while (next_pos < s1) {
+      if (next_pos >= s0) {
+        const uint32_t rel = uint32_t(next_pos - s0);
         if (lane == int(rel >> 4)) {
           const uint32_t j = rel & 15u;
           const uint32_t lo = (j < 4 ? lw.x : j < 8 ? lw.y : j < 12 ? lw.z : lw.w) >> (8 * (j & 3)) & 0xFFu;
@@ -527,6 +593,11 @@ __global__ void __launch_bounds__(kGemvWarps * 32) k12_gemv(const __grid_constan
         }
       }
       e++;
+      next_pos = locate();
+    }
+    if (bad) {
+      if (lane == 0) report(p.status, WC_ERR_CORRUPT);
+      return;
     }
     if (act) {
 #pragma unroll

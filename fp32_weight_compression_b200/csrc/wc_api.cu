@@ -2,11 +2,10 @@
 // into launches, and the kernel launch sequence.
 //
 // Encode, per launch of up to kMaxItems tensors (all on `stream`):
-//   k_prep     header fields, padding, scratch counters    (1 block / tensor)
+//   k_prep     header fields + scratch counters            (1 block / tensor)
 //   k_hist     coded-byte histogram -> 12-bit table        (1 block / 4 chunks)
-//   k_encode   persistent: raw planes + rANS per chunk + placement of the
-//              payloads through a look-back over the chunk sizes (a task
-//              per 16 chunks, one warp per 2 chunks)
+//   k_coder    raw planes + rANS per chunk + offset scan   (1 warp / 2 chunks)
+//   k_compact  payloads into the exponent section          (1 block / chunk)
 // Decode, per launch of up to kMaxItems containers:
 //   k_decode   persistent grid, one warp per 2 chunks
 // Block checksums (wc_crc32_blocks):
@@ -46,7 +45,6 @@ bool dtype_ok(int32_t dt) {
 struct DeviceInfo {
   int sms = 0;
   int dec_blocks_per_sm = 0;
-  int enc_blocks_per_sm = 0;
   int crc_blocks_per_sm = 0;
   cudaError_t crc_err = cudaSuccess;
 };
@@ -73,12 +71,7 @@ DeviceInfo device_info(int32_t *err) {
       *err = cuda_fail(cudaGetLastError(), "decoder set-up");
       return DeviceInfo{};
     }
-    const int eb = wc::encode_blocks_per_sm();
-    if (eb <= 0) {
-      *err = cuda_fail(cudaGetLastError(), "encoder set-up");
-      return DeviceInfo{};
-    }
-    cache[dev].enc_blocks_per_sm = eb;
+
     // the checksum kernel's set-up failing leaves the codec usable
     cache[dev].crc_blocks_per_sm = wc::crc_blocks_per_sm();
     if (cache[dev].crc_blocks_per_sm <= 0) cache[dev].crc_err = cudaGetLastError();
@@ -158,15 +151,12 @@ int32_t wc_encode_batch(const wc_encode_item *items, uint32_t count, void *strea
     if (it.scratch_cap < wc_scratch_bytes(it.n, it.dtype)) return WC_ERR_CAPACITY;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  int32_t err = WC_OK;
-  const DeviceInfo info = device_info(&err);
-  if (err != WC_OK) return err;
-  static thread_local wc::EncParams P;  // ~16 KiB: kept off the stack
+  static thread_local wc::EncParams P;  // ~14 KiB: kept off the stack
   for (uint32_t b0 = 0; b0 < count; b0 += wc::kMaxItems) {
     const uint32_t cnt = count - b0 < wc::kMaxItems ? count - b0 : wc::kMaxItems;
     memset(&P, 0, sizeof(P));
     P.count = cnt;
-    uint64_t tiles[wc::kMaxItems], coding[wc::kMaxItems];
+    uint64_t chunks = 0, blocks = 0, hblocks = 0;
     for (uint32_t i = 0; i < cnt; i++) {
       const wc_encode_item &src = items[b0 + i];
       wc::EncItem &d = P.items[i];
@@ -176,32 +166,23 @@ int32_t wc_encode_batch(const wc_encode_item *items, uint32_t count, void *strea
       d.out_size = src.out_size;
       d.n = src.n;
       d.dtype = uint32_t(src.dtype);
+      d.chunk_base = uint32_t(chunks);
+      d.block_base = uint32_t(blocks);
+      d.hist_base = uint32_t(hblocks);
       const uint64_t nc = wc::num_chunks(src.n);
-      tiles[i] = (nc + wc::kHistChunks - 1) / wc::kHistChunks;
-      coding[i] = (nc + wc::kCoderChunks - 1) / wc::kCoderChunks;
+      chunks += nc;
+      blocks += (nc + wc::kCoderChunks - 1) / wc::kCoderChunks;
+      hblocks += (nc + wc::kHistChunks - 1) / wc::kHistChunks;
+      if (chunks >= (uint64_t(1) << 31)) return WC_ERR_UNSUPPORTED;
     }
-    // the tiles and the coding tasks of each tensor, in item order
-    uint64_t tpos = 0, cpos = 0;
-    for (uint32_t i = 0; i < cnt; i++) {
-      if (tiles[i]) {
-        P.tseg_start[P.ntseg] = uint32_t(tpos);
-        P.tseg_item[P.ntseg++] = i;
-        tpos += tiles[i];
-      }
-      if (coding[i]) {
-        P.cseg_start[P.ncseg] = uint32_t(cpos);
-        P.cseg_item[P.ncseg++] = i;
-        cpos += coding[i];
-      }
-    }
-    if (tpos >= (uint64_t(1) << 31)) return WC_ERR_UNSUPPORTED;
-    P.total_tiles = uint32_t(tpos);
-    P.total_tasks = uint32_t(cpos);
+    P.total_chunks = uint32_t(chunks);
+    P.total_coder_blocks = uint32_t(blocks);
+    P.total_hist_blocks = uint32_t(hblocks);
     cudaError_t e;
     if ((e = wc::launch_prep(P, s)) != cudaSuccess) return cuda_fail(e, "k_prep");
     if ((e = wc::launch_hist(P, s)) != cudaSuccess) return cuda_fail(e, "k_hist");
-    if ((e = wc::launch_encode(P, info.sms * info.enc_blocks_per_sm, s)) != cudaSuccess)
-      return cuda_fail(e, "k_encode");
+    if ((e = wc::launch_coder(P, s)) != cudaSuccess) return cuda_fail(e, "k_coder");
+    if ((e = wc::launch_compact(P, s)) != cudaSuccess) return cuda_fail(e, "k_compact");
   }
   return WC_OK;
 }

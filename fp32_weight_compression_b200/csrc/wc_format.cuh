@@ -30,29 +30,22 @@ constexpr uint32_t kGroupValues = 512;
 constexpr uint32_t kStepsPerGroup = 16;
 
 // Encoder scratch, per tensor (offsets in bytes from the tensor's scratch).
-//   hist     u64[256]       exponent counts
-//   ctr      u32[4]         [0] histogram tiles done, [1] unused,
-//                           [2] table written: 0 not yet, 1 narrow, 2 wide format,
-//                           [3] (first tensor of a launch) coding-task counter
-//   tab      uint4[256]     per-symbol coding entry: narrow {m, xmax, cmpl,
-//                           sh | bias << 5}, wide {ml, xmax, cmpl, mh}
+//   hist     u64[256]       coded-byte counts
+//   ctr      u32[4]         [0] histogram blocks done, [1] coder warps done,
+//                           [2] table written: 1 narrow, 2 wide format, [3] unused
+//   tab      uint4[256]     per-symbol coding entry (wc_coder.cuh): narrow {m,
+//                           xmax, cmpl, sh | bias << 5}, wide {ml, xmax, cmpl, mh}
 //   bias     u32[256]       per-symbol additive term (wide format)
-//   stat     u64[nc]        per-chunk look-back word: flag << 62 | bytes, flag
-//                           1 = the chunk's padded length, 2 = the padded
-//                           length of chunks 0..k, 3 = failed
+//   len      u32[nc]        chunk lengths
 //   windows  nc x kWin      coded chunk staging (states at the front,
 //                           words filled backwards from the end)
 constexpr uint64_t kScrHist = 0;
 constexpr uint64_t kScrCtr = 2048;
 constexpr uint64_t kScrTab = 2304;
 constexpr uint64_t kScrBias = kScrTab + 256 * 16;   // 6400
-constexpr uint64_t kScrStat = kScrBias + 256 * 4;   // 7424
+constexpr uint64_t kScrLen = kScrBias + 256 * 4;    // 7424
 constexpr uint64_t kWin = 65536 + 2048;             // 67584 bytes per chunk
 constexpr uint32_t kWinWords = kWin / 2;            // 33792
-constexpr uint64_t kStatAgg = uint64_t(1) << 62;
-constexpr uint64_t kStatInc = uint64_t(2) << 62;
-constexpr uint64_t kStatBad = uint64_t(3) << 62;
-constexpr uint64_t kStatVal = (uint64_t(1) << 62) - 1;
 
 // fp8 e4m3 and e5m2: one byte per value, the raw plane one nibble per value.
 __host__ __device__ constexpr bool is_fp8(int dt) { return dt == WC_FP8E4M3 || dt == WC_FP8E5M2; }
@@ -101,7 +94,7 @@ __host__ __device__ constexpr uint32_t dtype_bytes(int dtype) {
 }
 
 __host__ __device__ inline uint64_t scratch_win_offset(uint64_t nc) {
-  return round256(kScrStat + 8 * nc);
+  return round256(kScrLen + 4 * nc);
 }
 
 // ---------------------------------------------------------------------------
@@ -115,22 +108,18 @@ struct EncItem {
   uint8_t *scratch;
   uint64_t *out_size;
   uint64_t n;
+  uint32_t chunk_base;  // first global chunk index of this item in the launch
+  uint32_t block_base;  // first coder block of this item in the launch
   uint32_t dtype;
-  uint32_t pad;
+  uint32_t hist_base;   // first histogram block of this item in the launch
 };
 
-// The encoder's work, as runs of one tensor's tasks ("segments", empty ones
-// left out): histogram tiles (k_hist, one block per tile) and coding tasks
-// (k_encode, taken in order from a counter).  Segment s covers the tasks
-// [start[s], start[s + 1]) of its kernel, of item item[s].
 struct EncParams {
   uint32_t count;
-  uint32_t total_tiles, total_tasks;
-  uint32_t ntseg, ncseg;
-  uint32_t pad[3];
+  uint32_t total_chunks;
+  uint32_t total_coder_blocks;
+  uint32_t total_hist_blocks;
   EncItem items[kMaxItems];
-  uint32_t tseg_start[kMaxItems], tseg_item[kMaxItems];
-  uint32_t cseg_start[kMaxItems], cseg_item[kMaxItems];
 };
 
 struct DecItem {
@@ -151,28 +140,51 @@ struct DecParams {
 
 // Histogram blocks: one tile of up to 4 chunks of one tensor.
 constexpr uint32_t kHistChunks = 4;
-// Coding tasks: 8 warps, two chunks each, all of one tensor.
+// Encoder coder blocks: 8 warps, two chunks each, all of one tensor.
 constexpr uint32_t kCoderWarps = 8;
 constexpr uint32_t kCoderChunks = 2 * kCoderWarps;
 // Decoder blocks: 8 warps, two chunks each, all of one tensor.
 constexpr uint32_t kDecWarps = 8;
 
-// A bounded wait (a table, a predecessor's look-back word) gives up after
-// this many nanoseconds of the GPU's global timer.
-constexpr uint64_t kWaitNs = 4000000000ull;
-
 // Host launchers (one per kernel file).
 cudaError_t launch_prep(const EncParams &p, cudaStream_t s);
 cudaError_t launch_hist(const EncParams &p, cudaStream_t s);
-cudaError_t launch_encode(const EncParams &p, int grid, cudaStream_t s);
+cudaError_t launch_coder(const EncParams &p, cudaStream_t s);
+cudaError_t launch_compact(const EncParams &p, cudaStream_t s);
 cudaError_t launch_decode(const DecParams &p, int grid, cudaStream_t s);
 int decode_blocks_per_sm();
-int encode_blocks_per_sm();
 
 // ---------------------------------------------------------------------------
 // Device helpers.
 // ---------------------------------------------------------------------------
 #ifdef __CUDACC__
+__device__ __forceinline__ uint32_t find_item_by_chunk(const EncParams &p, uint32_t g) {
+  uint32_t lo = 0, hi = p.count - 1;
+  while (lo < hi) {
+    uint32_t mid = (lo + hi + 1) >> 1;
+    if (p.items[mid].chunk_base <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint32_t find_item_by_block(const EncParams &p, uint32_t b) {
+  uint32_t lo = 0, hi = p.count - 1;
+  while (lo < hi) {
+    uint32_t mid = (lo + hi + 1) >> 1;
+    if (p.items[mid].block_base <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ uint32_t find_item_by_hist(const EncParams &p, uint32_t b) {
+  uint32_t lo = 0, hi = p.count - 1;
+  while (lo < hi) {
+    uint32_t mid = (lo + hi + 1) >> 1;
+    if (p.items[mid].hist_base <= b) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
   uint32_t m;
   asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
