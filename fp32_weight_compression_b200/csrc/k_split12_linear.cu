@@ -8,31 +8,44 @@
 // Work split.  A CTA owns 128 weight rows (the MMA's M) and a range of K;
 // the host splits K across CTAs so that the grid is one wave, and the CTAs
 // of one row block add their partial sums into Y (fp32 atomics; Y is zeroed
-// first).  Per stage of 64 K-values:
-//   * cp.async brings the rows' 64 index nibbles and 64 low bytes each (12
-//     bits a value, as stored) and the tokens' X slice (n_mma x 64, rows past
-//     M zero-filled, straight into the B operand layout) into a ring slot,
-//     three stages ahead of the stage being expanded;
-//   * the 128 threads expand the 128 x 64 values from the ring slot in
-//     segments of 16 (8 index bytes + 16 low bytes -> 16 bf16, two 16-byte
-//     rows of core matrices) into one of two A operand slots and patch the
-//     tile's exceptions;
-//   * one thread issues four MMAs (M = 128, N = n_mma = M rounded up to 16,
-//     K = 16) and commits them to the slot's mbarrier; once the previous
-//     stage's MMAs are done its ring slot takes the next loads.
-// At the end each warp reads its 32 TMEM lanes (rows) and adds them into Y.
+// first).  Per stage of 64 K-values, in a pipeline without block-wide
+// barriers (mbarriers between the roles):
+//   * lane 0 of the load warp brings, with TMA, the rows' 64 index nibbles
+//     and 64 low bytes each (12 bits a value, as stored) and the tokens' X
+//     slice (n_mma x 64, rows past M zero-filled, eight 8-value groups each
+//     landing as n_mma rows of 16 bytes: the B operand layout) into a ring
+//     slot, up to four stages ahead, once the MMAs that read the slot last
+//     are done; the slot's mbarrier completes when the bytes have landed;
+//   * the 8 expanding warps expand the 128 x 64 values from the ring slot
+//     in segments of 16 (8 index bytes + 16 low bytes -> 16 bf16, two
+//     16-byte rows of core matrices) into one of two A operand slots, patch
+//     the tile's exceptions and arrive on the A slot's mbarrier.  A quarter
+//     warp takes 8 consecutive rows of one segment; with the loads' 32- and
+//     64-byte swizzles its index and low-byte reads, and its 16-byte stores,
+//     each cover 8 distinct bank groups;
+//   * lane 0 of the MMA warp waits for the A slot, issues four MMAs (M =
+//     128, N = n_mma = M rounded up to 16, K = 16) and commits them to the A
+//     slot's and the ring slot's "free" mbarriers, which the expanding warps
+//     and the load lane wait on before they reuse either.
+// At the end each expanding warp reads its 32 TMEM lanes (rows) and adds them
+// into Y.
 //
-// Operand layout (K-major, no swizzle): a core matrix is 8 rows x 16 bytes
-// stored as 128 contiguous bytes; the two 8-value halves of a K = 16 slice
-// are 128 bytes apart (leading byte offset) and consecutive 8-row groups 256
-// bytes apart (stride byte offset).  A slice of A is 16 groups = 4 KiB; a
-// slice of B is n_mma / 8 groups.
+// Operand layouts (K-major, no swizzle): a core matrix is 8 rows x 16 bytes
+// stored as 128 contiguous bytes.  A: the two 8-value halves of a K = 16
+// slice are 128 bytes apart (leading byte offset) and consecutive 8-row
+// groups 256 bytes apart (stride byte offset); a slice is 16 groups = 4 KiB.
+// B: each 8-value group of the stage is n_mma rows x 16 bytes, so the halves
+// are 16 n_mma bytes apart and 8-row groups 128 bytes apart.
 //
-// Waits: every mbarrier wait is bounded; when one runs out the kernel records
+// Waits: every mbarrier wait is bounded (and gives up once another thread has
+// failed); when one runs out the kernel records
 // WC_ERR_TIMEOUT, stops issuing, waits (bounded) for what it issued, frees its
 // tensor memory and returns.
 #include <cstdint>
 #include <mutex>
+
+#include <cuda.h>
+#include <cudaTypedefs.h>
 
 #include "wc.h"
 #include "wc_split12.cuh"
@@ -41,11 +54,15 @@ namespace wc12l {
 
 using wc12::kChunk;
 
-constexpr int kThreads = 256;  // 8 warps: all expand; warps 0-3 (TMEM lanes) and 4-7 split the epilogue
+constexpr int kExpThreads = 256;         // 8 warps expand; warps 0-3 (TMEM lanes) and 4-7 split the epilogue
+constexpr int kMmaWarp = 8;              // lane 0 issues the MMAs
+constexpr int kLoadWarp = 9;             // lane 0 issues the TMA loads
+constexpr int kThreads = kExpThreads + 64;
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr uint32_t kASlice = kBM * 16 * 2;   // bytes of one K = 16 slice of A
 constexpr uint32_t kAStage = 4 * kASlice;
+constexpr uint32_t kASlots = 2;
 constexpr uint32_t kMaxTokens = 256;
 constexpr uint32_t kSpinLimit = 1u << 24;
 // A CTA's exceptions (its 128 rows, its range of K) are gathered once into a
@@ -53,8 +70,15 @@ constexpr uint32_t kSpinLimit = 1u << 24;
 // row | high byte << 16 | low byte << 24}; a CTA with more walks its chunks'
 // exception lists at every stage instead.
 constexpr uint32_t kExcCap = 512;
+// chunk offsets of a CTA's row block kept in shared memory for the gather
+constexpr uint32_t kGatherChunks = 255;
 
 struct Params {
+  // tensor maps (tensor-core path): index plane [N rows][K / 2 bytes], box
+  // 128 x 32 B, 32-byte swizzle; low plane [N][K bytes], box 128 x 64 B,
+  // 64-byte swizzle; X [M][K bf16], box n_mma x 8 values (one per 8-value
+  // group of a stage; rows past M read as zeros)
+  CUtensorMap tm_idx, tm_lo, tm_x;
   const uint8_t *w;
   uint64_t w_bytes;
   const uint16_t *x;  // [M, K]
@@ -71,6 +95,9 @@ struct Params {
 // and the tokens' X slice already in the B operand layout), the mbarriers,
 // and the CTA's exception list.
 constexpr uint32_t kDepth = 4;
+// mbarriers (full, slot_free: kDepth each; a_full, a_free: kASlots each),
+// the TMEM address, the failure flag and the exception count
+constexpr uint32_t kBarBytes = 8 * (2 * kDepth + 2 * kASlots) + 16;
 constexpr uint32_t kIdxBytes = kBM * kBK / 2;  // 4 KiB
 constexpr uint32_t kLoBytes = kBM * kBK;       // 8 KiB
 
@@ -79,7 +106,8 @@ __host__ __device__ inline uint32_t slot_bytes(uint32_t n_mma) { return kIdxByte
 // per-stage exception bins: a count (then start) per stage of the CTA
 constexpr uint32_t kMaxStagesPerCta = 256;
 __host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma) {
-  return 1024 + 2 * kAStage + kDepth * slot_bytes(n_mma) + 64 + 2 * 8 * kExcCap + 2 * 4 * (kMaxStagesPerCta + 1);
+  return 1024 + kASlots * kAStage + kDepth * slot_bytes(n_mma) + kBarBytes + 2 * 8 * kExcCap +
+         2 * 4 * (kMaxStagesPerCta + 1) + 8 * (kGatherChunks + 1);
 }
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
@@ -88,10 +116,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// shared-memory matrix descriptor: K-major, no swizzle, LBO 128 B, SBO 256 B
-__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr) {
-  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t(128 >> 4) << 16) | (uint64_t(256 >> 4) << 32) |
-         (uint64_t(1) << 46);
+// shared-memory matrix descriptor: K-major, no swizzle, leading and stride
+// byte offsets lbo and sbo
+__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46);
 }
 
 // instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128, N = n
@@ -151,29 +180,89 @@ __device__ __forceinline__ uint32_t op_offset(uint32_t row, uint32_t k, uint32_t
   return (k >> 4) * slice_bytes + (row >> 3) * 256 + ((k >> 3) & 1) * 128 + (row & 7) * 16 + (k & 7) * 2;
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+// Where TMA puts 16-byte part `part` of row `row` of a plane's box: rows of
+// 32 bytes (index plane, 32-byte swizzle: part ^= bit 2 of the row) or 64
+// bytes (low plane, 64-byte swizzle: part ^= bits 1-2 of the row).
+__device__ __forceinline__ uint32_t idx_gran(uint32_t row, uint32_t part) {
+  return row * 32 + ((part ^ ((row >> 2) & 1u)) << 4);
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ uint32_t lo_gran(uint32_t row, uint32_t part) {
+  return row * 64 + ((part ^ ((row >> 1) & 3u)) << 4);
+}
 
-__global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant__ Params p) {
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+// 2-D tile load (no multicast) into this CTA's shared memory, completing on bar
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
+                                            uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Named barrier 1 over the expanding threads, returning whether ok holds for
+// all of them.
+__device__ __forceinline__ bool expanders_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(ok)), "n"(kExpThreads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void expanders_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kExpThreads) : "memory"); }
+
+// A bounded wait that also gives up once another thread of the CTA has
+// recorded a failure in *flag.
+__device__ __forceinline__ bool mbar_wait_or_flag(uint64_t *bar, uint32_t parity, const volatile int *flag) {
+  const uint32_t a = smem_u32(bar);
+  for (uint32_t i = 0; i < kSpinLimit; i++) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (*flag) return false;
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant__ Params p) {
   extern __shared__ uint8_t dyn[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
-  uint8_t *a_op = base;                       // 2 x kAStage
-  uint8_t *ring = base + 2 * kAStage;         // kDepth x slot_bytes
+  uint8_t *a_op = base;                       // kASlots x kAStage
+  uint8_t *ring = base + kASlots * kAStage;   // kDepth x slot_bytes
   const uint32_t sb = slot_bytes(p.n_mma);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(ring + kDepth * sb);  // kDepth
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bar + kDepth);
+  uint64_t *full = reinterpret_cast<uint64_t *>(ring + kDepth * sb);  // [kDepth] a slot's loads landed
+  uint64_t *slot_free = full + kDepth;                                // [kDepth] its MMAs are done
+  uint64_t *a_full = slot_free + kDepth;                              // [kASlots] A slot expanded
+  uint64_t *a_free = a_full + kASlots;                                // [kASlots] its MMAs are done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(a_free + kASlots);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
   uint32_t *exc_n = tmem_slot + 2;
-  uint2 *exc_raw = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(bar) + 64);  // gathered
-  uint2 *exc_bin = exc_raw + kExcCap;                                                  // by stage
-  uint32_t *bin = reinterpret_cast<uint32_t *>(exc_bin + kExcCap);                     // per stage
-  uint32_t *cur = bin + kMaxStagesPerCta + 1;                                          // scatter cursors
+  uint2 *exc_raw = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(full) + kBarBytes);  // gathered
+  uint2 *exc_bin = exc_raw + kExcCap;                                                        // by stage
+  uint32_t *bin = reinterpret_cast<uint32_t *>(exc_bin + kExcCap);                           // per stage
+  uint32_t *cur = bin + kMaxStagesPerCta + 1;                                                // cursors
+  uint64_t *g_off = reinterpret_cast<uint64_t *>(cur + kMaxStagesPerCta + 1);                 // gather offsets
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool expander = tid < kExpThreads;
   const uint32_t K = p.K, N = p.N;
   const uint32_t n0 = blockIdx.x * kBM;
   const uint32_t split = blockIdx.y;
@@ -209,42 +298,20 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   const uint8_t *lo_plane = w + L.off_lo;
   const uint64_t c_lo = uint64_t(n0) * K / kChunk, c_hi = (uint64_t(n0 + kBM) * K - 1) / kChunk;
 
-  // This thread's copies of every stage, with their sources at stage 0 of
-  // the CTA (a stage adds 32 bytes to an index-plane source, 64 to a
-  // low-plane source, 128 to an X source): three of the 768 copies of the
-  // rows' index and low bytes, and n_mma / 32 of the X slice's (tokens >= M
-  // are zero-filled).
+  // stage j's TMA loads into ring slot j % kDepth (the load lane)
   const uint32_t ring_s = smem_u32(ring);
   const uint32_t k_first = s_begin * kBK;
-  const uint8_t *a_src[3];
-  uint32_t a_dst[3];
-#pragma unroll
-  for (int r = 0; r < 3; r++) {
-    const uint32_t i = uint32_t(tid) + kThreads * r;
-    if (i < 2 * kBM) {
-      const uint32_t row = i >> 1, part = i & 1;
-      a_src[r] = w + L.off_idx + (uint64_t(n0 + row) * K + k_first) / 2 + 16 * part;
-      a_dst[r] = row * 32 + 16 * part;
-    } else {
-      const uint32_t j2 = i - 2 * kBM, row = j2 >> 2, part = j2 & 3;
-      a_src[r] = lo_plane + uint64_t(n0 + row) * K + k_first + 16 * part;
-      a_dst[r] = kIdxBytes + row * 64 + 16 * part;
-    }
-  }
-  const uint32_t nb = p.n_mma * 8;  // X copies per stage
-  auto issue_loads = [&](uint32_t j) {
-    const uint32_t slot = ring_s + (j % kDepth) * sb;
-    const uint32_t kofs = j * kBK;  // values past the CTA's first stage
-#pragma unroll
-    for (int r = 0; r < 3; r++) cp_async16(slot + a_dst[r], a_src[r] + (r == 0 && tid < 2 * kBM ? kofs / 2 : kofs), 16);
-    for (uint32_t j3 = tid; j3 < nb; j3 += kThreads) {
-      const uint32_t t = j3 >> 3, jj = j3 & 7;
-      const bool real = t < p.M;
-      cp_async16(slot + kIdxBytes + kLoBytes + op_offset(t, 8 * jj, p.n_mma * 32),
-                 real ? static_cast<const void *>(p.x + uint64_t(t) * K + k_first + kofs + 8 * jj) : p.x,
-                 real ? 16 : 0);
-    }
+  const uint32_t stage_bytes = kIdxBytes + kLoBytes + b_stage_bytes(p.n_mma);
+  auto load_stage = [&](uint32_t j) {
+    const uint32_t d = j % kDepth, slot = ring_s + d * sb;
+    const int32_t k = int32_t(k_first + j * kBK);
+    mbar_expect_tx(&full[d], stage_bytes);
+    tma_load_2d(slot, &p.tm_idx, k / 2, int32_t(n0), &full[d]);
+    tma_load_2d(slot + kIdxBytes, &p.tm_lo, k, int32_t(n0), &full[d]);
+    for (uint32_t g = 0; g < kBK / 8; g++)
+      tma_load_2d(slot + kIdxBytes + kLoBytes + g * p.n_mma * 16, &p.tm_x, k + int32_t(8 * g), 0, &full[d]);
   };
+  const bool loader = warp == kLoadWarp && lane == 0;
 
   // tensor memory: n_mma fp32 columns, rounded up to a power of two >= 32
   uint32_t cols = 32;
@@ -256,23 +323,28 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
   if (tid == 0) {
-    for (uint32_t d = 0; d < kDepth; d++) mbar_init(&bar[d], 1);
+    for (uint32_t d = 0; d < kDepth; d++) {
+      mbar_init(&full[d], 1);
+      mbar_init(&slot_free[d], 1);
+    }
+    for (uint32_t d = 0; d < kASlots; d++) {
+      mbar_init(&a_full[d], kExpThreads);
+      mbar_init(&a_free[d], 1);
+    }
     *flag = 0;
     *exc_n = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   for (uint32_t i = tid; i <= nst && i <= kMaxStagesPerCta; i += kThreads) bin[i] = 0;
-  // the first kDepth - 1 stages' loads are in flight while the exceptions
-  // are gathered
-  for (uint32_t j = 0; j + 1 < kDepth; j++) {
-    if (j < nst) issue_loads(j);
-    cp_async_commit();
-  }
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t idesc = instr_desc(p.n_mma);
+  // the first kDepth stages' loads are in flight while the exceptions are
+  // gathered
+  uint32_t loaded = 0;  // load lane: stages whose loads were issued
+  if (loader)
+    for (; loaded < kDepth && loaded < nst; loaded++) load_stage(loaded);
 
   // The CTA's exceptions, once: positions within a chunk become (row, column)
   // relative to the CTA's tile with 32-bit arithmetic when 128 K fits it,
@@ -281,37 +353,64 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
   const uint64_t f_base = uint64_t(n0) * K, f_span = uint64_t(kBM) * K;
   const uint32_t k_beg = s_begin * kBK, k_end = s_end * kBK;
   const bool binned = nst <= kMaxStagesPerCta;
-  for (uint64_t c = c_lo; c <= c_hi; c++) {
-    const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
-    if (e0 > e1 || e1 > ne) {
-      if (tid == 0) report(p.status, WC_ERR_CORRUPT);
-      continue;
-    }
+  // The chunks' lists follow one another in the container, so the row
+  // block's exceptions are the one range [exc_off[c_lo], exc_off[c_hi + 1]);
+  // its entries are taken by all threads at once, each finding its chunk by
+  // a search in a shared copy of the offsets (up to kGatherChunks chunks;
+  // beyond that, chunk after chunk).
+  const uint32_t nch = uint32_t(c_hi - c_lo + 1);
+  auto gather_one = [&](uint64_t c, uint64_t e) {
     const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
-    for (uint64_t e = e0 + tid; e < e1; e += kThreads) {
-      const uint32_t pos = exc_pos[e];
-      if (pos >= cnt) {
-        report(p.status, WC_ERR_CORRUPT);
+    const uint32_t pos = exc_pos[e];
+    if (pos >= cnt) {
+      report(p.status, WC_ERR_CORRUPT);
+      return;
+    }
+    const uint64_t f = c * kChunk + pos;
+    if (f < f_base || f - f_base >= f_span) return;
+    const uint64_t lf = f - f_base;
+    uint32_t row, col;
+    if (f_span <= 0xFFFFFFFFull) {
+      row = uint32_t(lf) / K;
+      col = uint32_t(lf) - row * K;
+    } else {
+      row = uint32_t(lf / K);
+      col = uint32_t(lf - uint64_t(row) * K);
+    }
+    if (col < k_beg || col >= k_end) return;
+    const uint32_t slot = atomicAdd(exc_n, 1u);
+    if (slot < kExcCap) {
+      exc_raw[slot] = make_uint2(col - k_beg, row | (uint32_t(exc_val[e]) << 16) |
+                                                  (uint32_t(lo_plane[f]) << 24));
+      if (binned) atomicAdd(&bin[(col - k_beg) / kBK], 1u);
+    }
+  };
+  if (nch <= kGatherChunks) {
+    for (uint32_t j = tid; j <= nch; j += kThreads) g_off[j] = exc_off[c_lo + j];
+    __syncthreads();
+    bool bad = false;
+    for (uint32_t j = tid; j < nch; j += kThreads) bad |= g_off[j] > g_off[j + 1] || g_off[j + 1] > ne;
+    if (__syncthreads_or(bad)) {
+      if (tid == 0) report(p.status, WC_ERR_CORRUPT);
+    } else {
+      const uint64_t e_beg = g_off[0], e_end = g_off[nch];
+      for (uint64_t e = e_beg + tid; e < e_end; e += kThreads) {
+        uint32_t lo = 0, hi = nch - 1;  // the last chunk j with g_off[j] <= e
+        while (lo < hi) {
+          const uint32_t mid = (lo + hi + 1) >> 1;
+          if (g_off[mid] <= e) lo = mid; else hi = mid - 1;
+        }
+        gather_one(c_lo + lo, e);
+      }
+    }
+  } else {
+    for (uint64_t c = c_lo; c <= c_hi; c++) {
+      const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
+      if (e0 > e1 || e1 > ne) {
+        if (tid == 0) report(p.status, WC_ERR_CORRUPT);
         continue;
       }
-      const uint64_t f = c * kChunk + pos;
-      if (f < f_base || f - f_base >= f_span) continue;
-      const uint64_t lf = f - f_base;
-      uint32_t row, col;
-      if (f_span <= 0xFFFFFFFFull) {
-        row = uint32_t(lf) / K;
-        col = uint32_t(lf) - row * K;
-      } else {
-        row = uint32_t(lf / K);
-        col = uint32_t(lf - uint64_t(row) * K);
-      }
-      if (col < k_beg || col >= k_end) continue;
-      const uint32_t slot = atomicAdd(exc_n, 1u);
-      if (slot < kExcCap) {
-        exc_raw[slot] = make_uint2(col - k_beg, row | (uint32_t(exc_val[e]) << 16) |
-                                                    (uint32_t(lo_plane[f]) << 24));
-        if (binned) atomicAdd(&bin[(col - k_beg) / kBK], 1u);
-      }
+      for (uint64_t e = e0 + tid; e < e1; e += kThreads) gather_one(c, e);
     }
   }
   __syncthreads();
@@ -344,99 +443,140 @@ __global__ void __launch_bounds__(kThreads, 1) k12_linear(const __grid_constant_
     __syncthreads();
   }
 
-  uint32_t it = 0;
-  for (; it < nst; it++) {
-    const uint32_t st = s_begin + it;
-    const uint32_t k0 = st * kBK;
-    uint8_t *A = a_op + (it & 1) * kAStage;
-    const uint8_t *slot = ring + (it % kDepth) * sb;
-    cp_async_wait<kDepth - 2>();  // this stage's loads (later stages may still be in flight)
-    __syncthreads();
-
-    // A: 512 segments of 16 values (row = i / 4, values 16 (i % 4) ..), two
-    // per thread, expanded from the ring slot into the operand slot
+  // The pipeline.  Expanding threads, stage s: wait for slot s % kDepth's
+  // loads and for A slot s % 2 to be free (the MMAs of stage s - 2), expand
+  // into it, arrive on its a_full; then load stage s + kDepth - 1 into the
+  // slot stage s - 1 used, once that stage's MMAs are done.  The MMA thread,
+  // stage s: wait for a_full, issue the four MMAs, commit them to a_free and
+  // slot_free.  No block-wide barrier inside the loop.
+  const volatile int *vflag = flag;
+  uint32_t issued = 0;  // MMA thread: stages whose MMAs were issued
+  if (expander) {
+    // this thread's two segments: offsets of their index and low bytes in a
+    // ring slot and of their two 16-byte rows in an A slot
+    uint32_t o_idx[2], o_lo[2], o_a[2];
 #pragma unroll
     for (int q = 0; q < 2; q++) {
-      const uint32_t i = uint32_t(tid) + kThreads * q, row = i >> 2, seg = i & 3;
-      const uint2 iw = *reinterpret_cast<const uint2 *>(slot + row * 32 + 8 * seg);
-      const uint4 lw = *reinterpret_cast<const uint4 *>(slot + kIdxBytes + row * 64 + 16 * seg);
-      const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
-      const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
-      *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg, kASlice)) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-      *reinterpret_cast<uint4 *>(A + op_offset(row, 16 * seg + 8, kASlice)) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+      const uint32_t i = uint32_t(tid) + kExpThreads * q, row = ((i >> 5) << 3) | (i & 7), seg = (i >> 3) & 3;
+      o_idx[q] = idx_gran(row, seg >> 1) + 8 * (seg & 1);
+      o_lo[q] = kIdxBytes + lo_gran(row, seg);
+      o_a[q] = op_offset(row, 16 * seg, kASlice);  // + 128: the segment's second 8 values
     }
-    // exceptions that fall in this tile
-    if (!exc_walk) {
-      // each is patched by the thread that expanded its segment (program
-      // order after that thread's stores: no barrier needed)
-      for (uint32_t i = bin[it]; i < bin[it + 1]; i++) {
-        const uint2 ex = exc_bin[i];
-        const uint32_t row = ex.y & 0xFFFFu, col = ex.x - it * kBK;
-        if ((row * 4 + (col >> 4)) % kThreads != uint32_t(tid)) continue;
-        *reinterpret_cast<uint16_t *>(A + op_offset(row, col, kASlice)) =
-            uint16_t(((ex.y >> 16) & 0xFFu) << 8 | (ex.y >> 24));
+    for (uint32_t s = 0; s < nst; s++) {
+      const uint32_t as = s % kASlots;
+      uint8_t *A = a_op + as * kAStage;
+      const uint8_t *slot = ring + (s % kDepth) * sb;
+      // the stage's loads have landed; A slot s % 2 is free once the MMAs of
+      // stage s - 2 are done
+      bool okw = mbar_wait_or_flag(&full[s % kDepth], (s / kDepth) & 1u, vflag) &&
+                 (s < kASlots || mbar_wait_or_flag(&a_free[as], ((s / kASlots) & 1u) ^ 1u, vflag));
+      // with the per-stage walk the expanders meet at named barriers, so
+      // they decide together whether to go on
+      if (exc_walk) okw = expanders_all(okw);
+      if (!okw) {
+        if (!*vflag) report(p.status, WC_ERR_TIMEOUT);
+        *flag = 1;
+        break;
       }
-    } else {
-      __syncthreads();  // every segment expanded before any thread patches
-      for (uint64_t c = c_lo; c <= c_hi; c++) {
-        const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
-        if (e0 > e1 || e1 > ne) continue;  // reported by the gathering pass
-        const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
-        for (uint64_t e = e0 + tid; e < e1; e += kThreads) {
-          const uint32_t pos = exc_pos[e];
-          if (pos >= cnt) continue;
-          const uint64_t f = c * kChunk + pos;
-          const uint64_t row = f / K, col = f % K;
-          if (row < n0 || row >= n0 + kBM || col < k0 || col >= k0 + kBK) continue;
-          *reinterpret_cast<uint16_t *>(A + op_offset(uint32_t(row - n0), uint32_t(col - k0), kASlice)) =
-              uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[f]);
+      const uint32_t k0 = (s_begin + s) * kBK;
+      const uint32_t eb0 = exc_walk ? 0u : bin[s], eb1 = exc_walk ? 0u : bin[s + 1];
+      // A: 512 segments of 16 values, two per thread: segment i is row
+      // 8 (i / 32) + i % 8, values 16 ((i / 8) % 4) .., expanded from the
+      // ring slot into the operand slot
+#pragma unroll
+      for (int q = 0; q < 2; q++) {
+        const uint2 iw = *reinterpret_cast<const uint2 *>(slot + o_idx[q]);
+        const uint4 lw = *reinterpret_cast<const uint4 *>(slot + o_lo[q]);
+        const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
+        const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
+        *reinterpret_cast<uint4 *>(A + o_a[q]) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+        *reinterpret_cast<uint4 *>(A + o_a[q] + 128) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+      }
+      // exceptions that fall in this tile
+      if (!exc_walk) {
+        // each is patched by the thread that expanded its segment (program
+        // order after that thread's stores)
+        for (uint32_t i = eb0; i < eb1; i++) {
+          const uint2 ex = exc_bin[i];
+          const uint32_t row = ex.y & 0xFFFFu, col = ex.x - s * kBK;
+          if ((((row >> 3) << 5) | ((col >> 4) << 3) | (row & 7)) % kExpThreads != uint32_t(tid)) continue;
+          *reinterpret_cast<uint16_t *>(A + op_offset(row, col, kASlice)) =
+              uint16_t(((ex.y >> 16) & 0xFFu) << 8 | (ex.y >> 24));
+        }
+      } else {
+        // each expanding thread patches the entries it finds, which may lie in
+        // another thread's segment: the expanders meet first
+        expanders_sync();
+        for (uint64_t c = c_lo; c <= c_hi; c++) {
+          const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
+          if (e0 > e1 || e1 > ne) continue;  // reported by the gathering pass
+          const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
+          for (uint64_t e = e0 + tid; e < e1; e += kExpThreads) {
+            const uint32_t pos = exc_pos[e];
+            if (pos >= cnt) continue;
+            const uint64_t f = c * kChunk + pos;
+            const uint64_t row = f / K, col = f % K;
+            if (row < n0 || row >= n0 + kBM || col < k0 || col >= k0 + kBK) continue;
+            *reinterpret_cast<uint16_t *>(A + op_offset(uint32_t(row - n0), uint32_t(col - k0), kASlice)) =
+                uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[f]);
+          }
         }
       }
+      fence_proxy_async();  // generic-proxy writes -> visible to the tensor cores
+      mbar_arrive(&a_full[as]);
     }
-    fence_proxy_async();  // generic-proxy writes -> visible to the tensor cores
-    __syncthreads();
-    if (tid == 0) {
+  } else if (warp == kMmaWarp && lane == 0) {
+    const uint32_t idesc = instr_desc(p.n_mma);
+    for (uint32_t s = 0; s < nst; s++) {
+      const uint32_t as = s % kASlots;
+      if (!mbar_wait_or_flag(&a_full[as], (s / kASlots) & 1u, vflag)) {
+        if (!*vflag) report(p.status, WC_ERR_TIMEOUT);
+        *flag = 1;
+        break;
+      }
       fence_after_sync();
-      const uint32_t a0 = smem_u32(A), b0 = smem_u32(slot + kIdxBytes + kLoBytes);
+      const uint32_t a0 = smem_u32(a_op + as * kAStage), b0 = ring_s + (s % kDepth) * sb + kIdxBytes + kLoBytes;
+      const uint32_t b_lbo = p.n_mma * 16;  // one 8-value group of B
 #pragma unroll
       for (uint32_t sl = 0; sl < 4; sl++)
-        mma_bf16(tmem, operand_desc(a0 + sl * kASlice), operand_desc(b0 + sl * p.n_mma * 32), idesc,
-                 (it > 0 || sl > 0) ? 1u : 0u);
-      mma_commit(&bar[it % kDepth]);
-      // the slot of stage it - 1 is free once its MMAs are done (which also
-      // frees the A slot stage it + 1 writes); one thread waits, the rest
-      // wait at the barrier below
-      if (it >= 1) {
-        const uint32_t prev = it - 1;
-        if (!mbar_wait(&bar[prev % kDepth], (prev / kDepth) & 1u)) {
-          report(p.status, WC_ERR_TIMEOUT);
-          *flag = 1;
-        }
+        mma_bf16(tmem, operand_desc(a0 + sl * kASlice, 128, 256), operand_desc(b0 + sl * 2 * b_lbo, b_lbo, 128),
+                 idesc, (s > 0 || sl > 0) ? 1u : 0u);
+      mma_commit(&a_free[as]);
+      mma_commit(&slot_free[s % kDepth]);
+      issued = s + 1;
+    }
+  } else if (loader) {
+    // stage j reuses the slot of stage j - kDepth once its MMAs are done
+    for (; loaded < nst; loaded++) {
+      const uint32_t prev = loaded - kDepth;
+      if (!mbar_wait_or_flag(&slot_free[prev % kDepth], (prev / kDepth) & 1u, vflag)) {
+        if (!*vflag) report(p.status, WC_ERR_TIMEOUT);
+        *flag = 1;
+        break;
       }
+      load_stage(loaded);
     }
-    __syncthreads();
-    if (*flag) {
-      it++;  // stage it was issued
-      break;
-    }
-    if (it + kDepth - 1 < nst) issue_loads(it + kDepth - 1);
-    cp_async_commit();
+    // no load may still be in flight when the CTA ends: wait (bounded, also
+    // after a failure) for the last stage issued into each slot
+    for (uint32_t j = loaded > kDepth ? loaded - kDepth : 0; j < loaded; j++)
+      if (!mbar_wait(&full[j % kDepth], (j / kDepth) & 1u)) report(p.status, WC_ERR_TIMEOUT);
   }
-  cp_async_wait<0>();
 
-  // wait for the last stage issued (its commit covers all earlier MMAs)
-  const uint32_t issued = it;
+  // The MMA thread waits for the last stage it issued (the commit covers all
+  // earlier MMAs), without giving up on a flag: tensor memory is read and
+  // freed only after its MMAs are done.
   bool done = true;
-  if (issued > 0 && tid == 0) {
+  if (warp == kMmaWarp && lane == 0 && issued > 0) {
     const uint32_t last = issued - 1;
-    done = mbar_wait(&bar[last % kDepth], (last / kDepth) & 1u);
+    done = mbar_wait(&slot_free[last % kDepth], (last / kDepth) & 1u);
   }
+  if (!expander) __syncwarp();
   // every thread takes the same branch below: the tensor-memory loads are
   // warp-collective (.sync.aligned)
   done = __syncthreads_and(done) != 0;
-  if (!done && tid == 0) report(p.status, WC_ERR_TIMEOUT);
+  if (!done && tid == kExpThreads) report(p.status, WC_ERR_TIMEOUT);
   fence_after_sync();
-  if (done && !*flag && issued > 0) {
+  if (done && !*flag && expander) {
     // warp w reads TMEM lanes 32 (w % 4) .. (its rows); warps 0-3 take the
     // even 8-column groups, warps 4-7 the odd ones
     const uint32_t lane_base = 32 * (warp & 3);
@@ -654,6 +794,7 @@ struct DevInfo {
   bool attr = false;
   int smem_per_sm = 0;     // shared memory of one SM
   int smem_reserved = 0;   // per CTA, taken by the system
+  int regs = 0;            // registers a thread of k12_linear
 };
 
 // Dynamic shared memory for a launch with n_mma token columns: at least what
@@ -670,6 +811,36 @@ uint32_t launch_smem(const DevInfo &d, uint32_t n_mma) {
   const uint32_t floor_smem = per_sm / (max_ctas + 1) + 1;
   if (floor_smem > rsv && need + rsv < floor_smem) need = floor_smem - rsv;
   return need;
+}
+
+// cuTensorMapEncodeTiled, from the driver (once)
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void *f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// A 2-D map over rows of `inner` elements, `row_bytes` apart, loaded in
+// boxes of box_rows x box_inner.
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t rows,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows, CUtensorMapSwizzle sw,
+              CUtensorMapL2promotion l2) {
+  const PFN_cuTensorMapEncodeTiled_v12000 fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, l2,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 DevInfo dev_info() {
@@ -695,6 +866,9 @@ DevInfo dev_info() {
     }
     d.attr = cudaFuncSetAttribute(k12_linear, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   int(most)) == cudaSuccess;
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, k12_linear) != cudaSuccess) return DevInfo{};
+    d.regs = fa.numRegs;
     d.sms = sms;
   }
   return d;
@@ -731,6 +905,16 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   if (di.sms <= 0 || !di.attr) return WC_ERR_CUDA;
   const uint32_t blocks = N / wc12l::kBM, stages = K / wc12l::kBK;
   if (blocks == 0) return WC_ERR_INVALID_ARG;
+  // the planes the tensor maps cover must lie inside the buffer (their
+  // offsets depend on N K only; the kernel checks the header itself)
+  const uint64_t n = uint64_t(N) * K;
+  const wc12::Lay L = wc12::lay(n, 0);
+  if (w_bytes < L.off_lo + n) return WC_ERR_INVALID_ARG;
+  if (!wc12l::make_map(&p.tm_idx, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w + L.off_idx, K / 2, N, K / 2, 32,
+                       wc12l::kBM, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+      !wc12l::make_map(&p.tm_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w + L.off_lo, K, N, K, 64, wc12l::kBM,
+                       CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B))
+    return WC_ERR_CUDA;
   // tokens in slices of at most kMaxTokens (the MMA's N); each slice's rows
   // of X and Y are contiguous
   for (uint32_t t0 = 0; t0 < M; t0 += wc12l::kMaxTokens) {
@@ -739,12 +923,22 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
     p.y = d_y + uint64_t(t0) * N;
     p.M = m;
     p.n_mma = (m + 15) / 16 * 16;
+    if (!wc12l::make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, K, m, uint64_t(K) * 2, 8, p.n_mma,
+                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+      return WC_ERR_CUDA;
     // split K so that the grid is one wave of the CTAs an SM holds, with at
-    // least 4 stages a CTA when K allows (the load ring runs 3 ahead)
+    // least 4 stages a CTA when K allows (the load ring runs 4 ahead)
     const uint32_t smem = wc12l::launch_smem(di, p.n_mma);
     uint32_t cols = 32;
     while (cols < p.n_mma) cols <<= 1;
+    // CTAs an SM holds: shared memory, registers (whole warps of 8-register
+    // granules), threads, and the two the kernel is compiled for
     uint32_t per_sm = uint32_t(di.smem_per_sm) / (smem + uint32_t(di.smem_reserved));
+    const uint32_t warp_regs = (uint32_t(di.regs) + 7) / 8 * 8 * 32;
+    const uint32_t by_regs = 65536 / (warp_regs * (wc12l::kThreads / 32));
+    if (per_sm > by_regs) per_sm = by_regs;
+    if (per_sm > 2048 / wc12l::kThreads) per_sm = 2048 / wc12l::kThreads;
+    if (per_sm > 2) per_sm = 2;
     if (per_sm > 512 / cols) per_sm = 512 / cols;
     if (per_sm < 1) per_sm = 1;
     uint32_t splits = uint32_t(di.sms) * per_sm / blocks;
