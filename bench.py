@@ -596,7 +596,7 @@ def linear_leg(ins, specs_mine, dev, reps: int = 20):
     """wc12_linear (Y = X W^T with W held as a Split12 container, expanded
     into the tensor cores' operand layout inside the kernel) against
     torch.matmul on the bf16 weights (cuBLAS), for token counts M = 1 .. 256
-    (M <= 8: the library's CUDA-core path; more: its tensor-core path).
+    (the tensor-core path at every M).
     W: the first four gate projections of the set (4096 x 14336 bf16, 117 MB
     each, 470 MB together > L2), used in rotation so that every call reads its
     weights from HBM.  Reported per M: microseconds per call and the weight

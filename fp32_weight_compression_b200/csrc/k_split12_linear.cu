@@ -12,17 +12,18 @@
 // barriers (mbarriers between the roles):
 //   * lane 0 of the load warp brings, with TMA, the rows' 64 index nibbles
 //     and 64 low bytes each (12 bits a value, as stored) and the tokens' X
-//     slice (n_mma x 64, rows past M zero-filled, eight 8-value groups each
-//     landing as n_mma rows of 16 bytes: the B operand layout) into a ring
-//     slot, up to four stages ahead, once the MMAs that read the slot last
-//     are done; the slot's mbarrier completes when the bytes have landed;
+//     slice (n_mma rows of 128 bytes, rows past M zero-filled, 128-byte
+//     swizzle: the B operand layout) into a ring slot, up to four stages
+//     ahead, once the MMAs that read the slot last are done; the slot's
+//     mbarrier completes when the bytes have landed;
 //   * the 8 expanding warps expand the 128 x 64 values from the ring slot
 //     in segments of 16 (8 index bytes + 16 low bytes -> 16 bf16, two
 //     16-byte rows of core matrices) into one of two A operand slots, patch
-//     the tile's exceptions and arrive on the A slot's mbarrier.  A quarter
-//     warp takes 8 consecutive rows of one segment; with the loads' 32- and
-//     64-byte swizzles its index and low-byte reads, and its 16-byte stores,
-//     each cover 8 distinct bank groups;
+//     the tile's exceptions (after a named barrier among them, one thread
+//     an exception, its high byte) and arrive on the A slot's mbarrier.  A
+//     quarter warp takes 8 consecutive rows of one segment; with the loads'
+//     32- and 64-byte swizzles its index and low-byte reads, and its 16-byte
+//     stores, each cover 8 distinct bank groups;
 //   * lane 0 of the MMA warp waits for the A slot, issues four MMAs (M =
 //     128, N = n_mma = M rounded up to 16, K = 16) and commits them to the A
 //     slot's and the ring slot's "free" mbarriers, which the expanding warps
@@ -30,12 +31,12 @@
 // At the end each expanding warp reads its 32 TMEM lanes (rows) and adds them
 // into Y.
 //
-// Operand layouts (K-major, no swizzle): a core matrix is 8 rows x 16 bytes
-// stored as 128 contiguous bytes.  A: the two 8-value halves of a K = 16
+// Operand layouts (K-major).  A, no swizzle: a core matrix is 8 rows x 16
+// bytes stored as 128 contiguous bytes; the two 8-value halves of a K = 16
 // slice are 128 bytes apart (leading byte offset) and consecutive 8-row
 // groups 256 bytes apart (stride byte offset); a slice is 16 groups = 4 KiB.
-// B: each 8-value group of the stage is n_mma rows x 16 bytes, so the halves
-// are 16 n_mma bytes apart and 8-row groups 128 bytes apart.
+// B, 128-byte swizzle: a token's 64 values are one 128-byte row, 8-row
+// groups 1024 bytes apart; the K = 16 slice sl starts 32 sl bytes in.
 //
 // Waits: every mbarrier wait is bounded (and gives up once another thread has
 // failed); when one runs out the kernel records
@@ -67,8 +68,9 @@ constexpr uint32_t kMaxTokens = 256;
 constexpr uint32_t kSpinLimit = 1u << 24;
 // A CTA's exceptions (its 128 rows, its range of K) are gathered once into a
 // shared-memory list of up to kExcCap entries {column in the CTA's K range,
-// row | high byte << 16 | low byte << 24}; a CTA with more walks its chunks'
-// exception lists at every stage instead.
+// row | high byte << 16}; a CTA with more walks its chunks' exception lists
+// at every stage instead.  Either way an exception's value differs from the
+// expanded one only in its high byte (the low byte is stored for every value).
 constexpr uint32_t kExcCap = 512;
 // chunk offsets of a CTA's row block kept in shared memory for the gather
 constexpr uint32_t kGatherChunks = 255;
@@ -76,8 +78,8 @@ constexpr uint32_t kGatherChunks = 255;
 struct Params {
   // tensor maps (tensor-core path): index plane [N rows][K / 2 bytes], box
   // 128 x 32 B, 32-byte swizzle; low plane [N][K bytes], box 128 x 64 B,
-  // 64-byte swizzle; X [M][K bf16], box n_mma x 8 values (one per 8-value
-  // group of a stage; rows past M read as zeros)
+  // 64-byte swizzle; X [M][K bf16], box n_mma x 64 values, 128-byte swizzle
+  // (rows past M read as zeros)
   CUtensorMap tm_idx, tm_lo, tm_x;
   const uint8_t *w;
   uint64_t w_bytes;
@@ -116,11 +118,11 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-// shared-memory matrix descriptor: K-major, no swizzle, leading and stride
-// byte offsets lbo and sbo
-__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// shared-memory matrix descriptor, K-major: leading and stride byte offsets
+// lbo and sbo, layout 0 (no swizzle) or 2 (128-byte swizzle)
+__device__ __forceinline__ uint64_t operand_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
   return uint64_t((saddr >> 4) & 0x3FFFu) | (uint64_t((lbo >> 4) & 0x3FFFu) << 16) |
-         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46);
+         (uint64_t((sbo >> 4) & 0x3FFFu) << 32) | (uint64_t(1) << 46) | (uint64_t(layout) << 61);
 }
 
 // instruction descriptor: bf16 x bf16 -> f32, both K-major, M = 128, N = n
@@ -221,7 +223,7 @@ __device__ __forceinline__ bool expanders_all(bool ok) {
       : "memory");
   return r != 0;
 }
-__device__ __forceinline__ void expanders_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kExpThreads) : "memory"); }
+
 
 // A bounded wait that also gives up once another thread of the CTA has
 // recorded a failure in *flag.
@@ -295,7 +297,6 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
   const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(w + wc12::kExcOffOff);
   const uint16_t *exc_pos = reinterpret_cast<const uint16_t *>(w + L.off_exc);
   const uint8_t *exc_val = w + L.off_excval;
-  const uint8_t *lo_plane = w + L.off_lo;
   const uint64_t c_lo = uint64_t(n0) * K / kChunk, c_hi = (uint64_t(n0 + kBM) * K - 1) / kChunk;
 
   // stage j's TMA loads into ring slot j % kDepth (the load lane)
@@ -308,8 +309,7 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
     mbar_expect_tx(&full[d], stage_bytes);
     tma_load_2d(slot, &p.tm_idx, k / 2, int32_t(n0), &full[d]);
     tma_load_2d(slot + kIdxBytes, &p.tm_lo, k, int32_t(n0), &full[d]);
-    for (uint32_t g = 0; g < kBK / 8; g++)
-      tma_load_2d(slot + kIdxBytes + kLoBytes + g * p.n_mma * 16, &p.tm_x, k + int32_t(8 * g), 0, &full[d]);
+    tma_load_2d(slot + kIdxBytes + kLoBytes, &p.tm_x, k, 0, &full[d]);
   };
   const bool loader = warp == kLoadWarp && lane == 0;
 
@@ -359,9 +359,8 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
   // a search in a shared copy of the offsets (up to kGatherChunks chunks;
   // beyond that, chunk after chunk).
   const uint32_t nch = uint32_t(c_hi - c_lo + 1);
-  auto gather_one = [&](uint64_t c, uint64_t e) {
+  auto gather_one = [&](uint64_t c, uint64_t e, uint32_t pos) {
     const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
-    const uint32_t pos = exc_pos[e];
     if (pos >= cnt) {
       report(p.status, WC_ERR_CORRUPT);
       return;
@@ -380,8 +379,7 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
     if (col < k_beg || col >= k_end) return;
     const uint32_t slot = atomicAdd(exc_n, 1u);
     if (slot < kExcCap) {
-      exc_raw[slot] = make_uint2(col - k_beg, row | (uint32_t(exc_val[e]) << 16) |
-                                                  (uint32_t(lo_plane[f]) << 24));
+      exc_raw[slot] = make_uint2(col - k_beg, row | (uint32_t(exc_val[e]) << 16));
       if (binned) atomicAdd(&bin[(col - k_beg) / kBK], 1u);
     }
   };
@@ -394,13 +392,25 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
       if (tid == 0) report(p.status, WC_ERR_CORRUPT);
     } else {
       const uint64_t e_beg = g_off[0], e_end = g_off[nch];
-      for (uint64_t e = e_beg + tid; e < e_end; e += kThreads) {
-        uint32_t lo = 0, hi = nch - 1;  // the last chunk j with g_off[j] <= e
-        while (lo < hi) {
-          const uint32_t mid = (lo + hi + 1) >> 1;
-          if (g_off[mid] <= e) lo = mid; else hi = mid - 1;
+      constexpr uint32_t kG = 4;  // positions loaded together
+      for (uint64_t e = e_beg + tid; e < e_end; e += kThreads * kG) {
+        uint32_t pos[kG];
+#pragma unroll
+        for (uint32_t u = 0; u < kG; u++) {
+          const uint64_t eu = e + uint64_t(u) * kThreads;
+          pos[u] = eu < e_end ? exc_pos[eu] : 0u;
         }
-        gather_one(c_lo + lo, e);
+#pragma unroll
+        for (uint32_t u = 0; u < kG; u++) {
+          const uint64_t eu = e + uint64_t(u) * kThreads;
+          if (eu >= e_end) break;
+          uint32_t lo = 0, hi = nch - 1;  // the last chunk j with g_off[j] <= eu
+          while (lo < hi) {
+            const uint32_t mid = (lo + hi + 1) >> 1;
+            if (g_off[mid] <= eu) lo = mid; else hi = mid - 1;
+          }
+          gather_one(c_lo + lo, eu, pos[u]);
+        }
       }
     }
   } else {
@@ -410,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
         if (tid == 0) report(p.status, WC_ERR_CORRUPT);
         continue;
       }
-      for (uint64_t e = e0 + tid; e < e1; e += kThreads) gather_one(c, e);
+      for (uint64_t e = e0 + tid; e < e1; e += kThreads) gather_one(c, e, exc_pos[e]);
     }
   }
   __syncthreads();
@@ -468,45 +478,39 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
       const uint8_t *slot = ring + (s % kDepth) * sb;
       // the stage's loads have landed; A slot s % 2 is free once the MMAs of
       // stage s - 2 are done
-      bool okw = mbar_wait_or_flag(&full[s % kDepth], (s / kDepth) & 1u, vflag) &&
-                 (s < kASlots || mbar_wait_or_flag(&a_free[as], ((s / kASlots) & 1u) ^ 1u, vflag));
-      // with the per-stage walk the expanders meet at named barriers, so
-      // they decide together whether to go on
-      if (exc_walk) okw = expanders_all(okw);
-      if (!okw) {
+      const bool okw = mbar_wait_or_flag(&full[s % kDepth], (s / kDepth) & 1u, vflag) &&
+                       (s < kASlots || mbar_wait_or_flag(&a_free[as], ((s / kASlots) & 1u) ^ 1u, vflag));
+      const uint32_t k0 = (s_begin + s) * kBK;
+      const uint32_t eb0 = exc_walk ? 0u : bin[s], eb1 = exc_walk ? 0u : bin[s + 1];
+      if (okw) {
+        // A: 512 segments of 16 values, two per thread: segment i is row
+        // 8 (i / 32) + i % 8, values 16 ((i / 8) % 4) .., expanded from the
+        // ring slot into the operand slot
+#pragma unroll
+        for (int q = 0; q < 2; q++) {
+          const uint2 iw = *reinterpret_cast<const uint2 *>(slot + o_idx[q]);
+          const uint4 lw = *reinterpret_cast<const uint4 *>(slot + o_lo[q]);
+          const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
+          const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
+          *reinterpret_cast<uint4 *>(A + o_a[q]) = make_uint4(e0.x, e0.y, e1.x, e1.y);
+          *reinterpret_cast<uint4 *>(A + o_a[q] + 128) = make_uint4(e2.x, e2.y, e3.x, e3.y);
+        }
+      }
+      // The expanders meet (named barrier 1): every segment of the stage is
+      // written, and all decide together whether to go on.
+      if (!expanders_all(okw)) {
         if (!*vflag) report(p.status, WC_ERR_TIMEOUT);
         *flag = 1;
         break;
       }
-      const uint32_t k0 = (s_begin + s) * kBK;
-      const uint32_t eb0 = exc_walk ? 0u : bin[s], eb1 = exc_walk ? 0u : bin[s + 1];
-      // A: 512 segments of 16 values, two per thread: segment i is row
-      // 8 (i / 32) + i % 8, values 16 ((i / 8) % 4) .., expanded from the
-      // ring slot into the operand slot
-#pragma unroll
-      for (int q = 0; q < 2; q++) {
-        const uint2 iw = *reinterpret_cast<const uint2 *>(slot + o_idx[q]);
-        const uint4 lw = *reinterpret_cast<const uint4 *>(slot + o_lo[q]);
-        const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
-        const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
-        *reinterpret_cast<uint4 *>(A + o_a[q]) = make_uint4(e0.x, e0.y, e1.x, e1.y);
-        *reinterpret_cast<uint4 *>(A + o_a[q] + 128) = make_uint4(e2.x, e2.y, e3.x, e3.y);
-      }
-      // exceptions that fall in this tile
+      // the exceptions that fall in this tile get their high bytes, one
+      // thread an exception
       if (!exc_walk) {
-        // each is patched by the thread that expanded its segment (program
-        // order after that thread's stores)
-        for (uint32_t i = eb0; i < eb1; i++) {
+        for (uint32_t i = eb0 + uint32_t(tid); i < eb1; i += kExpThreads) {
           const uint2 ex = exc_bin[i];
-          const uint32_t row = ex.y & 0xFFFFu, col = ex.x - s * kBK;
-          if ((((row >> 3) << 5) | ((col >> 4) << 3) | (row & 7)) % kExpThreads != uint32_t(tid)) continue;
-          *reinterpret_cast<uint16_t *>(A + op_offset(row, col, kASlice)) =
-              uint16_t(((ex.y >> 16) & 0xFFu) << 8 | (ex.y >> 24));
+          A[op_offset(ex.y & 0xFFFFu, ex.x - s * kBK, kASlice) + 1] = uint8_t(ex.y >> 16);
         }
       } else {
-        // each expanding thread patches the entries it finds, which may lie in
-        // another thread's segment: the expanders meet first
-        expanders_sync();
         for (uint64_t c = c_lo; c <= c_hi; c++) {
           const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
           if (e0 > e1 || e1 > ne) continue;  // reported by the gathering pass
@@ -517,8 +521,7 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
             const uint64_t f = c * kChunk + pos;
             const uint64_t row = f / K, col = f % K;
             if (row < n0 || row >= n0 + kBM || col < k0 || col >= k0 + kBK) continue;
-            *reinterpret_cast<uint16_t *>(A + op_offset(uint32_t(row - n0), uint32_t(col - k0), kASlice)) =
-                uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[f]);
+            A[op_offset(uint32_t(row - n0), uint32_t(col - k0), kASlice) + 1] = exc_val[e];
           }
         }
       }
@@ -536,10 +539,9 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
       }
       fence_after_sync();
       const uint32_t a0 = smem_u32(a_op + as * kAStage), b0 = ring_s + (s % kDepth) * sb + kIdxBytes + kLoBytes;
-      const uint32_t b_lbo = p.n_mma * 16;  // one 8-value group of B
 #pragma unroll
       for (uint32_t sl = 0; sl < 4; sl++)
-        mma_bf16(tmem, operand_desc(a0 + sl * kASlice, 128, 256), operand_desc(b0 + sl * 2 * b_lbo, b_lbo, 128),
+        mma_bf16(tmem, operand_desc(a0 + sl * kASlice, 128, 256, 0), operand_desc(b0 + 32 * sl, 16, 1024, 2),
                  idesc, (s > 0 || sl > 0) ? 1u : 0u);
       mma_commit(&a_free[as]);
       mma_commit(&slot_free[s % kDepth]);
@@ -608,181 +610,6 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
-// Few tokens (M <= kGemvMaxM): the layer is bound by reading W, so it runs on
-// the CUDA cores, one warp per weight row, streaming the row's index nibbles
-// and low bytes (12 bits a value) and expanding them in registers: each lane
-// takes 16 consecutive values per step of 512, expands them with the
-// codebook (four byte permutes and a select per 4 values), patches the
-// tile's exceptions, and adds the exact bf16 x bf16 products into fp32 sums
-// (one per token); a warp reduction ends the row.  Exceptions are met in
-// order: a warp-uniform cursor walks the container's exception list, which
-// is sorted by position within each chunk and chunk after chunk.
-constexpr int kGemvWarps = 8;
-constexpr uint32_t kGemvMaxM = 8;
-
-template <int MT>
-__global__ void __launch_bounds__(kGemvWarps * 32) k12_gemv(const __grid_constant__ Params p) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint32_t K = p.K, N = p.N;
-  const uint8_t *w = p.w;
-  const uint32_t *h32 = reinterpret_cast<const uint32_t *>(w);
-  const uint64_t *h64 = reinterpret_cast<const uint64_t *>(w);
-  const uint64_t n = h64[1], ne = h64[3];
-  const uint32_t kk = h32[1] >> 24;
-  bool ok = h32[0] == wc12::kMagic && (h32[1] & 0xFFFFFFu) == (1u | (1u << 16)) &&
-            kk >= 1 && kk <= 16 && n == uint64_t(N) * K && ne <= n && h32[4] == uint32_t(kChunk);
-  wc12::Lay L{};
-  if (ok) {
-    L = wc12::lay(n, ne);
-    ok = h32[5] == uint32_t(L.nc) && h64[4] == L.off_idx && h64[5] == L.off_lo && h64[6] == L.off_exc &&
-         h64[7] == L.total && L.total <= p.w_bytes;
-  }
-  if (!ok) {
-    if (blockIdx.x == 0 && threadIdx.x == 0) report(p.status, WC_ERR_CORRUPT);
-    return;
-  }
-  const uint32_t row = blockIdx.x * kGemvWarps + warp;
-  if (row >= N) return;
-  const uint4 book = *reinterpret_cast<const uint4 *>(w + wc12::kBookOff);
-  const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(w + wc12::kExcOffOff);
-  const uint16_t *exc_pos = reinterpret_cast<const uint16_t *>(w + L.off_exc);
-  const uint8_t *exc_val = w + L.off_excval;
-  const uint8_t *idx_plane = w + L.off_idx;
-  const uint8_t *lo_plane = w + L.off_lo;
-  const uint64_t r0 = uint64_t(row) * K;
-
-  // exception cursor: chunk c, list index e = the first exception at or
-  // after value r0 (a search in chunk c's sorted positions); next_pos is its
-  // position among all values (~0 when the list is done), kept in a register
-  // so that a step reads the list only when an exception falls in it
-  uint64_t c = r0 / kChunk;
-  uint64_t c_end = exc_off[c + 1];
-  uint64_t e;
-  {
-    uint64_t lo = exc_off[c], hi = c_end;
-    if (lo > hi || hi > ne) {
-      if (lane == 0) report(p.status, WC_ERR_CORRUPT);
-      return;
-    }
-    const uint32_t target = uint32_t(r0 % kChunk);
-    while (lo < hi) {
-      const uint64_t mid = (lo + hi) >> 1;
-      if (exc_pos[mid] < target) lo = mid + 1; else hi = mid;
-    }
-    e = lo;
-  }
-  bool bad = false;
-  auto locate = [&]() -> uint64_t {  // position of exception e (warp-uniform)
-    while (e >= c_end && c + 1 < L.nc) {  // on to the next chunk's list
-      c++;
-      const uint64_t nxt = exc_off[c + 1];
-      if (exc_off[c] != c_end || nxt < c_end || nxt > ne) {
-        bad = true;
-        return ~uint64_t(0);
-      }
-      c_end = nxt;
-    }
-    if (e >= c_end) return ~uint64_t(0);
-    const uint32_t cpos = exc_pos[e];
-    const uint64_t cnt = n - c * kChunk < kChunk ? n - c * kChunk : kChunk;
-    if (cpos >= cnt) {
-      bad = true;
-      return ~uint64_t(0);
-    }
-    return c * kChunk + cpos;
-  };
-  uint64_t next_pos = locate();
-
-  float acc[MT];
-#pragma unroll
-  for (int m = 0; m < MT; m++) acc[m] = 0.0f;
-  // the planes of the next step are loaded while this one is worked on
-  uint2 iw_n = make_uint2(0, 0);
-  uint4 lw_n = make_uint4(0, 0, 0, 0);
-  if (uint32_t(16 * lane) < K) {
-    iw_n = __ldg(reinterpret_cast<const uint2 *>(idx_plane + (r0 + 16 * lane) / 2));
-    lw_n = __ldg(reinterpret_cast<const uint4 *>(lo_plane + r0 + 16 * lane));
-  }
-  for (uint32_t k0 = 0; k0 < K; k0 += 512) {
-    const uint32_t col = k0 + 16 * lane;
-    const bool act = col < K;  // K is a multiple of 64: a lane holds 16 values or none
-    const uint2 iw = iw_n;
-    const uint4 lw = lw_n;
-    if (col + 512 < K) {
-      iw_n = __ldg(reinterpret_cast<const uint2 *>(idx_plane + (r0 + col + 512) / 2));
-      lw_n = __ldg(reinterpret_cast<const uint4 *>(lo_plane + r0 + col + 512));
-    }
-    uint32_t v[8];
-    {
-      const uint2 e0 = wc12::expand4(iw.x, book, lw.x), e1 = wc12::expand4(iw.x >> 16, book, lw.y);
-      const uint2 e2 = wc12::expand4(iw.y, book, lw.z), e3 = wc12::expand4(iw.y >> 16, book, lw.w);
-      v[0] = e0.x; v[1] = e0.y; v[2] = e1.x; v[3] = e1.y; v[4] = e2.x; v[5] = e2.y; v[6] = e3.x; v[7] = e3.y;
-    }
-    // the exceptions among values [r0 + k0, r0 + min(k0 + 512, K))
-    const uint64_t s0 = r0 + k0, s1 = r0 + (k0 + 512 < K ? k0 + 512 : K);
-    while (next_pos < s1) {
-      if (next_pos >= s0) {
-        const uint32_t rel = uint32_t(next_pos - s0);
-        if (lane == int(rel >> 4)) {
-          const uint32_t j = rel & 15u;
-          const uint32_t lo = (j < 4 ? lw.x : j < 8 ? lw.y : j < 12 ? lw.z : lw.w) >> (8 * (j & 3)) & 0xFFu;
-          const uint32_t val = (uint32_t(exc_val[e]) << 8) | lo;
-#pragma unroll
-          for (int q = 0; q < 8; q++)
-            if (int(j >> 1) == q) v[q] = (j & 1u) ? ((v[q] & 0xFFFFu) | (val << 16)) : ((v[q] & 0xFFFF0000u) | val);
-        }
-      }
-      e++;
-      next_pos = locate();
-    }
-    if (bad) {
-      if (lane == 0) report(p.status, WC_ERR_CORRUPT);
-      return;
-    }
-    if (act) {
-#pragma unroll
-      for (int m = 0; m < MT; m++) {
-        const uint4 *xp = reinterpret_cast<const uint4 *>(p.x + uint64_t(m) * K + col);
-        const uint4 xa = __ldg(xp), xb = __ldg(xp + 1);
-        const uint32_t xw[8] = {xa.x, xa.y, xa.z, xa.w, xb.x, xb.y, xb.z, xb.w};
-        float a = acc[m];
-#pragma unroll
-        for (int q = 0; q < 8; q++) {
-          a = fmaf(__uint_as_float(v[q] << 16), __uint_as_float(xw[q] << 16), a);
-          a = fmaf(__uint_as_float(v[q] & 0xFFFF0000u), __uint_as_float(xw[q] & 0xFFFF0000u), a);
-        }
-        acc[m] = a;
-      }
-    }
-  }
-#pragma unroll
-  for (int m = 0; m < MT; m++) {
-    float a = acc[m];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-    if (lane == 0) p.y[uint64_t(m) * N + row] = a;
-  }
-}
-
-template <int MT>
-cudaError_t launch_gemv(const Params &p, cudaStream_t s) {
-  k12_gemv<MT><<<(p.N + kGemvWarps - 1) / kGemvWarps, kGemvWarps * 32, 0, s>>>(p);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_gemv_m(const Params &p, cudaStream_t s) {
-  switch (p.M) {
-    case 1: return launch_gemv<1>(p, s);
-    case 2: return launch_gemv<2>(p, s);
-    case 3: return launch_gemv<3>(p, s);
-    case 4: return launch_gemv<4>(p, s);
-    case 5: return launch_gemv<5>(p, s);
-    case 6: return launch_gemv<6>(p, s);
-    case 7: return launch_gemv<7>(p, s);
-    default: return launch_gemv<8>(p, s);
-  }
-}
-
 __global__ void k12_zero(float *y, uint64_t count) {
   for (uint64_t i = uint64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < count;
        i += uint64_t(gridDim.x) * blockDim.x)
@@ -886,6 +713,11 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   if (N == 0 || K == 0 || N % wc12l::kBM != 0 || K % wc12l::kBK != 0 || M == 0)
     return WC_ERR_INVALID_ARG;
   if (w_bytes < 96) return WC_ERR_INVALID_ARG;  // shorter than any container's header
+  // the index and low planes of an N x K container must lie inside the
+  // buffer (their offsets depend on N K only; the kernels check the header)
+  const uint64_t n = uint64_t(N) * K;
+  const wc12::Lay L = wc12::lay(n, 0);
+  if (w_bytes < L.off_lo + n) return WC_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   wc12l::Params p;
   p.w = static_cast<const uint8_t *>(d_w);
@@ -893,23 +725,10 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   p.N = N;
   p.K = K;
   p.status = d_status;
-  if (M <= wc12l::kGemvMaxM) {  // reading W bounds it: CUDA cores, no tensor memory
-    p.x = static_cast<const uint16_t *>(d_x);
-    p.y = d_y;
-    p.M = M;
-    p.n_mma = 0;
-    p.per_split = p.splits = 1;
-    return wc12l::launch_gemv_m(p, s) == cudaSuccess ? WC_OK : WC_ERR_CUDA;
-  }
   const wc12l::DevInfo di = wc12l::dev_info();
   if (di.sms <= 0 || !di.attr) return WC_ERR_CUDA;
   const uint32_t blocks = N / wc12l::kBM, stages = K / wc12l::kBK;
   if (blocks == 0) return WC_ERR_INVALID_ARG;
-  // the planes the tensor maps cover must lie inside the buffer (their
-  // offsets depend on N K only; the kernel checks the header itself)
-  const uint64_t n = uint64_t(N) * K;
-  const wc12::Lay L = wc12::lay(n, 0);
-  if (w_bytes < L.off_lo + n) return WC_ERR_INVALID_ARG;
   if (!wc12l::make_map(&p.tm_idx, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w + L.off_idx, K / 2, N, K / 2, 32,
                        wc12l::kBM, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
       !wc12l::make_map(&p.tm_lo, CU_TENSOR_MAP_DATA_TYPE_UINT8, p.w + L.off_lo, K, N, K, 64, wc12l::kBM,
@@ -923,8 +742,8 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
     p.y = d_y + uint64_t(t0) * N;
     p.M = m;
     p.n_mma = (m + 15) / 16 * 16;
-    if (!wc12l::make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, K, m, uint64_t(K) * 2, 8, p.n_mma,
-                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+    if (!wc12l::make_map(&p.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, K, m, uint64_t(K) * 2, wc12l::kBK, p.n_mma,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
       return WC_ERR_CUDA;
     // split K so that the grid is one wave of the CTAs an SM holds, with at
     // least 4 stages a CTA when K allows (the load ring runs 4 ahead)

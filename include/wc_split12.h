@@ -79,19 +79,21 @@ WC_API int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out,
 
 /* Y = X W^T with W (N x K bf16, row-major) given as a Split12 container, the
  * weights crossing HBM at 12 bits a value ("weight-compression" README:
- * serving with the weights kept in this format).  For M <= 8 tokens the
- * layer is bound by reading W and runs on the CUDA cores, a warp per weight
- * row expanding the values in registers; for more tokens the weights are
- * expanded tile by tile into the tensor cores' operand layout and multiplied
- * with tcgen05.mma.  Both accumulate exact bf16 products in fp32.
- *   d_w, w_bytes  the container (16-byte aligned, at least 96 bytes), n = N * K
+ * serving with the weights kept in this format).  The weights' planes and X
+ * come in by TMA; the weights are expanded tile by tile into the tensor
+ * cores' operand layout and multiplied with tcgen05.mma, exact bf16 products
+ * accumulated in fp32.
+ *   d_w, w_bytes  the container (16-byte aligned, at least 96 bytes, and at
+ *                 least up to the end of the low plane an N x K container
+ *                 has), n = N * K
  *   N, K          N a multiple of 128, K a multiple of 64
- *   d_x           M x K bf16, row-major, 16-byte aligned; M >= 1 (more than 8
- *                 are taken in slices of 256 tokens, one launch each)
+ *   d_x           M x K bf16, row-major, 16-byte aligned; M >= 1 (taken in
+ *                 slices of 256 tokens, one launch each)
  *   d_y           M x N fp32, row-major (overwritten)
  *   d_status      device i32 set to 0 by the caller: WC_ERR_CORRUPT for a bad
  *                 container, WC_ERR_TIMEOUT if a bounded wait ran out
- * Returns WC_OK, WC_ERR_INVALID_ARG or WC_ERR_CUDA. */
+ * Returns WC_OK, WC_ERR_INVALID_ARG or WC_ERR_CUDA (also when the driver
+ * cannot describe the planes to TMA). */
 WC_API int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, uint32_t K,
                            const void *d_x, uint32_t M, float *d_y, int32_t *d_status,
                            void *stream);

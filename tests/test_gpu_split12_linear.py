@@ -2,9 +2,8 @@
 Y = X W^T with W held as a Split12 container ("weight-compression" README:
 bf16 weights rebuilt from a codebook index and the raw low byte inside the
 serving kernels), against the oracle's float64 sum of the exact bf16
-products (oracle/split12.py linear).  M <= 8 runs on the CUDA cores (one
-warp per weight row), larger M on the tensor cores (tcgen05); both are
-covered.
+products (oracle/split12.py linear): TMA loads, the weights expanded into
+the tensor cores' operand layout, tcgen05 MMAs.
 
 Tolerance, from the arithmetic: every product of two bf16 values is exact in
 fp32, so an output is a sum of K exact terms; the tensor cores and the split-K
@@ -86,7 +85,7 @@ def test_one_small_shape_first(s12):
 
 
 @pytest.mark.parametrize("N,K", [(128, 64), (256, 128), (128, 4096), (256, 4096)])
-@pytest.mark.parametrize("M", [1, 3, 8, 9, 17, 144, 256, 300])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 144, 256, 300])
 def test_shapes(s12, N, K, M):
     _check(s12, N, K, M, seed=N + K + M)
 
@@ -96,7 +95,7 @@ def test_exceptions_in_the_tile(s12, K):
     """Outliers become exceptions: a few per tile (gathered into the CTA's
     list) and, at 20 %, more than the list holds (walked per stage)."""
     for frac in (0.002, 0.2):
-        for M in (4, 33):  # the CUDA-core path (M <= 8) and the tensor-core path
+        for M in (1, 4, 33):
             ne = _check(s12, 256, K, M, seed=K + int(frac * 1000) + M, outliers=frac)
             assert ne > 0
 
@@ -105,7 +104,7 @@ def test_corrupt_header_is_reported(s12):
     from fp32_weight_compression_b200 import wc
     N, K = 128, 128
     cont = s12.encode(_weights(N, K, 3))
-    for M in (1, 17):  # both paths
+    for M in (1, 17):
         x = _bf16_dev(workloads.rne_bf16(np.ones(M * K, np.float32))).view(M, K)
         for off, val in ((0, 0x00), (8, 0x01), (16, 0x00)):   # magic, n, chunk size
             bad = cont.copy()
@@ -116,3 +115,17 @@ def test_corrupt_header_is_reported(s12):
         # the intact container still works after the refusals
         y = wc.split12_linear(torch.from_numpy(cont).to("cuda"), N, K, x)
         assert torch.isfinite(y).all()
+
+
+def test_short_buffer_is_refused(s12):
+    """A buffer that cannot hold the index and low planes of an N x K
+    container is refused before any launch."""
+    from fp32_weight_compression_b200 import wc
+    N, K = 128, 256
+    cont = s12.encode(_weights(N, K, 5))
+    short = torch.from_numpy(cont[:N * K]).to("cuda")  # header + index plane, not all low bytes
+    for M in (1, 2, 40):
+        x = _bf16_dev(workloads.rne_bf16(np.ones(M * K, np.float32))).view(M, K)
+        with pytest.raises(wc.WCError) as ei:
+            wc.split12_linear(short, N, K, x)
+        assert ei.value.code == wc.ERR_INVALID_ARG
