@@ -80,6 +80,9 @@ def parse(argv=None):
                     help="skip the Split12 serving-format leg (wc12_encode / wc12_decode on the "
                          "headline tensors and wc12_linear against cuBLAS bf16, timed after the "
                          "step; the 'split12' object)")
+    ap.add_argument("--linear-only", action="store_true",
+                    help="profiling only: draw the set's first four gate projections and run the "
+                         "wc12_linear leg alone (one JSON line with its 'linear' object)")
     ap.add_argument("--no-checksum", dest="checksum", action="store_false",
                     help="skip the block-checksum leg (wc_crc32_blocks, 1 MiB blocks, over the "
                          "container arena, timed after the step; the 'checksum' object)")
@@ -294,6 +297,16 @@ DECODE_SOURCES = ["fp32_weight_compression_b200/csrc/k_decode.cu",
                   "fp32_weight_compression_b200/csrc/wc_planes.cuh"]
 
 
+ENCODE_SOURCES = ["fp32_weight_compression_b200/csrc/k_hist.cu",
+                  "fp32_weight_compression_b200/csrc/k_encode.cu",
+                  "fp32_weight_compression_b200/csrc/k_compact.cu",
+                  "fp32_weight_compression_b200/csrc/wc_hist.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_coder.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_format.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_block.cuh",
+                  "fp32_weight_compression_b200/csrc/wc_planes.cuh"]
+
+
 def kernel_sources_sha(files) -> str:
     h = hashlib.sha256()
     for f in files:
@@ -301,7 +314,8 @@ def kernel_sources_sha(files) -> str:
     return h.hexdigest()
 
 
-def recorded_traffic(kernel: str, workload: int, src_files, values: int) -> float | None:
+def recorded_traffic(kernel: str, workload: int, src_files, values: int,
+                     key: str = "traffic_bytes_per_value") -> float | None:
     """DRAM bytes per launch of `kernel` on the given set, from the ncu
     summary in profiles/ (bytes per value there, times this launch's values),
     valid only while the kernel's sources are unchanged."""
@@ -312,7 +326,7 @@ def recorded_traffic(kernel: str, workload: int, src_files, values: int) -> floa
     for line in open(path):
         if line.startswith("source_sha256:"):
             want = line.split(":", 1)[1].strip()
-        if line.startswith("traffic_bytes_per_value:"):
+        if line.startswith(key + ":"):
             per_value = float(line.split(":", 1)[1].strip())
     if per_value is None or want != kernel_sources_sha(src_files):
         return None
@@ -672,6 +686,21 @@ def checksum_leg(arena, dev, stream, reps: int = 10):
 
 
 # ---------------------------------------------------------------------------
+def linear_only(cid: int, local: int):
+    """The wc12_linear leg on its own (profiling): the set's first four gate
+    projections drawn, moved to the device, timed against cuBLAS."""
+    import torch
+    specs = workloads.tensor_specs(cid)
+    pick = [i for i, s in enumerate(specs) if s.name.endswith(".gate")][:4]
+    host, offs, nbytes, numels, dts = generate_pinned(None, cid, pick)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ins = [host[o:o + b].to(dev).view(dt) for o, b, dt in zip(offs, nbytes, dts)]
+    torch.cuda.synchronize(dev)
+    res = linear_leg(ins, [specs[i] for i in pick], dev)
+    print(json.dumps({"workload": WORKLOAD_NAMES[cid], "linear": res}))
+
+
 def main(argv=None):
     args = parse(argv)
     rank = int(os.environ.get("RANK", "0"))
@@ -683,6 +712,9 @@ def main(argv=None):
         return
 
     cid = args.workload
+    if args.linear_only:
+        linear_only(cid, local)
+        return
     extra = [] if args.extra in ("", "none") else [int(x) for x in args.extra.split(",")]
     extra = [c for c in extra if c != cid]
 
@@ -765,6 +797,13 @@ def main(argv=None):
     pool.close()
 
     traffic = recorded_traffic("k_decode", cid, DECODE_SOURCES, values_mine) if world == 1 else None
+    enc_traffic = (recorded_traffic("k_coder", cid, ENCODE_SOURCES, values_mine, "encode_traffic_bytes_per_value")
+                   if world == 1 else None)
+    # DRAM bytes of the four encode launches per step, from the recorded ncu
+    # capture (null once a kernel source changed): against the algorithmic bytes
+    r["encode"]["traffic"] = enc_traffic
+    r["encode"]["traffic_over_algorithmic"] = (enc_traffic / (total_in + total_cont)
+                                               if enc_traffic else None)
     dec_achieved = r["decode"]["hbm_gbs"]
     line = {
         "metric": METRIC,
