@@ -49,6 +49,7 @@
 #include <cudaTypedefs.h>
 
 #include "wc.h"
+#include "wc12_plan.cuh"
 #include "wc_split12.cuh"
 
 namespace wc12l {
@@ -83,6 +84,8 @@ struct Params {
   CUtensorMap tm_idx, tm_lo, tm_x;
   const uint8_t *w;
   uint64_t w_bytes;
+  const uint8_t *plan;  // the container's serving plan (wc12_plan.cuh), or null
+  uint64_t plan_bytes;
   const uint16_t *x;  // [M, K]
   float *y;           // [M, N]
   uint32_t M, N, K;
@@ -288,6 +291,13 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
     ok = h32[5] == uint32_t(L.nc) && h64[4] == L.off_idx && h64[5] == L.off_lo && h64[6] == L.off_exc &&
          h64[7] == L.total && L.total <= p.w_bytes;
   }
+  if (ok && p.plan != nullptr) {  // a plan built from this container for this N x K
+    const uint32_t *q32 = reinterpret_cast<const uint32_t *>(p.plan);
+    const uint64_t *q64 = reinterpret_cast<const uint64_t *>(p.plan);
+    const wc12p::PlanLay P = wc12p::plan_lay(N, K, ne);
+    ok = q32[0] == wc12p::kMagic && q32[1] == 1 && q32[2] == N && q32[3] == K && q64[2] == ne &&
+         q64[3] == P.buckets && P.total <= p.plan_bytes;
+  }
   if (!ok || s_begin >= s_end) {
     if (!ok && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) report(p.status, WC_ERR_CORRUPT);
     return;
@@ -346,13 +356,49 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
   if (loader)
     for (; loaded < kDepth && loaded < nst; loaded++) load_stage(loaded);
 
+  // The CTA's exceptions and how they are patched (mode): 0 from a shared
+  // list binned by stage (bin[] relative starts), 1 from the plan's entries
+  // read at each stage (bin[] absolute starts, or the plan's own when the
+  // CTA has more stages than bin[] holds), 2 by walking the chunks' lists at
+  // each stage, 3 not at all (a corrupt plan, reported).
+  const bool binned = nst <= kMaxStagesPerCta;
+  uint32_t mode = 0;
+  const uint32_t *plan_start = nullptr, *plan_ent = nullptr;
+  if (p.plan != nullptr) {
+    // The plan holds the tile's exceptions as one range, by stage: its
+    // starts, then (up to kExcCap) its entries, into shared memory.
+    const wc12p::PlanLay P = wc12p::plan_lay(N, K, ne);
+    plan_start = reinterpret_cast<const uint32_t *>(p.plan + wc12p::kStartOff) +
+                 uint64_t(blockIdx.x) * (K / kBK) + s_begin;
+    plan_ent = reinterpret_cast<const uint32_t *>(p.plan + P.off_ent);
+    mode = 1;
+    if (binned) {
+      for (uint32_t i = tid; i <= nst; i += kThreads) bin[i] = plan_start[i];
+      __syncthreads();
+      bool bad = false;
+      for (uint32_t i = tid; i < nst; i += kThreads) bad |= bin[i] > bin[i + 1] || bin[i + 1] > ne;
+      if (__syncthreads_or(bad)) {
+        if (tid == 0) report(p.status, WC_ERR_CORRUPT);
+        mode = 3;
+      } else if (bin[nst] - bin[0] <= kExcCap) {
+        const uint32_t base = bin[0], total = bin[nst] - base;
+        for (uint32_t i = tid; i < total; i += kThreads) {
+          const uint32_t e = plan_ent[base + i];
+          exc_bin[i] = make_uint2(e & 63u, ((e >> 6) & 127u) | (((e >> 16) & 255u) << 16));
+        }
+        __syncthreads();  // every thread has read bin[0]
+        for (uint32_t i = tid; i <= nst; i += kThreads) bin[i] -= base;
+        __syncthreads();
+        mode = 0;
+      }
+    }
+  } else {
   // The CTA's exceptions, once: positions within a chunk become (row, column)
   // relative to the CTA's tile with 32-bit arithmetic when 128 K fits it,
   // counted per stage, then binned by stage so that each stage's are found
   // without a search and patched by the thread that expanded their segment.
   const uint64_t f_base = uint64_t(n0) * K, f_span = uint64_t(kBM) * K;
   const uint32_t k_beg = s_begin * kBK, k_end = s_end * kBK;
-  const bool binned = nst <= kMaxStagesPerCta;
   // The chunks' lists follow one another in the container, so the row
   // block's exceptions are the one range [exc_off[c_lo], exc_off[c_hi + 1]);
   // its entries are taken by all threads at once, each finding its chunk by
@@ -425,8 +471,8 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
   }
   __syncthreads();
   const uint32_t n_exc = *exc_n;
-  const bool exc_walk = n_exc > kExcCap || !binned;
-  if (!exc_walk) {
+  mode = n_exc > kExcCap || !binned ? 2 : 0;
+  if (mode == 0) {
     // counts -> starts (one warp), then scatter by stage
     if (warp == 0) {
       uint32_t run = 0;
@@ -447,10 +493,11 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
     for (uint32_t i = tid; i <= nst; i += kThreads) cur[i] = bin[i];
     __syncthreads();
     for (uint32_t i = tid; i < n_exc; i += kThreads) {
-      const uint2 ex = exc_raw[i];
-      exc_bin[atomicAdd(&cur[ex.x / kBK], 1u)] = ex;
+      const uint2 ex = exc_raw[i];  // column in the CTA's range -> in its stage
+      exc_bin[atomicAdd(&cur[ex.x / kBK], 1u)] = make_uint2(ex.x % kBK, ex.y);
     }
     __syncthreads();
+  }
   }
 
   // The pipeline.  Expanding threads, stage s: wait for slot s % kDepth's
@@ -481,7 +528,18 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
       const bool okw = mbar_wait_or_flag(&full[s % kDepth], (s / kDepth) & 1u, vflag) &&
                        (s < kASlots || mbar_wait_or_flag(&a_free[as], ((s / kASlots) & 1u) ^ 1u, vflag));
       const uint32_t k0 = (s_begin + s) * kBK;
-      const uint32_t eb0 = exc_walk ? 0u : bin[s], eb1 = exc_walk ? 0u : bin[s + 1];
+      uint32_t eb0 = 0, eb1 = 0;  // the stage's exceptions (modes 0, 1)
+      if (mode == 0 || (mode == 1 && binned)) {
+        eb0 = bin[s];
+        eb1 = bin[s + 1];
+      } else if (mode == 1) {
+        eb0 = plan_start[s];
+        eb1 = plan_start[s + 1];
+      }
+      // mode 1: this thread's first entry of the stage, loaded before the
+      // expansion hides its latency
+      uint32_t first_e = 0;
+      if (mode == 1 && eb0 <= eb1 && eb1 <= ne && eb0 + uint32_t(tid) < eb1) first_e = plan_ent[eb0 + tid];
       if (okw) {
         // A: 512 segments of 16 values, two per thread: segment i is row
         // 8 (i / 32) + i % 8, values 16 ((i / 8) % 4) .., expanded from the
@@ -505,12 +563,21 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
       }
       // the exceptions that fall in this tile get their high bytes, one
       // thread an exception
-      if (!exc_walk) {
+      if (mode == 0) {
         for (uint32_t i = eb0 + uint32_t(tid); i < eb1; i += kExpThreads) {
           const uint2 ex = exc_bin[i];
-          A[op_offset(ex.y & 0xFFFFu, ex.x - s * kBK, kASlice) + 1] = uint8_t(ex.y >> 16);
+          A[op_offset(ex.y & 0xFFFFu, ex.x, kASlice) + 1] = uint8_t(ex.y >> 16);
         }
-      } else {
+      } else if (mode == 1) {
+        if (eb0 > eb1 || eb1 > ne) {
+          if (tid == 0) report(p.status, WC_ERR_CORRUPT);
+        } else {
+          for (uint32_t i = eb0 + uint32_t(tid); i < eb1; i += kExpThreads) {
+            const uint32_t e = i == eb0 + uint32_t(tid) ? first_e : plan_ent[i];
+            A[op_offset((e >> 6) & 127u, e & 63u, kASlice) + 1] = uint8_t(e >> 16);
+          }
+        }
+      } else if (mode == 2) {
         for (uint64_t c = c_lo; c <= c_hi; c++) {
           const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
           if (e0 > e1 || e1 > ne) continue;  // reported by the gathering pass
@@ -703,9 +770,10 @@ DevInfo dev_info() {
 
 }  // namespace wc12l
 
-extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, uint32_t K,
-                               const void *d_x, uint32_t M, float *d_y, int32_t *d_status,
-                               void *stream) {
+namespace wc12l {
+
+int32_t linear(const void *d_w, uint64_t w_bytes, const void *d_plan, uint64_t plan_bytes, uint32_t N,
+               uint32_t K, const void *d_x, uint32_t M, float *d_y, int32_t *d_status, void *stream) {
   auto aligned = [](const void *q, uintptr_t a) { return (reinterpret_cast<uintptr_t>(q) & (a - 1)) == 0; };
   if (d_w == nullptr || d_x == nullptr || d_y == nullptr || d_status == nullptr) return WC_ERR_INVALID_ARG;
   if (!aligned(d_w, 16) || !aligned(d_x, 16) || !aligned(d_y, 4) || !aligned(d_status, 4))
@@ -718,10 +786,15 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   const uint64_t n = uint64_t(N) * K;
   const wc12::Lay L = wc12::lay(n, 0);
   if (w_bytes < L.off_lo + n) return WC_ERR_INVALID_ARG;
+  if (d_plan != nullptr &&
+      (!aligned(d_plan, 16) || plan_bytes < wc12p::plan_lay(N, K, 0).off_ent))  // header and starts
+    return WC_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   wc12l::Params p;
   p.w = static_cast<const uint8_t *>(d_w);
   p.w_bytes = w_bytes;
+  p.plan = static_cast<const uint8_t *>(d_plan);
+  p.plan_bytes = plan_bytes;
   p.N = N;
   p.K = K;
   p.status = d_status;
@@ -773,3 +846,19 @@ extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, ui
   }
   return WC_OK;
 }
+
+}  // namespace wc12l
+
+extern "C" int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, uint32_t K,
+                               const void *d_x, uint32_t M, float *d_y, int32_t *d_status,
+                               void *stream) {
+  return wc12l::linear(d_w, w_bytes, nullptr, 0, N, K, d_x, M, d_y, d_status, stream);
+}
+
+extern "C" int32_t wc12_linear_planned(const void *d_w, uint64_t w_bytes, const void *d_plan,
+                                       uint64_t plan_bytes, uint32_t N, uint32_t K, const void *d_x,
+                                       uint32_t M, float *d_y, int32_t *d_status, void *stream) {
+  if (d_plan == nullptr) return WC_ERR_INVALID_ARG;
+  return wc12l::linear(d_w, w_bytes, d_plan, plan_bytes, N, K, d_x, M, d_y, d_status, stream);
+}
+

@@ -124,6 +124,12 @@ def load() -> ctypes.CDLL:
     L.wc12_read_header.argtypes = [vp, u64, ctypes.POINTER(u64), ctypes.POINTER(u64), ctypes.POINTER(u32)]
     L.wc12_linear.restype = i32
     L.wc12_linear.argtypes = [vp, u64, u32, u32, vp, u32, vp, vp, vp]
+    L.wc12_plan_bytes.restype = u64
+    L.wc12_plan_bytes.argtypes = [u32, u32, u64]
+    L.wc12_plan.restype = i32
+    L.wc12_plan.argtypes = [vp, u64, u32, u32, u64, vp, u64, vp, vp]
+    L.wc12_linear_planned.restype = i32
+    L.wc12_linear_planned.argtypes = [vp, u64, vp, u64, u32, u32, vp, u32, vp, vp, vp]
     L.wc_crc32_blocks.restype = i32
     L.wc_crc32_blocks.argtypes = [vp, u64, u64, vp, vp]
     L.wc_check_coder_division.restype = i32
@@ -470,16 +476,42 @@ def split12_decode(cont: torch.Tensor, shape=None, out=None, stream=None) -> tor
     return out
 
 
-def split12_linear(cont: torch.Tensor, N: int, K: int, x: torch.Tensor, stream=None) -> torch.Tensor:
+def split12_plan_bytes(N: int, K: int, ne: int) -> int:
+    return int(load().wc12_plan_bytes(N, K, ne))
+
+
+def split12_plan(cont: torch.Tensor, N: int, K: int, stream=None) -> torch.Tensor:
+    """The serving plan of a Split12 container on the device (wc12_plan): its
+    exceptions grouped by the linear layer's 128 x 64 tiles.  Reads the
+    container's header to the host once, for its exception count."""
+    _n, ne, _k = split12_read_header(cont[:64].cpu().numpy(), cont.numel())
+    plan = torch.empty(split12_plan_bytes(N, K, ne), dtype=torch.uint8, device=cont.device)
+    status = torch.zeros(1, dtype=torch.int32, device=cont.device)
+    _check(load().wc12_plan(cont.data_ptr(), cont.numel(), N, K, ne, plan.data_ptr(), plan.numel(),
+                            status.data_ptr(), _stream(stream)), "wc12_plan")
+    st = int(status.item())
+    if st != OK:
+        raise WCError(st, "wc12_plan (device status)")
+    return plan
+
+
+def split12_linear(cont: torch.Tensor, N: int, K: int, x: torch.Tensor, plan=None,
+                   stream=None) -> torch.Tensor:
     """Y = x W^T (fp32, M x N) with W (N x K bf16) given as a Split12
-    container on the device (wc12_linear)."""
+    container on the device (wc12_linear, or wc12_linear_planned with the
+    container's plan)."""
     if x.dtype != torch.bfloat16 or x.dim() != 2 or x.shape[1] != K:
         raise ValueError("x must be a 2-D bf16 tensor with K columns")
     xf = x.contiguous()
     y = torch.empty(x.shape[0], N, dtype=torch.float32, device=x.device)
     status = torch.zeros(1, dtype=torch.int32, device=x.device)
-    _check(load().wc12_linear(cont.data_ptr(), cont.numel(), N, K, xf.data_ptr(), x.shape[0],
-                              y.data_ptr(), status.data_ptr(), _stream(stream)), "wc12_linear")
+    if plan is None:
+        _check(load().wc12_linear(cont.data_ptr(), cont.numel(), N, K, xf.data_ptr(), x.shape[0],
+                                  y.data_ptr(), status.data_ptr(), _stream(stream)), "wc12_linear")
+    else:
+        _check(load().wc12_linear_planned(cont.data_ptr(), cont.numel(), plan.data_ptr(), plan.numel(), N, K,
+                                          xf.data_ptr(), x.shape[0], y.data_ptr(), status.data_ptr(),
+                                          _stream(stream)), "wc12_linear_planned")
     st = int(status.item())
     if st != OK:
         raise WCError(st, "wc12_linear (device status)")

@@ -98,6 +98,41 @@ WC_API int32_t wc12_linear(const void *d_w, uint64_t w_bytes, uint32_t N, uint32
                            const void *d_x, uint32_t M, float *d_y, int32_t *d_status,
                            void *stream);
 
+/* The serving plan of a container for wc12_linear_planned: the container's
+ * exceptions grouped by the tiles the layer works in (128 weight rows x 64
+ * values of K), so that each tile finds its exceptions as one range instead
+ * of searching the container's per-chunk lists at every call.  Built once
+ * per weight matrix; it depends on the container and on N, K only.
+ * Layout (little-endian): u32 "W12P", u32 version 1, u32 N, u32 K, u64 ne,
+ * u64 buckets = N/128 * K/64; u32 start[buckets + 1] (bucket b * (K/64) + s
+ * holds the exceptions of row block b, stage s); then, 16-byte aligned,
+ * u32 entry[ne]: column in the stage (bits 0-5), row in the block (bits
+ * 6-12), the exception's high byte (bits 16-23), in any order within a
+ * bucket. */
+WC_API uint64_t wc12_plan_bytes(uint32_t N, uint32_t K, uint64_t ne);
+
+/* Build the plan of container d_w (w_bytes, 16-byte aligned; N x K weights,
+ * N a multiple of 128, K of 64; ne its exception count, from
+ * wc12_read_header) into d_plan (plan_bytes >= wc12_plan_bytes(N, K, ne),
+ * 16-byte aligned).  *d_status (device i32 set to 0 by the caller) receives
+ * WC_ERR_CORRUPT if the container's header disagrees with N, K, ne or its
+ * exception lists are corrupt; the plan is then marked invalid (its magic
+ * is 0) and wc12_linear_planned refuses it.  Four launches on the stream.
+ * Returns WC_OK, WC_ERR_INVALID_ARG, WC_ERR_CAPACITY (plan_bytes too small)
+ * or WC_ERR_CUDA. */
+WC_API int32_t wc12_plan(const void *d_w, uint64_t w_bytes, uint32_t N, uint32_t K, uint64_t ne,
+                         void *d_plan, uint64_t plan_bytes, int32_t *d_status, void *stream);
+
+/* wc12_linear with the container's plan (d_plan, plan_bytes; built by
+ * wc12_plan for this container and N x K): the same result, without the
+ * per-call search for each tile's exceptions.  A plan whose header does not
+ * match the container (N, K, ne) is reported as WC_ERR_CORRUPT, as are
+ * start offsets out of order.  Returns WC_OK, WC_ERR_INVALID_ARG (also for
+ * a null plan or plan_bytes below its header and starts) or WC_ERR_CUDA. */
+WC_API int32_t wc12_linear_planned(const void *d_w, uint64_t w_bytes, const void *d_plan,
+                                   uint64_t plan_bytes, uint32_t N, uint32_t K, const void *d_x,
+                                   uint32_t M, float *d_y, int32_t *d_status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -26,7 +26,7 @@ def declared_entry_points():
     for fn in sorted(os.listdir(os.path.join(ROOT, "include"))):
         if fn.endswith(".h"):
             text = open(os.path.join(ROOT, "include", fn)).read()
-            names += re.findall(r"WC_API\s+[\w\s\*]*?\b(wc_\w+)\s*\(", text)
+            names += re.findall(r"WC_API\s+[\w\s\*]*?\b(wc(?:12)?_\w+)\s*\(", text)
     return names
 
 
@@ -266,6 +266,37 @@ def test_split12_linear_bad_arguments_rejected_without_device(wcm):
     assert call(w=None) == wcm.ERR_INVALID_ARG
     assert call(st=None) == wcm.ERR_INVALID_ARG
     assert L.wc12_linear(b, 95, 256, 128, b, 4, b, b, None) == wcm.ERR_INVALID_ARG   # no room for a header
+
+
+def test_split12_plan_size_and_bad_arguments(wcm):
+    """wc12_plan_bytes from its layout; wc12_plan and wc12_linear_planned
+    refuse bad arguments before touching a device."""
+    L = wcm.load()
+    for N, K, ne in ((128, 64, 0), (128, 64, 5), (4096, 14336, 22572), (256, 128, 1000)):
+        nb = (N // 128) * (K // 64)
+        off_ent = (32 + 4 * (nb + 1) + 15) // 16 * 16
+        assert wcm.split12_plan_bytes(N, K, ne) == (off_ent + 4 * ne + 15) // 16 * 16
+    buf = (ctypes.c_uint8 * 8192)()
+    b = (ctypes.addressof(buf) + 255) // 256 * 256
+    N, K = 128, 64
+    pb = wcm.split12_plan_bytes(N, K, 3)
+    big = 1 << 20
+    assert L.wc12_plan(b + 8, big, N, K, 3, b, pb, b, None) == wcm.ERR_INVALID_ARG   # container alignment
+    assert L.wc12_plan(b, big, N, K, 3, b + 8, pb, b, None) == wcm.ERR_INVALID_ARG   # plan alignment
+    assert L.wc12_plan(b, big, 100, K, 3, b, pb, b, None) == wcm.ERR_INVALID_ARG     # N
+    assert L.wc12_plan(b, big, N, 96, 3, b, pb, b, None) == wcm.ERR_INVALID_ARG      # K
+    assert L.wc12_plan(b, big, N, K, N * K + 1, b, big, b, None) == wcm.ERR_INVALID_ARG  # ne > n
+    assert L.wc12_plan(b, 100, N, K, 3, b, pb, b, None) == wcm.ERR_INVALID_ARG      # container too short
+    assert L.wc12_plan(b, big, N, K, 3, b, pb - 16, b, None) == wcm.ERR_CAPACITY    # plan too short
+    assert L.wc12_plan(b, big, N, K, 3, None, pb, b, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_plan(b, big, N, K, 3, b, pb, None, None) == wcm.ERR_INVALID_ARG
+    def planned(plan=b, plan_bytes=pb, N=256, K=128, M=4):
+        return L.wc12_linear_planned(b, big, plan, plan_bytes, N, K, b, M, b, b, None)
+    assert planned(plan=None) == wcm.ERR_INVALID_ARG
+    assert planned(plan=b + 8) == wcm.ERR_INVALID_ARG
+    assert planned(plan_bytes=40) == wcm.ERR_INVALID_ARG        # below the header and starts
+    assert planned(N=100) == wcm.ERR_INVALID_ARG
+    assert planned(M=0) == wcm.ERR_INVALID_ARG
 
 
 def test_split12_read_header_matches_the_oracle(wcm):

@@ -129,3 +129,127 @@ def test_short_buffer_is_refused(s12):
         with pytest.raises(wc.WCError) as ei:
             wc.split12_linear(short, N, K, x)
         assert ei.value.code == wc.ERR_INVALID_ARG
+
+
+def _plan_from_oracle(s12, cont, N, K):
+    """The serving plan's starts and (per bucket, sorted) entries, built from
+    the container's exception lists in numpy: the definition the GPU plan
+    must meet (its order within a bucket is free)."""
+    h = s12.read_header(cont)
+    lay = s12.layout(h["n"], h["ne"])
+    nc = lay["nc"]
+    exc_off = np.frombuffer(cont[80:80 + 8 * (nc + 1)].tobytes(), np.uint64).astype(np.int64)
+    pos = np.frombuffer(cont[lay["off_exc"]:lay["off_exc"] + 2 * h["ne"]].tobytes(), np.uint16).astype(np.int64)
+    hi = cont[lay["off_excval"]:lay["off_excval"] + h["ne"]].astype(np.int64)
+    chunk = np.repeat(np.arange(nc), np.diff(exc_off))
+    f = chunk * 65536 + pos
+    row, col = f // K, f % K
+    S = K // 64
+    bucket = (row // 128) * S + col // 64
+    entry = (col % 64) | ((row % 128) << 6) | (hi << 16)
+    nb = (N // 128) * S
+    counts = np.bincount(bucket, minlength=nb)
+    starts = np.concatenate([[0], np.cumsum(counts)])
+    per = [np.sort(entry[bucket == b]) for b in range(nb)]
+    return h["ne"], starts, per
+
+
+@pytest.mark.parametrize("N,K,outliers", [(128, 64, 0.0), (256, 4096, 0.002), (384, 1024, 0.2)])
+def test_plan_matches_its_definition(s12, N, K, outliers):
+    from fp32_weight_compression_b200 import wc
+    cont = s12.encode(_weights(N, K, 21, outliers))
+    ne, starts, per = _plan_from_oracle(s12, cont, N, K)
+    plan = wc.split12_plan(torch.from_numpy(cont).to("cuda"), N, K).cpu().numpy()
+    assert plan.size == wc.split12_plan_bytes(N, K, ne)
+    h = np.frombuffer(plan[:32].tobytes(), np.uint32)
+    assert tuple(h[:4]) == (0x50323157, 1, N, K)
+    nb = (N // 128) * (K // 64)
+    assert tuple(np.frombuffer(plan[16:32].tobytes(), np.uint64)) == (ne, nb)
+    got_starts = np.frombuffer(plan[32:32 + 4 * (nb + 1)].tobytes(), np.uint32).astype(np.int64)
+    assert np.array_equal(got_starts, starts)
+    off_ent = (32 + 4 * (nb + 1) + 15) // 16 * 16
+    ent = np.frombuffer(plan[off_ent:off_ent + 4 * ne].tobytes(), np.uint32).astype(np.int64)
+    for b in range(nb):
+        assert np.array_equal(np.sort(ent[starts[b]:starts[b + 1]]), per[b]), b
+
+
+@pytest.mark.parametrize("N,K", [(128, 64), (256, 128), (128, 4096), (256, 4096)])
+@pytest.mark.parametrize("M", [1, 2, 16, 17, 256, 300])
+def test_planned_shapes(s12, N, K, M):
+    _check_planned(s12, N, K, M, seed=N + K + M + 7)
+
+
+def _check_planned(s12, N, K, M, seed, outliers=0.0):
+    from fp32_weight_compression_b200 import wc
+    wbits = _weights(N, K, seed, outliers)
+    cont = s12.encode(wbits)
+    rng = np.random.default_rng(seed + 1)
+    xbits = workloads.rne_bf16(rng.standard_normal(M * K).astype(np.float32))
+    y64 = s12.linear(xbits.reshape(M, K), cont, N)
+    absum = np.abs(_to_f64(xbits).reshape(M, K)) @ np.abs(_to_f64(wbits).reshape(N, K)).T
+    dcont = torch.from_numpy(cont).to("cuda")
+    plan = wc.split12_plan(dcont, N, K)
+    y = wc.split12_linear(dcont, N, K, _bf16_dev(xbits).view(M, K), plan=plan)
+    torch.cuda.synchronize()
+    m = K + K // 64
+    u = 2.0 ** -23
+    bound = m * u / (1 - m * u) * absum
+    err = np.abs(y.cpu().numpy().astype(np.float64) - y64)
+    assert (err <= bound).all(), int((err > bound).sum())
+    # the same bits as without the plan, up to the split-K atomics' order
+    y0 = wc.split12_linear(dcont, N, K, _bf16_dev(xbits).view(M, K))
+    assert (np.abs(y0.cpu().numpy().astype(np.float64) - y64) <= bound).all()
+
+
+@pytest.mark.parametrize("K", [64, 4096])
+def test_planned_exceptions(s12, K):
+    """1 in 500 values an exception (the plan's range copied to shared
+    memory) and 1 in 5 (more than a CTA's list holds: read at each stage)."""
+    for frac in (0.002, 0.2):
+        for M in (1, 33):
+            _check_planned(s12, 256, K, M, seed=K + int(frac * 1000) + M + 3, outliers=frac)
+
+
+def test_plan_mismatch_and_corruption_are_reported(s12):
+    from fp32_weight_compression_b200 import wc
+    N, K = 128, 256
+    cont = s12.encode(_weights(N, K, 8, 0.01))
+    other = s12.encode(_weights(N, K, 9, 0.03))
+    dcont, dother = torch.from_numpy(cont).to("cuda"), torch.from_numpy(other).to("cuda")
+    plan = wc.split12_plan(dcont, N, K)
+    x = _bf16_dev(workloads.rne_bf16(np.ones(4 * K, np.float32))).view(4, K)
+    # a plan built for another container (another exception count)
+    assert s12.read_header(cont)["ne"] != s12.read_header(other)["ne"]
+    with pytest.raises(wc.WCError) as ei:
+        wc.split12_linear(dother, N, K, x, plan=plan)
+    assert ei.value.code == wc.ERR_CORRUPT
+    # a plan whose header (magic, N) was damaged, or whose starts run past
+    # the exception count or out of order (a plan is an index, not a
+    # checksummed copy: damage that keeps the starts in order goes unseen)
+    for off, val in ((0, 0xFF), (8, 0x01)):
+        bad = plan.clone()
+        bad[off] ^= val
+        with pytest.raises(wc.WCError) as ei:
+            wc.split12_linear(dcont, N, K, x, plan=bad)
+        assert ei.value.code == wc.ERR_CORRUPT
+    for i, v in ((1, 0xFFFFFFFF), (4, 0)):
+        bad = plan.clone()
+        bad[32 + 4 * i:32 + 4 * i + 4] = torch.tensor(list(int(v).to_bytes(4, "little")), dtype=torch.uint8)
+        with pytest.raises(wc.WCError) as ei:
+            wc.split12_linear(dcont, N, K, x, plan=bad)
+        assert ei.value.code == wc.ERR_CORRUPT
+    # a plan too short for its starts is refused on the host
+    with pytest.raises(wc.WCError) as ei:
+        wc.split12_linear(dcont, N, K, x, plan=plan[:40])
+    assert ei.value.code == wc.ERR_INVALID_ARG
+    # a corrupt container yields an invalid plan, which is then refused
+    badc = cont.copy()
+    h = s12.read_header(cont)
+    lay = s12.layout(h["n"], h["ne"])
+    badc[lay["off_exc"]:lay["off_exc"] + 2] = 0xFF  # first exception position past its chunk
+    with pytest.raises(wc.WCError) as ei:
+        wc.split12_plan(torch.from_numpy(badc).to("cuda"), N, K)
+    assert ei.value.code == wc.ERR_CORRUPT
+    # the intact pair still works
+    y = wc.split12_linear(dcont, N, K, x, plan=plan)
+    assert torch.isfinite(y).all()
