@@ -613,8 +613,10 @@ def linear_leg(ins, specs_mine, dev, reps: int = 20):
     (the tensor-core path at every M).
     W: the first four gate projections of the set (4096 x 14336 bf16, 117 MB
     each, 470 MB together > L2), used in rotation so that every call reads its
-    weights from HBM.  Reported per M: microseconds per call and the weight
-    bytes each call reads over its time."""
+    weights from HBM.  Timed with and without the weights' serving plans
+    (wc12_plan, built once before the timing; wc12_linear_planned).  Reported
+    per M: microseconds per call and the weight bytes each call reads over
+    its time."""
     import torch
     from fp32_weight_compression_b200 import wc
     pick = [i for i, s in enumerate(specs_mine) if s.name.endswith(".gate")][:4]
@@ -623,6 +625,7 @@ def linear_leg(ins, specs_mine, dev, reps: int = 20):
     Ws = [ins[i].view(specs_mine[i].shape) for i in pick]
     N, K = Ws[0].shape
     conts = [wc.split12_encode(w.reshape(-1)) for w in Ws]
+    plans = [wc.split12_plan(c, N, K) for c in conts]
     L = wc.load()
     status = torch.zeros(1, dtype=torch.int32, device=dev)
     out = {}
@@ -636,11 +639,17 @@ def linear_leg(ins, specs_mine, dev, reps: int = 20):
             wc._check(L.wc12_linear(c.data_ptr(), c.numel(), N, K, x.data_ptr(), M, y.data_ptr(),
                                     status.data_ptr(), s), "wc12_linear")
 
+        def ours_planned(r):
+            c, pl = conts[r % len(conts)], plans[r % len(plans)]
+            wc._check(L.wc12_linear_planned(c.data_ptr(), c.numel(), pl.data_ptr(), pl.numel(), N, K,
+                                            x.data_ptr(), M, y.data_ptr(), status.data_ptr(), s),
+                      "wc12_linear_planned")
+
         def ref(r):
             torch.matmul(x, Ws[r % len(Ws)].t())
 
         res = {}
-        for name, fn in (("wc12_linear", ours), ("cublas_bf16", ref)):
+        for name, fn in (("wc12_linear", ours), ("wc12_linear_planned", ours_planned), ("cublas_bf16", ref)):
             for r in range(4):
                 fn(r)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -651,7 +660,7 @@ def linear_leg(ins, specs_mine, dev, reps: int = 20):
             b.record()
             torch.cuda.synchronize(dev)
             t = a.elapsed_time(b) / reps / 1e3
-            wbytes = conts[0].numel() if name == "wc12_linear" else 2 * N * K
+            wbytes = conts[0].numel() if name.startswith("wc12") else 2 * N * K
             res[name] = {"us": t * 1e6, "weight_gbs": wbytes / t / 1e9}
         assert int(status.item()) == 0
         ref_y = torch.matmul(x.float(), Ws[(reps - 1) % len(Ws)].float().t())
@@ -659,9 +668,10 @@ def linear_leg(ins, specs_mine, dev, reps: int = 20):
         torch.cuda.synchronize(dev)
         res["max_rel_err"] = float(((y - ref_y).abs().max() / ref_y.abs().max().clamp_min(1e-30)).item())
         res["speedup"] = res["cublas_bf16"]["us"] / res["wc12_linear"]["us"]
+        res["speedup_planned"] = res["cublas_bf16"]["us"] / res["wc12_linear_planned"]["us"]
         out[str(M)] = res
     return {"N": N, "K": K, "weights": len(Ws), "per_M": out,
-            "container_bytes": conts[0].numel(), "bf16_bytes": 2 * N * K}
+            "container_bytes": conts[0].numel(), "plan_bytes": plans[0].numel(), "bf16_bytes": 2 * N * K}
 
 
 def checksum_leg(arena, dev, stream, reps: int = 10):
