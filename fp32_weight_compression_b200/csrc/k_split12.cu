@@ -32,8 +32,53 @@ namespace wc12 {
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
 
+// Launch parameters of a batch (up to kBatchMax tensors per launch; passed by
+// value).  Encode: the kernels that work per chunk find their tensor by its
+// first chunk (chunk_base), k12_count by its first block (count_base); the
+// per-tensor kernels take one block per tensor.
+constexpr uint32_t kBatchMax = 256;
+struct EncItem12 {
+  const uint16_t *in;
+  uint8_t *out;
+  uint8_t *scr;
+  uint64_t *out_size;
+  uint64_t n;
+  uint32_t chunk_base;
+  uint32_t count_base;
+};
+struct EncBatch12 {
+  uint32_t count, total_chunks, total_count_blocks, pad;
+  EncItem12 items[kBatchMax];
+};
+struct DecItem12 {
+  const uint8_t *cont;
+  uint64_t cont_bytes;
+  uint16_t *out;
+  uint64_t n;         // the values the caller expects (the header must agree)
+  uint32_t unit_base; // first work unit: one per chunk, one for an empty tensor
+  uint32_t pad;
+};
+struct DecBatch12 {
+  uint32_t count, total_units;
+  int32_t *status;
+  DecItem12 items[kBatchMax];
+};
+
+template <typename Item, typename F>
+__device__ __forceinline__ uint32_t find_item(const Item *items, uint32_t count, uint32_t g, F base_of) {
+  uint32_t lo = 0, hi = count - 1;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi + 1) >> 1;
+    if (base_of(items[mid]) <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k12_prep(uint64_t n, uint8_t *out, uint8_t *scr) {
+__global__ void __launch_bounds__(256) k12_prep(const __grid_constant__ EncBatch12 b) {
+  const EncItem12 &it = b.items[blockIdx.x];
+  const uint64_t n = it.n;
+  uint8_t *out = it.out, *scr = it.scr;
   const int tid = threadIdx.x;
   const Lay L = lay(n, 0);
   reinterpret_cast<unsigned long long *>(scr + kScrHist)[tid] = 0;
@@ -75,11 +120,15 @@ __device__ __forceinline__ void count_group(uint32_t *sh, int lane, uint4 a, uin
   count_hi(sh, lane, b.x); count_hi(sh, lane, b.y); count_hi(sh, lane, b.z); count_hi(sh, lane, b.w);
 }
 
-__global__ void __launch_bounds__(kHistThreads, 2)
-k12_hist(const uint16_t *__restrict__ in, uint64_t n, uint8_t *scr) {
+__global__ void __launch_bounds__(kHistThreads, 2) k12_hist(const __grid_constant__ EncBatch12 b) {
   __shared__ __align__(16) uint32_t sh[256 * 32];  // [high byte][lane]
+  const EncItem12 &it =
+      b.items[find_item(b.items, b.count, blockIdx.x, [](const EncItem12 &x) { return x.chunk_base; })];
+  const uint16_t *__restrict__ in = it.in;
+  const uint64_t n = it.n;
+  uint8_t *scr = it.scr;
   const int tid = threadIdx.x, lane = tid & 31;
-  const uint64_t c = blockIdx.x, v0 = c * kChunk;
+  const uint64_t c = blockIdx.x - it.chunk_base, v0 = c * kChunk;
   const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
   const uint32_t nfull = count / 16;
   for (int i = tid; i < 256 * 32 / 4; i += kHistThreads)
@@ -111,7 +160,8 @@ k12_hist(const uint16_t *__restrict__ in, uint64_t n, uint8_t *scr) {
 }
 
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k12_book(uint8_t *out, uint8_t *scr) {
+__global__ void __launch_bounds__(256) k12_book(const __grid_constant__ EncBatch12 b) {
+  uint8_t *out = b.items[blockIdx.x].out, *scr = b.items[blockIdx.x].scr;
   __shared__ unsigned long long cnt[256];
   __shared__ uint32_t wsel[8];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -140,14 +190,20 @@ __global__ void __launch_bounds__(256) k12_book(uint8_t *out, uint8_t *scr) {
 }
 
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k12_count(uint64_t nc, uint8_t *out, const uint8_t *scr) {
+__global__ void __launch_bounds__(256) k12_count(const __grid_constant__ EncBatch12 b) {
   __shared__ uint8_t lut[256];
+  const EncItem12 &it =
+      b.items[find_item(b.items, b.count, blockIdx.x, [](const EncItem12 &x) { return x.count_base; })];
+  const uint64_t nc = (it.n + kChunk - 1) / kChunk;
+  uint8_t *out = it.out;
+  const uint8_t *scr = it.scr;
+  const uint32_t lb = blockIdx.x - it.count_base;  // block of this tensor
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   lut[tid] = scr[kScrLut + tid];
   __syncthreads();
-  const uint64_t c = uint64_t(blockIdx.x) * 8 + warp;
+  const uint64_t c = uint64_t(lb) * 8 + warp;
   uint64_t *exc_off = reinterpret_cast<uint64_t *>(out + kExcOffOff);
-  if (blockIdx.x == 0 && tid == 0) exc_off[0] = 0;
+  if (lb == 0 && tid == 0) exc_off[0] = 0;
   if (c >= nc) return;
   const uint32_t *h = reinterpret_cast<const uint32_t *>(scr + kScrChunkHist) + c * 256;
   uint32_t s = 0;
@@ -164,7 +220,10 @@ __global__ void __launch_bounds__(256) k12_count(uint64_t nc, uint8_t *out, cons
 // ---------------------------------------------------------------------------
 constexpr int kScanThreads = 1024;
 
-__global__ void __launch_bounds__(kScanThreads) k12_scan(uint64_t n, uint8_t *out, uint64_t *out_size) {
+__global__ void __launch_bounds__(kScanThreads) k12_scan(const __grid_constant__ EncBatch12 b) {
+  const uint64_t n = b.items[blockIdx.x].n;
+  uint8_t *out = b.items[blockIdx.x].out;
+  uint64_t *out_size = b.items[blockIdx.x].out_size;
   __shared__ uint64_t red[kScanThreads / 32 + 1];
   __shared__ uint64_t s_ne;
   const int tid = threadIdx.x;
@@ -216,13 +275,18 @@ __device__ __forceinline__ uint32_t nibbles4(uint32_t s4, uint32_t &missed) {
   return (idx & 0xFu) | ((idx >> 4) & 0xF0u) | ((idx >> 8) & 0xF00u) | ((idx >> 12) & 0xF000u);
 }
 
-__global__ void __launch_bounds__(kPackThreads)
-k12_pack(const uint16_t *__restrict__ in, uint64_t n, uint8_t *out, const uint8_t *scr) {
+__global__ void __launch_bounds__(kPackThreads) k12_pack(const __grid_constant__ EncBatch12 b) {
   __shared__ uint8_t lut[256];
   __shared__ uint64_t red[kPackThreads / 32 + 1];
+  const EncItem12 &it =
+      b.items[find_item(b.items, b.count, blockIdx.x, [](const EncItem12 &x) { return x.chunk_base; })];
+  const uint16_t *__restrict__ in = it.in;
+  const uint64_t n = it.n;
+  uint8_t *out = it.out;
+  const uint8_t *scr = it.scr;
   const int tid = threadIdx.x;
   lut[tid] = scr[kScrLut + tid];
-  const uint64_t c = blockIdx.x, v0 = c * kChunk;
+  const uint64_t c = blockIdx.x - it.chunk_base, v0 = c * kChunk;
   const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
   const uint32_t nfull = count / 16, tail = count % 16;
   const uint32_t ngroups = nfull + (tail ? 1u : 0u);
@@ -305,35 +369,49 @@ __device__ __forceinline__ uint32_t over8(uint32_t w, uint32_t add) {
   return ((e + add) | (o + add)) & 0x10101010u;
 }
 
-__global__ void __launch_bounds__(kDecThreads)
-k12_decode(const uint8_t *__restrict__ cont, uint64_t cont_bytes, uint16_t *__restrict__ out,
-           uint64_t out_cap, int32_t *status) {
-  const int tid = threadIdx.x;
-  // header checks (every block; block 0 reports)
-  if (cont_bytes < 96) {
-    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CORRUPT);
-    return;
-  }
+// A container's header and layout, checked (every block that decodes from
+// it checks them; the first reports): err is WC_OK, WC_ERR_CORRUPT or, when
+// its values do not fit out_cap bytes, WC_ERR_CAPACITY.
+struct View12 {
+  int32_t err;
+  uint64_t n, ne;
+  uint32_t k;
+  Lay L;
+};
+
+__device__ View12 view12(const uint8_t *cont, uint64_t cont_bytes, uint64_t out_cap) {
+  View12 v{};
+  v.err = WC_ERR_CORRUPT;
+  if (cont_bytes < 96) return v;
   const uint32_t *h32 = reinterpret_cast<const uint32_t *>(cont);
   const uint64_t *h64 = reinterpret_cast<const uint64_t *>(cont);
   const uint64_t n = h64[1], ne = h64[3];
   const uint32_t k = h32[1] >> 24;
   bool ok = h32[0] == kMagic && (h32[1] & 0xFFFFFFu) == (1u | (1u << 16)) && k <= 16 &&
             (n > 0) == (k > 0) && n <= kMaxN && ne <= n && h32[4] == uint32_t(kChunk);
-  Lay L{};
-  if (ok) {
-    L = lay(n, ne);
-    ok = h32[5] == uint32_t(L.nc) && h64[4] == L.off_idx && h64[5] == L.off_lo &&
-         h64[6] == L.off_exc && h64[7] == L.total && L.total <= cont_bytes;
-  }
-  if (!ok) {
-    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CORRUPT);
-    return;
-  }
-  if (2 * n > out_cap) {
-    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CAPACITY);
-    return;
-  }
+  if (!ok) return v;
+  const Lay L = lay(n, ne);
+  ok = h32[5] == uint32_t(L.nc) && h64[4] == L.off_idx && h64[5] == L.off_lo && h64[6] == L.off_exc &&
+       h64[7] == L.total && L.total <= cont_bytes;
+  if (!ok) return v;
+  // an empty tensor's table is one zero
+  if (L.nc == 0 && reinterpret_cast<const uint64_t *>(cont + kExcOffOff)[0] != 0) return v;
+  v.n = n;
+  v.ne = ne;
+  v.k = k;
+  v.L = L;
+  v.err = 2 * n > out_cap ? WC_ERR_CAPACITY : WC_OK;
+  return v;
+}
+
+// Chunk c of a checked container into out (whole block): 16 values per
+// thread per step, then the chunk's exceptions after a block barrier.
+__device__ __forceinline__ void decode_chunk12(const uint8_t *__restrict__ cont, const View12 &v, uint64_t c,
+                                               uint16_t *__restrict__ out, int32_t *status) {
+  const int tid = threadIdx.x;
+  const Lay &L = v.L;
+  const uint64_t n = v.n, ne = v.ne;
+  const uint32_t k = v.k;
   const uint4 book = *reinterpret_cast<const uint4 *>(cont + kBookOff);
   const uint32_t add = (16u - k) * 0x01010101u;
   const uint64_t *exc_off = reinterpret_cast<const uint64_t *>(cont + kExcOffOff);
@@ -341,53 +419,75 @@ k12_decode(const uint8_t *__restrict__ cont, uint64_t cont_bytes, uint16_t *__re
   const uint8_t *exc_val = cont + L.off_excval;
   const uint8_t *idx_plane = cont + L.off_idx;
   const uint8_t *lo_plane = cont + L.off_lo;
-  if (L.nc == 0 && exc_off[0] != 0) {  // an empty tensor's table is one zero
-    if (blockIdx.x == 0 && tid == 0) report(status, WC_ERR_CORRUPT);
+  const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
+  if (!(e0 <= e1 && e1 <= ne && (c != 0 || e0 == 0) && (c + 1 != L.nc || e1 == ne))) {
+    if (tid == 0) report(status, WC_ERR_CORRUPT);
     return;
   }
-
-  for (uint64_t c = blockIdx.x; c < L.nc; c += gridDim.x) {
-    const uint64_t e0 = exc_off[c], e1 = exc_off[c + 1];
-    if (!(e0 <= e1 && e1 <= ne && (c != 0 || e0 == 0) && (c + 1 != L.nc || e1 == ne))) {
-      if (tid == 0) report(status, WC_ERR_CORRUPT);
+  const uint64_t v0 = c * kChunk;
+  const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
+  const uint32_t nfull = count / 16, tail = count % 16;
+  uint32_t bad = 0;
+  for (uint32_t g = tid; g < nfull; g += kDecThreads) {
+    const uint2 q = *reinterpret_cast<const uint2 *>(idx_plane + v0 / 2 + 8 * g);
+    const uint4 lo = *reinterpret_cast<const uint4 *>(lo_plane + v0 + 16 * g);
+    bad |= over8(q.x, add) | over8(q.y, add);
+    const uint2 o0 = expand4(q.x, book, lo.x), o1 = expand4(q.x >> 16, book, lo.y);
+    const uint2 o2 = expand4(q.y, book, lo.z), o3 = expand4(q.y >> 16, book, lo.w);
+    uint4 *dst = reinterpret_cast<uint4 *>(out + v0 + 16 * g);
+    dst[0] = make_uint4(o0.x, o0.y, o1.x, o1.y);
+    dst[1] = make_uint4(o2.x, o2.y, o3.x, o3.y);
+  }
+  if (tid == 0) {  // the ragged tail, value by value
+    for (uint32_t j = 0; j < tail; j++) {
+      const uint64_t vv = v0 + 16 * uint64_t(nfull) + j;
+      const uint32_t nib = (uint32_t(idx_plane[vv / 2]) >> (4 * (vv & 1))) & 0xFu;
+      bad |= nib >= k ? 1u : 0u;
+      const uint32_t hi = (nib < 8 ? ((&book.x)[nib >> 2] >> (8 * (nib & 3)))
+                                   : ((&book.z)[(nib - 8) >> 2] >> (8 * (nib & 3)))) & 0xFFu;
+      out[vv] = uint16_t((hi << 8) | lo_plane[vv]);
+    }
+  }
+  if (bad) report(status, WC_ERR_CORRUPT);
+  __syncthreads();  // the chunk's values are written; patch its exceptions
+  for (uint64_t e = e0 + tid; e < e1; e += kDecThreads) {
+    const uint32_t p = exc_pos[e];
+    if (p >= count || (e > e0 && p <= exc_pos[e - 1])) {
+      report(status, WC_ERR_CORRUPT);
       continue;
     }
-    const uint64_t v0 = c * kChunk;
-    const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
-    const uint32_t nfull = count / 16, tail = count % 16;
-    uint32_t bad = 0;
-    for (uint32_t g = tid; g < nfull; g += kDecThreads) {
-      const uint2 q = *reinterpret_cast<const uint2 *>(idx_plane + v0 / 2 + 8 * g);
-      const uint4 lo = *reinterpret_cast<const uint4 *>(lo_plane + v0 + 16 * g);
-      bad |= over8(q.x, add) | over8(q.y, add);
-      const uint2 o0 = expand4(q.x, book, lo.x), o1 = expand4(q.x >> 16, book, lo.y);
-      const uint2 o2 = expand4(q.y, book, lo.z), o3 = expand4(q.y >> 16, book, lo.w);
-      uint4 *dst = reinterpret_cast<uint4 *>(out + v0 + 16 * g);
-      dst[0] = make_uint4(o0.x, o0.y, o1.x, o1.y);
-      dst[1] = make_uint4(o2.x, o2.y, o3.x, o3.y);
+    const uint64_t vv = v0 + p;
+    out[vv] = uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[vv]);
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kDecThreads)
+k12_decode(const uint8_t *__restrict__ cont, uint64_t cont_bytes, uint16_t *__restrict__ out,
+           uint64_t out_cap, int32_t *status) {
+  const View12 v = view12(cont, cont_bytes, out_cap);
+  if (v.err != WC_OK) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) report(status, v.err);
+    return;
+  }
+  for (uint64_t c = blockIdx.x; c < v.L.nc; c += gridDim.x) decode_chunk12(cont, v, c, out, status);
+}
+
+// Many containers in one launch: work unit g (a chunk, or the one unit of an
+// empty tensor) of the container whose units start at or before g.
+__global__ void __launch_bounds__(kDecThreads) k12_decode_batch(const __grid_constant__ DecBatch12 b) {
+  for (uint32_t g = blockIdx.x; g < b.total_units; g += gridDim.x) {
+    const DecItem12 &it =
+        b.items[find_item(b.items, b.count, g, [](const DecItem12 &x) { return x.unit_base; })];
+    const uint32_t u = g - it.unit_base;
+    const View12 v = view12(it.cont, it.cont_bytes, 2 * it.n);
+    // a header for another number of values is not the tensor the caller expects
+    const int32_t err = v.err != WC_ERR_CORRUPT && v.n != it.n ? WC_ERR_CORRUPT : v.err;
+    if (err != WC_OK) {
+      if (u == 0 && threadIdx.x == 0) report(b.status, err);
+      continue;
     }
-    if (tid == 0) {  // the ragged tail, value by value
-      for (uint32_t j = 0; j < tail; j++) {
-        const uint64_t v = v0 + 16 * uint64_t(nfull) + j;
-        const uint32_t nib = (uint32_t(idx_plane[v / 2]) >> (4 * (v & 1))) & 0xFu;
-        bad |= nib >= k ? 1u : 0u;
-        const uint32_t hi = (nib < 8 ? ((&book.x)[nib >> 2] >> (8 * (nib & 3)))
-                                     : ((&book.z)[(nib - 8) >> 2] >> (8 * (nib & 3)))) & 0xFFu;
-        out[v] = uint16_t((hi << 8) | lo_plane[v]);
-      }
-    }
-    if (bad) report(status, WC_ERR_CORRUPT);
-    __syncthreads();  // the chunk's values are written; patch its exceptions
-    for (uint64_t e = e0 + tid; e < e1; e += kDecThreads) {
-      const uint32_t p = exc_pos[e];
-      if (p >= count || (e > e0 && p <= exc_pos[e - 1])) {
-        report(status, WC_ERR_CORRUPT);
-        continue;
-      }
-      const uint64_t v = v0 + p;
-      out[v] = uint16_t((uint32_t(exc_val[e]) << 8) | lo_plane[v]);
-    }
-    __syncthreads();
+    if (v.L.nc > 0) decode_chunk12(it.cont, v, u, it.out, b.status);
   }
 }
 
@@ -421,31 +521,58 @@ uint64_t wc12_scratch_bytes(uint64_t n) {
   return wc12::kScrChunkHist + 1024 * ((n + wc12::kChunk - 1) / wc12::kChunk);
 }
 
+int32_t wc12_encode_batch(const wc12_encode_item *items, uint32_t count, void *stream) {
+  if (count == 0) return WC_OK;
+  if (items == nullptr) return WC_ERR_INVALID_ARG;
+  for (uint32_t i = 0; i < count; i++) {
+    const wc12_encode_item &it = items[i];
+    if (it.n > wc12::kMaxN || it.out == nullptr || it.scratch == nullptr || it.out_size == nullptr)
+      return WC_ERR_INVALID_ARG;
+    if (it.n > 0 && it.in == nullptr) return WC_ERR_INVALID_ARG;
+    if (!wc12::aligned(it.in, 16) || !wc12::aligned(it.out, 16) || !wc12::aligned(it.scratch, 16) ||
+        !wc12::aligned(it.out_size, 8))
+      return WC_ERR_INVALID_ARG;
+    if (it.out_cap < wc12_encode_bound(it.n) || it.scratch_cap < wc12_scratch_bytes(it.n)) return WC_ERR_CAPACITY;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  static thread_local wc12::EncBatch12 B;  // ~12 KiB: kept off the stack
+  for (uint32_t b0 = 0; b0 < count; b0 += wc12::kBatchMax) {
+    const uint32_t cnt = count - b0 < wc12::kBatchMax ? count - b0 : wc12::kBatchMax;
+    memset(&B, 0, sizeof(B));
+    B.count = cnt;
+    uint64_t chunks = 0, cblocks = 0;
+    for (uint32_t i = 0; i < cnt; i++) {
+      const wc12_encode_item &src = items[b0 + i];
+      wc12::EncItem12 &d = B.items[i];
+      d.in = static_cast<const uint16_t *>(src.in);
+      d.out = static_cast<uint8_t *>(src.out);
+      d.scr = static_cast<uint8_t *>(src.scratch);
+      d.out_size = src.out_size;
+      d.n = src.n;
+      d.chunk_base = uint32_t(chunks);
+      d.count_base = uint32_t(cblocks);
+      const uint64_t nc = (src.n + wc12::kChunk - 1) / wc12::kChunk;
+      chunks += nc;
+      cblocks += nc ? (nc + 7) / 8 : 1;  // an empty tensor's block writes exc_off[0]
+      if (chunks > 0x7FFFFFFFull || cblocks > 0x7FFFFFFFull) return WC_ERR_INVALID_ARG;
+    }
+    B.total_chunks = uint32_t(chunks);
+    B.total_count_blocks = uint32_t(cblocks);
+    wc12::k12_prep<<<cnt, 256, 0, s>>>(B);
+    if (chunks) wc12::k12_hist<<<unsigned(chunks), wc12::kHistThreads, 0, s>>>(B);
+    wc12::k12_book<<<cnt, 256, 0, s>>>(B);
+    wc12::k12_count<<<unsigned(cblocks), 256, 0, s>>>(B);
+    wc12::k12_scan<<<cnt, wc12::kScanThreads, 0, s>>>(B);
+    if (chunks) wc12::k12_pack<<<unsigned(chunks), wc12::kPackThreads, 0, s>>>(B);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+  }
+  return WC_OK;
+}
+
 int32_t wc12_encode(const void *d_in, uint64_t n, void *d_out, uint64_t out_cap, void *d_scratch,
                     uint64_t scratch_cap, uint64_t *d_out_size, void *stream) {
-  if (n > wc12::kMaxN || d_out == nullptr || d_scratch == nullptr || d_out_size == nullptr)
-    return WC_ERR_INVALID_ARG;
-  if (n > 0 && d_in == nullptr) return WC_ERR_INVALID_ARG;
-  if (!wc12::aligned(d_in, 16) || !wc12::aligned(d_out, 16) || !wc12::aligned(d_scratch, 16) ||
-      !wc12::aligned(d_out_size, 8))
-    return WC_ERR_INVALID_ARG;
-  if (out_cap < wc12_encode_bound(n) || scratch_cap < wc12_scratch_bytes(n)) return WC_ERR_CAPACITY;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const uint16_t *in = static_cast<const uint16_t *>(d_in);
-  uint8_t *out = static_cast<uint8_t *>(d_out);
-  uint8_t *scr = static_cast<uint8_t *>(d_scratch);
-  const uint64_t nc = (n + wc12::kChunk - 1) / wc12::kChunk;
-  if (nc > 0x7FFFFFFFull) return WC_ERR_INVALID_ARG;
-  wc12::k12_prep<<<1, 256, 0, s>>>(n, out, scr);
-  if (nc) wc12::k12_hist<<<unsigned(nc), wc12::kHistThreads, 0, s>>>(in, n, scr);
-  wc12::k12_book<<<1, 256, 0, s>>>(out, scr);
-  if (nc) wc12::k12_count<<<unsigned((nc + 7) / 8), 256, 0, s>>>(nc, out, scr);
-  else wc12::k12_count<<<1, 256, 0, s>>>(0, out, scr);  // writes exc_off[0]
-  wc12::k12_scan<<<1, wc12::kScanThreads, 0, s>>>(n, out, d_out_size);
-  if (nc) wc12::k12_pack<<<unsigned(nc), wc12::kPackThreads, 0, s>>>(in, n, out, scr);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return WC_ERR_CUDA;
-  return WC_OK;
+  wc12_encode_item it{d_in, n, d_out, out_cap, d_scratch, scratch_cap, d_out_size};
+  return wc12_encode_batch(&it, 1, stream);
 }
 
 int32_t wc12_read_header(const void *h_cont, uint64_t bytes, uint64_t *n, uint64_t *ne, uint32_t *k) {
@@ -467,6 +594,45 @@ int32_t wc12_read_header(const void *h_cont, uint64_t bytes, uint64_t *n, uint64
   *n = nn;
   *ne = nne;
   *k = kk;
+  return WC_OK;
+}
+
+int32_t wc12_decode_batch(const wc12_decode_item *items, uint32_t count, int32_t *d_status, void *stream) {
+  if (count == 0) return WC_OK;
+  if (items == nullptr || d_status == nullptr || !wc12::aligned(d_status, 4)) return WC_ERR_INVALID_ARG;
+  for (uint32_t i = 0; i < count; i++) {
+    const wc12_decode_item &it = items[i];
+    if (it.cont == nullptr || !wc12::aligned(it.cont, 16) || !wc12::aligned(it.out, 16) || it.n > wc12::kMaxN)
+      return WC_ERR_INVALID_ARG;
+    if (it.n > 0 && it.out == nullptr) return WC_ERR_INVALID_ARG;
+  }
+  const int sms = wc12::sms_of_current_device();
+  if (sms <= 0) return WC_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  static thread_local wc12::DecBatch12 B;
+  for (uint32_t b0 = 0; b0 < count; b0 += wc12::kBatchMax) {
+    const uint32_t cnt = count - b0 < wc12::kBatchMax ? count - b0 : wc12::kBatchMax;
+    memset(&B, 0, sizeof(B));
+    B.count = cnt;
+    B.status = d_status;
+    uint64_t units = 0;
+    for (uint32_t i = 0; i < cnt; i++) {
+      const wc12_decode_item &src = items[b0 + i];
+      wc12::DecItem12 &d = B.items[i];
+      d.cont = static_cast<const uint8_t *>(src.cont);
+      d.cont_bytes = src.cont_bytes;
+      d.out = static_cast<uint16_t *>(src.out);
+      d.n = src.n;
+      d.unit_base = uint32_t(units);
+      const uint64_t nc = (src.n + wc12::kChunk - 1) / wc12::kChunk;
+      units += nc ? nc : 1;
+      if (units > 0x7FFFFFFFull) return WC_ERR_INVALID_ARG;
+    }
+    B.total_units = uint32_t(units);
+    const uint64_t cap = uint64_t(sms) * 8;
+    wc12::k12_decode_batch<<<unsigned(units < cap ? units : cap), wc12::kDecThreads, 0, s>>>(B);
+    if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
+  }
   return WC_OK;
 }
 

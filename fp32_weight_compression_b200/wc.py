@@ -42,6 +42,17 @@ class EncodeItem(ctypes.Structure):
                 ("out_size", ctypes.c_void_p)]
 
 
+class Split12EncodeItem(ctypes.Structure):
+    _fields_ = [("in_", ctypes.c_void_p), ("n", ctypes.c_uint64), ("out", ctypes.c_void_p),
+                ("out_cap", ctypes.c_uint64), ("scratch", ctypes.c_void_p), ("scratch_cap", ctypes.c_uint64),
+                ("out_size", ctypes.c_void_p)]
+
+
+class Split12DecodeItem(ctypes.Structure):
+    _fields_ = [("cont", ctypes.c_void_p), ("cont_bytes", ctypes.c_uint64), ("out", ctypes.c_void_p),
+                ("n", ctypes.c_uint64)]
+
+
 class DecodeItem(ctypes.Structure):
     _fields_ = [("cont", ctypes.c_void_p), ("cont_bytes", ctypes.c_uint64),
                 ("out", ctypes.c_void_p), ("out_cap", ctypes.c_uint64)]
@@ -124,6 +135,10 @@ def load() -> ctypes.CDLL:
     L.wc12_read_header.argtypes = [vp, u64, ctypes.POINTER(u64), ctypes.POINTER(u64), ctypes.POINTER(u32)]
     L.wc12_linear.restype = i32
     L.wc12_linear.argtypes = [vp, u64, u32, u32, vp, u32, vp, vp, vp]
+    L.wc12_encode_batch.restype = i32
+    L.wc12_encode_batch.argtypes = [ctypes.POINTER(Split12EncodeItem), u32, vp]
+    L.wc12_decode_batch.restype = i32
+    L.wc12_decode_batch.argtypes = [ctypes.POINTER(Split12DecodeItem), u32, vp, vp]
     L.wc12_plan_bytes.restype = u64
     L.wc12_plan_bytes.argtypes = [u32, u32, u64]
     L.wc12_plan.restype = i32
@@ -474,6 +489,50 @@ def split12_decode(cont: torch.Tensor, shape=None, out=None, stream=None) -> tor
     if st != OK:
         raise WCError(st, "wc12_decode (device status)")
     return out
+
+
+def split12_encode_batch(tensors, stream=None) -> list[torch.Tensor]:
+    """Split12 containers of many bf16 CUDA tensors, one launch per encoder
+    kernel for the whole list (wc12_encode_batch)."""
+    flats = []
+    for t in tensors:
+        if t.dtype != torch.bfloat16:
+            raise TypeError("Split12 takes bf16 tensors")
+        flats.append(_flat(t))
+    outs, scrs, sizes = [], [], []
+    items = (Split12EncodeItem * max(1, len(flats)))()
+    for i, f in enumerate(flats):
+        n = f.numel()
+        outs.append(torch.empty(split12_encode_bound(n), dtype=torch.uint8, device=f.device))
+        scrs.append(torch.empty(split12_scratch_bytes(n), dtype=torch.uint8, device=f.device))
+        sizes.append(torch.zeros(1, dtype=torch.int64, device=f.device))
+        items[i] = Split12EncodeItem(f.data_ptr() if n else None, n, outs[-1].data_ptr(), outs[-1].numel(),
+                                     scrs[-1].data_ptr(), scrs[-1].numel(), sizes[-1].data_ptr())
+    if flats:
+        _check(load().wc12_encode_batch(items, len(flats), _stream(stream)), "wc12_encode_batch")
+    return [o[: int(z.item())] for o, z in zip(outs, sizes)]
+
+
+def split12_decode_batch(conts, shapes, stream=None) -> list[torch.Tensor]:
+    """Decode many device Split12 containers into bf16 tensors of the given
+    shapes, one launch (wc12_decode_batch)."""
+    if len(conts) != len(shapes):
+        raise ValueError("one shape per container")
+    outs = []
+    items = (Split12DecodeItem * max(1, len(conts)))()
+    dev = conts[0].device if conts else None
+    for i, (c, sh) in enumerate(zip(conts, shapes)):
+        o = torch.empty(sh, dtype=torch.bfloat16, device=c.device)
+        outs.append(o)
+        items[i] = Split12DecodeItem(c.data_ptr(), c.numel(), o.data_ptr() if o.numel() else None, o.numel())
+    if conts:
+        status = torch.zeros(1, dtype=torch.int32, device=dev)
+        _check(load().wc12_decode_batch(items, len(conts), status.data_ptr(), _stream(stream)),
+               "wc12_decode_batch")
+        st = int(status.item())
+        if st != OK:
+            raise WCError(st, "wc12_decode_batch (device status)")
+    return outs
 
 
 def split12_plan_bytes(N: int, K: int, ne: int) -> int:

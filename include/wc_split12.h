@@ -68,6 +68,20 @@ WC_API int32_t wc12_encode(const void *d_in, uint64_t n, void *d_out, uint64_t o
 WC_API int32_t wc12_read_header(const void *h_cont, uint64_t bytes, uint64_t *n, uint64_t *ne,
                                 uint32_t *k);
 
+/* Many tensors in one call: one launch per encoder kernel for the whole
+ * list (in groups of 256 tensors), each item exactly as wc12_encode's
+ * arguments.  All checks are made before anything is launched. */
+typedef struct {
+  const void *in;      /* n bf16 values, 16-byte aligned (may be NULL if n == 0) */
+  uint64_t n;
+  void *out;           /* container, 16-byte aligned, out_cap >= wc12_encode_bound(n) */
+  uint64_t out_cap;
+  void *scratch;       /* 16-byte aligned, scratch_cap >= wc12_scratch_bytes(n) */
+  uint64_t scratch_cap;
+  uint64_t *out_size;  /* device u64, 8-byte aligned: the container's size */
+} wc12_encode_item;
+WC_API int32_t wc12_encode_batch(const wc12_encode_item *items, uint32_t count, void *stream);
+
 /* Decode a container (d_cont, cont_bytes, 16-byte aligned) into out_cap bytes
  * at d_out (16-byte aligned).  *d_status (device i32, set to 0 by the caller)
  * receives WC_ERR_CORRUPT for a bad header, offset table, index >= K or
@@ -76,6 +90,20 @@ WC_API int32_t wc12_read_header(const void *h_cont, uint64_t bytes, uint64_t *n,
  * Returns WC_OK, WC_ERR_INVALID_ARG or WC_ERR_CUDA. */
 WC_API int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out, uint64_t out_cap,
                            int32_t *d_status, void *stream);
+
+/* Many containers in one launch (in groups of 256): item i decodes cont
+ * (16-byte aligned, cont_bytes) into out (16-byte aligned, room for 2 n
+ * bytes), where n is the number of values the caller expects; a container
+ * whose header gives another n is reported as WC_ERR_CORRUPT.  The other
+ * checks and reports are wc12_decode's, into the one *d_status. */
+typedef struct {
+  const void *cont;
+  uint64_t cont_bytes;
+  void *out;
+  uint64_t n;
+} wc12_decode_item;
+WC_API int32_t wc12_decode_batch(const wc12_decode_item *items, uint32_t count, int32_t *d_status,
+                                 void *stream);
 
 /* Y = X W^T with W (N x K bf16, row-major) given as a Split12 container, the
  * weights crossing HBM at 12 bits a value ("weight-compression" README:

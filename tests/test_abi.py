@@ -268,6 +268,37 @@ def test_split12_linear_bad_arguments_rejected_without_device(wcm):
     assert L.wc12_linear(b, 95, 256, 128, b, 4, b, b, None) == wcm.ERR_INVALID_ARG   # no room for a header
 
 
+def test_split12_batch_bad_arguments_rejected_without_device(wcm):
+    L = wcm.load()
+    buf = (ctypes.c_uint8 * 4096)()
+    b = (ctypes.addressof(buf) + 255) // 256 * 256
+    n = 100
+    cap, scr = wcm.split12_encode_bound(n), wcm.split12_scratch_bytes(n)
+    E = wcm.Split12EncodeItem
+    def enc(**kw):
+        f = dict(in_=b, n=n, out=b, out_cap=cap, scratch=b, scratch_cap=scr, out_size=b)
+        f.update(kw)
+        items = (E * 2)(E(**dict(f)), E(b, 1, b, wcm.split12_encode_bound(1), b, wcm.split12_scratch_bytes(1), b))
+        return L.wc12_encode_batch(items, 2, None)
+    assert enc(in_=b + 2) == wcm.ERR_INVALID_ARG
+    assert enc(out=b + 8) == wcm.ERR_INVALID_ARG
+    assert enc(out_size=b + 4) == wcm.ERR_INVALID_ARG
+    assert enc(scratch=None) == wcm.ERR_INVALID_ARG
+    assert enc(out_cap=cap - 1) == wcm.ERR_CAPACITY
+    assert enc(scratch_cap=scr - 1) == wcm.ERR_CAPACITY
+    assert L.wc12_encode_batch(None, 1, None) == wcm.ERR_INVALID_ARG
+    assert L.wc12_encode_batch(None, 0, None) == wcm.OK
+    D = wcm.Split12DecodeItem
+    items = (D * 1)(D(b + 4, 1000, b, 10))
+    assert L.wc12_decode_batch(items, 1, b, None) == wcm.ERR_INVALID_ARG
+    items = (D * 1)(D(b, 1000, b + 2, 10))
+    assert L.wc12_decode_batch(items, 1, b, None) == wcm.ERR_INVALID_ARG
+    items = (D * 1)(D(b, 1000, None, 10))
+    assert L.wc12_decode_batch(items, 1, b, None) == wcm.ERR_INVALID_ARG
+    items = (D * 1)(D(b, 1000, b, 10))
+    assert L.wc12_decode_batch(items, 1, None, None) == wcm.ERR_INVALID_ARG
+
+
 def test_split12_plan_size_and_bad_arguments(wcm):
     """wc12_plan_bytes from its layout; wc12_plan and wc12_linear_planned
     refuse bad arguments before touching a device."""

@@ -118,3 +118,45 @@ def test_decodes_oracle_containers_and_refuses_damage(s12):
         else:
             assert st == 0
             assert np.array_equal(out[: want.size].cpu().numpy().view(np.uint16), want)
+
+
+def test_batch_matches_single_calls_and_the_oracle(s12):
+    """wc12_encode_batch / wc12_decode_batch: every container byte-identical
+    to the oracle's, every value bit-exact, for a list of mixed sizes (empty,
+    ragged, several chunks, exceptions) longer than one launch's 256 items."""
+    from fp32_weight_compression_b200 import wc
+    rng = np.random.default_rng(44)
+    sizes = [0, 1, 17, C - 1, C, C + 1, 3 * C + 5] + [int(rng.integers(0, 3 * C)) for _ in range(290)]
+    bits = []
+    for i, n in enumerate(sizes):
+        w = workloads.rne_bf16(rng.standard_normal(n).astype(np.float32) * np.float32(0.02))
+        if n and i % 3 == 0:  # some exceptions
+            m = rng.random(n) < 0.01
+            w[m] = (rng.integers(0, 256, int(m.sum())) << 8).astype(np.uint16) | (w[m] & 0xFF)
+        bits.append(w)
+    conts = wc.split12_encode_batch([_dev(b) for b in bits])
+    for b, c in zip(bits, conts):
+        want = s12.encode(b)
+        got = c.cpu().numpy()
+        assert got.size == want.size and np.array_equal(got, want)
+    outs = wc.split12_decode_batch(conts, [(b.size,) for b in bits])
+    for b, o in zip(bits, outs):
+        assert np.array_equal(o.view(torch.int16).cpu().numpy().view(np.uint16), b)
+
+
+def test_batch_decode_refuses_a_wrong_count_and_damage(s12):
+    from fp32_weight_compression_b200 import wc
+    rng = np.random.default_rng(45)
+    a = workloads.rne_bf16(rng.standard_normal(C + 9).astype(np.float32))
+    b = workloads.rne_bf16(rng.standard_normal(2 * C).astype(np.float32))
+    ca, cb = (torch.from_numpy(s12.encode(x)).to("cuda") for x in (a, b))
+    with pytest.raises(wc.WCError) as ei:
+        wc.split12_decode_batch([ca, cb], [(a.size,), (b.size - 1,)])  # not the tensor expected
+    assert ei.value.code == wc.ERR_CORRUPT
+    bad = ca.clone()
+    bad[0] ^= 0xFF
+    with pytest.raises(wc.WCError) as ei:
+        wc.split12_decode_batch([bad, cb], [(a.size,), (b.size,)])
+    assert ei.value.code == wc.ERR_CORRUPT
+    outs = wc.split12_decode_batch([ca, cb], [(a.size,), (b.size,)])
+    assert np.array_equal(outs[1].view(torch.int16).cpu().numpy().view(np.uint16), b)
