@@ -31,7 +31,7 @@
 namespace wc {
 
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr uint32_t kDecGroup = kDecWarps * 2;  // chunks per block group
+constexpr uint32_t kDecGroup = kDecWarps * 2;  // most chunks per block group
 constexpr uint32_t kRing = 1024;                // words per chunk ring
 constexpr uint32_t kUnit = 256;                 // words per cp.async round (32 lanes x 16 B)
 constexpr uint32_t kHalf = 256;                 // values per half-group (8 steps)
@@ -625,13 +625,20 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
   const int tid = threadIdx.x, warp = tid >> 5;
   int32_t *status = p.status;
 
-  // prologue: groups per item -> prefix (one item per thread)
-  uint32_t g = 0;
+  // prologue: chunks per item (one item per thread); the group size: 16
+  // chunks (all 8 warps) when the launch has enough chunks for every block,
+  // else the even number that spreads them over all blocks (down to one
+  // warp's pair); groups per item -> prefix
+  uint64_t cnt = 0;
   if (uint32_t(tid) < p.count) {
     const ItemView v = view_item(p.items[tid]);
-    if (v.ok) g = uint32_t((v.cnt + kDecGroup - 1) / kDecGroup);
+    if (v.ok) cnt = v.cnt;
     else if (blockIdx.x == 0) report(status, v.err);
   }
+  const uint64_t chunks = block_sum_u64<kDecThreads>(cnt, s.red);
+  const uint64_t per_block = (chunks + 2 * uint64_t(gridDim.x) - 1) / (2 * uint64_t(gridDim.x));  // pairs
+  const uint32_t group = uint32_t(per_block >= kDecGroup / 2 ? kDecGroup : (per_block < 1 ? 2 : 2 * per_block));
+  const uint32_t g = uint32_t((cnt + group - 1) / group);
   const uint64_t ex = block_excl_scan_u64<kDecThreads>(g, s.red);
   s.gpre[tid] = uint32_t(ex);
   if (tid == kDecThreads - 1) s.gpre[kMaxItems] = uint32_t(ex) + g;
@@ -650,7 +657,8 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
     const ItemView v = view_item(it);
     if (ii != s.cur_item) build_table(it, ii, status);
     if (!s.tab_ok) continue;
-    const uint64_t kA = v.first + uint64_t(grp - s.gpre[ii]) * kDecGroup + 2 * warp;
+    if (uint32_t(2 * warp) >= group) continue;  // this warp has no pair in a small group
+    const uint64_t kA = v.first + uint64_t(grp - s.gpre[ii]) * group + 2 * warp;
     const uint64_t kend = v.first + v.cnt;
     if (v.dtype == WC_BF16) decode_warp_chunks<WC_BF16>(v, it, kA, kend, status);
     else if (v.dtype == WC_FP16) decode_warp_chunks<WC_FP16>(v, it, kA, kend, status);
