@@ -626,9 +626,11 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
   int32_t *status = p.status;
 
   // prologue: chunks per item (one item per thread); the group size: 16
-  // chunks (all 8 warps) when the launch has enough chunks for every block,
-  // else the even number that spreads them over all blocks (down to one
-  // warp's pair); groups per item -> prefix
+  // chunks (8 warps x 2, decoded in lock-step) when the launch has enough
+  // for every block; with more chunks than warps, the even number that
+  // spreads them over all blocks; with fewer, one chunk a warp (a chunk is a
+  // chain of dependent steps: few chunks go faster one chain per warp) and as
+  // many a block as spread them; groups per item -> prefix
   uint64_t cnt = 0;
   if (uint32_t(tid) < p.count) {
     const ItemView v = view_item(p.items[tid]);
@@ -636,8 +638,15 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
     else if (blockIdx.x == 0) report(status, v.err);
   }
   const uint64_t chunks = block_sum_u64<kDecThreads>(cnt, s.red);
-  const uint64_t per_block = (chunks + 2 * uint64_t(gridDim.x) - 1) / (2 * uint64_t(gridDim.x));  // pairs
-  const uint32_t group = uint32_t(per_block >= kDecGroup / 2 ? kDecGroup : (per_block < 1 ? 2 : 2 * per_block));
+  const bool single = chunks <= uint64_t(kDecWarps) * gridDim.x;
+  uint32_t group;
+  if (single) {
+    const uint64_t per_block = (chunks + gridDim.x - 1) / gridDim.x;
+    group = uint32_t(per_block < 1 ? 1 : per_block);  // <= kDecWarps
+  } else {
+    const uint64_t per_block = (chunks + 2 * uint64_t(gridDim.x) - 1) / (2 * uint64_t(gridDim.x));  // pairs
+    group = uint32_t(per_block >= kDecGroup / 2 ? kDecGroup : 2 * per_block);
+  }
   const uint32_t g = uint32_t((cnt + group - 1) / group);
   const uint64_t ex = block_excl_scan_u64<kDecThreads>(g, s.red);
   s.gpre[tid] = uint32_t(ex);
@@ -657,9 +666,9 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
     const ItemView v = view_item(it);
     if (ii != s.cur_item) build_table(it, ii, status);
     if (!s.tab_ok) continue;
-    if (uint32_t(2 * warp) >= group) continue;  // this warp has no pair in a small group
-    const uint64_t kA = v.first + uint64_t(grp - s.gpre[ii]) * group + 2 * warp;
-    const uint64_t kend = v.first + v.cnt;
+    if (uint32_t(single ? warp : 2 * warp) >= group) continue;  // no chunk for this warp in a small group
+    const uint64_t kA = v.first + uint64_t(grp - s.gpre[ii]) * group + (single ? warp : 2 * warp);
+    const uint64_t kend = single ? min(v.first + v.cnt, kA + 1) : v.first + v.cnt;
     if (v.dtype == WC_BF16) decode_warp_chunks<WC_BF16>(v, it, kA, kend, status);
     else if (v.dtype == WC_FP16) decode_warp_chunks<WC_FP16>(v, it, kA, kend, status);
     else if (v.dtype == WC_FP8E4M3) decode_warp_chunks<WC_FP8E4M3>(v, it, kA, kend, status);

@@ -468,8 +468,7 @@ __global__ void __launch_bounds__(kCoderThreads, 4) k_coder(const __grid_constan
   s_bias[tid] = reinterpret_cast<const uint32_t *>(it.scratch + kScrBias)[tid];
   __syncthreads();
 
-  if (uint32_t(2 * warp) >= p.coder_group) return;  // no pair for this warp in a small group
-  const uint64_t kA = uint64_t(b - it.block_base) * p.coder_group + 2 * warp;
+  const uint64_t kA = uint64_t(b - it.block_base) * kCoderChunks + 2 * warp;
   if (kA >= L.nc) return;
   const bool hasB = kA + 1 < L.nc;
   CoderOut co{reinterpret_cast<uint32_t *>(it.scratch + kScrLen), it.scratch + scratch_win_offset(L.nc)};

@@ -119,8 +119,6 @@ struct EncParams {
   uint32_t total_chunks;
   uint32_t total_coder_blocks;
   uint32_t total_hist_blocks;
-  uint32_t coder_group;  // chunks per coder block (even, <= kCoderChunks)
-  uint32_t pad[3];
   EncItem items[kMaxItems];
 };
 
@@ -142,8 +140,7 @@ struct DecParams {
 
 // Histogram blocks: one tile of up to 4 chunks of one tensor.
 constexpr uint32_t kHistChunks = 4;
-// Encoder coder blocks: 8 warps, two chunks each, all of one tensor
-// (EncParams::coder_group chunks a block; the warps past it have none).
+// Encoder coder blocks: 8 warps, two chunks each, all of one tensor.
 constexpr uint32_t kCoderWarps = 8;
 constexpr uint32_t kCoderChunks = 2 * kCoderWarps;
 // Decoder blocks: 8 warps, two chunks each, all of one tensor.
