@@ -199,7 +199,7 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
 }
-// 2-D tile load (no multicast) into this CTA's shared memory, completing on bar
+// 2-D tile load into this CTA's own shared memory, completing on bar
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int32_t x, int32_t y,
                                             uint64_t *bar) {
   asm volatile(
