@@ -83,6 +83,9 @@ def parse(argv=None):
     ap.add_argument("--linear-only", action="store_true",
                     help="profiling only: draw the set's first four gate projections and run the "
                          "wc12_linear leg alone (one JSON line with its 'linear' object)")
+    ap.add_argument("--no-dtypes", dest="dtypes", action="store_false",
+                    help="skip the fp16 / fp8 leg (the headline set's leading tensors cast on the "
+                         "device, batched encode and decode timed; the 'dtypes' object)")
     ap.add_argument("--no-checksum", dest="checksum", action="store_false",
                     help="skip the block-checksum leg (wc_crc32_blocks, 1 MiB blocks, over the "
                          "container arena, timed after the step; the 'checksum' object)")
@@ -709,6 +712,60 @@ def checksum_leg(arena, dev, stream, reps: int = 10):
             "gbs": nbytes / t / 1e9, "reps": reps}
 
 
+def dtypes_leg(ins, dev, stream, budget: int = 600_000_000, reps: int = 5):
+    """The other dtypes of the codec (fp16, fp8 e4m3, fp8 e5m2) on the
+    headline set's leading bf16 tensors (up to `budget` values), cast on the
+    device: one batched encode and one batched decode per dtype, round trip
+    checked bit-exact.  Algorithmic bytes: encode reads the input and writes
+    the containers, decode reads the containers and writes the values."""
+    import torch
+    from fp32_weight_compression_b200 import wc
+    src, total = [], 0
+    for t in ins:
+        if t.dtype != torch.bfloat16 or total + t.numel() > budget:
+            continue
+        src.append(t)
+        total += t.numel()
+    out = {"values": total, "tensors": len(src)}
+
+    def timed(fn):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps / 1e3
+
+    for name, dt in (("fp16", torch.float16), ("fp8_e4m3", torch.float8_e4m3fn), ("fp8_e5m2", torch.float8_e5m2)):
+        xs = [t.to(dt) for t in src]
+        enc = wc.BatchEncoder([x.numel() for x in xs], [x.dtype for x in xs], dev).prepare(xs)
+        enc.run(stream)
+        torch.cuda.synchronize(dev)
+        sizes = enc.sizes.cpu().tolist()
+        conts = enc.containers(sizes)
+        outs = [torch.empty_like(x) for x in xs]
+        dec = wc.BatchDecoder(dev).prepare(conts, outs)
+        dec.run(stream)
+        torch.cuda.synchronize(dev)
+        assert int(dec.status.item()) == 0
+        elem = xs[0].element_size()
+        ok = all(torch.equal(o.view(torch.uint8), x.view(torch.uint8)) for o, x in zip(outs, xs))
+        assert ok, f"{name} round trip"
+        B = total * elem
+        C = int(sum(sizes))
+        te, td = timed(lambda: enc.run(stream)), timed(lambda: dec.run(stream))
+        out[name] = {"ratio": C / B,
+                     "encode": {"ms": te * 1e3, "gbs": B / te / 1e9, "hbm_gbs": (B + C) / te / 1e9},
+                     "decode": {"ms": td * 1e3, "gbs": B / td / 1e9, "hbm_gbs": (B + C) / td / 1e9}}
+        del xs, enc, dec, conts, outs
+        torch.cuda.empty_cache()
+    return out
+
+
 # ---------------------------------------------------------------------------
 def linear_only(cid: int, local: int):
     """The wc12_linear leg on its own (profiling): the set's first four gate
@@ -781,6 +838,7 @@ def main(argv=None):
     r = legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak)
     values_mine = int(sum(numels))
     checksum = checksum_leg(ds.enc.out, dev, stream) if args.checksum else None
+    dtl = dtypes_leg(ds.ins, dev, stream) if args.dtypes and world == 1 else None
     s12 = split12_leg(ds.ins, dev, stream) if args.split12 else None
     if s12 is not None:
         try:
@@ -869,6 +927,11 @@ def main(argv=None):
         for leg in ("encode", "decode"):
             s12[leg]["roofline_frac"] = s12[leg]["hbm_gbs"] / peak
         line["split12"] = s12
+    if dtl is not None:
+        for name in ("fp16", "fp8_e4m3", "fp8_e5m2"):
+            for leg in ("encode", "decode"):
+                dtl[name][leg]["roofline_frac"] = dtl[name][leg]["hbm_gbs"] / peak
+        line["dtypes"] = dtl
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
