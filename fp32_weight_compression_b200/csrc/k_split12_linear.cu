@@ -357,41 +357,21 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
     for (; loaded < kDepth && loaded < nst; loaded++) load_stage(loaded);
 
   // The CTA's exceptions and how they are patched (mode): 0 from a shared
-  // list binned by stage (bin[] relative starts), 1 from the plan's entries
-  // read at each stage (bin[] absolute starts, or the plan's own when the
-  // CTA has more stages than bin[] holds), 2 by walking the chunks' lists at
-  // each stage, 3 not at all (a corrupt plan, reported).
+  // list binned by stage (bin[] relative starts), 1 from the plan (bounds
+  // and entries read a stage ahead), 2 by walking the chunks' lists at each
+  // stage.
   const bool binned = nst <= kMaxStagesPerCta;
   uint32_t mode = 0;
   const uint32_t *plan_start = nullptr, *plan_ent = nullptr;
   if (p.plan != nullptr) {
-    // The plan holds the tile's exceptions as one range, by stage: its
-    // starts, then (up to kExcCap) its entries, into shared memory.
+    // The plan holds the tile's exceptions as one range, by stage: each
+    // stage's bounds and a thread's first entry of it are read a stage ahead
+    // in the loop, so nothing waits for them before the first stage.
     const wc12p::PlanLay P = wc12p::plan_lay(N, K, ne);
     plan_start = reinterpret_cast<const uint32_t *>(p.plan + wc12p::kStartOff) +
                  uint64_t(blockIdx.x) * (K / kBK) + s_begin;
     plan_ent = reinterpret_cast<const uint32_t *>(p.plan + P.off_ent);
     mode = 1;
-    if (binned) {
-      for (uint32_t i = tid; i <= nst; i += kThreads) bin[i] = plan_start[i];
-      __syncthreads();
-      bool bad = false;
-      for (uint32_t i = tid; i < nst; i += kThreads) bad |= bin[i] > bin[i + 1] || bin[i + 1] > ne;
-      if (__syncthreads_or(bad)) {
-        if (tid == 0) report(p.status, WC_ERR_CORRUPT);
-        mode = 3;
-      } else if (bin[nst] - bin[0] <= kExcCap) {
-        const uint32_t base = bin[0], total = bin[nst] - base;
-        for (uint32_t i = tid; i < total; i += kThreads) {
-          const uint32_t e = plan_ent[base + i];
-          exc_bin[i] = make_uint2(e & 63u, ((e >> 6) & 127u) | (((e >> 16) & 255u) << 16));
-        }
-        __syncthreads();  // every thread has read bin[0]
-        for (uint32_t i = tid; i <= nst; i += kThreads) bin[i] -= base;
-        __syncthreads();
-        mode = 0;
-      }
-    }
   } else {
   // The CTA's exceptions, once: positions within a chunk become (row, column)
   // relative to the CTA's tile with 32-bit arithmetic when 128 K fits it,
@@ -519,6 +499,13 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
       o_lo[q] = kIdxBytes + lo_gran(row, seg);
       o_a[q] = op_offset(row, 16 * seg, kASlice);  // + 128: the segment's second 8 values
     }
+    // mode 1: bounds of the current stage and this thread's first entry of it
+    uint32_t pb0 = 0, pb1 = 0, pe = 0;
+    if (mode == 1) {
+      pb0 = plan_start[0];
+      pb1 = plan_start[1];
+      pe = pb0 + uint32_t(tid) < ne ? plan_ent[pb0 + tid] : 0u;
+    }
     for (uint32_t s = 0; s < nst; s++) {
       const uint32_t as = s % kASlots;
       uint8_t *A = a_op + as * kAStage;
@@ -528,18 +515,20 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
       const bool okw = mbar_wait_or_flag(&full[s % kDepth], (s / kDepth) & 1u, vflag) &&
                        (s < kASlots || mbar_wait_or_flag(&a_free[as], ((s / kASlots) & 1u) ^ 1u, vflag));
       const uint32_t k0 = (s_begin + s) * kBK;
-      uint32_t eb0 = 0, eb1 = 0;  // the stage's exceptions (modes 0, 1)
-      if (mode == 0 || (mode == 1 && binned)) {
+      uint32_t eb0 = 0, eb1 = 0, first_e = 0;  // the stage's exceptions (modes 0, 1)
+      if (mode == 0) {
         eb0 = bin[s];
         eb1 = bin[s + 1];
       } else if (mode == 1) {
-        eb0 = plan_start[s];
-        eb1 = plan_start[s + 1];
+        // this stage's bounds and entry, read during the previous one; the
+        // next stage's now (the entry speculatively, within the plan)
+        eb0 = pb0;
+        eb1 = pb1;
+        first_e = pe;
+        pb0 = pb1;
+        pb1 = s + 2 <= nst ? plan_start[s + 2] : pb1;
+        pe = eb1 + uint32_t(tid) < ne ? plan_ent[eb1 + tid] : 0u;
       }
-      // mode 1: this thread's first entry of the stage, loaded before the
-      // expansion hides its latency
-      uint32_t first_e = 0;
-      if (mode == 1 && eb0 <= eb1 && eb1 <= ne && eb0 + uint32_t(tid) < eb1) first_e = plan_ent[eb0 + tid];
       if (okw) {
         // A: 512 segments of 16 values, two per thread: segment i is row
         // 8 (i / 32) + i % 8, values 16 ((i / 8) % 4) .., expanded from the
