@@ -29,7 +29,9 @@
 //     slot's and the ring slot's "free" mbarriers, which the expanding warps
 //     and the load lane wait on before they reuse either.
 // At the end each expanding warp reads its 32 TMEM lanes (rows) and adds them
-// into Y.
+// into Y.  The tile's exceptions: gathered once per CTA from the container's
+// per-chunk lists, or, with the weight's serving plan (wc12_linear_planned,
+// wc12_plan.cuh), read from the plan a stage ahead.
 //
 // Operand layouts (K-major).  A, no swizzle: a core matrix is 8 rows x 16
 // bytes stored as 128 contiguous bytes; the two 8-value halves of a K = 16
@@ -67,10 +69,10 @@ constexpr uint32_t kAStage = 4 * kASlice;
 constexpr uint32_t kASlots = 2;
 constexpr uint32_t kMaxTokens = 256;
 constexpr uint32_t kSpinLimit = 1u << 24;
-// A CTA's exceptions (its 128 rows, its range of K) are gathered once into a
-// shared-memory list of up to kExcCap entries {column in the CTA's K range,
-// row | high byte << 16}; a CTA with more walks its chunks' exception lists
-// at every stage instead.  Either way an exception's value differs from the
+// Without a plan, a CTA's exceptions (its 128 rows, its range of K) are
+// gathered once into a shared-memory list of up to kExcCap entries binned by
+// stage, {column in the stage, row | high byte << 16}; a CTA with more walks
+// its chunks' exception lists at every stage instead.  Either way an exception's value differs from the
 // expanded one only in its high byte (the low byte is stored for every value).
 constexpr uint32_t kExcCap = 512;
 // chunk offsets of a CTA's row block kept in shared memory for the gather
