@@ -13,9 +13,10 @@
 //   * lane 0 of the load warp brings, with TMA, the rows' 64 index nibbles
 //     and 64 low bytes each (12 bits a value, as stored) and the tokens' X
 //     slice (n_mma rows of 128 bytes, rows past M zero-filled, 128-byte
-//     swizzle: the B operand layout) into a ring slot, up to four stages
-//     ahead, once the MMAs that read the slot last are done; the slot's
-//     mbarrier completes when the bytes have landed;
+//     swizzle: the B operand layout) into a ring slot, up to D stages ahead
+//     (D = 4, or 3 or 2 where that lets two CTAs share an SM), once the MMAs
+//     that read the slot last are done; the slot's mbarrier completes when
+//     the bytes have landed;
 //   * the 8 expanding warps expand the 128 x 64 values from the ring slot
 //     in segments of 16 (8 index bytes + 16 low bytes -> 16 bf16, two
 //     16-byte rows of core matrices) into one of two A operand slots, patch
@@ -97,14 +98,16 @@ struct Params {
   int32_t *status;
 };
 
-// Shared memory: two expanded A operand slots, then a ring of kDepth load
-// slots (the stage's index bytes and low bytes of the 128 rows, as stored,
-// and the tokens' X slice already in the B operand layout), the mbarriers,
-// and the CTA's exception list.
-constexpr uint32_t kDepth = 4;
-// mbarriers (full, slot_free: kDepth each; a_full, a_free: kASlots each),
+// Shared memory: two expanded A operand slots, then a ring of D load slots
+// (the stage's index bytes and low bytes of the 128 rows, as stored, and the
+// tokens' X slice already in the B operand layout), the mbarriers and,
+// without a plan, the CTA's exception list.  The kernel is compiled for
+// D = 4, 3 and 2 (a constant, so that slot and phase indices are shifts and
+// masks).
+constexpr uint32_t kMaxDepth = 4;
+// mbarriers (full, slot_free: kMaxDepth each; a_full, a_free: kASlots each),
 // the TMEM address, the failure flag and the exception count
-constexpr uint32_t kBarBytes = 8 * (2 * kDepth + 2 * kASlots) + 16;
+constexpr uint32_t kBarBytes = 8 * (2 * kMaxDepth + 2 * kASlots) + 16;
 constexpr uint32_t kIdxBytes = kBM * kBK / 2;  // 4 KiB
 constexpr uint32_t kLoBytes = kBM * kBK;       // 8 KiB
 
@@ -112,9 +115,10 @@ __host__ __device__ inline uint32_t b_stage_bytes(uint32_t n_mma) { return n_mma
 __host__ __device__ inline uint32_t slot_bytes(uint32_t n_mma) { return kIdxBytes + kLoBytes + b_stage_bytes(n_mma); }
 // per-stage exception bins: a count (then start) per stage of the CTA
 constexpr uint32_t kMaxStagesPerCta = 256;
-__host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma) {
-  return 1024 + kASlots * kAStage + kDepth * slot_bytes(n_mma) + kBarBytes + 2 * 8 * kExcCap +
-         2 * 4 * (kMaxStagesPerCta + 1) + 8 * (kGatherChunks + 1);
+// the gathered exception list, its bins and cursors, the chunk offsets
+constexpr uint32_t kExcBytes = 2 * 8 * kExcCap + 2 * 4 * (kMaxStagesPerCta + 1) + 8 * (kGatherChunks + 1);
+__host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma, uint32_t depth, bool plan) {
+  return 1024 + kASlots * kAStage + depth * slot_bytes(n_mma) + kBarBytes + (plan ? 0u : kExcBytes);
 }
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
@@ -249,19 +253,22 @@ __device__ __forceinline__ bool mbar_wait_or_flag(uint64_t *bar, uint32_t parity
   return false;
 }
 
+template <uint32_t kDepth>
 __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant__ Params p) {
+  static_assert(kDepth >= 2 && kDepth <= kMaxDepth, "ring depth");
   extern __shared__ uint8_t dyn[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint8_t *a_op = base;                       // kASlots x kAStage
   uint8_t *ring = base + kASlots * kAStage;   // kDepth x slot_bytes
   const uint32_t sb = slot_bytes(p.n_mma);
   uint64_t *full = reinterpret_cast<uint64_t *>(ring + kDepth * sb);  // [kDepth] a slot's loads landed
-  uint64_t *slot_free = full + kDepth;                                // [kDepth] its MMAs are done
-  uint64_t *a_full = slot_free + kDepth;                              // [kASlots] A slot expanded
+  uint64_t *slot_free = full + kMaxDepth;                             // [kDepth] its MMAs are done
+  uint64_t *a_full = slot_free + kMaxDepth;                              // [kASlots] A slot expanded
   uint64_t *a_free = a_full + kASlots;                                // [kASlots] its MMAs are done
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(a_free + kASlots);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
   uint32_t *exc_n = tmem_slot + 2;
+  // without a plan only:
   uint2 *exc_raw = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(full) + kBarBytes);  // gathered
   uint2 *exc_bin = exc_raw + kExcCap;                                                        // by stage
   uint32_t *bin = reinterpret_cast<uint32_t *>(exc_bin + kExcCap);                           // per stage
@@ -347,7 +354,8 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
     *exc_n = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  for (uint32_t i = tid; i <= nst && i <= kMaxStagesPerCta; i += kThreads) bin[i] = 0;
+  if (p.plan == nullptr)
+    for (uint32_t i = tid; i <= nst && i <= kMaxStagesPerCta; i += kThreads) bin[i] = 0;
   fence_before_sync();
   __syncthreads();
   fence_after_sync();
@@ -679,18 +687,32 @@ struct DevInfo {
   bool attr = false;
   int smem_per_sm = 0;     // shared memory of one SM
   int smem_reserved = 0;   // per CTA, taken by the system
-  int regs = 0;            // registers a thread of k12_linear
+  int regs[kMaxDepth + 1] = {};  // registers a thread of k12_linear<D>
 };
 
-// Dynamic shared memory for a launch with n_mma token columns: at least what
-// the stages need, padded so that the CTAs that fit on one SM hold at most
-// the SM's 512 tensor-memory columns between them (otherwise a CTA's
-// tcgen05.alloc would wait for another CTA to finish).
-uint32_t launch_smem(const DevInfo &d, uint32_t n_mma) {
+using LinearKernel = void (*)(Params);
+LinearKernel kernel_for(uint32_t depth) {
+  return depth == 2 ? k12_linear<2> : (depth == 3 ? k12_linear<3> : k12_linear<kMaxDepth>);
+}
+
+// The ring depth of a launch: the deepest of 4, 3 and 2 that lets two CTAs
+// share an SM (the weights stream at twice the rate of one CTA's ring), else
+// 4 with one CTA an SM.
+uint32_t pick_depth(const DevInfo &d, uint32_t n_mma, bool plan) {
+  for (uint32_t dd = kMaxDepth; dd >= 2; dd--)
+    if (2 * (smem_bytes(n_mma, dd, plan) + uint32_t(d.smem_reserved)) <= uint32_t(d.smem_per_sm)) return dd;
+  return kMaxDepth;
+}
+
+// Dynamic shared memory for a launch with n_mma token columns and a ring of
+// `depth` slots: at least what the stages need, padded so that the CTAs that
+// fit on one SM hold at most the SM's 512 tensor-memory columns between them
+// (otherwise a CTA's tcgen05.alloc would wait for another CTA to finish).
+uint32_t launch_smem(const DevInfo &d, uint32_t n_mma, uint32_t depth, bool plan) {
   uint32_t cols = 32;
   while (cols < n_mma) cols <<= 1;
   const uint32_t max_ctas = 512 / cols;
-  uint32_t need = smem_bytes(n_mma);
+  uint32_t need = smem_bytes(n_mma, depth, plan);
   const uint32_t per_sm = uint32_t(d.smem_per_sm), rsv = uint32_t(d.smem_reserved);
   // CTAs per SM = floor(per_sm / (smem + rsv)); make it <= max_ctas
   const uint32_t floor_smem = per_sm / (max_ctas + 1) + 1;
@@ -744,16 +766,19 @@ DevInfo dev_info() {
       return DevInfo{};
     d.smem_per_sm = per_sm;
     d.smem_reserved = rsv;
-    uint32_t most = 0;
-    for (uint32_t m = 16; m <= kMaxTokens; m += 16) {
-      const uint32_t b = launch_smem(d, m);
-      most = b > most ? b : most;
+    d.attr = true;
+    for (uint32_t dd = 2; dd <= kMaxDepth; dd++) {
+      uint32_t most = 0;  // the largest launch of this depth (without a plan: the exception list)
+      for (uint32_t m = 16; m <= kMaxTokens; m += 16) {
+        const uint32_t b = launch_smem(d, m, dd, false);
+        most = b > most ? b : most;
+      }
+      d.attr = d.attr && cudaFuncSetAttribute(kernel_for(dd), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              int(most)) == cudaSuccess;
+      cudaFuncAttributes fa{};
+      if (cudaFuncGetAttributes(&fa, kernel_for(dd)) != cudaSuccess) return DevInfo{};
+      d.regs[dd] = fa.numRegs;
     }
-    d.attr = cudaFuncSetAttribute(k12_linear, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  int(most)) == cudaSuccess;
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, k12_linear) != cudaSuccess) return DevInfo{};
-    d.regs = fa.numRegs;
     d.sms = sms;
   }
   return d;
@@ -810,14 +835,15 @@ int32_t linear(const void *d_w, uint64_t w_bytes, const void *d_plan, uint64_t p
                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
       return WC_ERR_CUDA;
     // split K so that the grid is one wave of the CTAs an SM holds, with at
-    // least 4 stages a CTA when K allows (the load ring runs 4 ahead)
-    const uint32_t smem = wc12l::launch_smem(di, p.n_mma);
+    // least 4 stages a CTA when K allows (the load ring runs up to 4 ahead)
+    const uint32_t depth = wc12l::pick_depth(di, p.n_mma, d_plan != nullptr);
+    const uint32_t smem = wc12l::launch_smem(di, p.n_mma, depth, d_plan != nullptr);
     uint32_t cols = 32;
     while (cols < p.n_mma) cols <<= 1;
     // CTAs an SM holds: shared memory, registers (whole warps of 8-register
     // granules), threads, and the two the kernel is compiled for
     uint32_t per_sm = uint32_t(di.smem_per_sm) / (smem + uint32_t(di.smem_reserved));
-    const uint32_t warp_regs = (uint32_t(di.regs) + 7) / 8 * 8 * 32;
+    const uint32_t warp_regs = (uint32_t(di.regs[depth]) + 7) / 8 * 8 * 32;
     const uint32_t by_regs = 65536 / (warp_regs * (wc12l::kThreads / 32));
     if (per_sm > by_regs) per_sm = by_regs;
     if (per_sm > 2048 / wc12l::kThreads) per_sm = 2048 / wc12l::kThreads;
@@ -832,7 +858,7 @@ int32_t linear(const void *d_w, uint64_t w_bytes, const void *d_plan, uint64_t p
     p.splits = (stages + p.per_split - 1) / p.per_split;
     if (p.splits > 1) wc12l::k12_zero<<<unsigned(2 * di.sms), 256, 0, s>>>(p.y, uint64_t(m) * N);
     dim3 grid(blocks, p.splits);
-    wc12l::k12_linear<<<grid, wc12l::kThreads, smem, s>>>(p);
+    wc12l::kernel_for(depth)<<<grid, wc12l::kThreads, smem, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
   }
   return WC_OK;
