@@ -448,7 +448,7 @@ class DeviceSet:
 def time_steps(ds, K, W, stream, dev, barrier, sampler=None):
     """W warm-up steps, then exactly K timed steps (encode + decode each),
     bracketed by barrier + synchronize.  Returns (total, encode, decode)
-    seconds on this rank."""
+    seconds on this rank and the per-step encode and decode seconds."""
     import torch
     for _ in range(max(W, 1)):
         ds.enc.run()
@@ -476,15 +476,23 @@ def time_steps(ds, K, W, stream, dev, barrier, sampler=None):
         sampler.mark(t_wall0, t_wall1)
     ds.check()
     t_total = start.elapsed_time(end) / 1e3
-    t_enc = sum(e[0].elapsed_time(e[1]) for e in ev) / 1e3
-    t_dec = sum(e[1].elapsed_time(e[2]) for e in ev) / 1e3
-    return t_total, t_enc, t_dec
+    enc_steps = [e[0].elapsed_time(e[1]) / 1e3 for e in ev]
+    dec_steps = [e[1].elapsed_time(e[2]) / 1e3 for e in ev]
+    return t_total, sum(enc_steps), sum(dec_steps), enc_steps, dec_steps
 
 
-def legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak):
+def step_stats(steps):
+    """[median, best] of per-step seconds."""
+    return [statistics.median(steps), min(steps)]
+
+
+def legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak, enc_stats=None, dec_stats=None):
+    """The line's figures from the K timed steps; enc_stats / dec_stats:
+    [median, best] seconds of one step's encode / decode (added as
+    ms_median and ms_best)."""
     enc_bytes = total_in + total_cont  # read input, write container
     dec_bytes = total_cont + total_in  # read container, write output
-    return {
+    r = {
         "value": job_gbs(total_in, K, t_total),
         "ms_per_step": t_total / K * 1e3,
         "encode": {"gbs": job_gbs(total_in, K, t_enc), "ms": t_enc / K * 1e3,
@@ -496,6 +504,11 @@ def legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak):
         "ratio": total_cont / total_in,
         "dec_bytes": dec_bytes,
     }
+    for half, st in (("encode", enc_stats), ("decode", dec_stats)):
+        if st is not None:
+            r[half]["ms_median"] = st[0] * 1e3
+            r[half]["ms_best"] = st[1] * 1e3
+    return r
 
 
 def e2e_leg(args, host, offs, nbytes, dts, dev, stream, barrier, world):
@@ -829,13 +842,15 @@ def main(argv=None):
     peak, peak_note = peak_hbm()
     ds = DeviceSet(host, offs, nbytes, numels, dts, dev)
     sampler = ClockSampler(local)
-    t_total, t_enc, t_dec = time_steps(ds, args.steps, args.warmup, stream, dev, barrier, sampler)
+    t_total, t_enc, t_dec, enc_steps, dec_steps = time_steps(ds, args.steps, args.warmup, stream, dev,
+                                                             barrier, sampler)
     clocks = sampler.stop()
     total_cont = ds.container_bytes()
-    t_total, t_enc, t_dec = max_over_ranks([t_total, t_enc, t_dec], dev, world)
+    t_total, t_enc, t_dec, *st = max_over_ranks(
+        [t_total, t_enc, t_dec] + step_stats(enc_steps) + step_stats(dec_steps), dev, world)
     total_in, total_cont = (int(v) for v in sum_over_ranks([ds.bytes, total_cont], dev, world))
     K = args.steps
-    r = legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak)
+    r = legs(total_in, total_cont, K, t_total, t_enc, t_dec, peak, st[:2], st[2:])
     values_mine = int(sum(numels))
     checksum = checksum_leg(ds.enc.out, dev, stream) if args.checksum else None
     dtl = dtypes_leg(ds.ins, dev, stream) if args.dtypes and world == 1 else None
@@ -866,8 +881,9 @@ def main(argv=None):
             cs = workloads.tensor_specs(c)
             h, o, nb, nu, dt = generate_pinned(pool, c, list(range(len(cs))))
             d = DeviceSet(h, o, nb, nu, dt, dev)
-            tt, te, td = time_steps(d, args.extra_steps, 3, stream, dev, barrier)
-            rr = legs(d.bytes, d.container_bytes(), args.extra_steps, tt, te, td, peak)
+            tt, te, td, es, ds_ = time_steps(d, args.extra_steps, 3, stream, dev, barrier)
+            rr = legs(d.bytes, d.container_bytes(), args.extra_steps, tt, te, td, peak,
+                      step_stats(es), step_stats(ds_))
             rr.pop("dec_bytes")
             rr["workload"] = WORKLOAD_NAMES[c]
             rr["input_bytes"] = d.bytes
