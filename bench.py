@@ -155,13 +155,15 @@ def job_gbs(total_bytes, steps, seconds):
 def _oracle_worker(args):
     """Encode + decode the given tensors of a workload with the oracle, over
     and over, until `budget` seconds of oracle time are spent; the tensors
-    are drawn first and the timing starts when every worker is ready."""
-    cid, idx_list, budget, barrier = args
+    are drawn first (or arrive drawn) and the timing starts when every worker
+    is ready."""
+    cid, idx_list, budget, barrier = args[:4]
+    given = args[4] if len(args) > 4 else None
     sys.path.insert(0, ROOT)
     sys.path.insert(0, os.path.join(ROOT, "oracle"))
     import oracle
     import workloads as wl
-    data = [wl.generate_tensor(cid, i) for i in idx_list]
+    data = given if given is not None else [wl.generate_tensor(cid, i) for i in idx_list]
     oracle.decode(oracle.encode(data[0]))  # loads the library
     if barrier is not None:
         barrier.wait()
@@ -180,28 +182,34 @@ def _oracle_worker(args):
 
 def cpu_oracle_baseline(cid: int, budget: float, workers: int):
     """GB/s of oracle encode + decode on `workers` processes at once (one per
-    host core), each coding its own tensors of workload cid."""
+    host core), each coding its own tensors of workload cid (workload 5, one
+    2^28-value tensor: its first 64 chunks, 16 of each kind, drawn once here)."""
     import multiprocessing as mp
     specs = workloads.tensor_specs(cid)
-    if cid == 4:   # the k and v projections (4096x1024): many equal, modest tensors
+    given = None
+    if cid in (2, 4):   # the k and v projections: many equal, modest tensors
         pool_idx = [i for i, s in enumerate(specs) if s.name.endswith((".k", ".v"))]
-    elif cid == 2:
-        pool_idx = [i for i, s in enumerate(specs) if s.name.endswith((".k", ".v"))]
+    elif cid == 5:
+        pool_idx = [0]
+        given = [workloads.generate_tensor(5, 0)[: 64 * workloads.CHUNK].copy()]
     else:
         pool_idx = [i for i, s in enumerate(specs) if s.numel <= (1 << 22)] or [0]
     ctx = mp.get_context("spawn")
     barrier = ctx.Manager().Barrier(workers)
     assign = [[pool_idx[(w + k * workers) % len(pool_idx)] for k in range(2)] for w in range(workers)]
     with ctx.Pool(workers) as pool:
-        res = pool.map(_oracle_worker, [(cid, a, budget, barrier) for a in assign])
+        res = pool.map(_oracle_worker, [(cid, a, budget, barrier, given) for a in assign])
     total = sum(r[0] for r in res)
     wall = max(r[1] for r in res)
-    names = sorted({specs[i].name.split(".")[-1] for a in assign for i in a})
+    if given is not None:
+        what = "its first 64 chunks (16 of each adversarial kind)"
+    else:
+        names = sorted({specs[i].name.split(".")[-1] for a in assign for i in a})
+        what = f"2 of the {'/'.join(names)} tensors of the set"
     return {"value": total / wall / 1e9, "unit": "GB/s", "cores": workers, "kind": "oracle",
             "sample": (f"workload {cid}: {workers} processes at once (one per host core), each "
-                       f"coding 2 of the {'/'.join(names)} tensors of the set over and over "
-                       f"for {budget:.0f} s (encode + decode, {sum(r[2] for r in res)} tensor "
-                       f"round trips, {total / 1e9:.2f} GB)")}
+                       f"coding {what} over and over for {budget:.1f} s (encode + decode, "
+                       f"{sum(r[2] for r in res)} tensor round trips, {total / 1e9:.2f} GB)")}
 
 
 def cpu_oracle_single(budget: float):
@@ -815,9 +823,12 @@ def main(argv=None):
     # Host-side work first: the CPU baseline (all cores, then one), the
     # input draw.  Both use spawn-started processes, before any CUDA call.
     cpu_base = None
+    cpu_extra = {}  # the other sets' all-core figures, shorter samples
     if rank == 0 and world == 1 and args.cpu_seconds > 0:
         cpu_base = cpu_oracle_baseline(cid, args.cpu_seconds, host_cores())
         cpu_base["single_thread"] = cpu_oracle_single(min(3.0, args.cpu_seconds))
+        for c in extra:
+            cpu_extra[c] = cpu_oracle_baseline(c, min(2.5, args.cpu_seconds), host_cores())
     specs = workloads.tensor_specs(cid)
     idx = list(range(len(specs) if args.tensors <= 0 else min(args.tensors, len(specs))))
     shares = partition([specs[i].numel * specs[i].itemsize for i in idx], world)
@@ -887,6 +898,8 @@ def main(argv=None):
             rr.pop("dec_bytes")
             rr["workload"] = WORKLOAD_NAMES[c]
             rr["input_bytes"] = d.bytes
+            if c in cpu_extra:
+                rr["cpu_baseline"] = cpu_extra[c]
             rr["steps"] = args.extra_steps
             per_workload[str(c)] = rr
             launches += d.launches_per_step * args.extra_steps
