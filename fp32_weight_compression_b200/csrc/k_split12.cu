@@ -1,6 +1,6 @@
 // k_split12.cu -- the Split12 serving format for bf16 (include/wc_split12.h;
 // "weight-compression" README: the high byte from a codebook, the low byte
-// raw): encoder in five kernels, decoder in one, and their C ABI.
+// raw): encoder in six kernels, decoder in one, and their C ABI.
 //
 // Encode (all on one stream, sizes from n alone):
 //   k12_prep   1 block    header fields that depend on n, zero padding,
@@ -14,8 +14,9 @@
 //   k12_count  1 warp / chunk   the chunk's exceptions from its histogram
 //   k12_scan   1 block    exclusive scan -> exc_off[], ne, total size, the
 //                         padding after the exception lists
-//   k12_pack   1 block / chunk   index nibbles and low bytes; exceptions in
-//                         ascending position at the chunk's exc_off
+//   k12_pack   1 block / chunk   index nibbles and low bytes, a warp per
+//                         eighth of the chunk; exceptions in ascending
+//                         position at the chunk's exc_off
 // Decode: k12_decode, a persistent grid, one block per chunk at a time:
 // expands 16 values per thread per step (the codebook lives in four
 // registers; byte permutes do the lookup), then patches the chunk's
@@ -275,9 +276,90 @@ __device__ __forceinline__ uint32_t nibbles4(uint32_t s4, uint32_t &missed) {
   return (idx & 0xFu) | ((idx >> 4) & 0xF0u) | ((idx >> 8) & 0xF00u) | ((idx >> 12) & 0xF000u);
 }
 
+// The values of group g (16 values, or the chunk's ragged tail) that the
+// codebook misses, in ascending position: fn(position in the chunk, high
+// byte), for the first `missed` of them.
+template <typename F>
+__device__ __forceinline__ void for_misses(const uint8_t *lut, const uint16_t *src, uint32_t g, uint32_t nfull,
+                                           uint32_t tail, const uint4 &a, const uint4 &b, uint32_t missed,
+                                           F fn) {
+  const uint32_t nv = g < nfull ? 16u : (g == nfull ? tail : 0u);
+  for (uint32_t j = 0; j < nv && missed; j++) {
+    uint32_t v;
+    if (g < nfull) {
+      const uint32_t w = j < 8 ? (&a.x)[j >> 1] : (&b.x)[(j - 8) >> 1];
+      v = (j & 1) ? (w >> 16) : (w & 0xFFFFu);
+    } else {
+      v = src[16 * g + j];
+    }
+    const uint32_t h = v >> 8;
+    if (lut[h] == 0xFFu) {
+      fn(16 * g + j, h);
+      missed--;
+    }
+  }
+}
+
+// exclusive prefix over the warp's lanes, and the warp's total
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v, uint32_t &total) {
+  const int lane = threadIdx.x & 31;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t u = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  total = __shfl_sync(0xffffffffu, incl, 31);
+  return incl - v;
+}
+
+// Warp w of a block takes the chunk's groups [512 w, 512 (w + 1)), 32 a step
+// (16 values a lane), so the warps run without block barriers: a warp's
+// exceptions come in ascending position and are staged in shared memory;
+// after the chunk, one barrier gives each warp the count of the warps before
+// it, and the staged entries go to the chunk's list at that offset.  A warp
+// with more than kStaged reads its range again and writes them in place.
+constexpr uint32_t kPackWarps = kPackThreads / 32;
+constexpr uint32_t kWarpGroups = kChunk / 16 / kPackWarps;  // 512
+constexpr uint32_t kStaged = 256;
+
+// A warp's exceptions written in place, in ascending position from
+// exc_pos[e0] on, by reading its groups [g0, g1) again (the path for more
+// than fit in the staging list).
+__device__ __noinline__ void rewrite_misses(const uint8_t *lut, const uint16_t *src, uint32_t g0, uint32_t g1,
+                                            uint32_t nfull, uint32_t tail, uint64_t e0, uint16_t *exc_pos,
+                                            uint8_t *exc_val) {
+  const uint32_t lane = threadIdx.x & 31u;
+  uint32_t r = 0;
+  for (uint32_t gs = g0; gs < g1; gs += 32) {
+    const uint32_t g = gs + lane;
+    uint32_t missed = 0;
+    uint4 a = make_uint4(0, 0, 0, 0), bq = make_uint4(0, 0, 0, 0);
+    if (g < nfull) {
+      a = wc::ld_nc_v4(src + 16 * g);
+      bq = wc::ld_nc_v4(src + 16 * g + 8);
+      nibbles4(slots4(lut, a.x, a.y), missed);
+      nibbles4(slots4(lut, a.z, a.w), missed);
+      nibbles4(slots4(lut, bq.x, bq.y), missed);
+      nibbles4(slots4(lut, bq.z, bq.w), missed);
+    } else if (g == nfull && tail) {
+      for (uint32_t j = 0; j < tail; j++) missed += lut[src[16 * g + j] >> 8] == 0xFFu ? 1u : 0u;
+    }
+    uint32_t total;
+    uint64_t e = e0 + r + warp_excl_scan(missed, total);
+    for_misses(lut, src, g, nfull, tail, a, bq, missed, [&](uint32_t p, uint32_t h) {
+      exc_pos[e] = uint16_t(p);
+      exc_val[e] = uint8_t(h);
+      e++;
+    });
+    r += total;
+  }
+}
+
 __global__ void __launch_bounds__(kPackThreads) k12_pack(const __grid_constant__ EncBatch12 b) {
   __shared__ uint8_t lut[256];
-  __shared__ uint64_t red[kPackThreads / 32 + 1];
+  __shared__ uint32_t staged[kPackWarps][kStaged];  // position | high byte << 16
+  __shared__ uint32_t wcount[kPackWarps];
   const EncItem12 &it =
       b.items[find_item(b.items, b.count, blockIdx.x, [](const EncItem12 &x) { return x.chunk_base; })];
   const uint16_t *__restrict__ in = it.in;
@@ -285,6 +367,7 @@ __global__ void __launch_bounds__(kPackThreads) k12_pack(const __grid_constant__
   uint8_t *out = it.out;
   const uint8_t *scr = it.scr;
   const int tid = threadIdx.x;
+  const uint32_t w = uint32_t(tid) >> 5, lane = uint32_t(tid) & 31u;
   lut[tid] = scr[kScrLut + tid];
   const uint64_t c = blockIdx.x - it.chunk_base, v0 = c * kChunk;
   const uint32_t count = uint32_t(n - v0 < kChunk ? n - v0 : kChunk);
@@ -299,32 +382,34 @@ __global__ void __launch_bounds__(kPackThreads) k12_pack(const __grid_constant__
   uint8_t *idx_plane = out + L.off_idx + v0 / 2;
   uint8_t *lo_plane = out + L.off_lo + v0;
   const uint16_t *src = in + v0;
+  const uint32_t g0 = w * kWarpGroups;
+  const uint32_t g1 = g0 + kWarpGroups < ngroups ? g0 + kWarpGroups : ngroups;
   __syncthreads();
 
-  uint64_t run = 0;  // exceptions of this chunk written so far
-  // each step's group is loaded during the step before
+  uint32_t wrun = 0;  // this warp's exceptions so far
+  // each step's groups are loaded during the step before
   uint4 na = make_uint4(0, 0, 0, 0), nb = make_uint4(0, 0, 0, 0);
-  if (uint32_t(tid) < nfull) {
-    na = wc::ld_nc_v4(src + 16 * tid);
-    nb = wc::ld_nc_v4(src + 16 * tid + 8);
+  if (g0 + lane < nfull) {
+    na = wc::ld_nc_v4(src + 16 * (g0 + lane));
+    nb = wc::ld_nc_v4(src + 16 * (g0 + lane) + 8);
   }
-  for (uint32_t it = 0; it * kPackThreads < ngroups; it++) {
-    const uint32_t g = tid + it * kPackThreads;
+  for (uint32_t gs = g0; gs < g1; gs += 32) {
+    const uint32_t g = gs + lane;
     uint32_t missed = 0;
-    uint4 a = na, b = nb;
-    if (g + kPackThreads < nfull) {
-      na = wc::ld_nc_v4(src + 16 * (g + kPackThreads));
-      nb = wc::ld_nc_v4(src + 16 * (g + kPackThreads) + 8);
+    const uint4 a = na, bq = nb;
+    if (gs + 32 < g1 && g + 32 < nfull) {
+      na = wc::ld_nc_v4(src + 16 * (g + 32));
+      nb = wc::ld_nc_v4(src + 16 * (g + 32) + 8);
     }
     if (g < nfull) {
       const uint32_t q0 = nibbles4(slots4(lut, a.x, a.y), missed);
       const uint32_t q1 = nibbles4(slots4(lut, a.z, a.w), missed);
-      const uint32_t q2 = nibbles4(slots4(lut, b.x, b.y), missed);
-      const uint32_t q3 = nibbles4(slots4(lut, b.z, b.w), missed);
+      const uint32_t q2 = nibbles4(slots4(lut, bq.x, bq.y), missed);
+      const uint32_t q3 = nibbles4(slots4(lut, bq.z, bq.w), missed);
       *reinterpret_cast<uint2 *>(idx_plane + 8 * g) = make_uint2(q0 | (q1 << 16), q2 | (q3 << 16));
       *reinterpret_cast<uint4 *>(lo_plane + 16 * g) =
           make_uint4(__byte_perm(a.x, a.y, 0x6420), __byte_perm(a.z, a.w, 0x6420),
-                     __byte_perm(b.x, b.y, 0x6420), __byte_perm(b.z, b.w, 0x6420));
+                     __byte_perm(bq.x, bq.y, 0x6420), __byte_perm(bq.z, bq.w, 0x6420));
     } else if (g == nfull && tail) {
       uint32_t pair = 0;
       for (uint32_t j = 0; j < tail; j++) {
@@ -341,30 +426,29 @@ __global__ void __launch_bounds__(kPackThreads) k12_pack(const __grid_constant__
       }
       if (tail & 1) idx_plane[8 * g + tail / 2] = uint8_t(pair);  // high nibble 0
     }
-    // exceptions, in ascending position: this step's groups in thread order
-    if (__syncthreads_or(missed != 0)) {
-      const uint64_t before = wc::block_excl_scan_u64<kPackThreads>(missed, red);
-      const uint64_t total = wc::block_sum_u64<kPackThreads>(missed, red);
-      uint64_t e = e_base + run + before;
-      const uint32_t nv = g < nfull ? 16u : (g == nfull ? tail : 0u);
-      for (uint32_t j = 0; j < nv && missed; j++) {
-        uint32_t v;
-        if (g < nfull) {
-          const uint32_t w = j < 8 ? (&a.x)[j >> 1] : (&b.x)[(j - 8) >> 1];
-          v = (j & 1) ? (w >> 16) : (w & 0xFFFFu);
-        } else {
-          v = src[16 * g + j];
-        }
-        const uint32_t h = v >> 8;
-        if (lut[h] == 0xFFu) {
-          exc_pos[e] = uint16_t(16 * g + j);
-          exc_val[e] = uint8_t(h);
-          e++;
-          missed--;
-        }
-      }
-      run += total;
+    // this step's exceptions, in lane order, staged while there is room
+    if (__any_sync(0xffffffffu, missed != 0)) {
+      uint32_t total;
+      uint32_t pos = wrun + warp_excl_scan(missed, total);
+      for_misses(lut, src, g, nfull, tail, a, bq, missed, [&](uint32_t p, uint32_t h) {
+        if (pos < kStaged) staged[w][pos] = p | (h << 16);
+        pos++;
+      });
+      wrun += total;
     }
+  }
+  if (lane == 0) wcount[w] = wrun;
+  __syncthreads();
+  uint64_t e0 = e_base;
+  for (uint32_t q = 0; q < w; q++) e0 += wcount[q];
+  if (wrun <= kStaged) {
+    for (uint32_t i = lane; i < wrun; i += 32) {
+      const uint32_t v = staged[w][i];
+      exc_pos[e0 + i] = uint16_t(v);
+      exc_val[e0 + i] = uint8_t(v >> 16);
+    }
+  } else {
+    rewrite_misses(lut, src, g0, g1, nfull, tail, e0, exc_pos, exc_val);
   }
 }
 

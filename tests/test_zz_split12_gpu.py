@@ -62,6 +62,33 @@ def test_exceptions_across_chunks_and_steps(s12):
     _check(s12, b)
 
 
+def test_dense_exceptions_in_parts_of_a_chunk(s12):
+    """Exception counts around the encoder's per-warp staging (256 entries
+    for each eighth of a chunk, 8,192 values): exactly 256 in one eighth,
+    257 in the next, a dense run across the boundary of two eighths, dense
+    values in a ragged tail.  The other values take 16 high bytes only, so
+    the codebook is those 16 and every other byte is an exception."""
+    rng = np.random.default_rng(9)
+    n = 2 * C + 3000
+    book = np.array([0x3A, 0x3B, 0x3C, 0x3D, 0x3E, 0x3F, 0x40, 0x41,
+                     0xBA, 0xBB, 0xBC, 0xBD, 0xBE, 0xBF, 0xC0, 0xC1], np.uint16)
+    b = (book[rng.integers(0, 16, n)] << 8 | rng.integers(0, 256, n)).astype(np.uint16)
+    others = np.setdiff1d(np.arange(256, dtype=np.uint16), book)
+    rare = lambda k: (others[rng.integers(0, others.size, k)] << 8 | rng.integers(0, 256, k)).astype(np.uint16)
+    E = C // 8
+    for eighth, k in ((1, 256), (2, 257)):
+        b[eighth * E + rng.choice(E, k, replace=False)] = rare(k)
+    run = np.arange(C + 6 * E - 300, C + 6 * E + 400)          # across eighths 5 and 6 of chunk 1
+    b[run] = rare(run.size)
+    tail = np.arange(2 * C + 100, 2 * C + 2900)                 # the third chunk's 3,000 values
+    b[tail] = rare(tail.size)
+    hb = (b >> 8).astype(np.uint8)
+    assert np.array_equal(s12.codebook(hb), book.astype(np.uint8))
+    assert [int((~np.isin(hb[q * E:(q + 1) * E], book)).sum()) for q in (1, 2)] == [256, 257]
+    assert s12.read_header(s12.encode(b))["ne"] == 256 + 257 + run.size + tail.size
+    _check(s12, b)
+
+
 def test_every_pattern_and_tiny_alphabets(s12):
     _check(s12, np.arange(1 << 16, dtype=np.uint16))                      # ne at its bound
     _check(s12, np.full(3 * C + 5, 0x3F80, np.uint16))                    # K = 1
