@@ -67,7 +67,7 @@ constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr uint32_t kASlice = kBM * 16 * 2;   // bytes of one K = 16 slice of A
 constexpr uint32_t kAStage = 4 * kASlice;
-constexpr uint32_t kASlots = 2;
+constexpr uint32_t kMaxASlots = 2;
 constexpr uint32_t kMaxTokens = 256;
 constexpr uint32_t kSpinLimit = 1u << 24;
 // Without a plan, a CTA's exceptions (its 128 rows, its range of K) are
@@ -105,9 +105,9 @@ struct Params {
 // D = 4, 3 and 2 (a constant, so that slot and phase indices are shifts and
 // masks).
 constexpr uint32_t kMaxDepth = 4;
-// mbarriers (full, slot_free: kMaxDepth each; a_full, a_free: kASlots each),
-// the TMEM address, the failure flag and the exception count
-constexpr uint32_t kBarBytes = 8 * (2 * kMaxDepth + 2 * kASlots) + 16;
+// mbarriers (full, slot_free: kMaxDepth each; a_full, a_free: kMaxASlots
+// each), the TMEM address, the failure flag and the exception count
+constexpr uint32_t kBarBytes = 8 * (2 * kMaxDepth + 2 * kMaxASlots) + 16;
 constexpr uint32_t kIdxBytes = kBM * kBK / 2;  // 4 KiB
 constexpr uint32_t kLoBytes = kBM * kBK;       // 8 KiB
 
@@ -117,8 +117,8 @@ __host__ __device__ inline uint32_t slot_bytes(uint32_t n_mma) { return kIdxByte
 constexpr uint32_t kMaxStagesPerCta = 256;
 // the gathered exception list, its bins and cursors, the chunk offsets
 constexpr uint32_t kExcBytes = 2 * 8 * kExcCap + 2 * 4 * (kMaxStagesPerCta + 1) + 8 * (kGatherChunks + 1);
-__host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma, uint32_t depth, bool plan) {
-  return 1024 + kASlots * kAStage + depth * slot_bytes(n_mma) + kBarBytes + (plan ? 0u : kExcBytes);
+__host__ __device__ inline uint32_t smem_bytes(uint32_t n_mma, uint32_t depth, uint32_t aslots, bool plan) {
+  return 1024 + aslots * kAStage + depth * slot_bytes(n_mma) + kBarBytes + (plan ? 0u : kExcBytes);
 }
 
 __device__ __forceinline__ void report(int32_t *status, int32_t code) { atomicCAS(status, 0, code); }
@@ -253,9 +253,10 @@ __device__ __forceinline__ bool mbar_wait_or_flag(uint64_t *bar, uint32_t parity
   return false;
 }
 
-template <uint32_t kDepth>
+template <uint32_t kDepth, uint32_t kASlots>
 __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant__ Params p) {
   static_assert(kDepth >= 2 && kDepth <= kMaxDepth, "ring depth");
+  static_assert(kASlots >= 1 && kASlots <= kMaxASlots, "A slots");
   extern __shared__ uint8_t dyn[];
   uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(dyn) + 1023) & ~uintptr_t(1023));
   uint8_t *a_op = base;                       // kASlots x kAStage
@@ -264,8 +265,8 @@ __global__ void __launch_bounds__(kThreads, 2) k12_linear(const __grid_constant_
   uint64_t *full = reinterpret_cast<uint64_t *>(ring + kDepth * sb);  // [kDepth] a slot's loads landed
   uint64_t *slot_free = full + kMaxDepth;                             // [kDepth] its MMAs are done
   uint64_t *a_full = slot_free + kMaxDepth;                              // [kASlots] A slot expanded
-  uint64_t *a_free = a_full + kASlots;                                // [kASlots] its MMAs are done
-  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(a_free + kASlots);
+  uint64_t *a_free = a_full + kMaxASlots;                             // [kASlots] its MMAs are done
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(a_free + kMaxASlots);
   int *flag = reinterpret_cast<int *>(tmem_slot + 1);
   uint32_t *exc_n = tmem_slot + 2;
   // without a plan only:
@@ -687,32 +688,46 @@ struct DevInfo {
   bool attr = false;
   int smem_per_sm = 0;     // shared memory of one SM
   int smem_reserved = 0;   // per CTA, taken by the system
-  int regs[kMaxDepth + 1] = {};  // registers a thread of k12_linear<D>
+  int regs[4] = {};  // registers a thread of each compiled shape (kShapes)
 };
 
+// The compiled pipeline shapes {ring depth, A slots}, deepest first.
+struct Shape {
+  uint32_t depth, aslots;
+};
+constexpr Shape kShapes[4] = {{4, 2}, {3, 2}, {2, 2}, {2, 1}};
+
 using LinearKernel = void (*)(Params);
-LinearKernel kernel_for(uint32_t depth) {
-  return depth == 2 ? k12_linear<2> : (depth == 3 ? k12_linear<3> : k12_linear<kMaxDepth>);
+LinearKernel kernel_for(uint32_t shape) {
+  switch (shape) {
+    case 1: return k12_linear<3, 2>;
+    case 2: return k12_linear<2, 2>;
+    case 3: return k12_linear<2, 1>;
+    default: return k12_linear<4, 2>;
+  }
 }
 
-// The ring depth of a launch: the deepest of 4, 3 and 2 that lets two CTAs
-// share an SM (the weights stream at twice the rate of one CTA's ring), else
-// 4 with one CTA an SM.
-uint32_t pick_depth(const DevInfo &d, uint32_t n_mma, bool plan) {
-  for (uint32_t dd = kMaxDepth; dd >= 2; dd--)
-    if (2 * (smem_bytes(n_mma, dd, plan) + uint32_t(d.smem_reserved)) <= uint32_t(d.smem_per_sm)) return dd;
-  return kMaxDepth;
+// The shape of a launch: the first of kShapes (a 4-, 3- or 2-slot ring with
+// two A slots, then a 2-slot ring with one A slot, whose expansion of a stage
+// waits for the MMAs of the one before) that lets two CTAs share an SM —
+// two pipelines an SM, and every SM busy — else the deepest, one CTA an SM.
+uint32_t pick_shape(const DevInfo &d, uint32_t n_mma, bool plan) {
+  for (uint32_t i = 0; i < 4; i++)
+    if (2 * (smem_bytes(n_mma, kShapes[i].depth, kShapes[i].aslots, plan) + uint32_t(d.smem_reserved)) <=
+        uint32_t(d.smem_per_sm))
+      return i;
+  return 0;
 }
 
-// Dynamic shared memory for a launch with n_mma token columns and a ring of
-// `depth` slots: at least what the stages need, padded so that the CTAs that
+// Dynamic shared memory for a launch with n_mma token columns and pipeline
+// shape `shape`: at least what the stages need, padded so that the CTAs that
 // fit on one SM hold at most the SM's 512 tensor-memory columns between them
 // (otherwise a CTA's tcgen05.alloc would wait for another CTA to finish).
-uint32_t launch_smem(const DevInfo &d, uint32_t n_mma, uint32_t depth, bool plan) {
+uint32_t launch_smem(const DevInfo &d, uint32_t n_mma, uint32_t shape, bool plan) {
   uint32_t cols = 32;
   while (cols < n_mma) cols <<= 1;
   const uint32_t max_ctas = 512 / cols;
-  uint32_t need = smem_bytes(n_mma, depth, plan);
+  uint32_t need = smem_bytes(n_mma, kShapes[shape].depth, kShapes[shape].aslots, plan);
   const uint32_t per_sm = uint32_t(d.smem_per_sm), rsv = uint32_t(d.smem_reserved);
   // CTAs per SM = floor(per_sm / (smem + rsv)); make it <= max_ctas
   const uint32_t floor_smem = per_sm / (max_ctas + 1) + 1;
@@ -767,17 +782,17 @@ DevInfo dev_info() {
     d.smem_per_sm = per_sm;
     d.smem_reserved = rsv;
     d.attr = true;
-    for (uint32_t dd = 2; dd <= kMaxDepth; dd++) {
-      uint32_t most = 0;  // the largest launch of this depth (without a plan: the exception list)
+    for (uint32_t i = 0; i < 4; i++) {
+      uint32_t most = 0;  // the largest launch of this shape (without a plan: the exception list)
       for (uint32_t m = 16; m <= kMaxTokens; m += 16) {
-        const uint32_t b = launch_smem(d, m, dd, false);
+        const uint32_t b = launch_smem(d, m, i, false);
         most = b > most ? b : most;
       }
-      d.attr = d.attr && cudaFuncSetAttribute(kernel_for(dd), cudaFuncAttributeMaxDynamicSharedMemorySize,
+      d.attr = d.attr && cudaFuncSetAttribute(kernel_for(i), cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               int(most)) == cudaSuccess;
       cudaFuncAttributes fa{};
-      if (cudaFuncGetAttributes(&fa, kernel_for(dd)) != cudaSuccess) return DevInfo{};
-      d.regs[dd] = fa.numRegs;
+      if (cudaFuncGetAttributes(&fa, kernel_for(i)) != cudaSuccess) return DevInfo{};
+      d.regs[i] = fa.numRegs;
     }
     d.sms = sms;
   }
@@ -836,14 +851,14 @@ int32_t linear(const void *d_w, uint64_t w_bytes, const void *d_plan, uint64_t p
       return WC_ERR_CUDA;
     // split K so that the grid is one wave of the CTAs an SM holds, with at
     // least 4 stages a CTA when K allows (the load ring runs up to 4 ahead)
-    const uint32_t depth = wc12l::pick_depth(di, p.n_mma, d_plan != nullptr);
-    const uint32_t smem = wc12l::launch_smem(di, p.n_mma, depth, d_plan != nullptr);
+    const uint32_t shape = wc12l::pick_shape(di, p.n_mma, d_plan != nullptr);
+    const uint32_t smem = wc12l::launch_smem(di, p.n_mma, shape, d_plan != nullptr);
     uint32_t cols = 32;
     while (cols < p.n_mma) cols <<= 1;
     // CTAs an SM holds: shared memory, registers (whole warps of 8-register
     // granules), threads, and the two the kernel is compiled for
     uint32_t per_sm = uint32_t(di.smem_per_sm) / (smem + uint32_t(di.smem_reserved));
-    const uint32_t warp_regs = (uint32_t(di.regs[depth]) + 7) / 8 * 8 * 32;
+    const uint32_t warp_regs = (uint32_t(di.regs[shape]) + 7) / 8 * 8 * 32;
     const uint32_t by_regs = 65536 / (warp_regs * (wc12l::kThreads / 32));
     if (per_sm > by_regs) per_sm = by_regs;
     if (per_sm > 2048 / wc12l::kThreads) per_sm = 2048 / wc12l::kThreads;
@@ -858,7 +873,7 @@ int32_t linear(const void *d_w, uint64_t w_bytes, const void *d_plan, uint64_t p
     p.splits = (stages + p.per_split - 1) / p.per_split;
     if (p.splits > 1) wc12l::k12_zero<<<unsigned(2 * di.sms), 256, 0, s>>>(p.y, uint64_t(m) * N);
     dim3 grid(blocks, p.splits);
-    wc12l::kernel_for(depth)<<<grid, wc12l::kThreads, smem, s>>>(p);
+    wc12l::kernel_for(shape)<<<grid, wc12l::kThreads, smem, s>>>(p);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
   }
   return WC_OK;

@@ -85,7 +85,7 @@ def test_one_small_shape_first(s12):
 
 
 @pytest.mark.parametrize("N,K", [(128, 64), (256, 128), (128, 4096), (256, 4096)])
-@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 64, 144, 256, 300])
+@pytest.mark.parametrize("M", [1, 2, 3, 8, 9, 16, 17, 64, 144, 200, 256, 300])
 def test_shapes(s12, N, K, M):
     _check(s12, N, K, M, seed=N + K + M)
 
