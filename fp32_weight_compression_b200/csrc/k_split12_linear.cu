@@ -19,7 +19,8 @@
 //     the bytes have landed;
 //   * the 8 expanding warps expand the 128 x 64 values from the ring slot
 //     in segments of 16 (8 index bytes + 16 low bytes -> 16 bf16, two
-//     16-byte rows of core matrices) into one of two A operand slots, patch
+//     16-byte rows of core matrices) into one of two A operand slots (one,
+//     in the shape for the largest token counts), patch
 //     the tile's exceptions (after a named barrier among them, one thread
 //     an exception, its high byte) and arrive on the A slot's mbarrier.  A
 //     quarter warp takes 8 consecutive rows of one segment; with the loads'
