@@ -3,8 +3,11 @@
 // backwards; "SMEF" pass3_streams.py merge_streams).
 //
 // Persistent grid of 8-warp blocks.  Work is split into groups of 16
-// consecutive chunks of one tensor; a block takes groups blockIdx.x,
-// + gridDim.x, ...  The block stages its tensor's 4096-slot decoding table in
+// consecutive chunks of one tensor; a block takes the next group from the
+// launch's counter whenever it has finished one (the blocks an SM holds do
+// not progress at one rate -- the warp scheduler favours the older ones -- so
+// a fixed share each would leave fast blocks idle while slow ones finish).
+// The block stages its tensor's 4096-slot decoding table in
 // shared memory (entry = symbol | (slot - cum) << 8 | f << 20) and each warp
 // decodes two chunks.  When both are full 65,536-symbol coded chunks the warp
 // runs them in lock-step, so every lane carries two independent state chains;
@@ -24,6 +27,9 @@
 // length); a decoded chunk must end with every lane at 2^16 and every word
 // consumed.  Failures store a wc_status code in *status and skip the chunk.
 // No loop waits on another block; each wait is on this warp's own copies.
+#include <atomic>
+#include <mutex>
+
 #include "wc_block.cuh"
 #include "wc_format.cuh"
 #include "wc_planes.cuh"
@@ -42,6 +48,7 @@ struct DecSmem {
   uint32_t gpre[kMaxItems + 1];
   uint64_t red[kDecThreads / 32 + 1];
   int cur_item;
+  uint32_t next_grp;
   int tab_ok;
   int single_sym;
   // Word rings, kRing u16 per chunk, each on a 2 KiB boundary of the shared
@@ -655,7 +662,12 @@ __global__ void __launch_bounds__(kDecThreads, 4) k_decode(const __grid_constant
   __syncthreads();
   const uint32_t total = s.gpre[kMaxItems];
 
-  for (uint32_t grp = blockIdx.x; grp < total; grp += gridDim.x) {
+  for (;;) {
+    __syncthreads();  // every thread has read the previous group's number
+    if (tid == 0) s.next_grp = atomicAdd(p.queue, 1u);
+    __syncthreads();
+    const uint32_t grp = s.next_grp;
+    if (grp >= total) break;
     uint32_t lo = 0, hi = p.count - 1;  // last item with gpre <= grp
     while (lo < hi) {
       uint32_t mid = (lo + hi + 1) >> 1;
@@ -690,7 +702,43 @@ int decode_blocks_per_sm() {
   return nb;
 }
 
-cudaError_t launch_decode(const DecParams &p, int grid, cudaStream_t s) {
+// The launches' group counters: a library-held array of slots, one per
+// launch in rotation, each zeroed on the launch's stream before it runs, so
+// that calls overlapping on other streams (up to kQueueSlots of them) never
+// share one.
+constexpr uint32_t kQueueSlots = 4096;
+__device__ uint32_t g_dec_queue[kQueueSlots];
+
+// Device address of g_dec_queue on the current device, cached per device
+// together with the context it belongs to.
+static uint32_t *queue_base() {
+  struct Entry {
+    uint32_t *addr = nullptr;
+    unsigned long long ctx = 0;
+  };
+  static std::mutex mu;
+  static Entry cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  Entry &c = cache[dev];
+  const unsigned long long ctx = current_context_id();
+  if (c.addr == nullptr || ctx == 0 || c.ctx != ctx) {
+    void *a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_dec_queue) != cudaSuccess || a == nullptr) return nullptr;
+    c.addr = static_cast<uint32_t *>(a);
+    c.ctx = current_context_id();
+  }
+  return c.addr;
+}
+
+cudaError_t launch_decode(DecParams &p, int grid, cudaStream_t s) {
+  static std::atomic<uint32_t> next_slot{0};
+  uint32_t *base = queue_base();
+  if (base == nullptr) return cudaErrorInvalidSymbol;
+  p.queue = base + next_slot.fetch_add(1u) % kQueueSlots;
+  cudaError_t e = cudaMemsetAsync(p.queue, 0, sizeof(uint32_t), s);
+  if (e != cudaSuccess) return e;
   k_decode<<<grid, kDecThreads, sizeof(DecSmem), s>>>(p);
   return cudaGetLastError();
 }

@@ -135,6 +135,7 @@ struct DecParams {
   uint32_t count;
   uint32_t pad[3];
   int32_t *status;
+  uint32_t *queue;  // this launch's counter of groups taken (set by launch_decode)
   DecItem items[kMaxItems];
 };
 
@@ -151,8 +152,11 @@ cudaError_t launch_prep(const EncParams &p, cudaStream_t s);
 cudaError_t launch_hist(const EncParams &p, cudaStream_t s);
 cudaError_t launch_coder(const EncParams &p, cudaStream_t s);
 cudaError_t launch_compact(const EncParams &p, cudaStream_t s);
-cudaError_t launch_decode(const DecParams &p, int grid, cudaStream_t s);
+cudaError_t launch_decode(DecParams &p, int grid, cudaStream_t s);
 int decode_blocks_per_sm();
+// Identity of the CUDA context current on this thread, 0 if none (for
+// caching device addresses of the library's own device arrays).
+unsigned long long current_context_id();
 
 // ---------------------------------------------------------------------------
 // Device helpers.

@@ -35,6 +35,10 @@ uint64_t max_values() {
   return nc * wc::kChunk;
 }
 
+}  // namespace
+
+namespace wc {
+
 // Identity of the CUDA context current on this thread (0 if there is none or
 // the driver cannot say).  A device's array lives in the module loaded into
 // that device's context; if the context is destroyed and created again (a
@@ -67,6 +71,10 @@ unsigned long long current_context_id() {
   return id;
 }
 
+}  // namespace wc
+
+namespace {
+
 // Device address of g_noalloc_scratch on the current device, looked up with
 // that device current (in host code the symbol's name is only a host-side
 // stand-in, never a device address) and cached per device together with the
@@ -86,7 +94,7 @@ void *scratch_address(int32_t *err) {
   }
   std::lock_guard<std::mutex> lock(mu);
   Entry &c = cache[dev];
-  const unsigned long long ctx = current_context_id();
+  const unsigned long long ctx = wc::current_context_id();
   if (c.addr == nullptr || ctx == 0 || c.ctx != ctx) {
     void *p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
@@ -95,7 +103,7 @@ void *scratch_address(int32_t *err) {
       return nullptr;
     }
     c.addr = p;
-    c.ctx = current_context_id();  // the lookup made the device's context current
+    c.ctx = wc::current_context_id();  // the lookup made the device's context current
   }
   *err = WC_OK;
   return c.addr;

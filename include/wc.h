@@ -39,7 +39,12 @@
  *     h_* are host pointers.  The caller owns every buffer.  The library
  *     allocates no memory and never synchronises the device: all work is
  *     queued on `stream` (a cudaStream_t / CUstream handle; NULL is the
- *     legacy default stream) and the call returns before it runs.
+ *     legacy default stream) and the call returns before it runs.  It holds
+ *     two arrays in device memory of its own, loaded with it on every GPU:
+ *     wc_encode_noalloc's scratch (below) and 16 KiB of counters through
+ *     which a decode launch's blocks share out its work (4096 slots taken in
+ *     turn, each zeroed on the launch's stream first, so that up to 4096
+ *     decode launches may overlap on different streams).
  *   - Tensor and container buffers must be 16-byte aligned, scratch 256-byte
  *     aligned.  Values are passed as raw bits (bf16 = 2 bytes, fp32 = 4).
  *   - Argument, alignment and capacity errors are returned synchronously and
