@@ -17,7 +17,7 @@
 //   k12_pack   1 block / chunk   index nibbles and low bytes, a warp per
 //                         eighth of the chunk; exceptions in ascending
 //                         position at the chunk's exc_off
-// Decode: k12_decode, a persistent grid, one block per chunk at a time:
+// Decode: k12_decode, one block per chunk:
 // expands 16 values per thread per step (the codebook lives in four
 // registers; byte permutes do the lookup), then patches the chunk's
 // exceptions after a block barrier.
@@ -745,8 +745,10 @@ int32_t wc12_decode_batch(const wc12_decode_item *items, uint32_t count, int32_t
       if (units > 0x7FFFFFFFull) return WC_ERR_INVALID_ARG;
     }
     B.total_units = uint32_t(units);
-    const uint64_t cap = uint64_t(sms) * 8;
-    wc12::k12_decode_batch<<<unsigned(units < cap ? units : cap), wc12::kDecThreads, 0, s>>>(B);
+    // one block per unit: the hardware hands the next unit to whichever block
+    // slot frees first (a fixed share per block of a persistent grid left
+    // the faster blocks of an SM idle while its slower ones finished)
+    wc12::k12_decode_batch<<<unsigned(units), wc12::kDecThreads, 0, s>>>(B);
     if (cudaGetLastError() != cudaSuccess) return WC_ERR_CUDA;
   }
   return WC_OK;
@@ -760,7 +762,12 @@ int32_t wc12_decode(const void *d_cont, uint64_t cont_bytes, void *d_out, uint64
   if (out_cap > 0 && d_out == nullptr) return WC_ERR_INVALID_ARG;
   const int sms = wc12::sms_of_current_device();
   if (sms <= 0) return WC_ERR_CUDA;
-  wc12::k12_decode<<<unsigned(sms * 8), wc12::kDecThreads, 0, static_cast<cudaStream_t>(stream)>>>(
+  // one block per chunk the output can hold (the header, read on the device,
+  // gives the count; blocks past it have nothing to do)
+  uint64_t blocks = (out_cap / 2 + wc12::kChunk - 1) / wc12::kChunk;
+  if (blocks < 1) blocks = 1;
+  if (blocks > (uint64_t(1) << 24)) blocks = uint64_t(1) << 24;
+  wc12::k12_decode<<<unsigned(blocks), wc12::kDecThreads, 0, static_cast<cudaStream_t>(stream)>>>(
       static_cast<const uint8_t *>(d_cont), cont_bytes, static_cast<uint16_t *>(d_out), out_cap,
       d_status);
   const cudaError_t e = cudaGetLastError();
