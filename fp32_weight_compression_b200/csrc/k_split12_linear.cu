@@ -99,12 +99,12 @@ struct Params {
   int32_t *status;
 };
 
-// Shared memory: two expanded A operand slots, then a ring of D load slots
-// (the stage's index bytes and low bytes of the 128 rows, as stored, and the
-// tokens' X slice already in the B operand layout), the mbarriers and,
-// without a plan, the CTA's exception list.  The kernel is compiled for
-// D = 4, 3 and 2 (a constant, so that slot and phase indices are shifts and
-// masks).
+// Shared memory: the expanded A operand slots (two, or one), then a ring of
+// D load slots (the stage's index bytes and low bytes of the 128 rows, as
+// stored, and the tokens' X slice already in the B operand layout), the
+// mbarriers and, without a plan, the CTA's exception list.  The kernel is
+// compiled for four shapes, D = 4, 3 and 2 with two A slots and D = 2 with
+// one (constants, so that slot and phase indices are shifts and masks).
 constexpr uint32_t kMaxDepth = 4;
 // mbarriers (full, slot_free: kMaxDepth each; a_full, a_free: kMaxASlots
 // each), the TMEM address, the failure flag and the exception count
