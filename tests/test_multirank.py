@@ -77,6 +77,23 @@ def test_single_rank_needs_no_process_group():
     assert bench.job_gbs(2e9, 3, 2.0) == pytest.approx(3.0)
 
 
+def test_line_figures_from_the_timed_steps():
+    """legs(): the line's means from the K steps' totals, the per-step median
+    and best beside them, roofline fractions from the algorithmic bytes."""
+    import bench
+    enc_steps, dec_steps = [0.010, 0.012, 0.011], [0.007, 0.0072, 0.0071]
+    assert bench.step_stats(enc_steps) == [0.011, 0.010]
+    r = bench.legs(15e9, 10e9, 3, 0.06, sum(enc_steps), sum(dec_steps), 6540.0,
+                   bench.step_stats(enc_steps), bench.step_stats(dec_steps))
+    assert r["ms_per_step"] == pytest.approx(20.0)
+    assert r["encode"]["ms"] == pytest.approx(11.0) and r["decode"]["ms"] == pytest.approx(7.1)
+    assert (r["encode"]["ms_median"], r["encode"]["ms_best"]) == (pytest.approx(11.0), pytest.approx(10.0))
+    assert (r["decode"]["ms_median"], r["decode"]["ms_best"]) == (pytest.approx(7.1), pytest.approx(7.0))
+    assert r["decode"]["roofline_frac"] == pytest.approx(25e9 / 0.0071 / 1e9 / 6540.0)
+    assert r["ratio"] == pytest.approx(10 / 15)
+    assert "ms_median" not in bench.legs(1, 1, 1, 1.0, 0.5, 0.5, 1.0)["encode"]
+
+
 def test_partition_covers_every_tensor_once_and_balances():
     import bench
     for cid in (2, 3, 4):
