@@ -56,6 +56,12 @@
 #include "wc12_plan.cuh"
 #include "wc_split12.cuh"
 
+namespace wc {
+// Identity of the CUDA context current on this thread, 0 if none
+// (csrc/wc_noalloc.cu).
+unsigned long long current_context_id();
+}  // namespace wc
+
 namespace wc12l {
 
 using wc12::kChunk;
@@ -690,6 +696,7 @@ struct DevInfo {
   int smem_per_sm = 0;     // shared memory of one SM
   int smem_reserved = 0;   // per CTA, taken by the system
   int regs[4] = {};  // registers a thread of each compiled shape (kShapes)
+  unsigned long long ctx = 0;  // the context the attributes were set in
 };
 
 // The compiled pipeline shapes {ring depth, A slots}, deepest first.
@@ -773,7 +780,11 @@ DevInfo dev_info() {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return DevInfo{};
   std::lock_guard<std::mutex> lock(mu);
   DevInfo &d = cache[dev];
-  if (d.sms == 0) {
+  // once per device, and again in a context created afresh (after a
+  // cudaDeviceReset the kernels' shared-memory attributes must be set again)
+  const unsigned long long ctx = wc::current_context_id();
+  if (d.sms == 0 || (ctx != 0 && d.ctx != ctx)) {
+    d = DevInfo{};
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DevInfo{};
     int per_sm = 0, rsv = 0;
@@ -796,6 +807,7 @@ DevInfo dev_info() {
       d.regs[i] = fa.numRegs;
     }
     d.sms = sms;
+    d.ctx = wc::current_context_id();  // the set-up made the device's context current
   }
   return d;
 }

@@ -47,6 +47,7 @@ struct DeviceInfo {
   int dec_blocks_per_sm = 0;
   int crc_blocks_per_sm = 0;
   cudaError_t crc_err = cudaSuccess;
+  unsigned long long ctx = 0;  // the context the kernels' attributes were set in
 };
 
 DeviceInfo device_info(int32_t *err) {
@@ -59,7 +60,11 @@ DeviceInfo device_info(int32_t *err) {
     return DeviceInfo{};
   }
   std::lock_guard<std::mutex> lock(mu);
-  if (cache[dev].sms == 0) {
+  // once per device, and again in a context created afresh (after a
+  // cudaDeviceReset the kernels' shared-memory attributes must be set again)
+  const unsigned long long ctx = wc::current_context_id();
+  if (cache[dev].sms == 0 || (ctx != 0 && cache[dev].ctx != ctx)) {
+    cache[dev] = DeviceInfo{};
     int sms = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) {
@@ -77,6 +82,7 @@ DeviceInfo device_info(int32_t *err) {
     if (cache[dev].crc_blocks_per_sm <= 0) cache[dev].crc_err = cudaGetLastError();
     cache[dev].dec_blocks_per_sm = nb;
     cache[dev].sms = sms;
+    cache[dev].ctx = wc::current_context_id();  // the set-up made the device's context current
   }
   *err = WC_OK;
   return cache[dev];
